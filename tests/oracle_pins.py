@@ -1,0 +1,253 @@
+"""Pins that tie the float64 oracle to something other than itself.
+
+Each pin takes an ``oracle.Oracle`` instance and raises AssertionError when
+the oracle disagrees with: a hand-derived worked example (tests/golden), a
+closed form, an invariant the operator must satisfy, a library special case
+(numpy.fft for the hand-written FFT), or the direct definition on small
+inputs.  ``test_oracle.py`` runs every pin against the committed oracle and
+``test_oracle_mutations.py`` runs them against deliberately broken builds to
+show that a plausible mistake fails at least one pin.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _close(a, b, tol=1e-12, what=""):
+    a = np.asarray(a)
+    b = np.asarray(b)
+    if not (np.iscomplexobj(a) or np.iscomplexobj(b)):
+        a = a.astype(np.float64)
+        b = b.astype(np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} > {tol:.1e} * {scale:.3e}"
+
+
+# ------------------------------------------------------------------ FFT ---
+def pin_fft_matches_numpy(orc):
+    """The hand-written radix-2 FFT against numpy.fft (library special case)."""
+    rng = np.random.default_rng(1)
+    for m in range(0, 15):
+        n = 1 << m
+        z = rng.standard_normal(n) + 1j * rng.standard_normal(n)
+        _close(orc.fft(z), np.fft.fft(z), 1e-11, f"fft n={n}")
+        _close(orc.fft(z, inverse=True), np.fft.ifft(z) * n, 1e-11, f"ifft n={n}")
+
+
+def pin_fft_delta_and_parseval(orc):
+    n = 1024
+    d = np.zeros(n, complex); d[0] = 1.0
+    _close(orc.fft(d), np.ones(n), 1e-14, "fft(delta) = 1")
+    d2 = np.zeros(n, complex); d2[1] = 1.0
+    f = np.arange(n)
+    _close(orc.fft(d2), np.exp(-2j * np.pi * f / n), 1e-13, "fft(delta_1) = exp(-2 pi i f/n)")
+    z = np.random.default_rng(2).standard_normal(n) + 0j
+    Z = orc.fft(z)
+    assert abs(np.sum(np.abs(Z) ** 2) / n - np.sum(np.abs(z) ** 2)) < 1e-9 * np.sum(np.abs(z) ** 2)
+
+
+# ------------------------------------------------------------ worked examples
+def pin_golden_shortconv(orc):
+    g = _golden("shortconv_len4.json")
+    _close(orc.shortconv(g["u"], g["w"], g["bias"]), g["expected"], 1e-15, "shortconv golden")
+
+
+def pin_golden_fftconv(orc):
+    g = _golden("fftconv_len4.json")
+    _close(orc.causal_conv_direct(g["k"], g["D"], g["x"]), g["expected"], 1e-15, "direct golden")
+    _close(orc.causal_conv_fft(g["k"], g["D"], g["x"]), g["expected"], 1e-13, "fft golden")
+
+
+def pin_golden_operator_order2(orc):
+    g = _golden("operator_order2_len4.json")
+    u = np.array(g["u"], float)[None]
+    k = np.array(g["k"], float)[None]
+    D = np.array(g["D"], float)[None]
+    for method in (1, 2):
+        _close(orc.hyena_rows(u, k, D, method=method)[0], g["expected"], 1e-13,
+               f"operator order 2 golden, method {method}")
+
+
+def pin_golden_operator_order3(orc):
+    g = _golden("operator_order3_len3.json")
+    u = np.array(g["u"], float)[None]
+    k = np.array(g["k"], float)[None]
+    D = np.array(g["D"], float)[None]
+    for method in (1, 2):
+        _close(orc.hyena_rows(u, k, D, method=method)[0], g["expected"], 1e-13,
+               f"operator order 3 golden, method {method}")
+
+
+def pin_golden_conv2d(orc):
+    g = _golden("conv2d_2x2.json")
+    _close(orc.conv2d_direct(g["K"], g["D"], g["x"]), g["expected"], 1e-15, "conv2d direct golden")
+    _close(orc.conv2d_fft(g["K"], g["D"], g["x"]), g["expected"], 1e-13, "conv2d fft golden")
+
+
+def pin_golden_operator2d(orc):
+    g = _golden("operator2d_order2_2x2.json")
+    u = np.array(g["u"], float)[None]
+    k = np.array(g["k"], float)[None]
+    D = np.array(g["D"], float)[None]
+    for method in (1, 2):
+        _close(orc.hyena_rows(u, k, D, ndim=2, method=method)[0], g["expected"], 1e-13,
+               f"2-D operator golden, method {method}")
+
+
+# ---------------------------------------------------------- closed forms ---
+def pin_geometric_filter_closed_form(orc):
+    """k[t] = r^t, x = 1  ->  out[t] = (1 - r^(t+1)) / (1 - r) + D."""
+    L, r, D = 257, 0.97, -0.75
+    t = np.arange(L)
+    k = r ** t
+    want = (1 - r ** (t + 1)) / (1 - r) + D
+    _close(orc.causal_conv_direct(k, D, np.ones(L)), want, 1e-12, "geometric direct")
+    _close(orc.causal_conv_fft(k, D, np.ones(L)), want, 1e-11, "geometric fft")
+
+
+def pin_delta_invariant(orc):
+    """x0 = x1 = 1, v = delta_0, no short conv  ->  y = k + D delta_0 (order 2)."""
+    rng = np.random.default_rng(3)
+    for L in (16, 1024, 8192):
+        k = rng.standard_normal(L)
+        D = 0.625
+        u = np.ones((1, 3, L)); u[0, 2] = 0.0; u[0, 2, 0] = 1.0
+        want = k.copy(); want[0] += D
+        for method in (1, 2):
+            if method == 1 and L > 1024:
+                continue
+            y = orc.hyena_rows(u, k[None, None], np.array([[D]]), method=method)[0]
+            _close(y, want, 1e-12, f"delta invariant L={L} method {method}")
+
+
+# ------------------------------------------------------------ invariants ---
+def _rand_rows(rng, R, order, L, shortconv=True, bias=False):
+    u = rng.standard_normal((R, order + 1, L))
+    k = rng.standard_normal((R, order - 1, L)) * np.exp(-3.0 * np.arange(L) / L)
+    D = rng.standard_normal((R, order - 1))
+    w = rng.standard_normal((R, order + 1, 3)) * np.sqrt(1 / 3) if shortconv else None
+    b = rng.standard_normal((R, order + 1)) if (shortconv and bias) else None
+    return u, k, D, w, b
+
+
+def pin_fft_conv_equals_direct(orc):
+    rng = np.random.default_rng(4)
+    for L in (1, 2, 3, 5, 8, 17, 64, 100, 1024, 4096):
+        k = rng.standard_normal(L); x = rng.standard_normal(L); D = float(rng.standard_normal())
+        _close(orc.causal_conv_fft(k, D, x), orc.causal_conv_direct(k, D, x), 1e-11, f"L={L}")
+
+
+def pin_conv2d_fft_equals_direct(orc):
+    rng = np.random.default_rng(5)
+    for H, W in ((1, 1), (1, 8), (3, 5), (8, 8), (16, 32), (32, 32)):
+        K = rng.standard_normal((H, W)); x = rng.standard_normal((H, W))
+        _close(orc.conv2d_fft(K, 0.3, x), orc.conv2d_direct(K, 0.3, x), 1e-11, f"{H}x{W}")
+
+
+def pin_conv2d_single_row_is_1d(orc):
+    rng = np.random.default_rng(6)
+    W = 64
+    K = rng.standard_normal((1, W)); x = rng.standard_normal((1, W))
+    _close(orc.conv2d_direct(K, 0.5, x)[0], orc.causal_conv_direct(K[0], 0.5, x[0]), 1e-12, "H=1")
+    Kc = rng.standard_normal((W, 1)); xc = rng.standard_normal((W, 1))
+    _close(orc.conv2d_direct(Kc, 0.5, xc)[:, 0], orc.causal_conv_direct(Kc[:, 0], 0.5, xc[:, 0]),
+           1e-12, "W=1")
+
+
+def pin_operator_direct_equals_fft(orc):
+    rng = np.random.default_rng(7)
+    for order in (2, 3, 4):
+        u, k, D, w, b = _rand_rows(rng, 3, order, 300, bias=True)
+        y1 = orc.hyena_rows(u, k, D, w, b, method=1)
+        y2 = orc.hyena_rows(u, k, D, w, b, method=2)
+        _close(y2, y1, 1e-10, f"order {order}")
+
+
+def pin_causality(orc):
+    """Perturbing any chunk at t > s leaves y[0..s] bitwise unchanged."""
+    rng = np.random.default_rng(8)
+    L, s = 200, 117
+    for order in (2, 3):
+        u, k, D, w, b = _rand_rows(rng, 1, order, L, bias=True)
+        y = orc.hyena_rows(u, k, D, w, b, method=1)
+        u2 = u.copy()
+        u2[:, :, s + 1:] += rng.standard_normal(u2[:, :, s + 1:].shape)
+        y2 = orc.hyena_rows(u2, k, D, w, b, method=1)
+        assert np.array_equal(y[:, :s + 1], y2[:, :s + 1]), f"order {order}: not causal"
+        assert not np.array_equal(y[:, s + 1:], y2[:, s + 1:])
+
+
+def pin_linearity_in_v(orc):
+    """Order 2, no short conv: y is linear in the value chunk v."""
+    rng = np.random.default_rng(9)
+    L = 512
+    u, k, D, _, _ = _rand_rows(rng, 1, 2, L, shortconv=False)
+    a, c = rng.standard_normal(L), rng.standard_normal(L)
+    alpha, beta = 1.75, -0.5
+
+    def run(v):
+        uu = u.copy(); uu[0, 2] = v
+        return orc.hyena_rows(uu, k, D, method=2)[0]
+
+    _close(run(alpha * a + beta * c), alpha * run(a) + beta * run(c), 1e-11, "linearity")
+
+
+def pin_gating(orc):
+    """Order 2, no short conv: scaling x0 or x1 by alpha scales y by alpha; y/x0 is gate-free."""
+    rng = np.random.default_rng(10)
+    L = 256
+    u, k, D, _, _ = _rand_rows(rng, 1, 2, L, shortconv=False)
+    y = orc.hyena_rows(u, k, D, method=1)[0]
+    for j in (0, 1):
+        uu = u.copy(); uu[0, j] *= -2.5
+        _close(orc.hyena_rows(uu, k, D, method=1)[0], -2.5 * y, 1e-12, f"scale x{j}")
+    # y / x0 equals the ungated long conv of x1*v
+    conv = orc.causal_conv_direct(k[0, 0], D[0, 0], u[0, 1] * u[0, 2])
+    _close(y, u[0, 0] * conv, 1e-12, "output gate")
+
+
+def pin_order3_step_pairing(orc):
+    """Order 3 with one step made the identity isolates the other step's pairing."""
+    rng = np.random.default_rng(11)
+    L = 64
+    u, k, D, _, _ = _rand_rows(rng, 1, 3, L, shortconv=False)
+    delta = np.zeros(L); delta[0] = 1.0
+    # step 2 (gate x1, k[1], D[1]) is the identity: x1 = 1, k[1] = delta, D[1] = 0
+    u1 = u.copy(); u1[0, 1] = 1.0
+    k1 = k.copy(); k1[0, 1] = delta
+    D1 = D.copy(); D1[0, 1] = 0.0
+    want = u[0, 0] * orc.causal_conv_direct(k[0, 0], D[0, 0], u[0, 3] * u[0, 2])
+    _close(orc.hyena_rows(u1, k1, D1, method=1)[0], want, 1e-12, "step 1 = (x2, k[0], D[0])")
+    # step 1 (gate x2, k[0], D[0]) is the identity
+    u2 = u.copy(); u2[0, 2] = 1.0
+    k2 = k.copy(); k2[0, 0] = delta
+    D2 = D.copy(); D2[0, 0] = 0.0
+    want = u[0, 0] * orc.causal_conv_direct(k[0, 1], D[0, 1], u[0, 3] * u[0, 1])
+    _close(orc.hyena_rows(u2, k2, D2, method=1)[0], want, 1e-12, "step 2 = (x1, k[1], D[1])")
+
+
+def pin_shortconv_feeds_every_chunk(orc):
+    """With taps (0, 0, c_j) the short conv is a per-chunk scale c_j + bias b_j."""
+    rng = np.random.default_rng(12)
+    L = 128
+    u, k, D, _, _ = _rand_rows(rng, 1, 2, L, shortconv=False)
+    c = np.array([1.5, -0.5, 2.0]); bias = np.array([0.25, -1.0, 0.5])
+    w = np.zeros((1, 3, 3)); w[0, :, 2] = c
+    y = orc.hyena_rows(u, k, D, w, bias[None], method=1)[0]
+    us = u * c[None, :, None] + bias[None, :, None]
+    _close(y, orc.hyena_rows(us, k, D, method=1)[0], 1e-12, "per-chunk scale")
+
+
+ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -1,0 +1,60 @@
+"""Planted mistakes in the oracle must each fail at least one pin.
+
+Each case copies hyena_oracle.c, applies one textual change that a careless
+implementation could plausibly contain, compiles it with gcc into a
+temporary directory and runs every pin against it.  The committed oracle is
+never modified.  This shows the pins constrain every part of the oracle.
+"""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTATIONS = {
+    "shortconv taps reversed": ("out[t] = w[0] * um2 + w[1] * um1 + w[2] * u[t] + bias;",
+                                "out[t] = w[2] * um2 + w[1] * um1 + w[0] * u[t] + bias;"),
+    "shortconv bias dropped": ("out[t] = w[0] * um2 + w[1] * um1 + w[2] * u[t] + bias;",
+                               "out[t] = w[0] * um2 + w[1] * um1 + w[2] * u[t];"),
+    "conv skip D dropped": ("out[t] = acc + D * x[t];", "out[t] = acc;"),
+    "conv not causal-inclusive": ("for (int64_t tau = 0; tau <= t; ++tau)",
+                                  "for (int64_t tau = 0; tau < t; ++tau)"),
+    "fft sign flipped": ("sw[j] = sin(a) * (double)sign;", "sw[j] = -sin(a) * (double)sign;"),
+    "fft twiddle stride": ("double wr = cw[j * step], wi = sw[j * step];",
+                           "double wr = cw[j], wi = sw[j];"),
+    "fft conv circular (no padding)": ("int64_t n = next_pow2(2 * L);", "int64_t n = next_pow2(L);"),
+    "fft conv skip dropped": ("out[t] = xr[t] / (double)n + D * x[t];", "out[t] = xr[t] / (double)n;"),
+    "2-D kernel transposed": ("acc += K[i * W + j] * x[(p - i) * W + (q - j)];",
+                              "acc += K[j * W + i] * x[(p - i) * W + (q - j)];"),
+    "2-D fft conv circular": ("int64_t nh = next_pow2(2 * H), nw = next_pow2(2 * W);",
+                              "int64_t nh = next_pow2(H), nw = next_pow2(W);"),
+    "gate order not reversed": ("const double *gate = x + (int64_t)(order - s) * n;",
+                                "const double *gate = x + (int64_t)s * n;"),
+    "filters in reverse step order": ("const double *ks = k_row + (int64_t)(s - 1) * n;",
+                                      "const double *ks = k_row + (int64_t)(order - 1 - s) * n;"),
+    "skip from the wrong step": ("double Ds = D_row[s - 1];", "double Ds = D_row[order - 1 - s];"),
+    "output gated by x1": ("for (int64_t t = 0; t < n; ++t) y_row[t] = x[t] * v[t];",
+                           "for (int64_t t = 0; t < n; ++t) y_row[t] = x[n + t] * v[t];"),
+    "value chunk taken first": ("double *v = x + (int64_t)order * n;", "double *v = x;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name):
+    old, new = MUTATIONS[name]
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "hyena_oracle.c")).read()
+    assert src.count(old) == 1, f"mutation anchor not found exactly once: {old!r}"
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "mutant.c")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        mutant = oracle.Oracle(oracle.build(force=True, src=path, out=os.path.join(d, "libmutant.so")))
+        failed = []
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin(mutant)
+            except AssertionError:
+                failed.append(pin.__name__)
+        assert failed, f"no pin catches the planted mistake '{name}'"
