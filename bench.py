@@ -1,0 +1,363 @@
+"""Benchmark of the Hyena gated FFT long convolution on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload d768_l8k] [--no-cpu-baseline]
+
+A step is one hyena_gated_fftconv call over the whole workload (short conv,
+all order steps, output gate) with inputs resident in HBM.  Default workload:
+B=4, C=768, L=8192, order 2, bf16 storage / fp32 math (the 1-D operator at
+width 768 and 8K context).  The spectrum cache is built once, before timing.
+Every step reads ~252 MB (> the 126 MB L2), so no explicit L2 flush is needed.
+
+N > 1 (torchrun): every rank runs the same per-GPU workload on its own GPU
+(rows are independent: no exchange), so scaling is weak; the time is the max
+over ranks and value = all ranks' tokens / that time.
+
+`--impl reference` times the float64 CPU oracle on the host cores on a
+bounded sample of rows per step (the pages ship no runnable reference code).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Hyena op fwd tokens/s (B·L/s) at D=768, L=8K on 1×B200; % of HBM roofline"
+UNIT = "tokens/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
+    """One read of u (all order+1 chunks), one read of the stored spectra,
+    one write of y."""
+    es = 2 if p.dtype == "bf16" else 4
+    u = p.B * p.Ctot * p.n * es
+    y = p.B * p.C * p.n * es
+    spec = (p.order - 1) * p.C * spectrum_row_bytes
+    return u + spec + y
+
+
+def spectrum_row_bytes(p) -> int:
+    """Stored spectrum bytes per (step, channel) row of the library's layout."""
+    if p.ndim == 2:
+        return (p.W + 1) * 2 * p.H * 8
+    if p.L <= 16384:
+        return (p.L // 2 + 1) * 16
+    return 8 * p.L
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fft_long_convolution_02_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entries = json.load(f)
+    src = source_hash()
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_hash") == src:
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hyena_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def cpu_baseline(p, budget_s: float = 15.0):
+    """Time the float64 oracle (as it stands) on a bounded sample of rows."""
+    import oracle
+    from fft_long_convolution_02_b200 import inputs as I
+    cores = len(os.sched_getaffinity(0))
+    orc = oracle.default()
+    rng = np.random.default_rng(0)
+    rows = rng.choice(p.B * p.C, size=min(p.B * p.C, 8 * cores), replace=False)
+    args = I.oracle_rows(p, rows)
+    t0 = time.perf_counter()
+    orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores)
+    dt = time.perf_counter() - t0
+    # grow the sample to use about budget_s of CPU time
+    n_more = int(len(rows) * max(0.0, budget_s / max(dt, 1e-3) - 1.0))
+    n_more = min(n_more, p.B * p.C - len(rows))
+    total_rows, total_t = len(rows), dt
+    if n_more > 0:
+        rows2 = rng.choice(p.B * p.C, size=n_more, replace=False)
+        args = I.oracle_rows(p, rows2)
+        t0 = time.perf_counter()
+        orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores)
+        total_t += time.perf_counter() - t0
+        total_rows += n_more
+    # a row is one (b, c) pair; the operator's tokens are B*n over all C channels
+    tok_s = total_rows * p.n / (p.C * total_t)
+    return {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{total_rows} of {p.B * p.C} (b,c) rows, radix-2 FFT oracle in float64, "
+                      f"{total_t:.1f} s; tokens/s = rows*n/(C*t)"}
+
+
+def run_reference(args, p):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from fft_long_convolution_02_b200 import inputs as I
+    cores = len(os.sched_getaffinity(0))
+    orc = oracle.default()
+    rng = np.random.default_rng(1)
+    per_step = max(cores, 16)
+    samples = [I.oracle_rows(p, rng.choice(p.B * p.C, size=per_step, replace=False))
+               for _ in range(args.warmup + args.steps)]
+    for a in samples[:args.warmup]:
+        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores)
+    t0 = time.perf_counter()
+    for a in samples[args.warmup:]:
+        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores)
+    dt = time.perf_counter() - t0
+    tok_s = args.steps * per_step * p.n / (p.C * dt)
+    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": config_of(p),
+            "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} (b,c) rows per step of {p.B * p.C}; float64 radix-2 "
+                                       f"FFT oracle; tokens/s = rows*n/(C*t)"},
+            "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(p):
+    cfg = {"workload": p.name, "B": p.B, "C": p.C, "order": p.order,
+           "shortconv": p.shortconv, "storage": p.dtype, "math": "fp32"}
+    if p.ndim == 1:
+        cfg["L"] = p.L
+    else:
+        cfg["H"], cfg["W"] = p.H, p.W
+    return cfg
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="d768_l8k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from fft_long_convolution_02_b200 import inputs as I
+    p = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, p)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from fft_long_convolution_02_b200 import binding as hb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    hb.load()
+    dev = torch.device("cuda", local)
+    data = I.make_all(p)
+    if p.dtype == "bf16":
+        u_host = torch.from_numpy(data["u"].view(np.int16)).view(torch.bfloat16)
+        k_dev = torch.from_numpy(data["k"].view(np.int16)).view(torch.bfloat16).to(dev)
+        tdt = torch.bfloat16
+    else:
+        u_host = torch.from_numpy(data["u"])
+        k_dev = torch.from_numpy(data["k"]).to(dev)
+        tdt = torch.float32
+    u = u_host.to(dev)
+    D = torch.from_numpy(data["D"]).to(dev)
+    sc_w = torch.from_numpy(data["sc_w"]).to(dev) if data["sc_w"] is not None else None
+    spec = torch.empty(hb.hyena_spectrum_bytes(p.C, p.shape, p.order), dtype=torch.uint8, device=dev)
+    y = torch.empty((p.B, p.C) + p.shape, dtype=tdt, device=dev)
+    wsb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, p.shape, p.order)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+    stream = torch.cuda.current_stream()
+    hb.hyena_filter_spectrum(k_dev, D, p.C, p.shape, p.order, spec, stream)
+    torch.cuda.synchronize()
+
+    def step(uu=None):
+        hb.hyena_gated_fftconv(u if uu is None else uu, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws,
+                               stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    u_pin = u_host.pin_memory()
+    y_pin = torch.empty(y.shape, dtype=tdt).pin_memory()
+    u_e2e = torch.empty_like(u)
+    for _ in range(2):
+        u_e2e.copy_(u_pin, non_blocking=True)
+        step(u_e2e)
+        y_pin.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        u_e2e.copy_(u_pin, non_blocking=True)
+        step(u_e2e)
+        y_pin.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens_per_step = p.B * p.n
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    e2e_value = world * tokens_per_step * args.e2e_steps / (e2e_ms / 1e3)
+    peak, peak_kind = load_peaks()
+    spec_row = spectrum_row_bytes(p)
+    alg = algorithmic_bytes(p, spec_row)
+    avg_launch_s = float(np.mean(launch_ms)) / 1e3
+    achieved = alg / avg_launch_s / 1e9
+    kernel = "k_conv_onchip" if (p.ndim == 1 and p.L <= 16384) else ("multipass" if p.ndim == 1 else "grid2d")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if p.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": dict(config_of(p), parallelism=f"replicas{world}" if world > 1 else "single",
+                       l2="inputs larger than L2 (%.0f MB per step)" % (alg / 1e6)),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_8TBps": achieved / 8000.0,
+                     "traffic": committed_traffic(kernel, p.name),
+                     "algorithmic_bytes_per_launch": alg, "kernel": kernel,
+                     "avg_launch_us": avg_launch_s * 1e6},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": u.numel() * u.element_size(),
+                "d2h_bytes_per_step": y.numel() * y.element_size()},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(p)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+"""Thin ctypes binding of libhyena_b200.so (declared in include/hyena.h).
+
+Argument marshalling only: every step of the operator runs in the CUDA
+library.  Tensors are torch CUDA tensors (torch supplies device memory and
+streams); the functions take the same names as the C entry points.  There
+is no fallback: if the shared library is missing, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhyena_b200.so")
+
+HYENA_F32, HYENA_BF16 = 0, 1
+STATUS = {0: "HYENA_OK", 1: "HYENA_ERR_INVALID_ARG", 2: "HYENA_ERR_UNSUPPORTED_SHAPE",
+          3: "HYENA_ERR_MISALIGNED", 4: "HYENA_ERR_SPECTRUM_MISMATCH",
+          5: "HYENA_ERR_WORKSPACE_TOO_SMALL", 6: "HYENA_ERR_CUDA", 7: "HYENA_ERR_INTERNAL"}
+
+# every symbol include/hyena.h declares
+EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "hyena_spectrum_bytes",
+           "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
+           "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_spectrum_check"]
+
+_lock = threading.Lock()
+_lib = None
+
+
+class HyenaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m fft_long_convolution_02_b200.build`")
+        lib = ctypes.CDLL(path)
+        i64, vp, sz, fp = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        lib.hyena_version.restype = ctypes.c_int
+        lib.hyena_status_string.restype = ctypes.c_char_p
+        lib.hyena_status_string.argtypes = [ctypes.c_int]
+        lib.hyena_last_error_detail.restype = ctypes.c_char_p
+        lib.hyena_spectrum_bytes.restype = sz
+        lib.hyena_spectrum_bytes.argtypes = [i64, ctypes.c_int, i64p, ctypes.c_int]
+        lib.hyena_filter_spectrum.restype = ctypes.c_int
+        lib.hyena_filter_spectrum.argtypes = [vp, ctypes.c_int, fp, i64, ctypes.c_int, i64p, ctypes.c_int,
+                                              vp, sz, vp]
+        lib.hyena_shortconv.restype = ctypes.c_int
+        lib.hyena_shortconv.argtypes = [vp, vp, fp, fp, i64, i64, i64, ctypes.c_int, vp]
+        lib.hyena_gated_fftconv_workspace_bytes.restype = sz
+        lib.hyena_gated_fftconv_workspace_bytes.argtypes = [i64, i64, ctypes.c_int, i64p, ctypes.c_int]
+        lib.hyena_gated_fftconv_workspace_min_bytes.restype = sz
+        lib.hyena_gated_fftconv_workspace_min_bytes.argtypes = [i64, ctypes.c_int, i64p, ctypes.c_int]
+        lib.hyena_gated_fftconv.restype = ctypes.c_int
+        lib.hyena_gated_fftconv.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p, ctypes.c_int,
+                                            ctypes.c_int, vp, sz, vp]
+        lib.hyena_spectrum_check.restype = ctypes.c_int
+        lib.hyena_spectrum_check.argtypes = [vp, i64, ctypes.c_int, i64p, ctypes.c_int, vp]
+        _lib = lib
+    return _lib
+
+
+def _sizes(sizes):
+    sizes = [int(s) for s in sizes]
+    return (ctypes.c_int64 * len(sizes))(*sizes), len(sizes)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return HYENA_F32
+    if t.dtype == torch.bfloat16:
+        return HYENA_BF16
+    raise TypeError(f"unsupported tensor dtype {t.dtype}")
+
+
+def _check(rc: int):
+    if rc != 0:
+        detail = load().hyena_last_error_detail().decode()
+        raise HyenaError(rc, detail)
+
+
+def hyena_version() -> int:
+    return load().hyena_version()
+
+
+def hyena_spectrum_bytes(C: int, sizes, order: int) -> int:
+    arr, nd = _sizes(sizes)
+    return int(load().hyena_spectrum_bytes(C, nd, arr, order))
+
+
+def hyena_gated_fftconv_workspace_bytes(B: int, C: int, sizes, order: int) -> int:
+    arr, nd = _sizes(sizes)
+    return int(load().hyena_gated_fftconv_workspace_bytes(B, C, nd, arr, order))
+
+
+def hyena_gated_fftconv_workspace_min_bytes(C: int, sizes, order: int) -> int:
+    arr, nd = _sizes(sizes)
+    return int(load().hyena_gated_fftconv_workspace_min_bytes(C, nd, arr, order))
+
+
+def hyena_filter_spectrum(k, D, C: int, sizes, order: int, spectrum, stream=None) -> None:
+    """k: [order-1, C, *sizes] (f32/bf16 CUDA), D: [order-1, C] f32 or None,
+    spectrum: uint8 CUDA tensor of hyena_spectrum_bytes(...) bytes."""
+    arr, nd = _sizes(sizes)
+    _check(load().hyena_filter_spectrum(_ptr(k), _dtype_code(k), _ptr(D), C, nd, arr, order, _ptr(spectrum),
+                                        spectrum.numel() * spectrum.element_size(), _stream(stream)))
+
+
+def hyena_shortconv(u, out, w, bias=None, stream=None) -> None:
+    """u, out: [B, Ctot, L]; w: [Ctot, 3] f32; bias: [Ctot] f32 or None."""
+    B, Ctot, L = u.shape
+    _check(load().hyena_shortconv(_ptr(u), _ptr(out), _ptr(w), _ptr(bias), B, Ctot, L, _dtype_code(u),
+                                  _stream(stream)))
+
+
+def hyena_gated_fftconv(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int, workspace=None,
+                        stream=None) -> None:
+    """u: [B, (order+1)*C, *sizes], y: [B, C, *sizes] (same dtype), spectrum from
+    hyena_filter_spectrum, sc_w [(order+1)*C, 3] f32 or None, workspace uint8 or None."""
+    arr, nd = _sizes(sizes)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyena_gated_fftconv(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
+                                      _ptr(sc_w), _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
+                                      _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hyena_spectrum_check(spectrum, C: int, sizes, order: int, stream=None) -> None:
+    arr, nd = _sizes(sizes)
+    _check(load().hyena_spectrum_check(_ptr(spectrum), C, nd, arr, order, _stream(stream)))

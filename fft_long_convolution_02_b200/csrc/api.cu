@@ -1,0 +1,203 @@
+// api.cu -- the extern "C" boundary declared in include/hyena.h: argument
+// validation, planning, and dispatch to the kernel launchers.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "hyena.h"
+#include "kernels.h"
+#include "plan.h"
+
+using namespace hyena;
+
+namespace {
+
+thread_local std::string g_detail;
+
+hyena_status_t fail(hyena_status_t st, const std::string& why) {
+    g_detail = why;
+    return st;
+}
+
+hyena_status_t ok() {
+    g_detail.clear();
+    return HYENA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+size_t elem_size(hyena_dtype_t d) { return d == HYENA_BF16 ? 2 : 4; }
+
+bool valid_dtype(int d) { return d == HYENA_F32 || d == HYENA_BF16; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+hyena_status_t cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(HYENA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+hyena_status_t plan_or_fail(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p) {
+    std::string why;
+    if (C < 1) return fail(HYENA_ERR_INVALID_ARG, "C must be >= 1");
+    if (!sizes) return fail(HYENA_ERR_INVALID_ARG, "sizes is NULL");
+    if (ndim != 1 && ndim != 2) return fail(HYENA_ERR_INVALID_ARG, "ndim must be 1 or 2");
+    if (!make_plan(C, ndim, sizes, order, p, &why)) return fail(HYENA_ERR_UNSUPPORTED_SHAPE, why);
+    return HYENA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hyena_version(void) { return 100; }
+
+const char* hyena_status_string(hyena_status_t s) {
+    switch (s) {
+        case HYENA_OK: return "HYENA_OK";
+        case HYENA_ERR_INVALID_ARG: return "HYENA_ERR_INVALID_ARG";
+        case HYENA_ERR_UNSUPPORTED_SHAPE: return "HYENA_ERR_UNSUPPORTED_SHAPE";
+        case HYENA_ERR_MISALIGNED: return "HYENA_ERR_MISALIGNED";
+        case HYENA_ERR_SPECTRUM_MISMATCH: return "HYENA_ERR_SPECTRUM_MISMATCH";
+        case HYENA_ERR_WORKSPACE_TOO_SMALL: return "HYENA_ERR_WORKSPACE_TOO_SMALL";
+        case HYENA_ERR_CUDA: return "HYENA_ERR_CUDA";
+        case HYENA_ERR_INTERNAL: return "HYENA_ERR_INTERNAL";
+    }
+    return "HYENA_UNKNOWN_STATUS";
+}
+
+const char* hyena_last_error_detail(void) { return g_detail.c_str(); }
+
+size_t hyena_spectrum_bytes(int64_t C, int ndim, const int64_t* sizes, int order) {
+    Plan p;
+    std::string why;
+    if (!sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    return p.total_bytes;
+}
+
+hyena_status_t hyena_filter_spectrum(const void* k, hyena_dtype_t k_dtype, const float* D, int64_t C, int ndim,
+                                     const int64_t* sizes, int order, void* spectrum, size_t spectrum_bytes,
+                                     void* stream) {
+    Plan p;
+    hyena_status_t st = plan_or_fail(C, ndim, sizes, order, &p);
+    if (st != HYENA_OK) return st;
+    if (!k || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "k and spectrum must not be NULL");
+    if (!valid_dtype(k_dtype)) return fail(HYENA_ERR_INVALID_ARG, "k_dtype must be HYENA_F32 or HYENA_BF16");
+    if (!aligned16(k) || !aligned16(spectrum)) return fail(HYENA_ERR_MISALIGNED, "k and spectrum must be 16-byte aligned");
+    if (D && !aligned4(D)) return fail(HYENA_ERR_MISALIGNED, "D must be 4-byte aligned");
+    if (spectrum_bytes != p.total_bytes)
+        return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum_bytes must equal hyena_spectrum_bytes() = " +
+                                                      std::to_string(p.total_bytes));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* sp = static_cast<uint8_t*>(spectrum);
+    cudaError_t e = launch_header_and_tables(p, sp, s);
+    if (e != cudaSuccess) return cuda_status(e, "table fill");
+    SpectrumArgs a{k, int(k_dtype), D, sp};
+    switch (p.path) {
+        case PATH_ONCHIP_1D: e = launch_spectrum_onchip(p, a, s); break;
+        case PATH_MULTIPASS_1D: e = launch_spectrum_multipass(p, a, s); break;
+        case PATH_GRID_2D: e = launch_spectrum_2d(p, a, s); break;
+        default: return fail(HYENA_ERR_INTERNAL, "no path");
+    }
+    return cuda_status(e, "spectrum kernel");
+}
+
+hyena_status_t hyena_shortconv(const void* u, void* out, const float* w, const float* bias, int64_t B, int64_t Ctot,
+                               int64_t L, hyena_dtype_t dtype, void* stream) {
+    if (!u || !out || !w) return fail(HYENA_ERR_INVALID_ARG, "u, out and w must not be NULL");
+    if (!valid_dtype(dtype)) return fail(HYENA_ERR_INVALID_ARG, "dtype must be HYENA_F32 or HYENA_BF16");
+    if (B < 1 || Ctot < 1) return fail(HYENA_ERR_INVALID_ARG, "B and Ctot must be >= 1");
+    if (L < kMin1D || L > kMaxL || (L & (L - 1)) != 0)
+        return fail(HYENA_ERR_UNSUPPORTED_SHAPE, "L must be a power of two in [16, 2^20]");
+    if (!aligned16(u) || !aligned16(out)) return fail(HYENA_ERR_MISALIGNED, "u and out must be 16-byte aligned");
+    if (!aligned4(w) || (bias && !aligned4(bias))) return fail(HYENA_ERR_MISALIGNED, "w and bias must be 4-byte aligned");
+    const size_t nbytes = size_t(B) * size_t(Ctot) * size_t(L) * elem_size(dtype);
+    if (overlap(u, nbytes, out, nbytes)) return fail(HYENA_ERR_INVALID_ARG, "u and out overlap");
+    return cuda_status(launch_shortconv(u, out, w, bias, B, Ctot, L, int(dtype), static_cast<cudaStream_t>(stream)),
+                       "shortconv kernel");
+}
+
+size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_t* sizes, int order) {
+    Plan p;
+    std::string why;
+    if (!sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    return p.ws_row_bytes;
+}
+
+size_t hyena_gated_fftconv_workspace_bytes(int64_t B, int64_t C, int ndim, const int64_t* sizes, int order) {
+    Plan p;
+    std::string why;
+    if (B < 1 || !sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    return size_t(default_group_rows(p, B * C)) * p.ws_row_bytes;
+}
+
+hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    Plan p;
+    hyena_status_t st = plan_or_fail(C, ndim, sizes, order, &p);
+    if (st != HYENA_OK) return st;
+    if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
+    if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
+    if (!valid_dtype(dtype)) return fail(HYENA_ERR_INVALID_ARG, "dtype must be HYENA_F32 or HYENA_BF16");
+    if (ndim == 2 && sc_w) return fail(HYENA_ERR_INVALID_ARG, "the 2-D form has no short conv: sc_w must be NULL");
+    if (!aligned16(u) || !aligned16(y) || !aligned16(spectrum))
+        return fail(HYENA_ERR_MISALIGNED, "u, y and spectrum must be 16-byte aligned");
+    if ((sc_w && !aligned4(sc_w)) || (sc_bias && !aligned4(sc_bias)))
+        return fail(HYENA_ERR_MISALIGNED, "sc_w and sc_bias must be 4-byte aligned");
+    if (spectrum_bytes != p.total_bytes)
+        return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum_bytes must equal hyena_spectrum_bytes() = " +
+                                                      std::to_string(p.total_bytes));
+    const size_t es = elem_size(dtype);
+    const size_t ubytes = size_t(B) * size_t(order + 1) * size_t(C) * size_t(p.n) * es;
+    const size_t ybytes = size_t(B) * size_t(C) * size_t(p.n) * es;
+    if (overlap(u, ubytes, y, ybytes)) return fail(HYENA_ERR_INVALID_ARG, "u and y overlap");
+    int64_t group = 0;
+    if (p.ws_row_bytes > 0) {
+        if (!workspace || workspace_bytes < p.ws_row_bytes)
+            return fail(HYENA_ERR_WORKSPACE_TOO_SMALL,
+                        "workspace must hold at least " + std::to_string(p.ws_row_bytes) + " bytes");
+        if (!aligned16(workspace)) return fail(HYENA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+        if (overlap(workspace, workspace_bytes, y, ybytes) || overlap(workspace, workspace_bytes, u, ubytes) ||
+            overlap(workspace, workspace_bytes, spectrum, spectrum_bytes))
+            return fail(HYENA_ERR_INVALID_ARG, "workspace overlaps an operand");
+        group = int64_t(workspace_bytes / p.ws_row_bytes);
+        if (group > B * C) group = B * C;
+    }
+    ConvArgs a{u, y, static_cast<const uint8_t*>(spectrum), sc_w, sc_w ? sc_bias : nullptr, B, int(dtype),
+               static_cast<float2*>(workspace), group};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (p.path) {
+        case PATH_ONCHIP_1D: e = launch_conv_onchip(p, a, s); break;
+        case PATH_MULTIPASS_1D: e = launch_conv_multipass(p, a, s); break;
+        case PATH_GRID_2D: e = launch_conv_2d(p, a, s); break;
+        default: return fail(HYENA_ERR_INTERNAL, "no path");
+    }
+    return cuda_status(e, "gated fftconv kernel");
+}
+
+hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
+                                    void* stream) {
+    Plan p;
+    hyena_status_t st = plan_or_fail(C, ndim, sizes, order, &p);
+    if (st != HYENA_OK) return st;
+    if (!spectrum) return fail(HYENA_ERR_INVALID_ARG, "spectrum must not be NULL");
+    SpecHeader h{};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&h, spectrum, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e, "header read");
+    if (h.magic != kSpecMagic || h.version != kSpecVersion || h.path != p.path || h.C != p.C || h.L != p.L ||
+        h.H != p.H || h.W != p.W || h.order != p.order || size_t(h.total_bytes) != p.total_bytes)
+        return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum header does not match (C, sizes, order)");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// kernels.h -- internal launcher declarations (host side).  Every launcher
+// enqueues on the given stream and returns cudaGetLastError().
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plan.h"
+
+namespace hyena {
+
+enum DType { DT_F32 = 0, DT_BF16 = 1 };
+
+struct SpectrumArgs {
+    const void* k;        // [order-1, C, n]
+    int k_dtype;
+    const float* D;       // [order-1, C] or nullptr
+    uint8_t* spectrum;    // buffer start (header at offset 0)
+};
+
+struct ConvArgs {
+    const void* u;        // [B, (order+1)*C, n]
+    void* y;              // [B, C, n]
+    const uint8_t* spectrum;
+    const float* sc_w;    // [(order+1)*C, 3] or nullptr
+    const float* sc_b;    // [(order+1)*C] or nullptr
+    int64_t B;
+    int dtype;
+    float2* workspace;    // multi-pass / 2-D only
+    int64_t group_rows;   // rows per workspace group
+};
+
+cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);
+cudaError_t launch_spectrum_onchip(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+cudaError_t launch_conv_onchip(const Plan& p, const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_shortconv(const void* u, void* out, const float* w, const float* bias, int64_t B,
+                             int64_t Ctot, int64_t L, int dtype, cudaStream_t s);
+
+}  // namespace hyena

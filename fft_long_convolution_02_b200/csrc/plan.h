@@ -1,0 +1,89 @@
+// plan.h -- host-side planning for the Hyena gated FFT long convolution.
+//
+// A plan is a pure function of (C, ndim, sizes, order).  It fixes the kernel
+// path, the FFT factorisations, and the byte layout of the caller-owned
+// spectrum buffer:
+//
+//   [0, 256)               SpecHeader (magic, shape, layout offsets)
+//   [256, spec_off)        twiddle tables (float2, double-precision values
+//                          rounded to fp32), described by TableSpec entries
+//   [spec_off, total)      filter spectra, [order-1][C] rows of spec_row_bytes
+//
+// Paths (N = 2L zero-padded transform, computed as two M = L/2-point chains):
+//   PATH_ONCHIP_1D    16 <= L <= 16384: one CTA per (b, c) row, everything in
+//                     shared memory.  Spectrum row = (M+1) float4 pair entries.
+//   PATH_MULTIPASS_1D 32768 <= L <= 2^20: four-step M = M1 x M2 with three
+//                     passes through a caller workspace (kept L2-resident by
+//                     processing rows in groups).  Spectrum row = M1 units of
+//                     M2 float4 pair entries.
+//   PATH_GRID_2D      2-D H x W (16..512 each), zero-padded to 2H x 2W: a row
+//                     pass (packed real FFT of each image row), a column pass
+//                     (2H-point FFT, spectrum multiply, inverse) and an
+//                     inverse row pass.  Spectrum per channel = (W+1) columns
+//                     x 2H complex64 in the column pass's position order.
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace hyena {
+
+enum Path { PATH_NONE = 0, PATH_ONCHIP_1D = 1, PATH_MULTIPASS_1D = 2, PATH_GRID_2D = 3 };
+
+constexpr uint32_t kSpecMagic = 0x4853504Eu;  // "NPSH"
+constexpr uint32_t kSpecVersion = 1;
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxTableSpecs = 24;
+
+constexpr int64_t kOnchipMaxL = 16384;
+constexpr int64_t kMaxL = int64_t(1) << 20;
+constexpr int64_t kMin1D = 16;
+constexpr int64_t kMin2D = 16;
+constexpr int64_t kMax2D = 512;
+constexpr int kMaxOrder = 8;
+
+struct SpecHeader {
+    uint32_t magic, version;
+    int32_t ndim, order, path, reserved0;
+    int64_t C, L, H, W, M, M1, M2;
+    int64_t tables_off, tables_count, spec_off, spec_row_bytes, total_bytes;
+    int64_t reserved[17];
+};
+static_assert(sizeof(SpecHeader) == kHeaderBytes, "header must be 256 bytes");
+
+// entry[i][j] (i < na, j < nb) = w_N^(((a0 + i) (b0 + j) mult + add) mod N),
+// w_N = exp(-2 pi i / N), stored at tables[dst + i * nb + j].
+struct TableSpec {
+    int64_t dst, N, a0, na, b0, nb, mult, add;
+};
+struct TableSpecs {
+    TableSpec s[kMaxTableSpecs];
+    int n;
+    int64_t total;
+};
+
+struct Plan {
+    int ndim = 0, order = 0, path = PATH_NONE;
+    int64_t C = 0, L = 0, H = 0, W = 0;
+    int64_t M = 0, M1 = 0, M2 = 0;   // chain size; multi-pass factors; 2-D: M1 = W/2, M2 = H
+    int64_t n = 0;                   // samples per row (L or H*W)
+    // table offsets in float2 units from the start of the tables
+    int64_t t_fft_a = 0, t_fft_b = 0, t_twist = 0, t_untangle = 0, t_four = 0;
+    int64_t t_twist_hi = 0, t_twist_lo = 0, t_unt1 = 0, t_unt2 = 0, t_unt_c = 0, t_twist_h = 0;
+    TableSpecs specs{};
+    size_t tables_off = kHeaderBytes;
+    size_t spec_off = 0;
+    size_t spec_row_bytes = 0;
+    size_t total_bytes = 0;
+    // workspace (multi-pass and 2-D): bytes per (b, c) row in flight
+    size_t ws_row_bytes = 0;
+};
+
+// Returns false (and a reason) for unsupported shapes / orders.
+bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, std::string* why);
+
+// Default number of rows processed per group on the workspace paths.
+int64_t default_group_rows(const Plan& p, int64_t rows);
+
+}  // namespace hyena

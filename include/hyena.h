@@ -1,0 +1,163 @@
+/*
+ * hyena.h -- C ABI of the B200-native Hyena gated FFT long convolution.
+ *
+ * The operation ([P4] "HyenaDNA operator walk-through" (adg.csdn.net),
+ * section 二.1, HyenaOperator.forward, and section 二.2, fftconv; [P5]
+ * "Native Multi-Dimensional Subquadratic Operators via Input Dependent Long
+ * Convolutions", 方法论 -- 原生 ND 卷积 and 边界处理 -- for the 2-D form):
+ *
+ *   uc      = short_conv(u)            width-3 causal depthwise conv (optional)
+ *   x0..x(order-1), v = uc split along channels in blocks of C
+ *   for s = 1 .. order-1:
+ *       v = x_{order-s} * v                         (elementwise gate)
+ *       v = (k_s conv v)[0:L] + D_s * v              (causal long conv + skip)
+ *   y  = x0 * v
+ *
+ * The long convolution is evaluated as the 2L-point (2-D: 2H x 2W) zero-padded
+ * FFT product with a cached filter spectrum, which makes it non-circular.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them.  They must be 16-byte aligned.
+ *  - Tensors are row-major, last dimension contiguous: 1-D [.., L], 2-D
+ *    [.., H, W].  sizes = {L} for ndim 1, {H, W} for ndim 2.
+ *  - dtype selects the storage of u, y (and of k in hyena_filter_spectrum):
+ *    HYENA_F32 or HYENA_BF16 (round-to-nearest-even on store).  Arithmetic is
+ *    fp32 throughout; spectra are stored as complex64.
+ *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream) and is asynchronous: no call synchronises the host.
+ *  - Arguments are validated before anything is enqueued; on any error
+ *    nothing is launched and a status other than HYENA_OK is returned, with a
+ *    thread-local message available from hyena_last_error_detail().
+ *  - Supported shapes: 1-D L a power of two in [16, 2^20]; 2-D H, W powers of
+ *    two in [16, 512]; order in [2, 8]; C >= 1, B >= 1.
+ *  - The library keeps no state between calls; all entry points are
+ *    thread-safe.  Calls on one stream are ordered; calls that write the
+ *    same buffers from different streams race.
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype_t;
+
+typedef enum {
+    HYENA_OK = 0,
+    HYENA_ERR_INVALID_ARG = 1,        /* NULL pointer, bad dtype, B or C < 1, ...     */
+    HYENA_ERR_UNSUPPORTED_SHAPE = 2,  /* L / H / W / order outside the supported set  */
+    HYENA_ERR_MISALIGNED = 3,         /* a tensor pointer is not 16-byte aligned      */
+    HYENA_ERR_SPECTRUM_MISMATCH = 4,  /* spectrum_bytes does not match the shape      */
+    HYENA_ERR_WORKSPACE_TOO_SMALL = 5,/* workspace smaller than one row's share       */
+    HYENA_ERR_CUDA = 6,               /* a CUDA launch reported an error              */
+    HYENA_ERR_INTERNAL = 7
+} hyena_status_t;
+
+/* Version of this ABI (major * 100 + minor). */
+int hyena_version(void);
+
+/* Static name of a status code. */
+const char* hyena_status_string(hyena_status_t status);
+
+/* Thread-local description of the last error returned on this thread ("" if
+ * none).  Valid until the next call on the same thread. */
+const char* hyena_last_error_detail(void);
+
+/*
+ * Bytes of the spectrum buffer for C channels, shape sizes[ndim], order.
+ * Returns 0 for unsupported arguments.
+ */
+size_t hyena_spectrum_bytes(int64_t C, int ndim, const int64_t* sizes, int order);
+
+/*
+ * hyena_filter_spectrum -- S0, the filter-spectrum cache.
+ *
+ * Source: [P4] section 二.1 (k = filter(l) rearranged 'l (o d) -> o d l',
+ * bias 'o d'), section 二.2 (fftconv(v, k[o], bias[o])); the zero-padded FFT
+ * evaluation of the long convolution.
+ *
+ *   k        [order-1, C, sizes...] long filters in step order (k_dtype)
+ *   D        [order-1, C] fp32 skip ("bias") per step and channel, or NULL (= 0)
+ *   spectrum caller-allocated device buffer of spectrum_bytes =
+ *            hyena_spectrum_bytes(C, ndim, sizes, order) bytes; receives a
+ *            header, the twiddle tables of this shape (double-precision values
+ *            rounded to fp32) and, for every (step, channel), the zero-padded
+ *            spectrum of k with D folded in (D * v = (D delta) conv v) and the
+ *            inverse-FFT normalisation folded in.
+ *
+ * The buffer is the cache: keep it while k and D are unchanged and pass it to
+ * every hyena_gated_fftconv call with the same (C, sizes, order).
+ */
+hyena_status_t hyena_filter_spectrum(const void* k, hyena_dtype_t k_dtype, const float* D, int64_t C,
+                                     int ndim, const int64_t* sizes, int order, void* spectrum,
+                                     size_t spectrum_bytes, void* stream);
+
+/*
+ * hyena_shortconv -- S1 on its own (1-D only).
+ *
+ * Source: [P4] section 二.1, short_filter = Conv1d(inner, inner, 3, padding=2,
+ * groups=inner) truncated to the first L samples:
+ *   out[b, j, t] = w[j,0] u[b,j,t-2] + w[j,1] u[b,j,t-1] + w[j,2] u[b,j,t] + bias[j],
+ *   with u[.., t<0] = 0.
+ *
+ *   u, out [B, Ctot, L] (dtype); may not overlap.
+ *   w      [Ctot, 3] fp32;  bias [Ctot] fp32 or NULL (= 0).
+ */
+hyena_status_t hyena_shortconv(const void* u, void* out, const float* w, const float* bias, int64_t B,
+                               int64_t Ctot, int64_t L, hyena_dtype_t dtype, void* stream);
+
+/*
+ * Workspace bytes hyena_gated_fftconv uses for this shape by default (0 for
+ * the on-chip path, 1-D L <= 16384).  Any workspace at least as large as one
+ * row's share (hyena_gated_fftconv_workspace_min_bytes) is accepted; larger
+ * workspaces let more rows share each pass.
+ */
+size_t hyena_gated_fftconv_workspace_bytes(int64_t B, int64_t C, int ndim, const int64_t* sizes, int order);
+size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_t* sizes, int order);
+
+/*
+ * hyena_gated_fftconv -- S1..S9, the hot path.
+ *
+ * Source: [P4] section 二.1 (split *x, v = uc.split(d_model); for o, x_i in
+ * enumerate(reversed(x[1:])): v = v * x_i; v = fftconv(v, k[o], bias[o]);
+ * y = v * x[0]); [P5] 方法论 for ndim = 2 (non-circular global convolution by
+ * zero padding each axis to twice its length; output cropped to [0:H, 0:W],
+ * kernel anchored at (0, 0)).
+ *
+ *   u        [B, (order+1)*C, sizes...] projected stream, channel blocks in the
+ *            order x0, x1, ..., x(order-1), v (dtype)
+ *   y        [B, C, sizes...] output (dtype); may not overlap u
+ *   spectrum buffer filled by hyena_filter_spectrum for the same C, sizes,
+ *            order; spectrum_bytes must equal hyena_spectrum_bytes(...)
+ *   sc_w     [(order+1)*C, 3] fp32 short-conv taps applied to every chunk while
+ *            loading, or NULL when u is already short-convolved (1-D only;
+ *            must be NULL for ndim 2)
+ *   sc_bias  [(order+1)*C] fp32 or NULL (= 0); ignored when sc_w is NULL
+ *   workspace, workspace_bytes  device scratch for the multi-pass (L >= 32768)
+ *            and 2-D paths; may be NULL/0 for the on-chip path.  Its contents
+ *            are undefined after the call.
+ */
+hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * Debug helper (synchronous): copies the spectrum header to the host and
+ * checks it against (C, sizes, order).  Returns HYENA_OK when it matches,
+ * HYENA_ERR_SPECTRUM_MISMATCH when not (e.g. never filled, or filled for
+ * another shape).  Synchronises `stream`.
+ */
+hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
+                                    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_B200_H */

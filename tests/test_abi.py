@@ -1,0 +1,104 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fft_long_convolution_02_b200 import binding as hb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fft_long_convolution_02_b200 import build
+    build.build()
+    return hb.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hyena.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyena_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(hb.EXPORTS) == names
+
+
+def test_version_and_status_strings(lib):
+    assert lib.hyena_version() == 100
+    for code, name in hb.STATUS.items():
+        assert lib.hyena_status_string(code).decode() == name
+
+
+def _sz(*s):
+    return (ctypes.c_int64 * len(s))(*s)
+
+
+def test_spectrum_bytes_and_workspace(lib):
+    # on-chip: header + tables + (order-1) C (L/2+1) 16 bytes
+    b = lib.hyena_spectrum_bytes(768, 1, _sz(8192), 2)
+    assert b >= 768 * (4096 + 1) * 16 and b < 768 * (4096 + 1) * 16 + (1 << 20)
+    assert lib.hyena_gated_fftconv_workspace_bytes(4, 768, 1, _sz(8192), 2) == 0
+    # multi-pass: spectrum rows of 8L bytes, workspace 8L bytes per row
+    L = 1 << 20
+    b = lib.hyena_spectrum_bytes(256, 1, _sz(L), 2)
+    assert 256 * 8 * L <= b < 256 * 8 * L + (64 << 20)
+    assert lib.hyena_gated_fftconv_workspace_min_bytes(256, 1, _sz(L), 2) == 8 * L
+    # 2-D: (W+1) * 2H complex64 per channel
+    b = lib.hyena_spectrum_bytes(256, 2, _sz(256, 256), 2)
+    assert 256 * 257 * 512 * 8 <= b < 256 * 257 * 512 * 8 + (1 << 20)
+    # unsupported shapes
+    for bad in [(1, _sz(12), 2), (1, _sz(8), 2), (1, _sz(1 << 21), 2), (2, _sz(16, 1024), 2),
+                (1, _sz(1024), 1), (1, _sz(1024), 9)]:
+        assert lib.hyena_spectrum_bytes(64, *bad) == 0
+
+
+def _detail(lib):
+    return lib.hyena_last_error_detail().decode()
+
+
+def test_validation_errors_before_launch(lib):
+    fake = 1 << 20            # never dereferenced: validation fails first
+    sizes = _sz(1024)
+    nbytes = lib.hyena_spectrum_bytes(64, 1, sizes, 2)
+    gf = lib.hyena_gated_fftconv
+    # NULL tensors
+    assert gf(None, fake, fake, nbytes, None, None, 1, 64, 1, sizes, 2, 0, None, 0, None) == 1
+    # bad dtype
+    assert gf(fake, fake * 4, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 7, None, 0, None) == 1
+    # unsupported length / order
+    assert gf(fake, fake * 4, fake * 8, nbytes, None, None, 1, 64, 1, _sz(1000), 2, 0, None, 0, None) == 2
+    assert gf(fake, fake * 4, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 1, 0, None, 0, None) == 2
+    # misaligned pointers
+    assert gf(fake + 4, fake * 4, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0, None, 0, None) == 3
+    assert "16-byte" in _detail(lib)
+    # spectrum size mismatch
+    assert gf(fake, fake * 4, fake * 8, nbytes + 16, None, None, 1, 64, 1, sizes, 2, 0, None, 0, None) == 4
+    # overlapping u and y
+    assert gf(fake, fake + 64, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0, None, 0, None) == 1
+    # 2-D with a short conv
+    s2 = _sz(32, 32)
+    n2 = lib.hyena_spectrum_bytes(8, 2, s2, 2)
+    ws = lib.hyena_gated_fftconv_workspace_bytes(1, 8, 2, s2, 2)
+    assert gf(fake, fake * 4, fake * 8, n2, fake * 16, None, 1, 8, 2, s2, 2, 0, fake * 32, ws, None) == 1
+    # workspace too small on a workspace path
+    assert gf(fake, fake * 4, fake * 8, n2, None, None, 1, 8, 2, s2, 2, 0, None, 0, None) == 5
+    # B < 1
+    assert gf(fake, fake * 4, fake * 8, nbytes, None, None, 0, 64, 1, sizes, 2, 0, None, 0, None) == 1
+    # filter spectrum: size mismatch and NULLs
+    fs = lib.hyena_filter_spectrum
+    assert fs(fake, 0, None, 64, 1, sizes, 2, fake * 8, nbytes - 16, None) == 4
+    assert fs(None, 0, None, 64, 1, sizes, 2, fake * 8, nbytes, None) == 1
+    # short conv
+    sc = lib.hyena_shortconv
+    assert sc(fake, fake * 4, None, None, 1, 3, 64, 0, None) == 1
+    assert sc(fake, fake * 4, fake * 8, None, 1, 3, 63, 0, None) == 2
+    assert sc(fake, fake + 16, fake * 8, None, 1, 3, 64, 0, None) == 1
