@@ -1,6 +1,389 @@
-// grid2d.cu -- placeholder launchers.
+// grid2d.cu -- the 2-D non-circular form (H x W grids, 16..512 each).
+//
+// [P5] "Native Multi-Dimensional Subquadratic Operators via Input Dependent
+// Long Convolutions", 方法论 (原生 ND 卷积, 边界处理): the global convolution
+// runs on the native grid through an N-D FFT, made non-circular by zero
+// padding every axis to twice its length; with the gating of [P4] section
+// 二.1 (v <- x_{order-s} * v, conv, y = x0 * v).  Kernel anchored at (0,0),
+// output cropped to [0:H, 0:W].
+//
+// The 2H x 2W transform of a real, zero-padded image is evaluated as:
+//   row pass (A2)    each image row: packed real FFT of length 2W via two
+//                    W/2-point chains + untangle -> bins fq = 0..W (W+1 of them)
+//                    -> workspace [fq][p]
+//   column pass (B2) each bin column fq: 2H-point FFT of the zero-padded column
+//                    (two H-point chains), times K~, inverse, keep p < H
+//   row pass (C2)    re-tangle, inverse row chains, output gate -> y
+// K~[fp][fq] = (DFT_2Hx2W(k padded)[fp][fq] + D) / (8 H W) is stored per
+// channel as [fq][chain][position] so the column pass multiplies in the
+// digit-reversed order its forward DIF leaves behind.
+#include "common.cuh"
+#include "cta_fft.cuh"
 #include "kernels.h"
+
 namespace hyena {
-cudaError_t launch_spectrum_2d(const Plan&, const SpectrumArgs&, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_conv_2d(const Plan&, const ConvArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+constexpr int kRB = 16;        // image rows per CTA in the row passes
+constexpr int kCB = 4;         // bin columns per CTA in the column pass
+constexpr int kRowThreads = 256;
+constexpr int kColThreads2 = 128;
+
+struct T2d {
+    const float2* fftW;     // CTA FFT of size W/2
+    const float2* fftH;     // CTA FFT of size H
+    const float2* twist_w;  // w_W^n, n < W/2
+    const float2* untw;     // pair twiddles w_2W^f, chain e then chain o
+    const float2* twist_h;  // w_2H^p, p < H
+};
+
+T2d t2d(const Plan& p, const uint8_t* spectrum) {
+    const float2* t = reinterpret_cast<const float2*>(spectrum + p.tables_off);
+    return T2d{t + p.t_fft_a, t + p.t_fft_b, t + p.t_twist, t + p.t_untangle, t + p.t_twist_h};
 }
+
+template <int MW>
+__device__ __forceinline__ float2* rowbuf(float2* smem, int ch, int r) {
+    return smem + (ch * kRB + r) * fft_padded_size(MW);
+}
+
+// Row forward: rows of z (already in smem at natural positions) -> DIF ->
+// untangle -> ws[fq][p0 + r] for fq in [0, W].
+template <int MW>
+__device__ __forceinline__ void rows_forward_store(float2* smem, const T2d& tb, float2* __restrict__ ws_img,
+                                                   int H, int p0, float dscale, float d) {
+    constexpr int W = 2 * MW;
+    __syncthreads();
+    cta_fft_forward<MW>(smem, 2 * kRB, fft_padded_size(MW), tb.fftW);
+    // pairs q: chain e q = 0..MW/2, chain o q = MW/2+1..MW; rows r fastest
+    for (int idx = threadIdx.x; idx < (MW + 1) * kRB; idx += blockDim.x) {
+        const int q = idx / kRB;
+        const int r = idx - q * kRB;
+        const bool odd = q > MW / 2;
+        const int j = odd ? q - (MW / 2 + 1) : q;
+        const float2* buf = rowbuf<MW>(smem, odd ? 1 : 0, r);
+        const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
+        const float2 A = buf[fft_pad(fft_bin_pos<MW>(j))];
+        const float2 B = buf[fft_pad(fft_bin_pos<MW>(mb))];
+        const int f = odd ? 2 * j + 1 : 2 * j;
+        const int g = W - f;
+        float2 Xf, Xg;
+        if (q == 0) {
+            Xf = make_float2(2.0f * (A.x + A.y), 0.0f);
+            Xg = make_float2(2.0f * (A.x - A.y), 0.0f);
+        } else {
+            const float2 w = __ldg(tb.untw + q);
+            const float2 S = cadd(A, cconj(B));
+            const float2 T = cmul_i(cmul(w, csub(A, cconj(B))));
+            Xf = csub(S, T);
+            Xg = cconj(cadd(S, T));
+        }
+        // dscale/d turn X2 into the stored quantity (spectrum build) or leave it
+        Xf = make_float2(Xf.x * dscale + d, Xf.y * dscale);
+        Xg = make_float2(Xg.x * dscale + d, Xg.y * dscale);
+        ws_img[int64_t(f) * H + p0 + r] = Xf;
+        if (g != f) ws_img[int64_t(g) * H + p0 + r] = Xg;
+    }
+}
+
+// MODE 0: gated input x_{order-1} * v from u; MODE 1: the filter k.
+template <int MW, typename T, int MODE>
+__global__ void __launch_bounds__(kRowThreads)
+k_2d_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
+              int64_t img0, int64_t ws_img_stride, int64_t ws_img_offset) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * kRB;
+    const int64_t n = int64_t(H) * W;
+    const T* xg;
+    const T* vr = nullptr;
+    if (MODE == 0) {
+        const int64_t c = img / B, b = img - (img / B) * B;
+        const int64_t Ctot = int64_t(order + 1) * C;
+        const T* ub = src + b * Ctot * n;
+        xg = ub + (int64_t(order - 1) * C + c) * n;
+        vr = ub + (int64_t(order) * C + c) * n;
+    } else {
+        xg = src + img * n;
+    }
+    for (int idx = threadIdx.x; idx < kRB * MW; idx += blockDim.x) {
+        const int r = idx / MW;
+        const int nn = idx - r * MW;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        float2 z = load2(xg + off);
+        if (MODE == 0) {
+            const float2 v = load2(vr + off);
+            z = make_float2(z.x * v.x, z.y * v.y);
+        }
+        rowbuf<MW>(smem, 0, r)[fft_pad(nn)] = z;
+        rowbuf<MW>(smem, 1, r)[fft_pad(nn)] = cmul(z, __ldg(tb.twist_w + nn));
+    }
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
+    rows_forward_store<MW>(smem, tb, ws_img, H, p0, 1.0f, 0.0f);
+}
+
+// Column pass.  MODE 0: convolution in place.  MODE 1: spectrum build, one
+// CTA per (step, channel) walking the bin columns in increasing order (the
+// row-pass output sits in the upper half of the channel's region).
+template <int MH, int MODE>
+__global__ void __launch_bounds__(kColThreads2)
+k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
+          int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, const float* __restrict__ D, float s8) {
+    extern __shared__ float2 smem[];
+    constexpr int PS = fft_padded_size(MH);
+    const int64_t img = img0 + blockIdx.y;
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    const int ncol = W + 1;
+    const float2* sp = nullptr;
+    float d = 0.0f;
+    if (MODE == 0) {
+        const int64_t c = img / B;
+        sp = spec + (int64_t(step) * C + c) * spec_row_stride;
+    } else {
+        d = D ? __ldg(D + img) : 0.0f;
+    }
+    const int f_begin = MODE == 0 ? int(blockIdx.x) * kCB : 0;
+    const int f_end = MODE == 0 ? min(f_begin + kCB, ncol) : ncol;
+    const int per = MODE == 0 ? kCB : 1;
+    for (int f0 = f_begin; f0 < f_end; f0 += per) {
+        const int nc = min(per, f_end - f0);
+        const float2* src = MODE == 0 ? ws_img : ws_img + int64_t(ncol) * MH;   // spectrum build: upper half
+        for (int idx = threadIdx.x; idx < nc * MH; idx += blockDim.x) {
+            const int cc = idx / MH;
+            const int p = idx - cc * MH;
+            const float2 v = src[int64_t(f0 + cc) * MH + p];
+            smem[(2 * cc) * PS + fft_pad(p)] = v;
+            smem[(2 * cc + 1) * PS + fft_pad(p)] = cmul(v, __ldg(tb.twist_h + p));
+        }
+        __syncthreads();
+        cta_fft_forward<MH>(smem, 2 * nc, PS, tb.fftH);
+        if (MODE == 0) {
+            for (int idx = threadIdx.x; idx < 2 * nc * MH; idx += blockDim.x) {
+                const int tcol = idx / MH;            // 2*cc + chain
+                const int pos = idx - tcol * MH;
+                const int cc = tcol >> 1, ch = tcol & 1;
+                const float2 k = __ldg(sp + int64_t(f0 + cc) * (2 * MH) + ch * MH + pos);
+                float2* e = smem + tcol * PS + fft_pad(pos);
+                *e = cmul(*e, k);
+            }
+            __syncthreads();
+            cta_fft_inverse<MH>(smem, 2 * nc, PS, tb.fftH);
+            for (int idx = threadIdx.x; idx < nc * MH; idx += blockDim.x) {
+                const int cc = idx / MH;
+                const int p = idx - cc * MH;
+                const float2 e = smem[(2 * cc) * PS + fft_pad(p)];
+                const float2 o = smem[(2 * cc + 1) * PS + fft_pad(p)];
+                ws_img[int64_t(f0 + cc) * MH + p] = cadd(e, cmulc(o, __ldg(tb.twist_h + p)));
+            }
+        } else {
+            // K~ = (X2D / 2 + D) * s8, positions in order, chain e then chain o
+            for (int idx = threadIdx.x; idx < 2 * MH; idx += blockDim.x) {
+                const int ch = idx / MH;
+                const int pos = idx - ch * MH;
+                const float2 v = smem[ch * PS + fft_pad(pos)];
+                ws_img[int64_t(f0) * (2 * MH) + idx] = make_float2((0.5f * v.x + d) * s8, 0.5f * v.y * s8);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Row inverse pass: re-tangle, inverse row chains, output gate (FINAL) or
+// next gate + next step's row forward pass.
+template <int MW, typename T, bool FINAL>
+__global__ void __launch_bounds__(kRowThreads)
+k_2d_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C,
+              int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * kRB;
+    const int64_t n = int64_t(H) * W;
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    for (int idx = threadIdx.x; idx < (MW + 1) * kRB; idx += blockDim.x) {
+        const int q = idx / kRB;
+        const int r = idx - q * kRB;
+        const bool odd = q > MW / 2;
+        const int j = odd ? q - (MW / 2 + 1) : q;
+        float2* buf = rowbuf<MW>(smem, odd ? 1 : 0, r);
+        const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
+        const int f = odd ? 2 * j + 1 : 2 * j;
+        const int g = W - f;
+        const float2 Yf = ws_img[int64_t(f) * H + p0 + r];
+        const float2 Yg = ws_img[int64_t(g) * H + p0 + r];
+        const float2 w = (q == 0) ? make_float2(1.0f, 0.0f) : __ldg(tb.untw + q);
+        const float2 P = cadd(Yf, cconj(Yg));
+        const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+        buf[fft_pad(fft_bin_pos<MW>(j))] = cadd(P, U);
+        if (q != 0) buf[fft_pad(fft_bin_pos<MW>(mb))] = cconj(csub(P, U));
+    }
+    __syncthreads();
+    cta_fft_inverse<MW>(smem, 2 * kRB, fft_padded_size(MW), tb.fftW);
+    const int64_t c = img / B, b = img - (img / B) * B;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const T* ub = u + b * Ctot * n;
+    const int gate = FINAL ? 0 : gnext;
+    const T* xg = ub + (int64_t(gate) * C + c) * n;
+    T* yr = y + (b * C + c) * n;
+    for (int idx = threadIdx.x; idx < kRB * MW; idx += blockDim.x) {
+        const int r = idx / MW;
+        const int nn = idx - r * MW;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        float2* e = rowbuf<MW>(smem, 0, r) + fft_pad(nn);
+        float2* o = rowbuf<MW>(smem, 1, r) + fft_pad(nn);
+        const float2 tw = __ldg(tb.twist_w + nn);
+        const float2 zp = cadd(*e, cmulc(*o, tw));
+        const float2 x = load2(xg + off);
+        const float2 z = make_float2(x.x * zp.x, x.y * zp.y);
+        if (FINAL) {
+            store2(yr + off, z);
+        } else {
+            *e = z;
+            *o = cmul(z, tw);
+        }
+    }
+    if (!FINAL) rows_forward_store<MW>(smem, tb, ws_img, H, p0, 1.0f, 0.0f);
+}
+
+template <int MW>
+size_t row_smem() {
+    return size_t(2) * kRB * fft_padded_size(MW) * sizeof(float2);
+}
+
+template <int MH>
+size_t col_smem2(int per) {
+    return size_t(2) * per * fft_padded_size(MH) * sizeof(float2);
+}
+
+template <int MW, int MH>
+cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    float2* rows = reinterpret_cast<float2*>(a.spectrum + p.spec_off);
+    const int64_t nimg = (p.order - 1) * p.C;
+    const int64_t stride = int64_t(p.spec_row_bytes / sizeof(float2));    // (W+1) * 2H
+    const int H = int(p.H), W = int(p.W);
+    const size_t smA = row_smem<MW>();
+    const size_t smB = col_smem2<MH>(1);
+    auto kf = k_2d_rows_fwd<MW, float, 1>;
+    auto kh = k_2d_rows_fwd<MW, __nv_bfloat16, 1>;
+    auto kb = k_2d_cols<MH, 1>;
+    cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    const float s8 = 1.0f / (8.0f * float(H) * float(W));
+    for (int64_t i0 = 0; i0 < nimg; i0 += 32768) {
+        const int64_t g = nimg - i0 < 32768 ? nimg - i0 : 32768;
+        const dim3 gridA(H / kRB, unsigned(g));
+        // row pass output goes to the upper half of each channel's region
+        const int64_t upper = int64_t(W + 1) * H;
+        if (a.k_dtype == DT_F32)
+            kf<<<gridA, kRowThreads, smA, s>>>(static_cast<const float*>(a.k), rows + i0 * stride, tb, 1, 1, 2, H, i0,
+                                               stride, upper);
+        else
+            kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
+                                               2, H, i0, stride, upper);
+        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, nullptr, tb, W, 1, p.C, 0, i0, stride,
+                                                           0, a.D, s8);
+    }
+    return cudaGetLastError();
+}
+
+template <int MW, int MH, typename T>
+cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    const float2* spec = reinterpret_cast<const float2*>(a.spectrum + p.spec_off);
+    const T* u = static_cast<const T*>(a.u);
+    T* y = static_cast<T*>(a.y);
+    const int64_t nimg = a.B * p.C;
+    const int64_t G = a.group_rows < 65535 ? a.group_rows : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
+    const int64_t spec_stride = int64_t(p.spec_row_bytes / sizeof(float2));
+    const int H = int(p.H), W = int(p.W);
+    const size_t smA = row_smem<MW>();
+    const size_t smB = col_smem2<MH>(kCB);
+    auto ka = k_2d_rows_fwd<MW, T, 0>;
+    auto kb = k_2d_cols<MH, 0>;
+    auto kc = k_2d_rows_inv<MW, T, true>;
+    auto kca = k_2d_rows_inv<MW, T, false>;
+    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    const unsigned ncolblk = unsigned((W + 1 + kCB - 1) / kCB);
+    for (int64_t i0 = 0; i0 < nimg; i0 += G) {
+        const int64_t g = nimg - i0 < G ? nimg - i0 : G;
+        const dim3 gridR(H / kRB, unsigned(g));
+        ka<<<gridR, kRowThreads, smA, s>>>(u, a.workspace, tb, a.B, p.C, p.order, H, i0, stride, 0);
+        for (int st = 1; st < p.order; ++st) {
+            kb<<<dim3(ncolblk, unsigned(g)), kColThreads2, smB, s>>>(a.workspace, spec, tb, W, a.B, p.C, st - 1, i0,
+                                                                     stride, spec_stride, nullptr, 0.0f);
+            if (st < p.order - 1)
+                kca<<<gridR, kRowThreads, smA, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, p.order - st - 1, H, i0,
+                                                     stride);
+            else
+                kc<<<gridR, kRowThreads, smA, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, 0, H, i0, stride);
+        }
+    }
+    return cudaGetLastError();
+}
+
+template <int MW, int MH>
+cudaError_t conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    return a.dtype == DT_F32 ? conv_2d_t<MW, MH, float>(p, a, s) : conv_2d_t<MW, MH, __nv_bfloat16>(p, a, s);
+}
+
+template <int MW>
+cudaError_t dispatch_h_spec(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    switch (p.H) {
+        case 16: return spectrum_2d_t<MW, 16>(p, a, s);
+        case 32: return spectrum_2d_t<MW, 32>(p, a, s);
+        case 64: return spectrum_2d_t<MW, 64>(p, a, s);
+        case 128: return spectrum_2d_t<MW, 128>(p, a, s);
+        case 256: return spectrum_2d_t<MW, 256>(p, a, s);
+        case 512: return spectrum_2d_t<MW, 512>(p, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int MW>
+cudaError_t dispatch_h_conv(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    switch (p.H) {
+        case 16: return conv_2d<MW, 16>(p, a, s);
+        case 32: return conv_2d<MW, 32>(p, a, s);
+        case 64: return conv_2d<MW, 64>(p, a, s);
+        case 128: return conv_2d<MW, 128>(p, a, s);
+        case 256: return conv_2d<MW, 256>(p, a, s);
+        case 512: return conv_2d<MW, 512>(p, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    switch (p.W) {
+        case 16: return dispatch_h_spec<8>(p, a, s);
+        case 32: return dispatch_h_spec<16>(p, a, s);
+        case 64: return dispatch_h_spec<32>(p, a, s);
+        case 128: return dispatch_h_spec<64>(p, a, s);
+        case 256: return dispatch_h_spec<128>(p, a, s);
+        case 512: return dispatch_h_spec<256>(p, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    switch (p.W) {
+        case 16: return dispatch_h_conv<8>(p, a, s);
+        case 32: return dispatch_h_conv<16>(p, a, s);
+        case 64: return dispatch_h_conv<32>(p, a, s);
+        case 128: return dispatch_h_conv<64>(p, a, s);
+        case 256: return dispatch_h_conv<128>(p, a, s);
+        case 512: return dispatch_h_conv<256>(p, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace hyena

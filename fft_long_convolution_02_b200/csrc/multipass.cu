@@ -1,6 +1,433 @@
-// multipass.cu -- placeholder launchers (implemented below in this file).
+// multipass.cu -- the four-step path for 32768 <= L <= 2^20.
+//
+// Same method as the on-chip path ([P4] "HyenaDNA operator walk-through"
+// (adg.csdn.net), section 二.1 gating loop, section 二.2 fftconv; zero-padded
+// 2L FFT as two M = L/2-point chains with a pairwise untangle / spectrum
+// multiply / re-tangle), but an M-point chain no longer fits in one SM, so
+// each chain DFT is split four-step style with M = M1 * M2,
+// n = M2 n1 + n2, m = m1 + M1 m2:
+//
+//   DFT_M(x)[m1 + M1 m2] = sum_n2 w_M2^(n2 m2) w_M^(n2 m1) sum_n1 x[M2 n1 + n2] w_M1^(n1 m1)
+//
+//   pass A  (per block of 16 columns n2): gated input -> column DFT_M1 for
+//           both chains -> times w_M^(m1 n2) -> workspace
+//   pass B  (per unit = two rows m1 that hold every partner bin): row DFT_M2,
+//           pair step with the spectrum, row IDFT_M2 -> workspace (in place)
+//   pass C  (per block of columns): times w_M^(-m1 n2) -> column IDFT_M1 ->
+//           combine the chains -> output gate -> y; for order > 2 the next
+//           gate and the next step's pass A run in the same kernel (pass CA)
+//
+// Workspace row layout (complex64): [chain e | chain o], each M1 rows of M2
+// stored as M1/2 "units" of two rows.  Chain e unit 0 holds rows (0, M1/2),
+// unit u > 0 rows (u, M1-u); chain o unit u holds rows (u, M1-1-u).  Bin
+// m = m1 + M1 m2 pairs with M-m (chain e) or M-1-m (chain o), which always
+// lies in the same unit, so pass B needs nothing outside its unit.
+// The spectrum row has the same shape: one float4 pair entry per workspace
+// complex pair, written in place by the spectrum build.
+//
+// Rows are processed in groups sized to the caller's workspace (default
+// about 48 MB) so the intermediate data stays in the 126 MB L2 between passes.
+#include "common.cuh"
+#include "cta_fft.cuh"
 #include "kernels.h"
+
 namespace hyena {
-cudaError_t launch_spectrum_multipass(const Plan&, const SpectrumArgs&, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_conv_multipass(const Plan&, const ConvArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+constexpr int kNB2 = 16;          // columns per CTA in passes A and C
+constexpr int kColThreads = 256;
+
+struct MpTables {
+    const float2* fftA;     // CTA FFT of size M1
+    const float2* fftB;     // CTA FFT of size M2
+    const float2* four;     // w_M^(m1 n2), [M1][M2]
+    const float2* twist_hi; // w_L^(M2 n1)
+    const float2* twist_lo; // w_L^(n2)
+    const float2* unt1;     // w_L^(m1)
+    const float2* unt2;     // w_(2 M2)^(m2)
+    const float2* unt_c;    // w_2L^1
+};
+
+MpTables mp_tables(const Plan& p, const uint8_t* spectrum) {
+    const float2* t = reinterpret_cast<const float2*>(spectrum + p.tables_off);
+    return MpTables{t + p.t_fft_a, t + p.t_fft_b, t + p.t_four, t + p.t_twist_hi,
+                    t + p.t_twist_lo, t + p.t_unt1, t + p.t_unt2, t + p.t_unt_c};
 }
+
+// (unit, which) slot of row m1 in a chain's workspace block.
+template <int M1>
+__device__ __forceinline__ int mp_slot(bool odd, int m1) {
+    if (!odd) {
+        if (m1 == 0) return 0;
+        if (m1 == M1 / 2) return 1;
+        return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - m1) + 1;
+    }
+    return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - 1 - m1) + 1;
+}
+
+__device__ __forceinline__ float2 twist_of(const MpTables& tb, int n1, int n2) {
+    return cmul(__ldg(tb.twist_hi + n1), __ldg(tb.twist_lo + n2));
+}
+
+// Column block in shared memory: chain ch, column j, padded row index.
+template <int M1>
+__device__ __forceinline__ float2* col_ptr(float2* smem, int ch, int j) {
+    return smem + (ch * kNB2 + j) * fft_padded_size(M1);
+}
+
+// Forward column DFT of both chains, four-step twiddle, store to the
+// workspace (or the spectrum row when building the spectrum).
+template <int M1>
+__device__ __forceinline__ void cols_forward_store(float2* smem, const MpTables& tb, float2* __restrict__ ws_row,
+                                                   int M2, int n2_0) {
+    __syncthreads();
+    cta_fft_forward<M1>(smem, 2 * kNB2, fft_padded_size(M1), tb.fftA);
+    const int M = M1 * M2;
+    for (int idx = threadIdx.x; idx < 2 * M1 * kNB2; idx += blockDim.x) {
+        const int ch = idx / (M1 * kNB2);
+        const int rem = idx - ch * (M1 * kNB2);
+        const int m1 = rem / kNB2;
+        const int j = rem - m1 * kNB2;
+        const int n2 = n2_0 + j;
+        float2 v = col_ptr<M1>(smem, ch, j)[fft_pad(fft_bin_pos<M1>(m1))];
+        v = cmul(v, __ldg(tb.four + int64_t(m1) * M2 + n2));
+        ws_row[int64_t(ch) * M + int64_t(mp_slot<M1>(ch == 1, m1)) * M2 + n2] = v;
+    }
+}
+
+// ------------------------------------------------------------------ pass A
+// MODE 0: gated input from u (first order step); MODE 1: the filter k.
+template <int M1, typename T, int MODE>
+__global__ void __launch_bounds__(kColThreads)
+k_mp_pass_a(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, const float* __restrict__ sc_w,
+            const float* __restrict__ sc_b, int64_t B, int64_t C, int order, int M2, int64_t row0,
+            int64_t ws_row_stride) {
+    extern __shared__ float2 smem[];
+    const int64_t r = row0 + blockIdx.y;
+    const int n2_0 = blockIdx.x * kNB2;
+    const int64_t L = int64_t(2) * M1 * M2;
+    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    const T* xg;
+    const T* vr = nullptr;
+    Taps tg{}, tv{};
+    if (MODE == 0) {
+        const int64_t c = r / B, b = r - (r / B) * B;
+        const int64_t Ctot = int64_t(order + 1) * C;
+        const T* ub = src + b * Ctot * L;
+        const int g = order - 1;
+        xg = ub + (int64_t(g) * C + c) * L;
+        vr = ub + (int64_t(order) * C + c) * L;
+        tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
+        tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+    } else {
+        xg = src + r * L;
+    }
+    for (int idx = threadIdx.x; idx < M1 * kNB2; idx += blockDim.x) {
+        const int n1 = idx / kNB2;
+        const int j = idx - n1 * kNB2;
+        const int n2 = n2_0 + j;
+        const int64_t t = 2 * (int64_t(M2) * n1 + n2);
+        float2 z;
+        if (MODE == 0) {
+            const float2 a = shortconv_pair(xg, t, tg);
+            const float2 v = shortconv_pair(vr, t, tv);
+            z = make_float2(a.x * v.x, a.y * v.y);
+        } else {
+            z = load2(xg + t);
+        }
+        col_ptr<M1>(smem, 0, j)[fft_pad(n1)] = z;
+        col_ptr<M1>(smem, 1, j)[fft_pad(n1)] = cmul(z, twist_of(tb, n1, n2));
+    }
+    cols_forward_store<M1>(smem, tb, ws_row, M2, n2_0);
+}
+
+// ------------------------------------------------------------------ pass B
+// The pair step for one pair entry: A at bin m (row a), B at its partner.
+__device__ __forceinline__ void pair_conv(float2& A, float2& Bv, float2 w, float4 kk) {
+    const float2 S = cadd(A, cconj(Bv));
+    const float2 T = cmul_i(cmul(w, csub(A, cconj(Bv))));
+    const float2 Yf = cmul(csub(S, T), make_float2(kk.x, kk.y));
+    const float2 Yg = cmul(cconj(cadd(S, T)), make_float2(kk.z, kk.w));
+    const float2 P = cadd(Yf, cconj(Yg));
+    const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+    A = cadd(P, U);
+    Bv = cconj(csub(P, U));
+}
+
+__device__ __forceinline__ float4 pair_spec(float2 A, float2 Bv, float2 w, float d, float s4) {
+    const float2 S = cadd(A, cconj(Bv));
+    const float2 T = cmul_i(cmul(w, csub(A, cconj(Bv))));
+    const float2 Xf = cscale(csub(S, T), 0.5f);
+    const float2 Xg = cscale(cconj(cadd(S, T)), 0.5f);
+    return make_float4((Xf.x + d) * s4, Xf.y * s4, (Xg.x + d) * s4, Xg.y * s4);
+}
+
+// MODE 0: convolution (multiply by the spectrum, inverse row DFT, store back);
+//         workspace row i of the launch is (b, c) row r = row0 + i, r = c*B + b,
+//         and uses spectrum row (step, c).
+// MODE 1: spectrum build: workspace row i is spectrum row r = row0 + i
+//         (= step*C + c); the pair entries of K~ replace the unit in place.
+template <int M2, int MODE>
+__global__ void k_mp_pass_b(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1,
+                            int64_t row0, int64_t ws_row_stride, int64_t spec_row_stride4, int step,
+                            int64_t B, int64_t C, const float* __restrict__ D) {
+    extern __shared__ float2 smem[];
+    constexpr int PS = fft_padded_size(M2);
+    const int M = M1 * M2;
+    const int64_t L = int64_t(2) * M;
+    const bool odd = blockIdx.x >= unsigned(M1 / 2);
+    const int u = odd ? int(blockIdx.x) - M1 / 2 : int(blockIdx.x);
+    const int ra = u;                       // first row of the unit (0 for chain e unit 0)
+    const int64_t r = row0 + blockIdx.y;
+    float2* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
+    float2* b0 = smem;
+    float2* b1 = smem + PS;
+    for (int i = threadIdx.x; i < M2; i += blockDim.x) {
+        b0[fft_pad(i)] = unit[i];
+        b1[fft_pad(i)] = unit[M2 + i];
+    }
+    __syncthreads();
+    cta_fft_forward<M2>(smem, 2, PS, tb.fftB);
+    const float2 wodd = odd ? __ldg(tb.unt_c) : make_float2(1.0f, 0.0f);
+    const float2 wa = __ldg(tb.unt1 + ra);
+    const float2 wb0 = __ldg(tb.unt1 + M1 / 2);
+    const float4* sp = nullptr;
+    float4* sp_out = nullptr;
+    float d = 0.0f;
+    const float s4 = 1.0f / float(4 * L);
+    if (MODE == 0) {
+        const int64_t c = r / B;
+        sp = spec + (int64_t(step) * C + c) * spec_row_stride4 + (odd ? M / 2 : 0) + int64_t(u) * M2;
+    } else {
+        sp_out = reinterpret_cast<float4*>(unit);   // the unit's 2*M2 complex = M2 float4 entries
+        d = D ? __ldg(D + r) : 0.0f;
+    }
+    for (int e = threadIdx.x; e < M2; e += blockDim.x) {
+        float2* bufA;
+        float2* bufB;
+        int pa, pb;
+        float2 w;
+        bool special = false;
+        if (!odd && u == 0) {
+            if (e == 0) {
+                special = true;
+                bufA = b0; bufB = b0;
+                pa = fft_pad(fft_bin_pos<M2>(0));
+                pb = fft_pad(fft_bin_pos<M2>(M2 / 2));
+                w = make_float2(0.0f, -1.0f);   // w_2L^(L/2)
+            } else if (e < M2 / 2) {
+                bufA = b0; bufB = b0;
+                pa = fft_pad(fft_bin_pos<M2>(e));
+                pb = fft_pad(fft_bin_pos<M2>(M2 - e));
+                w = __ldg(tb.unt2 + e);
+            } else {
+                const int jj = e - M2 / 2;
+                bufA = b1; bufB = b1;
+                pa = fft_pad(fft_bin_pos<M2>(jj));
+                pb = fft_pad(fft_bin_pos<M2>(M2 - 1 - jj));
+                w = cmul(wb0, __ldg(tb.unt2 + jj));
+            }
+        } else {
+            bufA = b0; bufB = b1;
+            pa = fft_pad(fft_bin_pos<M2>(e));
+            pb = fft_pad(fft_bin_pos<M2>(M2 - 1 - e));
+            w = cmul(cmul(wa, __ldg(tb.unt2 + e)), wodd);
+        }
+        if (special) {
+            // f = 0 and f = L from Z[0]; the self pair f = L/2 (bin m = M/2)
+            const float2 A = bufA[pa];
+            const float2 Cc = bufB[pb];
+            if (MODE == 0) {
+                const float4 kk = __ldg(sp + e);
+                const float y0 = 2.0f * (A.x + A.y) * kk.x;
+                const float yL = 2.0f * (A.x - A.y) * kk.y;
+                float2 c1 = Cc, c2 = Cc;
+                pair_conv(c1, c2, w, make_float4(kk.z, kk.w, kk.z, kk.w));
+                bufA[pa] = make_float2(y0 + yL, y0 - yL);
+                bufB[pb] = c1;
+            } else {
+                const float4 h = pair_spec(Cc, Cc, w, d, s4);
+                sp_out[e] = make_float4((A.x + A.y + d) * s4, (A.x - A.y + d) * s4, h.x, h.y);
+            }
+        } else {
+            float2 A = bufA[pa];
+            float2 Bv = bufB[pb];
+            if (MODE == 0) {
+                pair_conv(A, Bv, w, __ldg(sp + e));
+                bufA[pa] = A;
+                bufB[pb] = Bv;
+            } else {
+                sp_out[e] = pair_spec(A, Bv, w, d, s4);
+            }
+        }
+    }
+    if (MODE == 1) return;
+    __syncthreads();
+    cta_fft_inverse<M2>(smem, 2, PS, tb.fftB);
+    for (int i = threadIdx.x; i < M2; i += blockDim.x) {
+        unit[i] = b0[fft_pad(i)];
+        unit[M2 + i] = b1[fft_pad(i)];
+    }
+}
+
+// ------------------------------------------------------------------ pass C
+// FINAL: output gate x0 and store y.  Otherwise: gate with x_{gnext}, then
+// run the next step's pass A on the same columns.
+template <int M1, typename T, bool FINAL>
+__global__ void __launch_bounds__(kColThreads)
+k_mp_pass_c(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, MpTables tb,
+            const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
+            int gnext, int M2, int64_t row0, int64_t ws_row_stride) {
+    extern __shared__ float2 smem[];
+    const int64_t r = row0 + blockIdx.y;
+    const int n2_0 = blockIdx.x * kNB2;
+    const int M = M1 * M2;
+    const int64_t L = int64_t(2) * M;
+    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    const int64_t c = r / B, b = r - (r / B) * B;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const T* ub = u + b * Ctot * L;
+    for (int idx = threadIdx.x; idx < 2 * M1 * kNB2; idx += blockDim.x) {
+        const int ch = idx / (M1 * kNB2);
+        const int rem = idx - ch * (M1 * kNB2);
+        const int m1 = rem / kNB2;
+        const int j = rem - m1 * kNB2;
+        const int n2 = n2_0 + j;
+        float2 v = ws_row[int64_t(ch) * M + int64_t(mp_slot<M1>(ch == 1, m1)) * M2 + n2];
+        v = cmulc(v, __ldg(tb.four + int64_t(m1) * M2 + n2));
+        col_ptr<M1>(smem, ch, j)[fft_pad(fft_bin_pos<M1>(m1))] = v;
+    }
+    __syncthreads();
+    cta_fft_inverse<M1>(smem, 2 * kNB2, fft_padded_size(M1), tb.fftA);
+    const int gate = FINAL ? 0 : gnext;
+    const T* xg = ub + (int64_t(gate) * C + c) * L;
+    const Taps tg = load_taps(sc_w, sc_b, int64_t(gate) * C + c);
+    T* yr = y + (b * C + c) * L;
+    for (int idx = threadIdx.x; idx < M1 * kNB2; idx += blockDim.x) {
+        const int n1 = idx / kNB2;
+        const int j = idx - n1 * kNB2;
+        const int n2 = n2_0 + j;
+        const int64_t n = int64_t(M2) * n1 + n2;
+        const float2 tw = twist_of(tb, n1, n2);
+        float2* ce = col_ptr<M1>(smem, 0, j) + fft_pad(n1);
+        float2* co = col_ptr<M1>(smem, 1, j) + fft_pad(n1);
+        const float2 zp = cadd(*ce, cmulc(*co, tw));
+        const float2 x = shortconv_pair(xg, 2 * n, tg);
+        const float2 z = make_float2(x.x * zp.x, x.y * zp.y);
+        if (FINAL) {
+            store2(yr + 2 * n, z);
+        } else {
+            *ce = z;
+            *co = cmul(z, tw);
+        }
+    }
+    if (!FINAL) cols_forward_store<M1>(smem, tb, ws_row, M2, n2_0);
+}
+
+template <int M1>
+size_t col_smem() {
+    return size_t(2) * kNB2 * fft_padded_size(M1) * sizeof(float2);
+}
+
+template <int M2>
+int row_threads() {
+    return M2 >= 2048 ? 256 : (M2 >= 1024 ? 128 : 64);
+}
+
+template <int M1, int M2>
+cudaError_t spectrum_mp(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    const MpTables tb = mp_tables(p, a.spectrum);
+    float2* rows = reinterpret_cast<float2*>(a.spectrum + p.spec_off);
+    const int64_t nrows = (p.order - 1) * p.C;
+    const int64_t stride = int64_t(p.spec_row_bytes / sizeof(float2));
+    const size_t smA = col_smem<M1>();
+    const size_t smB = size_t(2) * fft_padded_size(M2) * sizeof(float2);
+    auto kbf = k_mp_pass_a<M1, float, 1>;
+    auto kbh = k_mp_pass_a<M1, __nv_bfloat16, 1>;
+    auto kb = k_mp_pass_b<M2, 1>;
+    cudaFuncSetAttribute(kbf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kbh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    for (int64_t r0 = 0; r0 < nrows; r0 += 32768) {
+        const int64_t g = nrows - r0 < 32768 ? nrows - r0 : 32768;
+        if (a.k_dtype == DT_F32) {
+            kbf<<<dim3(M2 / kNB2, unsigned(g)), kColThreads, smA, s>>>(
+                static_cast<const float*>(a.k), rows + r0 * stride, tb, nullptr, nullptr, 1, 1, 2, M2, r0, stride);
+        } else {
+            kbh<<<dim3(M2 / kNB2, unsigned(g)), kColThreads, smA, s>>>(
+                static_cast<const __nv_bfloat16*>(a.k), rows + r0 * stride, tb, nullptr, nullptr, 1, 1, 2, M2, r0,
+                stride);
+        }
+        kb<<<dim3(M1, unsigned(g)), row_threads<M2>(), smB, s>>>(rows + r0 * stride, nullptr, tb, M1, r0, stride, 0,
+                                                                 0, 1, p.C, a.D);
+    }
+    return cudaGetLastError();
+}
+
+template <int M1, int M2, typename T>
+cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    const MpTables tb = mp_tables(p, a.spectrum);
+    const float4* spec = reinterpret_cast<const float4*>(a.spectrum + p.spec_off);
+    const T* u = static_cast<const T*>(a.u);
+    T* y = static_cast<T*>(a.y);
+    const int64_t rows = a.B * p.C;
+    int64_t G = a.group_rows < 65535 ? a.group_rows : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
+    const int64_t spec_stride4 = int64_t(p.spec_row_bytes / 16);
+    const size_t smA = col_smem<M1>();
+    const size_t smB = size_t(2) * fft_padded_size(M2) * sizeof(float2);
+    auto ka = k_mp_pass_a<M1, T, 0>;
+    auto kb = k_mp_pass_b<M2, 0>;
+    auto kc = k_mp_pass_c<M1, T, true>;
+    auto kca = k_mp_pass_c<M1, T, false>;
+    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    for (int64_t r0 = 0; r0 < rows; r0 += G) {
+        const int64_t g = rows - r0 < G ? rows - r0 : G;
+        const dim3 gridA(M2 / kNB2, unsigned(g));
+        ka<<<gridA, kColThreads, smA, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
+        for (int st = 1; st < p.order; ++st) {
+            kb<<<dim3(M1, unsigned(g)), row_threads<M2>(), smB, s>>>(a.workspace, spec, tb, M1, r0, stride,
+                                                                      spec_stride4, st - 1, a.B, p.C, nullptr);
+            if (st < p.order - 1) {
+                kca<<<gridA, kColThreads, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
+                                                     p.order - st - 1, M2, r0, stride);
+            } else {
+                kc<<<gridA, kColThreads, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2,
+                                                    r0, stride);
+            }
+        }
+    }
+    return cudaGetLastError();
+}
+
+template <int M1, int M2>
+cudaError_t conv_mp(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    return a.dtype == DT_F32 ? conv_mp_t<M1, M2, float>(p, a, s) : conv_mp_t<M1, M2, __nv_bfloat16>(p, a, s);
+}
+
+}  // namespace
+
+#define HYENA_MP_SWITCH(FN)                                   \
+    switch (p.M) {                                            \
+        case 1 << 14: return FN<128, 128>(p, a, s);           \
+        case 1 << 15: return FN<128, 256>(p, a, s);           \
+        case 1 << 16: return FN<256, 256>(p, a, s);           \
+        case 1 << 17: return FN<256, 512>(p, a, s);           \
+        case 1 << 18: return FN<256, 1024>(p, a, s);          \
+        case 1 << 19: return FN<256, 2048>(p, a, s);          \
+        default: return cudaErrorInvalidValue;                \
+    }
+
+cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    HYENA_MP_SWITCH(spectrum_mp)
+}
+
+cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    HYENA_MP_SWITCH(conv_mp)
+}
+
+}  // namespace hyena

@@ -185,6 +185,186 @@ k_conv_onchip(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restr
     }
 }
 
+// ---------------------------------------------------------------------------
+// Register-resident variant for M = 4096 (L = 8192): 256 threads, each holding
+// 16 points of each chain in registers through the three radix-16 stages.
+// Thread t owns n = t + 256 s in stage 1, (j, p) = (t/16, t%16) with
+// 256 j + p + 16 s in stage 2, and 16 t + s in stage 3.  The padding
+// pad(i) = i + i/16 + i/256 is linear along each of these strides (273, 17
+// and 1 padded slots), so every shared-memory access is a per-thread base
+// plus a compile-time offset.  Stage twiddles are copied to shared memory once
+// per CTA; CTAs are persistent (two per SM).  The step result stays in
+// registers between order steps.
+// ---------------------------------------------------------------------------
+namespace r16 {
+
+constexpr int M = 4096;
+constexpr int L = 8192;
+constexpr int NT = 256;
+constexpr int PS = fft_padded_size(M);        // 4368
+constexpr int NTW1 = 15 * 256;                // stage-1 twiddles w_4096^(t s)
+constexpr int NTW2 = 15 * 16;                 // stage-2 twiddles w_256^(p s)
+constexpr size_t kSmem = size_t(2 * PS + NTW1 + NTW2) * sizeof(float2);
+static_assert(fft_tw_size(M) == NTW1 + NTW2, "stage table layout");
+
+// cos(pi s / 16), s = 0..8 (mathematical constants)
+__device__ __forceinline__ float cos16(int s) {
+    switch (s) {
+        case 0: return 1.0f;
+        case 1: return 0.98078528040323044913f;
+        case 2: return 0.92387953251128675613f;
+        case 3: return 0.83146961230254523708f;
+        case 4: return 0.70710678118654752440f;
+        case 5: return 0.55557023301960222474f;
+        case 6: return 0.38268343236508977173f;
+        case 7: return 0.19509032201612826785f;
+        default: return 0.0f;
+    }
+}
+// w_32^s = exp(-2 pi i s / 32), s = 0..15
+__device__ __forceinline__ float2 w32(int s) {
+    const float c = s <= 8 ? cos16(s) : -cos16(16 - s);
+    const float sn = cos16(s <= 8 ? 8 - s : s - 8);
+    return make_float2(c, -sn);
+}
+
+template <bool INV>
+__device__ __forceinline__ void dft16x2(float2 (&e)[16], float2 (&o)[16]) {
+    DFT<16, INV>::run(e);
+    DFT<16, INV>::run(o);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT, 2)
+k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
+            const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
+            int64_t rows) {
+    extern __shared__ float2 smem[];
+    if (!header_ok(spectrum, C, L, order)) return;
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
+    const float2* twist = tables + fft_tw_size(M);
+    const float2* untw = twist + M;
+    const float4* spec = reinterpret_cast<const float4*>(spectrum + h->spec_off);
+    float2* E = smem;
+    float2* O = smem + PS;
+    float2* TW1 = smem + 2 * PS;
+    float2* TW2 = TW1 + NTW1;
+    for (int i = threadIdx.x; i < NTW1 + NTW2; i += NT) TW1[i] = __ldg(tables + i);
+
+    const int t = threadIdx.x;
+    const int base1 = t + (t >> 4);                       // pad(t + 256 s) = base1 + 273 s
+    const int jj = t >> 4, pp = t & 15;
+    const int base2 = 273 * jj + pp;                      // pad(256 j + p + 16 s) = base2 + 17 s
+    const int base3 = 17 * t + (t >> 4);                  // pad(16 t + s) = base3 + s
+    const float2 wt = __ldg(twist + t);                   // w_L^t
+    const int64_t Ctot = int64_t(order + 1) * C;
+    __syncthreads();
+
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int64_t c = r / B;
+        const int64_t b = r - c * B;
+        const T* ub = u + b * Ctot * L;
+        float2 v[16];     // value (packed pairs) at n = t + 256 s
+        {
+            const T* vr = ub + (int64_t(order) * C + c) * L;
+            const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) v[s] = shortconv_pair(vr, 2 * (t + 256 * s), tv);
+        }
+        for (int st = 1; st < order; ++st) {
+            const int g = order - st;
+            const T* xg = ub + (int64_t(g) * C + c) * L;
+            const Taps tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
+            float2 e[16], o[16];
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+                const float2 x = shortconv_pair(xg, 2 * (t + 256 * s), tg);
+                e[s] = make_float2(x.x * v[s].x, x.y * v[s].y);
+                o[s] = cmul(e[s], cmul(wt, w32(s)));
+            }
+            // stage 1: len 4096, P = 256
+            dft16x2<false>(e, o);
+#pragma unroll
+            for (int s = 1; s < 16; ++s) {
+                const float2 w = TW1[(s - 1) * 256 + t];
+                e[s] = cmul(e[s], w);
+                o[s] = cmul(o[s], w);
+            }
+            __syncthreads();   // previous users of E/O are done
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { E[base1 + 273 * s] = e[s]; O[base1 + 273 * s] = o[s]; }
+            __syncthreads();
+            // stage 2: len 256, P = 16
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { e[s] = E[base2 + 17 * s]; o[s] = O[base2 + 17 * s]; }
+            dft16x2<false>(e, o);
+#pragma unroll
+            for (int s = 1; s < 16; ++s) {
+                const float2 w = TW2[(s - 1) * 16 + pp];
+                e[s] = cmul(e[s], w);
+                o[s] = cmul(o[s], w);
+            }
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { E[base2 + 17 * s] = e[s]; O[base2 + 17 * s] = o[s]; }
+            __syncthreads();
+            // stage 3: len 16, P = 1
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { e[s] = E[base3 + s]; o[s] = O[base3 + s]; }
+            dft16x2<false>(e, o);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { E[base3 + s] = e[s]; O[base3 + s] = o[s]; }
+            __syncthreads();
+            conv_pairs<M>(E, O, spec + (int64_t(st - 1) * C + c) * (M + 1), untw);
+            __syncthreads();
+            // inverse stage 3
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { e[s] = E[base3 + s]; o[s] = O[base3 + s]; }
+            dft16x2<true>(e, o);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { E[base3 + s] = e[s]; O[base3 + s] = o[s]; }
+            __syncthreads();
+            // inverse stage 2
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { e[s] = E[base2 + 17 * s]; o[s] = O[base2 + 17 * s]; }
+#pragma unroll
+            for (int s = 1; s < 16; ++s) {
+                const float2 w = TW2[(s - 1) * 16 + pp];
+                e[s] = cmulc(e[s], w);
+                o[s] = cmulc(o[s], w);
+            }
+            dft16x2<true>(e, o);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { E[base2 + 17 * s] = e[s]; O[base2 + 17 * s] = o[s]; }
+            __syncthreads();
+            // inverse stage 1
+#pragma unroll
+            for (int s = 0; s < 16; ++s) { e[s] = E[base1 + 273 * s]; o[s] = O[base1 + 273 * s]; }
+#pragma unroll
+            for (int s = 1; s < 16; ++s) {
+                const float2 w = TW1[(s - 1) * 256 + t];
+                e[s] = cmulc(e[s], w);
+                o[s] = cmulc(o[s], w);
+            }
+            dft16x2<true>(e, o);
+            // combine the chains: z'[n] = e'[n] + w_L^(-n) o'[n]
+#pragma unroll
+            for (int s = 0; s < 16; ++s) v[s] = cadd(e[s], cmulc(o[s], cmul(wt, w32(s))));
+        }
+        const T* x0 = ub + c * L;
+        const Taps t0 = load_taps(sc_w, sc_b, c);
+        T* yr = y + (b * C + c) * L;
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {
+            const int n = t + 256 * s;
+            const float2 x = shortconv_pair(x0, 2 * n, t0);
+            store2(yr + 2 * n, make_float2(x.x * v[s].x, x.y * v[s].y));
+        }
+    }
+}
+
+}  // namespace r16
+
 template <int M>
 cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     constexpr int NT = onchip_threads<M>();
@@ -202,8 +382,26 @@ cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    auto kern = r16::k_conv_4096<T>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(r16::kSmem));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t rows = a.B * p.C;
+    int64_t grid = int64_t(2) * sms;
+    if (grid > rows) grid = rows;
+    kern<<<unsigned(grid), r16::NT, r16::kSmem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
+                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows);
+    return cudaGetLastError();
+}
+
 template <int M>
 cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    if constexpr (M == 4096) {
+        return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : conv_4096<__nv_bfloat16>(p, a, s);
+    }
     constexpr int NT = onchip_threads<M>();
     const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
     const unsigned grid = unsigned(a.B * p.C);

@@ -84,8 +84,9 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
             p->t_four = tb.add(p->M, 0, p->M1, 0, p->M2);             // w_M^(m1 n2), [m1][n2]
             p->t_twist_hi = tb.add(L, 0, p->M1, p->M2, 1);            // w_L^(M2 n1)
             p->t_twist_lo = tb.add(L, 0, p->M2, 1, 1);                // w_L^(n2)
-            p->t_unt1 = tb.add(p->M, 0, p->M1, 1, 1);                 // w_M^(m1)
-            p->t_unt2 = tb.add(p->M2, 0, p->M2, 1, 1);                // w_M2^(m2)
+            // pair twiddle w_2L^(2m) = w_L^m = w_L^(m1) * w_(2 M2)^(m2), m = m1 + M1 m2
+            p->t_unt1 = tb.add(L, 0, p->M1, 1, 1);                    // w_L^(m1)
+            p->t_unt2 = tb.add(2 * p->M2, 0, p->M2, 1, 1);            // w_(2 M2)^(m2)
             p->t_unt_c = tb.add(2 * L, 1, 1, 1, 1);                   // w_2L^1
             p->spec_row_bytes = size_t(p->M) * 16;                   // M1 units x M2 float4
             p->ws_row_bytes = size_t(2 * p->M) * 8;                  // two chains of M complex
