@@ -22,7 +22,8 @@ STATUS = {0: "HYENA_OK", 1: "HYENA_ERR_INVALID_ARG", 2: "HYENA_ERR_UNSUPPORTED_S
 # every symbol include/hyena.h declares
 EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "hyena_spectrum_bytes",
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
-           "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_spectrum_check"]
+           "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
+           "hyena_spectrum_check"]
 
 _lock = threading.Lock()
 _lib = None
@@ -65,6 +66,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hyena_gated_fftconv.restype = ctypes.c_int
         lib.hyena_gated_fftconv.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p, ctypes.c_int,
                                             ctypes.c_int, vp, sz, vp]
+        lib.hyena_gated_fftconv_noalloc.restype = ctypes.c_int
+        lib.hyena_gated_fftconv_noalloc.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
+                                                    ctypes.c_int, ctypes.c_int, vp]
         lib.hyena_spectrum_check.restype = ctypes.c_int
         lib.hyena_spectrum_check.argtypes = [vp, i64, ctypes.c_int, i64p, ctypes.c_int, vp]
         _lib = lib
@@ -151,6 +155,17 @@ def hyena_gated_fftconv(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, or
     _check(load().hyena_gated_fftconv(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
                                       _ptr(sc_w), _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
                                       _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hyena_gated_fftconv_noalloc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int,
+                                stream=None) -> None:
+    """hyena_gated_fftconv without a workspace argument: the library's fixed
+    scratch array is used instead (for callers that cannot allocate)."""
+    arr, nd = _sizes(sizes)
+    _check(load().hyena_gated_fftconv_noalloc(_ptr(u), _ptr(y), _ptr(spectrum),
+                                              spectrum.numel() * spectrum.element_size(), _ptr(sc_w),
+                                              _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
+                                              _stream(stream)))
 
 
 def hyena_spectrum_check(spectrum, C: int, sizes, order: int, stream=None) -> None:

@@ -53,6 +53,12 @@ hyena_status_t plan_or_fail(int64_t C, int ndim, const int64_t* sizes, int order
 
 }  // namespace
 
+namespace hyena {
+// Records the thread-local detail message reported by hyena_last_error_detail()
+// and returns st (used by entry points defined in other translation units).
+hyena_status_t set_last_error_detail(hyena_status_t st, const std::string& detail) { return fail(st, detail); }
+}  // namespace hyena
+
 extern "C" {
 
 int hyena_version(void) { return 100; }

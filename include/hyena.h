@@ -31,7 +31,8 @@
  *    thread-local message available from hyena_last_error_detail().
  *  - Supported shapes: 1-D L a power of two in [16, 2^20]; 2-D H, W powers of
  *    two in [16, 512]; order in [2, 8]; C >= 1, B >= 1.
- *  - The library keeps no state between calls; all entry points are
+ *  - Apart from the fixed scratch of hyena_gated_fftconv_noalloc (see there),
+ *    the library keeps no state between calls; all entry points are
  *    thread-safe.  Calls on one stream are ordered; calls that write the
  *    same buffers from different streams race.
  */
@@ -148,6 +149,43 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
                                    size_t workspace_bytes, void* stream);
 
 /*
+ * Size of the fixed scratch array used by hyena_gated_fftconv_noalloc (32 MiB).
+ */
+#define HYENA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * hyena_gated_fftconv_noalloc -- the same operation as hyena_gated_fftconv,
+ * for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart: this entry point exists for callers that have
+ * no way to provide a workspace, such as a plugin whose host framework owns
+ * every device allocation, or a serving loop that must never call cudaMalloc
+ * (an allocation can block, synchronise the device or fail under memory
+ * pressure at a point where the work cannot be dropped).  Instead of a
+ * caller workspace it uses a fixed device array of
+ * HYENA_NOALLOC_SCRATCH_BYTES that is part of the library image; every GPU
+ * that loads the library keeps that array until the process exits.  The
+ * caller still passes u, y and the spectrum; arguments and errors are those
+ * of hyena_gated_fftconv.  Nothing is allocated or freed.
+ *
+ *  - Limit: shapes whose workspace row (hyena_gated_fftconv_workspace_min_bytes)
+ *    exceeds HYENA_NOALLOC_SCRATCH_BYTES are rejected with
+ *    HYENA_ERR_WORKSPACE_TOO_SMALL; rows are processed in groups that fit.
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current), which may load
+ *    the library's device code; make that first call before any stream
+ *    capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    last call's contents.  No zeroing is needed: each call writes every
+ *    scratch element before reading it.  Calls that overlap on the GPU (for
+ *    example on two streams) race on the array and give wrong results.
+ */
+hyena_status_t hyena_gated_fftconv_noalloc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                           const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                           const int64_t* sizes, int order, hyena_dtype_t dtype, void* stream);
+
+/*
+ * Debug helper (synchronous)/*
  * Debug helper (synchronous): copies the spectrum header to the host and
  * checks it against (C, sizes, order).  Returns HYENA_OK when it matches,
  * HYENA_ERR_SPECTRUM_MISMATCH when not (e.g. never filled, or filled for
