@@ -15,6 +15,11 @@ __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&bits);
     return __bfloat1622float2(h);
 }
+// Two consecutive values from shared memory (even element index).
+__device__ __forceinline__ float2 load2_shared(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 load2_shared(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
 __device__ __forceinline__ void store2(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 __device__ __forceinline__ void store2(__nv_bfloat16* p, float2 v) {
     __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);

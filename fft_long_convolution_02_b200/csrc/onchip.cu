@@ -204,7 +204,6 @@ constexpr int NT = 256;
 constexpr int PS = fft_padded_size(M);        // 4368
 constexpr int NTW1 = 15 * 256;                // stage-1 twiddles w_4096^(t s)
 constexpr int NTW2 = 15 * 16;                 // stage-2 twiddles w_256^(p s)
-constexpr size_t kSmem = size_t(2 * PS + NTW1 + NTW2) * sizeof(float2);
 static_assert(fft_tw_size(M) == NTW1 + NTW2, "stage table layout");
 
 // cos(pi s / 16), s = 0..8 (mathematical constants)
@@ -234,6 +233,160 @@ __device__ __forceinline__ void dft16x2(float2 (&e)[16], float2 (&o)[16]) {
     DFT<16, INV>::run(o);
 }
 
+// cp.async of 16 bytes global -> shared (sm_80+ asynchronous copy).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Staging of one row of the step-1 gate and of the value: kHalo leading zero
+// elements (the short conv reads two samples before t = 0), then L samples.
+constexpr int kHalo = 8;
+
+template <typename T>
+__device__ __forceinline__ void prefetch_row(T* sx, T* sv, const T* gx, const T* gv) {
+    constexpr int per = 16 / sizeof(T);              // elements per 16-byte chunk
+    constexpr int chunks = L / per;
+    for (int i = threadIdx.x; i < chunks; i += NT) {
+        cp_async16(sx + kHalo + i * per, gx + i * per);
+        cp_async16(sv + kHalo + i * per, gv + i * per);
+    }
+    cp_async_commit();
+}
+
+// Two consecutive short-convolved samples t = 2n, 2n+1 from a staged row.
+template <typename T>
+__device__ __forceinline__ float2 staged_pair(const T* srow, int n, const Taps& tp) {
+    const float2 cur = load2_shared(srow + kHalo + 2 * n);
+    if (!tp.on) return cur;
+    const float2 prev = load2_shared(srow + kHalo + 2 * n - 2);
+    float2 r;
+    r.x = fmaf(tp.w0, prev.x, fmaf(tp.w1, prev.y, fmaf(tp.w2, cur.x, tp.b)));
+    r.y = fmaf(tp.w0, prev.y, fmaf(tp.w1, cur.x, fmaf(tp.w2, cur.y, tp.b)));
+    return r;
+}
+
+// Multiply e[s], o[s] (s = 1..15) by w_4096^(t s) (conjugate when CONJ),
+// generating the powers from w^t and w^(4t) on the fly: w^(4a+b) =
+// w^(4a) w^b with at most two rounded products (error a few ulp).
+template <bool CONJ>
+__device__ __forceinline__ void apply_stage1_twiddles(float2 (&e)[16], float2 (&o)[16],
+                                                      const float2* __restrict__ tw1_table) {
+    // w_4096^(t s): w^t and w^(4t) from the table, the rest by at most two
+    // rounded products (error a few ulp)
+    const int t = threadIdx.x;
+    const float2 w1 = __ldg(tw1_table + t);
+    const float2 w4 = __ldg(tw1_table + 3 * 256 + t);
+    const float2 w2 = cmul(w1, w1);
+    const float2 w3 = cmul(w2, w1);
+    const float2 w8 = cmul(w4, w4);
+    const float2 w12 = cmul(w8, w4);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const float2 wa = a == 0 ? make_float2(1.0f, 0.0f) : (a == 1 ? w4 : (a == 2 ? w8 : w12));
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int s = 4 * a + b;
+            if (s == 0) continue;
+            const float2 wb = b == 1 ? w1 : (b == 2 ? w2 : w3);
+            const float2 w = b == 0 ? wa : (a == 0 ? wb : cmul(wa, wb));
+            if (CONJ) {
+                e[s] = cmulc(e[s], w);
+                o[s] = cmulc(o[s], w);
+            } else {
+                e[s] = cmul(e[s], w);
+                o[s] = cmul(o[s], w);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void pair_conv4096(float2& A, float2& Bv, float2 w, float4 kk) {
+    const float2 S = cadd(A, cconj(Bv));
+    const float2 T = cmul_i(cmul(w, csub(A, cconj(Bv))));
+    const float2 Yf = cmul(csub(S, T), make_float2(kk.x, kk.y));
+    const float2 Yg = cmul(cconj(cadd(S, T)), make_float2(kk.z, kk.w));
+    const float2 P = cadd(Yf, cconj(Yg));
+    const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+    A = cadd(P, U);
+    Bv = cconj(csub(P, U));
+}
+
+// Pair step with a fixed thread mapping: thread t handles chain e pairs
+// j = t + 256 i (i < 8; thread 0 also j = 2048) and chain o pairs
+// j = t + 256 i (i < 8).  For t != 0 both members sit at compile-time
+// offsets from per-thread bases, and the pair twiddles are w_L^t w_32^i
+// (chain e) and w_2L^(2t+1) w_32^i (chain o).
+__device__ __forceinline__ void pairs_4096(float2* __restrict__ E, float2* __restrict__ O,
+                                           const float4* __restrict__ spec, const float2* __restrict__ twist,
+                                           const float2* __restrict__ untw) {
+    const int t = threadIdx.x;
+    const float2 wt = __ldg(twist + t);                   // w_L^t
+    const float2 wt_odd = __ldg(untw + (M / 2 + 1) + t);  // w_2L^(2t+1)
+    // position of bin j = t + 256 i: (t & 15) * 256 + (t >> 4) * 16 + i  (padded)
+    const int pa0 = fft_pad((t & 15) * 256 + (t >> 4) * 16);
+    // chain e partner M - j = (256 - t) + 256 (15 - i) for t != 0
+    const int te = (256 - t) & 255;
+    const int pbe0 = fft_pad((te & 15) * 256 + (te >> 4) * 16);
+    // chain o partner M - 1 - j = (255 - t) + 256 (15 - i)
+    const int to = 255 - t;
+    const int pbo0 = fft_pad((to & 15) * 256 + (to >> 4) * 16);
+#pragma unroll
+    for (int i0 = 0; i0 < 8; i0 += 4) {
+        float4 ke[4], ko[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ke[k] = __ldg(spec + t + 256 * (i0 + k));
+            ko[k] = __ldg(spec + (M / 2 + 1) + t + 256 * (i0 + k));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = i0 + k;
+            const float2 w32i = w32(i);
+            // chain e
+            if (t == 0 && i == 0) {
+                const float2 A = E[pa0];
+                const float y0 = 2.0f * (A.x + A.y) * ke[0].x;
+                const float yL = 2.0f * (A.x - A.y) * ke[0].z;
+                E[pa0] = make_float2(y0 + yL, y0 - yL);
+            } else {
+                // partner: t != 0 -> pbe0 + (15 - i); t == 0, i >= 1 -> bin 256 (16 - i)
+                const int pb = (t != 0) ? pbe0 + (15 - i) : (16 - i);
+                float2 A = E[pa0 + i];
+                float2 Bv = E[pb];
+                pair_conv4096(A, Bv, cmul(wt, w32i), ke[k]);
+                E[pa0 + i] = A;
+                E[pb] = Bv;
+            }
+            // chain o
+            {
+                const int pb = pbo0 + (15 - i);
+                float2 A = O[pa0 + i];
+                float2 Bv = O[pb];
+                pair_conv4096(A, Bv, cmul(wt_odd, w32i), ko[k]);
+                O[pa0 + i] = A;
+                O[pb] = Bv;
+            }
+        }
+    }
+    if (t == 0) {
+        // chain e self pair j = M/2 = 2048: bin 2048 -> position 8 (w = w_L^2048 = -i)
+        const int p = fft_pad(8);
+        float2 A = E[p];
+        const float4 kk = __ldg(spec + M / 2);
+        const float2 w = make_float2(0.0f, -1.0f);
+        const float2 S = cadd(A, cconj(A));
+        const float2 T = cmul_i(cmul(w, csub(A, cconj(A))));
+        const float2 Yf = cmul(csub(S, T), make_float2(kk.x, kk.y));
+        const float2 Yg = cmul(cconj(cadd(S, T)), make_float2(kk.z, kk.w));
+        const float2 P = cadd(Yf, cconj(Yg));
+        const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+        E[p] = cadd(P, U);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(NT, 2)
 k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
@@ -248,50 +401,73 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
     const float4* spec = reinterpret_cast<const float4*>(spectrum + h->spec_off);
     float2* E = smem;
     float2* O = smem + PS;
-    float2* TW1 = smem + 2 * PS;
-    float2* TW2 = TW1 + NTW1;
-    for (int i = threadIdx.x; i < NTW1 + NTW2; i += NT) TW1[i] = __ldg(tables + i);
+    float2* TW2 = smem + 2 * PS;
+    T* SX = reinterpret_cast<T*>(TW2 + NTW2);
+    T* SV = SX + (kHalo + L);
 
     const int t = threadIdx.x;
-    const int base1 = t + (t >> 4);                       // pad(t + 256 s) = base1 + 273 s
-    const int jj = t >> 4, pp = t & 15;
-    const int base2 = 273 * jj + pp;                      // pad(256 j + p + 16 s) = base2 + 17 s
-    const int base3 = 17 * t + (t >> 4);                  // pad(16 t + s) = base3 + s
-    const float2 wt = __ldg(twist + t);                   // w_L^t
     const int64_t Ctot = int64_t(order + 1) * C;
-    __syncthreads();
+    auto row_ptrs = [&](int64_t r, const T*& ub, int64_t& c, int64_t& b) {
+        c = r / B;
+        b = r - c * B;
+        ub = u + b * Ctot * L;
+    };
+    // first prefetch, then the per-CTA constants
+    if (int64_t(blockIdx.x) < rows) {
+        const T* ub; int64_t c, b;
+        row_ptrs(blockIdx.x, ub, c, b);
+        prefetch_row(SX, SV, ub + (int64_t(order - 1) * C + c) * L, ub + (int64_t(order) * C + c) * L);
+    }
+    if (t < kHalo) { SX[t] = T(0.0f); SV[t] = T(0.0f); }
+    for (int i = t; i < NTW2; i += NT) TW2[i] = __ldg(tables + NTW1 + i);
+    const int base1 = t + (t >> 4);                       // pad(t + 256 s) = base1 + 273 s
+    const int pp = t & 15;
+    const int base2 = 273 * (t >> 4) + pp;                // pad(256 j + p + 16 s) = base2 + 17 s
+    const int base3 = 17 * t + (t >> 4);                  // pad(16 t + s) = base3 + s
 
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const int64_t c = r / B;
-        const int64_t b = r - c * B;
-        const T* ub = u + b * Ctot * L;
-        float2 v[16];     // value (packed pairs) at n = t + 256 s
-        {
-            const T* vr = ub + (int64_t(order) * C + c) * L;
-            const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
-#pragma unroll
-            for (int s = 0; s < 16; ++s) v[s] = shortconv_pair(vr, 2 * (t + 256 * s), tv);
-        }
+        const T* ub; int64_t c, b;
+        row_ptrs(r, ub, c, b);
+        const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+        cp_async_wait_all();
+        __syncthreads();                                  // staging of row r complete
         for (int st = 1; st < order; ++st) {
             const int g = order - st;
-            const T* xg = ub + (int64_t(g) * C + c) * L;
             const Taps tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
             float2 e[16], o[16];
+            if (st == 1) {
 #pragma unroll
-            for (int s = 0; s < 16; ++s) {
-                const float2 x = shortconv_pair(xg, 2 * (t + 256 * s), tg);
-                e[s] = make_float2(x.x * v[s].x, x.y * v[s].y);
-                o[s] = cmul(e[s], cmul(wt, w32(s)));
+                for (int s = 0; s < 16; ++s) {
+                    const float2 x = staged_pair(SX, t + 256 * s, tg);
+                    const float2 vv = staged_pair(SV, t + 256 * s, tv);
+                    e[s] = make_float2(x.x * vv.x, x.y * vv.y);
+                }
+                __syncthreads();                          // staging consumed: prefetch the next row
+                const int64_t rn = r + gridDim.x;
+                if (rn < rows) {
+                    const T* ubn; int64_t cn, bn;
+                    row_ptrs(rn, ubn, cn, bn);
+                    prefetch_row(SX, SV, ubn + (int64_t(order - 1) * C + cn) * L,
+                                 ubn + (int64_t(order) * C + cn) * L);
+                }
+            } else {
+                // the previous step left v at this thread's stage-1 positions of E
+                const T* xg = ub + (int64_t(g) * C + c) * L;
+#pragma unroll
+                for (int s = 0; s < 16; ++s) {
+                    const float2 x = shortconv_pair(xg, 2 * (t + 256 * s), tg);
+                    const float2 vv = E[base1 + 273 * s];
+                    e[s] = make_float2(x.x * vv.x, x.y * vv.y);
+                }
+            }
+            {
+                const float2 wt = __ldg(twist + t);       // w_L^t
+#pragma unroll
+                for (int s = 0; s < 16; ++s) o[s] = cmul(e[s], cmul(wt, w32(s)));
             }
             // stage 1: len 4096, P = 256
             dft16x2<false>(e, o);
-#pragma unroll
-            for (int s = 1; s < 16; ++s) {
-                const float2 w = TW1[(s - 1) * 256 + t];
-                e[s] = cmul(e[s], w);
-                o[s] = cmul(o[s], w);
-            }
-            __syncthreads();   // previous users of E/O are done
+            apply_stage1_twiddles<false>(e, o, tables);
 #pragma unroll
             for (int s = 0; s < 16; ++s) { E[base1 + 273 * s] = e[s]; O[base1 + 273 * s] = o[s]; }
             __syncthreads();
@@ -315,7 +491,7 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
 #pragma unroll
             for (int s = 0; s < 16; ++s) { E[base3 + s] = e[s]; O[base3 + s] = o[s]; }
             __syncthreads();
-            conv_pairs<M>(E, O, spec + (int64_t(st - 1) * C + c) * (M + 1), untw);
+            pairs_4096(E, O, spec + (int64_t(st - 1) * C + c) * (M + 1), twist, untw);
             __syncthreads();
             // inverse stage 3
 #pragma unroll
@@ -340,27 +516,36 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
             // inverse stage 1
 #pragma unroll
             for (int s = 0; s < 16; ++s) { e[s] = E[base1 + 273 * s]; o[s] = O[base1 + 273 * s]; }
-#pragma unroll
-            for (int s = 1; s < 16; ++s) {
-                const float2 w = TW1[(s - 1) * 256 + t];
-                e[s] = cmulc(e[s], w);
-                o[s] = cmulc(o[s], w);
-            }
+            apply_stage1_twiddles<true>(e, o, tables);
             dft16x2<true>(e, o);
             // combine the chains: z'[n] = e'[n] + w_L^(-n) o'[n]
+            const float2 wt = __ldg(twist + t);           // w_L^t
+            if (st == order - 1) {
+                // last step: output gate y = x0 * v, straight from registers
+                const T* x0 = ub + c * L;
+                const Taps t0 = load_taps(sc_w, sc_b, c);
+                T* yr = y + (b * C + c) * L;
 #pragma unroll
-            for (int s = 0; s < 16; ++s) v[s] = cadd(e[s], cmulc(o[s], cmul(wt, w32(s))));
-        }
-        const T* x0 = ub + c * L;
-        const Taps t0 = load_taps(sc_w, sc_b, c);
-        T* yr = y + (b * C + c) * L;
+                for (int s = 0; s < 16; ++s) {
+                    const int n = t + 256 * s;
+                    const float2 vv = cadd(e[s], cmulc(o[s], cmul(wt, w32(s))));
+                    const float2 x = shortconv_pair(x0, 2 * n, t0);
+                    store2(yr + 2 * n, make_float2(x.x * vv.x, x.y * vv.y));
+                }
+            } else {
+                __syncthreads();                          // every thread has read E (inverse stage 1)
 #pragma unroll
-        for (int s = 0; s < 16; ++s) {
-            const int n = t + 256 * s;
-            const float2 x = shortconv_pair(x0, 2 * n, t0);
-            store2(yr + 2 * n, make_float2(x.x * v[s].x, x.y * v[s].y));
+                for (int s = 0; s < 16; ++s) E[base1 + 273 * s] = cadd(e[s], cmulc(o[s], cmul(wt, w32(s))));
+            }
+            __syncthreads();                              // E/O free for the next step / row
         }
     }
+    cp_async_wait_all();
+}
+
+template <typename T>
+constexpr size_t conv_4096_smem() {
+    return size_t(2 * PS + NTW2) * sizeof(float2) + size_t(2 * (kHalo + L)) * sizeof(T);
 }
 
 }  // namespace r16
@@ -385,14 +570,15 @@ cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
 template <typename T>
 cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     auto kern = r16::k_conv_4096<T>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(r16::kSmem));
+    constexpr size_t smem = r16::conv_4096_smem<T>();
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t rows = a.B * p.C;
     int64_t grid = int64_t(2) * sms;
     if (grid > rows) grid = rows;
-    kern<<<unsigned(grid), r16::NT, r16::kSmem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
+    kern<<<unsigned(grid), r16::NT, smem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
                                                     a.sc_w, a.sc_b, a.B, p.C, p.order, rows);
     return cudaGetLastError();
 }
