@@ -63,26 +63,27 @@ def spectrum_row_bytes(p) -> int:
     return 8 * p.L
 
 
-def source_hash() -> str:
+def source_hash(files) -> str:
+    """Hash of the kernel sources a profile was taken on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fft_long_convolution_02_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def committed_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    only if it was taken on the kernel's current sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         entries = json.load(f)
-    src = source_hash()
     for e in entries:
-        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_hash") == src:
+        if e.get("kernel") == kernel and e.get("workload") == workload and \
+                e.get("source_hash") == source_hash(e.get("sources", [])):
             return e.get("dram_bytes_per_launch")
     return None
 
@@ -331,7 +332,12 @@ def main():
     alg = algorithmic_bytes(p, spec_row)
     avg_launch_s = float(np.mean(launch_ms)) / 1e3
     achieved = alg / avg_launch_s / 1e9
-    kernel = "k_conv_onchip" if (p.ndim == 1 and p.L <= 16384) else ("multipass" if p.ndim == 1 else "grid2d")
+    if p.ndim == 1 and p.L == 8192:
+        kernel = "k_conv_4096"
+    elif p.ndim == 1 and p.L <= 16384:
+        kernel = "k_conv_onchip"
+    else:
+        kernel = "multipass" if p.ndim == 1 else "grid2d"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
