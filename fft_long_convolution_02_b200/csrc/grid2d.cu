@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"
+#include "reg_fft.cuh"
 
 namespace hyena {
 
@@ -179,11 +180,14 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
             }
         } else {
             // K~ = (X2D / 2 + D) * s8, positions in order, chain e then chain o
+            // stored in the fast column pass's thread order: position 16 g + k
+            // of chain ch goes to entry ch * MH + k * (MH / 16) + g
             for (int idx = threadIdx.x; idx < 2 * MH; idx += blockDim.x) {
                 const int ch = idx / MH;
                 const int pos = idx - ch * MH;
                 const float2 v = smem[ch * PS + fft_pad(pos)];
-                ws_img[int64_t(f0) * (2 * MH) + idx] = make_float2((0.5f * v.x + d) * s8, 0.5f * v.y * s8);
+                const int e = ch * MH + (pos & 15) * (MH / 16) + (pos >> 4);
+                ws_img[int64_t(f0) * (2 * MH) + e] = make_float2((0.5f * v.x + d) * s8, 0.5f * v.y * s8);
             }
         }
         __syncthreads();
@@ -247,6 +251,213 @@ k_2d_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ w
     if (!FINAL) rows_forward_store<MW>(smem, tb, ws_img, H, p0, 1.0f, 0.0f);
 }
 
+// ===========================================================================
+// Register-resident 2-D passes (reg_fft.cuh).
+//   rows   : a CTA of 32 image rows x (W/32) threads; thread (r, g) holds 16
+//            points of both row chains; the untangle / re-tangle pairs go
+//            through padded shared buffers (odd stride, conflict-free).
+//   columns: a CTA of 16 bin columns x (H/16) threads, both column chains per
+//            thread; K~ is read in the same thread order ([chain][k][g]).
+// ===========================================================================
+constexpr int kFC = 16;   // bin columns per CTA in the fast column pass
+
+template <int MW>
+__host__ __device__ constexpr int row_stride_f() {
+    return fft_padded_size(MW) | 1;   // odd stride: rows of a warp hit different banks
+}
+
+template <int MW, int FR>
+__device__ __forceinline__ void frows_store(float2 (&x)[2][16], float2* smem, const T2d& tb,
+                                            float2* __restrict__ ws_img, int H, int p0, int r, int g) {
+    constexpr int W = 2 * MW;
+    constexpr int RS = row_stride_f<MW>();
+    // positions 16 g + k of both chains to shared memory
+    float2* be = smem + (0 * FR + r) * RS;
+    float2* bo = smem + (1 * FR + r) * RS;
+    const int base = fft_pad(16 * g);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) { be[base + k] = x[0][k]; bo[base + k] = x[1][k]; }
+    __syncthreads();
+    // untangle: pairs q (chain e 0..MW/2, chain o MW/2+1..MW), rows fastest
+    for (int idx = threadIdx.x; idx < (MW + 1) * FR; idx += blockDim.x) {
+        const int q = idx / FR;
+        const int rr = idx - q * FR;
+        const bool odd = q > MW / 2;
+        const int j = odd ? q - (MW / 2 + 1) : q;
+        const float2* buf = smem + ((odd ? 1 : 0) * FR + rr) * RS;
+        const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
+        const float2 A = buf[fft_pad(fft_bin_pos<MW>(j))];
+        const float2 B = buf[fft_pad(fft_bin_pos<MW>(mb))];
+        const int f = odd ? 2 * j + 1 : 2 * j;
+        const int gg = W - f;
+        float2 Xf, Xg;
+        if (q == 0) {
+            Xf = make_float2(2.0f * (A.x + A.y), 0.0f);
+            Xg = make_float2(2.0f * (A.x - A.y), 0.0f);
+        } else {
+            const float2 w = __ldg(tb.untw + q);
+            const float2 S = cadd(A, cconj(B));
+            const float2 T = cmul_i(cmul(w, csub(A, cconj(B))));
+            Xf = csub(S, T);
+            Xg = cconj(cadd(S, T));
+        }
+        ws_img[int64_t(f) * H + p0 + rr] = Xf;
+        if (gg != f) ws_img[int64_t(gg) * H + p0 + rr] = Xg;
+    }
+}
+
+// Forward rows: MODE 0 gated x_{order-1} * v from u, MODE 1 the filter k.
+template <int MW, int FR, typename T, int MODE>
+__global__ void __launch_bounds__(FR * (MW / 16), (512 / (FR * (MW / 16))) > 0 ? 512 / (FR * (MW / 16)) : 1)
+k_2df_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
+               int64_t img0, int64_t ws_img_stride, int64_t ws_img_offset) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    constexpr int TPT = MW / 16;
+    constexpr int RS = row_stride_f<MW>();
+    const int t = threadIdx.x, r = t / TPT, g = t - (t / TPT) * TPT;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * FR;
+    const int64_t n = int64_t(H) * W;
+    const T* xg;
+    const T* vr = nullptr;
+    if (MODE == 0) {
+        const int64_t c = img / B, b = img - (img / B) * B;
+        const int64_t Ctot = int64_t(order + 1) * C;
+        const T* ub = src + b * Ctot * n;
+        xg = ub + (int64_t(order - 1) * C + c) * n;
+        vr = ub + (int64_t(order) * C + c) * n;
+    } else {
+        xg = src + img * n;
+    }
+    float2 x[2][16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int nn = g + TPT * s;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        float2 z = load2(xg + off);
+        if (MODE == 0) {
+            const float2 v = load2(vr + off);
+            z = make_float2(z.x * v.x, z.y * v.y);
+        }
+        x[0][s] = z;
+        x[1][s] = cmul(z, __ldg(tb.twist_w + nn));
+    }
+    float2* const buf[2] = {smem + (0 * FR + r) * RS, smem + (1 * FR + r) * RS};
+    reg_fft_forward<MW, 2>(x, buf, g, tb.fftW);
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
+    frows_store<MW, FR>(x, smem, tb, ws_img, H, p0, r, g);
+}
+
+// Inverse rows: re-tangle, inverse chains, output gate (FINAL) or next gate +
+// next step's forward rows.
+template <int MW, int FR, typename T, bool FINAL>
+__global__ void __launch_bounds__(FR * (MW / 16), (512 / (FR * (MW / 16))) > 0 ? 512 / (FR * (MW / 16)) : 1)
+k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C,
+               int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    constexpr int TPT = MW / 16;
+    constexpr int RS = row_stride_f<MW>();
+    const int t = threadIdx.x, r = t / TPT, g = t - (t / TPT) * TPT;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * FR;
+    const int64_t n = int64_t(H) * W;
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    for (int idx = threadIdx.x; idx < (MW + 1) * FR; idx += blockDim.x) {
+        const int q = idx / FR;
+        const int rr = idx - q * FR;
+        const bool odd = q > MW / 2;
+        const int j = odd ? q - (MW / 2 + 1) : q;
+        float2* buf = smem + ((odd ? 1 : 0) * FR + rr) * RS;
+        const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
+        const int f = odd ? 2 * j + 1 : 2 * j;
+        const int gg = W - f;
+        const float2 Yf = ws_img[int64_t(f) * H + p0 + rr];
+        const float2 Yg = ws_img[int64_t(gg) * H + p0 + rr];
+        const float2 w = (q == 0) ? make_float2(1.0f, 0.0f) : __ldg(tb.untw + q);
+        const float2 P = cadd(Yf, cconj(Yg));
+        const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+        buf[fft_pad(fft_bin_pos<MW>(j))] = cadd(P, U);
+        if (q != 0) buf[fft_pad(fft_bin_pos<MW>(mb))] = cconj(csub(P, U));
+    }
+    __syncthreads();
+    float2* const buf[2] = {smem + (0 * FR + r) * RS, smem + (1 * FR + r) * RS};
+    float2 x[2][16];
+    const int base = fft_pad(16 * g);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) { x[0][k] = buf[0][base + k]; x[1][k] = buf[1][base + k]; }
+    __syncthreads();
+    reg_fft_inverse<MW, 2>(x, buf, g, tb.fftW);
+    const int64_t c = img / B, b = img - (img / B) * B;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const T* ub = u + b * Ctot * n;
+    const int gate = FINAL ? 0 : gnext;
+    const T* xg = ub + (int64_t(gate) * C + c) * n;
+    T* yr = y + (b * C + c) * n;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int nn = g + TPT * s;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        const float2 tw = __ldg(tb.twist_w + nn);
+        const float2 zp = cadd(x[0][s], cmulc(x[1][s], tw));
+        const float2 xv = load2(xg + off);
+        const float2 z = make_float2(xv.x * zp.x, xv.y * zp.y);
+        if (FINAL) {
+            store2(yr + off, z);
+        } else {
+            x[0][s] = z;
+            x[1][s] = cmul(z, tw);
+        }
+    }
+    if (!FINAL) {
+        reg_fft_forward<MW, 2>(x, buf, g, tb.fftW);
+        frows_store<MW, FR>(x, smem, tb, ws_img, H, p0, r, g);
+    }
+}
+
+// Column pass (convolution): 2H-point FFT of each zero-padded bin column as two
+// H-point chains, times K~ (thread order), inverse, keep p < H.
+template <int MH>
+__global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
+k_2df_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
+           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = MH / 16;
+    constexpr int PS = fft_padded_size(MH);
+    const int t = threadIdx.x, cc = t / TPT, g = t - (t / TPT) * TPT;
+    const int64_t img = img0 + blockIdx.y;
+    const int f = blockIdx.x * kFC + cc;
+    const bool active = f <= W;
+    const int fc = active ? f : W;
+    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    const int64_t c = img / B;
+    const float2* sp = spec + (int64_t(step) * C + c) * spec_row_stride + int64_t(fc) * (2 * MH);
+    float2 x[2][16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int p = g + TPT * s;
+        const float2 v = ws_img[int64_t(fc) * MH + p];
+        x[0][s] = v;
+        x[1][s] = cmul(v, __ldg(tb.twist_h + p));
+    }
+    float2* const buf[2] = {smem + (2 * cc) * PS, smem + (2 * cc + 1) * PS};
+    reg_fft_forward<MH, 2>(x, buf, g, tb.fftH);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        x[0][k] = cmul(x[0][k], __ldg(sp + k * TPT + g));
+        x[1][k] = cmul(x[1][k], __ldg(sp + MH + k * TPT + g));
+    }
+    reg_fft_inverse<MH, 2>(x, buf, g, tb.fftH);
+    if (active) {
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {
+            const int p = g + TPT * s;
+            ws_img[int64_t(fc) * MH + p] = cadd(x[0][s], cmulc(x[1][s], __ldg(tb.twist_h + p)));
+        }
+    }
+}
+
 template <int MW>
 size_t row_smem() {
     return size_t(2) * kRB * fft_padded_size(MW) * sizeof(float2);
@@ -301,29 +512,47 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
     const int64_t spec_stride = int64_t(p.spec_row_bytes / sizeof(float2));
     const int H = int(p.H), W = int(p.W);
-    const size_t smA = row_smem<MW>();
-    const size_t smB = col_smem2<MH>(kCB);
-    auto ka = k_2d_rows_fwd<MW, T, 0>;
-    auto kb = k_2d_cols<MH, 0>;
-    auto kc = k_2d_rows_inv<MW, T, true>;
-    auto kca = k_2d_rows_inv<MW, T, false>;
-    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
-    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    const unsigned ncolblk = unsigned((W + 1 + kCB - 1) / kCB);
+    constexpr int FR = MH < 32 ? MH : 32;   // image rows per CTA
+    constexpr int NTR = FR * (MW / 16);
+    constexpr int NTC = kFC * (MH / 16);
+    const size_t smR = size_t(2 * FR) * row_stride_f<MW>() * sizeof(float2);
+    const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
+    auto kb = k_2df_cols<MH>;
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+    const unsigned ncolblk = unsigned((W + 1 + kFC - 1) / kFC);
+    // row passes: register-resident for W/2 >= 16, the generic engine for W = 16
+    auto launch_rows_fwd = [&](int64_t i0, int64_t g) {
+        if constexpr (MW >= 16) {
+            auto ka = k_2df_rows_fwd<MW, FR, T, 0>;
+            cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
+            ka<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, a.workspace, tb, a.B, p.C, p.order, H, i0, stride, 0);
+        } else {
+            auto ka = k_2d_rows_fwd<MW, T, 0>;
+            cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+            ka<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, a.workspace, tb, a.B, p.C, p.order,
+                                                                              H, i0, stride, 0);
+        }
+    };
+    auto launch_rows_inv = [&](int64_t i0, int64_t g, bool final_step, int gnext) {
+        if constexpr (MW >= 16) {
+            auto kc = final_step ? k_2df_rows_inv<MW, FR, T, true> : k_2df_rows_inv<MW, FR, T, false>;
+            cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
+            kc<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, gnext, H, i0,
+                                                            stride);
+        } else {
+            auto kc = final_step ? k_2d_rows_inv<MW, T, true> : k_2d_rows_inv<MW, T, false>;
+            cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+            kc<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, y, a.workspace, tb, a.B, p.C,
+                                                                              p.order, gnext, H, i0, stride);
+        }
+    };
     for (int64_t i0 = 0; i0 < nimg; i0 += G) {
         const int64_t g = nimg - i0 < G ? nimg - i0 : G;
-        const dim3 gridR(H / kRB, unsigned(g));
-        ka<<<gridR, kRowThreads, smA, s>>>(u, a.workspace, tb, a.B, p.C, p.order, H, i0, stride, 0);
+        launch_rows_fwd(i0, g);
         for (int st = 1; st < p.order; ++st) {
-            kb<<<dim3(ncolblk, unsigned(g)), kColThreads2, smB, s>>>(a.workspace, spec, tb, W, a.B, p.C, st - 1, i0,
-                                                                     stride, spec_stride, nullptr, 0.0f);
-            if (st < p.order - 1)
-                kca<<<gridR, kRowThreads, smA, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, p.order - st - 1, H, i0,
-                                                     stride);
-            else
-                kc<<<gridR, kRowThreads, smA, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, 0, H, i0, stride);
+            kb<<<dim3(ncolblk, unsigned(g)), NTC, smC, s>>>(a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride,
+                                                            spec_stride);
+            launch_rows_inv(i0, g, st == p.order - 1, st < p.order - 1 ? p.order - st - 1 : 0);
         }
     }
     return cudaGetLastError();

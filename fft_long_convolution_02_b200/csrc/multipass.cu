@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"
+#include "reg_fft.cuh"
 
 namespace hyena {
 
@@ -169,15 +170,15 @@ __device__ __forceinline__ float4 pair_spec(float2 A, float2 Bv, float2 w, float
 // MODE 1: spectrum build: workspace row i is spectrum row r = row0 + i
 //         (= step*C + c); the pair entries of K~ replace the unit in place.
 template <int M2, int MODE>
-__global__ void k_mp_pass_b(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1,
-                            int64_t row0, int64_t ws_row_stride, int64_t spec_row_stride4, int step,
-                            int64_t B, int64_t C, const float* __restrict__ D) {
-    extern __shared__ float2 smem[];
+__device__ __forceinline__ void mp_unit_generic(float2* __restrict__ ws, const float4* __restrict__ spec,
+                                                const MpTables& tb, int M1, int64_t row0, int64_t ws_row_stride,
+                                                int64_t spec_row_stride4, int step, int64_t B, int64_t C,
+                                                const float* __restrict__ D, int unit_index, float2* smem) {
     constexpr int PS = fft_padded_size(M2);
     const int M = M1 * M2;
     const int64_t L = int64_t(2) * M;
-    const bool odd = blockIdx.x >= unsigned(M1 / 2);
-    const int u = odd ? int(blockIdx.x) - M1 / 2 : int(blockIdx.x);
+    const bool odd = unit_index >= M1 / 2;
+    const int u = odd ? unit_index - M1 / 2 : unit_index;
     const int ra = u;                       // first row of the unit (0 for chain e unit 0)
     const int64_t r = row0 + blockIdx.y;
     float2* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
@@ -271,6 +272,15 @@ __global__ void k_mp_pass_b(float2* __restrict__ ws, const float4* __restrict__ 
     }
 }
 
+template <int M2, int MODE>
+__global__ void k_mp_pass_b(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1,
+                            int64_t row0, int64_t ws_row_stride, int64_t spec_row_stride4, int step,
+                            int64_t B, int64_t C, const float* __restrict__ D) {
+    extern __shared__ float2 smem[];
+    mp_unit_generic<M2, MODE>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D,
+                              int(blockIdx.x), smem);
+}
+
 // ------------------------------------------------------------------ pass C
 // FINAL: output gate x0 and store y.  Otherwise: gate with x_{gnext}, then
 // run the next step's pass A on the same columns.
@@ -325,6 +335,229 @@ k_mp_pass_c(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws,
     if (!FINAL) cols_forward_store<M1>(smem, tb, ws_row, M2, n2_0);
 }
 
+// ===========================================================================
+// Register-resident passes (reg_fft.cuh).  Column passes: a CTA of M1 threads
+// handles 16 columns n2; thread t = 16 g + j holds 16 points of column j for
+// both chains.  Row pass: a CTA handles NU units of two rows; thread g of a
+// unit holds 16 points of both rows.  After the forward row FFT, row a's
+// position q pairs with row b's position M2-1-q (every digit of the bin is
+// complemented), so thread g finds its partners at thread M2/16-1-g, slot
+// 15-k; the spectrum entries of these units are stored in that thread order,
+// entry [k][g].  Chain e unit 0 (rows 0 and M1/2, partners inside each row)
+// keeps the natural entry order and the generic kernel above.
+// ===========================================================================
+
+template <int M1>
+__device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables& tb, float2* __restrict__ ws_row,
+                                              int M2, int n2, int g) {
+    const int M = M1 * M2;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int m1 = fft_pos_bin<M1>(16 * g + k);
+        const float2 tw = __ldg(tb.four + int64_t(m1) * M2 + n2);
+        ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2] = cmul(x[0][k], tw);
+        ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2] = cmul(x[1][k], tw);
+    }
+}
+
+// MODE 0: gated input x_{order-1} * v from u (first order step); MODE 1: filter k.
+template <int M1, typename T, int MODE>
+__global__ void __launch_bounds__(M1, 512 / M1)
+k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, const float* __restrict__ sc_w,
+               const float* __restrict__ sc_b, int64_t B, int64_t C, int order, int M2, int64_t row0,
+               int64_t ws_row_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = M1 / 16;
+    constexpr int PS = fft_padded_size(M1);
+    const int t = threadIdx.x, j = t & 15, g = t >> 4;
+    const int n2 = blockIdx.x * 16 + j;
+    const int64_t r = row0 + blockIdx.y;
+    const int64_t L = int64_t(2) * M1 * M2;
+    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    const T* xg;
+    const T* vr = nullptr;
+    Taps tg{}, tv{};
+    if (MODE == 0) {
+        const int64_t c = r / B, b = r - (r / B) * B;
+        const int64_t Ctot = int64_t(order + 1) * C;
+        const T* ub = src + b * Ctot * L;
+        xg = ub + (int64_t(order - 1) * C + c) * L;
+        vr = ub + (int64_t(order) * C + c) * L;
+        tg = load_taps(sc_w, sc_b, int64_t(order - 1) * C + c);
+        tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+    } else {
+        xg = src + r * L;
+    }
+    float2 x[2][16];
+    const float2 tlo = __ldg(tb.twist_lo + n2);
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int n1 = g + TPT * s;
+        const int64_t tt = 2 * (int64_t(M2) * n1 + n2);
+        float2 z;
+        if (MODE == 0) {
+            const float2 a = shortconv_pair(xg, tt, tg);
+            const float2 v = shortconv_pair(vr, tt, tv);
+            z = make_float2(a.x * v.x, a.y * v.y);
+        } else {
+            z = load2(xg + tt);
+        }
+        x[0][s] = z;
+        x[1][s] = cmul(z, cmul(__ldg(tb.twist_hi + n1), tlo));
+    }
+    float2* const buf[2] = {smem + j * PS, smem + (16 + j) * PS};
+    reg_fft_forward<M1, 2>(x, buf, g, tb.fftA);
+    cols_store_ws<M1>(x, tb, ws_row, M2, n2, g);
+}
+
+// Inverse columns.  FINAL: output gate x0, store y.  Otherwise gate with
+// x_{gnext} and run the next step's forward column pass in place.
+template <int M1, typename T, bool FINAL>
+__global__ void __launch_bounds__(M1, 512 / M1)
+k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, MpTables tb,
+               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
+               int gnext, int M2, int64_t row0, int64_t ws_row_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = M1 / 16;
+    constexpr int PS = fft_padded_size(M1);
+    const int t = threadIdx.x, j = t & 15, g = t >> 4;
+    const int n2 = blockIdx.x * 16 + j;
+    const int M = M1 * M2;
+    const int64_t r = row0 + blockIdx.y;
+    const int64_t L = int64_t(2) * M;
+    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    float2 x[2][16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int m1 = fft_pos_bin<M1>(16 * g + k);
+        const float2 tw = __ldg(tb.four + int64_t(m1) * M2 + n2);
+        x[0][k] = cmulc(ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2], tw);
+        x[1][k] = cmulc(ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2], tw);
+    }
+    float2* const buf[2] = {smem + j * PS, smem + (16 + j) * PS};
+    reg_fft_inverse<M1, 2>(x, buf, g, tb.fftA);
+    const int64_t c = r / B, b = r - (r / B) * B;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const T* ub = u + b * Ctot * L;
+    const int gate = FINAL ? 0 : gnext;
+    const T* xg = ub + (int64_t(gate) * C + c) * L;
+    const Taps tg = load_taps(sc_w, sc_b, int64_t(gate) * C + c);
+    T* yr = y + (b * C + c) * L;
+    const float2 tlo = __ldg(tb.twist_lo + n2);
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int n1 = g + TPT * s;
+        const int64_t n = int64_t(M2) * n1 + n2;
+        const float2 tw = cmul(__ldg(tb.twist_hi + n1), tlo);
+        const float2 zp = cadd(x[0][s], cmulc(x[1][s], tw));
+        const float2 a = shortconv_pair(xg, 2 * n, tg);
+        const float2 z = make_float2(a.x * zp.x, a.y * zp.y);
+        if (FINAL) {
+            store2(yr + 2 * n, z);
+        } else {
+            x[0][s] = z;
+            x[1][s] = cmul(z, tw);
+        }
+    }
+    if (!FINAL) {
+        reg_fft_forward<M1, 2>(x, buf, g, tb.fftA);
+        cols_store_ws<M1>(x, tb, ws_row, M2, n2, g);
+    }
+}
+
+// Row pass over the units other than chain e unit 0.  Units are numbered
+// 0 .. M1-2: chain e units 1 .. M1/2-1, then chain o units 0 .. M1/2-1.
+// MODE 0: convolution; MODE 1: spectrum build (pair entries in [k][g] order).
+template <int M2, int NU, int MODE>
+__global__ void __launch_bounds__(NU * (M2 / 16), 512 / (NU * (M2 / 16)) > 0 ? 512 / (NU * (M2 / 16)) : 1)
+k_mpf_rows(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1, int64_t row0,
+           int64_t ws_row_stride, int64_t spec_row_stride4, int step, int64_t B, int64_t C,
+           const float* __restrict__ D) {
+    extern __shared__ float2 smem[];
+    if (blockIdx.x == gridDim.x - 1) {
+        // chain e unit 0 (rows 0 and M1/2; partners inside each row, natural entry order)
+        mp_unit_generic<M2, MODE>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D, 0, smem);
+        return;
+    }
+    constexpr int TPT = M2 / 16;
+    constexpr int PS = fft_padded_size(M2);
+    const int t = threadIdx.x, w = t / TPT, g = t - (t / TPT) * TPT;
+    const int M = M1 * M2;
+    const int64_t L = int64_t(2) * M;
+    const int units = M1 - 1;
+    const int ug = int(blockIdx.x) * NU + w;
+    const bool active = ug < units;
+    const int ugc = active ? ug : units - 1;
+    const bool odd = ugc >= M1 / 2 - 1;
+    const int u = odd ? ugc - (M1 / 2 - 1) : ugc + 1;
+    const int ra = u;
+    float2* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
+    float2* const buf[2] = {smem + (2 * w) * PS, smem + (2 * w + 1) * PS};
+    float2 x[2][16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        x[0][s] = unit[g + TPT * s];
+        x[1][s] = unit[M2 + g + TPT * s];
+    }
+    reg_fft_forward<M2, 2>(x, buf, g, tb.fftB);
+    // pair step: row b goes through shared memory to its partner thread
+    const int base = fft_pad(16 * g);
+    const int pbase = fft_pad(16 * (TPT - 1 - g));
+#pragma unroll
+    for (int k = 0; k < 16; ++k) buf[1][base + k] = x[1][k];
+    __syncthreads();
+    const int64_t r = row0 + blockIdx.y;
+    float2 wa = __ldg(tb.unt1 + ra);
+    if (odd) wa = cmul(wa, __ldg(tb.unt_c));
+    if (MODE == 0) {
+        const int64_t c = r / B;
+        const float4* sp = spec + (int64_t(step) * C + c) * spec_row_stride4 + (odd ? M / 2 : 0) + int64_t(u) * M2;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int m2 = fft_pos_bin<M2>(16 * g + k);
+            const float2 wk = cmul(wa, __ldg(tb.unt2 + m2));
+            float2 A = x[0][k];
+            float2 Bv = buf[1][pbase + 15 - k];
+            pair_conv(A, Bv, wk, __ldg(sp + k * TPT + g));
+            x[0][k] = A;
+            buf[1][pbase + 15 - k] = Bv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[1][k] = buf[1][base + k];
+        __syncthreads();
+        reg_fft_inverse<M2, 2>(x, buf, g, tb.fftB);
+        if (active) {
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+                unit[g + TPT * s] = x[0][s];
+                unit[M2 + g + TPT * s] = x[1][s];
+            }
+        }
+    } else {
+        const float d = D ? __ldg(D + r) : 0.0f;
+        const float s4 = 1.0f / float(4 * L);
+        float4 out[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int m2 = fft_pos_bin<M2>(16 * g + k);
+            const float2 wk = cmul(wa, __ldg(tb.unt2 + m2));
+            out[k] = pair_spec(x[0][k], buf[1][pbase + 15 - k], wk, d, s4);
+        }
+        __syncthreads();   // every thread of the block has loaded its unit
+        if (active) {
+            float4* sp_out = reinterpret_cast<float4*>(unit);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sp_out[k * TPT + g] = out[k];
+        }
+    }
+}
+
+template <int M2>
+constexpr int rows_nu() {
+    return (M2 / 16) >= 256 ? 1 : 256 / (M2 / 16);
+}
+
 template <int M1>
 size_t col_smem() {
     return size_t(2) * kNB2 * fft_padded_size(M1) * sizeof(float2);
@@ -341,26 +574,28 @@ cudaError_t spectrum_mp(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     float2* rows = reinterpret_cast<float2*>(a.spectrum + p.spec_off);
     const int64_t nrows = (p.order - 1) * p.C;
     const int64_t stride = int64_t(p.spec_row_bytes / sizeof(float2));
-    const size_t smA = col_smem<M1>();
+    constexpr int NU = rows_nu<M2>();
+    const size_t smA = size_t(32) * fft_padded_size(M1) * sizeof(float2);
     const size_t smB = size_t(2) * fft_padded_size(M2) * sizeof(float2);
-    auto kbf = k_mp_pass_a<M1, float, 1>;
-    auto kbh = k_mp_pass_a<M1, __nv_bfloat16, 1>;
-    auto kb = k_mp_pass_b<M2, 1>;
-    cudaFuncSetAttribute(kbf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kbh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    const size_t smR = size_t(2 * NU) * fft_padded_size(M2) * sizeof(float2);
+    auto kaf = k_mpf_cols_fwd<M1, float, 1>;
+    auto kah = k_mpf_cols_fwd<M1, __nv_bfloat16, 1>;
+    auto kr = k_mpf_rows<M2, NU, 1>;
+    cudaFuncSetAttribute(kaf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kah, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
+    const unsigned rblocks = unsigned((M1 - 1 + NU - 1) / NU);
     for (int64_t r0 = 0; r0 < nrows; r0 += 32768) {
         const int64_t g = nrows - r0 < 32768 ? nrows - r0 : 32768;
-        if (a.k_dtype == DT_F32) {
-            kbf<<<dim3(M2 / kNB2, unsigned(g)), kColThreads, smA, s>>>(
-                static_cast<const float*>(a.k), rows + r0 * stride, tb, nullptr, nullptr, 1, 1, 2, M2, r0, stride);
-        } else {
-            kbh<<<dim3(M2 / kNB2, unsigned(g)), kColThreads, smA, s>>>(
-                static_cast<const __nv_bfloat16*>(a.k), rows + r0 * stride, tb, nullptr, nullptr, 1, 1, 2, M2, r0,
-                stride);
-        }
-        kb<<<dim3(M1, unsigned(g)), row_threads<M2>(), smB, s>>>(rows + r0 * stride, nullptr, tb, M1, r0, stride, 0,
-                                                                 0, 1, p.C, a.D);
+        if (a.k_dtype == DT_F32)
+            kaf<<<dim3(M2 / 16, unsigned(g)), M1, smA, s>>>(static_cast<const float*>(a.k), rows + r0 * stride, tb,
+                                                             nullptr, nullptr, 1, 1, 2, M2, r0, stride);
+        else
+            kah<<<dim3(M2 / 16, unsigned(g)), M1, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + r0 * stride,
+                                                             tb, nullptr, nullptr, 1, 1, 2, M2, r0, stride);
+        // every unit; the last block of each row takes chain e unit 0
+        kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(rows + r0 * stride, nullptr, tb, M1, r0,
+                                                                       stride, 0, 0, 1, p.C, a.D);
     }
     return cudaGetLastError();
 }
@@ -375,29 +610,32 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     int64_t G = a.group_rows < 65535 ? a.group_rows : 65535;
     const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
     const int64_t spec_stride4 = int64_t(p.spec_row_bytes / 16);
-    const size_t smA = col_smem<M1>();
+    constexpr int NU = rows_nu<M2>();
+    const size_t smA = size_t(32) * fft_padded_size(M1) * sizeof(float2);
     const size_t smB = size_t(2) * fft_padded_size(M2) * sizeof(float2);
-    auto ka = k_mp_pass_a<M1, T, 0>;
-    auto kb = k_mp_pass_b<M2, 0>;
-    auto kc = k_mp_pass_c<M1, T, true>;
-    auto kca = k_mp_pass_c<M1, T, false>;
+    const size_t smR = size_t(2 * NU) * fft_padded_size(M2) * sizeof(float2);
+    auto ka = k_mpf_cols_fwd<M1, T, 0>;
+    auto kr = k_mpf_rows<M2, NU, 0>;
+    auto kc = k_mpf_cols_inv<M1, T, true>;
+    auto kca = k_mpf_cols_inv<M1, T, false>;
     cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
     cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
     cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    const unsigned rblocks = unsigned((M1 - 1 + NU - 1) / NU);
     for (int64_t r0 = 0; r0 < rows; r0 += G) {
         const int64_t g = rows - r0 < G ? rows - r0 : G;
-        const dim3 gridA(M2 / kNB2, unsigned(g));
-        ka<<<gridA, kColThreads, smA, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
+        const dim3 gridA(M2 / 16, unsigned(g));
+        ka<<<gridA, M1, smA, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
         for (int st = 1; st < p.order; ++st) {
-            kb<<<dim3(M1, unsigned(g)), row_threads<M2>(), smB, s>>>(a.workspace, spec, tb, M1, r0, stride,
-                                                                      spec_stride4, st - 1, a.B, p.C, nullptr);
+            kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(a.workspace, spec, tb, M1, r0, stride,
+                                                                           spec_stride4, st - 1, a.B, p.C, nullptr);
             if (st < p.order - 1) {
-                kca<<<gridA, kColThreads, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
-                                                     p.order - st - 1, M2, r0, stride);
+                kca<<<gridA, M1, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
+                                            p.order - st - 1, M2, r0, stride);
             } else {
-                kc<<<gridA, kColThreads, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2,
-                                                    r0, stride);
+                kc<<<gridA, M1, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2, r0,
+                                           stride);
             }
         }
     }
