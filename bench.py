@@ -58,6 +58,8 @@ def spectrum_row_bytes(p) -> int:
     """Stored spectrum bytes per (step, channel) row of the library's layout."""
     if p.ndim == 2:
         return (p.W + 1) * 2 * p.H * 8
+    if p.L == 8192:
+        return 16 * p.L                     # all 2L bins, complex64
     if p.L <= 16384:
         return (p.L // 2 + 1) * 16
     return 8 * p.L

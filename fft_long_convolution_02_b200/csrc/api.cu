@@ -203,6 +203,8 @@ hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, c
     if (h.magic != kSpecMagic || h.version != kSpecVersion || h.path != p.path || h.C != p.C || h.L != p.L ||
         h.H != p.H || h.W != p.W || h.order != p.order || size_t(h.total_bytes) != p.total_bytes)
         return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum header does not match (C, sizes, order)");
+    if (h.device_status != 0)
+        return fail(HYENA_ERR_INTERNAL, "a convolution with this spectrum gave up waiting for the tensor cores");
     return ok();
 }
 

@@ -32,6 +32,7 @@ struct ConvArgs {
 cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);
 cudaError_t launch_spectrum_onchip(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_onchip(const Plan& p, const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);

@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"
+#include "pairs4096.cuh"
 
 namespace hyena {
 
@@ -303,90 +304,6 @@ __device__ __forceinline__ void apply_stage1_twiddles(float2 (&e)[16], float2 (&
     }
 }
 
-__device__ __forceinline__ void pair_conv4096(float2& A, float2& Bv, float2 w, float4 kk) {
-    const float2 S = cadd(A, cconj(Bv));
-    const float2 T = cmul_i(cmul(w, csub(A, cconj(Bv))));
-    const float2 Yf = cmul(csub(S, T), make_float2(kk.x, kk.y));
-    const float2 Yg = cmul(cconj(cadd(S, T)), make_float2(kk.z, kk.w));
-    const float2 P = cadd(Yf, cconj(Yg));
-    const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
-    A = cadd(P, U);
-    Bv = cconj(csub(P, U));
-}
-
-// Pair step with a fixed thread mapping: thread t handles chain e pairs
-// j = t + 256 i (i < 8; thread 0 also j = 2048) and chain o pairs
-// j = t + 256 i (i < 8).  For t != 0 both members sit at compile-time
-// offsets from per-thread bases, and the pair twiddles are w_L^t w_32^i
-// (chain e) and w_2L^(2t+1) w_32^i (chain o).
-__device__ __forceinline__ void pairs_4096(float2* __restrict__ E, float2* __restrict__ O,
-                                           const float4* __restrict__ spec, const float2* __restrict__ twist,
-                                           const float2* __restrict__ untw) {
-    const int t = threadIdx.x;
-    const float2 wt = __ldg(twist + t);                   // w_L^t
-    const float2 wt_odd = __ldg(untw + (M / 2 + 1) + t);  // w_2L^(2t+1)
-    // position of bin j = t + 256 i: (t & 15) * 256 + (t >> 4) * 16 + i  (padded)
-    const int pa0 = fft_pad((t & 15) * 256 + (t >> 4) * 16);
-    // chain e partner M - j = (256 - t) + 256 (15 - i) for t != 0
-    const int te = (256 - t) & 255;
-    const int pbe0 = fft_pad((te & 15) * 256 + (te >> 4) * 16);
-    // chain o partner M - 1 - j = (255 - t) + 256 (15 - i)
-    const int to = 255 - t;
-    const int pbo0 = fft_pad((to & 15) * 256 + (to >> 4) * 16);
-#pragma unroll
-    for (int i0 = 0; i0 < 8; i0 += 4) {
-        float4 ke[4], ko[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            ke[k] = __ldg(spec + t + 256 * (i0 + k));
-            ko[k] = __ldg(spec + (M / 2 + 1) + t + 256 * (i0 + k));
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = i0 + k;
-            const float2 w32i = w32(i);
-            // chain e
-            if (t == 0 && i == 0) {
-                const float2 A = E[pa0];
-                const float y0 = 2.0f * (A.x + A.y) * ke[0].x;
-                const float yL = 2.0f * (A.x - A.y) * ke[0].z;
-                E[pa0] = make_float2(y0 + yL, y0 - yL);
-            } else {
-                // partner: t != 0 -> pbe0 + (15 - i); t == 0, i >= 1 -> bin 256 (16 - i)
-                const int pb = (t != 0) ? pbe0 + (15 - i) : (16 - i);
-                float2 A = E[pa0 + i];
-                float2 Bv = E[pb];
-                pair_conv4096(A, Bv, cmul(wt, w32i), ke[k]);
-                E[pa0 + i] = A;
-                E[pb] = Bv;
-            }
-            // chain o
-            {
-                const int pb = pbo0 + (15 - i);
-                float2 A = O[pa0 + i];
-                float2 Bv = O[pb];
-                pair_conv4096(A, Bv, cmul(wt_odd, w32i), ko[k]);
-                O[pa0 + i] = A;
-                O[pb] = Bv;
-            }
-        }
-    }
-    if (t == 0) {
-        // chain e self pair j = M/2 = 2048: bin 2048 -> position 8 (w = w_L^2048 = -i)
-        const int p = fft_pad(8);
-        float2 A = E[p];
-        const float4 kk = __ldg(spec + M / 2);
-        const float2 w = make_float2(0.0f, -1.0f);
-        const float2 S = cadd(A, cconj(A));
-        const float2 T = cmul_i(cmul(w, csub(A, cconj(A))));
-        const float2 Yf = cmul(csub(S, T), make_float2(kk.x, kk.y));
-        const float2 Yg = cmul(cconj(cadd(S, T)), make_float2(kk.z, kk.w));
-        const float2 P = cadd(Yf, cconj(Yg));
-        const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
-        E[p] = cadd(P, U);
-    }
-}
-
 template <typename T>
 __global__ void __launch_bounds__(NT, 2)
 k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
@@ -491,11 +408,48 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
 #pragma unroll
             for (int s = 0; s < 16; ++s) { E[base3 + s] = e[s]; O[base3 + s] = o[s]; }
             __syncthreads();
-            pairs_4096(E, O, spec + (int64_t(st - 1) * C + c) * (M + 1), twist, untw);
+            {
+                // pair step (position layout): every thread computes its own
+                // bins from its own and the partner's value; chain e first (own
+                // values in registers), then chain o (own values from O)
+                const float2* sp = reinterpret_cast<const float2*>(spec) + (int64_t(st - 1) * C + c) * (4 * M) +
+                                   kSpec8192Plane / 2;
+                const int lo = t & 15, hi = t >> 4;
+                const float2 we = __ldg(twist + (hi + 16 * lo));
+                const int pre = p4096::partner_row_e(t);
+                const int pbe = fft_pad(16 * pre);
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    const float2 Kf = __ldg(sp + cc * 256 + t);
+                    if (t == 0 && cc == 0) {
+                        const float2 Av = e[0];
+                        const float y0 = 2.0f * (Av.x + Av.y) * Kf.x;
+                        const float yL = 2.0f * (Av.x - Av.y) * Kf.y;
+                        e[0] = make_float2(y0 + yL, y0 - yL);
+                    } else {
+                        const int cp = (t == 0) ? 16 - cc : 15 - cc;
+                        const float2 Bv = E[(t == 0) ? (16 - cc) : (pbe + 15 - cc)];
+                        const float2 Kg = __ldg(sp + cp * 256 + pre);
+                        e[cc] = p4096::pair_own(e[cc], Bv, Kf, Kg, cmul(we, p4096::w32c(cc)));
+                    }
+                }
+                __syncthreads();                          // all partner reads of E done
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) E[base3 + cc] = e[cc];
+                const float2 wo = cmul(we, __ldg(untw + (M / 2 + 1)));   // times w_2L^1
+                const int pro = p4096::partner_row_o(t);
+                const int pbo = fft_pad(16 * pro);
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    const float2 Kf = __ldg(sp + M + cc * 256 + t);
+                    const float2 Kg = __ldg(sp + M + (15 - cc) * 256 + pro);
+                    o[cc] = p4096::pair_own(O[base3 + cc], O[pbo + 15 - cc], Kf, Kg, cmul(wo, p4096::w32c(cc)));
+                }
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) e[cc] = E[base3 + cc];
+            }
             __syncthreads();
             // inverse stage 3
-#pragma unroll
-            for (int s = 0; s < 16; ++s) { e[s] = E[base3 + s]; o[s] = O[base3 + s]; }
             dft16x2<true>(e, o);
 #pragma unroll
             for (int s = 0; s < 16; ++s) { E[base3 + s] = e[s]; O[base3 + s] = o[s]; }
@@ -550,8 +504,97 @@ constexpr size_t conv_4096_smem() {
 
 }  // namespace r16
 
+// Spectrum of the L = 8192 kernels: K~[f] = (X[f] + D) / (2L) for all 2L bins
+// of the zero-padded transform X = FFT_2L(k), in the two planes described in
+// pairs4096.cuh.  X[f] for f <= L comes from the
+// packed transform Z = FFT_L(k[2n] + i k[2n+1]) (chains e, o as in the
+// convolution kernels):
+//   X[f] = ((Z[f] + conj Z[L-f]) - i w_2L^f (Z[f] - conj Z[L-f])) / 2,
+// X[0] = Re Z[0] + Im Z[0], X[L] = Re Z[0] - Im Z[0]; X[2L-f] = conj X[f].
+
+template <typename TK>
+__global__ void __launch_bounds__(512)
+k_spectrum_8192(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* __restrict__ spectrum) {
+    extern __shared__ float2 smem[];
+    constexpr int M = 4096, L = 8192;
+    constexpr int PS = fft_padded_size(M);
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
+    const float2* tw_fft = tables;
+    const float2* twist = tables + fft_tw_size(M);
+    const float2* untw = twist + M;
+    const int64_t row = blockIdx.x;  // s * C + c
+    const TK* kr = k + row * L;
+    const float d = D ? __ldg(D + row) : 0.0f;
+    float2* be = smem;
+    float2* bo = smem + PS;
+    for (int n = threadIdx.x; n < M; n += blockDim.x) {
+        const float2 z = load2(kr + 2 * n);
+        be[fft_pad(n)] = z;
+        bo[fft_pad(n)] = cmul(z, __ldg(twist + n));
+    }
+    __syncthreads();
+    cta_fft_forward<M>(smem, 2, PS, tw_fft);
+    // bin m of a chain sits at position 256 (m & 15) + 16 ((m >> 4) & 15) + (m >> 8)
+    auto at = [&](const float2* buf, int m) {
+        return buf[fft_pad(256 * (m & 15) + 16 * ((m >> 4) & 15) + (m >> 8))];
+    };
+    uint32_t* out = reinterpret_cast<uint32_t*>(spectrum + h->spec_off + size_t(row) * size_t(16 * L));
+    const float sN = 1.0f / float(2 * L);
+    const float2 w2l = __ldg(untw + (M / 2 + 1));          // w_2L^1
+    for (int f = threadIdx.x; f < 2 * L; f += blockDim.x) {
+        const bool mir = f > L;
+        const int ff = mir ? 2 * L - f : f;
+        float2 X;
+        if (ff == 0 || ff == L) {
+            const float2 Z0 = at(be, 0);
+            X = make_float2(ff == 0 ? Z0.x + Z0.y : Z0.x - Z0.y, 0.0f);
+        } else {
+            const int m = ff >> 1;
+            const bool o = ff & 1;
+            const float2 Av = o ? at(bo, m) : at(be, m);
+            const float2 Bv = o ? at(bo, M - 1 - m) : at(be, M - m);
+            float2 w = __ldg(twist + m);                        // w_L^m = w_2L^(2m)
+            if (o) w = cmul(w, w2l);                            // w_2L^(2m+1)
+            const float2 S = cadd(Av, cconj(Bv));
+            const float2 T = cmul_i(cmul(w, csub(Av, cconj(Bv))));
+            X = cscale(csub(S, T), 0.5f);
+        }
+        const float2 K = make_float2((X.x + d) * sN, (mir ? -X.y : X.y) * sN);
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(K.x, K.y);
+        out[spec8192_pos(f)] = *reinterpret_cast<const uint32_t*>(&hb);
+        // plane 1 (position layout, half scale)
+        float* p1 = reinterpret_cast<float*>(out + kSpec8192Plane);
+        if (f == 0) {
+            p1[0] = 0.5f * K.x;
+        } else if (f == L) {
+            p1[1] = 0.5f * K.x;
+        } else if (f < L) {
+            const int m = f >> 1;
+            const int pos = 256 * (m & 15) + 16 * ((m >> 4) & 15) + (m >> 8);
+            const int e = (f & 1) * M + (pos & 15) * 256 + (pos >> 4);
+            p1[2 * e] = 0.5f * K.x;
+            p1[2 * e + 1] = 0.5f * K.y;
+        }
+    }
+}
+
 template <int M>
 cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    if constexpr (M == 4096) {
+        const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
+        const unsigned grid = unsigned((p.order - 1) * p.C);
+        if (a.k_dtype == DT_F32) {
+            auto kern = k_spectrum_8192<float>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            kern<<<grid, 512, smem, s>>>(static_cast<const float*>(a.k), a.D, a.spectrum);
+        } else {
+            auto kern = k_spectrum_8192<__nv_bfloat16>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            kern<<<grid, 512, smem, s>>>(static_cast<const __nv_bfloat16*>(a.k), a.D, a.spectrum);
+        }
+        return cudaGetLastError();
+    }
     constexpr int NT = onchip_threads<M>();
     const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
     const unsigned grid = unsigned((p.order - 1) * p.C);
@@ -586,7 +629,8 @@ cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
 template <int M>
 cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     if constexpr (M == 4096) {
-        return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : conv_4096<__nv_bfloat16>(p, a, s);
+        // bf16 storage: DFT stages on the tensor cores; fp32 storage: fp32 FFT
+        return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : launch_conv_8192_tc(p, a, s);
     }
     constexpr int NT = onchip_threads<M>();
     const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);

@@ -1,0 +1,550 @@
+// onchip_tc.cu -- L = 8192, bf16 storage: the gated FFT convolution with its
+// DFT stages on the tensor cores (tcgen05).
+//
+// Two batch rows b0, b1 of one channel share the filter, and the filter is
+// real, so they travel as one complex signal z = g[b0] + i g[b1] (g = the
+// gated input of the order step): the circular convolution of z with the
+// zero-padded filter k has real part y[b0] and imaginary part y[b1].  Each
+// CTA therefore runs one complex FFT of N = 2L = 16384 points (upper half of
+// the input zero), a point-wise product with K~ = (FFT_N(k) + D) / N, and the
+// inverse FFT, keeping the first L outputs -- no real-to-complex untangling.
+//
+// FFT_N factors as 16 x 32 x 32 (decimation in frequency):
+//   n = a + 1024 s (s < 8 non-zero), a = b + 32 q,   f = k1 + 16 k2 + 512 k3
+//   stage 1: Y1[a][k1]    = sum_s z[a + 1024 s] w16^(s k1)     x w_N^(a k1)
+//   stage 2: Y2[k1,b][k2] = sum_q Y1[b + 32 q][k1] w32^(q k2)  x w1024^(b k2)
+//   stage 3: X[k1,k2][k3] = sum_b Y2[k1,b][k2] w32^(b k3)
+// and the inverse runs the same stages backwards.  Every stage is one batched
+// product of the stage's vectors (rows) with the real form of a DFT matrix:
+// operands bf16 in shared memory, fp32 accumulators in tensor memory.  The
+// inverse uses the forward matrices through IDFT(x) = conj(DFT(conj x)); the
+// spectrum pass stores conj(X K~) and the final conjugation folds into the
+// output gate.
+//
+// Between stages every thread reads accumulator rows from tensor memory,
+// applies the twiddles in fp32 and scatters the values into the next stage's
+// operand.  The row orders below are chosen so that each thread's values for
+// one destination row are four consecutive slots: one 16-byte store.
+//   stage-1 rows   rho1(a)     = 128 T + 32 Q + b, q = a >> 5, b = a & 31,
+//                                T = (q & 3) + 4 (q >> 4), Q = (q >> 2) & 3
+//   stage-2 rows   rho2(k1, b) = 128 (b & 3) + 32 (k1 >> 2) + 8 (k1 & 3) + (b >> 2)
+//   stage-3 rows   rho2(k1, k2)
+//   stage-2' rows  128 (k1 & 3) + 32 (k1 >> 2) + b
+//   stage-1' rows  a
+// Thread (warp w, lane): lane quarter Q = w & 3, half h = w >> 2.
+//
+// Precision: the stage operands and the DFT matrices are rounded to bf16 (8
+// significant bits) six times per order step; the resulting row error is a
+// few 1e-3 relative to the output, inside the bf16-storage tolerance.  fp32
+// storage keeps the fp32 kernel.
+#include "common.cuh"
+#include "kernels.h"
+#include "plan_common.h"
+#include "tc_util.cuh"
+
+namespace hyena {
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int L = 8192;
+constexpr int N = 16384;
+constexpr int NT = 256;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSBO16 = 2 * tc::kLBO;   // operand with K = 16
+constexpr uint32_t kSBO32 = 4 * tc::kLBO;   // K = 32
+constexpr uint32_t kSBO64 = 8 * tc::kLBO;   // K = 64
+constexpr uint32_t kAbytes = 64 * kSBO64;   // 512 rows x K 64 = 1024 rows x K 32
+constexpr uint32_t kB1bytes = 4 * kSBO16;   // N 32 x K 16
+constexpr uint32_t kB32bytes = 8 * kSBO64;  // N 64 x K 64
+constexpr uint32_t kB1ibytes = 2 * kSBO32;  // N 16 x K 32
+constexpr uint32_t kTW2bytes = 4 * 16 * 8 * 16;
+constexpr uint32_t kOffB1 = kAbytes;
+constexpr uint32_t kOffB32 = kOffB1 + kB1bytes;
+constexpr uint32_t kOffB1i = kOffB32 + kB32bytes;
+constexpr uint32_t kOffTW2 = kOffB1i + kB1ibytes;
+constexpr size_t kSmem = size_t(kOffTW2) + kTW2bytes;
+constexpr int kWaitLimit = 1 << 22;
+static_assert(2 * L * sizeof(float) <= kAbytes, "output staging must fit the operand buffer");
+static_assert(kOffTW2 % 16 == 0, "twiddle table alignment");
+
+__device__ __forceinline__ uint32_t pack_bf16(float re, float im) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(re, im);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+__device__ __forceinline__ void sts128(uint8_t* base, uint32_t off, uint32_t x, uint32_t y, uint32_t z,
+                                       uint32_t w) {
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(x, y, z, w);
+}
+
+__device__ __forceinline__ int rho1(int a) {
+    const int q = a >> 5, b = a & 31;
+    return 128 * ((q & 3) + 4 * (q >> 4)) + 32 * ((q >> 2) & 3) + b;
+}
+
+// w_N^e for any integer e: quarter-turn reduction onto the tables
+// (twist[j] = w_N^(2j), odd[j] = w_N^(2j+1), j < 2048).
+__device__ __forceinline__ float2 wN(int e, const float2* __restrict__ twist, const float2* __restrict__ odd) {
+    e &= N - 1;
+    const int q = e >> 12, r = e & 4095;
+    float2 v = (r & 1) ? __ldg(odd + (r >> 1)) : __ldg(twist + (r >> 1));
+    if (q & 1) v = make_float2(v.y, -v.x);   // times -i
+    if (q & 2) v = make_float2(-v.x, -v.y);  // times -1
+    return v;
+}
+
+// Width-3 causal short conv of 8 consecutive samples n0 .. n0+7 (n0 % 8 == 0).
+__device__ __forceinline__ void sc8(const bf16* __restrict__ x, int n0, const Taps& tp, float (&o)[8]) {
+    const uint4 cur = __ldg(reinterpret_cast<const uint4*>(x + n0));
+    const uint32_t halo = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x + n0 - 2)) : 0u;
+    float v[10];
+    v[0] = bf_lo(halo); v[1] = bf_hi(halo);
+    v[2] = bf_lo(cur.x); v[3] = bf_hi(cur.x); v[4] = bf_lo(cur.y); v[5] = bf_hi(cur.y);
+    v[6] = bf_lo(cur.z); v[7] = bf_hi(cur.z); v[8] = bf_lo(cur.w); v[9] = bf_hi(cur.w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = fmaf(tp.w0, v[i], fmaf(tp.w1, v[i + 1], fmaf(tp.w2, v[i + 2], tp.b)));
+}
+__device__ __forceinline__ float sc1(const bf16* __restrict__ x, int n, const Taps& tp) {
+    const float c = __bfloat162float(x[n]);
+    const float p1 = n >= 1 ? __bfloat162float(x[n - 1]) : 0.0f;
+    const float p2 = n >= 2 ? __bfloat162float(x[n - 2]) : 0.0f;
+    return fmaf(tp.w0, p2, fmaf(tp.w1, p1, fmaf(tp.w2, c, tp.b)));
+}
+
+// Real form of a DFT matrix as a K-major B operand: row n = 2 k + (0: re, 1: im)
+// of output k, column j = 2 s + (0: re, 1: im) of input s, entry of w_R^(s k).
+__device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo) {
+    for (int idx = threadIdx.x; idx < 4 * nout * nin; idx += NT) {
+        const int n = idx / (2 * nin), j = idx % (2 * nin);
+        const int e = ((n >> 1) * (j >> 1)) % R;
+        float sv, cv;
+        sincospif(2.0f * float(e) / float(R), &sv, &cv);   // w = cv - i sv
+        float v;
+        if ((n & 1) == 0) v = (j & 1) == 0 ? cv : sv;       // re: Re w xr - Im w xi
+        else v = (j & 1) == 0 ? -sv : cv;                   // im: Im w xr + Re w xi
+        *reinterpret_cast<bf16*>(Bm + tc::kmaj_off(n, j, sbo)) = __float2bfloat16_rn(v);
+    }
+}
+
+// Publish this thread's operand writes and issue the stage's MMAs from one
+// thread (tiles x ksteps MMAs of M = 128), committed to `mbar`.
+__device__ __forceinline__ void stage_issue(uint32_t a, uint32_t sbo_a, uint32_t b, uint32_t sbo_b, int tiles,
+                                            int ksteps, uint32_t idesc, uint32_t tmem, uint32_t dcols,
+                                            uint64_t* mbar) {
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tc::fence_after_sync();
+        for (int T = 0; T < tiles; ++T)
+            for (int ks = 0; ks < ksteps; ++ks)
+                tc::mma_bf16(tmem + uint32_t(T) * dcols,
+                             tc::smem_desc(a + uint32_t(T) * 16u * sbo_a + uint32_t(ks) * 2u * tc::kLBO, sbo_a),
+                             tc::smem_desc(b + uint32_t(ks) * 2u * tc::kLBO, sbo_b), idesc, uint32_t(ks));
+        tc::commit(mbar);
+    }
+}
+// Wait (bounded) for the last issued stage.
+__device__ __forceinline__ bool stage_wait(uint64_t* mbar, uint32_t& phase) {
+    const bool ok = tc::mbar_wait(mbar, phase, kWaitLimit);
+    phase ^= 1u;
+    tc::fence_after_sync();
+    return ok;
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
+               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
+               int64_t npairs) {
+    extern __shared__ __align__(1024) uint8_t smem_tc[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    if (!(h->magic == kSpecMagic && h->path == PATH_ONCHIP_1D && h->C == C && h->L == L && h->order == order &&
+          h->spec_row_bytes == int64_t(N) * 8))
+        return;
+    const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
+    const float2* twist = tables + fft_tw_size(L / 2);        // w_L^j = w_N^(2j)
+    const float2* odd = twist + L / 2 + (L / 4 + 1);          // w_N^(2j+1)
+    const uint32_t* spec = reinterpret_cast<const uint32_t*>(spectrum + h->spec_off);   // plane 0 of each row
+    uint32_t* status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(spectrum) + offsetof(SpecHeader, device_status));
+
+    uint8_t* A = smem_tc;
+    float4* TW2 = reinterpret_cast<float4*>(smem_tc + kOffTW2);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const int64_t nbp = (B + 1) / 2;
+
+    fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16);
+    fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64);
+    fill_dft(smem_tc + kOffB1i, 16, 8, 16, kSBO32);
+    // TW2[(T * 16 + kp) * 8 + l] = (w1024^(b k), w1024^(b (k+1))), b = 4 l + T, k = 2 kp
+    for (int idx = t; idx < 4 * 16 * 8; idx += NT) {
+        const int l = idx & 7, kp = (idx >> 3) & 15, T = idx >> 7;
+        const int bb = 4 * l + T, k = 2 * kp;
+        const float2 w0 = wN(16 * ((bb * k) & 1023), twist, odd);
+        const float2 w1 = wN(16 * ((bb * (k + 1)) & 1023), twist, odd);
+        TW2[idx] = make_float4(w0.x, w0.y, w1.x, w1.y);
+    }
+    if (t == 0) tc::mbar_init(&mbar, 1);
+    if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);     // this warp's lane quarter
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t b1_addr = tc::smem_u32(smem_tc + kOffB1);
+    const uint32_t b32_addr = tc::smem_u32(smem_tc + kOffB32);
+    const uint32_t b1i_addr = tc::smem_u32(smem_tc + kOffB1i);
+    uint32_t phase = 0;
+    bool ok = true;
+
+    for (int64_t P = blockIdx.x; P < npairs; P += gridDim.x) {
+        const int64_t c = P / nbp;
+        const int64_t b0 = 2 * (P - c * nbp);
+        const bool has1 = b0 + 1 < B;
+        const bf16* u0 = u + b0 * Ctot * L;
+        const bf16* u1 = has1 ? u0 + Ctot * L : u0;
+        if (t == 0) {
+            // warm L2 with this pair's spectrum rows (hi plane) and the next pair's rows
+            for (int st = 1; st < order; ++st)
+                tc::prefetch_l2(spec + (int64_t(st - 1) * C + c) * (2 * N), N * 4);
+            const int64_t Pn = P + gridDim.x;
+            if (Pn < npairs) {
+                const int64_t cn = Pn / nbp, bn = 2 * (Pn - cn * nbp);
+                for (int r = 0; r < 2 && bn + r < B; ++r)
+                    for (int g = 0; g <= order; ++g)
+                        tc::prefetch_l2(u + ((bn + r) * Ctot + int64_t(g) * C + cn) * L, L * 2);
+            }
+        }
+        for (int st = 1; st < order; ++st) {
+            const int g = order - st;
+            const Taps tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
+            const bf16* xg0 = u0 + (int64_t(g) * C + c) * L;
+            const bf16* xg1 = u1 + (int64_t(g) * C + c) * L;
+            // ---------------- stage-1 operand: z = g[b0] + i g[b1]
+            if (st == 1) {
+                const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+                const bf16* v0 = u0 + (int64_t(order) * C + c) * L;
+                const bf16* v1 = u1 + (int64_t(order) * C + c) * L;
+                const int chalf = t >> 7, a0 = 8 * (t & 127);
+                uint32_t pk[8][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int n0 = a0 + 1024 * (4 * chalf + j);
+                    float xa[8], va[8], xb[8], vb[8];
+                    sc8(xg0, n0, tg, xa);
+                    sc8(v0, n0, tv, va);
+                    if (has1) {
+                        sc8(xg1, n0, tg, xb);
+                        sc8(v1, n0, tv, vb);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) { xb[i] = 0.0f; vb[i] = 0.0f; }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) pk[i][j] = pack_bf16(xa[i] * va[i], xb[i] * vb[i]);
+                }
+                __syncthreads();                        // operand buffer free (previous pair's output read)
+                // rows rho1(a0 + i) = rho1(a0) + i (a0 % 8 == 0)
+                const uint32_t base = uint32_t(rho1(a0) >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sts128(A, base + 16u * i, pk[i][0], pk[i][1], pk[i][2], pk[i][3]);
+            } else {
+                // previous step's output v = conj(stage-1' accumulators), row a, output s
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int a = 128 * (4 * hh + j) + 32 * Q + lane;
+                    float d[16];
+                    tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
+                    tc::tmem_ld_wait();
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        const int n = a + 1024 * s;
+                        const float za = sc1(xg0, n, tg) * d[2 * s];
+                        const float zb = has1 ? sc1(xg1, n, tg) * -d[2 * s + 1] : 0.0f;
+                        pk[s] = pack_bf16(za, zb);
+                    }
+                    sts128(A, tc::chunk_off(rho1(a), 0, kSBO16), pk[0], pk[1], pk[2], pk[3]);
+                    sts128(A, tc::chunk_off(rho1(a), 1, kSBO16), pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            // ---------------- stage 1: 8 tiles x (K 16 -> N 32)
+            stage_issue(a_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
+            ok &= stage_wait(&mbar, phase);
+            {
+                // twiddle w_N^(a k1); vector a = lane + 32 q, q = j + 4 Q + 16 h
+                // -> stage-2 row (k1, lane), chunk Q + 4 h (slots q, j = 0..3)
+                float2 beta[4], pw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    beta[j] = wN(lane + 32 * (j + 4 * Q + 16 * hh), twist, odd);
+                    pw[j] = make_float2(1.0f, 0.0f);
+                }
+                // row rho2(k1, lane): row / 8 = 16 (lane & 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane >> 2
+                const uint32_t base = uint32_t(16 * (lane & 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
+                                      uint32_t(lane >> 2) * 16u;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float d[4][16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int k1 = 8 * half + kk;
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 v = cmul(make_float2(d[j][2 * kk], d[j][2 * kk + 1]), pw[j]);
+                            pw[j] = cmul(pw[j], beta[j]);
+                            pk[j] = pack_bf16(v.x, v.y);
+                        }
+                        sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64, pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            // ---------------- stage 2: 4 tiles x (K 64 -> N 64)
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            ok &= stage_wait(&mbar, phase);
+            {
+                // rows (k1 = 4 Q + lane / 8, b = 4 (lane & 7) + T), outputs k2 = 16 h + ..
+                // twiddle w1024^(b k2) -> stage-3 row (k1, k2), chunk lane & 7
+                // row rho2(k1, k2), k2 = 16 h + 4 gq + i: row / 8 = 16 i + 4 Q + (lane >> 3), row % 8 = 4 h + gq
+                const uint32_t base = uint32_t(4 * Q + (lane >> 3)) * kSBO64 + uint32_t(lane & 7) * tc::kLBO +
+                                      uint32_t(4 * hh) * 16u;
+                const float4* tw = TW2 + 64 * hh + (lane & 7);
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    float d[4][8];
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int ip = 0; ip < 2; ++ip) {
+                        float4 w[4];
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) w[T] = tw[(T * 16 + 2 * gq + ip) * 8];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = 2 * ip + e;
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int T = 0; T < 4; ++T) {
+                                const float2 ww = e ? make_float2(w[T].z, w[T].w) : make_float2(w[T].x, w[T].y);
+                                const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), ww);
+                                pk[T] = pack_bf16(v.x, v.y);
+                            }
+                            sts128(A, base + uint32_t(16 * i) * kSBO64 + uint32_t(gq) * 16u, pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+            }
+            // ---------------- stage 3; meanwhile this thread loads its spectrum values
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            {
+                // row (k1 = 4 Q + lane / 8, k2 = 4 (lane & 7) + T) keeps its place, slots
+                // k3 = 16 h + 4 i + e; spectrum entry uint4 (T * 4 + i) of this thread
+                // holds K~ at e = 0..3 (bf16 hi plane).  Stores conj(X K~).
+                const uint4* kq = reinterpret_cast<const uint4*>(spec + (int64_t(st - 1) * C + c) * (2 * N)) +
+                                  (Q * 2 + hh) * 16 * 32 + lane;
+                uint4 kv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) kv[i] = __ldg(kq + 32 * i);
+                ok &= stage_wait(&mbar, phase);
+#pragma unroll
+                for (int T = 0; T < 4; ++T) {
+                    float d[32];
+                    tc::tmem_ld32(tl + uint32_t(64 * T + 32 * hh), d);
+                    tc::tmem_ld_wait();
+                    const uint32_t rowoff = uint32_t(16 * T + 4 * Q + (lane >> 3)) * kSBO64 + uint32_t(4 * hh) * tc::kLBO +
+                                            uint32_t(lane & 7) * 16u;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint4 kk = kv[4 * T + q4];
+                        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 4 * q4 + e;
+                            const float2 K = make_float2(bf_lo(kw[e]), bf_hi(kw[e]));
+                            const float2 v = cmul(make_float2(d[2 * i], d[2 * i + 1]), K);
+                            pk[e] = pack_bf16(v.x, -v.y);
+                        }
+                        sts128(A, rowoff + q4 * tc::kLBO, pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            // ---------------- stage 3' (inverse, on conj)
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            ok &= stage_wait(&mbar, phase);
+            {
+                // rows (k1 = 4 Q + lane / 8, k2 = 4 (lane & 7) + T), outputs b = 16 h + ..
+                // twiddle w1024^(b k2) -> stage-2' row (k1, b), chunk lane & 7
+                // row 128 (lane >> 3) + 32 Q + b, b = 16 h + 4 gq + i:
+                // row / 8 = 16 (lane >> 3) + 4 Q + 2 h + (gq >> 1), row % 8 = 4 (gq & 1) + i
+                const uint32_t base = uint32_t(16 * (lane >> 3) + 4 * Q + 2 * hh) * kSBO64 + uint32_t(lane & 7) * tc::kLBO;
+                const float4* tw = TW2 + 64 * hh + (lane & 7);
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    float d[4][8];
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int ip = 0; ip < 2; ++ip) {
+                        float4 w[4];
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) w[T] = tw[(T * 16 + 2 * gq + ip) * 8];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = 2 * ip + e;
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int T = 0; T < 4; ++T) {
+                                const float2 ww = e ? make_float2(w[T].z, w[T].w) : make_float2(w[T].x, w[T].y);
+                                const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), ww);
+                                pk[T] = pack_bf16(v.x, v.y);
+                            }
+                            sts128(A, base + uint32_t(gq >> 1) * kSBO64 + uint32_t(4 * (gq & 1) + i) * 16u, pk[0], pk[1],
+                                   pk[2], pk[3]);
+                        }
+                    }
+                }
+            }
+            // ---------------- stage 2'
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            ok &= stage_wait(&mbar, phase);
+            {
+                // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w_N^((b + 32 q) k1)
+                // -> stage-1' row a = b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
+                // row a = lane + 32 (16 h + 4 gq + i): a / 8 = (lane >> 3) + 64 h + 16 gq + 4 i, a % 8 = lane & 7
+                const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
+                                      uint32_t(lane & 7) * 16u;
+                float2 pw[4], stp[4];
+#pragma unroll
+                for (int T = 0; T < 4; ++T) {
+                    const int k1 = 4 * Q + T;
+                    pw[T] = wN((lane + 512 * hh) * k1, twist, odd);
+                    stp[T] = wN(32 * k1, twist, odd);
+                }
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    float d[4][8];
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) {
+                            const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), pw[T]);
+                            pw[T] = cmul(pw[T], stp[T]);
+                            pk[T] = pack_bf16(v.x, v.y);
+                        }
+                        sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            // ---------------- stage 1': 8 tiles x (K 32 -> N 16), outputs s < 8 only
+            stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar);
+            if (st < order - 1) ok &= stage_wait(&mbar, phase);
+        }
+        // ---------------- output: v = conj(D1') -> staging (fp32, natural order) -> y = sc(x0) v
+        {
+            // x0 samples n0 .. n0+7 (n0 = 8 (t + 256 jj)) of both rows, loaded while stage 1' runs
+            uint4 xr[2][4];
+            uint32_t xh[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const bf16* x0 = (r ? u1 : u0) + c * L;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int n0 = 8 * (t + 256 * jj);
+                    xr[r][jj] = __ldg(reinterpret_cast<const uint4*>(x0 + n0));
+                    xh[r][jj] = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x0 + n0 - 2)) : 0u;
+                }
+            }
+            ok &= stage_wait(&mbar, phase);
+            float* V0 = reinterpret_cast<float*>(A);
+            float* V1 = V0 + L;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int a = 128 * (4 * hh + j) + 32 * Q + lane;
+                float d[16];
+                tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8) {
+                    V0[a + 1024 * s8] = d[2 * s8];
+                    V1[a + 1024 * s8] = -d[2 * s8 + 1];
+                }
+            }
+            tc::fence_before_sync();
+            __syncthreads();
+            const Taps t0 = load_taps(sc_w, sc_b, c);
+            const float nanv = ok ? 1.0f : __int_as_float(0x7fc00000);   // a timed-out wait poisons the output
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (r == 1 && !has1) break;
+                bf16* yr = y + ((b0 + r) * C + c) * L;
+                const float* Vr = r ? V1 : V0;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int n0 = 8 * (t + 256 * jj);
+                    const uint4 cur = xr[r][jj];
+                    const uint32_t hb = xh[r][jj];
+                    const float xv[10] = {bf_lo(hb), bf_hi(hb), bf_lo(cur.x), bf_hi(cur.x), bf_lo(cur.y),
+                                          bf_hi(cur.y), bf_lo(cur.z), bf_hi(cur.z), bf_lo(cur.w), bf_hi(cur.w)};
+                    float xs[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        xs[i] = nanv * fmaf(t0.w0, xv[i], fmaf(t0.w1, xv[i + 1], fmaf(t0.w2, xv[i + 2], t0.b)));
+                    const float4 va = *reinterpret_cast<const float4*>(Vr + n0);
+                    const float4 vb = *reinterpret_cast<const float4*>(Vr + n0 + 4);
+                    uint4 o;
+                    o.x = pack_bf16(xs[0] * va.x, xs[1] * va.y);
+                    o.y = pack_bf16(xs[2] * va.z, xs[3] * va.w);
+                    o.z = pack_bf16(xs[4] * vb.x, xs[5] * vb.y);
+                    o.w = pack_bf16(xs[6] * vb.z, xs[7] * vb.w);
+                    *reinterpret_cast<uint4*>(yr + n0) = o;
+                }
+            }
+        }
+        if (!ok) {
+            if (t == 0) atomicOr(status, 1u);           // a tensor-core wait timed out
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    auto kern = k_conv_8192_tc;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t npairs = p.C * ((a.B + 1) / 2);
+    int64_t grid = int64_t(2) * sms;
+    if (grid > npairs) grid = npairs;
+    kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
+                                           a.sc_b, a.B, p.C, p.order, npairs);
+    return cudaGetLastError();
+}
+
+}  // namespace hyena

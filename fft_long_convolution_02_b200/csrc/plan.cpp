@@ -74,7 +74,10 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
             p->t_fft_a = tb.add_fft(int(p->M));
             p->t_twist = tb.add(L, 0, p->M, 1, 1);                  // w_L^n, n < M
             p->t_untangle = tb.add_untangle(L);
-            p->spec_row_bytes = size_t(p->M + 1) * 16;
+            // L = 8192: all 2L bins of the zero-padded transform (complex64, in
+            // the position order of its tensor-core kernel); other lengths the
+            // pair layout ((M+1) float4 entries)
+            p->spec_row_bytes = (L == 8192) ? size_t(16 * L) : size_t(p->M + 1) * 16;
         } else {
             p->path = PATH_MULTIPASS_1D;
             p->M1 = (p->M >= (int64_t(1) << 16)) ? 256 : 128;

@@ -11,7 +11,9 @@
 //
 // Paths (N = 2L zero-padded transform, computed as two M = L/2-point chains):
 //   PATH_ONCHIP_1D    16 <= L <= 16384: one CTA per (b, c) row, everything in
-//                     shared memory.  Spectrum row = (M+1) float4 pair entries.
+//                     shared memory.  Spectrum row = (M+1) float4 pair entries;
+//                     L = 8192: all 2L bins, complex64, in the position
+//                     order of the tensor-core kernel (onchip_tc.cu).
 //   PATH_MULTIPASS_1D 32768 <= L <= 2^20: four-step M = M1 x M2 with three
 //                     passes through a caller workspace (kept L2-resident by
 //                     processing rows in groups).  Spectrum row = M1 units of
@@ -48,7 +50,10 @@ struct SpecHeader {
     int32_t ndim, order, path, reserved0;
     int64_t C, L, H, W, M, M1, M2;
     int64_t tables_off, tables_count, spec_off, spec_row_bytes, total_bytes;
-    int64_t reserved[17];
+    // set (bit 0) by a convolution kernel whose bounded tensor-core wait gave
+    // up; reported by hyena_spectrum_check
+    uint32_t device_status, reserved1;
+    int64_t reserved[16];
 };
 static_assert(sizeof(SpecHeader) == kHeaderBytes, "header must be 256 bytes");
 

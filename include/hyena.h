@@ -185,11 +185,12 @@ hyena_status_t hyena_gated_fftconv_noalloc(const void* u, void* y, const void* s
                                            const int64_t* sizes, int order, hyena_dtype_t dtype, void* stream);
 
 /*
- * Debug helper (synchronous)/*
  * Debug helper (synchronous): copies the spectrum header to the host and
  * checks it against (C, sizes, order).  Returns HYENA_OK when it matches,
  * HYENA_ERR_SPECTRUM_MISMATCH when not (e.g. never filled, or filled for
- * another shape).  Synchronises `stream`.
+ * another shape), HYENA_ERR_INTERNAL when an earlier convolution with this
+ * spectrum gave up on a bounded tensor-core wait (its outputs were written as
+ * NaN).  Synchronises `stream`.
  */
 hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
                                     void* stream);

@@ -44,8 +44,11 @@ def _sz(*s):
 
 def test_spectrum_bytes_and_workspace(lib):
     # on-chip: header + tables + (order-1) C (L/2+1) 16 bytes
+    b = lib.hyena_spectrum_bytes(768, 1, _sz(1024), 2)
+    assert 768 * (512 + 1) * 16 <= b < 768 * (512 + 1) * 16 + (1 << 20)
+    # L = 8192: all 2L bins, 16L bytes per channel
     b = lib.hyena_spectrum_bytes(768, 1, _sz(8192), 2)
-    assert b >= 768 * (4096 + 1) * 16 and b < 768 * (4096 + 1) * 16 + (1 << 20)
+    assert 768 * 16 * 8192 <= b < 768 * 16 * 8192 + (1 << 20)
     assert lib.hyena_gated_fftconv_workspace_bytes(4, 768, 1, _sz(8192), 2) == 0
     # multi-pass: spectrum rows of 8L bytes, workspace 8L bytes per row
     L = 1 << 20
