@@ -60,13 +60,14 @@ constexpr uint32_t kB1bytes = 4 * kSBO16;   // N 32 x K 16
 constexpr uint32_t kB32bytes = 8 * kSBO64;  // N 64 x K 64
 constexpr uint32_t kB1ibytes = 2 * kSBO32;  // N 16 x K 32
 constexpr uint32_t kTW2bytes = 4 * 16 * 8 * 16;
+constexpr uint32_t kOffA1 = kAbytes - 128 * kSBO16;   // stage-1 operand (1024 rows x K 16)
 constexpr uint32_t kOffB1 = kAbytes;
 constexpr uint32_t kOffB32 = kOffB1 + kB1bytes;
 constexpr uint32_t kOffB1i = kOffB32 + kB32bytes;
 constexpr uint32_t kOffTW2 = kOffB1i + kB1ibytes;
 constexpr size_t kSmem = size_t(kOffTW2) + kTW2bytes;
 constexpr int kWaitLimit = 1 << 22;
-static_assert(2 * L * sizeof(float) <= kAbytes, "output staging must fit the operand buffer");
+static_assert(L * 4 <= kOffA1, "output staging must not overlap the stage-1 operand");
 static_assert(kOffTW2 % 16 == 0, "twiddle table alignment");
 
 __device__ __forceinline__ uint32_t pack_bf16(float re, float im) {
@@ -97,17 +98,6 @@ __device__ __forceinline__ float2 wN(int e, const float2* __restrict__ twist, co
     return v;
 }
 
-// Width-3 causal short conv of 8 consecutive samples n0 .. n0+7 (n0 % 8 == 0).
-__device__ __forceinline__ void sc8(const bf16* __restrict__ x, int n0, const Taps& tp, float (&o)[8]) {
-    const uint4 cur = __ldg(reinterpret_cast<const uint4*>(x + n0));
-    const uint32_t halo = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x + n0 - 2)) : 0u;
-    float v[10];
-    v[0] = bf_lo(halo); v[1] = bf_hi(halo);
-    v[2] = bf_lo(cur.x); v[3] = bf_hi(cur.x); v[4] = bf_lo(cur.y); v[5] = bf_hi(cur.y);
-    v[6] = bf_lo(cur.z); v[7] = bf_hi(cur.z); v[8] = bf_lo(cur.w); v[9] = bf_hi(cur.w);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = fmaf(tp.w0, v[i], fmaf(tp.w1, v[i + 1], fmaf(tp.w2, v[i + 2], tp.b)));
-}
 __device__ __forceinline__ float sc1(const bf16* __restrict__ x, int n, const Taps& tp) {
     const float c = __bfloat162float(x[n]);
     const float p1 = n >= 1 ? __bfloat162float(x[n - 1]) : 0.0f;
@@ -156,6 +146,64 @@ __device__ __forceinline__ bool stage_wait(uint64_t* mbar, uint32_t& phase) {
     return ok;
 }
 
+// Raw samples n0 .. n0+7 and the two before them (n0 % 8 == 0) of one row.
+struct Raw8 {
+    uint4 cur;
+    uint32_t halo;
+};
+__device__ __forceinline__ Raw8 load8(const bf16* __restrict__ x, int n0) {
+    Raw8 r;
+    r.cur = __ldg(reinterpret_cast<const uint4*>(x + n0));
+    r.halo = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x + n0 - 2)) : 0u;
+    return r;
+}
+// Width-3 causal short conv of the 8 samples of `r`.
+__device__ __forceinline__ void sc8(const Raw8& r, const Taps& tp, float (&o)[8]) {
+    const float v[10] = {bf_lo(r.halo),  bf_hi(r.halo),  bf_lo(r.cur.x), bf_hi(r.cur.x), bf_lo(r.cur.y),
+                         bf_hi(r.cur.y), bf_lo(r.cur.z), bf_hi(r.cur.z), bf_lo(r.cur.w), bf_hi(r.cur.w)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = fmaf(tp.w0, v[i], fmaf(tp.w1, v[i + 1], fmaf(tp.w2, v[i + 2], tp.b)));
+}
+
+// Step-1 input of a pair: thread t covers a = a0 .. a0+7 (a0 = 8 (t & 127)) at
+// s = 4 (t >> 7) + j, j < 4, i.e. samples n0 = a0 + 1024 s of x_g and v of
+// both rows.
+struct PairInput {
+    Raw8 x[2][4], v[2][4];
+};
+
+struct PairRef {
+    int64_t c, b0;
+    bool has1;
+};
+__device__ __forceinline__ PairRef pair_ref(int64_t P, int64_t B) {
+    const int64_t nbp = (B + 1) / 2;
+    PairRef r;
+    r.c = P / nbp;
+    r.b0 = 2 * (P - r.c * nbp);
+    r.has1 = r.b0 + 1 < B;
+    return r;
+}
+
+__device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __restrict__ u, const PairRef& pr,
+                                                int64_t C, int order, int j0) {
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const int t = threadIdx.x;
+    const int chalf = t >> 7, a0 = 8 * (t & 127);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const bf16* ub = u + (pr.b0 + (r && pr.has1 ? 1 : 0)) * Ctot * L;
+        const bf16* xg = ub + (int64_t(order - 1) * C + pr.c) * L;
+        const bf16* vv = ub + (int64_t(order) * C + pr.c) * L;
+#pragma unroll
+        for (int j = j0; j < j0 + 2; ++j) {
+            const int n0 = a0 + 1024 * (4 * chalf + j);
+            in.x[r][j] = load8(xg, n0);
+            in.v[r][j] = load8(vv, n0);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NT, 2)
 k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
                const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
@@ -173,13 +221,17 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     const uint32_t* spec = reinterpret_cast<const uint32_t*>(spectrum + h->spec_off);   // plane 0 of each row
     uint32_t* status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(spectrum) + offsetof(SpecHeader, device_status));
 
+    // A: stage operands.  The stage-1 operand sits in the upper part so that
+    // the previous pair's output staging (bf16 pairs, lower 32 KB) survives
+    // until its output gate has run.
     uint8_t* A = smem_tc;
+    uint8_t* A1 = smem_tc + kOffA1;
+    uint32_t* Vs = reinterpret_cast<uint32_t*>(smem_tc);      // output staging: (re, -im) as bf16 pairs
     float4* TW2 = reinterpret_cast<float4*>(smem_tc + kOffTW2);
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
     const int64_t Ctot = int64_t(order + 1) * C;
-    const int64_t nbp = (B + 1) / 2;
 
     fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16);
     fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64);
@@ -200,65 +252,112 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     const uint32_t tmem = tmem_base;
     const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);     // this warp's lane quarter
     const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t a1_addr = tc::smem_u32(A1);
     const uint32_t b1_addr = tc::smem_u32(smem_tc + kOffB1);
     const uint32_t b32_addr = tc::smem_u32(smem_tc + kOffB32);
     const uint32_t b1i_addr = tc::smem_u32(smem_tc + kOffB1i);
     uint32_t phase = 0;
     bool ok = true;
 
-    for (int64_t P = blockIdx.x; P < npairs; P += gridDim.x) {
-        const int64_t c = P / nbp;
-        const int64_t b0 = 2 * (P - c * nbp);
-        const bool has1 = b0 + 1 < B;
-        const bf16* u0 = u + b0 * Ctot * L;
-        const bf16* u1 = has1 ? u0 + Ctot * L : u0;
-        if (t == 0) {
-            // warm L2 with this pair's spectrum rows (hi plane) and the next pair's rows
-            for (int st = 1; st < order; ++st)
-                tc::prefetch_l2(spec + (int64_t(st - 1) * C + c) * (2 * N), N * 4);
-            const int64_t Pn = P + gridDim.x;
-            if (Pn < npairs) {
-                const int64_t cn = Pn / nbp, bn = 2 * (Pn - cn * nbp);
-                for (int r = 0; r < 2 && bn + r < B; ++r)
-                    for (int g = 0; g <= order; ++g)
-                        tc::prefetch_l2(u + ((bn + r) * Ctot + int64_t(g) * C + cn) * L, L * 2);
+    // Output gate of a finished pair: y = sc(x0) * v from the staging buffer.
+    // Thread t covers samples n0 = 8 (t + 256 jj) of both rows.
+    auto output_gate = [&](const PairRef& pr) {
+        const Taps t0 = load_taps(sc_w, sc_b, pr.c);
+        const float poison = ok ? 1.0f : __int_as_float(0x7fc00000);   // a timed-out wait poisons the output
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            if (r == 1 && !pr.has1) break;
+            const bf16* x0 = u + ((pr.b0 + r) * Ctot + pr.c) * L;
+            bf16* yr = y + ((pr.b0 + r) * C + pr.c) * L;
+            Raw8 xr[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) xr[jj] = load8(x0, 8 * (t + 256 * jj));
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int n0 = 8 * (t + 256 * jj);
+                const uint4 va = *reinterpret_cast<const uint4*>(Vs + n0);
+                const uint4 vb = *reinterpret_cast<const uint4*>(Vs + n0 + 4);
+                const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+                float xs[8];
+                sc8(xr[jj], t0, xs);
+                uint32_t o[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float v0 = r ? bf_hi(vw[2 * i]) : bf_lo(vw[2 * i]);
+                    const float v1 = r ? bf_hi(vw[2 * i + 1]) : bf_lo(vw[2 * i + 1]);
+                    o[i] = pack_bf16(poison * xs[2 * i] * v0, poison * xs[2 * i + 1] * v1);
+                }
+                *reinterpret_cast<uint4*>(yr + n0) = make_uint4(o[0], o[1], o[2], o[3]);
             }
         }
-        for (int st = 1; st < order; ++st) {
-            const int g = order - st;
-            const Taps tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
-            const bf16* xg0 = u0 + (int64_t(g) * C + c) * L;
-            const bf16* xg1 = u1 + (int64_t(g) * C + c) * L;
-            // ---------------- stage-1 operand: z = g[b0] + i g[b1]
-            if (st == 1) {
-                const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
-                const bf16* v0 = u0 + (int64_t(order) * C + c) * L;
-                const bf16* v1 = u1 + (int64_t(order) * C + c) * L;
-                const int chalf = t >> 7, a0 = 8 * (t & 127);
-                uint32_t pk[8][4];
+    };
+
+    PairInput in;
+    if (int64_t(blockIdx.x) < npairs) {
+        load_pair_input(in, u, pair_ref(blockIdx.x, B), C, order, 0);
+        load_pair_input(in, u, pair_ref(blockIdx.x, B), C, order, 2);
+    }
+    PairRef prev{0, 0, false};
+    bool have_prev = false;
+
+    for (int64_t P = blockIdx.x; P < npairs; P += gridDim.x) {
+        const PairRef pr = pair_ref(P, B);
+        const int64_t c = pr.c;
+        const bf16* u0 = u + pr.b0 * Ctot * L;
+        const bf16* u1 = pr.has1 ? u0 + Ctot * L : u0;
+        const int64_t Pn = P + gridDim.x;
+        if (t == 0) {
+            // warm L2 with this pair's spectrum rows (plane 0) and the next pair's rows
+            for (int st = 1; st < order; ++st)
+                tc::prefetch_l2(spec + (int64_t(st - 1) * C + c) * (2 * N), N * 4);
+            if (Pn < npairs) {
+                const PairRef pn = pair_ref(Pn, B);
+                for (int r = 0; r < 2 && pn.b0 + r < B; ++r)
+                    for (int g = 0; g <= order; ++g)
+                        tc::prefetch_l2(u + ((pn.b0 + r) * Ctot + int64_t(g) * C + pn.c) * L, L * 2);
+            }
+        }
+        // ---------------- step-1 operand: z = sc(x_{order-1}) sc(v), g[b0] + i g[b1]
+        {
+            const Taps tg = load_taps(sc_w, sc_b, int64_t(order - 1) * C + c);
+            const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+            const int chalf = t >> 7, a0 = 8 * (t & 127);
+            const float m1 = pr.has1 ? 1.0f : 0.0f;
+            // rows rho1(a0 + i) = rho1(a0) + i (a0 % 8 == 0); slots 4 chalf + j
+            const uint32_t base = uint32_t(rho1(a0) >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n0 = a0 + 1024 * (4 * chalf + j);
+            for (int jp = 0; jp < 4; jp += 2) {
+                uint32_t pk[8][2];
+#pragma unroll
+                for (int jo = 0; jo < 2; ++jo) {
+                    const int j = jp + jo;
                     float xa[8], va[8], xb[8], vb[8];
-                    sc8(xg0, n0, tg, xa);
-                    sc8(v0, n0, tv, va);
-                    if (has1) {
-                        sc8(xg1, n0, tg, xb);
-                        sc8(v1, n0, tv, vb);
-                    } else {
+                    sc8(in.x[0][j], tg, xa);
+                    sc8(in.v[0][j], tv, va);
+                    sc8(in.x[1][j], tg, xb);
+                    sc8(in.v[1][j], tv, vb);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) { xb[i] = 0.0f; vb[i] = 0.0f; }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) pk[i][j] = pack_bf16(xa[i] * va[i], xb[i] * vb[i]);
+                    for (int i = 0; i < 8; ++i) pk[i][jo] = pack_bf16(xa[i] * va[i], m1 * xb[i] * vb[i]);
                 }
-                __syncthreads();                        // operand buffer free (previous pair's output read)
-                // rows rho1(a0 + i) = rho1(a0) + i (a0 % 8 == 0)
-                const uint32_t base = uint32_t(rho1(a0) >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) sts128(A, base + 16u * i, pk[i][0], pk[i][1], pk[i][2], pk[i][3]);
-            } else {
-                // previous step's output v = conj(stage-1' accumulators), row a, output s
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<uint2*>(A1 + base + 16u * i + 4u * jp) = make_uint2(pk[i][0], pk[i][1]);
+            }
+            stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
+            if (have_prev) {
+                output_gate(prev);                  // overlaps the stage-1 MMAs
+                have_prev = false;
+            }
+            __syncthreads();                        // staging read by every thread before pass 1 overwrites it
+        }
+        for (int st = 1; st < order; ++st) {
+            if (st > 1) {
+                // previous step's output v = conj(stage-1' accumulators), row a, output s;
+                // z = sc(x_g) v with g = order - st
+                const int g = order - st;
+                const Taps tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
+                const bf16* xg0 = u0 + (int64_t(g) * C + c) * L;
+                const bf16* xg1 = u1 + (int64_t(g) * C + c) * L;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int a = 128 * (4 * hh + j) + 32 * Q + lane;
@@ -270,16 +369,15 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     for (int s = 0; s < 8; ++s) {
                         const int n = a + 1024 * s;
                         const float za = sc1(xg0, n, tg) * d[2 * s];
-                        const float zb = has1 ? sc1(xg1, n, tg) * -d[2 * s + 1] : 0.0f;
+                        const float zb = pr.has1 ? sc1(xg1, n, tg) * -d[2 * s + 1] : 0.0f;
                         pk[s] = pack_bf16(za, zb);
                     }
-                    sts128(A, tc::chunk_off(rho1(a), 0, kSBO16), pk[0], pk[1], pk[2], pk[3]);
-                    sts128(A, tc::chunk_off(rho1(a), 1, kSBO16), pk[4], pk[5], pk[6], pk[7]);
+                    sts128(A1, tc::chunk_off(rho1(a), 0, kSBO16), pk[0], pk[1], pk[2], pk[3]);
+                    sts128(A1, tc::chunk_off(rho1(a), 1, kSBO16), pk[4], pk[5], pk[6], pk[7]);
                 }
+                stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
             }
             // ---------------- stage 1: 8 tiles x (K 16 -> N 32)
-            stage_issue(a_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
-            ok &= stage_wait(&mbar, phase);
             {
                 // twiddle w_N^(a k1); vector a = lane + 32 q, q = j + 4 Q + 16 h
                 // -> stage-2 row (k1, lane), chunk Q + 4 h (slots q, j = 0..3)
@@ -289,6 +387,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     beta[j] = wN(lane + 32 * (j + 4 * Q + 16 * hh), twist, odd);
                     pw[j] = make_float2(1.0f, 0.0f);
                 }
+                ok &= stage_wait(&mbar, phase);
                 // row rho2(k1, lane): row / 8 = 16 (lane & 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane >> 2
                 const uint32_t base = uint32_t(16 * (lane & 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
                                       uint32_t(lane >> 2) * 16u;
@@ -422,7 +521,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             }
             // ---------------- stage 2'
             stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
-            ok &= stage_wait(&mbar, phase);
             {
                 // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w_N^((b + 32 q) k1)
                 // -> stage-1' row a = b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
@@ -436,6 +534,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     pw[T] = wN((lane + 512 * hh) * k1, twist, odd);
                     stp[T] = wN(32 * k1, twist, odd);
                 }
+                ok &= stage_wait(&mbar, phase);
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     float d[4][8];
@@ -459,72 +558,34 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar);
             if (st < order - 1) ok &= stage_wait(&mbar, phase);
         }
-        // ---------------- output: v = conj(D1') -> staging (fp32, natural order) -> y = sc(x0) v
-        {
-            // x0 samples n0 .. n0+7 (n0 = 8 (t + 256 jj)) of both rows, loaded while stage 1' runs
-            uint4 xr[2][4];
-            uint32_t xh[2][4];
+        // the next pair's step-1 input: half loaded while stage 1' runs, half after the
+        // staging (unconditional, so that the registers' live range ends here; past the
+        // last pair this pair's rows are reloaded and not used)
+        const PairRef pnext = pair_ref(Pn < npairs ? Pn : P, B);
+        load_pair_input(in, u, pnext, C, order, 0);
+        ok &= stage_wait(&mbar, phase);
+        // output staging v = conj(D1') as (re, -im) bf16 pairs in natural order;
+        // the output gate runs during the next pair's stage 1
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const bf16* x0 = (r ? u1 : u0) + c * L;
+        for (int j = 0; j < 4; ++j) {
+            const int a = 128 * (4 * hh + j) + 32 * Q + lane;
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
+            tc::tmem_ld_wait();
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int n0 = 8 * (t + 256 * jj);
-                    xr[r][jj] = __ldg(reinterpret_cast<const uint4*>(x0 + n0));
-                    xh[r][jj] = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x0 + n0 - 2)) : 0u;
-                }
-            }
-            ok &= stage_wait(&mbar, phase);
-            float* V0 = reinterpret_cast<float*>(A);
-            float* V1 = V0 + L;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int a = 128 * (4 * hh + j) + 32 * Q + lane;
-                float d[16];
-                tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int s8 = 0; s8 < 8; ++s8) {
-                    V0[a + 1024 * s8] = d[2 * s8];
-                    V1[a + 1024 * s8] = -d[2 * s8 + 1];
-                }
-            }
-            tc::fence_before_sync();
-            __syncthreads();
-            const Taps t0 = load_taps(sc_w, sc_b, c);
-            const float nanv = ok ? 1.0f : __int_as_float(0x7fc00000);   // a timed-out wait poisons the output
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (r == 1 && !has1) break;
-                bf16* yr = y + ((b0 + r) * C + c) * L;
-                const float* Vr = r ? V1 : V0;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int n0 = 8 * (t + 256 * jj);
-                    const uint4 cur = xr[r][jj];
-                    const uint32_t hb = xh[r][jj];
-                    const float xv[10] = {bf_lo(hb), bf_hi(hb), bf_lo(cur.x), bf_hi(cur.x), bf_lo(cur.y),
-                                          bf_hi(cur.y), bf_lo(cur.z), bf_hi(cur.z), bf_lo(cur.w), bf_hi(cur.w)};
-                    float xs[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        xs[i] = nanv * fmaf(t0.w0, xv[i], fmaf(t0.w1, xv[i + 1], fmaf(t0.w2, xv[i + 2], t0.b)));
-                    const float4 va = *reinterpret_cast<const float4*>(Vr + n0);
-                    const float4 vb = *reinterpret_cast<const float4*>(Vr + n0 + 4);
-                    uint4 o;
-                    o.x = pack_bf16(xs[0] * va.x, xs[1] * va.y);
-                    o.y = pack_bf16(xs[2] * va.z, xs[3] * va.w);
-                    o.z = pack_bf16(xs[4] * vb.x, xs[5] * vb.y);
-                    o.w = pack_bf16(xs[6] * vb.z, xs[7] * vb.w);
-                    *reinterpret_cast<uint4*>(yr + n0) = o;
-                }
-            }
+            for (int s8 = 0; s8 < 8; ++s8) Vs[a + 1024 * s8] = pack_bf16(d[2 * s8], -d[2 * s8 + 1]);
         }
+        load_pair_input(in, u, pnext, C, order, 2);
+        prev = pr;
+        have_prev = true;
         if (!ok) {
             if (t == 0) atomicOr(status, 1u);           // a tensor-core wait timed out
             break;
         }
     }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (have_prev) output_gate(prev);
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
