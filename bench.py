@@ -55,11 +55,11 @@ def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
 
 
 def spectrum_row_bytes(p) -> int:
-    """Stored spectrum bytes per (step, channel) row of the library's layout."""
+    """Spectrum bytes per (step, channel) row the convolution kernel reads."""
     if p.ndim == 2:
         return (p.W + 1) * 2 * p.H * 8
     if p.L == 8192:
-        return 16 * p.L                     # all 2L bins, complex64
+        return 8 * p.L                      # one plane: bf16 2L bins, or fp32 position layout
     if p.L <= 16384:
         return (p.L // 2 + 1) * 16
     return 8 * p.L
@@ -335,7 +335,7 @@ def main():
     avg_launch_s = float(np.mean(launch_ms)) / 1e3
     achieved = alg / avg_launch_s / 1e9
     if p.ndim == 1 and p.L == 8192:
-        kernel = "k_conv_4096"
+        kernel = "k_conv_8192_tc" if p.dtype == "bf16" else "k_conv_4096"
     elif p.ndim == 1 and p.L <= 16384:
         kernel = "k_conv_onchip"
     else:

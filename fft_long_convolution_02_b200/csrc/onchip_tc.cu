@@ -25,8 +25,8 @@
 // applies the twiddles in fp32 and scatters the values into the next stage's
 // operand.  The row orders below are chosen so that each thread's values for
 // one destination row are four consecutive slots: one 16-byte store.
-//   stage-1 rows   rho1(a)     = 128 T + 32 Q + b, q = a >> 5, b = a & 31,
-//                                T = (q & 3) + 4 (q >> 4), Q = (q >> 2) & 3
+//   stage-1 rows   rho1(a)     = 128 T + 32 Q + 8 (b & 3) + (b >> 2), q = a >> 5,
+//                                b = a & 31, T = (q & 3) + 4 (q >> 4), Q = (q >> 2) & 3
 //   stage-2 rows   rho2(k1, b) = 128 (b & 3) + 32 (k1 >> 2) + 8 (k1 & 3) + (b >> 2)
 //   stage-3 rows   rho2(k1, k2)
 //   stage-2' rows  128 (k1 & 3) + 32 (k1 >> 2) + b
@@ -84,7 +84,7 @@ __device__ __forceinline__ void sts128(uint8_t* base, uint32_t off, uint32_t x, 
 
 __device__ __forceinline__ int rho1(int a) {
     const int q = a >> 5, b = a & 31;
-    return 128 * ((q & 3) + 4 * (q >> 4)) + 32 * ((q >> 2) & 3) + b;
+    return 128 * ((q & 3) + 4 * (q >> 4)) + 32 * ((q >> 2) & 3) + 8 * (b & 3) + (b >> 2);
 }
 
 // w_N^e for any integer e: quarter-turn reduction onto the tables
@@ -263,7 +263,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     // Thread t covers samples n0 = 8 (t + 256 jj) of both rows.
     auto output_gate = [&](const PairRef& pr) {
         const Taps t0 = load_taps(sc_w, sc_b, pr.c);
-        const float poison = ok ? 1.0f : __int_as_float(0x7fc00000);   // a timed-out wait poisons the output
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             if (r == 1 && !pr.has1) break;
@@ -285,9 +284,11 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 for (int i = 0; i < 4; ++i) {
                     const float v0 = r ? bf_hi(vw[2 * i]) : bf_lo(vw[2 * i]);
                     const float v1 = r ? bf_hi(vw[2 * i + 1]) : bf_lo(vw[2 * i + 1]);
-                    o[i] = pack_bf16(poison * xs[2 * i] * v0, poison * xs[2 * i + 1] * v1);
+                    o[i] = pack_bf16(xs[2 * i] * v0, xs[2 * i + 1] * v1);
                 }
-                *reinterpret_cast<uint4*>(yr + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(yr + n0) = ok ? make_uint4(o[0], o[1], o[2], o[3])   // a timed-out
+                                                        : make_uint4(0x7fc07fc0u, 0x7fc07fc0u,   // wait poisons
+                                                                     0x7fc07fc0u, 0x7fc07fc0u);  // the output
             }
         }
     };
@@ -323,8 +324,9 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
             const int chalf = t >> 7, a0 = 8 * (t & 127);
             const float m1 = pr.has1 ? 1.0f : 0.0f;
-            // rows rho1(a0 + i) = rho1(a0) + i (a0 % 8 == 0); slots 4 chalf + j
-            const uint32_t base = uint32_t(rho1(a0) >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO;
+            // rows rho1(a0 + i) = rho1(a0) + 8 (i & 3) + (i >> 2) (a0 % 8 == 0); slots 4 chalf + j
+            const int r0 = rho1(a0);
+            const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
 #pragma unroll
             for (int jp = 0; jp < 4; jp += 2) {
                 uint32_t pk[8][2];
@@ -341,7 +343,8 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    *reinterpret_cast<uint2*>(A1 + base + 16u * i + 4u * jp) = make_uint2(pk[i][0], pk[i][1]);
+                    *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u + 4u * jp) =
+                        make_uint2(pk[i][0], pk[i][1]);
             }
             stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
             if (have_prev) {
@@ -379,19 +382,20 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             }
             // ---------------- stage 1: 8 tiles x (K 16 -> N 32)
             {
-                // twiddle w_N^(a k1); vector a = lane + 32 q, q = j + 4 Q + 16 h
-                // -> stage-2 row (k1, lane), chunk Q + 4 h (slots q, j = 0..3)
+                // twiddle w_N^(a k1); vector a = b + 32 q, b = 4 (lane & 7) + (lane >> 3),
+                // q = j + 4 Q + 16 h -> stage-2 row (k1, b), chunk Q + 4 h (slots q, j = 0..3)
+                const int b1 = 4 * (lane & 7) + (lane >> 3);
                 float2 beta[4], pw[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    beta[j] = wN(lane + 32 * (j + 4 * Q + 16 * hh), twist, odd);
+                    beta[j] = wN(b1 + 32 * (j + 4 * Q + 16 * hh), twist, odd);
                     pw[j] = make_float2(1.0f, 0.0f);
                 }
                 ok &= stage_wait(&mbar, phase);
-                // row rho2(k1, lane): row / 8 = 16 (lane & 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane >> 2
-                const uint32_t base = uint32_t(16 * (lane & 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
-                                      uint32_t(lane >> 2) * 16u;
-#pragma unroll
+                // row rho2(k1, b): row / 8 = 16 (lane >> 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane & 7
+                const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
+                                      uint32_t(lane & 7) * 16u;
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     float d[4][16];
 #pragma unroll
@@ -421,7 +425,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 const uint32_t base = uint32_t(4 * Q + (lane >> 3)) * kSBO64 + uint32_t(lane & 7) * tc::kLBO +
                                       uint32_t(4 * hh) * 16u;
                 const float4* tw = TW2 + 64 * hh + (lane & 7);
-#pragma unroll
+#pragma unroll 1
                 for (int gq = 0; gq < 4; ++gq) {
                     float d[4][8];
 #pragma unroll
@@ -492,7 +496,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 // row / 8 = 16 (lane >> 3) + 4 Q + 2 h + (gq >> 1), row % 8 = 4 (gq & 1) + i
                 const uint32_t base = uint32_t(16 * (lane >> 3) + 4 * Q + 2 * hh) * kSBO64 + uint32_t(lane & 7) * tc::kLBO;
                 const float4* tw = TW2 + 64 * hh + (lane & 7);
-#pragma unroll
+#pragma unroll 1
                 for (int gq = 0; gq < 4; ++gq) {
                     float d[4][8];
 #pragma unroll
@@ -535,7 +539,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     stp[T] = wN(32 * k1, twist, odd);
                 }
                 ok &= stage_wait(&mbar, phase);
-#pragma unroll
+#pragma unroll 1
                 for (int gq = 0; gq < 4; ++gq) {
                     float d[4][8];
 #pragma unroll
@@ -558,11 +562,12 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar);
             if (st < order - 1) ok &= stage_wait(&mbar, phase);
         }
-        // the next pair's step-1 input: half loaded while stage 1' runs, half after the
-        // staging (unconditional, so that the registers' live range ends here; past the
-        // last pair this pair's rows are reloaded and not used)
+        // the next pair's step-1 input, loaded while stage 1' runs (unconditional, so
+        // that the registers' live range ends here; past the last pair this pair's
+        // rows are reloaded and not used)
         const PairRef pnext = pair_ref(Pn < npairs ? Pn : P, B);
         load_pair_input(in, u, pnext, C, order, 0);
+        load_pair_input(in, u, pnext, C, order, 2);
         ok &= stage_wait(&mbar, phase);
         // output staging v = conj(D1') as (re, -im) bf16 pairs in natural order;
         // the output gate runs during the next pair's stage 1
@@ -575,7 +580,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8) Vs[a + 1024 * s8] = pack_bf16(d[2 * s8], -d[2 * s8 + 1]);
         }
-        load_pair_input(in, u, pnext, C, order, 2);
         prev = pr;
         have_prev = true;
         if (!ok) {
