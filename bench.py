@@ -221,11 +221,17 @@ def main():
     ap.add_argument("--workload", default="d768_l8k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--channels", type=int, default=0,
+                    help="override the workload's channel count C (smaller captures for ncu; "
+                         "lines printed with it are not the workload's bench line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from fft_long_convolution_02_b200 import inputs as I
     p = I.WORKLOADS[args.workload]
+    if args.channels:
+        import dataclasses
+        p = dataclasses.replace(p, C=args.channels)
     if args.impl == "reference":
         run_reference(args, p)
         return
