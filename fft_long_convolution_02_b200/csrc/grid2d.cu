@@ -165,7 +165,8 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
                 const int tcol = idx / MH;            // 2*cc + chain
                 const int pos = idx - tcol * MH;
                 const int cc = tcol >> 1, ch = tcol & 1;
-                const float2 k = __ldg(sp + int64_t(f0 + cc) * (2 * MH) + ch * MH + pos);
+                // spectrum entries in the fast column pass's order (see MODE 1)
+                const float2 k = __ldg(sp + int64_t(f0 + cc) * (2 * MH) + ch * MH + (pos & 15) * (MH / 16) + (pos >> 4));
                 float2* e = smem + tcol * PS + fft_pad(pos);
                 *e = cmul(*e, k);
             }
@@ -501,7 +502,10 @@ cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
     return cudaGetLastError();
 }
 
-template <int MW, int MH, typename T>
+// Row passes: register-resident engine (ROWS_REG, W/2 >= 16) or the CTA
+// engine; column pass: register-resident (COLS_REG) or the CTA engine.  Both
+// write and read the same workspace layout ([bin column][H] per image).
+template <int MW, int MH, typename T, bool ROWS_REG, bool COLS_REG>
 cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const T2d tb = t2d(p, a.spectrum);
     const float2* spec = reinterpret_cast<const float2*>(a.spectrum + p.spec_off);
@@ -517,12 +521,22 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     constexpr int NTC = kFC * (MH / 16);
     const size_t smR = size_t(2 * FR) * row_stride_f<MW>() * sizeof(float2);
     const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
-    auto kb = k_2df_cols<MH>;
-    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
-    const unsigned ncolblk = unsigned((W + 1 + kFC - 1) / kFC);
-    // row passes: register-resident for W/2 >= 16, the generic engine for W = 16
+    const size_t smB = col_smem2<MH>(kCB);
+    auto launch_cols = [&](int64_t i0, int64_t g, int st) {
+        if constexpr (COLS_REG) {
+            auto kb = k_2df_cols<MH>;
+            cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+            kb<<<dim3(unsigned((W + 1 + kFC - 1) / kFC), unsigned(g)), NTC, smC, s>>>(
+                a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride);
+        } else {
+            auto kb = k_2d_cols<MH, 0>;
+            cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+            kb<<<dim3(unsigned((W + 1 + kCB - 1) / kCB), unsigned(g)), kColThreads2, smB, s>>>(
+                a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f);
+        }
+    };
     auto launch_rows_fwd = [&](int64_t i0, int64_t g) {
-        if constexpr (MW >= 16) {
+        if constexpr (ROWS_REG && MW >= 16) {
             auto ka = k_2df_rows_fwd<MW, FR, T, 0>;
             cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
             ka<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, a.workspace, tb, a.B, p.C, p.order, H, i0, stride, 0);
@@ -534,7 +548,7 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         }
     };
     auto launch_rows_inv = [&](int64_t i0, int64_t g, bool final_step, int gnext) {
-        if constexpr (MW >= 16) {
+        if constexpr (ROWS_REG && MW >= 16) {
             auto kc = final_step ? k_2df_rows_inv<MW, FR, T, true> : k_2df_rows_inv<MW, FR, T, false>;
             cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
             kc<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, gnext, H, i0,
@@ -550,17 +564,23 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         const int64_t g = nimg - i0 < G ? nimg - i0 : G;
         launch_rows_fwd(i0, g);
         for (int st = 1; st < p.order; ++st) {
-            kb<<<dim3(ncolblk, unsigned(g)), NTC, smC, s>>>(a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride,
-                                                            spec_stride);
+            launch_cols(i0, g, st);
             launch_rows_inv(i0, g, st == p.order - 1, st < p.order - 1 ? p.order - st - 1 : 0);
         }
     }
     return cudaGetLastError();
 }
 
+// Engine choice per pass, measured on B=2, C=256, 256 x 256, bf16 (us per
+// call): CTA rows + register columns 843, register rows + register columns
+// 921, CTA rows + CTA columns 939, register rows + CTA columns 1020.
+constexpr bool kRowsReg2D = false;
+constexpr bool kColsReg2D = true;
+
 template <int MW, int MH>
 cudaError_t conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s) {
-    return a.dtype == DT_F32 ? conv_2d_t<MW, MH, float>(p, a, s) : conv_2d_t<MW, MH, __nv_bfloat16>(p, a, s);
+    return a.dtype == DT_F32 ? conv_2d_t<MW, MH, float, kRowsReg2D, kColsReg2D>(p, a, s)
+                             : conv_2d_t<MW, MH, __nv_bfloat16, kRowsReg2D, kColsReg2D>(p, a, s);
 }
 
 template <int MW>
