@@ -105,16 +105,39 @@ __device__ __forceinline__ float sc1(const bf16* __restrict__ x, int n, const Ta
     return fmaf(tp.w0, p2, fmaf(tp.w1, p1, fmaf(tp.w2, c, tp.b)));
 }
 
-// Real form of a DFT matrix as a K-major B operand: row n = 2 k + (0: re, 1: im)
-// of output k, column j = 2 s + (0: re, 1: im) of input s, entry of w_R^(s k).
+// Two complex values in split form: re = (re_a, re_b), im = (im_a, im_b), so
+// that a complex multiply is two packed fp32x2 multiply-adds per value.
+struct C2 {
+    float2 re, im;
+};
+__device__ __forceinline__ C2 cmul2(const C2& a, const C2& w) {
+    C2 r;
+    r.re = __ffma2_rn(make_float2(-a.im.x, -a.im.y), w.im, __fmul2_rn(a.re, w.re));
+    r.im = __ffma2_rn(a.im, w.re, __fmul2_rn(a.re, w.im));
+    return r;
+}
+__device__ __forceinline__ C2 c2_splat(float2 w) { return C2{make_float2(w.x, w.x), make_float2(w.y, w.y)}; }
+__device__ __forceinline__ C2 c2_of(float2 a, float2 b) { return C2{make_float2(a.x, b.x), make_float2(a.y, b.y)}; }
+// Accumulator columns 4p .. 4p+3 hold outputs 2p, 2p+1 as (re, re, im, im).
+template <int NCOL>
+__device__ __forceinline__ C2 c2_at(const float (&d)[NCOL], int p) {
+    return C2{make_float2(d[4 * p], d[4 * p + 1]), make_float2(d[4 * p + 2], d[4 * p + 3])};
+}
+
+// Real form of a DFT matrix as a K-major B operand, entry of w_R^(s k): column
+// j = 2 s + (0: re, 1: im) of input s; row n holds output k = 2 (n >> 2) + (n & 1),
+// real part for (n >> 1) & 1 == 0, else imaginary part, so that the accumulator
+// columns of outputs 2p, 2p+1 read (re, re, im, im).
 __device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo) {
     for (int idx = threadIdx.x; idx < 4 * nout * nin; idx += NT) {
         const int n = idx / (2 * nin), j = idx % (2 * nin);
-        const int e = ((n >> 1) * (j >> 1)) % R;
+        const int k = 2 * (n >> 2) + (n & 1);
+        const bool im_row = (n >> 1) & 1;
+        const int e = (k * (j >> 1)) % R;
         float sv, cv;
         sincospif(2.0f * float(e) / float(R), &sv, &cv);   // w = cv - i sv
         float v;
-        if ((n & 1) == 0) v = (j & 1) == 0 ? cv : sv;       // re: Re w xr - Im w xi
+        if (!im_row) v = (j & 1) == 0 ? cv : sv;            // re: Re w xr - Im w xi
         else v = (j & 1) == 0 ? -sv : cv;                   // im: Im w xr + Re w xi
         *reinterpret_cast<bf16*>(Bm + tc::kmaj_off(n, j, sbo)) = __float2bfloat16_rn(v);
     }
@@ -236,13 +259,14 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16);
     fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64);
     fill_dft(smem_tc + kOffB1i, 16, 8, 16, kSBO32);
-    // TW2[(T * 16 + kp) * 8 + l] = (w1024^(b k), w1024^(b (k+1))), b = 4 l + T, k = 2 kp
+    // TW2[(T * 16 + kp) * 8 + l] = (Re w0, Re w1, Im w0, Im w1), w0 = w1024^(b k),
+    // w1 = w1024^(b (k+1)), b = 4 l + T, k = 2 kp
     for (int idx = t; idx < 4 * 16 * 8; idx += NT) {
         const int l = idx & 7, kp = (idx >> 3) & 15, T = idx >> 7;
         const int bb = 4 * l + T, k = 2 * kp;
         const float2 w0 = wN(16 * ((bb * k) & 1023), twist, odd);
         const float2 w1 = wN(16 * ((bb * (k + 1)) & 1023), twist, odd);
-        TW2[idx] = make_float4(w0.x, w0.y, w1.x, w1.y);
+        TW2[idx] = make_float4(w0.x, w1.x, w0.y, w1.y);
     }
     if (t == 0) tc::mbar_init(&mbar, 1);
     if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
@@ -371,8 +395,9 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
                         const int n = a + 1024 * s;
-                        const float za = sc1(xg0, n, tg) * d[2 * s];
-                        const float zb = pr.has1 ? sc1(xg1, n, tg) * -d[2 * s + 1] : 0.0f;
+                        const int col = 4 * (s >> 1) + (s & 1);            // re at col, im at col + 2
+                        const float za = sc1(xg0, n, tg) * d[col];
+                        const float zb = pr.has1 ? sc1(xg1, n, tg) * -d[col + 2] : 0.0f;
                         pk[s] = pack_bf16(za, zb);
                     }
                     sts128(A1, tc::chunk_off(rho1(a), 0, kSBO16), pk[0], pk[1], pk[2], pk[3]);
@@ -383,13 +408,15 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             // ---------------- stage 1: 8 tiles x (K 16 -> N 32)
             {
                 // twiddle w_N^(a k1); vector a = b + 32 q, b = 4 (lane & 7) + (lane >> 3),
-                // q = j + 4 Q + 16 h -> stage-2 row (k1, b), chunk Q + 4 h (slots q, j = 0..3)
+                // q = j + 4 Q + 16 h -> stage-2 row (k1, b), chunk Q + 4 h (slots q, j = 0..3).
+                // Twiddles run in pairs (k1, k1 + 1), stepped by beta^2.
                 const int b1 = 4 * (lane & 7) + (lane >> 3);
-                float2 beta[4], pw[4];
+                C2 pw[4], st2[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    beta[j] = wN(b1 + 32 * (j + 4 * Q + 16 * hh), twist, odd);
-                    pw[j] = make_float2(1.0f, 0.0f);
+                    const float2 beta = wN(b1 + 32 * (j + 4 * Q + 16 * hh), twist, odd);
+                    pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
+                    st2[j] = c2_splat(cmul(beta, beta));
                 }
                 ok &= stage_wait(&mbar, phase);
                 // row rho2(k1, b): row / 8 = 16 (lane >> 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane & 7
@@ -402,16 +429,20 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const int k1 = 8 * half + kk;
-                        uint32_t pk[4];
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const int k1 = 8 * half + 2 * pp;
+                        C2 v[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const float2 v = cmul(make_float2(d[j][2 * kk], d[j][2 * kk + 1]), pw[j]);
-                            pw[j] = cmul(pw[j], beta[j]);
-                            pk[j] = pack_bf16(v.x, v.y);
+                            v[j] = cmul2(c2_at(d[j], pp), pw[j]);
+                            pw[j] = cmul2(pw[j], st2[j]);
                         }
-                        sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64, pk[0], pk[1], pk[2], pk[3]);
+                        sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64,
+                               pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
+                               pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+                        sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64,
+                               pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
+                               pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
                     }
                 }
             }
@@ -433,21 +464,19 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int ip = 0; ip < 2; ++ip) {
-                        float4 w[4];
+                        C2 v[4];
 #pragma unroll
-                        for (int T = 0; T < 4; ++T) w[T] = tw[(T * 16 + 2 * gq + ip) * 8];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int i = 2 * ip + e;
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int T = 0; T < 4; ++T) {
-                                const float2 ww = e ? make_float2(w[T].z, w[T].w) : make_float2(w[T].x, w[T].y);
-                                const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), ww);
-                                pk[T] = pack_bf16(v.x, v.y);
-                            }
-                            sts128(A, base + uint32_t(16 * i) * kSBO64 + uint32_t(gq) * 16u, pk[0], pk[1], pk[2], pk[3]);
+                        for (int T = 0; T < 4; ++T) {
+                            const float4 w = tw[(T * 16 + 2 * gq + ip) * 8];
+                            v[T] = cmul2(c2_at(d[T], ip), C2{make_float2(w.x, w.y), make_float2(w.z, w.w)});
                         }
+                        const int i = 2 * ip;
+                        sts128(A, base + uint32_t(16 * i) * kSBO64 + uint32_t(gq) * 16u,
+                               pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
+                               pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+                        sts128(A, base + uint32_t(16 * (i + 1)) * kSBO64 + uint32_t(gq) * 16u,
+                               pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
+                               pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
                     }
                 }
             }
@@ -473,16 +502,13 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const uint4 kk = kv[4 * T + q4];
-                        const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w};
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 4 * q4 + e;
-                            const float2 K = make_float2(bf_lo(kw[e]), bf_hi(kw[e]));
-                            const float2 v = cmul(make_float2(d[2 * i], d[2 * i + 1]), K);
-                            pk[e] = pack_bf16(v.x, -v.y);
-                        }
-                        sts128(A, rowoff + q4 * tc::kLBO, pk[0], pk[1], pk[2], pk[3]);
+                        // bins i = 4 q4 .. 4 q4 + 3 as two split pairs
+                        const C2 K0{make_float2(bf_lo(kk.x), bf_lo(kk.y)), make_float2(bf_hi(kk.x), bf_hi(kk.y))};
+                        const C2 K1{make_float2(bf_lo(kk.z), bf_lo(kk.w)), make_float2(bf_hi(kk.z), bf_hi(kk.w))};
+                        const C2 v0 = cmul2(c2_at(d, 2 * q4), K0);
+                        const C2 v1 = cmul2(c2_at(d, 2 * q4 + 1), K1);
+                        sts128(A, rowoff + q4 * tc::kLBO, pack_bf16(v0.re.x, -v0.im.x), pack_bf16(v0.re.y, -v0.im.y),
+                               pack_bf16(v1.re.x, -v1.im.x), pack_bf16(v1.re.y, -v1.im.y));
                     }
                 }
             }
@@ -504,22 +530,19 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int ip = 0; ip < 2; ++ip) {
-                        float4 w[4];
+                        C2 v[4];
 #pragma unroll
-                        for (int T = 0; T < 4; ++T) w[T] = tw[(T * 16 + 2 * gq + ip) * 8];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int i = 2 * ip + e;
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int T = 0; T < 4; ++T) {
-                                const float2 ww = e ? make_float2(w[T].z, w[T].w) : make_float2(w[T].x, w[T].y);
-                                const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), ww);
-                                pk[T] = pack_bf16(v.x, v.y);
-                            }
-                            sts128(A, base + uint32_t(gq >> 1) * kSBO64 + uint32_t(4 * (gq & 1) + i) * 16u, pk[0], pk[1],
-                                   pk[2], pk[3]);
+                        for (int T = 0; T < 4; ++T) {
+                            const float4 w = tw[(T * 16 + 2 * gq + ip) * 8];
+                            v[T] = cmul2(c2_at(d[T], ip), C2{make_float2(w.x, w.y), make_float2(w.z, w.w)});
                         }
+                        const int i = 2 * ip;
+                        sts128(A, base + uint32_t(gq >> 1) * kSBO64 + uint32_t(4 * (gq & 1) + i) * 16u,
+                               pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
+                               pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+                        sts128(A, base + uint32_t(gq >> 1) * kSBO64 + uint32_t(4 * (gq & 1) + i + 1) * 16u,
+                               pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
+                               pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
                     }
                 }
             }
@@ -531,12 +554,14 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 // row a = lane + 32 (16 h + 4 gq + i): a / 8 = (lane >> 3) + 64 h + 16 gq + 4 i, a % 8 = lane & 7
                 const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
                                       uint32_t(lane & 7) * 16u;
-                float2 pw[4], stp[4];
+                // twiddles in pairs (q, q + 1), stepped by w_N^(64 k1)
+                C2 pw[4], st2[4];
 #pragma unroll
                 for (int T = 0; T < 4; ++T) {
                     const int k1 = 4 * Q + T;
-                    pw[T] = wN((lane + 512 * hh) * k1, twist, odd);
-                    stp[T] = wN(32 * k1, twist, odd);
+                    const float2 p0 = wN((lane + 512 * hh) * k1, twist, odd);
+                    pw[T] = c2_of(p0, cmul(p0, wN(32 * k1, twist, odd)));
+                    st2[T] = c2_splat(wN(64 * k1, twist, odd));
                 }
                 ok &= stage_wait(&mbar, phase);
 #pragma unroll 1
@@ -546,15 +571,20 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t pk[4];
+                    for (int ip = 0; ip < 2; ++ip) {
+                        C2 v[4];
 #pragma unroll
                         for (int T = 0; T < 4; ++T) {
-                            const float2 v = cmul(make_float2(d[T][2 * i], d[T][2 * i + 1]), pw[T]);
-                            pw[T] = cmul(pw[T], stp[T]);
-                            pk[T] = pack_bf16(v.x, v.y);
+                            v[T] = cmul2(c2_at(d[T], ip), pw[T]);
+                            pw[T] = cmul2(pw[T], st2[T]);
                         }
-                        sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pk[0], pk[1], pk[2], pk[3]);
+                        const int i = 2 * ip;
+                        sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
+                               pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x),
+                               pack_bf16(v[3].re.x, v[3].im.x));
+                        sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
+                               pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y),
+                               pack_bf16(v[3].re.y, v[3].im.y));
                     }
                 }
             }
@@ -578,7 +608,10 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int s8 = 0; s8 < 8; ++s8) Vs[a + 1024 * s8] = pack_bf16(d[2 * s8], -d[2 * s8 + 1]);
+            for (int s8 = 0; s8 < 8; ++s8) {
+                const int col = 4 * (s8 >> 1) + (s8 & 1);                 // re at col, im at col + 2
+                Vs[a + 1024 * s8] = pack_bf16(d[col], -d[col + 2]);
+            }
         }
         prev = pr;
         have_prev = true;
