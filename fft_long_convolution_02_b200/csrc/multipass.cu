@@ -347,16 +347,39 @@ k_mp_pass_c(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws,
 // keeps the natural entry order and the generic kernel above.
 // ===========================================================================
 
+// Four-step twiddles w_M^(m1 n2) of a thread's 16 column positions 16 g + k,
+// m1 = fft_pos_bin(16 g + k).  For M1 = 128 and 256 the bins of k = 0..7 and of
+// k = 8..15 are two runs with step 16, so three table entries and 14 complex
+// multiplies replace 16 scattered table reads (relative error < 1e-6).
+template <int M1>
+struct ColTw {
+    float2 a, b, step;
+    __device__ __forceinline__ ColTw(const MpTables& tb, int M2, int n2, int g) {
+        static_assert(M1 == 128 || M1 == 256, "run structure holds for M1 = 128, 256");
+        a = __ldg(tb.four + int64_t(fft_pos_bin<M1>(16 * g)) * M2 + n2);
+        b = __ldg(tb.four + int64_t(fft_pos_bin<M1>(16 * g + 8)) * M2 + n2);
+        step = __ldg(tb.four + int64_t(16) * M2 + n2);          // w_M^(16 n2)
+    }
+    // twiddle of position k (call with k = 0, 1, ..., 15 in order)
+    __device__ __forceinline__ float2 next(int k) {
+        float2 r;
+        if (k < 8) { r = a; a = cmul(a, step); }
+        else { r = b; b = cmul(b, step); }
+        return r;
+    }
+};
+
 template <int M1>
 __device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables& tb, float2* __restrict__ ws_row,
                                               int M2, int n2, int g) {
     const int M = M1 * M2;
+    ColTw<M1> tw(tb, M2, n2, g);
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
         const int m1 = fft_pos_bin<M1>(16 * g + k);
-        const float2 tw = __ldg(tb.four + int64_t(m1) * M2 + n2);
-        ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2] = cmul(x[0][k], tw);
-        ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2] = cmul(x[1][k], tw);
+        const float2 w = tw.next(k);
+        ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2] = cmul(x[0][k], w);
+        ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2] = cmul(x[1][k], w);
     }
 }
 
@@ -427,12 +450,15 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
     const int64_t L = int64_t(2) * M;
     float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
     float2 x[2][16];
+    {
+        ColTw<M1> tw(tb, M2, n2, g);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int m1 = fft_pos_bin<M1>(16 * g + k);
-        const float2 tw = __ldg(tb.four + int64_t(m1) * M2 + n2);
-        x[0][k] = cmulc(ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2], tw);
-        x[1][k] = cmulc(ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2], tw);
+        for (int k = 0; k < 16; ++k) {
+            const int m1 = fft_pos_bin<M1>(16 * g + k);
+            const float2 w = tw.next(k);
+            x[0][k] = cmulc(ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2], w);
+            x[1][k] = cmulc(ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2], w);
+        }
     }
     float2* const buf[2] = {smem + j * PS, smem + (16 + j) * PS};
     reg_fft_inverse<M1, 2>(x, buf, g, tb.fftA);
