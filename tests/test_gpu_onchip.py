@@ -56,6 +56,40 @@ def test_orders_at_8192(orc, order, dtype):
     _check_all_rows(orc, p)
 
 
+def test_tensor_core_single_row_order8_no_shortconv(orc):
+    """The bf16 L = 8192 tensor-core kernel with one batch row (every pair has an
+    empty imaginary half), seven order steps, and no short conv."""
+    p = I.WORKLOADS["d768_l8k"].with_(B=1, C=3, order=8, seed=4401)
+    _check_all_rows(orc, p, use_shortconv=False)
+
+
+def test_tensor_core_causality():
+    """bf16 L = 8192 (tensor-core kernel): replacing every sample of u after t0 by
+    fresh values of the same distribution leaves y[0:t0] unchanged within the bf16
+    tolerance; a transform without the zero padding would wrap the change into
+    y[0:t0] at full size."""
+    import torch
+    from gpu_helpers import from_torch
+    p = I.WORKLOADS["d768_l8k"].with_(B=2, C=6, seed=4402)
+    data = I.make_all(p)
+    r = Run(p, data)
+    y0 = r.run()
+    t0 = 3000
+    u2 = r.u.clone()
+    g = torch.Generator(device="cuda").manual_seed(7)
+    u2[..., t0:] = torch.randn(u2[..., t0:].shape, device="cuda", generator=g).to(u2.dtype)
+    y1 = torch.empty_like(r.y)
+    r.conv(u=u2, y=y1)
+    torch.cuda.synchronize()
+    y1 = from_torch(y1)
+    a = y0[..., :t0].reshape(p.B * p.C, -1)
+    b = y1[..., :t0].reshape(p.B * p.C, -1)
+    err = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
+    assert err.max() <= TOL["bf16"], err.max()
+    # and the tail did change
+    assert not np.allclose(y0[..., t0:], y1[..., t0:])
+
+
 def test_shortconv_bias_and_odd_batch(orc):
     p = I.WORKLOADS["d768_l8k"].with_(B=3, C=9, sc_bias=True, seed=77)
     _check_all_rows(orc, p)
