@@ -33,6 +33,7 @@ cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStrea
 cudaError_t launch_spectrum_onchip(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_onchip(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s);
+constexpr int kMaxOrderTc = 3;   // highest order the L = 8192 tensor-core kernel serves
 cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);

@@ -629,8 +629,11 @@ cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
 template <int M>
 cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     if constexpr (M == 4096) {
-        // bf16 storage: DFT stages on the tensor cores; fp32 storage: fp32 FFT
-        return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : launch_conv_8192_tc(p, a, s);
+        // bf16 storage, order <= 3: DFT stages on the tensor cores (bf16 operands,
+        // row error ~5e-3 per order step); more order steps or fp32 storage: the
+        // fp32 register kernel (the bf16-operand error of 7 steps reaches 2e-2)
+        if (a.dtype != DT_F32 && p.order <= kMaxOrderTc) return launch_conv_8192_tc(p, a, s);
+        return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : conv_4096<__nv_bfloat16>(p, a, s);
     }
     constexpr int NT = onchip_threads<M>();
     const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);

@@ -49,16 +49,23 @@ def test_orders(orc, order):
     _check_all_rows(orc, p)
 
 
-@pytest.mark.parametrize("order,dtype", [(3, "bf16"), (4, "f32")])
+@pytest.mark.parametrize("order,dtype", [(3, "bf16"), (4, "bf16"), (4, "f32"), (8, "bf16")])
 def test_orders_at_8192(orc, order, dtype):
-    """The register-resident L = 8192 kernel across several order steps."""
+    """L = 8192 across several order steps: bf16 order <= 3 on the tensor-core
+    kernel, higher orders and fp32 on the fp32 register kernel."""
     p = I.WORKLOADS["d768_l8k"].with_(B=2, C=5, order=order, dtype=dtype, sc_bias=True, seed=310 + order)
     _check_all_rows(orc, p)
 
 
-def test_tensor_core_single_row_order8_no_shortconv(orc):
+def test_tensor_core_single_row_order3_no_shortconv(orc):
     """The bf16 L = 8192 tensor-core kernel with one batch row (every pair has an
-    empty imaginary half), seven order steps, and no short conv."""
+    empty imaginary half), two order steps, and no short conv."""
+    p = I.WORKLOADS["d768_l8k"].with_(B=1, C=3, order=3, seed=4401)
+    _check_all_rows(orc, p, use_shortconv=False)
+
+
+def test_bf16_order8_single_row_no_shortconv(orc):
+    """bf16 L = 8192 at order 8 (seven steps, fp32 register kernel), one row."""
     p = I.WORKLOADS["d768_l8k"].with_(B=1, C=3, order=8, seed=4401)
     _check_all_rows(orc, p, use_shortconv=False)
 
