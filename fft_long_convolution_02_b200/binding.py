@@ -17,13 +17,14 @@ LIB_PATH = os.path.join(HERE, "libhyena_b200.so")
 HYENA_F32, HYENA_BF16 = 0, 1
 STATUS = {0: "HYENA_OK", 1: "HYENA_ERR_INVALID_ARG", 2: "HYENA_ERR_UNSUPPORTED_SHAPE",
           3: "HYENA_ERR_MISALIGNED", 4: "HYENA_ERR_SPECTRUM_MISMATCH",
-          5: "HYENA_ERR_WORKSPACE_TOO_SMALL", 6: "HYENA_ERR_CUDA", 7: "HYENA_ERR_INTERNAL"}
+          5: "HYENA_ERR_WORKSPACE_TOO_SMALL", 6: "HYENA_ERR_CUDA", 7: "HYENA_ERR_INTERNAL",
+          8: "HYENA_ERR_TIMEOUT"}
 
 # every symbol include/hyena.h declares
 EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "hyena_spectrum_bytes",
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
            "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
-           "hyena_spectrum_check"]
+           "hyena_spectrum_check", "hyena_debug_conv_tc"]
 
 _lock = threading.Lock()
 _lib = None
@@ -71,6 +72,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                     ctypes.c_int, ctypes.c_int, vp]
         lib.hyena_spectrum_check.restype = ctypes.c_int
         lib.hyena_spectrum_check.argtypes = [vp, i64, ctypes.c_int, i64p, ctypes.c_int, vp]
+        lib.hyena_debug_conv_tc.restype = ctypes.c_int
+        lib.hyena_debug_conv_tc.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, ctypes.c_uint64,
+                                            ctypes.c_int, vp]
         _lib = lib
     return _lib
 
@@ -171,3 +175,13 @@ def hyena_gated_fftconv_noalloc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, s
 def hyena_spectrum_check(spectrum, C: int, sizes, order: int, stream=None) -> None:
     arr, nd = _sizes(sizes)
     _check(load().hyena_spectrum_check(_ptr(spectrum), C, nd, arr, order, _stream(stream)))
+
+
+def hyena_debug_conv_tc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, order: int, wait_budget_ns: int,
+                        issue_mma: bool = True, stream=None) -> None:
+    """Test hook of the L = 8192 bf16 tensor-core kernel: its bounded waits give
+    up after wait_budget_ns; issue_mma=False issues no tensor-core work, so the
+    first wait runs out (read back with hyena_spectrum_check)."""
+    _check(load().hyena_debug_conv_tc(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
+                                      _ptr(sc_w), _ptr(sc_bias), B, C, order, int(wait_budget_ns),
+                                      1 if issue_mma else 0, _stream(stream)))

@@ -73,6 +73,7 @@ const char* hyena_status_string(hyena_status_t s) {
         case HYENA_ERR_WORKSPACE_TOO_SMALL: return "HYENA_ERR_WORKSPACE_TOO_SMALL";
         case HYENA_ERR_CUDA: return "HYENA_ERR_CUDA";
         case HYENA_ERR_INTERNAL: return "HYENA_ERR_INTERNAL";
+        case HYENA_ERR_TIMEOUT: return "HYENA_ERR_TIMEOUT";
     }
     return "HYENA_UNKNOWN_STATUS";
 }
@@ -142,11 +143,16 @@ size_t hyena_gated_fftconv_workspace_bytes(int64_t B, int64_t C, int ndim, const
     return size_t(default_group_rows(p, B * C)) * p.ws_row_bytes;
 }
 
-hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
-                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
-                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
-    Plan p;
+}  // extern "C"
+
+namespace {
+
+// Validation shared by the convolution entry points; fills the plan and the
+// kernel arguments.
+hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, const float* sc_w,
+                            const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes, int order,
+                            hyena_dtype_t dtype, void* workspace, size_t workspace_bytes, Plan* pp, ConvArgs* pa) {
+    Plan& p = *pp;
     hyena_status_t st = plan_or_fail(C, ndim, sizes, order, &p);
     if (st != HYENA_OK) return st;
     if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
@@ -176,8 +182,24 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
         group = int64_t(workspace_bytes / p.ws_row_bytes);
         if (group > B * C) group = B * C;
     }
-    ConvArgs a{u, y, static_cast<const uint8_t*>(spectrum), sc_w, sc_w ? sc_bias : nullptr, B, int(dtype),
-               static_cast<float2*>(workspace), group};
+    *pa = ConvArgs{u, y, static_cast<const uint8_t*>(spectrum), sc_w, sc_w ? sc_bias : nullptr, B, int(dtype),
+                   static_cast<float2*>(workspace), group};
+    return HYENA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    Plan p;
+    ConvArgs a;
+    hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype,
+                                     workspace, workspace_bytes, &p, &a);
+    if (st != HYENA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     switch (p.path) {
@@ -187,6 +209,23 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "gated fftconv kernel");
+}
+
+hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int order,
+                                   uint64_t wait_budget_ns, int issue_mma, void* stream) {
+    Plan p;
+    ConvArgs a;
+    const int64_t L = 8192;
+    hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, 1, &L, order, HYENA_BF16,
+                                     nullptr, 0, &p, &a);
+    if (st != HYENA_OK) return st;
+    if (order > kMaxOrderTc)
+        return fail(HYENA_ERR_UNSUPPORTED_SHAPE, "the tensor-core kernel serves order <= " + std::to_string(kMaxOrderTc));
+    if (wait_budget_ns == 0) return fail(HYENA_ERR_INVALID_ARG, "wait_budget_ns must be > 0");
+    a.wait_budget_ns = wait_budget_ns;
+    a.issue_mma = issue_mma ? 1 : 0;
+    return cuda_status(launch_conv_8192_tc(p, a, static_cast<cudaStream_t>(stream)), "tensor-core kernel");
 }
 
 hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
@@ -204,7 +243,7 @@ hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, c
         h.H != p.H || h.W != p.W || h.order != p.order || size_t(h.total_bytes) != p.total_bytes)
         return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum header does not match (C, sizes, order)");
     if (h.device_status != 0)
-        return fail(HYENA_ERR_INTERNAL, "a convolution with this spectrum gave up waiting for the tensor cores");
+        return fail(HYENA_ERR_TIMEOUT, "a convolution with this spectrum ran out of its tensor-core wait budget");
     return ok();
 }
 

@@ -10,6 +10,10 @@ namespace hyena {
 
 enum DType { DT_F32 = 0, DT_BF16 = 1 };
 
+// Default budget of a bounded device wait: far above a normal wait (us), and
+// long enough to ride out time-slicing with other contexts on a shared GPU.
+constexpr uint64_t kDefaultWaitBudgetNs = 2000000000ull;
+
 struct SpectrumArgs {
     const void* k;        // [order-1, C, n]
     int k_dtype;
@@ -27,6 +31,10 @@ struct ConvArgs {
     int dtype;
     float2* workspace;    // multi-pass / 2-D only
     int64_t group_rows;   // rows per workspace group
+    // L = 8192 tensor-core kernel only: budget of each bounded wait, and whether
+    // the tensor-core work is issued (0 only from the timeout test hook)
+    uint64_t wait_budget_ns = kDefaultWaitBudgetNs;
+    int issue_mma = 1;
 };
 
 cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);

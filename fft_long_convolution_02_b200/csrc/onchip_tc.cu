@@ -66,7 +66,6 @@ constexpr uint32_t kOffB32 = kOffB1 + kB1bytes;
 constexpr uint32_t kOffB1i = kOffB32 + kB32bytes;
 constexpr uint32_t kOffTW2 = kOffB1i + kB1ibytes;
 constexpr size_t kSmem = size_t(kOffTW2) + kTW2bytes;
-constexpr int kWaitLimit = 1 << 22;
 static_assert(L * 4 <= kOffA1, "output staging must not overlap the stage-1 operand");
 static_assert(kOffTW2 % 16 == 0, "twiddle table alignment");
 
@@ -144,14 +143,15 @@ __device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo) {
 }
 
 // Publish this thread's operand writes and issue the stage's MMAs from one
-// thread (tiles x ksteps MMAs of M = 128), committed to `mbar`.
+// thread (tiles x ksteps MMAs of M = 128), committed to `mbar`.  Nothing is
+// issued once a wait has run out (go == false), so nothing is left in flight.
 __device__ __forceinline__ void stage_issue(uint32_t a, uint32_t sbo_a, uint32_t b, uint32_t sbo_b, int tiles,
                                             int ksteps, uint32_t idesc, uint32_t tmem, uint32_t dcols,
-                                            uint64_t* mbar) {
+                                            uint64_t* mbar, bool go) {
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && go) {
         tc::fence_after_sync();
         for (int T = 0; T < tiles; ++T)
             for (int ks = 0; ks < ksteps; ++ks)
@@ -161,12 +161,14 @@ __device__ __forceinline__ void stage_issue(uint32_t a, uint32_t sbo_a, uint32_t
         tc::commit(mbar);
     }
 }
-// Wait (bounded) for the last issued stage.
-__device__ __forceinline__ bool stage_wait(uint64_t* mbar, uint32_t& phase) {
-    const bool ok = tc::mbar_wait(mbar, phase, kWaitLimit);
+// Wait (bounded by budget_ns) for the last issued stage; after a wait has run
+// out (ok == false) no further waits are made.
+__device__ __forceinline__ bool stage_wait(uint64_t* mbar, uint32_t& phase, bool ok, uint64_t budget_ns) {
+    if (!ok) return false;
+    const bool done = tc::mbar_wait(mbar, phase, budget_ns);
     phase ^= 1u;
     tc::fence_after_sync();
-    return ok;
+    return done;
 }
 
 // Raw samples n0 .. n0+7 and the two before them (n0 % 8 == 0) of one row.
@@ -230,7 +232,7 @@ __device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __res
 __global__ void __launch_bounds__(NT, 2)
 k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
                const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-               int64_t npairs) {
+               int64_t npairs, uint64_t wait_budget_ns, int issue_mma) {
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
@@ -370,7 +372,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u + 4u * jp) =
                         make_uint2(pk[i][0], pk[i][1]);
             }
-            stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
+            stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
             if (have_prev) {
                 output_gate(prev);                  // overlaps the stage-1 MMAs
                 have_prev = false;
@@ -403,7 +405,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     sts128(A1, tc::chunk_off(rho1(a), 0, kSBO16), pk[0], pk[1], pk[2], pk[3]);
                     sts128(A1, tc::chunk_off(rho1(a), 1, kSBO16), pk[4], pk[5], pk[6], pk[7]);
                 }
-                stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar);
+                stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
             }
             // ---------------- stage 1: 8 tiles x (K 16 -> N 32)
             {
@@ -418,7 +420,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
                     st2[j] = c2_splat(cmul(beta, beta));
                 }
-                ok &= stage_wait(&mbar, phase);
+                ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
                 // row rho2(k1, b): row / 8 = 16 (lane >> 3) + 4 (k1 >> 2) + (k1 & 3), row % 8 = lane & 7
                 const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
                                       uint32_t(lane & 7) * 16u;
@@ -447,8 +449,8 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
             }
             // ---------------- stage 2: 4 tiles x (K 64 -> N 64)
-            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
-            ok &= stage_wait(&mbar, phase);
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
             {
                 // rows (k1 = 4 Q + lane / 8, b = 4 (lane & 7) + T), outputs k2 = 16 h + ..
                 // twiddle w1024^(b k2) -> stage-3 row (k1, k2), chunk lane & 7
@@ -481,7 +483,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
             }
             // ---------------- stage 3; meanwhile this thread loads its spectrum values
-            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
             {
                 // row (k1 = 4 Q + lane / 8, k2 = 4 (lane & 7) + T) keeps its place, slots
                 // k3 = 16 h + 4 i + e; spectrum entry uint4 (T * 4 + i) of this thread
@@ -491,7 +493,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 uint4 kv[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) kv[i] = __ldg(kq + 32 * i);
-                ok &= stage_wait(&mbar, phase);
+                ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
 #pragma unroll
                 for (int T = 0; T < 4; ++T) {
                     float d[32];
@@ -513,8 +515,8 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
             }
             // ---------------- stage 3' (inverse, on conj)
-            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
-            ok &= stage_wait(&mbar, phase);
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
             {
                 // rows (k1 = 4 Q + lane / 8, k2 = 4 (lane & 7) + T), outputs b = 16 h + ..
                 // twiddle w1024^(b k2) -> stage-2' row (k1, b), chunk lane & 7
@@ -547,7 +549,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
             }
             // ---------------- stage 2'
-            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar);
+            stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
             {
                 // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w_N^((b + 32 q) k1)
                 // -> stage-1' row a = b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
@@ -563,7 +565,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                     pw[T] = c2_of(p0, cmul(p0, wN(32 * k1, twist, odd)));
                     st2[T] = c2_splat(wN(64 * k1, twist, odd));
                 }
-                ok &= stage_wait(&mbar, phase);
+                ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
 #pragma unroll 1
                 for (int gq = 0; gq < 4; ++gq) {
                     float d[4][8];
@@ -589,8 +591,8 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 }
             }
             // ---------------- stage 1': 8 tiles x (K 32 -> N 16), outputs s < 8 only
-            stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar);
-            if (st < order - 1) ok &= stage_wait(&mbar, phase);
+            stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
+            if (st < order - 1) ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         }
         // the next pair's step-1 input, loaded while stage 1' runs (unconditional, so
         // that the registers' live range ends here; past the last pair this pair's
@@ -598,7 +600,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
         const PairRef pnext = pair_ref(Pn < npairs ? Pn : P, B);
         load_pair_input(in, u, pnext, C, order, 0);
         load_pair_input(in, u, pnext, C, order, 2);
-        ok &= stage_wait(&mbar, phase);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         // output staging v = conj(D1') as (re, -im) bf16 pairs in natural order;
         // the output gate runs during the next pair's stage 1
 #pragma unroll
@@ -615,8 +617,9 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
         }
         prev = pr;
         have_prev = true;
-        if (!ok) {
-            if (t == 0) atomicOr(status, 1u);           // a tensor-core wait timed out
+        if (__syncthreads_or(!ok)) {                    // a tensor-core wait ran out (uniform decision)
+            ok = false;
+            if (t == 0) atomicOr(status, 1u);
             break;
         }
     }
@@ -641,7 +644,7 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
     int64_t grid = int64_t(2) * sms;
     if (grid > npairs) grid = npairs;
     kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
-                                           a.sc_b, a.B, p.C, p.order, npairs);
+                                           a.sc_b, a.B, p.C, p.order, npairs, a.wait_budget_ns, a.issue_mma);
     return cudaGetLastError();
 }
 

@@ -67,11 +67,19 @@ __device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Wait for the phase with parity `parity` to complete; gives up after
-// `limit` polls and returns false (the caller records the timeout).
-__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, int limit) {
+// `budget_ns` nanoseconds of global time and returns false (the caller
+// records the timeout).
+__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint64_t budget_ns) {
+    const uint64_t t0 = globaltimer_ns();
     uint32_t done = 0;
-    for (int it = 0; it < limit && !done; ++it) {
+    while (true) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -79,8 +87,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, int l
             : "=r"(done)
             : "r"(smem_u32(mbar)), "r"(parity)
             : "memory");
+        if (done) return true;
+        if (globaltimer_ns() - t0 > budget_ns) return false;
     }
-    return done != 0;
 }
 
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }

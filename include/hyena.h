@@ -56,7 +56,9 @@ typedef enum {
     HYENA_ERR_SPECTRUM_MISMATCH = 4,  /* spectrum_bytes does not match the shape      */
     HYENA_ERR_WORKSPACE_TOO_SMALL = 5,/* workspace smaller than one row's share       */
     HYENA_ERR_CUDA = 6,               /* a CUDA launch reported an error              */
-    HYENA_ERR_INTERNAL = 7
+    HYENA_ERR_INTERNAL = 7,
+    HYENA_ERR_TIMEOUT = 8             /* a bounded device wait ran out (reported by
+                                         hyena_spectrum_check)                       */
 } hyena_status_t;
 
 /* Version of this ABI (major * 100 + minor). */
@@ -188,12 +190,30 @@ hyena_status_t hyena_gated_fftconv_noalloc(const void* u, void* y, const void* s
  * Debug helper (synchronous): copies the spectrum header to the host and
  * checks it against (C, sizes, order).  Returns HYENA_OK when it matches,
  * HYENA_ERR_SPECTRUM_MISMATCH when not (e.g. never filled, or filled for
- * another shape), HYENA_ERR_INTERNAL when an earlier convolution with this
- * spectrum gave up on a bounded tensor-core wait (its outputs were written as
- * NaN).  Synchronises `stream`.
+ * another shape), HYENA_ERR_TIMEOUT when an earlier convolution with this
+ * spectrum ran out of the budget of a bounded tensor-core wait (the L = 8192
+ * bf16 path; the outputs of that row pair were written as NaN and nothing was
+ * left in flight).  Synchronises `stream`.  Rebuilding the spectrum clears the
+ * record.
  */
 hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
                                     void* stream);
+
+/*
+ * Test hook for the bounded waits of the tensor-core kernel (the L = 8192, bf16,
+ * order <= 3 path of hyena_gated_fftconv; same arguments with ndim = 1,
+ * sizes = {8192}, dtype = HYENA_BF16).  Each wait of that kernel on its
+ * tensor-core work gives up after `wait_budget_ns` nanoseconds (the normal entry
+ * point uses 2 s).  With issue_mma = 0 no tensor-core work is issued, so the
+ * first wait runs out on a barrier that nothing completes: the kernel records
+ * the timeout in the spectrum header (hyena_spectrum_check then returns
+ * HYENA_ERR_TIMEOUT), writes NaN to the outputs of the row pair it was on, and
+ * returns with nothing in flight.  Other shapes return
+ * HYENA_ERR_UNSUPPORTED_SHAPE.  Asynchronous on `stream`.
+ */
+hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int order,
+                                   uint64_t wait_budget_ns, int issue_mma, void* stream);
 
 #ifdef __cplusplus
 }

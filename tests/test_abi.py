@@ -105,3 +105,17 @@ def test_validation_errors_before_launch(lib):
     assert sc(fake, fake * 4, None, None, 1, 3, 64, 0, None) == 1
     assert sc(fake, fake * 4, fake * 8, None, 1, 3, 63, 0, None) == 2
     assert sc(fake, fake + 16, fake * 8, None, 1, 3, 64, 0, None) == 1
+    # tensor-core wait test hook: L = 8192 bf16 only, order <= 3, budget > 0
+    dg = lib.hyena_debug_conv_tc
+    n8 = lib.hyena_spectrum_bytes(4, 1, _sz(8192), 2)
+    n8o4 = lib.hyena_spectrum_bytes(4, 1, _sz(8192), 4)
+    big = 1 << 32
+    assert dg(None, big, big * 2, n8, None, None, 2, 4, 2, 1000, 0, None) == 1
+    assert dg(big, big * 2, big * 3, n8o4, None, None, 2, 4, 4, 1000, 0, None) == 2
+    assert dg(big, big * 2, big * 3, n8, None, None, 2, 4, 2, 0, 0, None) == 1
+    assert dg(big, big * 2, big * 3, n8 + 16, None, None, 2, 4, 2, 1000, 0, None) == 4
+
+
+def test_status_strings(lib):
+    assert lib.hyena_status_string(8) == b"HYENA_ERR_TIMEOUT"
+    assert lib.hyena_status_string(0) == b"HYENA_OK"

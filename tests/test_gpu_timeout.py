@@ -1,0 +1,55 @@
+"""GPU: the bounded waits of the L = 8192 tensor-core kernel.  The test hook
+issues no tensor-core work, so the kernel's first wait runs out on a barrier
+that nothing completes (1 ms budget, one CTA); the timeout must be reported
+through the spectrum header, the outputs of the pair must be NaN, and the
+context must stay usable.  Nothing faults, traps or hangs."""
+import numpy as np
+import pytest
+
+from fft_long_convolution_02_b200 import binding as hb
+from fft_long_convolution_02_b200 import inputs as I
+from gpu_helpers import TOL, Run, from_torch, gpu_rows, oracle_for_rows, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fft_long_convolution_02_b200 import build
+    build.build()
+
+
+def test_tensor_core_wait_timeout_is_reported(orc):
+    import torch
+    p = I.WORKLOADS["d768_l8k"].with_(B=2, C=1, seed=5101)     # one row pair: a 1-CTA launch
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    hb.hyena_spectrum_check(r.spectrum, p.C, p.shape, p.order)
+    y = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_tc(r.u, y, r.spectrum, r.sc_w, None, p.B, p.C, p.order, wait_budget_ns=1_000_000,
+                           issue_mma=False)
+    torch.cuda.synchronize()
+    with pytest.raises(hb.HyenaError) as ei:
+        hb.hyena_spectrum_check(r.spectrum, p.C, p.shape, p.order)
+    assert ei.value.status == 8                                   # HYENA_ERR_TIMEOUT
+    assert torch.isnan(y.float()).all()
+    # the context is still usable: rebuild the spectrum (clears the record) and run normally
+    r.build_spectrum()
+    hb.hyena_spectrum_check(r.spectrum, p.C, p.shape, p.order)
+    r.conv()
+    torch.cuda.synchronize()
+    got = from_torch(r.y)
+    rows = np.arange(p.B * p.C)
+    err = row_rel_err(gpu_rows(got, p, rows), oracle_for_rows(orc, p, rows, data))
+    assert err.max() <= TOL["bf16"], err.max()
+    # the hook with the tensor-core work issued and the default budget gives the same result
+    y2 = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_tc(r.u, y2, r.spectrum, r.sc_w, None, p.B, p.C, p.order, wait_budget_ns=2_000_000_000,
+                           issue_mma=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, r.y)
+    hb.hyena_spectrum_check(r.spectrum, p.C, p.shape, p.order)
