@@ -73,21 +73,29 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+__device__ __forceinline__ bool mbar_try(uint64_t* mbar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(mbar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the phase with parity `parity` to complete; gives up after
 // `budget_ns` nanoseconds of global time and returns false (the caller
-// records the timeout).
+// records the timeout).  The clock is read only once the first poll has
+// failed, and then every 8 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, uint64_t budget_ns) {
+    if (mbar_try(mbar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t done = 0;
     while (true) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(smem_u32(mbar)), "r"(parity)
-            : "memory");
-        if (done) return true;
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try(mbar, parity)) return true;
         if (globaltimer_ns() - t0 > budget_ns) return false;
     }
 }
