@@ -182,12 +182,25 @@ __device__ __forceinline__ Raw8 load8(const bf16* __restrict__ x, int n0) {
     r.halo = n0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(x + n0 - 2)) : 0u;
     return r;
 }
-// Width-3 causal short conv of the 8 samples of `r`.
-__device__ __forceinline__ void sc8(const Raw8& r, const Taps& tp, float (&o)[8]) {
-    const float v[10] = {bf_lo(r.halo),  bf_hi(r.halo),  bf_lo(r.cur.x), bf_hi(r.cur.x), bf_lo(r.cur.y),
-                         bf_hi(r.cur.y), bf_lo(r.cur.z), bf_hi(r.cur.z), bf_lo(r.cur.w), bf_hi(r.cur.w)};
+// Short conv of the same 8 samples of the two rows of a pair at once: o[i] =
+// (sc of row b0, sc of row b1) at sample i, with packed fp32x2 FMAs; tap pairs
+// (w for row b0, w for row b1).
+struct Taps2 {
+    float2 w0, w1, w2, b;
+};
+__device__ __forceinline__ Taps2 taps2(const Taps& t, float m1) {
+    return Taps2{make_float2(t.w0, m1 * t.w0), make_float2(t.w1, m1 * t.w1), make_float2(t.w2, m1 * t.w2),
+                 make_float2(t.b, m1 * t.b)};
+}
+__device__ __forceinline__ void sc8x2(const Raw8& r0, const Raw8& r1, const Taps2& tp, float2 (&o)[8]) {
+    const float2 v[10] = {make_float2(bf_lo(r0.halo), bf_lo(r1.halo)),   make_float2(bf_hi(r0.halo), bf_hi(r1.halo)),
+                          make_float2(bf_lo(r0.cur.x), bf_lo(r1.cur.x)), make_float2(bf_hi(r0.cur.x), bf_hi(r1.cur.x)),
+                          make_float2(bf_lo(r0.cur.y), bf_lo(r1.cur.y)), make_float2(bf_hi(r0.cur.y), bf_hi(r1.cur.y)),
+                          make_float2(bf_lo(r0.cur.z), bf_lo(r1.cur.z)), make_float2(bf_hi(r0.cur.z), bf_hi(r1.cur.z)),
+                          make_float2(bf_lo(r0.cur.w), bf_lo(r1.cur.w)), make_float2(bf_hi(r0.cur.w), bf_hi(r1.cur.w))};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = fmaf(tp.w0, v[i], fmaf(tp.w1, v[i + 1], fmaf(tp.w2, v[i + 2], tp.b)));
+    for (int i = 0; i < 8; ++i)
+        o[i] = __ffma2_rn(tp.w0, v[i], __ffma2_rn(tp.w1, v[i + 1], __ffma2_rn(tp.w2, v[i + 2], tp.b)));
 }
 
 // Step-1 input of a pair: thread t covers a = a0 .. a0+7 (a0 = 8 (t & 127)) at
@@ -288,33 +301,40 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     // Output gate of a finished pair: y = sc(x0) * v from the staging buffer.
     // Thread t covers samples n0 = 8 (t + 256 jj) of both rows.
     auto output_gate = [&](const PairRef& pr) {
-        const Taps t0 = load_taps(sc_w, sc_b, pr.c);
+        const Taps2 t0 = taps2(load_taps(sc_w, sc_b, pr.c), 1.0f);
+        const bf16* x00 = u + (pr.b0 * Ctot + pr.c) * L;
+        const bf16* x01 = pr.has1 ? x00 + Ctot * L : x00;
+        bf16* y0 = y + (pr.b0 * C + pr.c) * L;
+        bf16* y1 = y0 + C * L;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            if (r == 1 && !pr.has1) break;
-            const bf16* x0 = u + ((pr.b0 + r) * Ctot + pr.c) * L;
-            bf16* yr = y + ((pr.b0 + r) * C + pr.c) * L;
-            Raw8 xr[4];
+        for (int jh = 0; jh < 4; jh += 2) {
+            Raw8 xr[2][2];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) xr[jj] = load8(x0, 8 * (t + 256 * jj));
+            for (int jo = 0; jo < 2; ++jo) {
+                xr[0][jo] = load8(x00, 8 * (t + 256 * (jh + jo)));
+                xr[1][jo] = load8(x01, 8 * (t + 256 * (jh + jo)));
+            }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int n0 = 8 * (t + 256 * jj);
+            for (int jo = 0; jo < 2; ++jo) {
+                const int n0 = 8 * (t + 256 * (jh + jo));
                 const uint4 va = *reinterpret_cast<const uint4*>(Vs + n0);
                 const uint4 vb = *reinterpret_cast<const uint4*>(Vs + n0 + 4);
                 const uint32_t vw[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-                float xs[8];
-                sc8(xr[jj], t0, xs);
-                uint32_t o[4];
+                float2 xs[8];
+                sc8x2(xr[0][jo], xr[1][jo], t0, xs);
+                uint32_t o0[4], o1[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float v0 = r ? bf_hi(vw[2 * i]) : bf_lo(vw[2 * i]);
-                    const float v1 = r ? bf_hi(vw[2 * i + 1]) : bf_lo(vw[2 * i + 1]);
-                    o[i] = pack_bf16(xs[2 * i] * v0, xs[2 * i + 1] * v1);
+                    // v staging holds (row b0, row b1) per sample
+                    const float2 ya = __fmul2_rn(xs[2 * i], make_float2(bf_lo(vw[2 * i]), bf_hi(vw[2 * i])));
+                    const float2 yb = __fmul2_rn(xs[2 * i + 1], make_float2(bf_lo(vw[2 * i + 1]), bf_hi(vw[2 * i + 1])));
+                    o0[i] = pack_bf16(ya.x, yb.x);
+                    o1[i] = pack_bf16(ya.y, yb.y);
                 }
-                *reinterpret_cast<uint4*>(yr + n0) = ok ? make_uint4(o[0], o[1], o[2], o[3])   // a timed-out
-                                                        : make_uint4(0x7fc07fc0u, 0x7fc07fc0u,   // wait poisons
-                                                                     0x7fc07fc0u, 0x7fc07fc0u);  // the output
+                const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
+                // a timed-out wait poisons the output
+                *reinterpret_cast<uint4*>(y0 + n0) = ok ? make_uint4(o0[0], o0[1], o0[2], o0[3]) : nan4;
+                if (pr.has1) *reinterpret_cast<uint4*>(y1 + n0) = ok ? make_uint4(o1[0], o1[1], o1[2], o1[3]) : nan4;
             }
         }
     };
@@ -346,10 +366,10 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
         }
         // ---------------- step-1 operand: z = sc(x_{order-1}) sc(v), g[b0] + i g[b1]
         {
-            const Taps tg = load_taps(sc_w, sc_b, int64_t(order - 1) * C + c);
-            const Taps tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
+            // an odd batch's last pair has no row b1: its v taps are zero, so z = g[b0]
+            const Taps2 tg = taps2(load_taps(sc_w, sc_b, int64_t(order - 1) * C + c), 1.0f);
+            const Taps2 tv = taps2(load_taps(sc_w, sc_b, int64_t(order) * C + c), pr.has1 ? 1.0f : 0.0f);
             const int chalf = t >> 7, a0 = 8 * (t & 127);
-            const float m1 = pr.has1 ? 1.0f : 0.0f;
             // rows rho1(a0 + i) = rho1(a0) + 8 (i & 3) + (i >> 2) (a0 % 8 == 0); slots 4 chalf + j
             const int r0 = rho1(a0);
             const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
@@ -359,13 +379,14 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
 #pragma unroll
                 for (int jo = 0; jo < 2; ++jo) {
                     const int j = jp + jo;
-                    float xa[8], va[8], xb[8], vb[8];
-                    sc8(in.x[0][j], tg, xa);
-                    sc8(in.v[0][j], tv, va);
-                    sc8(in.x[1][j], tg, xb);
-                    sc8(in.v[1][j], tv, vb);
+                    float2 xs[8], vs[8];
+                    sc8x2(in.x[0][j], in.x[1][j], tg, xs);
+                    sc8x2(in.v[0][j], in.v[1][j], tv, vs);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) pk[i][jo] = pack_bf16(xa[i] * va[i], m1 * xb[i] * vb[i]);
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 z = __fmul2_rn(xs[i], vs[i]);         // (g[b0], g[b1]) = (re, im)
+                        pk[i][jo] = pack_bf16(z.x, z.y);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
