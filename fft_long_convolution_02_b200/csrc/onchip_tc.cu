@@ -353,17 +353,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
         const bf16* u0 = u + pr.b0 * Ctot * L;
         const bf16* u1 = pr.has1 ? u0 + Ctot * L : u0;
         const int64_t Pn = P + gridDim.x;
-        if (t == 0) {
-            // warm L2 with this pair's spectrum rows (plane 0) and the next pair's rows
-            for (int st = 1; st < order; ++st)
-                tc::prefetch_l2(spec + (int64_t(st - 1) * C + c) * (2 * N), N * 4);
-            if (Pn < npairs) {
-                const PairRef pn = pair_ref(Pn, B);
-                for (int r = 0; r < 2 && pn.b0 + r < B; ++r)
-                    for (int g = 0; g <= order; ++g)
-                        tc::prefetch_l2(u + ((pn.b0 + r) * Ctot + int64_t(g) * C + pn.c) * L, L * 2);
-            }
-        }
         // ---------------- step-1 operand: z = sc(x_{order-1}) sc(v), g[b0] + i g[b1]
         {
             // an odd batch's last pair has no row b1: its v taps are zero, so z = g[b0]
