@@ -26,7 +26,8 @@
 // complex pair, written in place by the spectrum build.
 //
 // Rows are processed in groups sized to the caller's workspace (default
-// about 48 MB) so the intermediate data stays in the 126 MB L2 between passes.
+// about 96 MB, chosen by timing) so that much of the intermediate data stays
+// in the 126 MB L2 between passes.
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"
@@ -36,8 +37,6 @@ namespace hyena {
 
 namespace {
 
-constexpr int kNB2 = 16;          // columns per CTA in passes A and C
-constexpr int kColThreads = 256;
 
 struct MpTables {
     const float2* fftA;     // CTA FFT of size M1
@@ -65,82 +64,6 @@ __device__ __forceinline__ int mp_slot(bool odd, int m1) {
         return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - m1) + 1;
     }
     return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - 1 - m1) + 1;
-}
-
-__device__ __forceinline__ float2 twist_of(const MpTables& tb, int n1, int n2) {
-    return cmul(__ldg(tb.twist_hi + n1), __ldg(tb.twist_lo + n2));
-}
-
-// Column block in shared memory: chain ch, column j, padded row index.
-template <int M1>
-__device__ __forceinline__ float2* col_ptr(float2* smem, int ch, int j) {
-    return smem + (ch * kNB2 + j) * fft_padded_size(M1);
-}
-
-// Forward column DFT of both chains, four-step twiddle, store to the
-// workspace (or the spectrum row when building the spectrum).
-template <int M1>
-__device__ __forceinline__ void cols_forward_store(float2* smem, const MpTables& tb, float2* __restrict__ ws_row,
-                                                   int M2, int n2_0) {
-    __syncthreads();
-    cta_fft_forward<M1>(smem, 2 * kNB2, fft_padded_size(M1), tb.fftA);
-    const int M = M1 * M2;
-    for (int idx = threadIdx.x; idx < 2 * M1 * kNB2; idx += blockDim.x) {
-        const int ch = idx / (M1 * kNB2);
-        const int rem = idx - ch * (M1 * kNB2);
-        const int m1 = rem / kNB2;
-        const int j = rem - m1 * kNB2;
-        const int n2 = n2_0 + j;
-        float2 v = col_ptr<M1>(smem, ch, j)[fft_pad(fft_bin_pos<M1>(m1))];
-        v = cmul(v, __ldg(tb.four + int64_t(m1) * M2 + n2));
-        ws_row[int64_t(ch) * M + int64_t(mp_slot<M1>(ch == 1, m1)) * M2 + n2] = v;
-    }
-}
-
-// ------------------------------------------------------------------ pass A
-// MODE 0: gated input from u (first order step); MODE 1: the filter k.
-template <int M1, typename T, int MODE>
-__global__ void __launch_bounds__(kColThreads)
-k_mp_pass_a(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, const float* __restrict__ sc_w,
-            const float* __restrict__ sc_b, int64_t B, int64_t C, int order, int M2, int64_t row0,
-            int64_t ws_row_stride) {
-    extern __shared__ float2 smem[];
-    const int64_t r = row0 + blockIdx.y;
-    const int n2_0 = blockIdx.x * kNB2;
-    const int64_t L = int64_t(2) * M1 * M2;
-    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
-    const T* xg;
-    const T* vr = nullptr;
-    Taps tg{}, tv{};
-    if (MODE == 0) {
-        const int64_t c = r / B, b = r - (r / B) * B;
-        const int64_t Ctot = int64_t(order + 1) * C;
-        const T* ub = src + b * Ctot * L;
-        const int g = order - 1;
-        xg = ub + (int64_t(g) * C + c) * L;
-        vr = ub + (int64_t(order) * C + c) * L;
-        tg = load_taps(sc_w, sc_b, int64_t(g) * C + c);
-        tv = load_taps(sc_w, sc_b, int64_t(order) * C + c);
-    } else {
-        xg = src + r * L;
-    }
-    for (int idx = threadIdx.x; idx < M1 * kNB2; idx += blockDim.x) {
-        const int n1 = idx / kNB2;
-        const int j = idx - n1 * kNB2;
-        const int n2 = n2_0 + j;
-        const int64_t t = 2 * (int64_t(M2) * n1 + n2);
-        float2 z;
-        if (MODE == 0) {
-            const float2 a = shortconv_pair(xg, t, tg);
-            const float2 v = shortconv_pair(vr, t, tv);
-            z = make_float2(a.x * v.x, a.y * v.y);
-        } else {
-            z = load2(xg + t);
-        }
-        col_ptr<M1>(smem, 0, j)[fft_pad(n1)] = z;
-        col_ptr<M1>(smem, 1, j)[fft_pad(n1)] = cmul(z, twist_of(tb, n1, n2));
-    }
-    cols_forward_store<M1>(smem, tb, ws_row, M2, n2_0);
 }
 
 // ------------------------------------------------------------------ pass B
@@ -270,69 +193,6 @@ __device__ __forceinline__ void mp_unit_generic(float2* __restrict__ ws, const f
         unit[i] = b0[fft_pad(i)];
         unit[M2 + i] = b1[fft_pad(i)];
     }
-}
-
-template <int M2, int MODE>
-__global__ void k_mp_pass_b(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1,
-                            int64_t row0, int64_t ws_row_stride, int64_t spec_row_stride4, int step,
-                            int64_t B, int64_t C, const float* __restrict__ D) {
-    extern __shared__ float2 smem[];
-    mp_unit_generic<M2, MODE>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D,
-                              int(blockIdx.x), smem);
-}
-
-// ------------------------------------------------------------------ pass C
-// FINAL: output gate x0 and store y.  Otherwise: gate with x_{gnext}, then
-// run the next step's pass A on the same columns.
-template <int M1, typename T, bool FINAL>
-__global__ void __launch_bounds__(kColThreads)
-k_mp_pass_c(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, MpTables tb,
-            const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-            int gnext, int M2, int64_t row0, int64_t ws_row_stride) {
-    extern __shared__ float2 smem[];
-    const int64_t r = row0 + blockIdx.y;
-    const int n2_0 = blockIdx.x * kNB2;
-    const int M = M1 * M2;
-    const int64_t L = int64_t(2) * M;
-    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
-    const int64_t c = r / B, b = r - (r / B) * B;
-    const int64_t Ctot = int64_t(order + 1) * C;
-    const T* ub = u + b * Ctot * L;
-    for (int idx = threadIdx.x; idx < 2 * M1 * kNB2; idx += blockDim.x) {
-        const int ch = idx / (M1 * kNB2);
-        const int rem = idx - ch * (M1 * kNB2);
-        const int m1 = rem / kNB2;
-        const int j = rem - m1 * kNB2;
-        const int n2 = n2_0 + j;
-        float2 v = ws_row[int64_t(ch) * M + int64_t(mp_slot<M1>(ch == 1, m1)) * M2 + n2];
-        v = cmulc(v, __ldg(tb.four + int64_t(m1) * M2 + n2));
-        col_ptr<M1>(smem, ch, j)[fft_pad(fft_bin_pos<M1>(m1))] = v;
-    }
-    __syncthreads();
-    cta_fft_inverse<M1>(smem, 2 * kNB2, fft_padded_size(M1), tb.fftA);
-    const int gate = FINAL ? 0 : gnext;
-    const T* xg = ub + (int64_t(gate) * C + c) * L;
-    const Taps tg = load_taps(sc_w, sc_b, int64_t(gate) * C + c);
-    T* yr = y + (b * C + c) * L;
-    for (int idx = threadIdx.x; idx < M1 * kNB2; idx += blockDim.x) {
-        const int n1 = idx / kNB2;
-        const int j = idx - n1 * kNB2;
-        const int n2 = n2_0 + j;
-        const int64_t n = int64_t(M2) * n1 + n2;
-        const float2 tw = twist_of(tb, n1, n2);
-        float2* ce = col_ptr<M1>(smem, 0, j) + fft_pad(n1);
-        float2* co = col_ptr<M1>(smem, 1, j) + fft_pad(n1);
-        const float2 zp = cadd(*ce, cmulc(*co, tw));
-        const float2 x = shortconv_pair(xg, 2 * n, tg);
-        const float2 z = make_float2(x.x * zp.x, x.y * zp.y);
-        if (FINAL) {
-            store2(yr + 2 * n, z);
-        } else {
-            *ce = z;
-            *co = cmul(z, tw);
-        }
-    }
-    if (!FINAL) cols_forward_store<M1>(smem, tb, ws_row, M2, n2_0);
 }
 
 // ===========================================================================
@@ -582,16 +442,6 @@ k_mpf_rows(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb
 template <int M2>
 constexpr int rows_nu() {
     return (M2 / 16) >= 256 ? 1 : 256 / (M2 / 16);
-}
-
-template <int M1>
-size_t col_smem() {
-    return size_t(2) * kNB2 * fft_padded_size(M1) * sizeof(float2);
-}
-
-template <int M2>
-int row_threads() {
-    return M2 >= 2048 ? 256 : (M2 >= 1024 ? 128 : 64);
 }
 
 template <int M1, int M2>
