@@ -243,6 +243,45 @@ __device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables
     }
 }
 
+// Input staging of the column passes: the CTA's columns n2_0 .. n2_0+15 of
+// every row n1 of one channel row are 32 consecutive samples from
+// 2 (M2 n1 + n2_0); they and the two samples before them (the short conv's
+// halo) are copied to shared memory with 16-byte loads.  Segment n1 sits at
+// seg + n1 kSegStride: the samples start at element 8, the halo at 6.
+constexpr int kSegStride = 40;
+
+template <int M1, typename T>
+__device__ __forceinline__ void stage_segments(const T* __restrict__ src, int M2, int n2_0, T* __restrict__ seg) {
+    constexpr int PER = 16 / int(sizeof(T));      // elements per 16-byte chunk
+    constexpr int NCH = 32 / PER;                  // chunks per segment
+    for (int idx = threadIdx.x; idx < M1 * (NCH + 1); idx += blockDim.x) {
+        const int n1 = idx / (NCH + 1), ch = idx - n1 * (NCH + 1);
+        const int64_t t0 = 2 * (int64_t(M2) * n1 + n2_0);
+        T* dst = seg + n1 * kSegStride;
+        if (ch < NCH) {
+            *reinterpret_cast<uint4*>(dst + 8 + ch * PER) = __ldg(reinterpret_cast<const uint4*>(src + t0 + ch * PER));
+        } else if (sizeof(T) == 2) {
+            *reinterpret_cast<uint32_t*>(dst + 6) = t0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(src + t0 - 2)) : 0u;
+        } else {
+            *reinterpret_cast<uint2*>(dst + 6) =
+                t0 >= 2 ? __ldg(reinterpret_cast<const uint2*>(src + t0 - 2)) : make_uint2(0u, 0u);
+        }
+    }
+}
+
+// Short conv (or the raw samples, taps off) at the two samples of column j of
+// a staged segment.
+template <typename T>
+__device__ __forceinline__ float2 seg_pair(const T* row, int j, const Taps& tp) {
+    const float2 cur = load2_shared(row + 8 + 2 * j);
+    if (!tp.on) return cur;
+    const float2 prev = load2_shared(row + 6 + 2 * j);
+    float2 r;
+    r.x = fmaf(tp.w0, prev.x, fmaf(tp.w1, prev.y, fmaf(tp.w2, cur.x, tp.b)));
+    r.y = fmaf(tp.w0, prev.y, fmaf(tp.w1, cur.x, fmaf(tp.w2, cur.y, tp.b)));
+    return r;
+}
+
 // MODE 0: gated input x_{order-1} * v from u (first order step); MODE 1: filter k.
 template <int M1, typename T, int MODE>
 __global__ void __launch_bounds__(M1, 512 / M1)
@@ -272,22 +311,27 @@ k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, 
         xg = src + r * L;
     }
     float2 x[2][16];
+    T* seg = reinterpret_cast<T*>(smem);
+    const int n2_0 = blockIdx.x * 16;
+    stage_segments<M1, T>(xg, M2, n2_0, seg);
+    __syncthreads();
+    const Taps raw{0.0f, 0.0f, 1.0f, 0.0f, false};
+#pragma unroll
+    for (int s = 0; s < 16; ++s) x[0][s] = seg_pair(seg + (g + TPT * s) * kSegStride, j, MODE == 0 ? tg : raw);
+    if (MODE == 0) {
+        __syncthreads();
+        stage_segments<M1, T>(vr, M2, n2_0, seg);
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {
+            const float2 v = seg_pair(seg + (g + TPT * s) * kSegStride, j, tv);
+            x[0][s] = make_float2(x[0][s].x * v.x, x[0][s].y * v.y);
+        }
+    }
+    __syncthreads();                                   // staging read: the FFT reuses the buffer
     const float2 tlo = __ldg(tb.twist_lo + n2);
 #pragma unroll
-    for (int s = 0; s < 16; ++s) {
-        const int n1 = g + TPT * s;
-        const int64_t tt = 2 * (int64_t(M2) * n1 + n2);
-        float2 z;
-        if (MODE == 0) {
-            const float2 a = shortconv_pair(xg, tt, tg);
-            const float2 v = shortconv_pair(vr, tt, tv);
-            z = make_float2(a.x * v.x, a.y * v.y);
-        } else {
-            z = load2(xg + tt);
-        }
-        x[0][s] = z;
-        x[1][s] = cmul(z, cmul(__ldg(tb.twist_hi + n1), tlo));
-    }
+    for (int s = 0; s < 16; ++s) x[1][s] = cmul(x[0][s], cmul(__ldg(tb.twist_hi + g + TPT * s), tlo));
     float2* const buf[2] = {smem + j * PS, smem + (16 + j) * PS};
     reg_fft_forward<M1, 2>(x, buf, g, tb.fftA);
     cols_store_ws<M1>(x, tb, ws_row, M2, n2, g);
@@ -328,6 +372,10 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
     const int gate = FINAL ? 0 : gnext;
     const T* xg = ub + (int64_t(gate) * C + c) * L;
     const Taps tg = load_taps(sc_w, sc_b, int64_t(gate) * C + c);
+    T* seg = reinterpret_cast<T*>(smem);
+    __syncthreads();                                   // the inverse FFT's exchanges are done
+    stage_segments<M1, T>(xg, M2, blockIdx.x * 16, seg);
+    __syncthreads();
     T* yr = y + (b * C + c) * L;
     const float2 tlo = __ldg(tb.twist_lo + n2);
 #pragma unroll
@@ -336,7 +384,7 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
         const int64_t n = int64_t(M2) * n1 + n2;
         const float2 tw = cmul(__ldg(tb.twist_hi + n1), tlo);
         const float2 zp = cadd(x[0][s], cmulc(x[1][s], tw));
-        const float2 a = shortconv_pair(xg, 2 * n, tg);
+        const float2 a = seg_pair(seg + n1 * kSegStride, j, tg);
         const float2 z = make_float2(a.x * zp.x, a.y * zp.y);
         if (FINAL) {
             store2(yr + 2 * n, z);
@@ -346,6 +394,7 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
         }
     }
     if (!FINAL) {
+        __syncthreads();                               // staging read: the FFT reuses the buffer
         reg_fft_forward<M1, 2>(x, buf, g, tb.fftA);
         cols_store_ws<M1>(x, tb, ws_row, M2, n2, g);
     }
