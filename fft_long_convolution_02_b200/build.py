@@ -1,7 +1,7 @@
 """Build libhyena_b200.so in-tree: nvcc for sm_100a, one object per source,
 compiled in parallel, linked with g++ against the CUDA runtime.
 
-    python -m fft_long_convolution_02_b200.build [--force] [--debug-bounds]
+    python -m fft_long_convolution_02_b200.build [--force]
 """
 from __future__ import annotations
 
@@ -51,12 +51,12 @@ def _compile(src: str, extra: list[str]) -> str:
     return obj
 
 
-def build(force: bool = False, debug_bounds: bool = False, jobs: int | None = None) -> str:
+def build(force: bool = False, jobs: int | None = None) -> str:
     """Compile every CUDA source for sm_100a and link the shared library."""
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
         return LIB
     os.makedirs(OBJ, exist_ok=True)
-    extra = ["-DHYENA_DEBUG_BOUNDS=1"] if debug_bounds else []
+    extra: list[str] = []
     srcs = [os.path.join(CSRC, s) for s in CU_SOURCES + CPP_SOURCES]
     jobs = jobs or min(len(srcs), os.cpu_count() or 4)
     with cf.ThreadPoolExecutor(jobs) as ex:
@@ -73,4 +73,4 @@ def build(force: bool = False, debug_bounds: bool = False, jobs: int | None = No
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))
+    print(build(force="--force" in sys.argv))
