@@ -237,20 +237,13 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
     from fft_long_convolution_02_b200 import binding as hb
+    from fft_long_convolution_02_b200 import dist as hd
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = hd.env_ranks()
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    hd.init("nccl", 120.0, torch.device("cuda", local))
+    barrier = hd.barrier
 
     hb.load()
     dev = torch.device("cuda", local)
@@ -302,10 +295,7 @@ def main():
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_stop)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = hd.max_over_ranks(elapsed_ms, dev)
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     u_pin = u_host.pin_memory()
@@ -327,10 +317,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = hd.max_over_ranks(e2e_ms, dev)
 
     tokens_per_step = p.B * p.n
     value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
@@ -370,6 +357,7 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
+        import torch.distributed as dist
         dist.destroy_process_group()
 
 
