@@ -251,6 +251,26 @@ __device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables
 constexpr int kSegStride = 40;
 
 template <int M1, typename T>
+constexpr size_t seg_bytes() {
+    return size_t(M1) * kSegStride * sizeof(T);
+}
+
+__device__ __forceinline__ void cp_async_bytes16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+template <int NB>
+__device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "n"(NB)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Issue (cp.async, not waited) the copies of one channel row's segments.
+template <int M1, typename T>
 __device__ __forceinline__ void stage_segments(const T* __restrict__ src, int M2, int n2_0, T* __restrict__ seg) {
     constexpr int PER = 16 / int(sizeof(T));      // elements per 16-byte chunk
     constexpr int NCH = 32 / PER;                  // chunks per segment
@@ -259,12 +279,12 @@ __device__ __forceinline__ void stage_segments(const T* __restrict__ src, int M2
         const int64_t t0 = 2 * (int64_t(M2) * n1 + n2_0);
         T* dst = seg + n1 * kSegStride;
         if (ch < NCH) {
-            *reinterpret_cast<uint4*>(dst + 8 + ch * PER) = __ldg(reinterpret_cast<const uint4*>(src + t0 + ch * PER));
-        } else if (sizeof(T) == 2) {
-            *reinterpret_cast<uint32_t*>(dst + 6) = t0 >= 2 ? __ldg(reinterpret_cast<const uint32_t*>(src + t0 - 2)) : 0u;
+            cp_async_bytes16(dst + 8 + ch * PER, src + t0 + ch * PER);
+        } else if (t0 >= 2) {
+            cp_async_small<2 * int(sizeof(T))>(dst + 6, src + t0 - 2);
         } else {
-            *reinterpret_cast<uint2*>(dst + 6) =
-                t0 >= 2 ? __ldg(reinterpret_cast<const uint2*>(src + t0 - 2)) : make_uint2(0u, 0u);
+            dst[6] = T(0.0f);
+            dst[7] = T(0.0f);
         }
     }
 }
@@ -311,20 +331,21 @@ k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, 
         xg = src + r * L;
     }
     float2 x[2][16];
-    T* seg = reinterpret_cast<T*>(smem);
+    T* seg = reinterpret_cast<T*>(smem);                  // x segments, then v segments
+    T* segv = seg + M1 * kSegStride;
     const int n2_0 = blockIdx.x * 16;
     stage_segments<M1, T>(xg, M2, n2_0, seg);
+    if (MODE == 0) stage_segments<M1, T>(vr, M2, n2_0, segv);
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
     const Taps raw{0.0f, 0.0f, 1.0f, 0.0f, false};
 #pragma unroll
-    for (int s = 0; s < 16; ++s) x[0][s] = seg_pair(seg + (g + TPT * s) * kSegStride, j, MODE == 0 ? tg : raw);
-    if (MODE == 0) {
-        __syncthreads();
-        stage_segments<M1, T>(vr, M2, n2_0, seg);
-        __syncthreads();
-#pragma unroll
-        for (int s = 0; s < 16; ++s) {
-            const float2 v = seg_pair(seg + (g + TPT * s) * kSegStride, j, tv);
+    for (int s = 0; s < 16; ++s) {
+        const int n1 = g + TPT * s;
+        x[0][s] = seg_pair(seg + n1 * kSegStride, j, MODE == 0 ? tg : raw);
+        if (MODE == 0) {
+            const float2 v = seg_pair(segv + n1 * kSegStride, j, tv);
             x[0][s] = make_float2(x[0][s].x * v.x, x[0][s].y * v.y);
         }
     }
@@ -353,6 +374,10 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
     const int64_t r = row0 + blockIdx.y;
     const int64_t L = int64_t(2) * M;
     float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    // the gate's channel row is copied (cp.async) while the inverse FFT runs;
+    // its region follows the FFT buffer
+    const int gate = FINAL ? 0 : gnext;
+    T* const seg = reinterpret_cast<T*>(smem + 32 * PS);
     float2 x[2][16];
     {
         ColTw<M1> tw(tb, M2, n2, g);
@@ -364,17 +389,17 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
             x[1][k] = cmulc(ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2], w);
         }
     }
+    {
+        const int64_t c = r / B, b = r - c * B;
+        const T* xg = u + (b * int64_t(order + 1) * C + int64_t(gate) * C + c) * L;
+        stage_segments<M1, T>(xg, M2, blockIdx.x * 16, seg);
+        cp_async_commit();
+    }
     float2* const buf[2] = {smem + j * PS, smem + (16 + j) * PS};
     reg_fft_inverse<M1, 2>(x, buf, g, tb.fftA);
-    const int64_t c = r / B, b = r - (r / B) * B;
-    const int64_t Ctot = int64_t(order + 1) * C;
-    const T* ub = u + b * Ctot * L;
-    const int gate = FINAL ? 0 : gnext;
-    const T* xg = ub + (int64_t(gate) * C + c) * L;
+    const int64_t c = r / B, b = r - c * B;
     const Taps tg = load_taps(sc_w, sc_b, int64_t(gate) * C + c);
-    T* seg = reinterpret_cast<T*>(smem);
-    __syncthreads();                                   // the inverse FFT's exchanges are done
-    stage_segments<M1, T>(xg, M2, blockIdx.x * 16, seg);
+    cp_async_wait_all();
     __syncthreads();
     T* yr = y + (b * C + c) * L;
     const float2 tlo = __ldg(tb.twist_lo + n2);
@@ -394,7 +419,7 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
         }
     }
     if (!FINAL) {
-        __syncthreads();                               // staging read: the FFT reuses the buffer
+        __syncthreads();
         reg_fft_forward<M1, 2>(x, buf, g, tb.fftA);
         cols_store_ws<M1>(x, tb, ws_row, M2, n2, g);
     }
@@ -537,29 +562,30 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const int64_t spec_stride4 = int64_t(p.spec_row_bytes / 16);
     constexpr int NU = rows_nu<M2>();
     const size_t smA = size_t(32) * fft_padded_size(M1) * sizeof(float2);
-    const size_t smB = size_t(2) * fft_padded_size(M2) * sizeof(float2);
+    const size_t smAf = smA > 2 * seg_bytes<M1, T>() ? smA : 2 * seg_bytes<M1, T>();   // x and v segments
+    const size_t smAi = smA + seg_bytes<M1, T>();                                       // FFT buffer + gate
     const size_t smR = size_t(2 * NU) * fft_padded_size(M2) * sizeof(float2);
     auto ka = k_mpf_cols_fwd<M1, T, 0>;
     auto kr = k_mpf_rows<M2, NU, 0>;
     auto kc = k_mpf_cols_inv<M1, T, true>;
     auto kca = k_mpf_cols_inv<M1, T, false>;
-    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smAf));
     cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
-    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
-    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smAi));
+    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smAi));
     const unsigned rblocks = unsigned((M1 - 1 + NU - 1) / NU);
     for (int64_t r0 = 0; r0 < rows; r0 += G) {
         const int64_t g = rows - r0 < G ? rows - r0 : G;
         const dim3 gridA(M2 / 16, unsigned(g));
-        ka<<<gridA, M1, smA, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
+        ka<<<gridA, M1, smAf, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
         for (int st = 1; st < p.order; ++st) {
             kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(a.workspace, spec, tb, M1, r0, stride,
                                                                            spec_stride4, st - 1, a.B, p.C, nullptr);
             if (st < p.order - 1) {
-                kca<<<gridA, M1, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
+                kca<<<gridA, M1, smAi, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
                                             p.order - st - 1, M2, r0, stride);
             } else {
-                kc<<<gridA, M1, smA, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2, r0,
+                kc<<<gridA, M1, smAi, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2, r0,
                                            stride);
             }
         }
