@@ -63,4 +63,21 @@ __device__ __forceinline__ float2 shortconv_pair(const T* __restrict__ x, int64_
     return r;
 }
 
+// Asynchronous global -> shared copies (cp.async): 16 bytes (L2 only), or
+// 4 / 8 bytes; src_bytes < NB fills the rest of the destination with zeros.
+__device__ __forceinline__ void cp_async_bytes16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+template <int NB>
+__device__ __forceinline__ void cp_async_small(void* dst, const void* src, int src_bytes = NB) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n" ::"r"(static_cast<unsigned>(
+                     __cvta_generic_to_shared(dst))),
+                 "l"(src), "n"(NB), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
 }  // namespace hyena

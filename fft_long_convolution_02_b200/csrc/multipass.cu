@@ -255,20 +255,6 @@ constexpr size_t seg_bytes() {
     return size_t(M1) * kSegStride * sizeof(T);
 }
 
-__device__ __forceinline__ void cp_async_bytes16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
-                 : "memory");
-}
-template <int NB>
-__device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(dst))),
-                 "l"(src), "n"(NB)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
-
 // Issue (cp.async, not waited) the copies of one channel row's segments.
 template <int M1, typename T>
 __device__ __forceinline__ void stage_segments(const T* __restrict__ src, int M2, int n2_0, T* __restrict__ seg) {

@@ -76,6 +76,53 @@ __device__ __forceinline__ void reg_stage_compute(float2 (&x)[16], int g, const 
     }
 }
 
+// The same stage on two transforms in split form (re[s] = (Re x0[s], Re x1[s]),
+// im[s] likewise): packed fp32x2 arithmetic for both at once.
+template <int M, int I, bool INV>
+__device__ __forceinline__ void reg_stage_compute2(float2 (&re)[16], float2 (&im)[16], int g,
+                                                   const float2* __restrict__ tw) {
+    using S = RegStage<M, I>;
+    if constexpr (S::R16) {
+        const float2* tws = tw + fft_stage_tw_offset(M, I);
+        const int p = g % S::P;
+        if (!INV) {
+            DFT2<16, false>::run(re, im);
+            if constexpr (S::P > 1) {
+#pragma unroll
+                for (int s = 1; s < 16; ++s) cmul_split<false>(re[s], im[s], __ldg(tws + (s - 1) * S::P + p));
+            }
+        } else {
+            if constexpr (S::P > 1) {
+#pragma unroll
+                for (int s = 1; s < 16; ++s) cmul_split<true>(re[s], im[s], __ldg(tws + (s - 1) * S::P + p));
+            }
+            DFT2<16, true>::run(re, im);
+        }
+    } else {
+        constexpr int R = S::R;
+#pragma unroll
+        for (int u = 0; u < 16 / R; ++u) {
+            float2 ar[R], ai[R];
+#pragma unroll
+            for (int k = 0; k < R; ++k) { ar[k] = re[u * R + k]; ai[k] = im[u * R + k]; }
+            DFT2<R, INV>::run(ar, ai);
+#pragma unroll
+            for (int k = 0; k < R; ++k) { re[u * R + k] = ar[k]; im[u * R + k] = ai[k]; }
+        }
+    }
+}
+
+// Complex values of two transforms <-> split form, in place:
+// (x0[s], x1[s]) <-> ((Re x0[s], Re x1[s]), (Im x0[s], Im x1[s])).
+__device__ __forceinline__ void split_pair(float2 (&x)[2][16]) {
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const float2 a = x[0][s], b = x[1][s];
+        x[0][s] = make_float2(a.x, b.x);
+        x[1][s] = make_float2(a.y, b.y);
+    }
+}
+
 // Stage I (input layout) -> stage I+1 (input layout) through shared memory.
 template <int M, int I, int NV>
 __device__ __forceinline__ void reg_exchange_fwd(float2 (&x)[NV][16], float2* const (&buf)[NV], int g) {
@@ -118,11 +165,18 @@ __device__ __forceinline__ void reg_exchange_inv(float2 (&x)[NV][16], float2* co
     __syncthreads();
 }
 
+// With NV == 2 the data are in split form (split_pair): x[0] holds the real
+// parts of both transforms, x[1] the imaginary parts; the exchanges move them
+// through buf[0] and buf[1] exactly as they would move two transforms.
 template <int M, int I, int NV>
 __device__ __forceinline__ void reg_fwd_from(float2 (&x)[NV][16], float2* const (&buf)[NV], int g,
                                              const float2* __restrict__ tw) {
+    if constexpr (NV == 2) {
+        reg_stage_compute2<M, I, false>(x[0], x[1], g, tw);
+    } else {
 #pragma unroll
-    for (int v = 0; v < NV; ++v) reg_stage_compute<M, I, false>(x[v], g, tw);
+        for (int v = 0; v < NV; ++v) reg_stage_compute<M, I, false>(x[v], g, tw);
+    }
     if constexpr (I + 1 < fft_nstages(M)) {
         reg_exchange_fwd<M, I, NV>(x, buf, g);
         reg_fwd_from<M, I + 1, NV>(x, buf, g, tw);
@@ -132,8 +186,12 @@ __device__ __forceinline__ void reg_fwd_from(float2 (&x)[NV][16], float2* const 
 template <int M, int I, int NV>
 __device__ __forceinline__ void reg_inv_from(float2 (&x)[NV][16], float2* const (&buf)[NV], int g,
                                              const float2* __restrict__ tw) {
+    if constexpr (NV == 2) {
+        reg_stage_compute2<M, I, true>(x[0], x[1], g, tw);
+    } else {
 #pragma unroll
-    for (int v = 0; v < NV; ++v) reg_stage_compute<M, I, true>(x[v], g, tw);
+        for (int v = 0; v < NV; ++v) reg_stage_compute<M, I, true>(x[v], g, tw);
+    }
     if constexpr (I > 0) {
         reg_exchange_inv<M, I - 1, NV>(x, buf, g);
         reg_inv_from<M, I - 1, NV>(x, buf, g, tw);
@@ -145,14 +203,18 @@ template <int M, int NV>
 __device__ __forceinline__ void reg_fft_forward(float2 (&x)[NV][16], float2* const (&buf)[NV], int g,
                                                 const float2* __restrict__ tw) {
     static_assert(M >= 16, "register FFT needs M >= 16");
+    if constexpr (NV == 2) split_pair(x);
     reg_fwd_from<M, 0, NV>(x, buf, g, tw);
+    if constexpr (NV == 2) split_pair(x);
 }
 
 // Inverse: positions 16 g + s -> natural order (unnormalised).
 template <int M, int NV>
 __device__ __forceinline__ void reg_fft_inverse(float2 (&x)[NV][16], float2* const (&buf)[NV], int g,
                                                 const float2* __restrict__ tw) {
+    if constexpr (NV == 2) split_pair(x);
     reg_inv_from<M, fft_nstages(M) - 1, NV>(x, buf, g, tw);
+    if constexpr (NV == 2) split_pair(x);
 }
 
 // Bin held at position pos after the forward transform (inverse of fft_bin_pos).
