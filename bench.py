@@ -106,7 +106,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -278,7 +278,13 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
+    # keep the GPU under the same load (untimed steps) for the sampler's first
+    # samples, so that the clocks it reports are the clocks under this load
+    t_load = time.perf_counter() + 0.4
+    while time.perf_counter() < t_load:
+        for _ in range(8):
+            step()
+        torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()

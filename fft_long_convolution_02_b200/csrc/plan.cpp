@@ -128,10 +128,13 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
 
 int64_t default_group_rows(const Plan& p, int64_t rows) {
     if (p.ws_row_bytes == 0) return rows;
-    // workspace in flight per group: 96 MB for the four-step path (measured on
-    // L = 2^20: 48 MB 6.86 ms, 64 MB 6.70 ms, 96 MB 6.41 ms per call; flat at
-    // L = 65536), 48 MB for the 2-D path (well inside the 126 MB L2)
-    const size_t target = (p.path == PATH_MULTIPASS_1D) ? (size_t(96) << 20) : (size_t(48) << 20);
+    // rows per workspace group: the whole batch, up to 4 GiB of workspace.
+    // Fewer, larger groups mean fewer launches and fewer partly filled last
+    // waves; measured per call on B200 (group rows: ms):
+    //   L = 2^20, B*C = 256:        12: 4.51  37: 3.91  128: 3.72  256: 3.67
+    //   L = 65536, B*C = 4096 (o3): 192: 6.58  592: 5.93  2048: 5.72  4096: 5.68
+    //   256 x 256, B*C = 512:       95: 0.76  256: 0.67  512: 0.64
+    const size_t target = size_t(4) << 30;
     int64_t g = int64_t(target / p.ws_row_bytes);
     if (g < 1) g = 1;
     if (g > rows) g = rows;
