@@ -66,6 +66,29 @@ __device__ __forceinline__ int mp_slot(bool odd, int m1) {
     return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - 1 - m1) + 1;
 }
 
+// Workspace element: complex64, or bf16 (re, im) when the operator stores
+// bf16 (the spectrum build always uses complex64 rows).
+template <typename T>
+struct WsOf {
+    using type = float2;
+};
+template <>
+struct WsOf<__nv_bfloat16> {
+    using type = __nv_bfloat162;
+};
+template <typename T, int MODE>
+struct WsSel {
+    using type = typename WsOf<T>::type;
+};
+template <typename T>
+struct WsSel<T, 1> {
+    using type = float2;
+};
+__device__ __forceinline__ float2 ws_ld(const float2* p) { return *p; }
+__device__ __forceinline__ float2 ws_ld(const __nv_bfloat162* p) { return __bfloat1622float2(*p); }
+__device__ __forceinline__ void ws_st(float2* p, float2 v) { *p = v; }
+__device__ __forceinline__ void ws_st(__nv_bfloat162* p, float2 v) { *p = __float22bfloat162_rn(v); }
+
 // ------------------------------------------------------------------ pass B
 // The pair step for one pair entry: A at bin m (row a), B at its partner.
 __device__ __forceinline__ void pair_conv(float2& A, float2& Bv, float2 w, float4 kk) {
@@ -92,8 +115,8 @@ __device__ __forceinline__ float4 pair_spec(float2 A, float2 Bv, float2 w, float
 //         and uses spectrum row (step, c).
 // MODE 1: spectrum build: workspace row i is spectrum row r = row0 + i
 //         (= step*C + c); the pair entries of K~ replace the unit in place.
-template <int M2, int MODE>
-__device__ __forceinline__ void mp_unit_generic(float2* __restrict__ ws, const float4* __restrict__ spec,
+template <int M2, int MODE, typename W>
+__device__ __forceinline__ void mp_unit_generic(W* __restrict__ ws, const float4* __restrict__ spec,
                                                 const MpTables& tb, int M1, int64_t row0, int64_t ws_row_stride,
                                                 int64_t spec_row_stride4, int step, int64_t B, int64_t C,
                                                 const float* __restrict__ D, int unit_index, float2* smem) {
@@ -104,12 +127,13 @@ __device__ __forceinline__ void mp_unit_generic(float2* __restrict__ ws, const f
     const int u = odd ? unit_index - M1 / 2 : unit_index;
     const int ra = u;                       // first row of the unit (0 for chain e unit 0)
     const int64_t r = row0 + blockIdx.y;
-    float2* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
+    static_assert(MODE == 0 || sizeof(W) == sizeof(float2), "the spectrum build writes complex64 rows");
+    W* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
     float2* b0 = smem;
     float2* b1 = smem + PS;
     for (int i = threadIdx.x; i < M2; i += blockDim.x) {
-        b0[fft_pad(i)] = unit[i];
-        b1[fft_pad(i)] = unit[M2 + i];
+        b0[fft_pad(i)] = ws_ld(unit + i);
+        b1[fft_pad(i)] = ws_ld(unit + M2 + i);
     }
     __syncthreads();
     cta_fft_forward<M2>(smem, 2, PS, tb.fftB);
@@ -190,8 +214,8 @@ __device__ __forceinline__ void mp_unit_generic(float2* __restrict__ ws, const f
     __syncthreads();
     cta_fft_inverse<M2>(smem, 2, PS, tb.fftB);
     for (int i = threadIdx.x; i < M2; i += blockDim.x) {
-        unit[i] = b0[fft_pad(i)];
-        unit[M2 + i] = b1[fft_pad(i)];
+        ws_st(unit + i, b0[fft_pad(i)]);
+        ws_st(unit + M2 + i, b1[fft_pad(i)]);
     }
 }
 
@@ -229,8 +253,8 @@ struct ColTw {
     }
 };
 
-template <int M1>
-__device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables& tb, float2* __restrict__ ws_row,
+template <int M1, typename W>
+__device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables& tb, W* __restrict__ ws_row,
                                               int M2, int n2, int g) {
     const int M = M1 * M2;
     ColTw<M1> tw(tb, M2, n2, g);
@@ -238,8 +262,8 @@ __device__ __forceinline__ void cols_store_ws(float2 (&x)[2][16], const MpTables
     for (int k = 0; k < 16; ++k) {
         const int m1 = fft_pos_bin<M1>(16 * g + k);
         const float2 w = tw.next(k);
-        ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2] = cmul(x[0][k], w);
-        ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2] = cmul(x[1][k], w);
+        ws_st(ws_row + int64_t(mp_slot<M1>(false, m1)) * M2 + n2, cmul(x[0][k], w));
+        ws_st(ws_row + M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2, cmul(x[1][k], w));
     }
 }
 
@@ -291,7 +315,8 @@ __device__ __forceinline__ float2 seg_pair(const T* row, int j, const Taps& tp) 
 // MODE 0: gated input x_{order-1} * v from u (first order step); MODE 1: filter k.
 template <int M1, typename T, int MODE>
 __global__ void __launch_bounds__(M1, 512 / M1)
-k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, const float* __restrict__ sc_w,
+k_mpf_cols_fwd(const T* __restrict__ src, typename WsSel<T, MODE>::type* __restrict__ ws, MpTables tb,
+               const float* __restrict__ sc_w,
                const float* __restrict__ sc_b, int64_t B, int64_t C, int order, int M2, int64_t row0,
                int64_t ws_row_stride) {
     extern __shared__ float2 smem[];
@@ -301,7 +326,7 @@ k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, 
     const int n2 = blockIdx.x * 16 + j;
     const int64_t r = row0 + blockIdx.y;
     const int64_t L = int64_t(2) * M1 * M2;
-    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    auto* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
     const T* xg;
     const T* vr = nullptr;
     Taps tg{}, tv{};
@@ -348,7 +373,7 @@ k_mpf_cols_fwd(const T* __restrict__ src, float2* __restrict__ ws, MpTables tb, 
 // x_{gnext} and run the next step's forward column pass in place.
 template <int M1, typename T, bool FINAL>
 __global__ void __launch_bounds__(M1, 512 / M1)
-k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, MpTables tb,
+k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::type* __restrict__ ws, MpTables tb,
                const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
                int gnext, int M2, int64_t row0, int64_t ws_row_stride) {
     extern __shared__ float2 smem[];
@@ -359,7 +384,7 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
     const int M = M1 * M2;
     const int64_t r = row0 + blockIdx.y;
     const int64_t L = int64_t(2) * M;
-    float2* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
+    auto* ws_row = ws + int64_t(blockIdx.y) * ws_row_stride;
     // the gate's channel row is copied (cp.async) while the inverse FFT runs;
     // its region follows the FFT buffer
     const int gate = FINAL ? 0 : gnext;
@@ -371,8 +396,8 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
         for (int k = 0; k < 16; ++k) {
             const int m1 = fft_pos_bin<M1>(16 * g + k);
             const float2 w = tw.next(k);
-            x[0][k] = cmulc(ws_row[int64_t(mp_slot<M1>(false, m1)) * M2 + n2], w);
-            x[1][k] = cmulc(ws_row[M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2], w);
+            x[0][k] = cmulc(ws_ld(ws_row + int64_t(mp_slot<M1>(false, m1)) * M2 + n2), w);
+            x[1][k] = cmulc(ws_ld(ws_row + M + int64_t(mp_slot<M1>(true, m1)) * M2 + n2), w);
         }
     }
     {
@@ -414,15 +439,15 @@ k_mpf_cols_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
 // Row pass over the units other than chain e unit 0.  Units are numbered
 // 0 .. M1-2: chain e units 1 .. M1/2-1, then chain o units 0 .. M1/2-1.
 // MODE 0: convolution; MODE 1: spectrum build (pair entries in [k][g] order).
-template <int M2, int NU, int MODE>
+template <int M2, int NU, int MODE, typename W>
 __global__ void __launch_bounds__(NU * (M2 / 16), 512 / (NU * (M2 / 16)) > 0 ? 512 / (NU * (M2 / 16)) : 1)
-k_mpf_rows(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1, int64_t row0,
+k_mpf_rows(W* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1, int64_t row0,
            int64_t ws_row_stride, int64_t spec_row_stride4, int step, int64_t B, int64_t C,
            const float* __restrict__ D) {
     extern __shared__ float2 smem[];
     if (blockIdx.x == gridDim.x - 1) {
         // chain e unit 0 (rows 0 and M1/2; partners inside each row, natural entry order)
-        mp_unit_generic<M2, MODE>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D, 0, smem);
+        mp_unit_generic<M2, MODE, W>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D, 0, smem);
         return;
     }
     constexpr int TPT = M2 / 16;
@@ -437,13 +462,13 @@ k_mpf_rows(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb
     const bool odd = ugc >= M1 / 2 - 1;
     const int u = odd ? ugc - (M1 / 2 - 1) : ugc + 1;
     const int ra = u;
-    float2* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
+    W* unit = ws + int64_t(blockIdx.y) * ws_row_stride + (odd ? M : 0) + int64_t(2 * u) * M2;
     float2* const buf[2] = {smem + (2 * w) * PS, smem + (2 * w + 1) * PS};
     float2 x[2][16];
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
-        x[0][s] = unit[g + TPT * s];
-        x[1][s] = unit[M2 + g + TPT * s];
+        x[0][s] = ws_ld(unit + g + TPT * s);
+        x[1][s] = ws_ld(unit + M2 + g + TPT * s);
     }
     reg_fft_forward<M2, 2>(x, buf, g, tb.fftB);
     // pair step: row b goes through shared memory to its partner thread
@@ -476,8 +501,8 @@ k_mpf_rows(float2* __restrict__ ws, const float4* __restrict__ spec, MpTables tb
         if (active) {
 #pragma unroll
             for (int s = 0; s < 16; ++s) {
-                unit[g + TPT * s] = x[0][s];
-                unit[M2 + g + TPT * s] = x[1][s];
+                ws_st(unit + g + TPT * s, x[0][s]);
+                ws_st(unit + M2 + g + TPT * s, x[1][s]);
             }
         }
     } else {
@@ -516,7 +541,7 @@ cudaError_t spectrum_mp(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     const size_t smR = size_t(2 * NU) * fft_padded_size(M2) * sizeof(float2);
     auto kaf = k_mpf_cols_fwd<M1, float, 1>;
     auto kah = k_mpf_cols_fwd<M1, __nv_bfloat16, 1>;
-    auto kr = k_mpf_rows<M2, NU, 1>;
+    auto kr = k_mpf_rows<M2, NU, 1, float2>;
     cudaFuncSetAttribute(kaf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
     cudaFuncSetAttribute(kah, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
     cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
@@ -543,8 +568,13 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const T* u = static_cast<const T*>(a.u);
     T* y = static_cast<T*>(a.y);
     const int64_t rows = a.B * p.C;
-    int64_t G = a.group_rows < 65535 ? a.group_rows : 65535;
-    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
+    // bf16 storage keeps the workspace in bf16 (re, im): rows of 2M elements
+    // of half the size, so the caller's workspace holds twice the rows
+    using W = typename WsOf<T>::type;
+    W* ws = reinterpret_cast<W*>(a.workspace);
+    const int64_t cap = int64_t(a.group_rows) * int64_t(sizeof(float2) / sizeof(W));
+    int64_t G = cap < 65535 ? cap : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));   // 2M elements
     const int64_t spec_stride4 = int64_t(p.spec_row_bytes / 16);
     constexpr int NU = rows_nu<M2>();
     const size_t smA = size_t(32) * fft_padded_size(M1) * sizeof(float2);
@@ -552,7 +582,7 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const size_t smAi = smA + seg_bytes<M1, T>();                                       // FFT buffer + gate
     const size_t smR = size_t(2 * NU) * fft_padded_size(M2) * sizeof(float2);
     auto ka = k_mpf_cols_fwd<M1, T, 0>;
-    auto kr = k_mpf_rows<M2, NU, 0>;
+    auto kr = k_mpf_rows<M2, NU, 0, W>;
     auto kc = k_mpf_cols_inv<M1, T, true>;
     auto kca = k_mpf_cols_inv<M1, T, false>;
     cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smAf));
@@ -563,15 +593,15 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     for (int64_t r0 = 0; r0 < rows; r0 += G) {
         const int64_t g = rows - r0 < G ? rows - r0 : G;
         const dim3 gridA(M2 / 16, unsigned(g));
-        ka<<<gridA, M1, smAf, s>>>(u, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
+        ka<<<gridA, M1, smAf, s>>>(u, ws, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
         for (int st = 1; st < p.order; ++st) {
-            kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(a.workspace, spec, tb, M1, r0, stride,
+            kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(ws, spec, tb, M1, r0, stride,
                                                                            spec_stride4, st - 1, a.B, p.C, nullptr);
             if (st < p.order - 1) {
-                kca<<<gridA, M1, smAi, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
+                kca<<<gridA, M1, smAi, s>>>(u, y, ws, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
                                             p.order - st - 1, M2, r0, stride);
             } else {
-                kc<<<gridA, M1, smAi, s>>>(u, y, a.workspace, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2, r0,
+                kc<<<gridA, M1, smAi, s>>>(u, y, ws, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, 0, M2, r0,
                                            stride);
             }
         }

@@ -38,6 +38,15 @@ def test_multipass_lengths_f32(orc, L):
     assert err < 1e-5
 
 
+@pytest.mark.parametrize("L", [1 << 15, 1 << 16, 1 << 17, 1 << 18, 1 << 19, 1 << 20])
+def test_multipass_lengths_bf16(orc, L):
+    """bf16 storage keeps the workspace in bf16: every (M1, M2) split of the
+    four-step path within the bf16 tolerance."""
+    p = I.WORKLOADS["dna_1m"].with_(B=2, C=1, L=L, seed=520 + L.bit_length())
+    err = _check(orc, p)
+    print(f"L={L} bf16 max row rel err {err:.3e}")
+
+
 @pytest.mark.parametrize("order", [2, 3, 4])
 def test_multipass_orders_bf16(orc, order):
     p = I.WORKLOADS["order3"].with_(B=3, C=3, L=1 << 15, order=order, sc_bias=True, seed=600 + order)
