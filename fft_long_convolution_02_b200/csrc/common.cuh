@@ -63,6 +63,30 @@ __device__ __forceinline__ float2 shortconv_pair(const T* __restrict__ x, int64_
     return r;
 }
 
+// Workspace element of the multi-pass and 2-D paths: complex64, or bf16
+// (re, im) when the operator stores bf16; WsSel<T, 1> (the spectrum build)
+// is always complex64.
+template <typename T>
+struct WsOf {
+    using type = float2;
+};
+template <>
+struct WsOf<__nv_bfloat16> {
+    using type = __nv_bfloat162;
+};
+template <typename T, int MODE>
+struct WsSel {
+    using type = typename WsOf<T>::type;
+};
+template <typename T>
+struct WsSel<T, 1> {
+    using type = float2;
+};
+__device__ __forceinline__ float2 ws_ld(const float2* p) { return *p; }
+__device__ __forceinline__ float2 ws_ld(const __nv_bfloat162* p) { return __bfloat1622float2(*p); }
+__device__ __forceinline__ void ws_st(float2* p, float2 v) { *p = v; }
+__device__ __forceinline__ void ws_st(__nv_bfloat162* p, float2 v) { *p = __float22bfloat162_rn(v); }
+
 // Asynchronous global -> shared copies (cp.async): 16 bytes (L2 only), or
 // 4 / 8 bytes; src_bytes < NB fills the rest of the destination with zeros.
 __device__ __forceinline__ void cp_async_bytes16(void* dst, const void* src) {

@@ -51,8 +51,8 @@ __device__ __forceinline__ float2* rowbuf(float2* smem, int ch, int r) {
 
 // Row forward: rows of z (already in smem at natural positions) -> DIF ->
 // untangle -> ws[fq][p0 + r] for fq in [0, W].
-template <int MW>
-__device__ __forceinline__ void rows_forward_store(float2* smem, const T2d& tb, float2* __restrict__ ws_img,
+template <int MW, typename WT>
+__device__ __forceinline__ void rows_forward_store(float2* smem, const T2d& tb, WT* __restrict__ ws_img,
                                                    int H, int p0, float dscale, float d) {
     constexpr int W = 2 * MW;
     __syncthreads();
@@ -83,15 +83,15 @@ __device__ __forceinline__ void rows_forward_store(float2* smem, const T2d& tb, 
         // dscale/d turn X2 into the stored quantity (spectrum build) or leave it
         Xf = make_float2(Xf.x * dscale + d, Xf.y * dscale);
         Xg = make_float2(Xg.x * dscale + d, Xg.y * dscale);
-        ws_img[int64_t(f) * H + p0 + r] = Xf;
-        if (g != f) ws_img[int64_t(g) * H + p0 + r] = Xg;
+        ws_st(ws_img + int64_t(f) * H + p0 + r, Xf);
+        if (g != f) ws_st(ws_img + int64_t(g) * H + p0 + r, Xg);
     }
 }
 
 // MODE 0: gated input x_{order-1} * v from u; MODE 1: the filter k.
 template <int MW, typename T, int MODE>
 __global__ void __launch_bounds__(kRowThreads)
-k_2d_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
+k_2d_rows_fwd(const T* __restrict__ src, typename WsSel<T, MODE>::type* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
               int64_t img0, int64_t ws_img_stride, int64_t ws_img_offset) {
     extern __shared__ float2 smem[];
     constexpr int W = 2 * MW;
@@ -121,21 +121,22 @@ k_2d_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64_
         rowbuf<MW>(smem, 0, r)[fft_pad(nn)] = z;
         rowbuf<MW>(smem, 1, r)[fft_pad(nn)] = cmul(z, __ldg(tb.twist_w + nn));
     }
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
+    auto* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
     rows_forward_store<MW>(smem, tb, ws_img, H, p0, 1.0f, 0.0f);
 }
 
 // Column pass.  MODE 0: convolution in place.  MODE 1: spectrum build, one
 // CTA per (step, channel) walking the bin columns in increasing order (the
 // row-pass output sits in the upper half of the channel's region).
-template <int MH, int MODE>
+template <int MH, int MODE, typename WT>
 __global__ void __launch_bounds__(kColThreads2)
-k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
+k_2d_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, const float* __restrict__ D, float s8) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(MH);
     const int64_t img = img0 + blockIdx.y;
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    static_assert(MODE == 0 || sizeof(WT) == sizeof(float2), "the spectrum build writes complex64 rows");
+    WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
     const int ncol = W + 1;
     const float2* sp = nullptr;
     float d = 0.0f;
@@ -150,11 +151,11 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
     const int per = MODE == 0 ? kCB : 1;
     for (int f0 = f_begin; f0 < f_end; f0 += per) {
         const int nc = min(per, f_end - f0);
-        const float2* src = MODE == 0 ? ws_img : ws_img + int64_t(ncol) * MH;   // spectrum build: upper half
+        const WT* src = MODE == 0 ? ws_img : ws_img + int64_t(ncol) * MH;   // spectrum build: upper half
         for (int idx = threadIdx.x; idx < nc * MH; idx += blockDim.x) {
             const int cc = idx / MH;
             const int p = idx - cc * MH;
-            const float2 v = src[int64_t(f0 + cc) * MH + p];
+            const float2 v = ws_ld(src + int64_t(f0 + cc) * MH + p);
             smem[(2 * cc) * PS + fft_pad(p)] = v;
             smem[(2 * cc + 1) * PS + fft_pad(p)] = cmul(v, __ldg(tb.twist_h + p));
         }
@@ -177,7 +178,7 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
                 const int p = idx - cc * MH;
                 const float2 e = smem[(2 * cc) * PS + fft_pad(p)];
                 const float2 o = smem[(2 * cc + 1) * PS + fft_pad(p)];
-                ws_img[int64_t(f0 + cc) * MH + p] = cadd(e, cmulc(o, __ldg(tb.twist_h + p)));
+                ws_st(ws_img + int64_t(f0 + cc) * MH + p, cadd(e, cmulc(o, __ldg(tb.twist_h + p))));
             }
         } else {
             // K~ = (X2D / 2 + D) * s8, positions in order, chain e then chain o
@@ -188,7 +189,7 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
                 const int pos = idx - ch * MH;
                 const float2 v = smem[ch * PS + fft_pad(pos)];
                 const int e = ch * MH + (pos & 15) * (MH / 16) + (pos >> 4);
-                ws_img[int64_t(f0) * (2 * MH) + e] = make_float2((0.5f * v.x + d) * s8, 0.5f * v.y * s8);
+                ws_st(ws_img + int64_t(f0) * (2 * MH) + e, make_float2((0.5f * v.x + d) * s8, 0.5f * v.y * s8));
             }
         }
         __syncthreads();
@@ -199,14 +200,14 @@ k_2d_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int 
 // next gate + next step's row forward pass.
 template <int MW, typename T, bool FINAL>
 __global__ void __launch_bounds__(kRowThreads)
-k_2d_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C,
-              int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
+k_2d_rows_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::type* __restrict__ ws, T2d tb, int64_t B,
+              int64_t C, int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
     extern __shared__ float2 smem[];
     constexpr int W = 2 * MW;
     const int64_t img = img0 + blockIdx.y;
     const int p0 = blockIdx.x * kRB;
     const int64_t n = int64_t(H) * W;
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    auto* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
     for (int idx = threadIdx.x; idx < (MW + 1) * kRB; idx += blockDim.x) {
         const int q = idx / kRB;
         const int r = idx - q * kRB;
@@ -216,8 +217,8 @@ k_2d_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ w
         const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
         const int f = odd ? 2 * j + 1 : 2 * j;
         const int g = W - f;
-        const float2 Yf = ws_img[int64_t(f) * H + p0 + r];
-        const float2 Yg = ws_img[int64_t(g) * H + p0 + r];
+        const float2 Yf = ws_ld(ws_img + int64_t(f) * H + p0 + r);
+        const float2 Yg = ws_ld(ws_img + int64_t(g) * H + p0 + r);
         const float2 w = (q == 0) ? make_float2(1.0f, 0.0f) : __ldg(tb.untw + q);
         const float2 P = cadd(Yf, cconj(Yg));
         const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
@@ -267,9 +268,9 @@ __host__ __device__ constexpr int row_stride_f() {
     return fft_padded_size(MW) | 1;   // odd stride: rows of a warp hit different banks
 }
 
-template <int MW, int FR>
+template <int MW, int FR, typename WT>
 __device__ __forceinline__ void frows_store(float2 (&x)[2][16], float2* smem, const T2d& tb,
-                                            float2* __restrict__ ws_img, int H, int p0, int r, int g) {
+                                            WT* __restrict__ ws_img, int H, int p0, int r, int g) {
     constexpr int W = 2 * MW;
     constexpr int RS = row_stride_f<MW>();
     // positions 16 g + k of both chains to shared memory
@@ -302,15 +303,15 @@ __device__ __forceinline__ void frows_store(float2 (&x)[2][16], float2* smem, co
             Xf = csub(S, T);
             Xg = cconj(cadd(S, T));
         }
-        ws_img[int64_t(f) * H + p0 + rr] = Xf;
-        if (gg != f) ws_img[int64_t(gg) * H + p0 + rr] = Xg;
+        ws_st(ws_img + int64_t(f) * H + p0 + rr, Xf);
+        if (gg != f) ws_st(ws_img + int64_t(gg) * H + p0 + rr, Xg);
     }
 }
 
 // Forward rows: MODE 0 gated x_{order-1} * v from u, MODE 1 the filter k.
 template <int MW, int FR, typename T, int MODE>
 __global__ void __launch_bounds__(FR * (MW / 16), (512 / (FR * (MW / 16))) > 0 ? 512 / (FR * (MW / 16)) : 1)
-k_2df_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
+k_2df_rows_fwd(const T* __restrict__ src, typename WsSel<T, MODE>::type* __restrict__ ws, T2d tb, int64_t B, int64_t C, int order, int H,
                int64_t img0, int64_t ws_img_stride, int64_t ws_img_offset) {
     extern __shared__ float2 smem[];
     constexpr int W = 2 * MW;
@@ -346,7 +347,7 @@ k_2df_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64
     }
     float2* const buf[2] = {smem + (0 * FR + r) * RS, smem + (1 * FR + r) * RS};
     reg_fft_forward<MW, 2>(x, buf, g, tb.fftW);
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
+    auto* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride + ws_img_offset;
     frows_store<MW, FR>(x, smem, tb, ws_img, H, p0, r, g);
 }
 
@@ -354,8 +355,8 @@ k_2df_rows_fwd(const T* __restrict__ src, float2* __restrict__ ws, T2d tb, int64
 // next step's forward rows.
 template <int MW, int FR, typename T, bool FINAL>
 __global__ void __launch_bounds__(FR * (MW / 16), (512 / (FR * (MW / 16))) > 0 ? 512 / (FR * (MW / 16)) : 1)
-k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ ws, T2d tb, int64_t B, int64_t C,
-               int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
+k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::type* __restrict__ ws, T2d tb, int64_t B,
+               int64_t C, int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
     extern __shared__ float2 smem[];
     constexpr int W = 2 * MW;
     constexpr int TPT = MW / 16;
@@ -364,7 +365,7 @@ k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
     const int64_t img = img0 + blockIdx.y;
     const int p0 = blockIdx.x * FR;
     const int64_t n = int64_t(H) * W;
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    auto* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
     for (int idx = threadIdx.x; idx < (MW + 1) * FR; idx += blockDim.x) {
         const int q = idx / FR;
         const int rr = idx - q * FR;
@@ -374,8 +375,8 @@ k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
         const int mb = odd ? (MW - 1 - j) : ((MW - j) & (MW - 1));
         const int f = odd ? 2 * j + 1 : 2 * j;
         const int gg = W - f;
-        const float2 Yf = ws_img[int64_t(f) * H + p0 + rr];
-        const float2 Yg = ws_img[int64_t(gg) * H + p0 + rr];
+        const float2 Yf = ws_ld(ws_img + int64_t(f) * H + p0 + rr);
+        const float2 Yg = ws_ld(ws_img + int64_t(gg) * H + p0 + rr);
         const float2 w = (q == 0) ? make_float2(1.0f, 0.0f) : __ldg(tb.untw + q);
         const float2 P = cadd(Yf, cconj(Yg));
         const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
@@ -419,9 +420,9 @@ k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, float2* __restrict__ 
 
 // Column pass (convolution): 2H-point FFT of each zero-padded bin column as two
 // H-point chains, times K~ (thread order), inverse, keep p < H.
-template <int MH>
+template <int MH, typename WT>
 __global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
-k_2df_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
+k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
            int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride) {
     extern __shared__ float2 smem[];
     constexpr int TPT = MH / 16;
@@ -431,14 +432,14 @@ k_2df_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int
     const int f = blockIdx.x * kFC + cc;
     const bool active = f <= W;
     const int fc = active ? f : W;
-    float2* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
     const int64_t c = img / B;
     const float2* sp = spec + (int64_t(step) * C + c) * spec_row_stride + int64_t(fc) * (2 * MH);
     float2 x[2][16];
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
         const int p = g + TPT * s;
-        const float2 v = ws_img[int64_t(fc) * MH + p];
+        const float2 v = ws_ld(ws_img + int64_t(fc) * MH + p);
         x[0][s] = v;
         x[1][s] = cmul(v, __ldg(tb.twist_h + p));
     }
@@ -454,7 +455,7 @@ k_2df_cols(float2* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int
 #pragma unroll
         for (int s = 0; s < 16; ++s) {
             const int p = g + TPT * s;
-            ws_img[int64_t(fc) * MH + p] = cadd(x[0][s], cmulc(x[1][s], __ldg(tb.twist_h + p)));
+            ws_st(ws_img + int64_t(fc) * MH + p, cadd(x[0][s], cmulc(x[1][s], __ldg(tb.twist_h + p))));
         }
     }
 }
@@ -480,7 +481,7 @@ cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
     const size_t smB = col_smem2<MH>(1);
     auto kf = k_2d_rows_fwd<MW, float, 1>;
     auto kh = k_2d_rows_fwd<MW, __nv_bfloat16, 1>;
-    auto kb = k_2d_cols<MH, 1>;
+    auto kb = k_2d_cols<MH, 1, float2>;
     cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
     cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
     cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
@@ -512,8 +513,14 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const T* u = static_cast<const T*>(a.u);
     T* y = static_cast<T*>(a.y);
     const int64_t nimg = a.B * p.C;
-    const int64_t G = a.group_rows < 65535 ? a.group_rows : 65535;
-    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));
+    // bf16 storage keeps the workspace in bf16 (re, im): images of the same
+    // element count at half the bytes, so the caller's workspace holds twice
+    // the images
+    using WT = typename WsOf<T>::type;
+    WT* ws = reinterpret_cast<WT*>(a.workspace);
+    const int64_t cap = int64_t(a.group_rows) * int64_t(sizeof(float2) / sizeof(WT));
+    const int64_t G = cap < 65535 ? cap : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));   // elements per image
     const int64_t spec_stride = int64_t(p.spec_row_bytes / sizeof(float2));
     const int H = int(p.H), W = int(p.W);
     constexpr int FR = MH < 32 ? MH : 32;   // image rows per CTA
@@ -524,26 +531,26 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const size_t smB = col_smem2<MH>(kCB);
     auto launch_cols = [&](int64_t i0, int64_t g, int st) {
         if constexpr (COLS_REG) {
-            auto kb = k_2df_cols<MH>;
+            auto kb = k_2df_cols<MH, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
             kb<<<dim3(unsigned((W + 1 + kFC - 1) / kFC), unsigned(g)), NTC, smC, s>>>(
-                a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride);
+                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride);
         } else {
-            auto kb = k_2d_cols<MH, 0>;
+            auto kb = k_2d_cols<MH, 0, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
             kb<<<dim3(unsigned((W + 1 + kCB - 1) / kCB), unsigned(g)), kColThreads2, smB, s>>>(
-                a.workspace, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f);
+                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f);
         }
     };
     auto launch_rows_fwd = [&](int64_t i0, int64_t g) {
         if constexpr (ROWS_REG && MW >= 16) {
             auto ka = k_2df_rows_fwd<MW, FR, T, 0>;
             cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
-            ka<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, a.workspace, tb, a.B, p.C, p.order, H, i0, stride, 0);
+            ka<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, ws, tb, a.B, p.C, p.order, H, i0, stride, 0);
         } else {
             auto ka = k_2d_rows_fwd<MW, T, 0>;
             cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
-            ka<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, a.workspace, tb, a.B, p.C, p.order,
+            ka<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, ws, tb, a.B, p.C, p.order,
                                                                               H, i0, stride, 0);
         }
     };
@@ -551,12 +558,12 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         if constexpr (ROWS_REG && MW >= 16) {
             auto kc = final_step ? k_2df_rows_inv<MW, FR, T, true> : k_2df_rows_inv<MW, FR, T, false>;
             cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smR));
-            kc<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, y, a.workspace, tb, a.B, p.C, p.order, gnext, H, i0,
+            kc<<<dim3(H / FR, unsigned(g)), NTR, smR, s>>>(u, y, ws, tb, a.B, p.C, p.order, gnext, H, i0,
                                                             stride);
         } else {
             auto kc = final_step ? k_2d_rows_inv<MW, T, true> : k_2d_rows_inv<MW, T, false>;
             cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
-            kc<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, y, a.workspace, tb, a.B, p.C,
+            kc<<<dim3(H / kRB, unsigned(g)), kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C,
                                                                               p.order, gnext, H, i0, stride);
         }
     };

@@ -66,29 +66,6 @@ __device__ __forceinline__ int mp_slot(bool odd, int m1) {
     return m1 < M1 / 2 ? 2 * m1 : 2 * (M1 - 1 - m1) + 1;
 }
 
-// Workspace element: complex64, or bf16 (re, im) when the operator stores
-// bf16 (the spectrum build always uses complex64 rows).
-template <typename T>
-struct WsOf {
-    using type = float2;
-};
-template <>
-struct WsOf<__nv_bfloat16> {
-    using type = __nv_bfloat162;
-};
-template <typename T, int MODE>
-struct WsSel {
-    using type = typename WsOf<T>::type;
-};
-template <typename T>
-struct WsSel<T, 1> {
-    using type = float2;
-};
-__device__ __forceinline__ float2 ws_ld(const float2* p) { return *p; }
-__device__ __forceinline__ float2 ws_ld(const __nv_bfloat162* p) { return __bfloat1622float2(*p); }
-__device__ __forceinline__ void ws_st(float2* p, float2 v) { *p = v; }
-__device__ __forceinline__ void ws_st(__nv_bfloat162* p, float2 v) { *p = __float22bfloat162_rn(v); }
-
 // ------------------------------------------------------------------ pass B
 // The pair step for one pair entry: A at bin m (row a), B at its partner.
 __device__ __forceinline__ void pair_conv(float2& A, float2& Bv, float2 w, float4 kk) {
