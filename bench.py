@@ -45,12 +45,12 @@ def load_peaks():
 
 
 def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
-    """One read of u (all order+1 chunks), one read of the stored spectra,
-    one write of y."""
+    """One read of u (all order+1 chunks), one read of the stored spectra
+    (C rows per order step, B*C with per-sample filters), one write of y."""
     es = 2 if p.dtype == "bf16" else 4
     u = p.B * p.Ctot * p.n * es
     y = p.B * p.C * p.n * es
-    spec = (p.order - 1) * p.C * spectrum_row_bytes
+    spec = (p.order - 1) * p.FC * spectrum_row_bytes
     return u + spec + y
 
 
@@ -205,6 +205,8 @@ def run_reference(args, p):
 def config_of(p):
     cfg = {"workload": p.name, "B": p.B, "C": p.C, "order": p.order,
            "shortconv": p.shortconv, "storage": p.dtype, "math": "fp32"}
+    if p.per_sample:
+        cfg["filters"] = "per-sample (one filter per (b, c) row)"
     if p.ndim == 1:
         cfg["L"] = p.L
     else:
@@ -259,16 +261,17 @@ def main():
     u = u_host.to(dev)
     D = torch.from_numpy(data["D"]).to(dev)
     sc_w = torch.from_numpy(data["sc_w"]).to(dev) if data["sc_w"] is not None else None
-    spec = torch.empty(hb.hyena_spectrum_bytes(p.C, p.shape, p.order), dtype=torch.uint8, device=dev)
+    spec = torch.empty(hb.hyena_spectrum_bytes(p.FC, p.shape, p.order), dtype=torch.uint8, device=dev)
     y = torch.empty((p.B, p.C) + p.shape, dtype=tdt, device=dev)
     wsb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, p.shape, p.order)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
     stream = torch.cuda.current_stream()
-    hb.hyena_filter_spectrum(k_dev, D, p.C, p.shape, p.order, spec, stream)
+    hb.hyena_filter_spectrum(k_dev, D, p.FC, p.shape, p.order, spec, stream)
+    conv = hb.hyena_gated_fftconv_per_sample if p.per_sample else hb.hyena_gated_fftconv
     torch.cuda.synchronize()
 
     def step(uu=None):
-        hb.hyena_gated_fftconv(u if uu is None else uu, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws,
+        conv(u if uu is None else uu, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws,
                                stream)
 
     for _ in range(args.warmup):
@@ -334,7 +337,7 @@ def main():
     avg_launch_s = float(np.mean(launch_ms)) / 1e3
     achieved = alg / avg_launch_s / 1e9
     if p.ndim == 1 and p.L == 8192:
-        kernel = "k_conv_8192_tc" if p.dtype == "bf16" else "k_conv_4096"
+        kernel = "k_conv_8192_tc" if (p.dtype == "bf16" and not p.per_sample) else "k_conv_4096"
     elif p.ndim == 1 and p.L <= 16384:
         kernel = "k_conv_onchip"
     else:

@@ -24,7 +24,7 @@ STATUS = {0: "HYENA_OK", 1: "HYENA_ERR_INVALID_ARG", 2: "HYENA_ERR_UNSUPPORTED_S
 EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "hyena_spectrum_bytes",
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
            "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
-           "hyena_spectrum_check", "hyena_debug_conv_tc"]
+           "hyena_gated_fftconv_per_sample", "hyena_spectrum_check", "hyena_debug_conv_tc"]
 
 _lock = threading.Lock()
 _lib = None
@@ -67,6 +67,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hyena_gated_fftconv.restype = ctypes.c_int
         lib.hyena_gated_fftconv.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p, ctypes.c_int,
                                             ctypes.c_int, vp, sz, vp]
+        lib.hyena_gated_fftconv_per_sample.restype = ctypes.c_int
+        lib.hyena_gated_fftconv_per_sample.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
+                                                       ctypes.c_int, ctypes.c_int, vp, sz, vp]
         lib.hyena_gated_fftconv_noalloc.restype = ctypes.c_int
         lib.hyena_gated_fftconv_noalloc.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
                                                     ctypes.c_int, ctypes.c_int, vp]
@@ -159,6 +162,18 @@ def hyena_gated_fftconv(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, or
     _check(load().hyena_gated_fftconv(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
                                       _ptr(sc_w), _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
                                       _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hyena_gated_fftconv_per_sample(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int,
+                                   workspace=None, stream=None) -> None:
+    """hyena_gated_fftconv with one filter per (b, c) row: spectrum from
+    hyena_filter_spectrum over B*C channels (k [order-1, B, C, *sizes])."""
+    arr, nd = _sizes(sizes)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyena_gated_fftconv_per_sample(_ptr(u), _ptr(y), _ptr(spectrum),
+                                                 spectrum.numel() * spectrum.element_size(), _ptr(sc_w),
+                                                 _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
+                                                 _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def hyena_gated_fftconv_noalloc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int,

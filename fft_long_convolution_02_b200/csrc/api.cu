@@ -151,10 +151,20 @@ namespace {
 // kernel arguments.
 hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, const float* sc_w,
                             const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes, int order,
-                            hyena_dtype_t dtype, void* workspace, size_t workspace_bytes, Plan* pp, ConvArgs* pa) {
+                            hyena_dtype_t dtype, void* workspace, size_t workspace_bytes, Plan* pp, ConvArgs* pa,
+                            bool per_sample = false) {
     Plan& p = *pp;
     hyena_status_t st = plan_or_fail(C, ndim, sizes, order, &p);
     if (st != HYENA_OK) return st;
+    // the spectrum holds C filters per order step, or B*C (one per (b, c) row)
+    size_t spec_total = p.total_bytes;
+    if (per_sample) {
+        Plan ps;
+        if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
+        st = plan_or_fail(B * C, ndim, sizes, order, &ps);
+        if (st != HYENA_OK) return st;
+        spec_total = ps.total_bytes;
+    }
     if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
     if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
     if (!valid_dtype(dtype)) return fail(HYENA_ERR_INVALID_ARG, "dtype must be HYENA_F32 or HYENA_BF16");
@@ -163,9 +173,10 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
         return fail(HYENA_ERR_MISALIGNED, "u, y and spectrum must be 16-byte aligned");
     if ((sc_w && !aligned4(sc_w)) || (sc_bias && !aligned4(sc_bias)))
         return fail(HYENA_ERR_MISALIGNED, "sc_w and sc_bias must be 4-byte aligned");
-    if (spectrum_bytes != p.total_bytes)
-        return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum_bytes must equal hyena_spectrum_bytes() = " +
-                                                      std::to_string(p.total_bytes));
+    if (spectrum_bytes != spec_total)
+        return fail(HYENA_ERR_SPECTRUM_MISMATCH, std::string("spectrum_bytes must equal hyena_spectrum_bytes(") +
+                                                      (per_sample ? "B*C" : "C") + ", ...) = " +
+                                                      std::to_string(spec_total));
     const size_t es = elem_size(dtype);
     const size_t ubytes = size_t(B) * size_t(order + 1) * size_t(C) * size_t(p.n) * es;
     const size_t ybytes = size_t(B) * size_t(C) * size_t(p.n) * es;
@@ -184,21 +195,19 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
     }
     *pa = ConvArgs{u, y, static_cast<const uint8_t*>(spectrum), sc_w, sc_w ? sc_bias : nullptr, B, int(dtype),
                    static_cast<float2*>(workspace), group};
+    pa->spec_C = per_sample ? B * C : C;
+    pa->spec_per_b = per_sample ? C : 0;
     return HYENA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
-                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
-                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+hyena_status_t gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, const float* sc_w,
+                             const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes, int order,
+                             hyena_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream,
+                             bool per_sample) {
     Plan p;
     ConvArgs a;
     hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype,
-                                     workspace, workspace_bytes, &p, &a);
+                                     workspace, workspace_bytes, &p, &a, per_sample);
     if (st != HYENA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
@@ -209,6 +218,26 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "gated fftconv kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                   const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                   const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    return gated_fftconv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype, workspace,
+                         workspace_bytes, stream, false);
+}
+
+hyena_status_t hyena_gated_fftconv_per_sample(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                              const float* sc_w, const float* sc_bias, int64_t B, int64_t C,
+                                              int ndim, const int64_t* sizes, int order, hyena_dtype_t dtype,
+                                              void* workspace, size_t workspace_bytes, void* stream) {
+    return gated_fftconv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype, workspace,
+                         workspace_bytes, stream, true);
 }
 
 hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,

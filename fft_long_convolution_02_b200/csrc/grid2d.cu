@@ -131,7 +131,8 @@ k_2d_rows_fwd(const T* __restrict__ src, typename WsSel<T, MODE>::type* __restri
 template <int MH, int MODE, typename WT>
 __global__ void __launch_bounds__(kColThreads2)
 k_2d_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
-          int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, const float* __restrict__ D, float s8) {
+          int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, const float* __restrict__ D, float s8,
+          int64_t SC, int64_t SB) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(MH);
     const int64_t img = img0 + blockIdx.y;
@@ -141,8 +142,8 @@ k_2d_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, i
     const float2* sp = nullptr;
     float d = 0.0f;
     if (MODE == 0) {
-        const int64_t c = img / B;
-        sp = spec + (int64_t(step) * C + c) * spec_row_stride;
+        const int64_t c = img / B, b = img - c * B;
+        sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride;
     } else {
         d = D ? __ldg(D + img) : 0.0f;
     }
@@ -423,7 +424,7 @@ k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::typ
 template <int MH, typename WT>
 __global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
 k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
-           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride) {
+           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, int64_t SC, int64_t SB) {
     extern __shared__ float2 smem[];
     constexpr int TPT = MH / 16;
     constexpr int PS = fft_padded_size(MH);
@@ -433,8 +434,8 @@ k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, 
     const bool active = f <= W;
     const int fc = active ? f : W;
     WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
-    const int64_t c = img / B;
-    const float2* sp = spec + (int64_t(step) * C + c) * spec_row_stride + int64_t(fc) * (2 * MH);
+    const int64_t c = img / B, b = img - c * B;
+    const float2* sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride + int64_t(fc) * (2 * MH);
     float2 x[2][16];
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
@@ -498,7 +499,7 @@ cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
             kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
                                                2, H, i0, stride, upper);
         kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, nullptr, tb, W, 1, p.C, 0, i0, stride,
-                                                           0, a.D, s8);
+                                                           0, a.D, s8, 0, 0);
     }
     return cudaGetLastError();
 }
@@ -534,12 +535,13 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
             auto kb = k_2df_cols<MH, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
             kb<<<dim3(unsigned((W + 1 + kFC - 1) / kFC), unsigned(g)), NTC, smC, s>>>(
-                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride);
+                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, a.spec_C, a.spec_per_b);
         } else {
             auto kb = k_2d_cols<MH, 0, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
             kb<<<dim3(unsigned((W + 1 + kCB - 1) / kCB), unsigned(g)), kColThreads2, smB, s>>>(
-                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f);
+                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f, a.spec_C,
+                a.spec_per_b);
         }
     };
     auto launch_rows_fwd = [&](int64_t i0, int64_t g) {

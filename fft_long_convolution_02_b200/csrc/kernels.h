@@ -35,6 +35,10 @@ struct ConvArgs {
     // the tensor-core work is issued (0 only from the timeout test hook)
     uint64_t wait_budget_ns = kDefaultWaitBudgetNs;
     int issue_mma = 1;
+    // spectrum row of (order step s, b, c) = s * spec_C + b * spec_per_b + c:
+    // (C, 0) for filters shared over the batch, (B*C, C) for per-sample filters
+    int64_t spec_C = 0;
+    int64_t spec_per_b = 0;
 };
 
 cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);

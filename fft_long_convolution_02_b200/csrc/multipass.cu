@@ -96,7 +96,8 @@ template <int M2, int MODE, typename W>
 __device__ __forceinline__ void mp_unit_generic(W* __restrict__ ws, const float4* __restrict__ spec,
                                                 const MpTables& tb, int M1, int64_t row0, int64_t ws_row_stride,
                                                 int64_t spec_row_stride4, int step, int64_t B, int64_t C,
-                                                const float* __restrict__ D, int unit_index, float2* smem) {
+                                                const float* __restrict__ D, int unit_index, float2* smem,
+                                                int64_t SC, int64_t SB) {
     constexpr int PS = fft_padded_size(M2);
     const int M = M1 * M2;
     const int64_t L = int64_t(2) * M;
@@ -122,8 +123,8 @@ __device__ __forceinline__ void mp_unit_generic(W* __restrict__ ws, const float4
     float d = 0.0f;
     const float s4 = 1.0f / float(4 * L);
     if (MODE == 0) {
-        const int64_t c = r / B;
-        sp = spec + (int64_t(step) * C + c) * spec_row_stride4 + (odd ? M / 2 : 0) + int64_t(u) * M2;
+        const int64_t c = r / B, b = r - c * B;
+        sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride4 + (odd ? M / 2 : 0) + int64_t(u) * M2;
     } else {
         sp_out = reinterpret_cast<float4*>(unit);   // the unit's 2*M2 complex = M2 float4 entries
         d = D ? __ldg(D + r) : 0.0f;
@@ -420,11 +421,12 @@ template <int M2, int NU, int MODE, typename W>
 __global__ void __launch_bounds__(NU * (M2 / 16), 512 / (NU * (M2 / 16)) > 0 ? 512 / (NU * (M2 / 16)) : 1)
 k_mpf_rows(W* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int M1, int64_t row0,
            int64_t ws_row_stride, int64_t spec_row_stride4, int step, int64_t B, int64_t C,
-           const float* __restrict__ D) {
+           const float* __restrict__ D, int64_t SC, int64_t SB) {
     extern __shared__ float2 smem[];
     if (blockIdx.x == gridDim.x - 1) {
         // chain e unit 0 (rows 0 and M1/2; partners inside each row, natural entry order)
-        mp_unit_generic<M2, MODE, W>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D, 0, smem);
+        mp_unit_generic<M2, MODE, W>(ws, spec, tb, M1, row0, ws_row_stride, spec_row_stride4, step, B, C, D, 0, smem,
+                                     SC, SB);
         return;
     }
     constexpr int TPT = M2 / 16;
@@ -458,8 +460,9 @@ k_mpf_rows(W* __restrict__ ws, const float4* __restrict__ spec, MpTables tb, int
     float2 wa = __ldg(tb.unt1 + ra);
     if (odd) wa = cmul(wa, __ldg(tb.unt_c));
     if (MODE == 0) {
-        const int64_t c = r / B;
-        const float4* sp = spec + (int64_t(step) * C + c) * spec_row_stride4 + (odd ? M / 2 : 0) + int64_t(u) * M2;
+        const int64_t c = r / B, b = r - c * B;
+        const float4* sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride4 + (odd ? M / 2 : 0) +
+                           int64_t(u) * M2;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const int m2 = fft_pos_bin<M2>(16 * g + k);
@@ -533,7 +536,7 @@ cudaError_t spectrum_mp(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
                                                              tb, nullptr, nullptr, 1, 1, 2, M2, r0, stride);
         // every unit; the last block of each row takes chain e unit 0
         kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(rows + r0 * stride, nullptr, tb, M1, r0,
-                                                                       stride, 0, 0, 1, p.C, a.D);
+                                                                       stride, 0, 0, 1, p.C, a.D, 0, 0);
     }
     return cudaGetLastError();
 }
@@ -573,7 +576,8 @@ cudaError_t conv_mp_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         ka<<<gridA, M1, smAf, s>>>(u, ws, tb, a.sc_w, a.sc_b, a.B, p.C, p.order, M2, r0, stride);
         for (int st = 1; st < p.order; ++st) {
             kr<<<dim3(rblocks + 1, unsigned(g)), NU * (M2 / 16), smR, s>>>(ws, spec, tb, M1, r0, stride,
-                                                                           spec_stride4, st - 1, a.B, p.C, nullptr);
+                                                                           spec_stride4, st - 1, a.B, p.C, nullptr,
+                                                                           a.spec_C, a.spec_per_b);
             if (st < p.order - 1) {
                 kca<<<gridA, M1, smAi, s>>>(u, y, ws, tb, a.sc_w, a.sc_b, a.B, p.C, p.order,
                                             p.order - st - 1, M2, r0, stride);

@@ -132,11 +132,11 @@ template <int M, typename T>
 __global__ void __launch_bounds__(onchip_threads<M>())
 k_conv_onchip(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C,
-              int order) {
+              int order, int64_t SC, int64_t SB) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(M);
     constexpr int L = 2 * M;
-    if (!header_ok(spectrum, C, L, order)) return;
+    if (!header_ok(spectrum, SC, L, order)) return;
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
     const float2* tw_fft = tables;
@@ -167,7 +167,7 @@ k_conv_onchip(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restr
         }
         __syncthreads();
         cta_fft_forward<M>(smem, 2, PS, tw_fft);
-        conv_pairs<M>(be, bo, spec + (int64_t(s - 1) * C + c) * (M + 1), untw);
+        conv_pairs<M>(be, bo, spec + (int64_t(s - 1) * SC + b * SB + c) * (M + 1), untw);
         __syncthreads();
         cta_fft_inverse<M>(smem, 2, PS, tw_fft);
         for (int n = threadIdx.x; n < M; n += blockDim.x) {
@@ -308,9 +308,9 @@ template <typename T>
 __global__ void __launch_bounds__(NT, 2)
 k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
             const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-            int64_t rows) {
+            int64_t rows, int64_t SC, int64_t SB) {
     extern __shared__ float2 smem[];
-    if (!header_ok(spectrum, C, L, order)) return;
+    if (!header_ok(spectrum, SC, L, order)) return;
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
     const float2* twist = tables + fft_tw_size(M);
@@ -412,7 +412,7 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
                 // pair step (position layout): every thread computes its own
                 // bins from its own and the partner's value; chain e first (own
                 // values in registers), then chain o (own values from O)
-                const float2* sp = reinterpret_cast<const float2*>(spec) + (int64_t(st - 1) * C + c) * (4 * M) +
+                const float2* sp = reinterpret_cast<const float2*>(spec) + (int64_t(st - 1) * SC + b * SB + c) * (4 * M) +
                                    kSpec8192Plane / 2;
                 const int lo = t & 15, hi = t >> 4;
                 const float2 we = __ldg(twist + (hi + 16 * lo));
@@ -622,7 +622,7 @@ cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     int64_t grid = int64_t(2) * sms;
     if (grid > rows) grid = rows;
     kern<<<unsigned(grid), r16::NT, smem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
-                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows);
+                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows, a.spec_C, a.spec_per_b);
     return cudaGetLastError();
 }
 
@@ -632,7 +632,8 @@ cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         // bf16 storage, order <= 3: DFT stages on the tensor cores (bf16 operands,
         // row error ~5e-3 per order step); more order steps or fp32 storage: the
         // fp32 register kernel (the bf16-operand error of 7 steps reaches 2e-2)
-        if (a.dtype != DT_F32 && p.order <= kMaxOrderTc) return launch_conv_8192_tc(p, a, s);
+        // (per-sample filters: the tensor-core kernel's two rows share one filter)
+        if (a.dtype != DT_F32 && p.order <= kMaxOrderTc && a.spec_per_b == 0) return launch_conv_8192_tc(p, a, s);
         return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : conv_4096<__nv_bfloat16>(p, a, s);
     }
     constexpr int NT = onchip_threads<M>();
@@ -642,12 +643,12 @@ cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         auto kern = k_conv_onchip<M, float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         kern<<<grid, NT, smem, s>>>(static_cast<const float*>(a.u), static_cast<float*>(a.y), a.spectrum,
-                                    a.sc_w, a.sc_b, a.B, p.C, p.order);
+                                    a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b);
     } else {
         auto kern = k_conv_onchip<M, __nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         kern<<<grid, NT, smem, s>>>(static_cast<const __nv_bfloat16*>(a.u), static_cast<__nv_bfloat16*>(a.y),
-                                    a.spectrum, a.sc_w, a.sc_b, a.B, p.C, p.order);
+                                    a.spectrum, a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b);
     }
     return cudaGetLastError();
 }

@@ -23,6 +23,8 @@ widths and lengths the pages discuss):
 * ``order3``   B=2 C=2048 L=65536 order 3, bf16.  a_c ~ U[0.5,8].
 * ``grid2d``   B=2 C=256 256x256 order 2, bf16, no short conv.
   K[c,i,j] = N(0,1) exp(-(i^2+j^2)/(2 s_c^2)), s_c ~ U[8,128].
+* ``d768_l8k_ps`` as ``d768_l8k`` with per-sample (input-dependent) filters:
+  k and D drawn for every (b, c) row, filter index b*C + c.
 
 "N(0, 1/3)" is read as variance 1/3 (standard deviation sqrt(1/3)).
 bf16 values are produced once here by round-to-nearest-even from float32,
@@ -52,6 +54,7 @@ class Problem:
     sigma: tuple = (8.0, 128.0)  # s_c range (2-D)
     u_kind: str = "normal"     # "normal" or "acgt"
     sc_bias: bool = False
+    per_sample: bool = False   # one long filter (and D) per (b, c) row
     seed: int = 20260000
 
     @property
@@ -70,6 +73,14 @@ class Problem:
     def Ctot(self) -> int:
         return (self.order + 1) * self.C
 
+    @property
+    def FC(self) -> int:
+        """Filter channels: C, or B*C with per-sample filters (index b*C + c)."""
+        return self.B * self.C if self.per_sample else self.C
+
+    def filter_index(self, b: int, c: int) -> int:
+        return b * self.C + c if self.per_sample else c
+
     def with_(self, **kw) -> "Problem":
         return replace(self, **kw)
 
@@ -85,6 +96,8 @@ WORKLOADS = {
                       decay=(0.5, 8.0), seed=20260003),
     "grid2d": Problem("grid2d", B=2, C=256, H=256, W=256, order=2, dtype="bf16",
                       shortconv=False, sigma=(8.0, 128.0), seed=20260004),
+    "d768_l8k_ps": Problem("d768_l8k_ps", B=4, C=768, L=8192, order=2, dtype="bf16",
+                           decay=(0.5, 6.0), per_sample=True, seed=20260005),
 }
 
 
@@ -156,8 +169,8 @@ def k_row(p: Problem, s: int, c: int) -> np.ndarray:
 
 
 def D_all(p: Problem) -> np.ndarray:
-    """[order-1, C] float32 skip values."""
-    return _rng(p, TAG_D).standard_normal((p.order - 1, p.C), dtype=np.float32)
+    """[order-1, FC] float32 skip values."""
+    return _rng(p, TAG_D).standard_normal((p.order - 1, p.FC), dtype=np.float32)
 
 
 def sc_w_all(p: Problem) -> np.ndarray | None:
@@ -185,10 +198,10 @@ def make_u(p: Problem) -> np.ndarray:
 
 
 def make_k(p: Problem) -> np.ndarray:
-    """Stored k: [order-1, C, *shape]."""
-    out = np.empty((p.order - 1, p.C) + p.shape, dtype=np.uint16 if p.dtype == "bf16" else np.float32)
+    """Stored k: [order-1, FC, *shape] (FC = B*C, index b*C + c, with per-sample filters)."""
+    out = np.empty((p.order - 1, p.FC) + p.shape, dtype=np.uint16 if p.dtype == "bf16" else np.float32)
     for s in range(p.order - 1):
-        for c in range(p.C):
+        for c in range(p.FC):
             out[s, c] = store(p, k_row(p, s, c)).reshape(p.shape)
     return out
 
@@ -222,15 +235,17 @@ def oracle_rows(p: Problem, rows, data: dict | None = None):
                 u_rows[i, j] = stored_values(p, data["u"][b, ch])
             else:
                 u_rows[i, j] = stored_values(p, store(p, u_row(p, b, ch, cache))).reshape(p.shape)
+        fi = p.filter_index(b, c)
         for s in range(p.order - 1):
             if data is not None:
-                k_rows[i, s] = stored_values(p, data["k"][s, c])
+                k_rows[i, s] = stored_values(p, data["k"][s, fi])
             else:
-                key = (s, c)
+                key = (s, fi)
                 if key not in kcache:
-                    kcache[key] = stored_values(p, store(p, k_row(p, s, c))).reshape(p.shape)
+                    kcache[key] = stored_values(p, store(p, k_row(p, s, fi))).reshape(p.shape)
                 k_rows[i, s] = kcache[key]
-    D_rows = D[:, rows % p.C].T.astype(np.float64)
+    fis = np.array([p.filter_index(int(r) // p.C, int(r) % p.C) for r in rows], dtype=np.int64)
+    D_rows = D[:, fis].T.astype(np.float64)
     chans = np.arange(p.order + 1)[None, :] * p.C + (rows % p.C)[:, None]
     scw_rows = None if scw is None else scw[chans].astype(np.float64)
     scb_rows = None if scb is None else scb[chans].astype(np.float64)

@@ -151,6 +151,33 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
                                    size_t workspace_bytes, void* stream);
 
 /*
+ * hyena_gated_fftconv_per_sample -- S1..S9 with one long filter per (b, c)
+ * row: input-dependent kernels.
+ *
+ * Source: [P5] 方法论 (通过寄存器与 FiLM 实现输入依赖型核: the kernel
+ * K(x) = w(c) * f_theta(c; z(x)) depends on the whole input sample, so every
+ * sample brings its own filters) and 实现 (nSubQ: the spectrum modulation
+ * applies the input-dependent kernel inside the fused FFT -> modulate -> IFFT).
+ * How the per-sample filters are generated is outside this call: they arrive
+ * as k, like the shared filters of hyena_gated_fftconv.
+ *
+ *   spectrum buffer filled by hyena_filter_spectrum(k, k_dtype, D, B*C, ...)
+ *            from k [order-1, B, C, sizes...] and D [order-1, B, C] (the
+ *            per-sample filters as B*C channels); spectrum_bytes must equal
+ *            hyena_spectrum_bytes(B*C, ndim, sizes, order).  Row (b, c) of
+ *            order step s uses filter (s, b*C + c).
+ *   everything else as hyena_gated_fftconv (same shapes, errors, workspace).
+ *
+ * The spectrum is read once per row instead of once per channel.  At L = 8192
+ * with bf16 storage this runs the fp32 register kernel (the tensor-core kernel
+ * pairs two batch rows of one channel, which needs a shared filter).
+ */
+hyena_status_t hyena_gated_fftconv_per_sample(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                              const float* sc_w, const float* sc_bias, int64_t B, int64_t C,
+                                              int ndim, const int64_t* sizes, int order, hyena_dtype_t dtype,
+                                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Size of the fixed scratch array used by hyena_gated_fftconv_noalloc (32 MiB).
  */
 #define HYENA_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -96,6 +96,11 @@ def test_validation_errors_before_launch(lib):
     assert gf(fake, fake * 4, fake * 8, n2, None, None, 1, 8, 2, s2, 2, 0, None, 0, None) == 5
     # B < 1
     assert gf(fake, fake * 4, fake * 8, nbytes, None, None, 0, 64, 1, sizes, 2, 0, None, 0, None) == 1
+    # per-sample filters: the spectrum must hold B*C rows per step
+    ps = lib.hyena_gated_fftconv_per_sample
+    assert ps(fake, fake * 4, fake * 8, nbytes, None, None, 2, 64, 1, sizes, 2, 0, None, 0, None) == 4
+    assert "B*C" in _detail(lib)
+    assert ps(fake, fake * 4, fake * 8, nbytes, None, None, 0, 64, 1, sizes, 2, 0, None, 0, None) == 1
     # filter spectrum: size mismatch and NULLs
     fs = lib.hyena_filter_spectrum
     assert fs(fake, 0, None, 64, 1, sizes, 2, fake * 8, nbytes - 16, None) == 4
