@@ -72,6 +72,8 @@ class Oracle:
         lib.oracle_fft.argtypes = [_dp, _dp, _i64, ctypes.c_int]
         lib.oracle_conv2d_direct.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
         lib.oracle_conv2d_fft.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
+        lib.oracle_conv2d_circ_direct.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
+        lib.oracle_conv2d_circ_fft.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
         lib.oracle_hyena_rows.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _dp]
@@ -123,8 +125,23 @@ class Oracle:
         self.lib.oracle_conv2d_fft(_ptr(K), float(D), _ptr(x), _ptr(out), x.shape[0], x.shape[1])
         return out
 
+    def conv2d_circ_direct(self, K, D: float, x) -> np.ndarray:
+        """Circular 2-D convolution by its direct sum ([P5] 边界处理)."""
+        K = _f64(K); x = _f64(x)
+        out = np.empty_like(x)
+        self.lib.oracle_conv2d_circ_direct(_ptr(K), float(D), _ptr(x), _ptr(out), x.shape[0], x.shape[1])
+        return out
+
+    def conv2d_circ_fft(self, K, D: float, x) -> np.ndarray:
+        """The same through an unpadded H x W radix-2 FFT."""
+        K = _f64(K); x = _f64(x)
+        out = np.empty_like(x)
+        self.lib.oracle_conv2d_circ_fft(_ptr(K), float(D), _ptr(x), _ptr(out), x.shape[0], x.shape[1])
+        return out
+
     def hyena_rows(self, u_rows, k_rows, D_rows, sc_w_rows=None, sc_b_rows=None, *,
-                   ndim: int = 1, method: int = 0, nthreads: int = 0) -> np.ndarray:
+                   ndim: int = 1, method: int = 0, nthreads: int = 0,
+                   circular: bool = False) -> np.ndarray:
         """The operator on self-contained rows.
 
         u_rows   : [R, order+1, L] (1-D) or [R, order+1, H, W] (2-D) -- chunks
@@ -133,8 +150,12 @@ class Oracle:
         D_rows   : [R, order-1]
         sc_w_rows: [R, order+1, 3] or None;  sc_b_rows: [R, order+1] or None
         method   : 1 direct sums, 2 FFT, 0 direct when small
+        circular : 2-D only: the circular (periodic) form instead of the
+                   zero-padded one
         Returns y: [R, L] or [R, H, W] in float64.
         """
+        if circular and ndim != 2:
+            raise ValueError("the circular form is 2-D")
         u_rows = _f64(u_rows); k_rows = _f64(k_rows); D_rows = _f64(D_rows)
         R, ch = u_rows.shape[0], u_rows.shape[1]
         order = ch - 1
@@ -150,8 +171,8 @@ class Oracle:
             raise ValueError("sc_w_rows must be [R, order+1, 3]")
         y = np.empty((R, H * W), dtype=np.float64)
         rc = self.lib.oracle_hyena_rows(_ptr(u_rows), _ptr(k_rows), _ptr(D_rows), _ptr(scw),
-                                        _ptr(scb), R, H, W, ndim, order, method, nthreads,
-                                        _ptr(y))
+                                        _ptr(scb), R, H, W, 3 if circular else ndim, order, method,
+                                        nthreads, _ptr(y))
         if rc != 0:
             raise ValueError("oracle_hyena_rows rejected its arguments")
         return y.reshape((R, W) if ndim == 1 else (R, H, W))
@@ -192,6 +213,14 @@ def conv2d_direct(K, D, x):
 
 def conv2d_fft(K, D, x):
     return default().conv2d_fft(K, D, x)
+
+
+def conv2d_circ_direct(K, D, x):
+    return default().conv2d_circ_direct(K, D, x)
+
+
+def conv2d_circ_fft(K, D, x):
+    return default().conv2d_circ_fft(K, D, x)
 
 
 def hyena_rows(u_rows, k_rows, D_rows, sc_w_rows=None, sc_b_rows=None, **kw):

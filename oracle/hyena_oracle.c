@@ -29,6 +29,9 @@
  *    kept, tap w[2] multiplies the current sample, w[0] the sample two back.
  *  - 2-D form: v[p][q] = sum_{i<=p, j<=q} K[i][j] w[p-i][q-j] + D w[p][q]
  *    (kernel anchored at (0,0), output cropped to [0:H, 0:W]).
+ *  - 2-D circular form ([P5] 边界处理: circular convolution for periodic
+ *    systems, no padding): v[p][q] = sum_{i<H, j<W} K[i][j]
+ *    w[(p-i) mod H][(q-j) mod W] + D w[p][q], with K on the same H x W grid.
  *
  * Every function works in double precision on exactly the values it is
  * given.  Radix-2 FFT twiddles come from cos/sin of the C library in double,
@@ -221,6 +224,49 @@ void oracle_conv2d_fft(const double *K, double D, const double *x,
 }
 
 /* ---------------------------------------------------------------------- */
+/* 2-D circular convolution ([P5] 边界处理, periodic systems).            */
+/* out[p][q] = sum_{i<H, j<W} K[i][j] x[(p-i) mod H][(q-j) mod W]         */
+/*             + D x[p][q]                                               */
+/* ---------------------------------------------------------------------- */
+void oracle_conv2d_circ_direct(const double *K, double D, const double *x,
+                               double *out, int64_t H, int64_t W)
+{
+    for (int64_t p = 0; p < H; ++p)
+        for (int64_t q = 0; q < W; ++q) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < H; ++i)
+                for (int64_t j = 0; j < W; ++j)
+                    acc += K[i * W + j] * x[((p - i + H) % H) * W + ((q - j + W) % W)];
+            out[p * W + q] = acc + D * x[p * W + q];
+        }
+}
+
+/* The same through an H x W FFT (powers of two; no padding: the DFT's own
+ * periodicity is the circular boundary). */
+void oracle_conv2d_circ_fft(const double *K, double D, const double *x,
+                            double *out, int64_t H, int64_t W)
+{
+    size_t n = (size_t)(H * W);
+    double *kr = (double *)malloc(sizeof(double) * n);
+    double *ki = (double *)calloc(n, sizeof(double));
+    double *xr = (double *)malloc(sizeof(double) * n);
+    double *xi = (double *)calloc(n, sizeof(double));
+    memcpy(kr, K, sizeof(double) * n);
+    memcpy(xr, x, sizeof(double) * n);
+    oracle_fft2(kr, ki, H, W, -1);
+    oracle_fft2(xr, xi, H, W, -1);
+    for (size_t f = 0; f < n; ++f) {
+        double a = xr[f] * kr[f] - xi[f] * ki[f];
+        double b = xr[f] * ki[f] + xi[f] * kr[f];
+        xr[f] = a; xi[f] = b;
+    }
+    oracle_fft2(xr, xi, H, W, +1);
+    double scale = 1.0 / (double)n;
+    for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale + D * x[t];
+    free(kr); free(ki); free(xr); free(xi);
+}
+
+/* ---------------------------------------------------------------------- */
 /* The Hyena operator on one (b, c) row ([P4] 二.1 forward loop).         */
 /*                                                                        */
 /* Each row is self-contained (n = L in 1-D, n = H*W in 2-D):             */
@@ -231,6 +277,7 @@ void oracle_conv2d_fft(const double *K, double D, const double *x,
 /*  scw_row: [order+1][3]  short-conv taps of the chunk channels, or NULL */
 /*  scb_row: [order+1]     short-conv bias, or NULL                       */
 /*  method : 1 direct sums, 2 FFT, 0 direct when small else FFT           */
+/*  ndim   : 1, 2 (non-circular) or 3 meaning the 2-D circular form       */
 /* Step s = 1..order-1 uses gate x_{order-s}, filter k[s-1], skip D[s-1]. */
 /* ---------------------------------------------------------------------- */
 static void hyena_row(const double *u_row, const double *k_row, const double *D_row,
@@ -261,13 +308,16 @@ static void hyena_row(const double *u_row, const double *k_row, const double *D_
         for (int64_t t = 0; t < n; ++t) w[t] = gate[t] * v[t];
         int direct = (method == 1) ||
                      (method == 0 && ((ndim == 1 && W <= 4096) ||
-                                      (ndim == 2 && H <= 64 && W <= 64)));
+                                      (ndim != 1 && H <= 64 && W <= 64)));
         if (ndim == 1) {
             if (direct) oracle_causal_conv_direct(ks, Ds, w, vn, W);
             else        oracle_causal_conv_fft(ks, Ds, w, vn, W);
-        } else {
+        } else if (ndim == 2) {
             if (direct) oracle_conv2d_direct(ks, Ds, w, vn, H, W);
             else        oracle_conv2d_fft(ks, Ds, w, vn, H, W);
+        } else {
+            if (direct) oracle_conv2d_circ_direct(ks, Ds, w, vn, H, W);
+            else        oracle_conv2d_circ_fft(ks, Ds, w, vn, H, W);
         }
         memcpy(v, vn, sizeof(double) * (size_t)n);
     }
@@ -288,9 +338,9 @@ int oracle_hyena_rows(const double *u_rows, const double *k_rows, const double *
 {
     if (!u_rows || !k_rows || !D_rows || !y || nrows < 0 || H < 1 || W < 1 || order < 2)
         return -1;
-    if (ndim != 1 && ndim != 2) return -1;
+    if (ndim != 1 && ndim != 2 && ndim != 3) return -1;
     if (ndim == 1 && H != 1) return -1;
-    if (ndim == 2 && scw_rows) return -1;
+    if (ndim != 1 && scw_rows) return -1;
     int64_t n = H * W;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);

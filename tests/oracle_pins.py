@@ -250,4 +250,82 @@ def pin_shortconv_feeds_every_chunk(orc):
     _close(y, orc.hyena_rows(us, k, D, method=1)[0], 1e-12, "per-chunk scale")
 
 
+# ------------------------------------------------- 2-D circular form ---
+# [P5] 边界处理: the circular (periodic) convolution, no padding.
+def pin_conv2d_circ_matches_numpy(orc):
+    """Direct sum and FFT form against numpy's unpadded FFT2 product (library
+    special case of circular convolution)."""
+    rng = np.random.default_rng(21)
+    for H, W in ((1, 8), (4, 4), (8, 16), (16, 8), (32, 32)):
+        K = rng.standard_normal((H, W)); x = rng.standard_normal((H, W))
+        ref = np.fft.ifft2(np.fft.fft2(K) * np.fft.fft2(x)).real + 0.7 * x
+        _close(orc.conv2d_circ_direct(K, 0.7, x), ref, 1e-11, f"direct {H}x{W}")
+        _close(orc.conv2d_circ_fft(K, 0.7, x), ref, 1e-11, f"fft {H}x{W}")
+
+
+def pin_conv2d_circ_delta_and_shift(orc):
+    """A delta at (0, 0) returns K + D delta; a cyclic shift of the input
+    shifts the output by the same amount (both the direct and the FFT form)."""
+    rng = np.random.default_rng(22)
+    H, W = 8, 16
+    K = rng.standard_normal((H, W))
+    d = np.zeros((H, W)); d[0, 0] = 1.0
+    want = K.copy(); want[0, 0] += 0.4
+    for f in (orc.conv2d_circ_direct, orc.conv2d_circ_fft):
+        _close(f(K, 0.4, d), want, 1e-12, "delta")
+        x = rng.standard_normal((H, W))
+        _close(f(K, 0.4, np.roll(x, (3, 5), axis=(0, 1))), np.roll(f(K, 0.4, x), (3, 5), axis=(0, 1)),
+               1e-11, "shift")
+
+
+def pin_conv2d_circ_without_wrap_is_linear(orc):
+    """Kernel and input supported in the top-left quarter never wrap, so the
+    circular form equals the zero-padded (non-circular) one; the whole
+    operator too."""
+    rng = np.random.default_rng(23)
+    H, W = 16, 32
+    K = np.zeros((H, W)); K[: H // 2, : W // 2] = rng.standard_normal((H // 2, W // 2))
+    x = np.zeros((H, W)); x[: H // 2, : W // 2] = rng.standard_normal((H // 2, W // 2))
+    _close(orc.conv2d_circ_direct(K, 0.3, x), orc.conv2d_direct(K, 0.3, x), 1e-12, "conv")
+    u = np.zeros((2, 3, H, W)); u[:, :, : H // 2, : W // 2] = rng.standard_normal((2, 3, H // 2, W // 2))
+    k = np.zeros((2, 1, H, W)); k[:, :, : H // 2, : W // 2] = rng.standard_normal((2, 1, H // 2, W // 2))
+    D = rng.standard_normal((2, 1))
+    _close(orc.hyena_rows(u, k, D, ndim=2, method=1, circular=True), orc.hyena_rows(u, k, D, ndim=2, method=1),
+           1e-12, "operator")
+    _close(orc.hyena_rows(u, k, D, ndim=2, method=2, circular=True), orc.hyena_rows(u, k, D, ndim=2, method=1),
+           1e-11, "operator fft")
+
+
+def pin_operator2d_circ_direct_equals_fft_and_numpy(orc):
+    """The circular operator (order 2, full-support data that wraps): direct
+    sums equal the FFT form, and both equal gating around numpy's circular
+    FFT2 product."""
+    rng = np.random.default_rng(25)
+    H, W = 8, 16
+    u = rng.standard_normal((3, 3, H, W)); k = rng.standard_normal((3, 1, H, W))
+    D = rng.standard_normal((3, 1))
+    yd = orc.hyena_rows(u, k, D, ndim=2, method=1, circular=True)
+    yf = orc.hyena_rows(u, k, D, ndim=2, method=2, circular=True)
+    _close(yd, yf, 1e-11, "direct vs fft")
+    for r in range(3):
+        w = u[r, 1] * u[r, 2]
+        v = np.fft.ifft2(np.fft.fft2(k[r, 0]) * np.fft.fft2(w)).real + D[r, 0] * w
+        _close(yd[r], u[r, 0] * v, 1e-11, "numpy composition")
+
+
+def pin_operator2d_circ_wraps(orc):
+    """With a kernel at the last row and column only, the circular operator
+    differs from the padded one exactly by the wrapped terms: the padded form
+    sees K[H-1][W-1] only at (H-1, W-1), the circular one at every output."""
+    rng = np.random.default_rng(24)
+    H, W = 8, 8
+    K = np.zeros((H, W)); K[H - 1, W - 1] = 2.0
+    x = rng.standard_normal((H, W))
+    circ = orc.conv2d_circ_direct(K, 0.0, x)
+    _close(circ, 2.0 * np.roll(x, (H - 1, W - 1), axis=(0, 1)), 1e-12, "wrapped shift")
+    lin = orc.conv2d_direct(K, 0.0, x)
+    want = np.zeros((H, W)); want[H - 1, W - 1] = 2.0 * x[0, 0]
+    _close(lin, want, 1e-12, "padded")
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

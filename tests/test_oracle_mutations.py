@@ -38,6 +38,12 @@ MUTATIONS = {
     "output gated by x1": ("for (int64_t t = 0; t < n; ++t) y_row[t] = x[t] * v[t];",
                            "for (int64_t t = 0; t < n; ++t) y_row[t] = x[n + t] * v[t];"),
     "value chunk taken first": ("double *v = x + (int64_t)order * n;", "double *v = x;"),
+    "2-D circular index not wrapped": ("acc += K[i * W + j] * x[((p - i + H) % H) * W + ((q - j + W) % W)];",
+                                       "acc += K[i * W + j] * x[((p + i) % H) * W + ((q + j) % W)];"),
+    "2-D circular fft skip dropped": ("for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale + D * x[t];",
+                                      "for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale;"),
+    "2-D circular form runs padded": ("if (direct) oracle_conv2d_circ_direct(ks, Ds, w, vn, H, W);",
+                                      "if (direct) oracle_conv2d_direct(ks, Ds, w, vn, H, W);"),
 }
 
 
