@@ -57,7 +57,7 @@ def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
 def spectrum_row_bytes(p) -> int:
     """Spectrum bytes per (step, channel) row the convolution kernel reads."""
     if p.ndim == 2:
-        return (p.W + 1) * 2 * p.H * 8
+        return (p.W // 2 + 1) * p.H * 8 if p.circular else (p.W + 1) * 2 * p.H * 8
     if p.L == 8192:
         return 8 * p.L                      # one plane: bf16 2L bins, or fp32 position layout
     if p.L <= 16384:
@@ -151,7 +151,7 @@ def cpu_baseline(p, budget_s: float = 15.0):
     rows = rng.choice(p.B * p.C, size=min(p.B * p.C, 8 * cores), replace=False)
     args = I.oracle_rows(p, rows)
     t0 = time.perf_counter()
-    orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores)
+    orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
     dt = time.perf_counter() - t0
     # grow the sample to use about budget_s of CPU time
     n_more = int(len(rows) * max(0.0, budget_s / max(dt, 1e-3) - 1.0))
@@ -161,7 +161,7 @@ def cpu_baseline(p, budget_s: float = 15.0):
         rows2 = rng.choice(p.B * p.C, size=n_more, replace=False)
         args = I.oracle_rows(p, rows2)
         t0 = time.perf_counter()
-        orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores)
+        orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
         total_t += time.perf_counter() - t0
         total_rows += n_more
     # a row is one (b, c) pair; the operator's tokens are B*n over all C channels
@@ -184,10 +184,10 @@ def run_reference(args, p):
     samples = [I.oracle_rows(p, rng.choice(p.B * p.C, size=per_step, replace=False))
                for _ in range(args.warmup + args.steps)]
     for a in samples[:args.warmup]:
-        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores)
+        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
     t0 = time.perf_counter()
     for a in samples[args.warmup:]:
-        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores)
+        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
     dt = time.perf_counter() - t0
     tok_s = args.steps * per_step * p.n / (p.C * dt)
     line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
@@ -207,6 +207,8 @@ def config_of(p):
            "shortconv": p.shortconv, "storage": p.dtype, "math": "fp32"}
     if p.per_sample:
         cfg["filters"] = "per-sample (one filter per (b, c) row)"
+    if p.circular:
+        cfg["boundary"] = "circular"
     if p.ndim == 1:
         cfg["L"] = p.L
     else:
@@ -261,17 +263,18 @@ def main():
     u = u_host.to(dev)
     D = torch.from_numpy(data["D"]).to(dev)
     sc_w = torch.from_numpy(data["sc_w"]).to(dev) if data["sc_w"] is not None else None
-    spec = torch.empty(hb.hyena_spectrum_bytes(p.FC, p.shape, p.order), dtype=torch.uint8, device=dev)
+    shape = hb.Circular(p.shape) if p.circular else p.shape      # the ABI's shape argument
+    spec = torch.empty(hb.hyena_spectrum_bytes(p.FC, shape, p.order), dtype=torch.uint8, device=dev)
     y = torch.empty((p.B, p.C) + p.shape, dtype=tdt, device=dev)
-    wsb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, p.shape, p.order)
+    wsb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, shape, p.order)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
     stream = torch.cuda.current_stream()
-    hb.hyena_filter_spectrum(k_dev, D, p.FC, p.shape, p.order, spec, stream)
+    hb.hyena_filter_spectrum(k_dev, D, p.FC, shape, p.order, spec, stream)
     conv = hb.hyena_gated_fftconv_per_sample if p.per_sample else hb.hyena_gated_fftconv
     torch.cuda.synchronize()
 
     def step(uu=None):
-        conv(u if uu is None else uu, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws,
+        conv(u if uu is None else uu, y, spec, sc_w, None, p.B, p.C, shape, p.order, ws,
                                stream)
 
     for _ in range(args.warmup):

@@ -82,9 +82,23 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     return _lib
 
 
+HYENA_CIRCULAR = 0x100   # include/hyena.h: OR-ed into ndim for the circular 2-D form
+
+
+class Circular(tuple):
+    """sizes (H, W) of the circular (periodic) 2-D form: pass Circular((H, W))
+    wherever a shape is taken."""
+
+
 def _sizes(sizes):
+    circ = isinstance(sizes, Circular)
     sizes = [int(s) for s in sizes]
-    return (ctypes.c_int64 * len(sizes))(*sizes), len(sizes)
+    nd = len(sizes)
+    if circ:
+        if nd != 2:
+            raise ValueError("the circular form is 2-D")
+        nd |= HYENA_CIRCULAR
+    return (ctypes.c_int64 * len(sizes))(*sizes), nd
 
 
 def _ptr(x):

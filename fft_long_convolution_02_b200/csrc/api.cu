@@ -42,11 +42,15 @@ hyena_status_t cuda_status(cudaError_t e, const char* what) {
     return fail(HYENA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
+
+// 1, 2, or 2 | HYENA_CIRCULAR (the circular 2-D form)
+bool valid_ndim(int ndim) { return ndim == 1 || ndim == 2 || ndim == (2 | kCircularFlag); }
+
 hyena_status_t plan_or_fail(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p) {
     std::string why;
     if (C < 1) return fail(HYENA_ERR_INVALID_ARG, "C must be >= 1");
     if (!sizes) return fail(HYENA_ERR_INVALID_ARG, "sizes is NULL");
-    if (ndim != 1 && ndim != 2) return fail(HYENA_ERR_INVALID_ARG, "ndim must be 1 or 2");
+    if (!valid_ndim(ndim)) return fail(HYENA_ERR_INVALID_ARG, "ndim must be 1, 2 or 2 | HYENA_CIRCULAR");
     if (!make_plan(C, ndim, sizes, order, p, &why)) return fail(HYENA_ERR_UNSUPPORTED_SHAPE, why);
     return HYENA_OK;
 }
@@ -83,7 +87,7 @@ const char* hyena_last_error_detail(void) { return g_detail.c_str(); }
 size_t hyena_spectrum_bytes(int64_t C, int ndim, const int64_t* sizes, int order) {
     Plan p;
     std::string why;
-    if (!sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    if (!sizes || !valid_ndim(ndim) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
     return p.total_bytes;
 }
 
@@ -108,7 +112,8 @@ hyena_status_t hyena_filter_spectrum(const void* k, hyena_dtype_t k_dtype, const
     switch (p.path) {
         case PATH_ONCHIP_1D: e = launch_spectrum_onchip(p, a, s); break;
         case PATH_MULTIPASS_1D: e = launch_spectrum_multipass(p, a, s); break;
-        case PATH_GRID_2D: e = launch_spectrum_2d(p, a, s); break;
+        case PATH_GRID_2D:
+        case PATH_GRID_2D_CIRC: e = launch_spectrum_2d(p, a, s); break;
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "spectrum kernel");
@@ -132,14 +137,14 @@ hyena_status_t hyena_shortconv(const void* u, void* out, const float* w, const f
 size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_t* sizes, int order) {
     Plan p;
     std::string why;
-    if (!sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    if (!sizes || !valid_ndim(ndim) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
     return p.ws_row_bytes;
 }
 
 size_t hyena_gated_fftconv_workspace_bytes(int64_t B, int64_t C, int ndim, const int64_t* sizes, int order) {
     Plan p;
     std::string why;
-    if (B < 1 || !sizes || (ndim != 1 && ndim != 2) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
+    if (B < 1 || !sizes || !valid_ndim(ndim) || !make_plan(C, ndim, sizes, order, &p, &why)) return 0;
     return size_t(default_group_rows(p, B * C)) * p.ws_row_bytes;
 }
 
@@ -168,7 +173,7 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
     if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
     if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
     if (!valid_dtype(dtype)) return fail(HYENA_ERR_INVALID_ARG, "dtype must be HYENA_F32 or HYENA_BF16");
-    if (ndim == 2 && sc_w) return fail(HYENA_ERR_INVALID_ARG, "the 2-D form has no short conv: sc_w must be NULL");
+    if (ndim != 1 && sc_w) return fail(HYENA_ERR_INVALID_ARG, "the 2-D form has no short conv: sc_w must be NULL");
     if (!aligned16(u) || !aligned16(y) || !aligned16(spectrum))
         return fail(HYENA_ERR_MISALIGNED, "u, y and spectrum must be 16-byte aligned");
     if ((sc_w && !aligned4(sc_w)) || (sc_bias && !aligned4(sc_bias)))
@@ -214,7 +219,8 @@ hyena_status_t gated_fftconv(const void* u, void* y, const void* spectrum, size_
     switch (p.path) {
         case PATH_ONCHIP_1D: e = launch_conv_onchip(p, a, s); break;
         case PATH_MULTIPASS_1D: e = launch_conv_multipass(p, a, s); break;
-        case PATH_GRID_2D: e = launch_conv_2d(p, a, s); break;
+        case PATH_GRID_2D:
+        case PATH_GRID_2D_CIRC: e = launch_conv_2d(p, a, s); break;
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "gated fftconv kernel");

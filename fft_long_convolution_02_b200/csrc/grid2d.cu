@@ -1,4 +1,5 @@
-// grid2d.cu -- the 2-D non-circular form (H x W grids, 16..512 each).
+// grid2d.cu -- the 2-D forms (H x W grids, 16..512 each): non-circular
+// (zero padded) and, further down, circular.
 //
 // [P5] "Native Multi-Dimensional Subquadratic Operators via Input Dependent
 // Long Convolutions", 方法论 (原生 ND 卷积, 边界处理): the global convolution
@@ -461,6 +462,191 @@ k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, 
     }
 }
 
+// ===========================================================================
+// Circular form ([P5] 边界处理: circular convolution for periodic systems):
+// no padding, so each axis is its own DFT length.  The W-point real FFT of a
+// row is the packed W/2-point complex FFT untangled: exactly the chain e of
+// the padded row pass (its even bins), giving bins k = 0..W/2 (W/2+1 columns
+// of H values).  Each column then takes one H-point chain: forward, times K~,
+// inverse.  K~[kh][kw] = (DFT_HxW(k)[kh][kw] + D) / (2 H W), per channel
+// [kw][position] with the H positions in the register column pass's thread
+// order.
+// ===========================================================================
+
+// Row forward, circular: rows of z (chain e slots of the CTA's row buffers)
+// -> packed FFT -> untangle -> ws[k][p0 + r], k = 0..W/2.
+template <int MW, typename WT>
+__device__ __forceinline__ void rowsc_forward_store(float2* smem, const T2d& tb, WT* __restrict__ ws_img, int H,
+                                                    int p0) {
+    __syncthreads();
+    cta_fft_forward<MW>(smem, kRB, fft_padded_size(MW), tb.fftW);
+    for (int idx = threadIdx.x; idx < (MW / 2 + 1) * kRB; idx += blockDim.x) {
+        const int j = idx / kRB;
+        const int r = idx - j * kRB;
+        const float2* buf = rowbuf<MW>(smem, 0, r);
+        const float2 A = buf[fft_pad(fft_bin_pos<MW>(j))];
+        const float2 B = buf[fft_pad(fft_bin_pos<MW>((MW - j) & (MW - 1)))];
+        float2 Xf, Xg;
+        if (j == 0) {
+            Xf = make_float2(2.0f * (A.x + A.y), 0.0f);
+            Xg = make_float2(2.0f * (A.x - A.y), 0.0f);
+        } else {
+            const float2 w = __ldg(tb.untw + j);   // w_W^j
+            const float2 S = cadd(A, cconj(B));
+            const float2 T = cmul_i(cmul(w, csub(A, cconj(B))));
+            Xf = csub(S, T);
+            Xg = cconj(cadd(S, T));
+        }
+        ws_st(ws_img + int64_t(j) * H + p0 + r, Xf);
+        if (MW - j != j) ws_st(ws_img + int64_t(MW - j) * H + p0 + r, Xg);
+    }
+}
+
+// MODE 0: gated input x_{order-1} * v from u; MODE 1: the filter k.
+template <int MW, typename T, int MODE>
+__global__ void __launch_bounds__(kRowThreads)
+k_2dc_rows_fwd(const T* __restrict__ src, typename WsSel<T, MODE>::type* __restrict__ ws, T2d tb, int64_t B,
+               int64_t C, int order, int H, int64_t img0, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * kRB;
+    const int64_t n = int64_t(H) * W;
+    const T* xg;
+    const T* vr = nullptr;
+    if (MODE == 0) {
+        const int64_t c = img / B, b = img - (img / B) * B;
+        const int64_t Ctot = int64_t(order + 1) * C;
+        const T* ub = src + b * Ctot * n;
+        xg = ub + (int64_t(order - 1) * C + c) * n;
+        vr = ub + (int64_t(order) * C + c) * n;
+    } else {
+        xg = src + img * n;
+    }
+    for (int idx = threadIdx.x; idx < kRB * MW; idx += blockDim.x) {
+        const int r = idx / MW;
+        const int nn = idx - r * MW;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        float2 z = load2(xg + off);
+        if (MODE == 0) {
+            const float2 v = load2(vr + off);
+            z = make_float2(z.x * v.x, z.y * v.y);
+        }
+        rowbuf<MW>(smem, 0, r)[fft_pad(nn)] = z;
+    }
+    rowsc_forward_store<MW>(smem, tb, ws + int64_t(blockIdx.y) * ws_img_stride, H, p0);
+}
+
+// Row inverse, circular: re-tangle, inverse packed FFT, output gate (FINAL)
+// or next gate + next step's row forward pass.
+template <int MW, typename T, bool FINAL>
+__global__ void __launch_bounds__(kRowThreads)
+k_2dc_rows_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::type* __restrict__ ws, T2d tb,
+               int64_t B, int64_t C, int order, int gnext, int H, int64_t img0, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int W = 2 * MW;
+    const int64_t img = img0 + blockIdx.y;
+    const int p0 = blockIdx.x * kRB;
+    const int64_t n = int64_t(H) * W;
+    auto* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    for (int idx = threadIdx.x; idx < (MW / 2 + 1) * kRB; idx += blockDim.x) {
+        const int j = idx / kRB;
+        const int r = idx - j * kRB;
+        float2* buf = rowbuf<MW>(smem, 0, r);
+        const int mb = (MW - j) & (MW - 1);
+        const float2 Yf = ws_ld(ws_img + int64_t(j) * H + p0 + r);
+        const float2 Yg = ws_ld(ws_img + int64_t(MW - j) * H + p0 + r);
+        const float2 w = (j == 0) ? make_float2(1.0f, 0.0f) : __ldg(tb.untw + j);
+        const float2 P = cadd(Yf, cconj(Yg));
+        const float2 U = cmul_i(cmulc(csub(Yf, cconj(Yg)), w));
+        buf[fft_pad(fft_bin_pos<MW>(j))] = cadd(P, U);
+        if (j != 0) buf[fft_pad(fft_bin_pos<MW>(mb))] = cconj(csub(P, U));
+    }
+    __syncthreads();
+    cta_fft_inverse<MW>(smem, kRB, fft_padded_size(MW), tb.fftW);
+    const int64_t c = img / B, b = img - (img / B) * B;
+    const int64_t Ctot = int64_t(order + 1) * C;
+    const T* ub = u + b * Ctot * n;
+    const int gate = FINAL ? 0 : gnext;
+    const T* xg = ub + (int64_t(gate) * C + c) * n;
+    T* yr = y + (b * C + c) * n;
+    for (int idx = threadIdx.x; idx < kRB * MW; idx += blockDim.x) {
+        const int r = idx / MW;
+        const int nn = idx - r * MW;
+        const int64_t off = int64_t(p0 + r) * W + 2 * nn;
+        float2* e = rowbuf<MW>(smem, 0, r) + fft_pad(nn);
+        const float2 x = load2(xg + off);
+        const float2 z = make_float2(x.x * e->x, x.y * e->y);
+        if (FINAL) store2(yr + off, z);
+        else *e = z;
+    }
+    if (!FINAL) rowsc_forward_store<MW>(smem, tb, ws_img, H, p0);
+}
+
+// Column pass, circular (convolution): thread group cc of the CTA takes the
+// two bin columns fa = 2 (blockIdx.x kFC + cc) and fa + 1 as its two register
+// transforms: H-point forward, times K~ (thread order), inverse.
+template <int MH, typename WT>
+__global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
+k_2dc_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int ncol, int64_t B, int step,
+           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, int64_t SC, int64_t SB) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = MH / 16;
+    constexpr int PS = fft_padded_size(MH);
+    const int t = threadIdx.x, cc = t / TPT, g = t - (t / TPT) * TPT;
+    const int64_t img = img0 + blockIdx.y;
+    const int fa = 2 * (int(blockIdx.x) * kFC + cc);
+    const int f[2] = {fa < ncol ? fa : ncol - 1, fa + 1 < ncol ? fa + 1 : ncol - 1};
+    WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    const int64_t c = img / B, b = img - c * B;
+    const float2* sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride;
+    float2 x[2][16];
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+#pragma unroll
+        for (int s = 0; s < 16; ++s) x[v][s] = ws_ld(ws_img + int64_t(f[v]) * MH + g + TPT * s);
+    }
+    float2* const buf[2] = {smem + (2 * cc) * PS, smem + (2 * cc + 1) * PS};
+    reg_fft_forward<MH, 2>(x, buf, g, tb.fftH);
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[v][k] = cmul(x[v][k], __ldg(sp + int64_t(f[v]) * MH + k * TPT + g));
+    }
+    reg_fft_inverse<MH, 2>(x, buf, g, tb.fftH);
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+        if (fa + v < ncol) {
+#pragma unroll
+            for (int s = 0; s < 16; ++s) ws_st(ws_img + int64_t(f[v]) * MH + g + TPT * s, x[v][s]);
+        }
+    }
+}
+
+// Spectrum build, circular: one CTA per (step, channel) walks the W/2+1 bin
+// columns of the row-pass output in place: H-point forward FFT, then
+// K~ = (X / 2 + D) / (2 H W) in the column pass's thread order.
+template <int MH>
+__global__ void __launch_bounds__(kColThreads2)
+k_2dc_cols_spec(float2* __restrict__ rows, T2d tb, int ncol, int64_t row0, int64_t row_stride,
+                const float* __restrict__ D, float s2) {
+    extern __shared__ float2 smem[];
+    const int64_t r = row0 + blockIdx.y;
+    float2* img = rows + int64_t(blockIdx.y) * row_stride;
+    const float d = D ? __ldg(D + r) : 0.0f;
+    for (int f = 0; f < ncol; ++f) {
+        for (int p = threadIdx.x; p < MH; p += blockDim.x) smem[fft_pad(p)] = img[int64_t(f) * MH + p];
+        __syncthreads();
+        cta_fft_forward<MH>(smem, 1, fft_padded_size(MH), tb.fftH);
+        for (int pos = threadIdx.x; pos < MH; pos += blockDim.x) {
+            const float2 v = smem[fft_pad(pos)];
+            const int e = (pos & 15) * (MH / 16) + (pos >> 4);
+            img[int64_t(f) * MH + e] = make_float2((0.5f * v.x + d) * s2, 0.5f * v.y * s2);
+        }
+        __syncthreads();
+    }
+}
+
 template <int MW>
 size_t row_smem() {
     return size_t(2) * kRB * fft_padded_size(MW) * sizeof(float2);
@@ -580,6 +766,79 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <int MW, int MH>
+cudaError_t spectrum_2dc_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    float2* rows = reinterpret_cast<float2*>(a.spectrum + p.spec_off);
+    const int64_t nimg = (p.order - 1) * p.C;
+    const int64_t stride = int64_t(p.spec_row_bytes / sizeof(float2));    // (W/2+1) * H
+    const int H = int(p.H), W = int(p.W);
+    const size_t smA = row_smem<MW>();
+    const size_t smB = size_t(fft_padded_size(MH)) * sizeof(float2);
+    auto kf = k_2dc_rows_fwd<MW, float, 1>;
+    auto kh = k_2dc_rows_fwd<MW, __nv_bfloat16, 1>;
+    auto kb = k_2dc_cols_spec<MH>;
+    cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    const float s2 = 1.0f / (2.0f * float(H) * float(W));
+    for (int64_t i0 = 0; i0 < nimg; i0 += 32768) {
+        const int64_t g = nimg - i0 < 32768 ? nimg - i0 : 32768;
+        const dim3 gridA(H / kRB, unsigned(g));
+        if (a.k_dtype == DT_F32)
+            kf<<<gridA, kRowThreads, smA, s>>>(static_cast<const float*>(a.k), rows + i0 * stride, tb, 1, 1, 2, H, i0,
+                                               stride);
+        else
+            kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
+                                               2, H, i0, stride);
+        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, tb, W / 2 + 1, i0, stride, a.D, s2);
+    }
+    return cudaGetLastError();
+}
+
+template <int MW, int MH, typename T>
+cudaError_t conv_2dc_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    const float2* spec = reinterpret_cast<const float2*>(a.spectrum + p.spec_off);
+    const T* u = static_cast<const T*>(a.u);
+    T* y = static_cast<T*>(a.y);
+    const int64_t nimg = a.B * p.C;
+    using WT = typename WsOf<T>::type;
+    WT* ws = reinterpret_cast<WT*>(a.workspace);
+    const int64_t cap = int64_t(a.group_rows) * int64_t(sizeof(float2) / sizeof(WT));
+    const int64_t G = cap < 65535 ? cap : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));     // (W/2+1) * H elements
+    const int64_t spec_stride = int64_t(p.spec_row_bytes / sizeof(float2));
+    const int H = int(p.H), W = int(p.W);
+    const int ncol = W / 2 + 1;
+    constexpr int NTC = kFC * (MH / 16);
+    const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
+    auto ka = k_2dc_rows_fwd<MW, T, 0>;
+    auto kb = k_2dc_cols<MH, WT>;
+    auto kc = k_2dc_rows_inv<MW, T, true>;
+    auto kca = k_2dc_rows_inv<MW, T, false>;
+    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    const unsigned cblocks = unsigned((ncol + 2 * kFC - 1) / (2 * kFC));
+    for (int64_t i0 = 0; i0 < nimg; i0 += G) {
+        const int64_t g = nimg - i0 < G ? nimg - i0 : G;
+        const dim3 gridR(H / kRB, unsigned(g));
+        ka<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, ws, tb, a.B, p.C, p.order, H, i0, stride);
+        for (int st = 1; st < p.order; ++st) {
+            kb<<<dim3(cblocks, unsigned(g)), NTC, smC, s>>>(ws, spec, tb, ncol, a.B, st - 1, i0, stride, spec_stride,
+                                                            a.spec_C, a.spec_per_b);
+            if (st < p.order - 1)
+                kca<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C, p.order, p.order - st - 1, H,
+                                                               i0, stride);
+            else
+                kc<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C, p.order, 0, H, i0, stride);
+        }
+    }
+    return cudaGetLastError();
+}
+
 // Engine choice per pass, measured on B=2, C=256, 256 x 256, bf16 (us per
 // call): CTA rows + register columns 843, register rows + register columns
 // 921, CTA rows + CTA columns 939, register rows + CTA columns 1020.
@@ -588,19 +847,27 @@ constexpr bool kColsReg2D = true;
 
 template <int MW, int MH>
 cudaError_t conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    if (p.path == PATH_GRID_2D_CIRC)
+        return a.dtype == DT_F32 ? conv_2dc_t<MW, MH, float>(p, a, s) : conv_2dc_t<MW, MH, __nv_bfloat16>(p, a, s);
     return a.dtype == DT_F32 ? conv_2d_t<MW, MH, float, kRowsReg2D, kColsReg2D>(p, a, s)
                              : conv_2d_t<MW, MH, __nv_bfloat16, kRowsReg2D, kColsReg2D>(p, a, s);
+}
+
+template <int MW, int MH>
+cudaError_t spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    if (p.path == PATH_GRID_2D_CIRC) return spectrum_2dc_t<MW, MH>(p, a, s);
+    return spectrum_2d_t<MW, MH>(p, a, s);
 }
 
 template <int MW>
 cudaError_t dispatch_h_spec(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     switch (p.H) {
-        case 16: return spectrum_2d_t<MW, 16>(p, a, s);
-        case 32: return spectrum_2d_t<MW, 32>(p, a, s);
-        case 64: return spectrum_2d_t<MW, 64>(p, a, s);
-        case 128: return spectrum_2d_t<MW, 128>(p, a, s);
-        case 256: return spectrum_2d_t<MW, 256>(p, a, s);
-        case 512: return spectrum_2d_t<MW, 512>(p, a, s);
+        case 16: return spectrum_2d<MW, 16>(p, a, s);
+        case 32: return spectrum_2d<MW, 32>(p, a, s);
+        case 64: return spectrum_2d<MW, 64>(p, a, s);
+        case 128: return spectrum_2d<MW, 128>(p, a, s);
+        case 256: return spectrum_2d<MW, 256>(p, a, s);
+        case 512: return spectrum_2d<MW, 512>(p, a, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -53,6 +53,9 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
     if (C < 1) { *why = "C must be >= 1"; return false; }
     if (order < 2 || order > kMaxOrder) { *why = "order must be in [2, 8]"; return false; }
     if (!sizes) { *why = "sizes is NULL"; return false; }
+    const bool circular = (ndim & kCircularFlag) != 0;
+    ndim &= ~kCircularFlag;
+    if (circular && ndim != 2) { *why = "the circular form is 2-D only"; return false; }
     p->C = C;
     p->ndim = ndim;
     p->order = order;
@@ -100,7 +103,7 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
             *why = "2-D sizes must be powers of two in [16, 512]";
             return false;
         }
-        p->path = PATH_GRID_2D;
+        p->path = circular ? PATH_GRID_2D_CIRC : PATH_GRID_2D;
         p->H = H;
         p->W = W;
         p->L = 0;
@@ -112,8 +115,13 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
         p->t_twist = tb.add(W, 0, p->M1, 1, 1);                        // w_W^n, n < W/2
         p->t_untangle = tb.add_untangle(W);
         p->t_twist_h = tb.add(2 * H, 0, H, 1, 1);                      // w_2H^p, p < H
-        p->spec_row_bytes = size_t(W + 1) * size_t(2 * H) * 8;
-        p->ws_row_bytes = size_t(W + 1) * size_t(H) * 8;
+        if (circular) {
+            p->spec_row_bytes = size_t(W / 2 + 1) * size_t(H) * 8;
+            p->ws_row_bytes = size_t(W / 2 + 1) * size_t(H) * 8;
+        } else {
+            p->spec_row_bytes = size_t(W + 1) * size_t(2 * H) * 8;
+            p->ws_row_bytes = size_t(W + 1) * size_t(H) * 8;
+        }
     } else {
         *why = "ndim must be 1 or 2";
         return false;

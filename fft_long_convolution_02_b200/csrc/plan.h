@@ -23,6 +23,10 @@
 //                     (2H-point FFT, spectrum multiply, inverse) and an
 //                     inverse row pass.  Spectrum per channel = (W+1) columns
 //                     x 2H complex64 in the column pass's position order.
+//   PATH_GRID_2D_CIRC 2-D circular (ndim = 2 | kCircularFlag): no padding, the
+//                     W-point row FFT (packed, one W/2-point chain) and the
+//                     H-point column FFT.  Spectrum per channel = (W/2+1)
+//                     columns x H complex64.
 #pragma once
 #include <stddef.h>
 #include <stdint.h>
@@ -31,7 +35,10 @@
 
 namespace hyena {
 
-enum Path { PATH_NONE = 0, PATH_ONCHIP_1D = 1, PATH_MULTIPASS_1D = 2, PATH_GRID_2D = 3 };
+enum Path { PATH_NONE = 0, PATH_ONCHIP_1D = 1, PATH_MULTIPASS_1D = 2, PATH_GRID_2D = 3, PATH_GRID_2D_CIRC = 4 };
+
+// OR-ed into ndim (2-D only): the circular (periodic) form (HYENA_CIRCULAR).
+constexpr int kCircularFlag = 0x100;
 
 constexpr uint32_t kSpecMagic = 0x4853504Eu;  // "NPSH"
 constexpr uint32_t kSpecVersion = 1;

@@ -23,6 +23,8 @@ widths and lengths the pages discuss):
 * ``order3``   B=2 C=2048 L=65536 order 3, bf16.  a_c ~ U[0.5,8].
 * ``grid2d``   B=2 C=256 256x256 order 2, bf16, no short conv.
   K[c,i,j] = N(0,1) exp(-(i^2+j^2)/(2 s_c^2)), s_c ~ U[8,128].
+* ``grid2d_circ`` as ``grid2d`` in the circular (periodic) 2-D form; the
+  filter is the same Gaussian-windowed N(0,1) field on the H x W grid.
 * ``d768_l8k_ps`` as ``d768_l8k`` with per-sample (input-dependent) filters:
   k and D drawn for every (b, c) row, filter index b*C + c.
 
@@ -55,6 +57,7 @@ class Problem:
     u_kind: str = "normal"     # "normal" or "acgt"
     sc_bias: bool = False
     per_sample: bool = False   # one long filter (and D) per (b, c) row
+    circular: bool = False     # 2-D only: periodic boundary, no padding
     seed: int = 20260000
 
     @property
@@ -96,6 +99,8 @@ WORKLOADS = {
                       decay=(0.5, 8.0), seed=20260003),
     "grid2d": Problem("grid2d", B=2, C=256, H=256, W=256, order=2, dtype="bf16",
                       shortconv=False, sigma=(8.0, 128.0), seed=20260004),
+    "grid2d_circ": Problem("grid2d_circ", B=2, C=256, H=256, W=256, order=2, dtype="bf16",
+                           shortconv=False, sigma=(8.0, 128.0), circular=True, seed=20260006),
     "d768_l8k_ps": Problem("d768_l8k_ps", B=4, C=768, L=8192, order=2, dtype="bf16",
                            decay=(0.5, 6.0), per_sample=True, seed=20260005),
 }

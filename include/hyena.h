@@ -61,6 +61,17 @@ typedef enum {
                                          hyena_spectrum_check)                       */
 } hyena_status_t;
 
+/*
+ * ndim: 1 (L), 2 (H x W, non-circular: zero padded, output cropped), or
+ * 2 | HYENA_CIRCULAR (H x W, circular: periodic boundary, the filter on the
+ * same H x W grid, v[p][q] = sum_{i,j} K[i][j] w[(p-i) mod H][(q-j) mod W] +
+ * D w[p][q]).  Source: [P5] 方法论 (边界处理: circular convolution for
+ * periodic physical systems, non-circular by zero padding for images and
+ * volumes).  Every call that takes ndim accepts the flag; a spectrum built
+ * for one form is rejected by the other (its size differs).
+ */
+#define HYENA_CIRCULAR 0x100
+
 /* Version of this ABI (major * 100 + minor). */
 int hyena_version(void);
 

@@ -11,6 +11,11 @@ from fft_long_convolution_02_b200 import inputs as I
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 
 
+def api_shape(p: I.Problem):
+    """The shape argument of the C ABI calls (the circular 2-D form flagged)."""
+    return hb.Circular(p.shape) if p.circular else p.shape
+
+
 def to_torch(p: I.Problem, stored: np.ndarray, device="cuda"):
     import torch
     if p.dtype == "bf16":
@@ -37,21 +42,21 @@ class Run:
         self.sc_w = torch.from_numpy(data["sc_w"]).cuda() if (use_shortconv and data["sc_w"] is not None) else None
         self.sc_b = (torch.from_numpy(data["sc_b"]).cuda()
                      if (self.sc_w is not None and data.get("sc_b") is not None) else None)
-        self.spectrum = torch.empty(hb.hyena_spectrum_bytes(p.C, p.shape, p.order), dtype=torch.uint8,
+        self.spectrum = torch.empty(hb.hyena_spectrum_bytes(p.C, api_shape(p), p.order), dtype=torch.uint8,
                                     device="cuda")
         self.y = torch.empty((p.B, p.C) + p.shape, dtype=self.u.dtype, device="cuda")
         if workspace_bytes is None:
-            workspace_bytes = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, p.shape, p.order)
+            workspace_bytes = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, api_shape(p), p.order)
         self.workspace = (torch.empty(workspace_bytes, dtype=torch.uint8, device="cuda")
                           if workspace_bytes else None)
 
     def build_spectrum(self):
-        hb.hyena_filter_spectrum(self.k, self.D, self.p.C, self.p.shape, self.p.order, self.spectrum)
+        hb.hyena_filter_spectrum(self.k, self.D, self.p.C, api_shape(self.p), self.p.order, self.spectrum)
 
     def conv(self, u=None, y=None):
         p = self.p
         hb.hyena_gated_fftconv(self.u if u is None else u, self.y if y is None else y, self.spectrum,
-                               self.sc_w, self.sc_b, p.B, p.C, p.shape, p.order, self.workspace)
+                               self.sc_w, self.sc_b, p.B, p.C, api_shape(p), p.order, self.workspace)
 
     def run(self) -> np.ndarray:
         import torch
@@ -72,7 +77,7 @@ def oracle_for_rows(orc, p: I.Problem, rows, data=None, use_shortconv=True, meth
     u, k, D, w, b = I.oracle_rows(p, rows, data)
     if not use_shortconv:
         w, b = None, None
-    return orc.hyena_rows(u, k, D, w, b, ndim=p.ndim, method=method)
+    return orc.hyena_rows(u, k, D, w, b, ndim=p.ndim, method=method, circular=p.circular)
 
 
 def gpu_rows(y: np.ndarray, p: I.Problem, rows) -> np.ndarray:

@@ -58,6 +58,12 @@ def test_spectrum_bytes_and_workspace(lib):
     # 2-D: (W+1) * 2H complex64 per channel
     b = lib.hyena_spectrum_bytes(256, 2, _sz(256, 256), 2)
     assert 256 * 257 * 512 * 8 <= b < 256 * 257 * 512 * 8 + (1 << 20)
+    # 2-D circular: (W/2+1) * H complex64 per channel; 1-D circular is refused
+    circ = 2 | 0x100
+    b = lib.hyena_spectrum_bytes(256, circ, _sz(256, 128), 2)
+    assert 256 * 65 * 256 * 8 <= b < 256 * 65 * 256 * 8 + (1 << 20)
+    assert lib.hyena_gated_fftconv_workspace_min_bytes(256, circ, _sz(256, 128), 2) == 65 * 256 * 8
+    assert lib.hyena_spectrum_bytes(64, 1 | 0x100, _sz(1024), 2) == 0
     # unsupported shapes
     for bad in [(1, _sz(12), 2), (1, _sz(8), 2), (1, _sz(1 << 21), 2), (2, _sz(16, 1024), 2),
                 (1, _sz(1024), 1), (1, _sz(1024), 9)]:
