@@ -73,6 +73,11 @@ class Oracle:
         lib.oracle_conv2d_direct.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
         lib.oracle_conv2d_fft.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
         lib.oracle_conv2d_circ_direct.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
+        lib.oracle_conv3d_direct.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64, _i64]
+        lib.oracle_conv3d_fft.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64, _i64]
+        lib.oracle_hyena_rows3.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, _dp]
+        lib.oracle_hyena_rows3.restype = ctypes.c_int
         lib.oracle_conv2d_circ_fft.argtypes = [_dp, ctypes.c_double, _dp, _dp, _i64, _i64]
         lib.oracle_hyena_rows.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -138,6 +143,36 @@ class Oracle:
         out = np.empty_like(x)
         self.lib.oracle_conv2d_circ_fft(_ptr(K), float(D), _ptr(x), _ptr(out), x.shape[0], x.shape[1])
         return out
+
+    def conv3d_direct(self, K, D: float, x) -> np.ndarray:
+        """3-D non-circular convolution by its direct sum ([P5] 原生 ND 卷积)."""
+        K = _f64(K); x = _f64(x)
+        out = np.empty_like(x)
+        self.lib.oracle_conv3d_direct(_ptr(K), float(D), _ptr(x), _ptr(out), *x.shape)
+        return out
+
+    def conv3d_fft(self, K, D: float, x) -> np.ndarray:
+        """The same through a zero-padded (2x per axis) radix-2 3-D FFT."""
+        K = _f64(K); x = _f64(x)
+        out = np.empty_like(x)
+        self.lib.oracle_conv3d_fft(_ptr(K), float(D), _ptr(x), _ptr(out), *x.shape)
+        return out
+
+    def hyena_rows3(self, u_rows, k_rows, D_rows, *, method: int = 2, nthreads: int = 0) -> np.ndarray:
+        """The operator on self-contained 3-D rows: u_rows [R, order+1, N1, N2, N3],
+        k_rows [R, order-1, N1, N2, N3], D_rows [R, order-1]; y [R, N1, N2, N3]."""
+        u_rows = _f64(u_rows); k_rows = _f64(k_rows); D_rows = _f64(D_rows)
+        R, ch = u_rows.shape[0], u_rows.shape[1]
+        order = ch - 1
+        N1, N2, N3 = u_rows.shape[2:]
+        if k_rows.shape != (R, order - 1, N1, N2, N3) or D_rows.shape != (R, order - 1):
+            raise ValueError("k_rows / D_rows shape does not match u_rows")
+        y = np.empty((R, N1, N2, N3), dtype=np.float64)
+        rc = self.lib.oracle_hyena_rows3(_ptr(u_rows), _ptr(k_rows), _ptr(D_rows), R, N1, N2, N3, order, method,
+                                         nthreads, _ptr(y))
+        if rc != 0:
+            raise ValueError("oracle_hyena_rows3 rejected its arguments")
+        return y
 
     def hyena_rows(self, u_rows, k_rows, D_rows, sc_w_rows=None, sc_b_rows=None, *,
                    ndim: int = 1, method: int = 0, nthreads: int = 0,
@@ -221,6 +256,18 @@ def conv2d_circ_direct(K, D, x):
 
 def conv2d_circ_fft(K, D, x):
     return default().conv2d_circ_fft(K, D, x)
+
+
+def conv3d_direct(K, D, x):
+    return default().conv3d_direct(K, D, x)
+
+
+def conv3d_fft(K, D, x):
+    return default().conv3d_fft(K, D, x)
+
+
+def hyena_rows3(u_rows, k_rows, D_rows, **kw):
+    return default().hyena_rows3(u_rows, k_rows, D_rows, **kw)
 
 
 def hyena_rows(u_rows, k_rows, D_rows, sc_w_rows=None, sc_b_rows=None, **kw):

@@ -29,6 +29,10 @@
  *    kept, tap w[2] multiplies the current sample, w[0] the sample two back.
  *  - 2-D form: v[p][q] = sum_{i<=p, j<=q} K[i][j] w[p-i][q-j] + D w[p][q]
  *    (kernel anchored at (0,0), output cropped to [0:H, 0:W]).
+ *  - 3-D form ([P5] 原生 ND 卷积 on L1 x L2 x L3 grids, e.g. 3-D medical
+ *    volumes): v[a][p][q] = sum_{h<=a, i<=p, j<=q} K[h][i][j]
+ *    w[a-h][p-i][q-j] + D w[a][p][q], kernel anchored at the origin, output
+ *    cropped to the input grid (zero padding every axis to twice its length).
  *  - 2-D circular form ([P5] 边界处理: circular convolution for periodic
  *    systems, no padding): v[p][q] = sum_{i<H, j<W} K[i][j]
  *    w[(p-i) mod H][(q-j) mod W] + D w[p][q], with K on the same H x W grid.
@@ -264,6 +268,119 @@ void oracle_conv2d_circ_fft(const double *K, double D, const double *x,
     double scale = 1.0 / (double)n;
     for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale + D * x[t];
     free(kr); free(ki); free(xr); free(xi);
+}
+
+/* ---------------------------------------------------------------------- */
+/* 3-D non-circular convolution ([P5] 原生 ND 卷积, 边界处理).            */
+/* out[a][p][q] = sum_{h<=a, i<=p, j<=q} K[h][i][j] x[a-h][p-i][q-j]      */
+/*                + D x[a][p][q]                                         */
+/* ---------------------------------------------------------------------- */
+void oracle_conv3d_direct(const double *K, double D, const double *x,
+                          double *out, int64_t N1, int64_t N2, int64_t N3)
+{
+    for (int64_t a = 0; a < N1; ++a)
+        for (int64_t p = 0; p < N2; ++p)
+            for (int64_t q = 0; q < N3; ++q) {
+                double acc = 0.0;
+                for (int64_t h = 0; h <= a; ++h)
+                    for (int64_t i = 0; i <= p; ++i)
+                        for (int64_t j = 0; j <= q; ++j)
+                            acc += K[(h * N2 + i) * N3 + j] * x[((a - h) * N2 + (p - i)) * N3 + (q - j)];
+                out[(a * N2 + p) * N3 + q] = acc + D * x[(a * N2 + p) * N3 + q];
+            }
+}
+
+/* 3-D FFT of an n1 x n2 x n3 complex array: each axis in turn, radix-2. */
+static void oracle_fft3(double *re, double *im, int64_t n1, int64_t n2, int64_t n3, int sign)
+{
+    int64_t nmax = n1 > n2 ? (n1 > n3 ? n1 : n3) : (n2 > n3 ? n2 : n3);
+    double *lr = (double *)malloc(sizeof(double) * (size_t)nmax);
+    double *li = (double *)malloc(sizeof(double) * (size_t)nmax);
+    for (int64_t a = 0; a < n1; ++a)            /* axis 3: contiguous lines */
+        for (int64_t p = 0; p < n2; ++p)
+            oracle_fft(re + (a * n2 + p) * n3, im + (a * n2 + p) * n3, n3, sign);
+    for (int64_t a = 0; a < n1; ++a)            /* axis 2 */
+        for (int64_t q = 0; q < n3; ++q) {
+            for (int64_t p = 0; p < n2; ++p) { lr[p] = re[(a * n2 + p) * n3 + q]; li[p] = im[(a * n2 + p) * n3 + q]; }
+            oracle_fft(lr, li, n2, sign);
+            for (int64_t p = 0; p < n2; ++p) { re[(a * n2 + p) * n3 + q] = lr[p]; im[(a * n2 + p) * n3 + q] = li[p]; }
+        }
+    for (int64_t p = 0; p < n2; ++p)            /* axis 1 */
+        for (int64_t q = 0; q < n3; ++q) {
+            for (int64_t a = 0; a < n1; ++a) { lr[a] = re[(a * n2 + p) * n3 + q]; li[a] = im[(a * n2 + p) * n3 + q]; }
+            oracle_fft(lr, li, n1, sign);
+            for (int64_t a = 0; a < n1; ++a) { re[(a * n2 + p) * n3 + q] = lr[a]; im[(a * n2 + p) * n3 + q] = li[a]; }
+        }
+    free(lr); free(li);
+}
+
+/* Zero-padded (every axis to twice its length, powers of two) 3-D FFT convolution. */
+void oracle_conv3d_fft(const double *K, double D, const double *x,
+                       double *out, int64_t N1, int64_t N2, int64_t N3)
+{
+    int64_t n1 = next_pow2(2 * N1), n2 = next_pow2(2 * N2), n3 = next_pow2(2 * N3);
+    size_t n = (size_t)(n1 * n2 * n3);
+    double *kr = (double *)calloc(n, sizeof(double));
+    double *ki = (double *)calloc(n, sizeof(double));
+    double *xr = (double *)calloc(n, sizeof(double));
+    double *xi = (double *)calloc(n, sizeof(double));
+    for (int64_t a = 0; a < N1; ++a)
+        for (int64_t p = 0; p < N2; ++p)
+            for (int64_t q = 0; q < N3; ++q) {
+                kr[(a * n2 + p) * n3 + q] = K[(a * N2 + p) * N3 + q];
+                xr[(a * n2 + p) * n3 + q] = x[(a * N2 + p) * N3 + q];
+            }
+    oracle_fft3(kr, ki, n1, n2, n3, -1);
+    oracle_fft3(xr, xi, n1, n2, n3, -1);
+    for (size_t f = 0; f < n; ++f) {
+        double a = xr[f] * kr[f] - xi[f] * ki[f];
+        double b = xr[f] * ki[f] + xi[f] * kr[f];
+        xr[f] = a; xi[f] = b;
+    }
+    oracle_fft3(xr, xi, n1, n2, n3, +1);
+    double scale = 1.0 / (double)n;
+    for (int64_t a = 0; a < N1; ++a)
+        for (int64_t p = 0; p < N2; ++p)
+            for (int64_t q = 0; q < N3; ++q)
+                out[(a * N2 + p) * N3 + q] = xr[(a * n2 + p) * n3 + q] * scale + D * x[(a * N2 + p) * N3 + q];
+    free(kr); free(ki); free(xr); free(xi);
+}
+
+/*
+ * The operator on nrows self-contained 3-D rows (N1 x N2 x N3 each, no short
+ * conv: the pages give none for N-D): u_rows [nrows][order+1][n], k_rows
+ * [nrows][order-1][n], D_rows [nrows][order-1], y [nrows][n]; the same gating
+ * as the 1-D and 2-D forms ([P4] 二.1).  method: 1 direct, 2 FFT.
+ */
+int oracle_hyena_rows3(const double *u_rows, const double *k_rows, const double *D_rows, int64_t nrows,
+                       int64_t N1, int64_t N2, int64_t N3, int order, int method, int nthreads, double *y)
+{
+    if (!u_rows || !k_rows || !D_rows || !y || nrows < 0 || N1 < 1 || N2 < 1 || N3 < 1 || order < 2)
+        return -1;
+    int64_t n = N1 * N2 * N3;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        const double *x = u_rows + r * (order + 1) * n;
+        double *v = (double *)malloc(sizeof(double) * (size_t)n);
+        double *w = (double *)malloc(sizeof(double) * (size_t)n);
+        memcpy(v, x + (int64_t)order * n, sizeof(double) * (size_t)n);
+        for (int s = 1; s <= order - 1; ++s) {
+            const double *g = x + (int64_t)(order - s) * n;   /* gate x_{order-s} */
+            for (int64_t t = 0; t < n; ++t) w[t] = g[t] * v[t];
+            const double *ks = k_rows + (r * (order - 1) + (s - 1)) * n;
+            double Ds = D_rows[r * (order - 1) + (s - 1)];
+            if (method == 1) oracle_conv3d_direct(ks, Ds, w, v, N1, N2, N3);
+            else             oracle_conv3d_fft(ks, Ds, w, v, N1, N2, N3);
+        }
+        for (int64_t t = 0; t < n; ++t) y[r * n + t] = x[t] * v[t];
+        free(v); free(w);
+    }
+    return 0;
 }
 
 /* ---------------------------------------------------------------------- */

@@ -328,4 +328,48 @@ def pin_operator2d_circ_wraps(orc):
     _close(lin, want, 1e-12, "padded")
 
 
+# -------------------------------------------------------------- 3-D form ---
+# [P5] 原生 ND 卷积 / 边界处理: N-D global convolution, zero padded per axis.
+def _np_linear3(K, x):
+    n = [2 * s for s in x.shape]
+    ax = (0, 1, 2)
+    y = np.fft.ifftn(np.fft.fftn(K, n, axes=ax) * np.fft.fftn(x, n, axes=ax), axes=ax).real
+    return y[: x.shape[0], : x.shape[1], : x.shape[2]]
+
+
+def pin_conv3d_matches_numpy(orc):
+    """Direct sum and FFT form against numpy's zero-padded fftn product."""
+    rng = np.random.default_rng(31)
+    for shape in ((1, 4, 8), (4, 4, 4), (2, 8, 4), (8, 4, 16)):
+        K = rng.standard_normal(shape); x = rng.standard_normal(shape)
+        ref = _np_linear3(K, x) + 0.6 * x
+        _close(orc.conv3d_direct(K, 0.6, x), ref, 1e-11, f"direct {shape}")
+        _close(orc.conv3d_fft(K, 0.6, x), ref, 1e-11, f"fft {shape}")
+
+
+def pin_conv3d_single_slice_is_2d(orc):
+    """N1 = 1 reduces to the 2-D form, and the delta returns K + D delta."""
+    rng = np.random.default_rng(32)
+    K = rng.standard_normal((1, 8, 16)); x = rng.standard_normal((1, 8, 16))
+    _close(orc.conv3d_direct(K, 0.2, x)[0], orc.conv2d_direct(K[0], 0.2, x[0]), 1e-12, "N1=1")
+    K = rng.standard_normal((4, 4, 8))
+    d = np.zeros((4, 4, 8)); d[0, 0, 0] = 1.0
+    want = K.copy(); want[0, 0, 0] += 0.2
+    _close(orc.conv3d_direct(K, 0.2, d), want, 1e-12, "delta direct")
+    _close(orc.conv3d_fft(K, 0.2, d), want, 1e-12, "delta fft")
+
+
+def pin_operator3d(orc):
+    """The 3-D operator: direct equals FFT (orders 2 and 3), and one slice
+    equals the 2-D operator."""
+    rng = np.random.default_rng(33)
+    for order in (2, 3):
+        u = rng.standard_normal((2, order + 1, 2, 4, 8)); k = rng.standard_normal((2, order - 1, 2, 4, 8))
+        D = rng.standard_normal((2, order - 1))
+        _close(orc.hyena_rows3(u, k, D, method=1), orc.hyena_rows3(u, k, D, method=2), 1e-11, f"order {order}")
+    u = rng.standard_normal((2, 3, 1, 8, 8)); k = rng.standard_normal((2, 1, 1, 8, 8)); D = rng.standard_normal((2, 1))
+    _close(orc.hyena_rows3(u, k, D, method=1)[:, 0], orc.hyena_rows(u[:, :, 0], k[:, :, 0], D, ndim=2, method=1),
+           1e-12, "N1=1 operator")
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

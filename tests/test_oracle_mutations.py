@@ -42,6 +42,12 @@ MUTATIONS = {
                                        "acc += K[i * W + j] * x[((p + i) % H) * W + ((q + j) % W)];"),
     "2-D circular fft skip dropped": ("for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale + D * x[t];",
                                       "for (size_t t = 0; t < n; ++t) out[t] = xr[t] * scale;"),
+    "3-D kernel axes swapped": ("acc += K[(h * N2 + i) * N3 + j] * x[((a - h) * N2 + (p - i)) * N3 + (q - j)];",
+                                "acc += K[(i * N2 + h) * N3 + j] * x[((a - h) * N2 + (p - i)) * N3 + (q - j)];"),
+    "3-D fft depth axis not padded": ("int64_t n1 = next_pow2(2 * N1), n2 = next_pow2(2 * N2), n3 = next_pow2(2 * N3);",
+                                      "int64_t n1 = next_pow2(N1), n2 = next_pow2(2 * N2), n3 = next_pow2(2 * N3);"),
+    "3-D operator gates with v's chunk": ("const double *g = x + (int64_t)(order - s) * n;",
+                                          "const double *g = x + (int64_t)order * n;"),
     "2-D circular form runs padded": ("if (direct) oracle_conv2d_circ_direct(ks, Ds, w, vn, H, W);",
                                       "if (direct) oracle_conv2d_direct(ks, Ds, w, vn, H, W);"),
 }
