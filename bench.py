@@ -56,6 +56,8 @@ def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
 
 def spectrum_row_bytes(p) -> int:
     """Spectrum bytes per (step, channel) row the convolution kernel reads."""
+    if p.ndim == 3:
+        return (p.W + 1) * 2 * p.H * 2 * p.N1 * 8
     if p.ndim == 2:
         return (p.W // 2 + 1) * p.H * 8 if p.circular else (p.W + 1) * 2 * p.H * 8
     if p.L == 8192:
@@ -141,6 +143,13 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def _oracle_rows(orc, p, args, cores):
+    """The float64 oracle on self-contained rows of problem p (FFT form)."""
+    if p.ndim == 3:
+        return orc.hyena_rows3(*args[:3], method=2, nthreads=cores)
+    return orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+
+
 def cpu_baseline(p, budget_s: float = 15.0):
     """Time the float64 oracle (as it stands) on a bounded sample of rows."""
     import oracle
@@ -151,7 +160,7 @@ def cpu_baseline(p, budget_s: float = 15.0):
     rows = rng.choice(p.B * p.C, size=min(p.B * p.C, 8 * cores), replace=False)
     args = I.oracle_rows(p, rows)
     t0 = time.perf_counter()
-    orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+    _oracle_rows(orc, p, args, cores)
     dt = time.perf_counter() - t0
     # grow the sample to use about budget_s of CPU time
     n_more = int(len(rows) * max(0.0, budget_s / max(dt, 1e-3) - 1.0))
@@ -161,7 +170,7 @@ def cpu_baseline(p, budget_s: float = 15.0):
         rows2 = rng.choice(p.B * p.C, size=n_more, replace=False)
         args = I.oracle_rows(p, rows2)
         t0 = time.perf_counter()
-        orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+        _oracle_rows(orc, p, args, cores)
         total_t += time.perf_counter() - t0
         total_rows += n_more
     # a row is one (b, c) pair; the operator's tokens are B*n over all C channels
@@ -184,10 +193,10 @@ def run_reference(args, p):
     samples = [I.oracle_rows(p, rng.choice(p.B * p.C, size=per_step, replace=False))
                for _ in range(args.warmup + args.steps)]
     for a in samples[:args.warmup]:
-        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+        _oracle_rows(orc, p, a, cores)
     t0 = time.perf_counter()
     for a in samples[args.warmup:]:
-        orc.hyena_rows(*a, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+        _oracle_rows(orc, p, a, cores)
     dt = time.perf_counter() - t0
     tok_s = args.steps * per_step * p.n / (p.C * dt)
     line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
@@ -211,8 +220,10 @@ def config_of(p):
         cfg["boundary"] = "circular"
     if p.ndim == 1:
         cfg["L"] = p.L
-    else:
+    elif p.ndim == 2:
         cfg["H"], cfg["W"] = p.H, p.W
+    else:
+        cfg["N1"], cfg["H"], cfg["W"] = p.N1, p.H, p.W
     return cfg
 
 
@@ -344,7 +355,7 @@ def main():
     elif p.ndim == 1 and p.L <= 16384:
         kernel = "k_conv_onchip"
     else:
-        kernel = "multipass" if p.ndim == 1 else "grid2d"
+        kernel = "multipass" if p.ndim == 1 else ("grid2d" if p.ndim == 2 else "grid3d")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,

@@ -43,14 +43,14 @@ hyena_status_t cuda_status(cudaError_t e, const char* what) {
 }
 
 
-// 1, 2, or 2 | HYENA_CIRCULAR (the circular 2-D form)
-bool valid_ndim(int ndim) { return ndim == 1 || ndim == 2 || ndim == (2 | kCircularFlag); }
+// 1, 2, 3, or 2 | HYENA_CIRCULAR (the circular 2-D form)
+bool valid_ndim(int ndim) { return ndim == 1 || ndim == 2 || ndim == 3 || ndim == (2 | kCircularFlag); }
 
 hyena_status_t plan_or_fail(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p) {
     std::string why;
     if (C < 1) return fail(HYENA_ERR_INVALID_ARG, "C must be >= 1");
     if (!sizes) return fail(HYENA_ERR_INVALID_ARG, "sizes is NULL");
-    if (!valid_ndim(ndim)) return fail(HYENA_ERR_INVALID_ARG, "ndim must be 1, 2 or 2 | HYENA_CIRCULAR");
+    if (!valid_ndim(ndim)) return fail(HYENA_ERR_INVALID_ARG, "ndim must be 1, 2, 3 or 2 | HYENA_CIRCULAR");
     if (!make_plan(C, ndim, sizes, order, p, &why)) return fail(HYENA_ERR_UNSUPPORTED_SHAPE, why);
     return HYENA_OK;
 }
@@ -114,6 +114,7 @@ hyena_status_t hyena_filter_spectrum(const void* k, hyena_dtype_t k_dtype, const
         case PATH_MULTIPASS_1D: e = launch_spectrum_multipass(p, a, s); break;
         case PATH_GRID_2D:
         case PATH_GRID_2D_CIRC: e = launch_spectrum_2d(p, a, s); break;
+        case PATH_GRID_3D: e = launch_spectrum_3d(p, a, s); break;
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "spectrum kernel");
@@ -173,7 +174,7 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
     if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
     if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
     if (!valid_dtype(dtype)) return fail(HYENA_ERR_INVALID_ARG, "dtype must be HYENA_F32 or HYENA_BF16");
-    if (ndim != 1 && sc_w) return fail(HYENA_ERR_INVALID_ARG, "the 2-D form has no short conv: sc_w must be NULL");
+    if (ndim != 1 && sc_w) return fail(HYENA_ERR_INVALID_ARG, "the 2-D and 3-D forms have no short conv: sc_w must be NULL");
     if (!aligned16(u) || !aligned16(y) || !aligned16(spectrum))
         return fail(HYENA_ERR_MISALIGNED, "u, y and spectrum must be 16-byte aligned");
     if ((sc_w && !aligned4(sc_w)) || (sc_bias && !aligned4(sc_bias)))
@@ -221,6 +222,7 @@ hyena_status_t gated_fftconv(const void* u, void* y, const void* spectrum, size_
         case PATH_MULTIPASS_1D: e = launch_conv_multipass(p, a, s); break;
         case PATH_GRID_2D:
         case PATH_GRID_2D_CIRC: e = launch_conv_2d(p, a, s); break;
+        case PATH_GRID_3D: e = launch_conv_3d(p, a, s); break;
         default: return fail(HYENA_ERR_INTERNAL, "no path");
     }
     return cuda_status(e, "gated fftconv kernel");

@@ -647,6 +647,81 @@ k_2dc_cols_spec(float2* __restrict__ rows, T2d tb, int ncol, int64_t row0, int64
     }
 }
 
+// ===========================================================================
+// 3-D non-circular form ([P5] 原生 ND 卷积 on N1 x H x W grids, e.g. 3-D
+// medical volumes; every axis zero padded to twice its length).  The volume
+// is N1 H rows of W samples for the row passes (the 2-D row kernels with
+// N1 H image rows), so the first workspace region ws1 is [fw][d][h] (fw =
+// 0..W).  The column passes run one padded 2H-point transform per (fw, d)
+// and store both chains' H positions as depth lines: ws2 [fw][chain][pos][d].
+// The depth pass is the 2-D register column pass over those lines (2N1-point,
+// times K~, inverse); the inverse column pass brings the lines back to ws1.
+// K~ = (DFT_2N1x2Hx2W(k) + D) / (16 N1 H W), per channel [line][chain][pos]
+// with line = (fw, chain, pos) of the column pass.
+// ===========================================================================
+
+// Forward column pass of the 3-D form: columns (fw, d) of ws1 -> ws2 lines.
+// Thread group cc of the CTA takes column d = d0 + cc of bin fw.
+template <int MH, typename WT>
+__global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
+k_3d_cols_fwd(WT* __restrict__ ws, T2d tb, int N1, int64_t ws1_off, int64_t ws2_off, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = MH / 16;
+    constexpr int PS = fft_padded_size(MH);
+    const int t = threadIdx.x, cc = t / TPT, g = t - (t / TPT) * TPT;
+    const int dblocks = N1 / kFC;
+    const int fw = int(blockIdx.x) / dblocks;
+    const int d = (int(blockIdx.x) - fw * dblocks) * kFC + cc;
+    WT* ws1 = ws + int64_t(blockIdx.y) * ws_img_stride + ws1_off;
+    WT* ws2 = ws + int64_t(blockIdx.y) * ws_img_stride + ws2_off;
+    const WT* col = ws1 + (int64_t(fw) * N1 + d) * MH;
+    float2 x[2][16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int h = g + TPT * s;
+        const float2 v = ws_ld(col + h);
+        x[0][s] = v;
+        x[1][s] = cmul(v, __ldg(tb.twist_h + h));
+    }
+    float2* const buf[2] = {smem + (2 * cc) * PS, smem + (2 * cc + 1) * PS};
+    reg_fft_forward<MH, 2>(x, buf, g, tb.fftH);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            ws_st(ws2 + ((int64_t(fw) * 2 + ch) * MH + 16 * g + k) * N1 + d, x[ch][k]);
+    }
+}
+
+// Inverse column pass of the 3-D form: ws2 lines -> columns (fw, d) of ws1.
+template <int MH, typename WT>
+__global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
+k_3d_cols_inv(WT* __restrict__ ws, T2d tb, int N1, int64_t ws1_off, int64_t ws2_off, int64_t ws_img_stride) {
+    extern __shared__ float2 smem[];
+    constexpr int TPT = MH / 16;
+    constexpr int PS = fft_padded_size(MH);
+    const int t = threadIdx.x, cc = t / TPT, g = t - (t / TPT) * TPT;
+    const int dblocks = N1 / kFC;
+    const int fw = int(blockIdx.x) / dblocks;
+    const int d = (int(blockIdx.x) - fw * dblocks) * kFC + cc;
+    WT* ws1 = ws + int64_t(blockIdx.y) * ws_img_stride + ws1_off;
+    WT* ws2 = ws + int64_t(blockIdx.y) * ws_img_stride + ws2_off;
+    float2 x[2][16];
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[ch][k] = ws_ld(ws2 + ((int64_t(fw) * 2 + ch) * MH + 16 * g + k) * N1 + d);
+    }
+    float2* const buf[2] = {smem + (2 * cc) * PS, smem + (2 * cc + 1) * PS};
+    reg_fft_inverse<MH, 2>(x, buf, g, tb.fftH);
+    WT* col = ws1 + (int64_t(fw) * N1 + d) * MH;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const int h = g + TPT * s;
+        ws_st(col + h, cadd(x[0][s], cmulc(x[1][s], __ldg(tb.twist_h + h))));
+    }
+}
+
 template <int MW>
 size_t row_smem() {
     return size_t(2) * kRB * fft_padded_size(MW) * sizeof(float2);
@@ -839,6 +914,114 @@ cudaError_t conv_2dc_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Depth tables of the 3-D form: the depth pass is the 2-D register column
+// pass with the H tables swapped for the N1 ones.
+T2d t2d_depth(const Plan& p, const uint8_t* spectrum) {
+    const float2* t = reinterpret_cast<const float2*>(spectrum + p.tables_off);
+    T2d tb = t2d(p, spectrum);
+    tb.fftH = t + p.t_fft_d;
+    tb.twist_h = t + p.t_twist_d;
+    return tb;
+}
+
+// 3-D spectrum build: row pass of k into the lower quarter of each channel's
+// region, forward column pass into the upper half, then the depth lines in
+// spectrum mode (one CTA per channel walking the lines in increasing order,
+// so each line's output only overwrites consumed input).
+template <int MW, int MH, int MD>
+cudaError_t spectrum_3d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    const T2d tbd = t2d_depth(p, a.spectrum);
+    float2* rows = reinterpret_cast<float2*>(a.spectrum + p.spec_off);
+    const int64_t nimg = (p.order - 1) * p.C;
+    const int64_t stride = int64_t(p.spec_row_bytes / sizeof(float2));    // lines * 2 N1
+    const int N1 = int(p.L), H = int(p.H), W = int(p.W);
+    const int64_t nlines = int64_t(W + 1) * 2 * H;
+    const int64_t ws2_off = nlines * N1;                                  // upper half
+    const size_t smA = row_smem<MW>();
+    const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
+    const size_t smB = col_smem2<MD>(1);
+    auto kf = k_2d_rows_fwd<MW, float, 1>;
+    auto kh = k_2d_rows_fwd<MW, __nv_bfloat16, 1>;
+    auto kcf = k_3d_cols_fwd<MH, float2>;
+    auto kb = k_2d_cols<MD, 1, float2>;
+    cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smA));
+    cudaFuncSetAttribute(kcf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
+    const float s16 = 1.0f / (16.0f * float(N1) * float(H) * float(W));
+    for (int64_t i0 = 0; i0 < nimg; i0 += 32768) {
+        const int64_t g = nimg - i0 < 32768 ? nimg - i0 : 32768;
+        const dim3 gridA(N1 * H / kRB, unsigned(g));
+        if (a.k_dtype == DT_F32)
+            kf<<<gridA, kRowThreads, smA, s>>>(static_cast<const float*>(a.k), rows + i0 * stride, tb, 1, 1, 2,
+                                               N1 * H, i0, stride, 0);
+        else
+            kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
+                                               2, N1 * H, i0, stride, 0);
+        kcf<<<dim3(unsigned((W + 1) * (N1 / kFC)), unsigned(g)), kFC * (MH / 16), smC, s>>>(rows + i0 * stride, tb,
+                                                                                          N1, 0, ws2_off, stride);
+        // k_2d_cols in spectrum mode reads its columns from the upper half
+        // (offset ncol * MD = nlines * N1) and writes 2 N1 entries per line
+        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, nullptr, tbd, int(nlines - 1), 1, p.C,
+                                                           0, i0, stride, 0, a.D, s16, 0, 0);
+    }
+    return cudaGetLastError();
+}
+
+template <int MW, int MH, int MD, typename T>
+cudaError_t conv_3d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    const T2d tb = t2d(p, a.spectrum);
+    const T2d tbd = t2d_depth(p, a.spectrum);
+    const float2* spec = reinterpret_cast<const float2*>(a.spectrum + p.spec_off);
+    const T* u = static_cast<const T*>(a.u);
+    T* y = static_cast<T*>(a.y);
+    const int64_t nimg = a.B * p.C;
+    using WT = typename WsOf<T>::type;
+    WT* ws = reinterpret_cast<WT*>(a.workspace);
+    const int64_t cap = int64_t(a.group_rows) * int64_t(sizeof(float2) / sizeof(WT));
+    const int64_t G = cap < 65535 ? cap : 65535;
+    const int64_t stride = int64_t(p.ws_row_bytes / sizeof(float2));      // ws1 + ws2 elements
+    const int64_t spec_stride = int64_t(p.spec_row_bytes / sizeof(float2));
+    const int N1 = int(p.L), H = int(p.H), W = int(p.W);
+    const int64_t nlines = int64_t(W + 1) * 2 * H;
+    const int64_t ws2_off = int64_t(W + 1) * N1 * H;
+    const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
+    const size_t smD = size_t(2 * kFC) * fft_padded_size(MD) * sizeof(float2);
+    auto ka = k_2d_rows_fwd<MW, T, 0>;
+    auto kcf = k_3d_cols_fwd<MH, WT>;
+    auto kd = k_2df_cols<MD, WT>;
+    auto kci = k_3d_cols_inv<MH, WT>;
+    auto kc = k_2d_rows_inv<MW, T, true>;
+    auto kca = k_2d_rows_inv<MW, T, false>;
+    cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    cudaFuncSetAttribute(kcf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+    cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smD));
+    cudaFuncSetAttribute(kci, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+    cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
+    const unsigned cblocks = unsigned((W + 1) * (N1 / kFC));
+    const unsigned dblocks = unsigned((nlines + kFC - 1) / kFC);
+    for (int64_t i0 = 0; i0 < nimg; i0 += G) {
+        const int64_t g = nimg - i0 < G ? nimg - i0 : G;
+        const dim3 gridR(N1 * H / kRB, unsigned(g));
+        ka<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, ws, tb, a.B, p.C, p.order, N1 * H, i0, stride, 0);
+        for (int st = 1; st < p.order; ++st) {
+            kcf<<<dim3(cblocks, unsigned(g)), kFC * (MH / 16), smC, s>>>(ws, tb, N1, 0, ws2_off, stride);
+            kd<<<dim3(dblocks, unsigned(g)), kFC * (MD / 16), smD, s>>>(ws + ws2_off, spec, tbd, int(nlines - 1),
+                                                                        a.B, p.C, st - 1, i0, stride, spec_stride,
+                                                                        a.spec_C, a.spec_per_b);
+            kci<<<dim3(cblocks, unsigned(g)), kFC * (MH / 16), smC, s>>>(ws, tb, N1, 0, ws2_off, stride);
+            if (st < p.order - 1)
+                kca<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C, p.order, p.order - st - 1,
+                                                               N1 * H, i0, stride);
+            else
+                kc<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C, p.order, 0, N1 * H, i0, stride);
+        }
+    }
+    return cudaGetLastError();
+}
+
 // Engine choice per pass, measured on B=2, C=256, 256 x 256, bf16 (us per
 // call): CTA rows + register columns 843, register rows + register columns
 // 921, CTA rows + CTA columns 939, register rows + CTA columns 1020.
@@ -885,7 +1068,56 @@ cudaError_t dispatch_h_conv(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     }
 }
 
+template <int MW, int MH>
+cudaError_t dispatch_d(const Plan& p, const void* args, cudaStream_t s, bool spectrum) {
+    switch (p.L) {
+#define HYENA_3D_CASE(N)                                                                          \
+    case N:                                                                                       \
+        if (spectrum) return spectrum_3d_t<MW, MH, N>(p, *static_cast<const SpectrumArgs*>(args), s); \
+        {                                                                                         \
+            const ConvArgs& a = *static_cast<const ConvArgs*>(args);                              \
+            return a.dtype == DT_F32 ? conv_3d_t<MW, MH, N, float>(p, a, s)                      \
+                                     : conv_3d_t<MW, MH, N, __nv_bfloat16>(p, a, s);              \
+        }
+        HYENA_3D_CASE(16)
+        HYENA_3D_CASE(32)
+        HYENA_3D_CASE(64)
+        HYENA_3D_CASE(128)
+#undef HYENA_3D_CASE
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int MW>
+cudaError_t dispatch_3d_h(const Plan& p, const void* args, cudaStream_t s, bool spectrum) {
+    switch (p.H) {
+        case 16: return dispatch_d<MW, 16>(p, args, s, spectrum);
+        case 32: return dispatch_d<MW, 32>(p, args, s, spectrum);
+        case 64: return dispatch_d<MW, 64>(p, args, s, spectrum);
+        case 128: return dispatch_d<MW, 128>(p, args, s, spectrum);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t dispatch_3d(const Plan& p, const void* args, cudaStream_t s, bool spectrum) {
+    switch (p.W) {
+        case 16: return dispatch_3d_h<8>(p, args, s, spectrum);
+        case 32: return dispatch_3d_h<16>(p, args, s, spectrum);
+        case 64: return dispatch_3d_h<32>(p, args, s, spectrum);
+        case 128: return dispatch_3d_h<64>(p, args, s, spectrum);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_spectrum_3d(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    return dispatch_3d(p, &a, s, true);
+}
+
+cudaError_t launch_conv_3d(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    return dispatch_3d(p, &a, s, false);
+}
 
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     switch (p.W) {

@@ -50,6 +50,8 @@ cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cuda
 cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_spectrum_3d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+cudaError_t launch_conv_3d(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_shortconv(const void* u, void* out, const float* w, const float* bias, int64_t B,
                              int64_t Ctot, int64_t L, int dtype, cudaStream_t s);
 

@@ -122,8 +122,31 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
             p->spec_row_bytes = size_t(W + 1) * size_t(2 * H) * 8;
             p->ws_row_bytes = size_t(W + 1) * size_t(H) * 8;
         }
+    } else if (ndim == 3) {
+        const int64_t N1 = sizes[0], H = sizes[1], W = sizes[2];
+        if (!is_pow2(N1) || !is_pow2(H) || !is_pow2(W) || N1 < kMin3D || H < kMin3D || W < kMin3D ||
+            N1 > kMax3D || H > kMax3D || W > kMax3D) {
+            *why = "3-D sizes must be powers of two in [16, 128]";
+            return false;
+        }
+        p->path = PATH_GRID_3D;
+        p->L = N1;
+        p->H = H;
+        p->W = W;
+        p->n = N1 * H * W;
+        p->M1 = W / 2;
+        p->M2 = H;
+        p->t_fft_a = tb.add_fft(int(p->M1));
+        p->t_fft_b = tb.add_fft(int(p->M2));
+        p->t_twist = tb.add(W, 0, p->M1, 1, 1);                        // w_W^n, n < W/2
+        p->t_untangle = tb.add_untangle(W);
+        p->t_twist_h = tb.add(2 * H, 0, H, 1, 1);                      // w_2H^p, p < H
+        p->t_fft_d = tb.add_fft(int(N1));
+        p->t_twist_d = tb.add(2 * N1, 0, N1, 1, 1);                    // w_2N1^d, d < N1
+        p->spec_row_bytes = size_t(W + 1) * size_t(2 * H) * size_t(2 * N1) * 8;
+        p->ws_row_bytes = size_t(3) * size_t(W + 1) * size_t(H) * size_t(N1) * 8;   // ws1 + ws2
     } else {
-        *why = "ndim must be 1 or 2";
+        *why = "ndim must be 1, 2 or 3";
         return false;
     }
     if (!tb.ok) { *why = "internal: too many twiddle tables"; return false; }

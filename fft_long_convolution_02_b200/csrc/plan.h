@@ -27,6 +27,12 @@
 //                     W-point row FFT (packed, one W/2-point chain) and the
 //                     H-point column FFT.  Spectrum per channel = (W/2+1)
 //                     columns x H complex64.
+//   PATH_GRID_3D      3-D N1 x H x W (16..128 each), zero padded on every
+//                     axis: the 2-D row passes over N1 H rows, a forward and
+//                     an inverse column pass (2H points) and a depth pass
+//                     (2N1 points, spectrum multiply) between them.  Spectrum
+//                     per channel = (W+1) 2H depth lines x 2N1 complex64.
+//                     N1 is kept in the L field.
 #pragma once
 #include <stddef.h>
 #include <stdint.h>
@@ -35,7 +41,9 @@
 
 namespace hyena {
 
-enum Path { PATH_NONE = 0, PATH_ONCHIP_1D = 1, PATH_MULTIPASS_1D = 2, PATH_GRID_2D = 3, PATH_GRID_2D_CIRC = 4 };
+enum Path {
+    PATH_NONE = 0, PATH_ONCHIP_1D = 1, PATH_MULTIPASS_1D = 2, PATH_GRID_2D = 3, PATH_GRID_2D_CIRC = 4, PATH_GRID_3D = 5
+};
 
 // OR-ed into ndim (2-D only): the circular (periodic) form (HYENA_CIRCULAR).
 constexpr int kCircularFlag = 0x100;
@@ -50,6 +58,8 @@ constexpr int64_t kMaxL = int64_t(1) << 20;
 constexpr int64_t kMin1D = 16;
 constexpr int64_t kMin2D = 16;
 constexpr int64_t kMax2D = 512;
+constexpr int64_t kMin3D = 16;
+constexpr int64_t kMax3D = 128;
 constexpr int kMaxOrder = 8;
 
 struct SpecHeader {
@@ -83,6 +93,7 @@ struct Plan {
     // table offsets in float2 units from the start of the tables
     int64_t t_fft_a = 0, t_fft_b = 0, t_twist = 0, t_untangle = 0, t_four = 0;
     int64_t t_twist_hi = 0, t_twist_lo = 0, t_unt1 = 0, t_unt2 = 0, t_unt_c = 0, t_twist_h = 0;
+    int64_t t_fft_d = 0, t_twist_d = 0;   // 3-D depth axis
     TableSpecs specs{};
     size_t tables_off = kHeaderBytes;
     size_t spec_off = 0;

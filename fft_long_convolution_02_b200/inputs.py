@@ -25,6 +25,8 @@ widths and lengths the pages discuss):
   K[c,i,j] = N(0,1) exp(-(i^2+j^2)/(2 s_c^2)), s_c ~ U[8,128].
 * ``grid2d_circ`` as ``grid2d`` in the circular (periodic) 2-D form; the
   filter is the same Gaussian-windowed N(0,1) field on the H x W grid.
+* ``vol3d``    B=2 C=32 64x64x64 order 2, bf16, no short conv (3-D volumes).
+  K[c,a,i,j] = N(0,1) exp(-(a^2+i^2+j^2)/(2 s_c^2)), s_c ~ U[4,32].
 * ``d768_l8k_ps`` as ``d768_l8k`` with per-sample (input-dependent) filters:
   k and D drawn for every (b, c) row, filter index b*C + c.
 
@@ -48,9 +50,10 @@ class Problem:
     C: int
     order: int
     dtype: str                 # "f32" or "bf16" storage of u, k and y
-    L: int = 0                 # 1-D length (0 for 2-D)
-    H: int = 0                 # 2-D grid (0 for 1-D)
+    L: int = 0                 # 1-D length (0 for 2-D / 3-D)
+    H: int = 0                 # 2-D grid (0 for 1-D); 3-D: second axis
     W: int = 0
+    N1: int = 0                # 3-D: first axis (0 otherwise)
     shortconv: bool = True
     decay: tuple = (1.0, 8.0)  # a_c range (1-D)
     sigma: tuple = (8.0, 128.0)  # s_c range (2-D)
@@ -62,14 +65,16 @@ class Problem:
 
     @property
     def ndim(self) -> int:
-        return 2 if self.H else 1
+        return 3 if self.N1 else (2 if self.H else 1)
 
     @property
     def n(self) -> int:
-        return self.H * self.W if self.H else self.L
+        return self.N1 * self.H * self.W if self.N1 else (self.H * self.W if self.H else self.L)
 
     @property
     def shape(self) -> tuple:
+        if self.N1:
+            return (self.N1, self.H, self.W)
         return (self.H, self.W) if self.H else (self.L,)
 
     @property
@@ -101,6 +106,8 @@ WORKLOADS = {
                       shortconv=False, sigma=(8.0, 128.0), seed=20260004),
     "grid2d_circ": Problem("grid2d_circ", B=2, C=256, H=256, W=256, order=2, dtype="bf16",
                            shortconv=False, sigma=(8.0, 128.0), circular=True, seed=20260006),
+    "vol3d": Problem("vol3d", B=2, C=32, N1=64, H=64, W=64, order=2, dtype="bf16",
+                     shortconv=False, sigma=(4.0, 32.0), seed=20260007),
     "d768_l8k_ps": Problem("d768_l8k_ps", B=4, C=768, L=8192, order=2, dtype="bf16",
                            decay=(0.5, 6.0), per_sample=True, seed=20260005),
 }
@@ -167,6 +174,12 @@ def k_row(p: Problem, s: int, c: int) -> np.ndarray:
         env = np.exp(-a * t / p.L)
         return (g.standard_normal(p.L) * env).astype(np.float32)
     sig = g.uniform(p.sigma[0], p.sigma[1])
+    if p.ndim == 3:
+        a = np.arange(p.N1, dtype=np.float64)[:, None, None]
+        i = np.arange(p.H, dtype=np.float64)[None, :, None]
+        j = np.arange(p.W, dtype=np.float64)[None, None, :]
+        env = np.exp(-(a * a + i * i + j * j) / (2.0 * sig * sig))
+        return (g.standard_normal(p.shape) * env).astype(np.float32).reshape(-1)
     i = np.arange(p.H, dtype=np.float64)[:, None]
     j = np.arange(p.W, dtype=np.float64)[None, :]
     env = np.exp(-(i * i + j * j) / (2.0 * sig * sig))

@@ -62,7 +62,10 @@ typedef enum {
 } hyena_status_t;
 
 /*
- * ndim: 1 (L), 2 (H x W, non-circular: zero padded, output cropped), or
+ * ndim: 1 (L), 2 (H x W, non-circular: zero padded, output cropped),
+ * 3 (N1 x H x W volumes, each a power of two in [16, 128], non-circular:
+ * every axis zero padded to twice its length, kernel anchored at the origin,
+ * output cropped; [P5] 原生 ND 卷积 and 3-D medical volumes), or
  * 2 | HYENA_CIRCULAR (H x W, circular: periodic boundary, the filter on the
  * same H x W grid, v[p][q] = sum_{i,j} K[i][j] w[(p-i) mod H][(q-j) mod W] +
  * D w[p][q]).  Source: [P5] 方法论 (边界处理: circular convolution for

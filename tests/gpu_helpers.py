@@ -75,6 +75,8 @@ def row_rel_err(y_gpu_rows: np.ndarray, y_ref_rows: np.ndarray) -> np.ndarray:
 
 def oracle_for_rows(orc, p: I.Problem, rows, data=None, use_shortconv=True, method=0):
     u, k, D, w, b = I.oracle_rows(p, rows, data)
+    if p.ndim == 3:
+        return orc.hyena_rows3(u, k, D, method=2 if method == 0 else method)
     if not use_shortconv:
         w, b = None, None
     return orc.hyena_rows(u, k, D, w, b, ndim=p.ndim, method=method, circular=p.circular)

@@ -64,6 +64,12 @@ def test_spectrum_bytes_and_workspace(lib):
     assert 256 * 65 * 256 * 8 <= b < 256 * 65 * 256 * 8 + (1 << 20)
     assert lib.hyena_gated_fftconv_workspace_min_bytes(256, circ, _sz(256, 128), 2) == 65 * 256 * 8
     assert lib.hyena_spectrum_bytes(64, 1 | 0x100, _sz(1024), 2) == 0
+    # 3-D: (W+1) 2H depth lines x 2 N1 complex64 per channel; workspace 3 (W+1) H N1 complex64
+    b = lib.hyena_spectrum_bytes(8, 3, _sz(16, 32, 64), 2)
+    assert 8 * 65 * 64 * 32 * 8 <= b < 8 * 65 * 64 * 32 * 8 + (1 << 20)
+    assert lib.hyena_gated_fftconv_workspace_min_bytes(8, 3, _sz(16, 32, 64), 2) == 3 * 65 * 32 * 16 * 8
+    assert lib.hyena_spectrum_bytes(8, 3, _sz(8, 32, 64), 2) == 0
+    assert lib.hyena_spectrum_bytes(8, 3, _sz(16, 32, 256), 2) == 0
     # unsupported shapes
     for bad in [(1, _sz(12), 2), (1, _sz(8), 2), (1, _sz(1 << 21), 2), (2, _sz(16, 1024), 2),
                 (1, _sz(1024), 1), (1, _sz(1024), 9)]:
