@@ -24,7 +24,8 @@ STATUS = {0: "HYENA_OK", 1: "HYENA_ERR_INVALID_ARG", 2: "HYENA_ERR_UNSUPPORTED_S
 EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "hyena_spectrum_bytes",
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
            "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
-           "hyena_gated_fftconv_per_sample", "hyena_spectrum_check", "hyena_debug_conv_tc"]
+           "hyena_gated_fftconv_per_sample", "hyena_gated_fftconv_host", "hyena_spectrum_check",
+           "hyena_debug_conv_tc"]
 
 _lock = threading.Lock()
 _lib = None
@@ -70,6 +71,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hyena_gated_fftconv_per_sample.restype = ctypes.c_int
         lib.hyena_gated_fftconv_per_sample.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
                                                        ctypes.c_int, ctypes.c_int, vp, sz, vp]
+        lib.hyena_gated_fftconv_host.restype = ctypes.c_int
+        lib.hyena_gated_fftconv_host.argtypes = [vp, vp, vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
+                                                 ctypes.c_int, ctypes.c_int, vp, sz, i64, vp]
         lib.hyena_gated_fftconv_noalloc.restype = ctypes.c_int
         lib.hyena_gated_fftconv_noalloc.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
                                                     ctypes.c_int, ctypes.c_int, vp]
@@ -188,6 +192,22 @@ def hyena_gated_fftconv_per_sample(u, y, spectrum, sc_w, sc_bias, B: int, C: int
                                                  spectrum.numel() * spectrum.element_size(), _ptr(sc_w),
                                                  _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
                                                  _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def hyena_gated_fftconv_host(u_host, y_host, u_dev, y_dev, spectrum, sc_w, sc_bias, B: int, C: int, sizes,
+                             order: int, workspace=None, chunk_rows: int = 0, stream=None) -> None:
+    """u_host / y_host: CPU tensors (pinned for overlap); u_dev / y_dev: CUDA
+    tensors of the same shapes; the copies are pipelined against the kernels."""
+    if u_host.is_cuda or y_host.is_cuda:
+        raise ValueError("u_host and y_host must be host (CPU) tensors")
+    if not (u_host.is_contiguous() and y_host.is_contiguous()):
+        raise ValueError("u_host and y_host must be contiguous")
+    arr, nd = _sizes(sizes)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyena_gated_fftconv_host(u_host.data_ptr(), y_host.data_ptr(), _ptr(u_dev), _ptr(y_dev),
+                                           _ptr(spectrum), spectrum.numel() * spectrum.element_size(), _ptr(sc_w),
+                                           _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u_dev),
+                                           _ptr(workspace), ws_bytes, int(chunk_rows), _stream(stream)))
 
 
 def hyena_gated_fftconv_noalloc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int,

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
 
 #include "hyena.h"
@@ -263,6 +264,91 @@ hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum,
     a.wait_budget_ns = wait_budget_ns;
     a.issue_mma = issue_mma ? 1 : 0;
     return cuda_status(launch_conv_8192_tc(p, a, static_cast<cudaStream_t>(stream)), "tensor-core kernel");
+}
+
+}  // extern "C"
+
+namespace {
+
+// Per-device second stream and events of the host-buffer pipeline, created
+// on first use and kept for the life of the process.
+struct HostPipe {
+    cudaStream_t aux = nullptr;
+    cudaEvent_t entry = nullptr, aux_done = nullptr, conv_done[2] = {nullptr, nullptr};
+};
+constexpr int kMaxPipeDevices = 64;
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kMaxPipeDevices];
+
+cudaError_t host_pipe(int dev, HostPipe** out) {
+    HostPipe& hp = g_pipe[dev];
+    if (!hp.aux) {
+        cudaError_t e = cudaStreamCreateWithFlags(&hp.aux, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.aux_done, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.conv_done[0], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.conv_done[1], cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+    }
+    *out = &hp;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* u_dev, void* y_dev,
+                                        const void* spectrum, size_t spectrum_bytes, const float* sc_w,
+                                        const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes,
+                                        int order, hyena_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                        int64_t chunk_rows, void* stream) {
+    Plan p;
+    ConvArgs a;
+    hyena_status_t st = prepare_conv(u_dev, y_dev, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order,
+                                     dtype, workspace, workspace_bytes, &p, &a);
+    if (st != HYENA_OK) return st;
+    if (!u_host || !y_host) return fail(HYENA_ERR_INVALID_ARG, "u_host and y_host must not be NULL");
+    if (chunk_rows < 0) return fail(HYENA_ERR_INVALID_ARG, "chunk_rows must be >= 0 (0: default)");
+    const int64_t chunk = chunk_rows > 0 ? (chunk_rows < B ? chunk_rows : B) : (B + 3) / 4;
+    const size_t es = elem_size(dtype);
+    const size_t ub = size_t(order + 1) * size_t(C) * size_t(p.n) * es;    // u bytes per batch row
+    const size_t yb = size_t(C) * size_t(p.n) * es;                        // y bytes per batch row
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxPipeDevices) return fail(HYENA_ERR_INVALID_ARG, "device index beyond 64");
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    HostPipe* hp = nullptr;
+    e = host_pipe(dev, &hp);
+    if (e != cudaSuccess) return cuda_status(e, "host pipeline set-up");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaStream_t streams[2] = {s, hp->aux};
+    // the second stream starts after the work already queued on the caller's stream
+    e = cudaEventRecord(hp->entry, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->aux, hp->entry, 0);
+    const uint8_t* uh = static_cast<const uint8_t*>(u_host);
+    uint8_t* yh = static_cast<uint8_t*>(y_host);
+    uint8_t* ud = static_cast<uint8_t*>(u_dev);
+    uint8_t* yd = static_cast<uint8_t*>(y_dev);
+    int i = 0;
+    for (int64_t b0 = 0; b0 < B && e == cudaSuccess; b0 += chunk, ++i) {
+        const int64_t nb = B - b0 < chunk ? B - b0 : chunk;
+        cudaStream_t cs = streams[i & 1];
+        e = cudaMemcpyAsync(ud + b0 * ub, uh + b0 * ub, nb * ub, cudaMemcpyHostToDevice, cs);
+        // chunks share the workspace: their convolutions run one after another
+        if (e == cudaSuccess && i > 0 && p.ws_row_bytes > 0) e = cudaStreamWaitEvent(cs, hp->conv_done[(i - 1) & 1], 0);
+        if (e != cudaSuccess) break;
+        st = gated_fftconv(ud + b0 * ub, yd + b0 * yb, spectrum, spectrum_bytes, sc_w, sc_bias, nb, C, ndim, sizes,
+                           order, dtype, workspace, workspace_bytes, cs, false);
+        if (st != HYENA_OK) return st;
+        e = cudaEventRecord(hp->conv_done[i & 1], cs);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(yh + b0 * yb, yd + b0 * yb, nb * yb, cudaMemcpyDeviceToHost, cs);
+    }
+    // the caller's stream completes after every chunk
+    if (e == cudaSuccess) e = cudaEventRecord(hp->aux_done, hp->aux);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->aux_done, 0);
+    return cuda_status(e, "host pipeline");
 }
 
 hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,

@@ -192,6 +192,34 @@ hyena_status_t hyena_gated_fftconv_per_sample(const void* u, void* y, const void
                                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * hyena_gated_fftconv_host -- hyena_gated_fftconv on inputs and outputs that
+ * live in host memory, with the host<->device copies pipelined against the
+ * kernels.
+ *
+ * The paper has no counterpart: this entry point is for callers whose stream
+ * of inputs sits in host memory (serving, or data larger than the device).
+ * The batch is cut into chunks of chunk_rows batch rows (0: ceil(B/4)); each
+ * chunk is copied to u_dev, convolved and copied back to y_host, alternately
+ * on `stream` and on a second stream the library keeps per device, so one
+ * chunk's host-to-device copy overlaps the previous chunk's kernel and
+ * device-to-host copy.  Chunks share the workspace, so on the workspace paths
+ * their kernels run one after another.
+ *
+ *   u_host   [B, (order+1)*C, sizes...] host memory (page-locked for overlap;
+ *            pageable memory works but its copies do not overlap)
+ *   y_host   [B, C, sizes...] host memory, written when `stream` completes
+ *   u_dev, y_dev  device buffers of the full u and y sizes (caller-owned)
+ *   everything else as hyena_gated_fftconv (shared filters).
+ * Returns after queueing; the results are in y_host once `stream` completes.
+ * Argument errors are reported before anything is queued.
+ */
+hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* u_dev, void* y_dev,
+                                        const void* spectrum, size_t spectrum_bytes, const float* sc_w,
+                                        const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes,
+                                        int order, hyena_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                        int64_t chunk_rows, void* stream);
+
+/*
  * Size of the fixed scratch array used by hyena_gated_fftconv_noalloc (32 MiB).
  */
 #define HYENA_NOALLOC_SCRATCH_BYTES (32u << 20)

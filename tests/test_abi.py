@@ -122,6 +122,14 @@ def test_validation_errors_before_launch(lib):
     assert sc(fake, fake * 4, None, None, 1, 3, 64, 0, None) == 1
     assert sc(fake, fake * 4, fake * 8, None, 1, 3, 63, 0, None) == 2
     assert sc(fake, fake + 16, fake * 8, None, 1, 3, 64, 0, None) == 1
+    # host-buffer pipeline: device-side checks first, then the host pointers and chunk size
+    hp = lib.hyena_gated_fftconv_host
+    assert hp(fake, fake * 2, fake * 4 + 4, fake * 6, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0,
+              None, 0, 0, None) == 3
+    assert hp(None, fake * 2, fake * 4, fake * 6, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0,
+              None, 0, 0, None) == 1
+    assert hp(fake, fake * 2, fake * 4, fake * 6, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0,
+              None, 0, -1, None) == 1
     # tensor-core wait test hook: L = 8192 bf16 only, order <= 3, budget > 0
     dg = lib.hyena_debug_conv_tc
     n8 = lib.hyena_spectrum_bytes(4, 1, _sz(8192), 2)
