@@ -25,9 +25,10 @@
 // The spectrum row has the same shape: one float4 pair entry per workspace
 // complex pair, written in place by the spectrum build.
 //
-// Rows are processed in groups sized to the caller's workspace (default
-// about 96 MB, chosen by timing) so that much of the intermediate data stays
-// in the 126 MB L2 between passes.
+// Rows are processed in groups sized to the caller's workspace (by default
+// the whole batch up to 4 GiB: fewer launches and fewer partly filled last
+// waves measured faster than groups small enough to stay in the 126 MB L2).
+// With bf16 storage the workspace holds bf16 (re, im) pairs.
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"

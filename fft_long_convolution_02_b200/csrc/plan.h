@@ -15,9 +15,10 @@
 //                     L = 8192: all 2L bins, complex64, in the position
 //                     order of the tensor-core kernel (onchip_tc.cu).
 //   PATH_MULTIPASS_1D 32768 <= L <= 2^20: four-step M = M1 x M2 with three
-//                     passes through a caller workspace (kept L2-resident by
-//                     processing rows in groups).  Spectrum row = M1 units of
-//                     M2 float4 pair entries.
+//                     passes through a caller workspace (rows processed in
+//                     groups that fit it; by default the whole batch up to
+//                     4 GiB).  Spectrum row = M1 units of M2 float4 pair
+//                     entries.
 //   PATH_GRID_2D      2-D H x W (16..512 each), zero-padded to 2H x 2W: a row
 //                     pass (packed real FFT of each image row), a column pass
 //                     (2H-point FFT, spectrum multiply, inverse) and an
