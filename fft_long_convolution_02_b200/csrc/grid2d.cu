@@ -1,5 +1,7 @@
-// grid2d.cu -- the 2-D forms (H x W grids, 16..512 each): non-circular
-// (zero padded) and, further down, circular.
+// grid2d.cu -- the N-D forms: 2-D non-circular (zero padded, H x W grids of
+// 16..512 each), further down the 2-D circular form and the 3-D non-circular
+// form (N1 x H x W volumes of 16..128 per axis, reusing the row and column
+// engines).
 //
 // [P5] "Native Multi-Dimensional Subquadratic Operators via Input Dependent
 // Long Convolutions", 方法论 (原生 ND 卷积, 边界处理): the global convolution

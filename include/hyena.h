@@ -142,9 +142,10 @@ size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_
  *
  * Source: [P4] section 二.1 (split *x, v = uc.split(d_model); for o, x_i in
  * enumerate(reversed(x[1:])): v = v * x_i; v = fftconv(v, k[o], bias[o]);
- * y = v * x[0]); [P5] 方法论 for ndim = 2 (non-circular global convolution by
- * zero padding each axis to twice its length; output cropped to [0:H, 0:W],
- * kernel anchored at (0, 0)).
+ * y = v * x[0]); [P5] 方法论 for ndim = 2 and 3 (non-circular global
+ * convolution by zero padding each axis to twice its length; output cropped
+ * to the input grid, kernel anchored at the origin) and for
+ * ndim = 2 | HYENA_CIRCULAR (circular, periodic boundary).
  *
  *   u        [B, (order+1)*C, sizes...] projected stream, channel blocks in the
  *            order x0, x1, ..., x(order-1), v (dtype)
