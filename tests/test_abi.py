@@ -144,3 +144,40 @@ def test_validation_errors_before_launch(lib):
 def test_status_strings(lib):
     assert lib.hyena_status_string(8) == b"HYENA_ERR_TIMEOUT"
     assert lib.hyena_status_string(0) == b"HYENA_OK"
+
+
+def test_spectrum_and_workspace_sizes_every_path(lib):
+    """Byte counts of every path against their closed forms (header + tables
+    below 1 MiB), and the shapes each path refuses."""
+    hdr = 1 << 20
+    C, order = 4, 3
+    S = order - 1
+
+    def spec(nd, *sizes):
+        return lib.hyena_spectrum_bytes(C, nd, _sz(*sizes), order)
+
+    def wsmin(nd, *sizes):
+        return lib.hyena_gated_fftconv_workspace_min_bytes(C, nd, _sz(*sizes), order)
+
+    for L in (16, 64, 1024, 4096, 16384):                      # on-chip pair layout
+        assert S * C * (L // 2 + 1) * 16 <= spec(1, L) < S * C * (L // 2 + 1) * 16 + hdr
+        assert wsmin(1, L) == 0
+    assert S * C * 16 * 8192 <= spec(1, 8192) < S * C * 16 * 8192 + hdr   # two planes at L = 8192
+    for L in (1 << 15, 1 << 17, 1 << 20):                      # four-step
+        assert S * C * 8 * L <= spec(1, L) < S * C * 8 * L + (64 << 20)
+        assert wsmin(1, L) == 8 * L
+    for H, W in ((16, 16), (512, 32), (32, 512)):              # 2-D padded and circular
+        assert S * C * (W + 1) * 2 * H * 8 <= spec(2, H, W) < S * C * (W + 1) * 2 * H * 8 + hdr
+        assert wsmin(2, H, W) == (W + 1) * H * 8
+        circ = 2 | 0x100
+        assert S * C * (W // 2 + 1) * H * 8 <= spec(circ, H, W) < S * C * (W // 2 + 1) * H * 8 + hdr
+        assert wsmin(circ, H, W) == (W // 2 + 1) * H * 8
+    for N1, H, W in ((16, 16, 16), (128, 16, 32)):             # 3-D
+        lines = (W + 1) * 2 * H
+        assert S * C * lines * 2 * N1 * 8 <= spec(3, N1, H, W) < S * C * lines * 2 * N1 * 8 + hdr
+        assert wsmin(3, N1, H, W) == 3 * (W + 1) * H * N1 * 8
+    refused = [(1, (8,)), (1, (48,)), (1, (1 << 21,)), (2, (8, 16)), (2, (16, 1024)), (2, (24, 16)),
+               (3, (8, 16, 16)), (3, (16, 256, 16)), (1 | 0x100, (1024,)),
+               (3 | 0x100, (16, 16, 16)), (4, (16, 16, 16, 16))]
+    for nd, sizes in refused:
+        assert lib.hyena_spectrum_bytes(C, nd, _sz(*sizes), order) == 0, (nd, sizes)
