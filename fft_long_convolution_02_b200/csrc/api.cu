@@ -341,13 +341,16 @@ hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* 
         if (e != cudaSuccess) break;
         st = gated_fftconv(ud + b0 * ub, yd + b0 * yb, spectrum, spectrum_bytes, sc_w, sc_bias, nb, C, ndim, sizes,
                            order, dtype, workspace, workspace_bytes, cs, false);
-        if (st != HYENA_OK) return st;
+        if (st != HYENA_OK) break;
         e = cudaEventRecord(hp->conv_done[i & 1], cs);
         if (e == cudaSuccess) e = cudaMemcpyAsync(yh + b0 * yb, yd + b0 * yb, nb * yb, cudaMemcpyDeviceToHost, cs);
     }
-    // the caller's stream completes after every chunk
-    if (e == cudaSuccess) e = cudaEventRecord(hp->aux_done, hp->aux);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->aux_done, 0);
+    // the caller's stream completes after every chunk queued on the second
+    // stream, also when queueing stopped early on an error
+    cudaError_t ej = cudaEventRecord(hp->aux_done, hp->aux);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp->aux_done, 0);
+    if (st != HYENA_OK) return st;
+    if (e == cudaSuccess) e = ej;
     return cuda_status(e, "host pipeline");
 }
 
