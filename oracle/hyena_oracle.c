@@ -21,7 +21,7 @@
  *       边界处理): the N-D global convolution is evaluated with an N-D FFT;
  *       the non-circular form zero-pads every axis to twice its length.
  *
- * Readings of points the pages leave open (listed again in the design doc):
+ * Readings of points the pages leave open:
  *  - fftconv(x, k, D) = (k * x)[0:L] + D * x  (causal linear convolution plus
  *    a per-channel skip); evaluated either by its direct sum or by a
  *    zero-padded FFT of size >= 2L.
