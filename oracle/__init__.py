@@ -20,7 +20,12 @@ ctypes.  Sources, per function:
 * ``hyena_rows`` -- [P4] section 二.1, ``HyenaOperator.forward``: split into
   gates and value, ``for o, x_i in enumerate(reversed(x[1:]))`` gate then
   long conv, output gate ``y = v * x[0]``.
+* ``conv2d_circ_*`` -- [P5] 边界处理: the circular (periodic) 2-D form.
+* ``conv3d_*`` / ``hyena_rows3`` -- [P5] 原生 ND 卷积: the 3-D form.
 * ``fft`` -- a hand-written iterative radix-2 FFT (the textbook algorithm).
+* ``filter_gen`` (submodule) -- [P4] section 二.2: the implicit filter
+  (positional embedding -> MLP with Sin -> exponential modulation), plain
+  numpy in float64.
 """
 from __future__ import annotations
 
