@@ -2,7 +2,10 @@
 
 This module is shared by the tests, the benchmark and the oracle checks.  It
 holds none of the operator's arithmetic: it only draws random numbers and
-rounds them to the storage type.
+rounds them to the storage type, producing tensors in the layouts of the C
+ABI (u [B, (order+1)*C, ...], k [order-1, FC, ...], D [order-1, FC], taps
+[(order+1)*C, 3]).  How a (b, c) row reads its chunks from them (the split)
+is part of the operator and lives in the oracle.
 
 Every row of every tensor has its own counter-keyed numpy PCG64 stream,
 ``SeedSequence([seed, tag, i, j])``, so any row can be produced without
@@ -85,9 +88,6 @@ class Problem:
     def FC(self) -> int:
         """Filter channels: C, or B*C with per-sample filters (index b*C + c)."""
         return self.B * self.C if self.per_sample else self.C
-
-    def filter_index(self, b: int, c: int) -> int:
-        return b * self.C + c if self.per_sample else c
 
     def with_(self, **kw) -> "Problem":
         return replace(self, **kw)
@@ -226,45 +226,3 @@ def make_k(p: Problem) -> np.ndarray:
 
 def make_all(p: Problem) -> dict:
     return {"u": make_u(p), "k": make_k(p), "D": D_all(p), "sc_w": sc_w_all(p), "sc_b": sc_b_all(p)}
-
-
-def oracle_rows(p: Problem, rows, data: dict | None = None):
-    """Float64 self-contained rows (the oracle's input format) for row ids b*C + c.
-
-    When ``data`` (from make_all) is given the rows are cut from it; otherwise
-    they are generated directly, which is how large workloads are sampled.
-    Returns u_rows [R, order+1, *shape], k_rows [R, order-1, *shape],
-    D_rows [R, order-1], sc_w_rows [R, order+1, 3] or None, sc_b_rows or None.
-    """
-    rows = np.asarray(rows, dtype=np.int64)
-    R = rows.size
-    u_rows = np.empty((R, p.order + 1) + p.shape, dtype=np.float64)
-    k_rows = np.empty((R, p.order - 1) + p.shape, dtype=np.float64)
-    D = D_all(p)
-    scw = sc_w_all(p)
-    scb = sc_b_all(p)
-    cache: dict = {}
-    kcache: dict = {}
-    for i, r in enumerate(rows):
-        b, c = int(r) // p.C, int(r) % p.C
-        for j in range(p.order + 1):
-            ch = j * p.C + c
-            if data is not None:
-                u_rows[i, j] = stored_values(p, data["u"][b, ch])
-            else:
-                u_rows[i, j] = stored_values(p, store(p, u_row(p, b, ch, cache))).reshape(p.shape)
-        fi = p.filter_index(b, c)
-        for s in range(p.order - 1):
-            if data is not None:
-                k_rows[i, s] = stored_values(p, data["k"][s, fi])
-            else:
-                key = (s, fi)
-                if key not in kcache:
-                    kcache[key] = stored_values(p, store(p, k_row(p, s, fi))).reshape(p.shape)
-                k_rows[i, s] = kcache[key]
-    fis = np.array([p.filter_index(int(r) // p.C, int(r) % p.C) for r in rows], dtype=np.int64)
-    D_rows = D[:, fis].T.astype(np.float64)
-    chans = np.arange(p.order + 1)[None, :] * p.C + (rows % p.C)[:, None]
-    scw_rows = None if scw is None else scw[chans].astype(np.float64)
-    scb_rows = None if scb is None else scb[chans].astype(np.float64)
-    return u_rows, k_rows, D_rows, scw_rows, scb_rows

@@ -17,9 +17,18 @@ ctypes.  Sources, per function:
   Subquadratic Operators via Input Dependent Long Convolutions", 方法论
   (原生 ND 卷积, 边界处理): N-D FFT convolution, non-circular by zero-padding
   each axis to twice its length.
-* ``hyena_rows`` -- [P4] section 二.1, ``HyenaOperator.forward``: split into
-  gates and value, ``for o, x_i in enumerate(reversed(x[1:]))`` gate then
-  long conv, output gate ``y = v * x[0]``.
+* ``split_rows`` -- [P4] section 二.1, ``*x, v = uc.split(d_model, dim=1)``:
+  chunk j of row (b, c) of the stacked stream is channel j*C + c (taps and
+  bias alike); filters at index c, or b*C + c for per-sample filters.
+* ``hyena_rows`` -- [P4] section 二.1, ``HyenaOperator.forward`` on one row's
+  chunks: ``for o, x_i in enumerate(reversed(x[1:]))`` gate then long conv,
+  output gate ``y = v * x[0]``.
+* ``hyena_stacked`` -- the two above on the stacked tensors the CUDA path
+  receives.
+* ``in_proj`` / ``out_proj`` -- [P4] section 二.1: ``in_proj =
+  nn.Linear(d_model, (order+1) d_model)`` followed by ``rearrange(u, 'b l d
+  -> b d l')``, and ``out_proj = nn.Linear(d_model, d_model)`` applied to
+  ``rearrange(y, 'b d l -> b l d')`` (``nn.Linear(x) = x W^T + bias``).
 * ``conv2d_circ_*`` -- [P5] 边界处理: the circular (periodic) 2-D form.
 * ``conv3d_*`` / ``hyena_rows3`` -- [P5] 原生 ND 卷积: the 3-D form.
 * ``fft`` -- a hand-written iterative radix-2 FFT (the textbook algorithm).
@@ -88,6 +97,12 @@ class Oracle:
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _dp]
         lib.oracle_hyena_rows.restype = ctypes.c_int
+        lib.oracle_split_rows.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, _dp, _dp,
+                                          _dp, _i64, _i64, ctypes.c_int, _i64, ctypes.c_int,
+                                          ctypes.POINTER(_i64), _i64, _dp, _dp, _dp, _dp, _dp]
+        lib.oracle_split_rows.restype = ctypes.c_int
+        lib.oracle_in_proj.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, _dp]
+        lib.oracle_out_proj.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _i64, _dp]
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -217,6 +232,118 @@ class Oracle:
             raise ValueError("oracle_hyena_rows rejected its arguments")
         return y.reshape((R, W) if ndim == 1 else (R, H, W))
 
+    def split_rows(self, u, k, D, sc_w=None, sc_b=None, *, B: int, C: int, order: int, shape,
+                   rows=None, per_sample: bool = False):
+        """The split of the stacked projected stream ([P4] 二.1,
+        ``*x, v = uc.split(d_model, dim=1)``), done by ``oracle_split_rows``.
+
+        u    : [B, (order+1)*C, *shape] -- float64, float32, or uint16 holding
+               bfloat16 bit patterns (exact values are used)
+        k    : [order-1, FC, *shape] (same element kinds); FC = C, or B*C with
+               per_sample (filter of row (b, c) at index b*C + c)
+        D    : [order-1, FC] or None;  sc_w: [(order+1)*C, 3] or None;
+        sc_b : [(order+1)*C] or None
+        rows : row ids b*C + c (default: all B*C rows in order)
+        Returns the self-contained rows of ``hyena_rows``: u_rows
+        [R, order+1, *shape], k_rows [R, order-1, *shape], D_rows
+        [R, order-1], sc_w_rows [R, order+1, 3] or None, sc_b_rows or None.
+        """
+        shape = tuple(int(x) for x in shape)
+        n = int(np.prod(shape))
+        rows = np.ascontiguousarray(np.arange(B * C) if rows is None else rows, dtype=np.int64).reshape(-1)
+        R = rows.size
+        FC = B * C if per_sample else C
+        u = np.ascontiguousarray(u)
+        k = np.ascontiguousarray(k)
+        if u.shape != (B, (order + 1) * C) + shape:
+            raise ValueError(f"u must be [B, (order+1)*C, *shape] = {(B, (order + 1) * C) + shape}, got {u.shape}")
+        if k.shape != (order - 1, FC) + shape:
+            raise ValueError(f"k must be [order-1, FC, *shape] = {(order - 1, FC) + shape}, got {k.shape}")
+        Dd = None if D is None else _f64(D)
+        if Dd is not None and Dd.shape != (order - 1, FC):
+            raise ValueError("D must be [order-1, FC]")
+        scw = None if sc_w is None else _f64(sc_w)
+        scb = None if (sc_w is None or sc_b is None) else _f64(sc_b)
+        if scw is not None and scw.shape != ((order + 1) * C, 3):
+            raise ValueError("sc_w must be [(order+1)*C, 3]")
+        u_rows = np.empty((R, order + 1) + shape, dtype=np.float64)
+        k_rows = np.empty((R, order - 1) + shape, dtype=np.float64)
+        D_rows = np.empty((R, order - 1), dtype=np.float64)
+        scw_rows = np.empty((R, order + 1, 3), dtype=np.float64) if scw is not None else None
+        scb_rows = np.empty((R, order + 1), dtype=np.float64) if scw is not None else None
+        rc = self.lib.oracle_split_rows(u.ctypes.data, _kind(u), k.ctypes.data, _kind(k), _ptr(Dd), _ptr(scw),
+                                        _ptr(scb), B, C, order, n, 1 if per_sample else 0,
+                                        rows.ctypes.data_as(ctypes.POINTER(_i64)), R, _ptr(u_rows),
+                                        _ptr(k_rows), _ptr(D_rows), _ptr(scw_rows), _ptr(scb_rows))
+        if rc != 0:
+            raise ValueError("oracle_split_rows rejected its arguments")
+        return u_rows, k_rows, D_rows, scw_rows, scb_rows
+
+    def hyena_stacked(self, u, k, D, sc_w=None, sc_b=None, *, B: int, C: int, order: int, shape,
+                      rows=None, per_sample: bool = False, circular: bool = False, method: int = 0,
+                      nthreads: int = 0) -> np.ndarray:
+        """The operator on the stacked tensors the CUDA path receives
+        (u [B, (order+1)*C, *shape] -> y rows [R, *shape], R = len(rows),
+        default all B*C rows in order b*C + c): ``split_rows`` followed by
+        ``hyena_rows`` (1-D, 2-D) or ``hyena_rows3`` (3-D)."""
+        shape = tuple(int(x) for x in shape)
+        u_rows, k_rows, D_rows, w, b = self.split_rows(u, k, D, sc_w, sc_b, B=B, C=C, order=order, shape=shape,
+                                                       rows=rows, per_sample=per_sample)
+        if len(shape) == 3:
+            if w is not None:
+                raise ValueError("the 3-D form has no short conv")
+            return self.hyena_rows3(u_rows, k_rows, D_rows, method=2 if method == 0 else method,
+                                    nthreads=nthreads)
+        return self.hyena_rows(u_rows, k_rows, D_rows, w, b, ndim=len(shape), method=method, nthreads=nthreads,
+                               circular=circular)
+
+    def in_proj(self, x, W, bias=None) -> np.ndarray:
+        """x [B, L, D], W [J, D] (nn.Linear weight), bias [J] or None ->
+        u [B, J, L] = rearrange(x W^T + bias, 'b l d -> b d l').  Arrays may
+        be float64, float32 or uint16 bfloat16 bit patterns."""
+        x = _values(x); W = _values(W)
+        B, L, D = x.shape
+        J = W.shape[0]
+        if W.shape != (J, D):
+            raise ValueError("W must be [J, D]")
+        b = None if bias is None else _f64(bias)
+        u = np.empty((B, J, L), dtype=np.float64)
+        self.lib.oracle_in_proj(_ptr(x), _ptr(W), _ptr(b), B, L, D, J, _ptr(u))
+        return u
+
+    def out_proj(self, y, W, bias=None) -> np.ndarray:
+        """y [B, D, L], W [J, D], bias [J] or None -> out [B, L, J] =
+        rearrange(y, 'b d l -> b l d') W^T + bias."""
+        y = _values(y); W = _values(W)
+        B, D, L = y.shape
+        J = W.shape[0]
+        if W.shape != (J, D):
+            raise ValueError("W must be [J, D]")
+        b = None if bias is None else _f64(bias)
+        out = np.empty((B, L, J), dtype=np.float64)
+        self.lib.oracle_out_proj(_ptr(y), _ptr(W), _ptr(b), B, L, D, J, _ptr(out))
+        return out
+
+
+def _values(a) -> np.ndarray:
+    """Exact float64 values of an array of float64, float32 or uint16
+    bfloat16 bit patterns (the upper 16 bits of an IEEE binary32)."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64))
+    return _f64(a)
+
+
+def _kind(a: np.ndarray) -> int:
+    """Element kind of a stacked tensor for oracle_split_rows."""
+    if a.dtype == np.float64:
+        return 0
+    if a.dtype == np.float32:
+        return 1
+    if a.dtype == np.uint16:
+        return 2          # bfloat16 bit patterns
+    raise ValueError(f"unsupported element type {a.dtype} (float64, float32 or uint16 bf16 bits)")
+
 
 def default() -> Oracle:
     """The oracle built from hyena_oracle.c as committed."""
@@ -277,3 +404,19 @@ def hyena_rows3(u_rows, k_rows, D_rows, **kw):
 
 def hyena_rows(u_rows, k_rows, D_rows, sc_w_rows=None, sc_b_rows=None, **kw):
     return default().hyena_rows(u_rows, k_rows, D_rows, sc_w_rows, sc_b_rows, **kw)
+
+
+def split_rows(u, k, D, sc_w=None, sc_b=None, **kw):
+    return default().split_rows(u, k, D, sc_w, sc_b, **kw)
+
+
+def hyena_stacked(u, k, D, sc_w=None, sc_b=None, **kw):
+    return default().hyena_stacked(u, k, D, sc_w, sc_b, **kw)
+
+
+def in_proj(x, W, bias=None):
+    return default().in_proj(x, W, bias)
+
+
+def out_proj(y, W, bias=None):
+    return default().out_proj(y, W, bias)

@@ -475,6 +475,117 @@ int oracle_hyena_rows(const double *u_rows, const double *k_rows, const double *
     return 0;
 }
 
+/* ---------------------------------------------------------------------- */
+/* Split of the projected stream ([P4] 二.1: after in_proj and the short   */
+/* filter the stream u[b][(order+1) d][l] is cut along the channel axis   */
+/* into blocks of d, `*x, v = uc.split(d_model, dim=1)`, so x_0..x_(order-1) */
+/* come first and v last).  Chunk j of row (b, c) is channel j*C + c of   */
+/* batch b.  The short filter is depthwise over all (order+1) C channels, */
+/* so its taps and bias split the same way.  The long filters            */
+/* k[order-1][FC][n] and skips D[order-1][FC] of step s are taken at      */
+/* index c (shared by the batch, [P4] 二.1 'l (o d) -> o d l'), or at     */
+/* b*C + c when every sample brings its own filters ([P5] 方法论, input-   */
+/* dependent kernels; FC = B*C).                                          */
+/*                                                                        */
+/* Stored values are read exactly: kind 0 = float64, 1 = float32,         */
+/* 2 = bfloat16 bit patterns (the upper 16 bits of an IEEE binary32).     */
+/* ---------------------------------------------------------------------- */
+static double stored_value(const void *base, int kind, int64_t i)
+{
+    if (kind == 0) return ((const double *)base)[i];
+    if (kind == 1) return (double)((const float *)base)[i];
+    uint32_t bits = (uint32_t)((const uint16_t *)base)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Gathers the self-contained rows (layouts of oracle_hyena_rows) of the
+ * listed row ids r = b*C + c from the stacked tensors.
+ *   u     [B][(order+1)*C][n] (u_kind)      k  [order-1][FC][n] (k_kind)
+ *   D     [order-1][FC] or NULL (= 0)       sc_w [(order+1)*C][3] or NULL,
+ *   sc_b  [(order+1)*C] or NULL (= 0)
+ * Outputs: u_rows [R][order+1][n], k_rows [R][order-1][n], D_rows
+ * [R][order-1], scw_rows [R][order+1][3] and scb_rows [R][order+1] (both
+ * only when sc_w is given).  Returns 0, or -1 on bad arguments.
+ */
+int oracle_split_rows(const void *u, int u_kind, const void *k, int k_kind, const double *D,
+                      const double *sc_w, const double *sc_b, int64_t B, int64_t C, int order,
+                      int64_t n, int per_sample, const int64_t *rows, int64_t nrows,
+                      double *u_rows, double *k_rows, double *D_rows, double *scw_rows,
+                      double *scb_rows)
+{
+    if (!u || !k || !rows || !u_rows || !k_rows || !D_rows || B < 1 || C < 1 || order < 2 || n < 1)
+        return -1;
+    if (u_kind < 0 || u_kind > 2 || k_kind < 0 || k_kind > 2) return -1;
+    if (sc_w && (!scw_rows || !scb_rows)) return -1;
+    const int64_t Ctot = (int64_t)(order + 1) * C;
+    const int64_t FC = per_sample ? B * C : C;
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t r = rows[i];
+        if (r < 0 || r >= B * C) return -1;
+        const int64_t b = r / C, c = r % C;
+        for (int j = 0; j <= order; ++j) {
+            const int64_t ch = (int64_t)j * C + c;             /* block j, channel c */
+            const int64_t src = (b * Ctot + ch) * n;
+            double *dst = u_rows + (i * (order + 1) + j) * n;
+            for (int64_t t = 0; t < n; ++t) dst[t] = stored_value(u, u_kind, src + t);
+            if (sc_w) {
+                for (int m = 0; m < 3; ++m) scw_rows[(i * (order + 1) + j) * 3 + m] = sc_w[ch * 3 + m];
+                scb_rows[i * (order + 1) + j] = sc_b ? sc_b[ch] : 0.0;
+            }
+        }
+        const int64_t f = per_sample ? b * C + c : c;          /* filter index */
+        for (int s = 0; s < order - 1; ++s) {
+            const int64_t src = ((int64_t)s * FC + f) * n;
+            double *dst = k_rows + (i * (order - 1) + s) * n;
+            for (int64_t t = 0; t < n; ++t) dst[t] = stored_value(k, k_kind, src + t);
+            D_rows[i * (order - 1) + s] = D ? D[(int64_t)s * FC + f] : 0.0;
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Projections around the operator ([P4] 二.1, HyenaOperator: in_proj =   */
+/* nn.Linear(d_model, (order+1) d_model) on u[b][l][:], then              */
+/* rearrange 'b l d -> b d l'; at the end y = rearrange(v * x[0],         */
+/* 'b d l -> b l d') and out_proj = nn.Linear(d_model, d_model)).          */
+/* nn.Linear(x) = x W^T + bias with the weight stored W[out][in].          */
+/* ---------------------------------------------------------------------- */
+/* x [B][L][D] -> u [B][J][L]:  u[b][j][l] = sum_i x[b][l][i] W[j][i] + bias[j] */
+void oracle_in_proj(const double *x, const double *W, const double *bias, int64_t B, int64_t L,
+                    int64_t D, int64_t J, double *u)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t j = 0; j < J; ++j) {
+            for (int64_t l = 0; l < L; ++l) {
+                double acc = bias ? bias[j] : 0.0;
+                for (int64_t i = 0; i < D; ++i) acc += x[(b * L + l) * D + i] * W[j * D + i];
+                u[(b * J + j) * L + l] = acc;
+            }
+        }
+    }
+}
+
+/* y [B][D][L] -> out [B][L][J]:  out[b][l][j] = sum_i y[b][i][l] W[j][i] + bias[j] */
+void oracle_out_proj(const double *y, const double *W, const double *bias, int64_t B, int64_t L,
+                     int64_t D, int64_t J, double *out)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t l = 0; l < L; ++l) {
+            for (int64_t j = 0; j < J; ++j) {
+                double acc = bias ? bias[j] : 0.0;
+                for (int64_t i = 0; i < D; ++i) acc += y[(b * D + i) * L + l] * W[j * D + i];
+                out[(b * L + l) * J + j] = acc;
+            }
+        }
+    }
+}
+
 /* Number of threads an OpenMP parallel region would use. */
 int oracle_max_threads(void)
 {

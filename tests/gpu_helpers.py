@@ -73,13 +73,13 @@ def row_rel_err(y_gpu_rows: np.ndarray, y_ref_rows: np.ndarray) -> np.ndarray:
     return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-300)
 
 
-def oracle_for_rows(orc, p: I.Problem, rows, data=None, use_shortconv=True, method=0):
-    u, k, D, w, b = I.oracle_rows(p, rows, data)
-    if p.ndim == 3:
-        return orc.hyena_rows3(u, k, D, method=2 if method == 0 else method)
-    if not use_shortconv:
-        w, b = None, None
-    return orc.hyena_rows(u, k, D, w, b, ndim=p.ndim, method=method, circular=p.circular)
+def oracle_for_rows(orc, p: I.Problem, rows, data, use_shortconv=True, method=0):
+    """The oracle's y for row ids b*C + c of the stacked tensors in ``data``
+    (from inputs.make_all): the oracle does the split itself."""
+    w = data["sc_w"] if use_shortconv else None
+    b = data.get("sc_b") if use_shortconv else None
+    return orc.hyena_stacked(data["u"], data["k"], data["D"], w, b, B=p.B, C=p.C, order=p.order, shape=p.shape,
+                             rows=rows, per_sample=p.per_sample, circular=p.circular, method=method)
 
 
 def gpu_rows(y: np.ndarray, p: I.Problem, rows) -> np.ndarray:

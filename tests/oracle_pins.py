@@ -106,6 +106,122 @@ def pin_golden_operator2d(orc):
                f"2-D operator golden, method {method}")
 
 
+def pin_golden_split_order3(orc):
+    """Stacked [B, (order+1) C, L] -> chunk j of channel c is channel j*C + c."""
+    g = _golden("operator_split_order3_c2.json")
+    u = np.array(g["u"], float)
+    k = np.array(g["k"], float)
+    D = np.array(g["D"], float)
+    want = np.array(g["expected"], float).reshape(g["B"] * g["C"], -1)
+    for method in (1, 2):
+        y = orc.hyena_stacked(u, k, D, B=g["B"], C=g["C"], order=g["order"], shape=u.shape[2:], method=method)
+        _close(y, want, 1e-13, f"split golden (order 3), method {method}")
+
+
+def pin_golden_split_taps(orc):
+    """Short-conv taps and bias of chunk j of channel c are those of channel j*C + c."""
+    g = _golden("operator_split_taps_order2_c2.json")
+    u = np.array(g["u"], float)
+    want = np.array(g["expected"], float).reshape(g["B"] * g["C"], -1)
+    for method in (1, 2):
+        y = orc.hyena_stacked(u, np.array(g["k"], float), np.array(g["D"], float), np.array(g["sc_w"], float),
+                              np.array(g["sc_b"], float), B=g["B"], C=g["C"], order=g["order"],
+                              shape=u.shape[2:], method=method)
+        _close(y, want, 1e-13, f"split taps golden, method {method}")
+
+
+def pin_split_batches_rows_and_storage(orc):
+    """Batch b of a stacked call equals a call on u[b] alone; a row subset
+    equals those rows of the full call; bf16 bit patterns decode to the same
+    values as float32 (values chosen exactly representable in bf16)."""
+    rng = np.random.default_rng(21)
+    B, C, order, L = 3, 4, 3, 32
+    u = rng.integers(-8, 9, size=(B, (order + 1) * C, L)).astype(np.float32) / 4
+    k = rng.integers(-8, 9, size=(order - 1, C, L)).astype(np.float32) / 8
+    D = rng.standard_normal((order - 1, C))
+    w = rng.standard_normal(((order + 1) * C, 3))
+    bias = rng.standard_normal((order + 1) * C)
+    kw = dict(C=C, order=order, shape=(L,), method=1)
+    full = orc.hyena_stacked(u, k, D, w, bias, B=B, **kw).reshape(B, C, L)
+    for b in range(B):
+        one = orc.hyena_stacked(u[b:b + 1], k, D, w, bias, B=1, **kw).reshape(C, L)
+        _close(full[b], one, 0.0, f"batch {b} on its own")
+    rows = np.array([7, 0, 11, 5])
+    sub = orc.hyena_stacked(u, k, D, w, bias, B=B, rows=rows, **kw)
+    _close(sub, full.reshape(B * C, L)[rows], 0.0, "row subset")
+    ubits = (u.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    kbits = (k.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    assert np.array_equal((ubits.astype(np.uint32) << np.uint32(16)).view(np.float32), u)
+    viabits = orc.hyena_stacked(ubits, kbits, D, w, bias, B=B, **kw).reshape(B, C, L)
+    _close(viabits, full, 0.0, "bf16 bit patterns")
+
+
+def pin_split_per_sample_filters(orc):
+    """Per-sample filters: row (b, c) takes filter b*C + c.  Filters repeated
+    over the batch give the shared-filter result, and batch b equals a
+    shared-filter call with the filters of sample b."""
+    rng = np.random.default_rng(22)
+    B, C, order, L = 2, 3, 3, 16
+    u = rng.standard_normal((B, (order + 1) * C, L))
+    k = rng.standard_normal((order - 1, B * C, L))
+    D = rng.standard_normal((order - 1, B * C))
+    w = rng.standard_normal(((order + 1) * C, 3))
+    kw = dict(C=C, order=order, shape=(L,), method=1)
+    ps = orc.hyena_stacked(u, k, D, w, B=B, per_sample=True, **kw).reshape(B, C, L)
+    for b in range(B):
+        shared = orc.hyena_stacked(u[b:b + 1], k[:, b * C:(b + 1) * C], D[:, b * C:(b + 1) * C], w, B=1,
+                                   **kw).reshape(C, L)
+        _close(ps[b], shared, 0.0, f"per-sample filters of sample {b}")
+    k_rep = np.concatenate([k[:, :C]] * B, axis=1)
+    D_rep = np.concatenate([D[:, :C]] * B, axis=1)
+    _close(orc.hyena_stacked(u, k_rep, D_rep, w, B=B, per_sample=True, **kw),
+           orc.hyena_stacked(u, k[:, :C], D[:, :C], w, B=B, **kw), 0.0, "repeated per-sample = shared")
+
+
+def pin_golden_projections(orc):
+    """in_proj with its 'b l d -> b d l' rearrangement and out_proj on the
+    rearranged y, against a hand-derived example."""
+    g = _golden("projections_2x2.json")
+    a = g["in_proj"]
+    _close(orc.in_proj(np.array(a["x"], float), np.array(a["W"], float), np.array(a["bias"], float)),
+           a["expected"], 1e-15, "in_proj golden")
+    b = g["out_proj"]
+    _close(orc.out_proj(np.array(b["y"], float), np.array(b["W"], float), np.array(b["bias"], float)),
+           b["expected"], 1e-15, "out_proj golden")
+
+
+def pin_projections_match_numpy(orc):
+    """Random shapes against numpy's matmul (a library special case), with and
+    without bias, and bf16 bit patterns decoded exactly."""
+    rng = np.random.default_rng(31)
+    for B, L, D, J in ((1, 5, 3, 7), (2, 16, 8, 24), (3, 9, 16, 16)):
+        x = rng.standard_normal((B, L, D)); W = rng.standard_normal((J, D)); bias = rng.standard_normal(J)
+        _close(orc.in_proj(x, W, bias), np.einsum("bld,jd->bjl", x, W) + bias[None, :, None], 1e-12, "in_proj")
+        _close(orc.in_proj(x, W), np.matmul(x, W.T).transpose(0, 2, 1), 1e-12, "in_proj no bias")
+        y = rng.standard_normal((B, D, L)); W2 = rng.standard_normal((J, D))
+        _close(orc.out_proj(y, W2, bias), np.matmul(y.transpose(0, 2, 1), W2.T) + bias, 1e-12, "out_proj")
+    xq = (rng.integers(-64, 64, size=(2, 8, 4)) / 16).astype(np.float32)
+    Wq = (rng.integers(-64, 64, size=(6, 4)) / 16).astype(np.float32)
+    bits = lambda a: (a.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    _close(orc.in_proj(bits(xq), bits(Wq)), orc.in_proj(xq, Wq), 0.0, "in_proj on bf16 bits")
+
+
+def pin_layer_with_identity_projections(orc):
+    """W_in = [I; I; I] copies x into every chunk and W_out = I: the layer is
+    then the operator on the stacked x^T (the projections compose with the
+    split in the order [P4] 二.1 gives)."""
+    rng = np.random.default_rng(32)
+    B, L, D, order = 2, 16, 3, 2
+    x = rng.standard_normal((B, L, D))
+    W_in = np.concatenate([np.eye(D)] * (order + 1), axis=0)
+    k = rng.standard_normal((order - 1, D, L)); Dk = rng.standard_normal((order - 1, D))
+    u = orc.in_proj(x, W_in)
+    _close(u, np.concatenate([x.transpose(0, 2, 1)] * (order + 1), axis=1), 0.0, "identity in_proj")
+    y = orc.hyena_stacked(u, k, Dk, B=B, C=D, order=order, shape=(L,), method=1).reshape(B, D, L)
+    out = orc.out_proj(y, np.eye(D))
+    _close(out, y.transpose(0, 2, 1), 0.0, "identity out_proj")
+
+
 # ---------------------------------------------------------- closed forms ---
 def pin_geometric_filter_closed_form(orc):
     """k[t] = r^t, x = 1  ->  out[t] = (1 - r^(t+1)) / (1 - r) + D."""

@@ -28,7 +28,9 @@ def _worker(rank, world, port, outdir):
     p = I.WORKLOADS["tiny"].with_(B=2, C=7, L=256, seed=7001)
     c0, c1 = hd.channel_shard(p.C, world, rank)
     rows = np.array([b * p.C + c for b in range(p.B) for c in range(c0, c1)], dtype=np.int64)
-    y = oracle.hyena_rows(*I.oracle_rows(p, rows), method=1) if len(rows) else np.zeros((0, p.L))
+    data = I.make_all(p)
+    y = (oracle.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], B=p.B, C=p.C, order=p.order,
+                              shape=p.shape, rows=rows, method=1) if len(rows) else np.zeros((0, p.L)))
     np.save(os.path.join(outdir, f"r{rank}.npy"), y.reshape(p.B, c1 - c0, p.L))
     np.save(os.path.join(outdir, f"m{rank}.npy"), np.array([m, c0, c1]))
     hd.barrier()
@@ -59,5 +61,7 @@ def test_two_gloo_ranks_shard_and_reduce():
         shards = [np.load(os.path.join(d, f"r{r}.npy")) for r in range(world)]
     p = I.WORKLOADS["tiny"].with_(B=2, C=7, L=256, seed=7001)
     y_sharded = np.concatenate(shards, axis=1)
-    y_full = oracle.hyena_rows(*I.oracle_rows(p, np.arange(p.B * p.C)), method=1).reshape(p.B, p.C, p.L)
+    data = I.make_all(p)
+    y_full = oracle.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], B=p.B, C=p.C, order=p.order,
+                                  shape=p.shape, method=1).reshape(p.B, p.C, p.L)
     assert np.array_equal(y_sharded, y_full)

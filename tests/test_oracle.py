@@ -15,10 +15,9 @@ def test_tiny_workload_direct_equals_fft(orc):
     """The whole small workload: the direct-sum oracle and the FFT oracle agree."""
     p = I.WORKLOADS["tiny"]
     data = I.make_all(p)
-    rows = np.arange(p.B * p.C)
-    args = I.oracle_rows(p, rows, data)
-    y1 = orc.hyena_rows(*args, method=1)
-    y2 = orc.hyena_rows(*args, method=2)
+    kw = dict(B=p.B, C=p.C, order=p.order, shape=p.shape)
+    y1 = orc.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], data["sc_b"], method=1, **kw)
+    y2 = orc.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], data["sc_b"], method=2, **kw)
     rel = np.linalg.norm(y1 - y2, axis=-1) / np.linalg.norm(y1, axis=-1)
     assert rel.max() < 1e-12
 
@@ -27,10 +26,10 @@ def test_tiny_workload_direct_equals_fft(orc):
 def test_d768_l8k_sampled_rows_direct_equals_fft(orc):
     """Full L = 8192 on sampled rows: direct sums and the radix-2 FFT agree."""
     p = I.WORKLOADS["d768_l8k"]
-    rows = np.array([0, 767, 2 * 768 + 5])
-    args = I.oracle_rows(p, rows)
-    y1 = orc.hyena_rows(*args, method=1)
-    y2 = orc.hyena_rows(*args, method=2)
+    data = I.make_all(p)
+    kw = dict(B=p.B, C=p.C, order=p.order, shape=p.shape, rows=np.array([0, 767, 2 * 768 + 5]))
+    y1 = orc.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], method=1, **kw)
+    y2 = orc.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], method=2, **kw)
     rel = np.linalg.norm(y1 - y2, axis=-1) / np.linalg.norm(y1, axis=-1)
     assert rel.max() < 1e-11
 
@@ -49,17 +48,12 @@ def test_bf16_rounding_matches_torch():
 
 
 def test_generators_are_row_addressable():
-    """A row generated on its own equals the same row cut from the full tensor."""
-    p = I.WORKLOADS["tiny"].with_(C=8, L=64)
-    data = I.make_all(p)
-    rows = np.array([3, 7])
-    a = I.oracle_rows(p, rows, data)
-    b = I.oracle_rows(p, rows)
-    for x, y in zip(a, b):
-        if x is None:
-            assert y is None
-        else:
-            assert np.array_equal(x, y)
+    """A channel row generated on its own equals the same row of the full tensor."""
+    for p in (I.WORKLOADS["tiny"].with_(B=2, C=8, L=64), I.WORKLOADS["dna_1m"].with_(L=256)):
+        data = I.make_all(p)
+        for b, ch in ((0, 3), (p.B - 1, p.Ctot - 1)):
+            assert np.array_equal(I.store(p, I.u_row(p, b, ch)), data["u"][b, ch])
+        assert np.array_equal(I.store(p, I.k_row(p, 0, p.C - 1)), data["k"][0, p.C - 1])
 
 
 def test_generator_recipes():

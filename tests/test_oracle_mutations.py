@@ -48,6 +48,27 @@ MUTATIONS = {
                                       "int64_t n1 = next_pow2(N1), n2 = next_pow2(2 * N2), n3 = next_pow2(2 * N3);"),
     "3-D operator gates with v's chunk": ("const double *g = x + (int64_t)(order - s) * n;",
                                           "const double *g = x + (int64_t)order * n;"),
+    "split interleaved (chunk j of c at c*(order+1) + j)": ("const int64_t ch = (int64_t)j * C + c;",
+                                                            "const int64_t ch = c * (int64_t)(order + 1) + j;"),
+    "split batch stride of one chunk": ("const int64_t src = (b * Ctot + ch) * n;",
+                                        "const int64_t src = (b * C + ch) * n;"),
+    "split taps of the row's first chunk": ("scw_rows[(i * (order + 1) + j) * 3 + m] = sc_w[ch * 3 + m];",
+                                            "scw_rows[(i * (order + 1) + j) * 3 + m] = sc_w[c * 3 + m];"),
+    "split bias of the row's first chunk": ("scb_rows[i * (order + 1) + j] = sc_b ? sc_b[ch] : 0.0;",
+                                            "scb_rows[i * (order + 1) + j] = sc_b ? sc_b[c] : 0.0;"),
+    "split per-sample filter index transposed": ("const int64_t f = per_sample ? b * C + c : c;",
+                                                 "const int64_t f = per_sample ? c * B + b : c;"),
+    "split filters indexed by batch": ("const int64_t f = per_sample ? b * C + c : c;",
+                                       "const int64_t f = per_sample ? b * C + c : (c + b) % C;"),
+    "bf16 bits read as the low half": ("uint32_t bits = (uint32_t)((const uint16_t *)base)[i] << 16;",
+                                       "uint32_t bits = (uint32_t)((const uint16_t *)base)[i];"),
+    "in_proj weight transposed": ("for (int64_t i = 0; i < D; ++i) acc += x[(b * L + l) * D + i] * W[j * D + i];",
+                                  "for (int64_t i = 0; i < D; ++i) acc += x[(b * L + l) * D + i] * W[i * J + j];"),
+    "in_proj not rearranged": ("u[(b * J + j) * L + l] = acc;", "u[(b * L + l) * J + j] = acc;"),
+    "out_proj reads y unrearranged": ("for (int64_t i = 0; i < D; ++i) acc += y[(b * D + i) * L + l] * W[j * D + i];",
+                                      "for (int64_t i = 0; i < D; ++i) acc += y[(b * L + l) * D + i] * W[j * D + i];"),
+    "out_proj bias dropped": ("                double acc = bias ? bias[j] : 0.0;\n                for (int64_t i = 0; i < D; ++i) acc += y",
+                              "                double acc = 0.0;\n                for (int64_t i = 0; i < D; ++i) acc += y"),
     "2-D circular form runs padded": ("if (direct) oracle_conv2d_circ_direct(ks, Ds, w, vn, H, W);",
                                       "if (direct) oracle_conv2d_direct(ks, Ds, w, vn, H, W);"),
 }
