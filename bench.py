@@ -44,6 +44,78 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def load_bf16_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed alone (burst)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        if "bf16_tflops" in pk:
+            return float(pk["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def time_events(fn, stream, steps: int, warmup: int = 3) -> float:
+    """Median milliseconds per call of fn, CUDA events on `stream`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def layer_extras(p, dev, stream, steps: int):
+    """The layer around the operator on the same workload: in_proj and out_proj
+    (tcgen05 GEMMs, bf16 in/out, fp32 accumulation) against the bf16 peak, and
+    the spectrum build from the implicit filter (once per filter change)."""
+    import torch
+    from fft_long_convolution_02_b200 import binding as hb
+    from fft_long_convolution_02_b200 import inputs as I
+    out = {}
+    if p.dtype == "bf16" and p.ndim == 1 and not p.per_sample and p.C % 8 == 0 and p.L % 8 == 0:
+        lay = I.make_layer(p)
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        x, Wi, Wo = bf(lay["x"]), bf(lay["W_in"]), bf(lay["W_out"])
+        bi, bo = torch.from_numpy(lay["b_in"]).to(dev), torch.from_numpy(lay["b_out"]).to(dev)
+        u = torch.empty((p.B, p.Ctot, p.L), dtype=torch.bfloat16, device=dev)
+        yv = torch.empty((p.B, p.C, p.L), dtype=torch.bfloat16, device=dev).normal_()
+        o = torch.empty((p.B, p.L, p.C), dtype=torch.bfloat16, device=dev)
+        t_in = time_events(lambda: hb.hyena_in_proj(x, Wi, bi, u, p.order, stream), stream, steps)
+        t_out = time_events(lambda: hb.hyena_out_proj(yv, Wo, bo, o, stream), stream, steps)
+        peak, kind = load_bf16_peak()
+        f_in = 2.0 * p.B * p.L * p.C * p.Ctot
+        f_out = 2.0 * p.B * p.L * p.C * p.C
+        out["projections"] = {
+            "kernel": "k_gemm_bf16 (tcgen05, TMA, bf16 operands, fp32 accumulation in tensor memory)",
+            "in_proj_us": t_in * 1e3, "in_proj_tflops": f_in / (t_in / 1e3) / 1e12,
+            "out_proj_us": t_out * 1e3, "out_proj_tflops": f_out / (t_out / 1e3) / 1e12,
+            "peak_tflops": peak, "peak_kind": kind,
+            "in_proj_frac": f_in / (t_in / 1e3) / 1e12 / peak, "out_proj_frac": f_out / (t_out / 1e3) / 1e12 / peak}
+    if p.ndim == 1 and p.L <= 16384 and not p.per_sample:
+        prm = I.implicit_filter_params(p)
+        dprm = {k: (torch.from_numpy(v).to(dev) if isinstance(v, np.ndarray) else v) for k, v in prm.items()}
+        D = torch.from_numpy(I.D_all(p)).to(dev)
+        spec = torch.empty(hb.hyena_spectrum_bytes(p.C, p.shape, p.order), dtype=torch.uint8, device=dev)
+        ws = torch.empty(hb.hyena_implicit_filter_workspace_bytes(p.L, prm["width"]), dtype=torch.uint8, device=dev)
+        t_imp = time_events(lambda: hb.hyena_filter_spectrum_implicit(dprm, D, p.C, p.L, p.order, spec, ws,
+                                                                      stream=stream), stream, max(3, steps // 5))
+        k = torch.empty((p.order - 1, p.C, p.L), dtype=torch.float32, device=dev).normal_()
+        t_st = time_events(lambda: hb.hyena_filter_spectrum(k, D, p.C, p.shape, p.order, spec, stream), stream,
+                           max(3, steps // 5))
+        out["implicit_filter_spectrum"] = {
+            "what": "filter generation (embedding, Sin MLP width 64 with 2 inner layers, modulation) fused into the "
+                    "spectrum build, once per filter change; not in the timed step",
+            "ms": t_imp, "stored_filter_spectrum_ms": t_st}
+    hb.hyena_kernel_status(stream)
+    return out
+
+
 def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
     """One read of u (all order+1 chunks), one read of the stored spectra
     (C rows per order step, B*C with per-sample filters), one write of y."""
@@ -143,24 +215,22 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def _oracle_rows(orc, p, args, cores):
-    """The float64 oracle on self-contained rows of problem p (FFT form)."""
-    if p.ndim == 3:
-        return orc.hyena_rows3(*args[:3], method=2, nthreads=cores)
-    return orc.hyena_rows(*args, ndim=p.ndim, method=2, nthreads=cores, circular=p.circular)
+def _oracle_rows(orc, p, data, rows, cores):
+    """The float64 oracle (FFT form) on rows b*C + c of the stacked inputs."""
+    return orc.hyena_stacked(data["u"], data["k"], data["D"], data["sc_w"], data["sc_b"], B=p.B, C=p.C,
+                             order=p.order, shape=p.shape, rows=rows, per_sample=p.per_sample,
+                             circular=p.circular, method=2, nthreads=cores)
 
 
-def cpu_baseline(p, budget_s: float = 15.0):
+def cpu_baseline(p, data, budget_s: float = 15.0):
     """Time the float64 oracle (as it stands) on a bounded sample of rows."""
     import oracle
-    from fft_long_convolution_02_b200 import inputs as I
     cores = len(os.sched_getaffinity(0))
     orc = oracle.default()
     rng = np.random.default_rng(0)
     rows = rng.choice(p.B * p.C, size=min(p.B * p.C, 8 * cores), replace=False)
-    args = I.oracle_rows(p, rows)
     t0 = time.perf_counter()
-    _oracle_rows(orc, p, args, cores)
+    _oracle_rows(orc, p, data, rows, cores)
     dt = time.perf_counter() - t0
     # grow the sample to use about budget_s of CPU time
     n_more = int(len(rows) * max(0.0, budget_s / max(dt, 1e-3) - 1.0))
@@ -168,9 +238,8 @@ def cpu_baseline(p, budget_s: float = 15.0):
     total_rows, total_t = len(rows), dt
     if n_more > 0:
         rows2 = rng.choice(p.B * p.C, size=n_more, replace=False)
-        args = I.oracle_rows(p, rows2)
         t0 = time.perf_counter()
-        _oracle_rows(orc, p, args, cores)
+        _oracle_rows(orc, p, data, rows2, cores)
         total_t += time.perf_counter() - t0
         total_rows += n_more
     # a row is one (b, c) pair; the operator's tokens are B*n over all C channels
@@ -190,20 +259,20 @@ def run_reference(args, p):
     orc = oracle.default()
     rng = np.random.default_rng(1)
     per_step = max(cores, 16)
-    samples = [I.oracle_rows(p, rng.choice(p.B * p.C, size=per_step, replace=False))
-               for _ in range(args.warmup + args.steps)]
-    for a in samples[:args.warmup]:
-        _oracle_rows(orc, p, a, cores)
+    data = I.make_all(p)
+    samples = [rng.choice(p.B * p.C, size=per_step, replace=False) for _ in range(args.warmup + args.steps)]
+    for rows in samples[:args.warmup]:
+        _oracle_rows(orc, p, data, rows, cores)
     t0 = time.perf_counter()
-    for a in samples[args.warmup:]:
-        _oracle_rows(orc, p, a, cores)
+    for rows in samples[args.warmup:]:
+        _oracle_rows(orc, p, data, rows, cores)
     dt = time.perf_counter() - t0
     tok_s = args.steps * per_step * p.n / (p.C * dt)
     line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": config_of(p),
+            "config": config_of(p, "float64 (the oracle)"),
             "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{per_step} (b,c) rows per step of {p.B * p.C}; float64 radix-2 "
                                        f"FFT oracle; tokens/s = rows*n/(C*t)"},
@@ -211,9 +280,28 @@ def run_reference(args, p):
     print(json.dumps(line), flush=True)
 
 
-def config_of(p):
+def kernel_of(p) -> str:
+    """The dominant kernel hyena_gated_fftconv launches for problem p."""
+    if p.ndim == 1 and p.L == 8192:
+        return "k_conv_8192_tc" if (p.dtype == "bf16" and not p.per_sample and p.order <= 3) else "k_conv_4096"
+    if p.ndim == 1 and p.L <= 16384:
+        return "k_conv_onchip"
+    return "multipass" if p.ndim == 1 else ("grid2d" if p.ndim == 2 else "grid3d")
+
+
+def math_of(p, kernel: str) -> str:
+    """What the measured kernel computes in, as built."""
+    if kernel == "k_conv_8192_tc":
+        return ("DFT stages on tcgen05 tensor cores: bf16 operands and DFT matrices, fp32 accumulation; "
+                "short conv, gates, twiddles and spectrum products fp32; spectrum read as bf16 (re, im)")
+    if p.dtype == "bf16" and (p.ndim > 1 or p.L > 16384):
+        return "fp32 (intermediate kept as bf16 pairs in the workspace between passes)"
+    return "fp32"
+
+
+def config_of(p, math: str):
     cfg = {"workload": p.name, "B": p.B, "C": p.C, "order": p.order,
-           "shortconv": p.shortconv, "storage": p.dtype, "math": "fp32"}
+           "shortconv": p.shortconv, "storage": p.dtype, "math": math}
     if p.per_sample:
         cfg["filters"] = "per-sample (one filter per (b, c) row)"
     if p.circular:
@@ -320,6 +408,28 @@ def main():
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     elapsed_ms = hd.max_over_ranks(elapsed_ms, dev)
 
+    # the same workload with every transform multiply in fp32 (bf16 storage,
+    # fp32 arithmetic: HYENA_FLAG_FP32_TRANSFORM), where that changes the kernel
+    fp32_ms = None
+    if kernel_of(p) == "k_conv_8192_tc":
+        def step32():
+            hb.hyena_gated_fftconv_ex(u, y, spec, sc_w, None, p.B, p.C, shape, p.order, ws,
+                                      flags=hb.HYENA_FLAG_FP32_TRANSFORM, stream=stream)
+        for _ in range(args.warmup):
+            step32()
+        torch.cuda.synchronize()
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            step32()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fp32_ms = hd.max_over_ranks(f0.elapsed_time(f1), dev)
+
+    extras = layer_extras(p, dev, stream, args.steps)
+
     # end to end through the C ABI with host buffers (pinned), copies timed:
     # hyena_gated_fftconv_host pipelines each step's chunk copies against the
     # kernels (per-sample filters: copy, convolve, copy back on one stream)
@@ -358,18 +468,13 @@ def main():
     alg = algorithmic_bytes(p, spec_row)
     avg_launch_s = float(np.mean(launch_ms)) / 1e3
     achieved = alg / avg_launch_s / 1e9
-    if p.ndim == 1 and p.L == 8192:
-        kernel = "k_conv_8192_tc" if (p.dtype == "bf16" and not p.per_sample) else "k_conv_4096"
-    elif p.ndim == 1 and p.L <= 16384:
-        kernel = "k_conv_onchip"
-    else:
-        kernel = "multipass" if p.ndim == 1 else ("grid2d" if p.ndim == 2 else "grid3d")
+    kernel = kernel_of(p)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if p.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": dict(config_of(p), parallelism=f"replicas{world}" if world > 1 else "single",
+        "config": dict(config_of(p, math_of(p, kernel)), parallelism=f"replicas{world}" if world > 1 else "single",
                        l2="inputs larger than L2 (%.0f MB per step)" % (alg / 1e6)),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
@@ -381,10 +486,17 @@ def main():
                 "h2d_bytes_per_step": u.numel() * u.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},
         "gpu_launches": args.steps,
+        "fp32_transform": None if fp32_ms is None else {
+            "kernel": "k_conv_4096", "flag": "HYENA_FLAG_FP32_TRANSFORM",
+            "math": "fp32 throughout (register FFT on the CUDA cores; complex64 spectrum plane)",
+            "value": world * tokens_per_step * args.steps / (fp32_ms / 1e3), "unit": UNIT,
+            "ms_per_step": fp32_ms / args.steps,
+            "roofline_frac": alg / (fp32_ms / args.steps / 1e3) / 1e9 / peak},
         "clocks": clk,
     }
+    line.update(extras)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(p)
+        line["cpu_baseline"] = cpu_baseline(p, data)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -25,7 +25,8 @@ EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "h
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
            "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
            "hyena_gated_fftconv_per_sample", "hyena_gated_fftconv_host", "hyena_spectrum_check",
-           "hyena_debug_conv_tc"]
+           "hyena_debug_conv_tc", "hyena_gated_fftconv_ex", "hyena_kernel_status", "hyena_in_proj",
+           "hyena_out_proj", "hyena_implicit_filter_workspace_bytes", "hyena_filter_spectrum_implicit"]
 
 _lock = threading.Lock()
 _lib = None
@@ -77,6 +78,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hyena_gated_fftconv_noalloc.restype = ctypes.c_int
         lib.hyena_gated_fftconv_noalloc.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p,
                                                     ctypes.c_int, ctypes.c_int, vp]
+        lib.hyena_gated_fftconv_ex.restype = ctypes.c_int
+        lib.hyena_gated_fftconv_ex.argtypes = [vp, vp, vp, sz, fp, fp, i64, i64, ctypes.c_int, i64p, ctypes.c_int,
+                                               ctypes.c_int, vp, sz, ctypes.c_uint, vp]
+        lib.hyena_in_proj.restype = ctypes.c_int
+        lib.hyena_in_proj.argtypes = [vp, vp, fp, vp, i64, i64, i64, ctypes.c_int, vp]
+        lib.hyena_out_proj.restype = ctypes.c_int
+        lib.hyena_out_proj.argtypes = [vp, vp, fp, vp, i64, i64, i64, vp]
+        lib.hyena_implicit_filter_workspace_bytes.restype = sz
+        lib.hyena_implicit_filter_workspace_bytes.argtypes = [i64, ctypes.c_int]
+        lib.hyena_filter_spectrum_implicit.restype = ctypes.c_int
+        lib.hyena_filter_spectrum_implicit.argtypes = [ctypes.POINTER(ImplicitFilter), fp, i64, i64, ctypes.c_int, vp,
+                                                       sz, vp, sz, fp, vp]
+        lib.hyena_kernel_status.restype = ctypes.c_int
+        lib.hyena_kernel_status.argtypes = [vp]
         lib.hyena_spectrum_check.restype = ctypes.c_int
         lib.hyena_spectrum_check.argtypes = [vp, i64, ctypes.c_int, i64p, ctypes.c_int, vp]
         lib.hyena_debug_conv_tc.restype = ctypes.c_int
@@ -182,6 +197,66 @@ def hyena_gated_fftconv(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, or
                                       _ptr(workspace), ws_bytes, _stream(stream)))
 
 
+HYENA_FLAG_FP32_TRANSFORM = 0x1
+
+
+def hyena_gated_fftconv_ex(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int, workspace=None,
+                           flags: int = 0, stream=None) -> None:
+    """hyena_gated_fftconv with flags (HYENA_FLAG_FP32_TRANSFORM: the fp32
+    transform at L = 8192 with bf16 storage)."""
+    arr, nd = _sizes(sizes)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyena_gated_fftconv_ex(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
+                                         _ptr(sc_w), _ptr(sc_bias), B, C, nd, arr, order, _dtype_code(u),
+                                         _ptr(workspace), ws_bytes, int(flags), _stream(stream)))
+
+
+def hyena_in_proj(x, W, bias, u, order: int, stream=None) -> None:
+    """x [B, L, D] bf16, W [(order+1)*D, D] bf16, bias [(order+1)*D] f32 or
+    None -> u [B, (order+1)*D, L] bf16 (in_proj then 'b l d -> b d l')."""
+    B, L, D = x.shape
+    _check(load().hyena_in_proj(_ptr(x), _ptr(W), _ptr(bias), _ptr(u), B, L, D, int(order), _stream(stream)))
+
+
+def hyena_out_proj(y, W, bias, out, stream=None) -> None:
+    """y [B, D, L] bf16, W [D, D] bf16, bias [D] f32 or None -> out [B, L, D]
+    bf16 ('b d l -> b l d' then out_proj)."""
+    B, D, L = y.shape
+    _check(load().hyena_out_proj(_ptr(y), _ptr(W), _ptr(bias), _ptr(out), B, L, D, _stream(stream)))
+
+
+class ImplicitFilter(ctypes.Structure):
+    """hyena_implicit_filter_t (device pointers)."""
+    _fields_ = [("emb_dim", ctypes.c_int), ("width", ctypes.c_int), ("num_inner", ctypes.c_int),
+                ("W_in", ctypes.c_void_p), ("b_in", ctypes.c_void_p), ("W_inner", ctypes.c_void_p),
+                ("b_inner", ctypes.c_void_p), ("W_out", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("alpha", ctypes.c_void_p)]
+
+
+def hyena_implicit_filter_workspace_bytes(L: int, width: int) -> int:
+    return int(load().hyena_implicit_filter_workspace_bytes(L, width))
+
+
+def hyena_filter_spectrum_implicit(params: dict, D, C: int, L: int, order: int, spectrum, workspace, k_out=None,
+                                   stream=None) -> None:
+    """params: emb_dim, width, num_inner (ints) and CUDA float32 tensors W_in,
+    b_in, W_inner, b_inner (or None), W_out, w, alpha (hyena_implicit_filter_t)."""
+    f = ImplicitFilter(int(params["emb_dim"]), int(params["width"]), int(params["num_inner"]),
+                       _ptr(params["W_in"]), _ptr(params["b_in"]), _ptr(params.get("W_inner")),
+                       _ptr(params.get("b_inner")), _ptr(params["W_out"]), _ptr(params["w"]), _ptr(params["alpha"]))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().hyena_filter_spectrum_implicit(ctypes.byref(f), _ptr(D), C, L, int(order), _ptr(spectrum),
+                                                 spectrum.numel() * spectrum.element_size(), _ptr(workspace),
+                                                 ws_bytes, _ptr(k_out), _stream(stream)))
+
+
+def hyena_kernel_status(stream=None) -> None:
+    """Raises HyenaError (HYENA_ERR_TIMEOUT or HYENA_ERR_SPECTRUM_MISMATCH)
+    when a convolution kernel on the current device recorded one since the
+    last call; synchronises the stream and clears the record."""
+    _check(load().hyena_kernel_status(_stream(stream)))
+
+
 def hyena_gated_fftconv_per_sample(u, y, spectrum, sc_w, sc_bias, B: int, C: int, sizes, order: int,
                                    workspace=None, stream=None) -> None:
     """hyena_gated_fftconv with one filter per (b, c) row: spectrum from
@@ -230,7 +305,7 @@ def hyena_debug_conv_tc(u, y, spectrum, sc_w, sc_bias, B: int, C: int, order: in
                         issue_mma: bool = True, stream=None) -> None:
     """Test hook of the L = 8192 bf16 tensor-core kernel: its bounded waits give
     up after wait_budget_ns; issue_mma=False issues no tensor-core work, so the
-    first wait runs out (read back with hyena_spectrum_check)."""
+    first wait runs out (read back with hyena_kernel_status)."""
     _check(load().hyena_debug_conv_tc(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
                                       _ptr(sc_w), _ptr(sc_bias), B, C, order, int(wait_budget_ns),
                                       1 if issue_mma else 0, _stream(stream)))

@@ -66,7 +66,7 @@ hyena_status_t set_last_error_detail(hyena_status_t st, const std::string& detai
 
 extern "C" {
 
-int hyena_version(void) { return 100; }
+int hyena_version(void) { return 101; }
 
 const char* hyena_status_string(hyena_status_t s) {
     switch (s) {
@@ -210,14 +210,17 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
 hyena_status_t gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, const float* sc_w,
                              const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes, int order,
                              hyena_dtype_t dtype, void* workspace, size_t workspace_bytes, void* stream,
-                             bool per_sample) {
+                             bool per_sample, unsigned flags = 0) {
+    if (flags & ~unsigned(HYENA_FLAG_FP32_TRANSFORM)) return fail(HYENA_ERR_INVALID_ARG, "unknown flag bits");
     Plan p;
     ConvArgs a;
     hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype,
                                      workspace, workspace_bytes, &p, &a, per_sample);
     if (st != HYENA_OK) return st;
+    a.fp32_transform = (flags & HYENA_FLAG_FP32_TRANSFORM) != 0;
+    cudaError_t e = kernel_status_word(&a.status);
+    if (e != cudaSuccess) return cuda_status(e, "kernel status word");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
     switch (p.path) {
         case PATH_ONCHIP_1D: e = launch_conv_onchip(p, a, s); break;
         case PATH_MULTIPASS_1D: e = launch_conv_multipass(p, a, s); break;
@@ -239,6 +242,14 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
                                    size_t workspace_bytes, void* stream) {
     return gated_fftconv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype, workspace,
                          workspace_bytes, stream, false);
+}
+
+hyena_status_t hyena_gated_fftconv_ex(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                      const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                      const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                      size_t workspace_bytes, unsigned flags, void* stream) {
+    return gated_fftconv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, ndim, sizes, order, dtype, workspace,
+                         workspace_bytes, stream, false, flags);
 }
 
 hyena_status_t hyena_gated_fftconv_per_sample(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
@@ -263,6 +274,8 @@ hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum,
     if (wait_budget_ns == 0) return fail(HYENA_ERR_INVALID_ARG, "wait_budget_ns must be > 0");
     a.wait_budget_ns = wait_budget_ns;
     a.issue_mma = issue_mma ? 1 : 0;
+    cudaError_t e = kernel_status_word(&a.status);
+    if (e != cudaSuccess) return cuda_status(e, "kernel status word");
     return cuda_status(launch_conv_8192_tc(p, a, static_cast<cudaStream_t>(stream)), "tensor-core kernel");
 }
 
@@ -310,7 +323,11 @@ hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* 
     if (st != HYENA_OK) return st;
     if (!u_host || !y_host) return fail(HYENA_ERR_INVALID_ARG, "u_host and y_host must not be NULL");
     if (chunk_rows < 0) return fail(HYENA_ERR_INVALID_ARG, "chunk_rows must be >= 0 (0: default)");
-    const int64_t chunk = chunk_rows > 0 ? (chunk_rows < B ? chunk_rows : B) : (B + 3) / 4;
+    int64_t chunk = chunk_rows > 0 ? (chunk_rows < B ? chunk_rows : B) : (B + 3) / 4;
+    // default: an even number of batch rows, so that the L = 8192 bf16 kernel,
+    // which transforms two batch rows of a channel together, never pairs a
+    // row with zeros
+    if (chunk_rows == 0 && (chunk & 1) && chunk < B) ++chunk;
     const size_t es = elem_size(dtype);
     const size_t ub = size_t(order + 1) * size_t(C) * size_t(p.n) * es;    // u bytes per batch row
     const size_t yb = size_t(C) * size_t(p.n) * es;                        // y bytes per batch row
@@ -368,8 +385,6 @@ hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, c
     if (h.magic != kSpecMagic || h.version != kSpecVersion || h.path != p.path || h.C != p.C || h.L != p.L ||
         h.H != p.H || h.W != p.W || h.order != p.order || size_t(h.total_bytes) != p.total_bytes)
         return fail(HYENA_ERR_SPECTRUM_MISMATCH, "spectrum header does not match (C, sizes, order)");
-    if (h.device_status != 0)
-        return fail(HYENA_ERR_TIMEOUT, "a convolution with this spectrum ran out of its tensor-core wait budget");
     return ok();
 }
 

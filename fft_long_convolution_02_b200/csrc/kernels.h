@@ -14,11 +14,37 @@ enum DType { DT_F32 = 0, DT_BF16 = 1 };
 // long enough to ride out time-slicing with other contexts on a shared GPU.
 constexpr uint64_t kDefaultWaitBudgetNs = 2000000000ull;
 
+// Bits of the per-device kernel status word (status.cu, hyena_kernel_status).
+constexpr uint32_t kStatusTimeout = 1u;            // a bounded tensor-core wait ran out
+constexpr uint32_t kStatusSpectrumMismatch = 2u;   // spectrum header does not match the launch
+
+// Device address of this device's kernel status word (looked up once per device).
+cudaError_t kernel_status_word(uint32_t** out);
+
+// Records a kernel-detected condition in the status word (one thread per CTA).
+__device__ __forceinline__ void report_status(uint32_t* status, uint32_t bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// The implicit long filter (HyenaFilter): row r = s*C + c of the filters is
+// k[t] = exp(-alpha[r] t / (L-1)) * sum_j hT[j][t] W_out[r][j], where hT is
+// the last hidden layer of the filter MLP, transposed ([width][L]).
+struct ImplicitFilter {
+    const float* hT = nullptr;
+    const float* W_out = nullptr;   // [(order-1) C][width]
+    const float* alpha = nullptr;   // [(order-1) C]
+    float* k_out = nullptr;         // [(order-1) C][L] copy of the generated filters, or nullptr
+    int width = 0;
+};
+
 struct SpectrumArgs {
     const void* k;        // [order-1, C, n]
     int k_dtype;
     const float* D;       // [order-1, C] or nullptr
     uint8_t* spectrum;    // buffer start (header at offset 0)
+    // set: the filters are generated (k unused); 1-D on-chip lengths only
+    bool implicit = false;
+    ImplicitFilter imp{};
 };
 
 struct ConvArgs {
@@ -39,6 +65,11 @@ struct ConvArgs {
     // (C, 0) for filters shared over the batch, (B*C, C) for per-sample filters
     int64_t spec_C = 0;
     int64_t spec_per_b = 0;
+    // kernel status word of this device (kStatus* bits)
+    uint32_t* status = nullptr;
+    // L = 8192 with bf16 storage: run the fp32 CUDA-core transform instead of
+    // the tensor-core one (HYENA_FLAG_FP32_TRANSFORM)
+    bool fp32_transform = false;
 };
 
 cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);
@@ -52,6 +83,12 @@ cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_
 cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_3d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_3d(const Plan& p, const ConvArgs& a, cudaStream_t s);
+// Hidden layers of the implicit filter MLP for t < L -> hT [width][L] (filtergen.cu).
+struct ImplicitMlp {
+    int emb_dim, width, num_inner;
+    const float *W_in, *b_in, *W_inner, *b_inner, *w;
+};
+cudaError_t launch_filter_hidden(const ImplicitMlp& m, int64_t L, float* hT, cudaStream_t s);
 cudaError_t launch_shortconv(const void* u, void* out, const float* w, const float* bias, int64_t B,
                              int64_t Ctot, int64_t L, int dtype, cudaStream_t s);
 

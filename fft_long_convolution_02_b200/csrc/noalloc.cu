@@ -13,7 +13,9 @@
 // (32 MiB); every GPU that loads the library keeps it until the process
 // exits.  Its device address is looked up once per device with
 // cudaGetSymbolAddress (host code may not use the array's name as a device
-// pointer) and cached.  Nothing here allocates or frees memory.
+// pointer) and cached for the life of the process, so calls after a reset of
+// the device (which may move the array) are not supported.  Nothing here
+// allocates or frees memory.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -42,6 +42,29 @@ __device__ __forceinline__ bool header_ok(const uint8_t* spec, int64_t C, int64_
            h->order == order;
 }
 
+// Samples 2n, 2n+1 of filter row `row` from the implicit filter (ImplicitFilter);
+// wo = the row's output weights (shared memory).  Optionally records them.
+__device__ __forceinline__ float2 implicit_pair(const ImplicitFilter& f, const float* wo, int64_t row, int L, int n) {
+    float a0 = 0.0f, a1 = 0.0f;
+    const float2* h = reinterpret_cast<const float2*>(f.hT) + n;
+    for (int j = 0; j < f.width; ++j) {
+        const float2 v = __ldg(h + int64_t(j) * (L / 2));
+        a0 = fmaf(v.x, wo[j], a0);
+        a1 = fmaf(v.y, wo[j], a1);
+    }
+    const float al = __ldg(f.alpha + row);
+    const float inv = 1.0f / float(L - 1);
+    const float2 k = make_float2(a0 * expf(-al * (float(2 * n) * inv)), a1 * expf(-al * (float(2 * n + 1) * inv)));
+    if (f.k_out) reinterpret_cast<float2*>(f.k_out + row * L)[n] = k;
+    return k;
+}
+
+// The row's output weights of the implicit filter into shared memory `wo`.
+__device__ __forceinline__ void load_row_weights(const ImplicitFilter& f, float* wo, int64_t row) {
+    for (int j = threadIdx.x; j < f.width; j += blockDim.x) wo[j] = __ldg(f.W_out + row * f.width + j);
+    __syncthreads();
+}
+
 // Pair step of the convolution: untangle, multiply by K~, re-tangle.
 // Chain e pairs q = 0..M/2 -> (m, M-m); chain o pairs q = M/2+1..M -> (j, M-1-j).
 template <int M>
@@ -79,10 +102,10 @@ __device__ __forceinline__ void conv_pairs(float2* __restrict__ be, float2* __re
     }
 }
 
-template <int M, typename TK>
+template <int M, typename TK, bool IMP>
 __global__ void __launch_bounds__(onchip_threads<M>())
 k_spectrum_onchip(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* __restrict__ spectrum,
-                  int64_t C, int order) {
+                  int64_t C, int order, ImplicitFilter imp) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(M);
     constexpr int L = 2 * M;
@@ -93,12 +116,16 @@ k_spectrum_onchip(const TK* __restrict__ k, const float* __restrict__ D, uint8_t
     const float2* twist = tables + fft_tw_size(M);
     const float2* untw = twist + M;
     const int64_t row = blockIdx.x;  // s * C + c
-    const TK* kr = k + row * L;
+    const TK* kr = IMP ? nullptr : k + row * L;
     const float d = D ? __ldg(D + row) : 0.0f;
     float2* be = smem;
     float2* bo = smem + PS;
+    float* wo = reinterpret_cast<float*>(smem + 2 * PS);
+    if constexpr (IMP) load_row_weights(imp, wo, row);
     for (int n = threadIdx.x; n < M; n += blockDim.x) {
-        const float2 z = load2(kr + 2 * n);
+        float2 z;
+        if constexpr (IMP) z = implicit_pair(imp, wo, row, L, n);
+        else z = load2(kr + 2 * n);
         be[fft_pad(n)] = z;
         bo[fft_pad(n)] = cmul(z, __ldg(twist + n));
     }
@@ -132,11 +159,14 @@ template <int M, typename T>
 __global__ void __launch_bounds__(onchip_threads<M>())
 k_conv_onchip(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C,
-              int order, int64_t SC, int64_t SB) {
+              int order, int64_t SC, int64_t SB, uint32_t* status) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(M);
     constexpr int L = 2 * M;
-    if (!header_ok(spectrum, SC, L, order)) return;
+    if (!header_ok(spectrum, SC, L, order)) {
+        if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
     const float2* tw_fft = tables;
@@ -308,9 +338,12 @@ template <typename T>
 __global__ void __launch_bounds__(NT, 2)
 k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restrict__ spectrum,
             const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-            int64_t rows, int64_t SC, int64_t SB) {
+            int64_t rows, int64_t SC, int64_t SB, uint32_t* status) {
     extern __shared__ float2 smem[];
-    if (!header_ok(spectrum, SC, L, order)) return;
+    if (!header_ok(spectrum, SC, L, order)) {
+        if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
     const float2* twist = tables + fft_tw_size(M);
@@ -512,9 +545,10 @@ constexpr size_t conv_4096_smem() {
 //   X[f] = ((Z[f] + conj Z[L-f]) - i w_2L^f (Z[f] - conj Z[L-f])) / 2,
 // X[0] = Re Z[0] + Im Z[0], X[L] = Re Z[0] - Im Z[0]; X[2L-f] = conj X[f].
 
-template <typename TK>
+template <typename TK, bool IMP>
 __global__ void __launch_bounds__(512)
-k_spectrum_8192(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* __restrict__ spectrum) {
+k_spectrum_8192(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* __restrict__ spectrum,
+                ImplicitFilter imp) {
     extern __shared__ float2 smem[];
     constexpr int M = 4096, L = 8192;
     constexpr int PS = fft_padded_size(M);
@@ -524,12 +558,16 @@ k_spectrum_8192(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* 
     const float2* twist = tables + fft_tw_size(M);
     const float2* untw = twist + M;
     const int64_t row = blockIdx.x;  // s * C + c
-    const TK* kr = k + row * L;
+    const TK* kr = IMP ? nullptr : k + row * L;
     const float d = D ? __ldg(D + row) : 0.0f;
     float2* be = smem;
     float2* bo = smem + PS;
+    float* wo = reinterpret_cast<float*>(smem + 2 * PS);
+    if constexpr (IMP) load_row_weights(imp, wo, row);
     for (int n = threadIdx.x; n < M; n += blockDim.x) {
-        const float2 z = load2(kr + 2 * n);
+        float2 z;
+        if constexpr (IMP) z = implicit_pair(imp, wo, row, L, n);
+        else z = load2(kr + 2 * n);
         be[fft_pad(n)] = z;
         bo[fft_pad(n)] = cmul(z, __ldg(twist + n));
     }
@@ -581,31 +619,38 @@ k_spectrum_8192(const TK* __restrict__ k, const float* __restrict__ D, uint8_t* 
 
 template <int M>
 cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    // FFT buffers, then (implicit filters) one row of output weights
+    const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2) + (a.implicit ? size_t(a.imp.width) * 4 : 0);
+    const unsigned grid = unsigned((p.order - 1) * p.C);
     if constexpr (M == 4096) {
-        const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
-        const unsigned grid = unsigned((p.order - 1) * p.C);
-        if (a.k_dtype == DT_F32) {
-            auto kern = k_spectrum_8192<float>;
+        if (a.implicit) {
+            auto kern = k_spectrum_8192<float, true>;
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-            kern<<<grid, 512, smem, s>>>(static_cast<const float*>(a.k), a.D, a.spectrum);
+            kern<<<grid, 512, smem, s>>>(nullptr, a.D, a.spectrum, a.imp);
+        } else if (a.k_dtype == DT_F32) {
+            auto kern = k_spectrum_8192<float, false>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            kern<<<grid, 512, smem, s>>>(static_cast<const float*>(a.k), a.D, a.spectrum, a.imp);
         } else {
-            auto kern = k_spectrum_8192<__nv_bfloat16>;
+            auto kern = k_spectrum_8192<__nv_bfloat16, false>;
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-            kern<<<grid, 512, smem, s>>>(static_cast<const __nv_bfloat16*>(a.k), a.D, a.spectrum);
+            kern<<<grid, 512, smem, s>>>(static_cast<const __nv_bfloat16*>(a.k), a.D, a.spectrum, a.imp);
         }
         return cudaGetLastError();
     }
     constexpr int NT = onchip_threads<M>();
-    const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
-    const unsigned grid = unsigned((p.order - 1) * p.C);
-    if (a.k_dtype == DT_F32) {
-        auto kern = k_spectrum_onchip<M, float>;
+    if (a.implicit) {
+        auto kern = k_spectrum_onchip<M, float, true>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        kern<<<grid, NT, smem, s>>>(static_cast<const float*>(a.k), a.D, a.spectrum, p.C, p.order);
+        kern<<<grid, NT, smem, s>>>(nullptr, a.D, a.spectrum, p.C, p.order, a.imp);
+    } else if (a.k_dtype == DT_F32) {
+        auto kern = k_spectrum_onchip<M, float, false>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        kern<<<grid, NT, smem, s>>>(static_cast<const float*>(a.k), a.D, a.spectrum, p.C, p.order, a.imp);
     } else {
-        auto kern = k_spectrum_onchip<M, __nv_bfloat16>;
+        auto kern = k_spectrum_onchip<M, __nv_bfloat16, false>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        kern<<<grid, NT, smem, s>>>(static_cast<const __nv_bfloat16*>(a.k), a.D, a.spectrum, p.C, p.order);
+        kern<<<grid, NT, smem, s>>>(static_cast<const __nv_bfloat16*>(a.k), a.D, a.spectrum, p.C, p.order, a.imp);
     }
     return cudaGetLastError();
 }
@@ -622,7 +667,8 @@ cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     int64_t grid = int64_t(2) * sms;
     if (grid > rows) grid = rows;
     kern<<<unsigned(grid), r16::NT, smem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
-                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows, a.spec_C, a.spec_per_b);
+                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows, a.spec_C, a.spec_per_b,
+                                                    a.status);
     return cudaGetLastError();
 }
 
@@ -633,7 +679,9 @@ cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         // row error ~5e-3 per order step); more order steps or fp32 storage: the
         // fp32 register kernel (the bf16-operand error of 7 steps reaches 2e-2)
         // (per-sample filters: the tensor-core kernel's two rows share one filter)
-        if (a.dtype != DT_F32 && p.order <= kMaxOrderTc && a.spec_per_b == 0) return launch_conv_8192_tc(p, a, s);
+        // (HYENA_FLAG_FP32_TRANSFORM asks for the fp32 kernel with bf16 storage too)
+        if (a.dtype != DT_F32 && p.order <= kMaxOrderTc && a.spec_per_b == 0 && !a.fp32_transform)
+            return launch_conv_8192_tc(p, a, s);
         return a.dtype == DT_F32 ? conv_4096<float>(p, a, s) : conv_4096<__nv_bfloat16>(p, a, s);
     }
     constexpr int NT = onchip_threads<M>();
@@ -643,12 +691,13 @@ cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         auto kern = k_conv_onchip<M, float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         kern<<<grid, NT, smem, s>>>(static_cast<const float*>(a.u), static_cast<float*>(a.y), a.spectrum,
-                                    a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b);
+                                    a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b, a.status);
     } else {
         auto kern = k_conv_onchip<M, __nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         kern<<<grid, NT, smem, s>>>(static_cast<const __nv_bfloat16*>(a.u), static_cast<__nv_bfloat16*>(a.y),
-                                    a.spectrum, a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b);
+                                    a.spectrum, a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b,
+                                    a.status);
     }
     return cudaGetLastError();
 }

@@ -245,19 +245,20 @@ __device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __res
 __global__ void __launch_bounds__(NT, 2)
 k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
                const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-               int64_t npairs, uint64_t wait_budget_ns, int issue_mma) {
+               int64_t npairs, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     if (!(h->magic == kSpecMagic && h->path == PATH_ONCHIP_1D && h->C == C && h->L == L && h->order == order &&
-          h->spec_row_bytes == int64_t(N) * 8))
+          h->spec_row_bytes == int64_t(N) * 8)) {
+        if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return;
+    }
     const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
     const float2* twist = tables + fft_tw_size(L / 2);        // w_L^j = w_N^(2j)
     const float2* odd = twist + L / 2 + (L / 4 + 1);          // w_N^(2j+1)
     const uint32_t* spec = reinterpret_cast<const uint32_t*>(spectrum + h->spec_off);   // plane 0 of each row
-    uint32_t* status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(spectrum) + offsetof(SpecHeader, device_status));
 
     // A: stage operands.  The stage-1 operand sits in the upper part so that
     // the previous pair's output staging (bf16 pairs, lower 32 KB) survives
@@ -629,7 +630,7 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
         have_prev = true;
         if (__syncthreads_or(!ok)) {                    // a tensor-core wait ran out (uniform decision)
             ok = false;
-            if (t == 0) atomicOr(status, 1u);
+            if (t == 0) report_status(status, kStatusTimeout);
             break;
         }
     }
@@ -654,7 +655,8 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
     int64_t grid = int64_t(2) * sms;
     if (grid > npairs) grid = npairs;
     kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
-                                           a.sc_b, a.B, p.C, p.order, npairs, a.wait_budget_ns, a.issue_mma);
+                                           a.sc_b, a.B, p.C, p.order, npairs, a.wait_budget_ns, a.issue_mma,
+                                           a.status);
     return cudaGetLastError();
 }
 

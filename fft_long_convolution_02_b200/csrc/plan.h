@@ -68,9 +68,7 @@ struct SpecHeader {
     int32_t ndim, order, path, reserved0;
     int64_t C, L, H, W, M, M1, M2;
     int64_t tables_off, tables_count, spec_off, spec_row_bytes, total_bytes;
-    // set (bit 0) by a convolution kernel whose bounded tensor-core wait gave
-    // up; reported by hyena_spectrum_check
-    uint32_t device_status, reserved1;
+    uint32_t reserved1, reserved2;
     int64_t reserved[16];
 };
 static_assert(sizeof(SpecHeader) == kHeaderBytes, "header must be 256 bytes");

@@ -10,7 +10,7 @@
 // The 16 extra bytes per chunk put the 8 chunks of one row on different
 // shared-memory banks, so a warp storing whole chunks of 8 rows is
 // conflict-free.  A 16-element K step covers two chunks; step s starts at
-// +2 s LBO.
+// +2 s LBO.  Operands written once (the DFT matrices) may use LBO = 128.
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -25,18 +25,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 // byte offset of chunk `c` (elements 8c .. 8c+7) of row `row`
-__host__ __device__ constexpr uint32_t chunk_off(int row, int c, uint32_t sbo) {
-    return uint32_t(row >> 3) * sbo + uint32_t(c) * kLBO + uint32_t(row & 7) * 16u;
+__host__ __device__ constexpr uint32_t chunk_off(int row, int c, uint32_t sbo, uint32_t lbo = kLBO) {
+    return uint32_t(row >> 3) * sbo + uint32_t(c) * lbo + uint32_t(row & 7) * 16u;
 }
-__host__ __device__ constexpr uint32_t kmaj_off(int row, int k, uint32_t sbo) {
-    return chunk_off(row, k >> 3, sbo) + uint32_t(k & 7) * 2u;
+__host__ __device__ constexpr uint32_t kmaj_off(int row, int k, uint32_t sbo, uint32_t lbo = kLBO) {
+    return chunk_off(row, k >> 3, sbo, lbo) + uint32_t(k & 7) * 2u;
 }
 
 // Shared-memory matrix descriptor (sm_100 UMMA, version 1, no swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t sbo) {
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t sbo, uint32_t lbo = kLBO) {
     uint64_t d = 0;
     d |= uint64_t((saddr >> 4) & 0x3FFFu);
-    d |= uint64_t(kLBO >> 4) << 16;
+    d |= uint64_t(lbo >> 4) << 16;
     d |= uint64_t(sbo >> 4) << 32;
     d |= uint64_t(1) << 46;
     return d;
@@ -149,6 +149,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(v[i]);
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+// Arrive on `mbar` and expect `bytes` of asynchronous transactions (TMA).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
+                 : "memory");
+}
 
 }  // namespace tc
 }  // namespace hyena

@@ -44,6 +44,8 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 TAG_U, TAG_K, TAG_D, TAG_SCW, TAG_TOK, TAG_EMB, TAG_SCB = 1, 2, 3, 4, 5, 6, 7
+TAG_X, TAG_WIN, TAG_BIN, TAG_WOUT, TAG_BOUT = 8, 9, 10, 11, 12
+TAG_FILT = 13
 
 
 @dataclass(frozen=True)
@@ -222,6 +224,40 @@ def make_k(p: Problem) -> np.ndarray:
         for c in range(p.FC):
             out[s, c] = store(p, k_row(p, s, c)).reshape(p.shape)
     return out
+
+
+def make_layer(p: Problem) -> dict:
+    """Inputs of the layer around the operator (1-D, width D = C): the token
+    stream x [B, L, D] ~ N(0, 1), and the in/out projections with the default
+    nn.Linear initialisation ranges, weights and biases U(-1/sqrt(D), 1/sqrt(D)):
+    W_in [(order+1) D, D], b_in [(order+1) D], W_out [D, D], b_out [D].  x and
+    the weights in the problem's storage type, the biases float32."""
+    D, J = p.C, p.Ctot
+    r = 1.0 / np.sqrt(D)
+    x = np.empty((p.B, p.L, D), dtype=np.uint16 if p.dtype == "bf16" else np.float32)
+    for b in range(p.B):
+        x[b] = store(p, _rng(p, TAG_X, b).standard_normal((p.L, D), dtype=np.float32))
+    W_in = store(p, _rng(p, TAG_WIN).uniform(-r, r, (J, D)).astype(np.float32))
+    b_in = _rng(p, TAG_BIN).uniform(-r, r, J).astype(np.float32)
+    W_out = store(p, _rng(p, TAG_WOUT).uniform(-r, r, (D, D)).astype(np.float32))
+    b_out = _rng(p, TAG_BOUT).uniform(-r, r, D).astype(np.float32)
+    return {"x": x, "W_in": W_in, "b_in": b_in, "W_out": W_out, "b_out": b_out}
+
+
+def implicit_filter_params(p: Problem, width: int = 64, emb_dim: int = 3, num_inner: int = 2) -> dict:
+    """Synthetic parameters of the implicit filter (HyenaFilter) for the
+    (order-1) C filters of problem p: the default nn.Linear ranges
+    U(-1/sqrt(fan_in), 1/sqrt(fan_in)) for weights and biases, Sin
+    frequencies w ~ U[0.5, 2] around the default 1, decay rates alpha over
+    the workload's range p.decay (float32 arrays)."""
+    g = _rng(p, TAG_FILT)
+    dm = (p.order - 1) * p.C
+    u = lambda fan, shape: g.uniform(-1 / np.sqrt(fan), 1 / np.sqrt(fan), shape).astype(np.float32)
+    return {"emb_dim": emb_dim, "width": width, "num_inner": num_inner,
+            "W_in": u(emb_dim, (width, emb_dim)), "b_in": u(emb_dim, width),
+            "W_inner": u(width, (num_inner, width, width)), "b_inner": u(width, (num_inner, width)),
+            "W_out": u(width, (dm, width)), "w": g.uniform(0.5, 2.0, width).astype(np.float32),
+            "alpha": g.uniform(p.decay[0], p.decay[1], dm).astype(np.float32)}
 
 
 def make_all(p: Problem) -> dict:

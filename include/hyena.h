@@ -22,8 +22,18 @@
  *  - Tensors are row-major, last dimension contiguous: 1-D [.., L], 2-D
  *    [.., H, W].  sizes = {L} for ndim 1, {H, W} for ndim 2.
  *  - dtype selects the storage of u, y (and of k in hyena_filter_spectrum):
- *    HYENA_F32 or HYENA_BF16 (round-to-nearest-even on store).  Arithmetic is
- *    fp32 throughout; spectra are stored as complex64.
+ *    HYENA_F32 or HYENA_BF16 (round-to-nearest-even on store).  Arithmetic:
+ *    the short conv, the gates, the twiddles and the spectrum products are
+ *    fp32 on every path.  With fp32 storage, and on every path other than
+ *    1-D L = 8192 with bf16 storage, the transforms are fp32 too and the
+ *    spectrum is read as complex64.  At L = 8192 with bf16 storage (order
+ *    <= 3, shared filters) the DFT stages run on the tensor cores: their
+ *    operands and the DFT matrices are rounded to bf16 and accumulated in
+ *    fp32, and the spectrum is read as bf16 (re, im) pairs (row error a few
+ *    1e-3); HYENA_FLAG_FP32_TRANSFORM (hyena_gated_fftconv_ex) selects the
+ *    fp32 transform there instead.  With bf16 storage the intermediate of the
+ *    multi-pass (L >= 32768) and N-D paths is kept as bf16 pairs in the
+ *    workspace.
  *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
  *    stream) and is asynchronous: no call synchronises the host.
  *  - Arguments are validated before anything is enqueued; on any error
@@ -58,7 +68,7 @@ typedef enum {
     HYENA_ERR_CUDA = 6,               /* a CUDA launch reported an error              */
     HYENA_ERR_INTERNAL = 7,
     HYENA_ERR_TIMEOUT = 8             /* a bounded device wait ran out (reported by
-                                         hyena_spectrum_check)                       */
+                                         hyena_kernel_status)                        */
 } hyena_status_t;
 
 /*
@@ -115,6 +125,54 @@ hyena_status_t hyena_filter_spectrum(const void* k, hyena_dtype_t k_dtype, const
                                      size_t spectrum_bytes, void* stream);
 
 /*
+ * Parameters of the implicit long filter (device pointers, fp32, row-major).
+ * Source: [P4] section 二.2, HyenaFilter: filter(L) = modulation(t,
+ * implicit_filter(pos_emb(L))) with
+ *   pos_emb(l)   = [t_l, cos(2 pi b l / L), sin(2 pi b l / L)], b = 1 .. (emb_dim-1)/2,
+ *                  t_l = l / (L-1)
+ *   implicit_filter = Linear(emb_dim, width) -> Sin, num_inner x
+ *                  (Linear(width, width) -> Sin), Linear(width, d_model)
+ *                  without bias; Sin(x) = sin(w * x), w per feature
+ *   modulation   = h[l][c] exp(-alpha[c] t_l)
+ * with d_model = (order-1) C outputs taken as 'l (o d) -> o d l' (output
+ * channel s*C + c is the filter of order step s, channel c).
+ */
+typedef struct {
+    int emb_dim;            /* odd, 3 .. 33 */
+    int width;              /* 1 .. 128 (the HyenaOperator passes filter_order = 64) */
+    int num_inner;          /* 0 .. 8 */
+    const float* W_in;      /* [width, emb_dim] */
+    const float* b_in;      /* [width] */
+    const float* W_inner;   /* [num_inner, width, width], or NULL when num_inner = 0 */
+    const float* b_inner;   /* [num_inner, width], or NULL when num_inner = 0 */
+    const float* W_out;     /* [(order-1) C, width] */
+    const float* w;         /* [width] Sin frequencies */
+    const float* alpha;     /* [(order-1) C] decay rates */
+} hyena_implicit_filter_t;
+
+/* Workspace bytes of hyena_filter_spectrum_implicit: width x L fp32 (0 for bad arguments). */
+size_t hyena_implicit_filter_workspace_bytes(int64_t L, int width);
+
+/*
+ * hyena_filter_spectrum_implicit -- S0 from the implicit filter: the filters
+ * are generated on the device and go straight into the spectrum build.
+ *
+ * Fills `spectrum` exactly as hyena_filter_spectrum(k, HYENA_F32, D, C,
+ * ndim 1, {L}, order, ...) would for the filters k [order-1, C, L] the
+ * parameters generate; use it with hyena_gated_fftconv like any spectrum.
+ * The MLP's hidden layers are evaluated once for all t into `workspace`
+ * (hyena_implicit_filter_workspace_bytes), and each filter row is computed
+ * inside the spectrum kernel, so the filters are not written to memory
+ * unless k_out is given: k_out [order-1, C, L] fp32 (8-byte aligned)
+ * receives a copy of them (for checking), or NULL.
+ * L: the on-chip lengths, powers of two in [16, 16384]; D as in
+ * hyena_filter_spectrum.  Asynchronous on `stream`.
+ */
+hyena_status_t hyena_filter_spectrum_implicit(const hyena_implicit_filter_t* f, const float* D, int64_t C, int64_t L,
+                                              int order, void* spectrum, size_t spectrum_bytes, void* workspace,
+                                              size_t workspace_bytes, float* k_out, void* stream);
+
+/*
  * hyena_shortconv -- S1 on its own (1-D only).
  *
  * Source: [P4] section 二.1, short_filter = Conv1d(inner, inner, 3, padding=2,
@@ -159,11 +217,53 @@ size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_
  *   workspace, workspace_bytes  device scratch for the multi-pass (L >= 32768)
  *            and 2-D paths; may be NULL/0 for the on-chip path.  Its contents
  *            are undefined after the call.
+ *
+ * The spectrum is only read.  Conditions the kernels detect on the device (a
+ * spectrum whose header does not match the shape: that kernel writes no
+ * output; a bounded tensor-core wait that ran out: NaN outputs) are recorded
+ * in the device's status word, see hyena_kernel_status.
  */
 hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
                                    const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
                                    const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
                                    size_t workspace_bytes, void* stream);
+
+/* Flags of hyena_gated_fftconv_ex. */
+#define HYENA_FLAG_FP32_TRANSFORM 0x1u  /* every transform multiply in fp32 on the CUDA cores (no bf16 tensor-core
+                                           operands); changes only 1-D L = 8192 with bf16 storage */
+
+/*
+ * hyena_gated_fftconv_ex -- hyena_gated_fftconv with flags (shared filters).
+ * flags: 0 (same as hyena_gated_fftconv) or HYENA_FLAG_FP32_TRANSFORM; other
+ * bits are rejected with HYENA_ERR_INVALID_ARG.  The pages fix no precision
+ * for the transform; this lets a caller pick fp32 arithmetic throughout
+ * (bf16 storage, fp32 math) at the cost of speed at L = 8192.
+ */
+hyena_status_t hyena_gated_fftconv_ex(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                      const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int ndim,
+                                      const int64_t* sizes, int order, hyena_dtype_t dtype, void* workspace,
+                                      size_t workspace_bytes, unsigned flags, void* stream);
+
+/*
+ * hyena_kernel_status -- what the convolution kernels detected on this device
+ * since the last call (the current device's status word, which every
+ * convolution kernel on the device may set; reading clears it).
+ *
+ * The paper has no counterpart: a kernel cannot return an error, so this is
+ * how conditions seen on the device reach the caller.  Synchronises `stream`
+ * (make it the stream of the calls in question, or NULL), then returns
+ * HYENA_OK, HYENA_ERR_TIMEOUT (a bounded wait for tensor-core work ran out:
+ * the L = 8192 bf16 path wrote NaN to that row pair's outputs and left
+ * nothing in flight) or HYENA_ERR_SPECTRUM_MISMATCH (a kernel found a
+ * spectrum header that does not match the shape it was given -- never
+ * filled, or filled for another C, size or order of the same byte size --
+ * and wrote no output), or HYENA_ERR_CUDA.  The word is per device, not per
+ * stream or per call: kernels running on other streams meanwhile may set
+ * bits between the read and the clear, and those bits are lost.  Its address
+ * is looked up once per device (calls after a device reset are not
+ * supported).
+ */
+hyena_status_t hyena_kernel_status(void* stream);
 
 /*
  * hyena_gated_fftconv_per_sample -- S1..S9 with one long filter per (b, c)
@@ -199,7 +299,9 @@ hyena_status_t hyena_gated_fftconv_per_sample(const void* u, void* y, const void
  *
  * The paper has no counterpart: this entry point is for callers whose stream
  * of inputs sits in host memory (serving, or data larger than the device).
- * The batch is cut into chunks of chunk_rows batch rows (0: ceil(B/4)); each
+ * The batch is cut into chunks of chunk_rows batch rows (0: ceil(B/4), rounded
+ * up to an even count when B allows, because the L = 8192 bf16 kernel
+ * transforms two batch rows of a channel together); each
  * chunk is copied to u_dev, convolved and copied back to y_host, alternately
  * on `stream` and on a second stream the library keeps per device, so one
  * chunk's host-to-device copy overlaps the previous chunk's kernel and
@@ -219,6 +321,42 @@ hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* 
                                         const float* sc_bias, int64_t B, int64_t C, int ndim, const int64_t* sizes,
                                         int order, hyena_dtype_t dtype, void* workspace, size_t workspace_bytes,
                                         int64_t chunk_rows, void* stream);
+
+/*
+ * hyena_in_proj -- the input projection of the Hyena operator on the tensor
+ * cores.
+ *
+ * Source: [P4] section 二.1, HyenaOperator: in_proj = nn.Linear(d_model,
+ * (order+1) d_model) on u [b, l, d], then rearrange 'b l d -> b d l':
+ *   u[b][j][l] = sum_i x[b][l][i] W[j][i] + bias[j],   j < (order+1) D.
+ *
+ *   x     [B, L, D] bf16 (features contiguous)
+ *   W     [(order+1) D, D] bf16, the nn.Linear weight (out x in)
+ *   bias  [(order+1) D] fp32, or NULL (= 0)
+ *   u     [B, (order+1) D, L] bf16 out: the layout hyena_gated_fftconv reads
+ * bf16 operands, fp32 accumulation, bf16 result (round to nearest even).
+ * D and L multiples of 8; pointers 16-byte aligned (bias 4-byte); u may not
+ * overlap x or W.  Asynchronous on `stream`; errors as for the other calls; a
+ * bounded device wait that runs out is reported by hyena_kernel_status.
+ */
+hyena_status_t hyena_in_proj(const void* x, const void* W, const float* bias, void* u, int64_t B, int64_t L,
+                             int64_t D, int order, void* stream);
+
+/*
+ * hyena_out_proj -- the output projection on the tensor cores.
+ *
+ * Source: [P4] section 二.1: y = rearrange(v * x[0], 'b d l -> b l d'), then
+ * out_proj = nn.Linear(d_model, d_model):
+ *   out[b][l][j] = sum_i y[b][i][l] W[j][i] + bias[j],   j < D.
+ *
+ *   y     [B, D, L] bf16, the output of hyena_gated_fftconv (read in place,
+ *         no transposed copy)
+ *   W     [D, D] bf16 (out x in);  bias [D] fp32 or NULL
+ *   out   [B, L, D] bf16
+ * Same precision, shape, alignment and error rules as hyena_in_proj.
+ */
+hyena_status_t hyena_out_proj(const void* y, const void* W, const float* bias, void* out, int64_t B, int64_t L,
+                              int64_t D, void* stream);
 
 /*
  * Size of the fixed scratch array used by hyena_gated_fftconv_noalloc (32 MiB).
@@ -242,11 +380,16 @@ hyena_status_t hyena_gated_fftconv_host(const void* u_host, void* y_host, void* 
  *
  *  - Limit: shapes whose workspace row (hyena_gated_fftconv_workspace_min_bytes)
  *    exceeds HYENA_NOALLOC_SCRATCH_BYTES are rejected with
- *    HYENA_ERR_WORKSPACE_TOO_SMALL; rows are processed in groups that fit.
+ *    HYENA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued (a 128^3
+ *    volume, for example); rows are processed in groups that fit (at
+ *    L = 2^20: 4 rows per group with fp32 storage, 8 with bf16 storage).
  *  - Set-up: the first call on each device looks up the array's device
  *    address (cudaGetSymbolAddress, with that device current), which may load
  *    the library's device code; make that first call before any stream
- *    capture.
+ *    capture.  The address is kept for the life of the process: after
+ *    cudaDeviceReset (or anything else that tears down and recreates the
+ *    device's primary context) the array may live elsewhere, so calls after
+ *    such a reset are not supported.
  *  - Sharing: every call on a device uses the same array, which keeps the
  *    last call's contents.  No zeroing is needed: each call writes every
  *    scratch element before reading it.  Calls that overlap on the GPU (for
@@ -260,11 +403,7 @@ hyena_status_t hyena_gated_fftconv_noalloc(const void* u, void* y, const void* s
  * Debug helper (synchronous): copies the spectrum header to the host and
  * checks it against (C, sizes, order).  Returns HYENA_OK when it matches,
  * HYENA_ERR_SPECTRUM_MISMATCH when not (e.g. never filled, or filled for
- * another shape), HYENA_ERR_TIMEOUT when an earlier convolution with this
- * spectrum ran out of the budget of a bounded tensor-core wait (the L = 8192
- * bf16 path; the outputs of that row pair were written as NaN and nothing was
- * left in flight).  Synchronises `stream`.  Rebuilding the spectrum clears the
- * record.
+ * another shape).  Synchronises `stream`.
  */
 hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, const int64_t* sizes, int order,
                                     void* stream);
@@ -276,7 +415,7 @@ hyena_status_t hyena_spectrum_check(const void* spectrum, int64_t C, int ndim, c
  * tensor-core work gives up after `wait_budget_ns` nanoseconds (the normal entry
  * point uses 2 s).  With issue_mma = 0 no tensor-core work is issued, so the
  * first wait runs out on a barrier that nothing completes: the kernel records
- * the timeout in the spectrum header (hyena_spectrum_check then returns
+ * the timeout in the device's status word (hyena_kernel_status then returns
  * HYENA_ERR_TIMEOUT), writes NaN to the outputs of the row pair it was on, and
  * returns with nothing in flight.  Other shapes return
  * HYENA_ERR_UNSUPPORTED_SHAPE.  Asynchronous on `stream`.

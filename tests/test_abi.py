@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.hyena_version() == 100
+    assert lib.hyena_version() == 101
     for code, name in hb.STATUS.items():
         assert lib.hyena_status_string(code).decode() == name
 
@@ -139,6 +139,36 @@ def test_validation_errors_before_launch(lib):
     assert dg(big, big * 2, big * 3, n8o4, None, None, 2, 4, 4, 1000, 0, None) == 2
     assert dg(big, big * 2, big * 3, n8, None, None, 2, 4, 2, 0, 0, None) == 1
     assert dg(big, big * 2, big * 3, n8 + 16, None, None, 2, 4, 2, 1000, 0, None) == 4
+    # projections: NULLs, shapes, order, alignment, overlap (no launch)
+    ip, op = lib.hyena_in_proj, lib.hyena_out_proj
+    assert ip(None, fake, None, fake * 4, 1, 64, 64, 2, None) == 1
+    assert ip(fake, fake * 2, None, fake * 4, 1, 64, 60, 2, None) == 2          # D not a multiple of 8
+    assert ip(fake, fake * 2, None, fake * 4, 1, 60, 64, 2, None) == 2          # L not a multiple of 8
+    assert ip(fake, fake * 2, None, fake * 4, 1, 64, 64, 9, None) == 2          # order
+    assert ip(fake + 8, fake * 2, None, fake * 4, 1, 64, 64, 2, None) == 3
+    assert ip(fake, fake * 2, None, fake + 64, 1, 64, 64, 2, None) == 1          # u overlaps x
+    assert op(fake, fake * 2, fake * 3 + 2, fake * 4, 1, 64, 64, None) == 3      # bias misaligned
+    assert op(fake, fake * 2, None, fake + 16, 1, 64, 64, None) == 1             # out overlaps y
+    assert op(fake, fake * 2, None, fake * 4, 0, 64, 64, None) == 1
+    # implicit filters: parameter checks before any launch
+    assert lib.hyena_implicit_filter_workspace_bytes(8192, 64) == 8192 * 64 * 4
+    assert lib.hyena_implicit_filter_workspace_bytes(8192, 129) == 0
+    fi = lib.hyena_filter_spectrum_implicit
+    assert fi(None, None, 4, 1024, 2, fake, nbytes, fake, 1 << 20, None, None) == 1
+    prm = hb.ImplicitFilter(3, 64, 2, fake, fake, fake, fake, fake, fake, fake)
+    n1 = lib.hyena_spectrum_bytes(4, 1, _sz(1024), 2)
+    bad = hb.ImplicitFilter(4, 64, 2, fake, fake, fake, fake, fake, fake, fake)
+    assert fi(ctypes.byref(bad), None, 4, 1024, 2, fake, n1, fake, 1024 * 64 * 4, None, None) == 1
+    noinner = hb.ImplicitFilter(3, 64, 2, fake, fake, None, None, fake, fake, fake)
+    assert fi(ctypes.byref(noinner), None, 4, 1024, 2, fake, n1, fake, 1024 * 64 * 4, None, None) == 1
+    assert fi(ctypes.byref(prm), None, 4, 1024, 2, fake, n1, fake, 1024 * 64 * 4 - 4, None, None) == 5
+    assert fi(ctypes.byref(prm), None, 4, 1024, 2, fake, n1 + 16, fake, 1024 * 64 * 4, None, None) == 4
+    assert fi(ctypes.byref(prm), None, 4, 1 << 15, 2, fake, n1, fake, 1 << 30, None, None) == 2
+    # flags entry point: unknown bits first, then the same checks as hyena_gated_fftconv
+    gx = lib.hyena_gated_fftconv_ex
+    assert gx(fake, fake * 4, fake * 8, nbytes, None, None, 1, 64, 1, sizes, 2, 0, None, 0, 0x2, None) == 1
+    assert "flag" in _detail(lib)
+    assert gx(fake, fake * 4, fake * 8, nbytes + 16, None, None, 1, 64, 1, sizes, 2, 0, None, 0, 0x1, None) == 4
 
 
 def test_status_strings(lib):

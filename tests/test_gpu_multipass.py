@@ -67,17 +67,20 @@ def test_multipass_no_shortconv(orc):
 
 
 def test_order3_workload_full_size_sampled_rows(orc):
-    """B=2 C=2048 L=65536 order 3 bf16 at full size; 24 seeded rows vs the oracle."""
+    """B=2 C=2048 L=65536 order 3 bf16 at full size; 66 seeded rows (the
+    first, the last and 64 drawn) vs the oracle."""
     p = I.WORKLOADS["order3"]
-    rows = np.random.default_rng(8).choice(p.B * p.C, 22, replace=False)
+    rows = np.random.default_rng(8).choice(np.arange(1, p.B * p.C - 1), 64, replace=False)
     rows = np.concatenate([[0, p.B * p.C - 1], rows])
     _check(orc, p, rows=rows)
 
 
 def test_dna_1m_workload_full_size_sampled_rows(orc):
-    """B=1 C=256 L=2^20 order 2 bf16 (ACGT embedding) at full size; 8 rows vs the oracle."""
+    """B=1 C=256 L=2^20 order 2 bf16 (ACGT embedding) at full size; 66 seeded
+    rows (the first, the last and 64 drawn) vs the oracle."""
     p = I.WORKLOADS["dna_1m"]
-    rows = np.array([0, 1, 77, 128, 200, 254, 255, 31])
+    rows = np.random.default_rng(12).choice(np.arange(1, p.B * p.C - 1), 64, replace=False)
+    rows = np.concatenate([[0, p.B * p.C - 1], rows])
     _check(orc, p, rows=rows)
 
 
@@ -101,12 +104,10 @@ def test_grid2d_small_workspace(orc):
     _check(orc, p, workspace_bytes=one)
 
 
-def test_grid2d_workload_full_size_sampled_images(orc):
-    """B=2 C=256 256x256 order 2 bf16 at full size; 16 seeded images vs the oracle."""
+def test_grid2d_workload_full_size_all_images(orc):
+    """B=2 C=256 256x256 order 2 bf16 at full size; all 512 images vs the oracle."""
     p = I.WORKLOADS["grid2d"]
-    rows = np.random.default_rng(9).choice(p.B * p.C, 14, replace=False)
-    rows = np.concatenate([[0, p.B * p.C - 1], rows])
-    _check(orc, p, rows=rows)
+    _check(orc, p, rows=np.arange(p.B * p.C))
 
 
 def test_grid2d_delta_gives_kernel_plus_D():
