@@ -36,26 +36,65 @@ namespace {
 constexpr int kMaxWidth = 128;
 constexpr int kMaxEmb = 33;
 constexpr int kMaxInner = 8;
-constexpr int kTT = 32;            // time steps per block
-constexpr int kThreadsH = 128;     // thread j computes feature j (j < width)
+constexpr int kTT = 64;            // time steps per block
+constexpr int kThreadsH = 128;     // 16 feature groups of 4 x 8 time groups of 8
 
-// Dynamic shared memory: WT [max(emb, width)][width + 1] (a layer's weight,
-// transposed), h [2][kTT][width + 1], z [kTT][emb_dim].
+// One layer of the MLP on a tile of kTT time steps: out[j][t] = sin(w[j] *
+// (bias[j] + sum_i WT[i][j] in[i][t])) for j < W, with WT [K][WP4] (the
+// weight transposed, rows padded to a multiple of 4) and in/out [.][kTT]
+// (feature-major).  Thread (jg, tg) computes features 4 jg + 64 r (r <
+// ceil(W / 64)) at time steps 8 tg .. 8 tg + 7 as a 4 x 8 register tile.
+__device__ __forceinline__ void mlp_layer(const float* WT, int WP4, const float* in, int K, const float* bias,
+                                          const float* w, int W, float* out) {
+    const int jg = int(threadIdx.x) & 15, tg = int(threadIdx.x) >> 4;
+    for (int j0 = 4 * jg; j0 < W; j0 += 64) {
+        float acc[4][8];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float b = j0 + a < W ? __ldg(bias + j0 + a) : 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[a][e] = b;
+        }
+        for (int i = 0; i < K; ++i) {
+            const float4 wv = *reinterpret_cast<const float4*>(WT + i * WP4 + j0);
+            const float4 h0 = *reinterpret_cast<const float4*>(in + i * kTT + 8 * tg);
+            const float4 h1 = *reinterpret_cast<const float4*>(in + i * kTT + 8 * tg + 4);
+            const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            const float hh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(ww[a], hh[e], acc[a][e]);
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            if (j0 + a >= W) continue;
+            const float wj = __ldg(w + j0 + a);
+            float4* o = reinterpret_cast<float4*>(out + (j0 + a) * kTT + 8 * tg);
+            o[0] = make_float4(sinf(wj * acc[a][0]), sinf(wj * acc[a][1]), sinf(wj * acc[a][2]), sinf(wj * acc[a][3]));
+            o[1] = make_float4(sinf(wj * acc[a][4]), sinf(wj * acc[a][5]), sinf(wj * acc[a][6]), sinf(wj * acc[a][7]));
+        }
+    }
+}
+
+// Dynamic shared memory: WT [max(emb, width)][WP4] (a layer's weight,
+// transposed), h [2][width][kTT] (feature-major), z [emb_dim][kTT].
 __global__ void __launch_bounds__(kThreadsH)
 k_filter_hidden(ImplicitMlp m, int64_t L, float* __restrict__ hT) {
-    extern __shared__ float sm[];
-    const int W = m.width, E = m.emb_dim, WP = W + 1;
+    extern __shared__ __align__(16) float sm[];
+    const int W = m.width, E = m.emb_dim;
+    const int WP4 = (W + 3) & ~3;
     const int rows = E > W ? E : W;
     float* WT = sm;
-    float* h0 = WT + rows * WP;
-    float* h1 = h0 + kTT * WP;
-    float* z = h1 + kTT * WP;
+    float* h0 = WT + rows * WP4;
+    float* h1 = h0 + WP4 * kTT;
+    float* z = h1 + WP4 * kTT;
     const int64_t t0 = int64_t(blockIdx.x) * kTT;
-    const int j = int(threadIdx.x);
-    // positional embedding of the tile's time steps
+    const int tid = int(threadIdx.x);
+    // positional embedding of the tile's time steps (feature-major)
     const int nb = (E - 1) / 2;
-    for (int idx = j; idx < kTT * E; idx += kThreadsH) {
-        const int tt = idx / E, f = idx % E;
+    for (int idx = tid; idx < kTT * E; idx += kThreadsH) {
+        const int f = idx / kTT, tt = idx % kTT;
         const int64_t l = t0 + tt;
         float v = 0.0f;
         if (l < L) {
@@ -70,61 +109,36 @@ k_filter_hidden(ImplicitMlp m, int64_t L, float* __restrict__ hT) {
                 v = f <= nb ? cv : sv;
             }
         }
-        z[tt * E + f] = v;
+        z[f * kTT + tt] = v;
     }
     // first layer: h = Sin(W_in z + b_in)
-    for (int idx = j; idx < W * E; idx += kThreadsH) {
+    for (int idx = tid; idx < W * E; idx += kThreadsH) {
         const int o = idx / E, i = idx % E;
-        WT[i * WP + o] = __ldg(m.W_in + idx);
+        WT[i * WP4 + o] = __ldg(m.W_in + idx);
     }
     __syncthreads();
-    const float wj = j < W ? __ldg(m.w + j) : 0.0f;
-    if (j < W) {
-        const float bj = __ldg(m.b_in + j);
-        float acc[kTT];
-#pragma unroll
-        for (int tt = 0; tt < kTT; ++tt) acc[tt] = bj;
-        for (int i = 0; i < E; ++i) {
-            const float wv = WT[i * WP + j];
-#pragma unroll
-            for (int tt = 0; tt < kTT; ++tt) acc[tt] = fmaf(wv, z[tt * E + i], acc[tt]);
-        }
-#pragma unroll
-        for (int tt = 0; tt < kTT; ++tt) h0[tt * WP + j] = sinf(wj * acc[tt]);
-    }
+    mlp_layer(WT, WP4, z, E, m.b_in, m.w, W, h0);
     float* cur = h0;
     float* nxt = h1;
     // inner layers: h = Sin(W h + b)
     for (int layer = 0; layer < m.num_inner; ++layer) {
-        __syncthreads();                               // previous layer done with WT and cur complete
+        __syncthreads();                               // previous layer done with WT, cur complete
         const float* Wl = m.W_inner + int64_t(layer) * W * W;
-        for (int idx = j; idx < W * W; idx += kThreadsH) {
+        for (int idx = tid; idx < W * W; idx += kThreadsH) {
             const int o = idx / W, i = idx % W;
-            WT[i * WP + o] = __ldg(Wl + idx);
+            WT[i * WP4 + o] = __ldg(Wl + idx);
         }
         __syncthreads();
-        if (j < W) {
-            const float bj = __ldg(m.b_inner + int64_t(layer) * W + j);
-            float acc[kTT];
-#pragma unroll
-            for (int tt = 0; tt < kTT; ++tt) acc[tt] = bj;
-            for (int i = 0; i < W; ++i) {
-                const float wv = WT[i * WP + j];
-#pragma unroll
-                for (int tt = 0; tt < kTT; ++tt) acc[tt] = fmaf(wv, cur[tt * WP + i], acc[tt]);
-            }
-#pragma unroll
-            for (int tt = 0; tt < kTT; ++tt) nxt[tt * WP + j] = sinf(wj * acc[tt]);
-        }
+        mlp_layer(WT, WP4, cur, W, m.b_inner + int64_t(layer) * W, m.w, W, nxt);
         float* sw = cur;
         cur = nxt;
         nxt = sw;
     }
     __syncthreads();
     // hT[f][t] for the tile (consecutive t per feature row)
-    for (int idx = j; idx < W * kTT; idx += kThreadsH) {
+    for (int idx = tid; idx < W * kTT; idx += kThreadsH) {
         const int f = idx / kTT, tt = idx % kTT;
-        if (t0 + tt < L) hT[int64_t(f) * L + t0 + tt] = cur[tt * WP + f];
+        if (t0 + tt < L) hT[int64_t(f) * L + t0 + tt] = cur[f * kTT + tt];
     }
 }
 
@@ -134,7 +148,8 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 cudaError_t launch_filter_hidden(const ImplicitMlp& m, int64_t L, float* hT, cudaStream_t s) {
     const int rows = m.emb_dim > m.width ? m.emb_dim : m.width;
-    const size_t smem = (size_t(rows) * (m.width + 1) + size_t(2) * kTT * (m.width + 1) + size_t(kTT) * m.emb_dim) * 4;
+    const int wp4 = (m.width + 3) & ~3;
+    const size_t smem = (size_t(rows) * wp4 + size_t(2) * wp4 * kTT + size_t(kTT) * m.emb_dim) * 4;
     cudaError_t e = cudaFuncSetAttribute(k_filter_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     const unsigned grid = unsigned((L + kTT - 1) / kTT);

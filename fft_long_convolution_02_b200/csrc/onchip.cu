@@ -47,8 +47,21 @@ __device__ __forceinline__ bool header_ok(const uint8_t* spec, int64_t C, int64_
 __device__ __forceinline__ float2 implicit_pair(const ImplicitFilter& f, const float* wo, int64_t row, int L, int n) {
     float a0 = 0.0f, a1 = 0.0f;
     const float2* h = reinterpret_cast<const float2*>(f.hT) + n;
-    for (int j = 0; j < f.width; ++j) {
-        const float2 v = __ldg(h + int64_t(j) * (L / 2));
+    const int64_t hs = L / 2;                  // float2 stride between hidden features
+    int j = 0;
+    // eight independent loads in flight per batch
+    for (; j + 8 <= f.width; j += 8) {
+        float2 v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = __ldg(h + int64_t(j + e) * hs);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            a0 = fmaf(v[e].x, wo[j + e], a0);
+            a1 = fmaf(v[e].y, wo[j + e], a1);
+        }
+    }
+    for (; j < f.width; ++j) {
+        const float2 v = __ldg(h + int64_t(j) * hs);
         a0 = fmaf(v.x, wo[j], a0);
         a1 = fmaf(v.y, wo[j], a1);
     }

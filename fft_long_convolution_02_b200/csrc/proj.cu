@@ -16,11 +16,11 @@
 //             C = out[b] row-major [L][D].
 //
 // Kernel: persistent, one CTA per SM, 192 threads in three roles:
-//   warp 0   loads A and B tiles (128 x 64 and 256 x 64 bf16, 128-byte swizzle)
+//   warp 0   loads A and B tiles (128 x 64 and BN x 64 bf16, 128-byte swizzle)
 //            with TMA (cp.async.bulk.tensor, no multicast) into a ring of
 //            kStages stages, each completing on a "full" mbarrier;
-//   warp 1   issues tcgen05.mma (M 128, N 256, K 16; four per 64-wide K block)
-//            into one of two 256-column tensor-memory accumulators, frees each
+//   warp 1   issues tcgen05.mma (M 128, N BN, K 16; four per 64-wide K block)
+//            into one of two BN-column tensor-memory accumulators, frees each
 //            stage with tcgen05.commit to its "empty" mbarrier, and signals a
 //            finished tile with a commit to "acc_full";
 //   warps 2-5 (the epilogue) read the accumulator rows with tcgen05.ld, add the
@@ -48,16 +48,30 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kStages = 4;
+constexpr int BM = 128, BK = 64;
 constexpr uint32_t kATile = BM * BK * 2;          // 16 KB
-constexpr uint32_t kBTile = BN * BK * 2;          // 32 KB
-constexpr uint32_t kStageBytes = kATile + kBTile;
 constexpr int kThreadsG = 192;
-constexpr uint32_t kAccCols = 256;                // one fp32 accumulator (BN columns)
-constexpr uint32_t kTmemColsG = 2 * kAccCols;
-// shared memory: 1024-byte aligned stages, then the barriers
-constexpr size_t kSmemG = 1024 + size_t(kStages) * kStageBytes + 256;
+// Epilogue staging: per epilogue warp 32 rows x 64 columns of bf16, rows
+// 144 bytes apart (128 + 16), so that a thread writing its row's 16-byte
+// chunks and a warp reading 4 rows x 128 contiguous bytes are both free of
+// bank conflicts.
+constexpr uint32_t kEpiRow = 144;
+constexpr uint32_t kEpiWarp = 32 * kEpiRow;
+constexpr uint32_t kEpiBytes = 4 * kEpiWarp;
+
+// Tile width BN (256, or 128 when the wider tiles would leave the grid with
+// few waves): B tile, stage size, ring depth, tensor-memory columns (two
+// accumulators of BN fp32 columns) and shared memory (1024-byte aligned
+// stages, then the barriers).
+template <int BN>
+struct Cfg {
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr uint32_t kBTile = BN * BK * 2;
+    static constexpr uint32_t kStageBytes = kATile + kBTile;
+    static constexpr uint32_t kAccCols = BN;
+    static constexpr uint32_t kTmemCols = 2 * BN;
+    static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + 256 + (BN == 256 ? kEpiBytes : 0);
+};
 
 struct GemmParams {
     int64_t M, N, K, batches;
@@ -103,8 +117,13 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kThreadsG, 1)
 k_gemm_bf16(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, GemmParams p) {
+    constexpr int kStages = Cfg<BN>::kStages;
+    constexpr uint32_t kStageBytes = Cfg<BN>::kStageBytes;
+    constexpr uint32_t kAccCols = Cfg<BN>::kAccCols;
+    constexpr uint32_t kTmemColsG = Cfg<BN>::kTmemCols;
     extern __shared__ __align__(1024) uint8_t smem_g[];
     // the stages start at the first 1024-byte boundary (128-byte swizzle atoms)
     const uint32_t base_s = tc::smem_u32(smem_g);
@@ -115,6 +134,7 @@ k_gemm_bf16(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* mma_done = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint8_t* epi = stages + kStages * kStageBytes + 256;     // epilogue staging (kEpiBytes)
 
     const int warp = int(threadIdx.x) >> 5, lane = int(threadIdx.x) & 31;
     if (threadIdx.x == 0) {
@@ -218,8 +238,14 @@ k_gemm_bf16(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
         }
     } else {
         // ---------------- epilogue (warps 2..5: lane quarter warp % 4)
+        // Accumulator row `row` of the tile is tensor-memory lane `row`.  With
+        // 256-wide tiles each thread reads 64 columns of its row, rounds them to
+        // bf16 and stages them in shared memory; the warp then stores 4 rows x
+        // 128 contiguous bytes per instruction (whole lines instead of 16-byte
+        // pieces of 32 rows: half the written sectors).
         const int q = warp & 3;
         const int row = 32 * q + lane;
+        uint8_t* sw = epi + (warp - 2) * kEpiWarp;
         int it = 0;
         bool ok = true;
         for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
@@ -232,31 +258,63 @@ k_gemm_bf16(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
             tc::fence_after_sync();
             const int64_t b = tile / (p.tiles_m * p.tiles_n);
             const int64_t rem = tile - b * p.tiles_m * p.tiles_n;
-            const int64_t m = (rem / p.tiles_n) * BM + row;
+            const int64_t m_base = (rem / p.tiles_n) * BM + 32 * q;   // this warp's first row
             const int64_t n0 = (rem % p.tiles_n) * BN;
-            const bool row_ok = m < p.M;
-            bf16* crow = p.c + b * p.c_bstride + (row_ok ? m : 0) * p.ldc;
-            const float rb = (p.bias && p.bias_per_row && row_ok) ? __ldg(p.bias + m) : 0.0f;
+            const int64_t m = m_base + lane;
+            const float rb = (p.bias && p.bias_per_row && m < p.M) ? __ldg(p.bias + m) : 0.0f;
             const uint32_t t_acc = tmem + uint32_t(acc) * kAccCols + (uint32_t(32 * q) << 16);
+            bf16* cb = p.c + b * p.c_bstride;
+            if constexpr (BN == 256) {
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                float v[32];
-                tc::tmem_ld32(t_acc + uint32_t(32 * ch), v);
-                tc::tmem_ld_wait();
-                const int64_t n = n0 + 32 * ch;
-                if (!row_ok || n >= p.N) continue;
+                for (int ch = 0; ch < BN / 64; ++ch) {
+                    float v[64];
+                    tc::tmem_ld32(t_acc + uint32_t(64 * ch), *reinterpret_cast<float(*)[32]>(v));
+                    tc::tmem_ld32(t_acc + uint32_t(64 * ch + 32), *reinterpret_cast<float(*)[32]>(v + 32));
+                    tc::tmem_ld_wait();
+                    const int64_t n = n0 + 64 * ch;
+                    if (p.bias) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    float bi = rb;
-                    if (p.bias && !p.bias_per_row) bi = (n + i < p.N) ? __ldg(p.bias + n + i) : 0.0f;
-                    v[i] += bi;
+                        for (int i = 0; i < 64; ++i)
+                            v[i] += p.bias_per_row ? rb : ((n + i < p.N) ? __ldg(p.bias + n + i) : 0.0f);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(sw + lane * kEpiRow + 16 * c) =
+                            make_uint4(pack2(v[8 * c], v[8 * c + 1]), pack2(v[8 * c + 2], v[8 * c + 3]),
+                                       pack2(v[8 * c + 4], v[8 * c + 5]), pack2(v[8 * c + 6], v[8 * c + 7]));
+                    __syncwarp();
+                    // round k: rows 4 k + lane / 8, 16-byte chunk lane % 8 of the 64 columns
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int r = 4 * k + (lane >> 3), c = lane & 7;
+                        const uint4 w = *reinterpret_cast<const uint4*>(sw + r * kEpiRow + 16 * c);
+                        const int64_t mr = m_base + r, nc = n + 8 * c;
+                        if (mr < p.M && nc + 8 <= p.N) *reinterpret_cast<uint4*>(cb + mr * p.ldc + nc) = w;
+                    }
+                    __syncwarp();
                 }
+            } else {
+                // 128-wide tiles: each thread stores its row directly (measured faster here)
+#pragma unroll 1
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    float v[32];
+                    tc::tmem_ld32(t_acc + uint32_t(32 * ch), v);
+                    tc::tmem_ld_wait();
+                    const int64_t n = n0 + 32 * ch;
+                    if (m >= p.M || n >= p.N) continue;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    if (n + 8 * g + 8 <= p.N) {
-                        const uint4 w = make_uint4(pack2(v[8 * g], v[8 * g + 1]), pack2(v[8 * g + 2], v[8 * g + 3]),
-                                                   pack2(v[8 * g + 4], v[8 * g + 5]), pack2(v[8 * g + 6], v[8 * g + 7]));
-                        *reinterpret_cast<uint4*>(crow + n + 8 * g) = w;
+                    for (int i = 0; i < 32; ++i) {
+                        float bi = rb;
+                        if (p.bias && !p.bias_per_row) bi = (n + i < p.N) ? __ldg(p.bias + n + i) : 0.0f;
+                        v[i] += bi;
+                    }
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        if (n + 8 * g + 8 <= p.N) {
+                            const uint4 w = make_uint4(pack2(v[8 * g], v[8 * g + 1]), pack2(v[8 * g + 2], v[8 * g + 3]),
+                                                       pack2(v[8 * g + 4], v[8 * g + 5]), pack2(v[8 * g + 6], v[8 * g + 7]));
+                            *reinterpret_cast<uint4*>(cb + m * p.ldc + n + 8 * g) = w;
+                        }
                     }
                 }
             }
@@ -313,18 +371,32 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint
     return true;
 }
 
-cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, cudaStream_t s) {
-    auto kern = k_gemm_bf16;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemG));
-    if (e != cudaSuccess) return e;
+int sm_count() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// Tile width for an M x N output per batch: 256 unless that leaves fewer than
+// eight waves of tiles on the SMs (then the last, partly filled wave costs
+// more than the narrower tiles do).
+int pick_bn(int64_t M, int64_t N, int64_t batches) {
+    const int64_t tiles256 = batches * ((M + BM - 1) / BM) * ((N + 255) / 256);
+    return tiles256 >= 8 * int64_t(sm_count()) ? 256 : 128;
+}
+
+template <int BN>
+cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, cudaStream_t s) {
+    auto kern = k_gemm_bf16<BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg<BN>::kSmem));
+    if (e != cudaSuccess) return e;
+    const int sms = sm_count();
     p.tiles_m = (p.M + BM - 1) / BM;
     p.tiles_n = (p.N + BN - 1) / BN;
     const int64_t tiles = p.batches * p.tiles_m * p.tiles_n;
     const int64_t grid = tiles < sms ? tiles : sms;
-    kern<<<unsigned(grid), kThreadsG, kSmemG, s>>>(ma, mb, p);
+    kern<<<unsigned(grid), kThreadsG, Cfg<BN>::kSmem, s>>>(ma, mb, p);
     return cudaGetLastError();
 }
 
@@ -364,9 +436,10 @@ extern "C" hyena_status_t hyena_in_proj(const void* x, const void* W, const floa
         return set_last_error_detail(HYENA_ERR_INVALID_ARG, "u overlaps x or W");
     std::string why;
     CUtensorMap ma, mb;
+    const int bn = pick_bn(J, L, B);
     // A = W_in [J][D] (K-major), B = x [B][L][D] (K-major per position)
     if (!make_map(&ma, W, uint64_t(D), uint64_t(J), 1, uint64_t(D) * 2, uint64_t(J * D) * 2, BK, BM, &why) ||
-        !make_map(&mb, x, uint64_t(D), uint64_t(L), uint64_t(B), uint64_t(D) * 2, uint64_t(L * D) * 2, BK, BN, &why))
+        !make_map(&mb, x, uint64_t(D), uint64_t(L), uint64_t(B), uint64_t(D) * 2, uint64_t(L * D) * 2, BK, bn, &why))
         return set_last_error_detail(HYENA_ERR_CUDA, why);
     GemmParams p{};
     p.M = J; p.N = L; p.K = D; p.batches = B;
@@ -375,7 +448,9 @@ extern "C" hyena_status_t hyena_in_proj(const void* x, const void* W, const floa
     p.bias = bias; p.bias_per_row = 1;
     p.budget_ns = kDefaultWaitBudgetNs;
     cudaError_t e = kernel_status_word(&p.status);
-    if (e == cudaSuccess) e = launch_gemm(ma, mb, p, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)
+        e = bn == 256 ? launch_gemm<256>(ma, mb, p, static_cast<cudaStream_t>(stream))
+                      : launch_gemm<128>(ma, mb, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return set_last_error_detail(HYENA_ERR_CUDA, std::string("in_proj: ") + cudaGetErrorString(e));
     return set_last_error_detail(HYENA_OK, "");
 }
@@ -388,10 +463,11 @@ extern "C" hyena_status_t hyena_out_proj(const void* y, const void* W, const flo
         return set_last_error_detail(HYENA_ERR_INVALID_ARG, "out overlaps y or W");
     std::string why;
     CUtensorMap ma, mb;
+    const int bn = pick_bn(L, D, B);
     // A = y[b]^T: y [B][D][L] read as [64 l][64 k] boxes (positions contiguous);
     // B = W_out [D][D] (K-major)
     if (!make_map(&ma, y, uint64_t(L), uint64_t(D), uint64_t(B), uint64_t(L) * 2, uint64_t(D * L) * 2, 64, BK, &why) ||
-        !make_map(&mb, W, uint64_t(D), uint64_t(D), 1, uint64_t(D) * 2, uint64_t(D * D) * 2, BK, BN, &why))
+        !make_map(&mb, W, uint64_t(D), uint64_t(D), 1, uint64_t(D) * 2, uint64_t(D * D) * 2, BK, bn, &why))
         return set_last_error_detail(HYENA_ERR_CUDA, why);
     GemmParams p{};
     p.M = L; p.N = D; p.K = D; p.batches = B;
@@ -400,7 +476,9 @@ extern "C" hyena_status_t hyena_out_proj(const void* y, const void* W, const flo
     p.bias = bias; p.bias_per_row = 0;
     p.budget_ns = kDefaultWaitBudgetNs;
     cudaError_t e = kernel_status_word(&p.status);
-    if (e == cudaSuccess) e = launch_gemm(ma, mb, p, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)
+        e = bn == 256 ? launch_gemm<256>(ma, mb, p, static_cast<cudaStream_t>(stream))
+                      : launch_gemm<128>(ma, mb, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return set_last_error_detail(HYENA_ERR_CUDA, std::string("out_proj: ") + cudaGetErrorString(e));
     return set_last_error_detail(HYENA_OK, "");
 }
