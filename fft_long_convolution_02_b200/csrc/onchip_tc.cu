@@ -211,11 +211,11 @@ struct PairInput {
 };
 
 struct PairRef {
-    int64_t c, b0;
+    int c, b0;
     bool has1;
 };
-__device__ __forceinline__ PairRef pair_ref(int64_t P, int64_t B) {
-    const int64_t nbp = (B + 1) / 2;
+__device__ __forceinline__ PairRef pair_ref(int P, int B) {
+    const int nbp = (B + 1) / 2;
     PairRef r;
     r.c = P / nbp;
     r.b0 = 2 * (P - r.c * nbp);
@@ -224,13 +224,13 @@ __device__ __forceinline__ PairRef pair_ref(int64_t P, int64_t B) {
 }
 
 __device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __restrict__ u, const PairRef& pr,
-                                                int64_t C, int order, int j0) {
+                                                int C, int order, int j0) {
     const int64_t Ctot = int64_t(order + 1) * C;
     const int t = threadIdx.x;
     const int chalf = t >> 7, a0 = 8 * (t & 127);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-        const bf16* ub = u + (pr.b0 + (r && pr.has1 ? 1 : 0)) * Ctot * L;
+        const bf16* ub = u + int64_t(pr.b0 + (r && pr.has1 ? 1 : 0)) * Ctot * L;
         const bf16* xg = ub + (int64_t(order - 1) * C + pr.c) * L;
         const bf16* vv = ub + (int64_t(order) * C + pr.c) * L;
 #pragma unroll
@@ -244,8 +244,8 @@ __device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __res
 
 __global__ void __launch_bounds__(NT, 2)
 k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
-               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
-               int64_t npairs, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+               const float* __restrict__ sc_w, const float* __restrict__ sc_b, int B, int C, int order,
+               int npairs, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
@@ -303,10 +303,10 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     // Thread t covers samples n0 = 8 (t + 256 jj) of both rows.
     auto output_gate = [&](const PairRef& pr) {
         const Taps2 t0 = taps2(load_taps(sc_w, sc_b, pr.c), 1.0f);
-        const bf16* x00 = u + (pr.b0 * Ctot + pr.c) * L;
+        const bf16* x00 = u + (int64_t(pr.b0) * Ctot + pr.c) * L;
         const bf16* x01 = pr.has1 ? x00 + Ctot * L : x00;
-        bf16* y0 = y + (pr.b0 * C + pr.c) * L;
-        bf16* y1 = y0 + C * L;
+        bf16* y0 = y + (int64_t(pr.b0) * C + pr.c) * L;
+        bf16* y1 = y0 + int64_t(C) * L;
 #pragma unroll
         for (int jh = 0; jh < 4; jh += 2) {
             Raw8 xr[2][2];
@@ -341,19 +341,19 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     };
 
     PairInput in;
-    if (int64_t(blockIdx.x) < npairs) {
-        load_pair_input(in, u, pair_ref(blockIdx.x, B), C, order, 0);
-        load_pair_input(in, u, pair_ref(blockIdx.x, B), C, order, 2);
-    }
     PairRef prev{0, 0, false};
     bool have_prev = false;
 
-    for (int64_t P = blockIdx.x; P < npairs; P += gridDim.x) {
+    for (int P = blockIdx.x; P < npairs; P += gridDim.x) {
         const PairRef pr = pair_ref(P, B);
-        const int64_t c = pr.c;
-        const bf16* u0 = u + pr.b0 * Ctot * L;
+        const int c = pr.c;
+        const bf16* u0 = u + int64_t(pr.b0) * Ctot * L;
         const bf16* u1 = pr.has1 ? u0 + Ctot * L : u0;
-        const int64_t Pn = P + gridDim.x;
+        // this pair's step-1 input (the other CTA of the SM covers the load
+        // latency; holding the next pair's samples in registers instead costs
+        // spills that are slower than the wait)
+        load_pair_input(in, u, pr, C, order, 0);
+        load_pair_input(in, u, pr, C, order, 2);
         // ---------------- step-1 operand: z = sc(x_{order-1}) sc(v), g[b0] + i g[b1]
         {
             // an odd batch's last pair has no row b1: its v taps are zero, so z = g[b0]
@@ -605,12 +605,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
             stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
             if (st < order - 1) ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         }
-        // the next pair's step-1 input, loaded while stage 1' runs (unconditional, so
-        // that the registers' live range ends here; past the last pair this pair's
-        // rows are reloaded and not used)
-        const PairRef pnext = pair_ref(Pn < npairs ? Pn : P, B);
-        load_pair_input(in, u, pnext, C, order, 0);
-        load_pair_input(in, u, pnext, C, order, 2);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         // output staging v = conj(D1') as (re, -im) bf16 pairs in natural order;
         // the output gate runs during the next pair's stage 1
@@ -652,10 +646,11 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t npairs = p.C * ((a.B + 1) / 2);
+    if (npairs > INT32_MAX || a.B > INT32_MAX) return cudaErrorInvalidValue;   // 32-bit pair indices
     int64_t grid = int64_t(2) * sms;
     if (grid > npairs) grid = npairs;
     kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
-                                           a.sc_b, a.B, p.C, p.order, npairs, a.wait_budget_ns, a.issue_mma,
+                                           a.sc_b, int(a.B), int(p.C), p.order, int(npairs), a.wait_budget_ns, a.issue_mma,
                                            a.status);
     return cudaGetLastError();
 }
