@@ -245,20 +245,23 @@ __device__ __forceinline__ void load_pair_input(PairInput& in, const bf16* __res
 __global__ void __launch_bounds__(NT, 2)
 k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* __restrict__ spectrum,
                const float* __restrict__ sc_w, const float* __restrict__ sc_b, int B, int C, int order,
-               int npairs, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+               int npairs, int64_t tables_off, int64_t spec_off, int64_t Ctot, uint64_t wait_budget_ns,
+               int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     if (!(h->magic == kSpecMagic && h->path == PATH_ONCHIP_1D && h->C == C && h->L == L && h->order == order &&
-          h->spec_row_bytes == int64_t(N) * 8)) {
+          h->spec_row_bytes == int64_t(N) * 8 && h->tables_off == tables_off && h->spec_off == spec_off)) {
         if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return;
     }
-    const float2* tables = reinterpret_cast<const float2*>(spectrum + h->tables_off);
+    // the layout offsets are kernel parameters (checked against the header above),
+    // so that the table pointers need no registers of their own
+    const float2* tables = reinterpret_cast<const float2*>(spectrum + tables_off);
     const float2* twist = tables + fft_tw_size(L / 2);        // w_L^j = w_N^(2j)
     const float2* odd = twist + L / 2 + (L / 4 + 1);          // w_N^(2j+1)
-    const uint32_t* spec = reinterpret_cast<const uint32_t*>(spectrum + h->spec_off);   // plane 0 of each row
+    const uint32_t* spec = reinterpret_cast<const uint32_t*>(spectrum + spec_off);   // plane 0 of each row
 
     // A: stage operands.  The stage-1 operand sits in the upper part so that
     // the previous pair's output staging (bf16 pairs, lower 32 KB) survives
@@ -270,7 +273,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    const int64_t Ctot = int64_t(order + 1) * C;
 
     fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16);
     fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64);
@@ -506,20 +508,22 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                 for (int i = 0; i < 16; ++i) kv[i] = __ldg(kq + 32 * i);
                 ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
 #pragma unroll
-                for (int T = 0; T < 4; ++T) {
-                    float d[32];
-                    tc::tmem_ld32(tl + uint32_t(64 * T + 32 * hh), d);
+                for (int TH = 0; TH < 8; ++TH) {
+                    // half TH & 1 of tile T's 32 accumulator columns
+                    const int T = TH >> 1;
+                    float d[16];
+                    tc::tmem_ld16(tl + uint32_t(64 * T + 32 * hh + 16 * (TH & 1)), d);
                     tc::tmem_ld_wait();
                     const uint32_t rowoff = uint32_t(16 * T + 4 * Q + (lane >> 3)) * kSBO64 + uint32_t(4 * hh) * tc::kLBO +
                                             uint32_t(lane & 7) * 16u;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
+                    for (int q4 = 2 * (TH & 1); q4 < 2 * (TH & 1) + 2; ++q4) {
                         const uint4 kk = kv[4 * T + q4];
                         // bins i = 4 q4 .. 4 q4 + 3 as two split pairs
                         const C2 K0{make_float2(bf_lo(kk.x), bf_lo(kk.y)), make_float2(bf_hi(kk.x), bf_hi(kk.y))};
                         const C2 K1{make_float2(bf_lo(kk.z), bf_lo(kk.w)), make_float2(bf_hi(kk.z), bf_hi(kk.w))};
-                        const C2 v0 = cmul2(c2_at(d, 2 * q4), K0);
-                        const C2 v1 = cmul2(c2_at(d, 2 * q4 + 1), K1);
+                        const C2 v0 = cmul2(c2_at(d, 2 * (q4 & 1)), K0);
+                        const C2 v1 = cmul2(c2_at(d, 2 * (q4 & 1) + 1), K1);
                         sts128(A, rowoff + q4 * tc::kLBO, pack_bf16(v0.re.x, -v0.im.x), pack_bf16(v0.re.y, -v0.im.y),
                                pack_bf16(v1.re.x, -v1.im.x), pack_bf16(v1.re.y, -v1.im.y));
                     }
@@ -650,7 +654,8 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
     int64_t grid = int64_t(2) * sms;
     if (grid > npairs) grid = npairs;
     kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
-                                           a.sc_b, int(a.B), int(p.C), p.order, int(npairs), a.wait_budget_ns, a.issue_mma,
+                                           a.sc_b, int(a.B), int(p.C), p.order, int(npairs), int64_t(p.tables_off),
+                                           int64_t(p.spec_off), int64_t(p.order + 1) * p.C, a.wait_budget_ns, a.issue_mma,
                                            a.status);
     return cudaGetLastError();
 }
