@@ -126,15 +126,16 @@ __device__ __forceinline__ C2 c2_at(const float (&d)[NCOL], int p) {
 // Real form of a DFT matrix as a K-major B operand, entry of w_R^(s k): column
 // j = 2 s + (0: re, 1: im) of input s; row n holds output k = 2 (n >> 2) + (n & 1),
 // real part for (n >> 1) & 1 == 0, else imaginary part, so that the accumulator
-// columns of outputs 2p, 2p+1 read (re, re, im, im).
-__device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo) {
+// columns of outputs 2p, 2p+1 read (re, re, im, im).  w32 holds (cos, sin) of
+// 2 pi i / 32, i < 32 (R divides 32).
+__device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo, const float2* w32) {
     for (int idx = threadIdx.x; idx < 4 * nout * nin; idx += NT) {
         const int n = idx / (2 * nin), j = idx % (2 * nin);
         const int k = 2 * (n >> 2) + (n & 1);
         const bool im_row = (n >> 1) & 1;
         const int e = (k * (j >> 1)) % R;
-        float sv, cv;
-        sincospif(2.0f * float(e) / float(R), &sv, &cv);   // w = cv - i sv
+        const float2 cs = w32[e * (32 / R)];                // w = cv - i sv
+        const float cv = cs.x, sv = cs.y;
         float v;
         if (!im_row) v = (j & 1) == 0 ? cv : sv;            // re: Re w xr - Im w xi
         else v = (j & 1) == 0 ? -sv : cv;                   // im: Im w xr + Re w xi
@@ -274,9 +275,18 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
 
-    fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16);
-    fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64);
-    fill_dft(smem_tc + kOffB1i, 16, 8, 16, kSBO32);
+    // the 32 distinct entries of the DFT matrices once (in the operand area, free
+    // until the first pair), then the matrices by lookup
+    float2* w32 = reinterpret_cast<float2*>(smem_tc);
+    if (t < 32) {
+        float sv, cv;
+        sincospif(2.0f * float(t) / 32.0f, &sv, &cv);
+        w32[t] = make_float2(cv, sv);
+    }
+    __syncthreads();
+    fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16, w32);
+    fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64, w32);
+    fill_dft(smem_tc + kOffB1i, 16, 8, 16, kSBO32, w32);
     // TW2[(T * 16 + kp) * 8 + l] = (Re w0, Re w1, Im w0, Im w1), w0 = w1024^(b k),
     // w1 = w1024^(b (k+1)), b = 4 l + T, k = 2 kp
     for (int idx = t; idx < 4 * 16 * 8; idx += NT) {
