@@ -286,6 +286,8 @@ def kernel_of(p) -> str:
         return "k_conv_8192_tc" if (p.dtype == "bf16" and not p.per_sample and p.order <= 3) else "k_conv_4096"
     if p.ndim == 1 and p.L <= 16384:
         return "k_conv_onchip"
+    if p.ndim == 1 and p.L == 65536 and p.dtype == "bf16" and not p.per_sample and p.order <= 3:
+        return "k_conv_cluster"
     return "multipass" if p.ndim == 1 else ("grid2d" if p.ndim == 2 else "grid3d")
 
 
@@ -294,6 +296,10 @@ def math_of(p, kernel: str) -> str:
     if kernel == "k_conv_8192_tc":
         return ("DFT stages on tcgen05 tensor cores: bf16 operands and DFT matrices, fp32 accumulation; "
                 "short conv, gates, twiddles and spectrum products fp32; spectrum read as bf16 (re, im)")
+    if kernel == "k_conv_cluster":
+        return ("2L-point transform split over 8-CTA clusters: 8-point DFTs, short conv, gates and twiddles fp32 "
+                "on the CUDA cores; 16384-point DFT stages per CTA on tcgen05 tensor cores with bf16 operands and "
+                "fp32 accumulation; exchanges as bf16 pairs; spectrum read as bf16 (re, im)")
     if p.dtype == "bf16" and (p.ndim > 1 or p.L > 16384):
         return "fp32 (intermediate kept as bf16 pairs in the workspace between passes)"
     return "fp32"

@@ -79,6 +79,12 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
 constexpr int kMaxOrderTc = 3;   // highest order the L = 8192 tensor-core kernel serves
 cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s);
+// L = 65536, bf16 storage (cluster.cu): the cluster plane of the spectrum, and
+// the convolution on 8-CTA clusters with workspace_bytes of scratch (512 KB
+// per cluster in flight).
+cudaError_t launch_spectrum_cluster(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+bool cluster_path(const Plan& p, const ConvArgs& a);
+cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspace_bytes, cudaStream_t s);
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_3d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);

@@ -609,12 +609,26 @@ cudaError_t conv_mp(const Plan& p, const ConvArgs& a, cudaStream_t s) {
         default: return cudaErrorInvalidValue;                \
     }
 
-cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+cudaError_t spectrum_mp_any(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     HYENA_MP_SWITCH(spectrum_mp)
 }
 
-cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+cudaError_t conv_mp_any(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     HYENA_MP_SWITCH(conv_mp)
+}
+
+// The multi-pass rows, and at L = 65536 the cluster plane (cluster.cu) too.
+cudaError_t launch_spectrum_multipass(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
+    const cudaError_t e = spectrum_mp_any(p, a, s);
+    if (e != cudaSuccess) return e;
+    return launch_spectrum_cluster(p, a, s);
+}
+
+// bf16 storage at L = 65536 with shared filters runs on the cluster kernel,
+// its scratch taken from the workspace; the rest on the multi-pass kernels.
+cudaError_t launch_conv_multipass(const Plan& p, const ConvArgs& a, cudaStream_t s) {
+    if (cluster_path(p, a)) return launch_conv_cluster(p, a, size_t(a.group_rows) * p.ws_row_bytes, s);
+    return conv_mp_any(p, a, s);
 }
 
 }  // namespace hyena

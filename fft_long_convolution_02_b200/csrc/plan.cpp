@@ -96,6 +96,12 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
             p->t_unt_c = tb.add(2 * L, 1, 1, 1, 1);                   // w_2L^1
             p->spec_row_bytes = size_t(p->M) * 16;                   // M1 units x M2 float4
             p->ws_row_bytes = size_t(2 * p->M) * 8;                  // two chains of M complex
+            if (L == kClusterL) {
+                p->t_cl_fft = tb.add_fft(16384);
+                p->t_cl_wa = tb.add(2 * L, 0, 16384, 1, 1);              // w_2L^a
+                p->t_cl_even = tb.add(16384, 0, 2048, 1, 1, 2, 0);       // w_16384^(2j)
+                p->t_cl_odd = tb.add(16384, 0, 2048, 1, 1, 2, 1);        // w_16384^(2j+1)
+            }
         }
     } else if (ndim == 2) {
         const int64_t H = sizes[0], W = sizes[1];
@@ -154,6 +160,10 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
     p->tables_off = kHeaderBytes;
     p->spec_off = align_up(p->tables_off + size_t(tb.cursor) * 8, 256);
     p->total_bytes = p->spec_off + size_t(S) * size_t(C) * p->spec_row_bytes;
+    if (p->path == PATH_MULTIPASS_1D && p->L == kClusterL) {
+        p->cl_plane_off = align_up(p->total_bytes, 256);
+        p->total_bytes = p->cl_plane_off + size_t(S) * size_t(C) * size_t(2 * p->L) * 4;
+    }
     return true;
 }
 

@@ -18,7 +18,11 @@
 //                     passes through a caller workspace (rows processed in
 //                     groups that fit it; by default the whole batch up to
 //                     4 GiB).  Spectrum row = M1 units of M2 float4 pair
-//                     entries.
+//                     entries.  L = 65536 adds, after the rows, the cluster
+//                     plane (cluster.cu): per (step, c) all 2L bins of K~ as
+//                     bf16 (re, im), eight sub-planes of 16384 in the
+//                     tensor-core kernel's position order (header
+//                     reserved[0] holds its offset).
 //   PATH_GRID_2D      2-D H x W (16..512 each), zero-padded to 2H x 2W: a row
 //                     pass (packed real FFT of each image row), a column pass
 //                     (2H-point FFT, spectrum multiply, inverse) and an
@@ -55,6 +59,9 @@ constexpr size_t kHeaderBytes = 256;
 constexpr int kMaxTableSpecs = 24;
 
 constexpr int64_t kOnchipMaxL = 16384;
+// L served by the cluster kernel (bf16 storage): 2L = kClusterR x 16384
+constexpr int64_t kClusterL = 65536;
+constexpr int kClusterR = 8;
 constexpr int64_t kMaxL = int64_t(1) << 20;
 constexpr int64_t kMin1D = 16;
 constexpr int64_t kMin2D = 16;
@@ -93,6 +100,10 @@ struct Plan {
     int64_t t_fft_a = 0, t_fft_b = 0, t_twist = 0, t_untangle = 0, t_four = 0;
     int64_t t_twist_hi = 0, t_twist_lo = 0, t_unt1 = 0, t_unt2 = 0, t_unt_c = 0, t_twist_h = 0;
     int64_t t_fft_d = 0, t_twist_d = 0;   // 3-D depth axis
+    // L = kClusterL: CTA FFT of 16384 points, w_2L^a (a < 16384), and the
+    // even / odd powers w_16384^(2j), w_16384^(2j+1) (j < 2048)
+    int64_t t_cl_fft = 0, t_cl_wa = 0, t_cl_even = 0, t_cl_odd = 0;
+    size_t cl_plane_off = 0;               // 0: no cluster plane
     TableSpecs specs{};
     size_t tables_off = kHeaderBytes;
     size_t spec_off = 0;

@@ -112,7 +112,7 @@ __device__ __forceinline__ C2 c2_at(const float (&d)[NCOL], int p) {
 // real part for (n >> 1) & 1 == 0, else imaginary part, so that the accumulator
 // columns of outputs 2p, 2p+1 read (re, re, im, im).  w32 holds (cos, sin) of
 // 2 pi i / 32, i < 32 (R divides 32).
-__device__ void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo, const float2* w32) {
+__device__ inline void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo, const float2* w32) {
     for (int idx = threadIdx.x; idx < 4 * nout * nin; idx += blockDim.x) {
         const int n = idx / (2 * nin), j = idx % (2 * nin);
         const int k = 2 * (n >> 2) + (n & 1);
