@@ -167,8 +167,14 @@ constexpr uint32_t kB1fBytes = 4 * kSBO32;      // 16-point DFT, N 32 x K 32
 constexpr uint32_t kOffB1f = kAbytes;
 constexpr uint32_t kOffB32c = kOffB1f + kB1fBytes;
 constexpr uint32_t kOffTW2c = kOffB32c + kB32bytes;
-constexpr size_t kSmemC = size_t(kOffTW2c) + kTW2bytes;
-static_assert(kOffTW2c % 16 == 0, "twiddle table alignment");
+// F1 staging: per warp two buffers of up to 16 runs of 40 samples (bf16)
+constexpr uint32_t kStageRun = 80;
+constexpr uint32_t kStageBuf = 16 * kStageRun;
+constexpr uint32_t kOffStage = kOffTW2c + kTW2bytes;
+constexpr size_t kSmemC = size_t(kOffStage) + (NT / 32) * 2 * kStageBuf;
+static_assert(kOffTW2c % 16 == 0 && kOffStage % 16 == 0, "table / staging alignment");
+// two CTAs per SM: 2 x (dynamic + 1 KB static + 1 KB reserved) <= 228 KB
+static_assert(2 * (kSmemC + 2048) <= 233472, "two CTAs per SM");
 
 struct ClArgs {
     const bf16* u;            // [B, (order+1) C, L]
@@ -308,52 +314,130 @@ struct PairRows {
     float m1;         // 1, or 0 for a pair with one row
 };
 
-// F1 of one round: for each of the four s' (m < 4) of a' = sh.ap, the gated
-// samples z[s] = sc(x_g)[n] v[n] (n = a + NI s, a = a' + 1024 s'; STEP1: v =
-// sc(v) read from u, else v = I1 of the previous step at the same a), then
-// Y1[k1][a] = w_NO^(a k1) DFT_8(z)[k1].  The four s' of the row are one
-// 16-byte chunk (chunk `quad` of row rho1(a')) of CTA k1's stage-1 operand.
-template <bool STEP1>
-__device__ __forceinline__ void f1_round(const ClArgs& p, const PairRows& rw, int64_t cg, int64_t cv,
-                                         const Taps2& tg, const Taps2& tv, const Share& sh,
-                                         const uint32_t* __restrict__ scr, uint32_t a_addr) {
-    uint32_t v[RC][4];                          // [k1][m]: bf16 pairs
+// F1 of one order step.  Thread (warp w, lane l) takes, in round r < 2, the
+// row a' = 32 q + l, q = 16 half + 2 w + r, and its four s' = 4 quad + m
+// (m < 4): a = a' + 1024 s'.  For each (r, m) the warp stages the 34 samples
+// n - 2 .. n (n = a + NI s) of every input row it needs (the gate rows, and
+// at the first step the value rows, at s < 4) in shared memory with cp.async,
+// one item ahead of the arithmetic: z[s] = sc(x_g)[n] v[n] (STEP1: v = sc(v),
+// else v = the previous step's I1 at a), Y1[k1][a] = w_NO^(a k1) DFT_8(z)[k1].
+// The four s' of a row are one 16-byte chunk (chunk `quad` of row rho1(a'))
+// of CTA k1's stage-1 operand, written after each round.
+// MODE 2 runs the same loop for the output gate: I1 of the last step, times
+// sc(x0) (cg = x0's rows), stored to y (y0, y1: rows b0, b1 of y; ok = false
+// writes NaN).
+template <int MODE>
+__device__ __forceinline__ void f1_step(const ClArgs& p, const PairRows& rw, int64_t cg, int64_t cv,
+                                        const Taps2& tg, const Taps2& tv, int half, int quad, int warp, int lane,
+                                        const uint32_t* __restrict__ scr, uint32_t a_addr, uint8_t* stage,
+                                        bf16* y0 = nullptr, bf16* y1 = nullptr, bool ok = true) {
+    constexpr bool STEP1 = MODE == 0;
+    constexpr int NR = STEP1 ? 4 : 2;           // input rows per s
+    constexpr int NC = 4 * NR;                  // staged runs per item
+    auto issue = [&](int it) {
+        const int base = 32 * (16 * half + 2 * warp + (it >> 2)) + 1024 * (4 * quad + (it & 3));
+        uint8_t* dst = stage + (it & 1) * kStageBuf;
+        for (int k = lane; k < NC * 5; k += 32) {
+            const int c = k / 5, ch = k - 5 * (k / 5);
+            const int s = c / NR, rr = c - NR * (c / NR);
+            const bf16* row = (rr & 1 ? rw.u1 : rw.u0) + (rr < 2 ? cg : cv);
+            const int e = base + NI * s - 8 + 8 * ch;          // first sample of this 16-byte piece
+            const bool in = e >= 0;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tc::smem_u32(dst + c * kStageRun + 16 * ch)),
+                         "l"(row + (in ? e : 0)), "r"(in ? 16 : 0)
+                         : "memory");
+        }
+        cp_async_commit();
+    };
+    auto s3_at = [&](const uint8_t* buf, int c) {
+        const bf16* r = reinterpret_cast<const bf16*>(buf + c * kStageRun) + 6 + lane;
+        S3 o;
+        o.m2 = __bfloat162float(r[0]);
+        o.m1 = __bfloat162float(r[1]);
+        o.c = __bfloat162float(r[2]);
+        return o;
+    };
+    issue(0);
+#pragma unroll 1
+    for (int r = 0; r < 2; ++r) {
+        const int ap = 32 * (16 * half + 2 * warp + r) + lane;
+        uint32_t v[RC][4];                      // [k1][m]: bf16 pairs
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int a = sh.ap + 1024 * (4 * sh.quad + m);
-        float2 ys[4];
-        if constexpr (!STEP1) i1_one(ys, scr, a, p.wa);
-        float2 z[4];
+        for (int m = 0; m < 4; ++m) {
+            const int it = 4 * r + m;
+            if (it < 7) issue(it + 1);
+            else cp_async_commit();
+            const int a = ap + 1024 * (4 * quad + m);
+            const float2 w1 = __ldg(p.wa + a);
+            uint32_t sv[STEP1 ? 1 : RC];
+            if constexpr (!STEP1) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int n = a + NI * s;
-            const float2 xs = sc_pair(load3(rw.u0 + cg, n), load3(rw.u1 + cg, n), tg);
+                for (int k1 = 0; k1 < RC; ++k1) sv[k1] = __ldcg(scr + int64_t(k1) * NI + a);
+            }
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+            __syncwarp();
+            const uint8_t* buf = stage + (it & 1) * kStageBuf;
+            float2 z[4];
             if constexpr (STEP1) {
-                z[s] = __fmul2_rn(xs, sc_pair(load3(rw.u0 + cv, n), load3(rw.u1 + cv, n), tv));
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    z[s] = __fmul2_rn(sc_pair(s3_at(buf, 4 * s), s3_at(buf, 4 * s + 1), tg),
+                                      sc_pair(s3_at(buf, 4 * s + 2), s3_at(buf, 4 * s + 3), tv));
             } else {
-                z[s] = __fmul2_rn(xs, make_float2(ys[s].x, rw.m1 * ys[s].y));
+                // I1 of the previous step at a: conj U[k1] = w_NO^(a k1) conj V[k1][a]
+                float2 x[8];
+                float2 w = w1;
+#pragma unroll
+                for (int k1 = 0; k1 < RC; ++k1) {
+                    const float2 vc = make_float2(bf_lo(sv[k1]), bf_hi(sv[k1]));
+                    if (k1 == 0) {
+                        x[0] = vc;
+                    } else {
+                        x[k1] = cmul(vc, w);
+                        if (k1 + 1 < RC) w = cmul(w, w1);
+                    }
+                }
+                float2 o[4];
+                dft8_first4(x, o);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const float2 ys = make_float2(o[s].x, -rw.m1 * o[s].y);   // y = conj (row b1 masked)
+                    z[s] = __fmul2_rn(sc_pair(s3_at(buf, 2 * s), s3_at(buf, 2 * s + 1), tg), ys);
+                }
+            }
+            __syncwarp();                       // buffer read before the next issue refills it
+            if constexpr (MODE == 2) {
+                const bf16 nanv = __float2bfloat16_rn(__int_as_float(0x7fc00000));
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    // a timed-out wait poisons the output
+                    y0[a + NI * s] = ok ? __float2bfloat16_rn(z[s].x) : nanv;
+                    if (rw.m1 != 0.0f) y1[a + NI * s] = ok ? __float2bfloat16_rn(z[s].y) : nanv;
+                }
+                continue;
+            }
+            float2 o[8];
+            dft8_of4(z, o);
+            float2 w = w1;
+            v[0][m] = pack_bf16(o[0].x, o[0].y);
+#pragma unroll
+            for (int k1 = 1; k1 < RC; ++k1) {
+                const float2 tw = cmul(o[k1], w);
+                v[k1][m] = pack_bf16(tw.x, tw.y);
+                if (k1 + 1 < RC) w = cmul(w, w1);
             }
         }
-        float2 o[8];
-        dft8_of4(z, o);
-        const float2 w1 = __ldg(p.wa + a);
-        float2 w = w1;
-        v[0][m] = pack_bf16(o[0].x, o[0].y);
+        if constexpr (MODE == 2) continue;
+        const uint32_t off = a_addr + tc::chunk_off(rho1(ap), quad, kSBO32);
 #pragma unroll
-        for (int k1 = 1; k1 < RC; ++k1) {
-            const float2 tw = cmul(o[k1], w);
-            v[k1][m] = pack_bf16(tw.x, tw.y);
-            if (k1 + 1 < RC) w = cmul(w, w1);
+        for (int k1 = 0; k1 < RC; ++k1) {
+            const uint32_t dst = map_rank(off, uint32_t(k1));
+            asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k1][0]),
+                         "r"(v[k1][1]), "r"(v[k1][2]), "r"(v[k1][3])
+                         : "memory");
         }
     }
-    const uint32_t off = a_addr + tc::chunk_off(rho1(sh.ap), sh.quad, kSBO32);
-#pragma unroll
-    for (int k1 = 0; k1 < RC; ++k1) {
-        const uint32_t dst = map_rank(off, uint32_t(k1));
-        asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[k1][0]), "r"(v[k1][1]),
-                     "r"(v[k1][2]), "r"(v[k1][3])
-                     : "memory");
-    }
+    cp_async_wait_all();
 }
 
 __global__ void __launch_bounds__(NT, 2)
@@ -414,12 +498,9 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
                 const int64_t cg = (int64_t(g) * p.C + pr.c) * LC, cv = (int64_t(p.order) * p.C + pr.c) * LC;
                 const Taps2 tg = taps2(load_taps(p.sc_w, p.sc_b, int64_t(g) * p.C + pr.c), 1.0f);
                 const Taps2 tv = taps2(load_taps(p.sc_w, p.sc_b, int64_t(p.order) * p.C + pr.c), rw.m1);
-#pragma unroll 1
-                for (int r = 0; r < 2; ++r) {
-                    const Share sh{32 * (16 * half + 2 * warp + r) + lane, quad};
-                    if (st == 1) f1_round<true>(p, rw, cg, cv, tg, tv, sh, scr, a_addr);
-                    else f1_round<false>(p, rw, cg, cv, tg, tv, sh, scr, a_addr);
-                }
+                uint8_t* stage = smem_cl + kOffStage + warp * 2 * kStageBuf;
+                if (st == 1) f1_step<0>(p, rw, cg, cv, tg, tv, half, quad, warp, lane, scr, a_addr, stage);
+                else f1_step<1>(p, rw, cg, cv, tg, tv, half, quad, warp, lane, scr, a_addr, stage);
             }
             fence_proxy_async_cluster();
             cluster_sync();
@@ -470,30 +551,17 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
             tc::fence_after_sync();
         }
         // ---- I1 of the last step and the output gate y = sc(x0) v
-        const int64_t Ctot = int64_t(p.order + 1) * p.C;
-        const bf16* x00 = p.u + (int64_t(pr.b0) * Ctot + pr.c) * LC;
-        const bf16* x01 = pr.has1 ? x00 + Ctot * LC : x00;
-        bf16* y0 = p.y + (int64_t(pr.b0) * p.C + pr.c) * LC;
-        bf16* y1 = y0 + int64_t(p.C) * LC;
-        const Taps2 t0 = taps2(load_taps(p.sc_w, p.sc_b, pr.c), 1.0f);
-        const bf16 nanv = __float2bfloat16_rn(__int_as_float(0x7fc00000));
-#pragma unroll 1
-        for (int r = 0; r < 2; ++r) {
-            const int ap = 32 * (16 * half + 2 * warp + r) + lane;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int a = ap + 1024 * (4 * quad + m);
-                float2 ys[4];
-                i1_one(ys, scr, a, p.wa);
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int n = a + NI * s;
-                    const float2 yv = __fmul2_rn(sc_pair(load3(x00, n), load3(x01, n), t0), ys[s]);
-                    // a timed-out wait poisons the output
-                    y0[n] = ok ? __float2bfloat16_rn(yv.x) : nanv;
-                    if (pr.has1) y1[n] = ok ? __float2bfloat16_rn(yv.y) : nanv;
-                }
-            }
+        {
+            const int64_t Ctot = int64_t(p.order + 1) * p.C;
+            PairRows rw;
+            rw.u0 = p.u + int64_t(pr.b0) * Ctot * LC;
+            rw.u1 = pr.has1 ? rw.u0 + Ctot * LC : rw.u0;
+            rw.m1 = pr.has1 ? 1.0f : 0.0f;
+            const Taps2 t0 = taps2(load_taps(p.sc_w, p.sc_b, pr.c), 1.0f);
+            bf16* y0 = p.y + (int64_t(pr.b0) * p.C + pr.c) * LC;
+            uint8_t* stage = smem_cl + kOffStage + warp * 2 * kStageBuf;
+            f1_step<2>(p, rw, int64_t(pr.c) * LC, 0, t0, t0, half, quad, warp, lane, scr, a_addr, stage, y0,
+                       y0 + int64_t(p.C) * LC, ok);
         }
     }
     tc::fence_before_sync();
