@@ -51,8 +51,10 @@ CASES = [
     I.WORKLOADS["grid2d"].with_(B=2, C=5, H=64, W=128, dtype="f32", sigma=(4.0, 32.0), seed=1204),
     # on-chip path (no scratch needed), bf16
     I.WORKLOADS["d768_l8k"].with_(C=16, seed=1205),
+    # cluster path, bf16, order 3, L = 2^16: the scratch holds one 512 KB slice per cluster
+    I.WORKLOADS["order3"].with_(B=3, C=7, L=1 << 16, seed=1206),
 ]
-EXPECTED_GROUPS = [3, 2, 8, 1, None]
+EXPECTED_GROUPS = [3, 2, 8, 1, None, None]
 
 
 def test_cases_span_several_groups():
