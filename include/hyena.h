@@ -31,7 +31,13 @@
  *    operands and the DFT matrices are rounded to bf16 and accumulated in
  *    fp32, and the spectrum is read as bf16 (re, im) pairs (row error a few
  *    1e-3); HYENA_FLAG_FP32_TRANSFORM (hyena_gated_fftconv_ex) selects the
- *    fp32 transform there instead.  With bf16 storage the intermediate of the
+ *    fp32 transform there instead.  At L = 65536 with bf16 storage (order
+ *    <= 3, shared filters) the 2L-point transform of a row pair is split over
+ *    a cluster of 8 CTAs: the 8-point DFTs, gates and twiddles in fp32, the
+ *    16384-point part on the tensor cores as at L = 8192, the exchanges
+ *    between the CTAs and the spectrum as bf16 pairs (row error ~1e-2 at
+ *    order 3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 multi-pass
+ *    transform there.  With bf16 storage the intermediate of the other
  *    multi-pass (L >= 32768) and N-D paths is kept as bf16 pairs in the
  *    workspace.
  *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
@@ -115,7 +121,9 @@ size_t hyena_spectrum_bytes(int64_t C, int ndim, const int64_t* sizes, int order
  *            header, the twiddle tables of this shape (double-precision values
  *            rounded to fp32) and, for every (step, channel), the zero-padded
  *            spectrum of k with D folded in (D * v = (D delta) conv v) and the
- *            inverse-FFT normalisation folded in.
+ *            inverse-FFT normalisation folded in.  At L = 65536 it holds that
+ *            spectrum twice: in the multi-pass layout (complex64) and as the
+ *            bf16 plane the cluster path reads.
  *
  * The buffer is the cache: keep it while k and D are unchanged and pass it to
  * every hyena_gated_fftconv call with the same (C, sizes, order).
@@ -216,7 +224,9 @@ size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_
  *   sc_bias  [(order+1)*C] fp32 or NULL (= 0); ignored when sc_w is NULL
  *   workspace, workspace_bytes  device scratch for the multi-pass (L >= 32768)
  *            and 2-D paths; may be NULL/0 for the on-chip path.  Its contents
- *            are undefined after the call.
+ *            are undefined after the call.  The cluster path (L = 65536, bf16)
+ *            takes 512 KB per cluster in flight from it (up to 30 clusters
+ *            on a B200); the minimum workspace runs one cluster.
  *
  * The spectrum is only read.  Conditions the kernels detect on the device (a
  * spectrum whose header does not match the shape: that kernel writes no
@@ -230,7 +240,7 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
 
 /* Flags of hyena_gated_fftconv_ex. */
 #define HYENA_FLAG_FP32_TRANSFORM 0x1u  /* every transform multiply in fp32 on the CUDA cores (no bf16 tensor-core
-                                           operands); changes only 1-D L = 8192 with bf16 storage */
+                                           operands); changes only 1-D L = 8192 and 65536 with bf16 storage */
 
 /*
  * hyena_gated_fftconv_ex -- hyena_gated_fftconv with flags (shared filters).
