@@ -279,6 +279,27 @@ hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum,
     return cuda_status(launch_conv_8192_tc(p, a, static_cast<cudaStream_t>(stream)), "tensor-core kernel");
 }
 
+hyena_status_t hyena_debug_conv_cluster(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                        const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int order,
+                                        void* workspace, size_t workspace_bytes, uint64_t wait_budget_ns,
+                                        int issue_mma, void* stream) {
+    Plan p;
+    ConvArgs a;
+    const int64_t L = kClusterL;
+    hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, sc_w, sc_bias, B, C, 1, &L, order, HYENA_BF16,
+                                     workspace, workspace_bytes, &p, &a);
+    if (st != HYENA_OK) return st;
+    if (!cluster_path(p, a))
+        return fail(HYENA_ERR_UNSUPPORTED_SHAPE, "the cluster kernel serves order <= " + std::to_string(kMaxOrderTc));
+    if (wait_budget_ns == 0) return fail(HYENA_ERR_INVALID_ARG, "wait_budget_ns must be > 0");
+    a.wait_budget_ns = wait_budget_ns;
+    a.issue_mma = issue_mma ? 1 : 0;
+    cudaError_t e = kernel_status_word(&a.status);
+    if (e != cudaSuccess) return cuda_status(e, "kernel status word");
+    return cuda_status(launch_conv_cluster(p, a, size_t(a.group_rows) * p.ws_row_bytes, static_cast<cudaStream_t>(stream)),
+                       "cluster kernel");
+}
+
 }  // extern "C"
 
 namespace {

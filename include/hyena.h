@@ -434,6 +434,18 @@ hyena_status_t hyena_debug_conv_tc(const void* u, void* y, const void* spectrum,
                                    const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int order,
                                    uint64_t wait_budget_ns, int issue_mma, void* stream);
 
+/*
+ * The same test hook for the cluster kernel (1-D L = 65536, bf16, order <= 3,
+ * shared filters; workspace as in hyena_gated_fftconv).  A CTA whose wait ran
+ * out issues no more tensor-core work but still takes every cluster barrier,
+ * so the cluster finishes; its outputs are NaN and the timeout is recorded in
+ * the device's status word.  Other shapes return HYENA_ERR_UNSUPPORTED_SHAPE.
+ */
+hyena_status_t hyena_debug_conv_cluster(const void* u, void* y, const void* spectrum, size_t spectrum_bytes,
+                                        const float* sc_w, const float* sc_bias, int64_t B, int64_t C, int order,
+                                        void* workspace, size_t workspace_bytes, uint64_t wait_budget_ns,
+                                        int issue_mma, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -57,3 +57,32 @@ def test_tensor_core_wait_timeout_is_reported(orc):
     torch.cuda.synchronize()
     assert torch.equal(y2, r.y)
     hb.hyena_kernel_status()
+
+
+def test_cluster_wait_timeout_is_reported(orc):
+    """The cluster kernel (L = 65536, bf16): one pair, one cluster of 8 CTAs.
+    With no tensor-core work issued every CTA's first wait runs out; each
+    still takes every cluster barrier, so the launch completes, the timeout
+    is recorded, the outputs are NaN, and the next normal call is correct."""
+    import torch
+    p = I.WORKLOADS["order3"].with_(B=2, C=1, L=1 << 16, seed=5102)
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    hb.hyena_kernel_status()
+    spec_before = r.spectrum.clone()
+    y = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_cluster(r.u, y, r.spectrum, r.sc_w, None, p.B, p.C, p.order, r.workspace,
+                                wait_budget_ns=1_000_000, issue_mma=False)
+    torch.cuda.synchronize()
+    with pytest.raises(hb.HyenaError) as ei:
+        hb.hyena_kernel_status()
+    assert ei.value.status == 8                                   # HYENA_ERR_TIMEOUT
+    assert torch.isnan(y.float()).all()
+    assert torch.equal(r.spectrum, spec_before)
+    r.conv()
+    torch.cuda.synchronize()
+    hb.hyena_kernel_status()
+    rows = np.arange(p.B * p.C)
+    err = row_rel_err(gpu_rows(from_torch(r.y), p, rows), oracle_for_rows(orc, p, rows, data, method=2))
+    assert err.max() <= TOL["bf16"], err.max()
