@@ -45,6 +45,7 @@ CASES = [
     I.WORKLOADS["d768_l8k"].with_(B=3, C=5, seed=6002),                                   # tensor cores, bf16
     I.WORKLOADS["d768_l8k"].with_(B=2, C=3, dtype="f32", seed=6003),                      # fp32 register kernel
     I.WORKLOADS["order3"].with_(B=2, C=3, L=1 << 15, seed=6004),                          # four-step, order 3
+    I.WORKLOADS["order3"].with_(B=3, C=2, L=1 << 16, seed=6006),                          # 8-CTA clusters, order 3
     I.WORKLOADS["grid2d"].with_(B=2, C=3, H=64, W=32, sigma=(4.0, 16.0), seed=6005),      # 2-D
 ]
 

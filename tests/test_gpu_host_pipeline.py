@@ -27,6 +27,7 @@ CASES = [
     ("d768_l8k", dict(B=4, C=8), 0),                          # default chunk (2 rows): pairs kept whole
     ("d768_l8k", dict(B=3, C=8), 0),                          # default chunk rounded up to 2 rows
     ("order3", dict(B=3, C=2, L=1 << 15), 1),                 # four-step: chunks share the workspace
+    ("order3", dict(B=4, C=2, L=1 << 16), 2),                 # cluster kernel, pairs kept whole
     ("grid2d", dict(B=2, C=3, H=32, W=64), 1),                # 2-D
 ]
 
