@@ -233,79 +233,16 @@ __device__ __forceinline__ void dft8_first4(const float2 (&x)[8], float2 (&o)[4]
 }
 
 
-// Samples n-2, n-1, n of one row (zero before its start), from one aligned
-// pair load and one single load.
+// Samples n-2, n-1, n of one row (zero before its start).
 struct S3 {
     float m2, m1, c;
 };
-__device__ __forceinline__ S3 load3(const bf16* __restrict__ x, int n) {
-    const int odd = n & 1;
-    const int p2 = n - 2 + odd;                 // even: the pair (n-2, n-1) or (n-1, n)
-    const int ns = odd ? n - 2 : n;
-    const uint32_t pr = p2 >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(x + p2)) : 0u;
-    const float sg = ns >= 0 ? __bfloat162float(__ldg(x + ns)) : 0.0f;
-    S3 r;
-    if (odd) {
-        r.m2 = sg;
-        r.m1 = bf_lo(pr);
-        r.c = bf_hi(pr);
-    } else {
-        r.m2 = bf_lo(pr);
-        r.m1 = bf_hi(pr);
-        r.c = sg;
-    }
-    return r;
-}
 // Short conv at one sample of both rows: (row b0, row b1).
 __device__ __forceinline__ float2 sc_pair(const S3& r0, const S3& r1, const Taps2& tp) {
     return __ffma2_rn(tp.w0, make_float2(r0.m2, r1.m2),
                       __ffma2_rn(tp.w1, make_float2(r0.m1, r1.m1), __ffma2_rn(tp.w2, make_float2(r0.c, r1.c), tp.b)));
 }
 
-// A thread's share of F1 and I1 in round r (r < 2): one a' = 32 q + lane,
-// q = 16 half + 2 warp + r, with the four s' = 4 quad + m (m < 4) of its CTA
-// (rank = 2 quad + half), i.e. a = a' + 1024 s'; the samples are n = a + NI s.
-// Lane-consecutive a' make each warp's remote 16-byte stores whole 128-byte
-// rows-of-8 of the destination operand.
-struct Share {
-    int ap, quad;
-};
-
-// I1 at one a: reads conj V[k1][a] of the 8 CTAs from the cluster's scratch
-// and returns ys[s] = y[a + NI s] (s < 4) as (row b0, row b1).
-__device__ __forceinline__ void i1_one(float2 (&ys)[4], const uint32_t* __restrict__ scr, int a,
-                                       const float2* __restrict__ wa) {
-    uint32_t v[RC];
-#pragma unroll
-    for (int k1 = 0; k1 < RC; ++k1) v[k1] = __ldcg(scr + int64_t(k1) * NI + a);
-    const float2 w1 = __ldg(wa + a);
-    float2 x[8];
-    float2 w = w1;
-#pragma unroll
-    for (int k1 = 0; k1 < RC; ++k1) {
-        const float2 vc = make_float2(bf_lo(v[k1]), bf_hi(v[k1]));
-        // conj U[k1] = w_NO^(a k1) conj V[k1][a]
-        if (k1 == 0) {
-            x[0] = vc;
-        } else {
-            x[k1] = cmul(vc, w);
-            if (k1 + 1 < RC) w = cmul(w, w1);
-        }
-    }
-    float2 o[4];
-    dft8_first4(x, o);
-#pragma unroll
-    for (int s = 0; s < 4; ++s) ys[s] = make_float2(o[s].x, -o[s].y);   // y = conj
-}
-
-// L2 prefetch of this CTA's share of one input row (the samples a' + 1024 s'
-// + NI s of its a'-half and s'-quad: 16 runs of 512 samples), one run per
-// calling thread (run < 16).
-__device__ __forceinline__ void prefetch_share(const bf16* row, int half, int quad, int run) {
-    const int m = run & 3, s = run >> 2;
-    const bf16* src = row + 512 * half + 1024 * (4 * quad + m) + NI * s;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(1024u) : "memory");
-}
 
 // Row pair operands of one order step.
 struct PairRows {
@@ -504,20 +441,6 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
             }
             fence_proxy_async_cluster();
             cluster_sync();
-            // ---- the next gate's rows into L2 while the tensor cores work: x_(g-1),
-            // or after the last step x0 and the next pair's x_(order-1) and v
-            if (t < 96) {
-                const int64_t Ctot = int64_t(p.order + 1) * p.C;
-                const int which = t >> 4, run = t & 15;
-                const bool last = st == p.order - 1;
-                const int nrows = last ? (P + nq < p.npairs ? 6 : 2) : 2;
-                if (which < nrows) {
-                    const PairRef pn = which < 2 ? pr : pair_ref(P + nq, p.B);
-                    const int chunk = which < 2 ? (last ? 0 : g - 1) : (which < 4 ? p.order - 1 : p.order);
-                    const int b = pn.b0 + ((which & 1) && pn.has1 ? 1 : 0);
-                    prefetch_share(p.u + (int64_t(b) * Ctot + int64_t(chunk) * p.C + pn.c) * LC, half, quad, run);
-                }
-            }
             // ---- F2 and its inverse on this CTA's 16384 points
             stage_issue(a_addr, kSBO32, b1f_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 32), tmem, 32, &mbar,
                         ok && p.issue_mma);
