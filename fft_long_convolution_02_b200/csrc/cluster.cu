@@ -441,6 +441,11 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
             }
             fence_proxy_async_cluster();
             cluster_sync();
+            // ---- this CTA's spectrum sub-plane into L2 while the stages before its pass run
+            if (t < 4)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                                 p.plane + ((int64_t(st - 1) * p.C + pr.c) * RC + rank) * NI + t * (NI / 4)),
+                             "r"(uint32_t(NI)) : "memory");
             // ---- F2 and its inverse on this CTA's 16384 points
             stage_issue(a_addr, kSBO32, b1f_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 32), tmem, 32, &mbar,
                         ok && p.issue_mma);

@@ -439,6 +439,14 @@ k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, 
     WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
     const int64_t c = img / B, b = img - c * B;
     const float2* sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride + int64_t(fc) * (2 * MH);
+    if (t < kFC) {
+        // this CTA's spectrum columns into L2 while the forward transform runs
+        const int f2 = blockIdx.x * kFC + t;
+        if (f2 <= W)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sp + int64_t(f2 - fc) * (2 * MH)),
+                         "r"(uint32_t(2 * MH * sizeof(float2)))
+                         : "memory");
+    }
     float2 x[2][16];
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
