@@ -211,6 +211,9 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
                         make_uint2(pk[i][0], pk[i][1]);
             }
             stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
+            if (t < 4)   // this pair's spectrum plane into L2 before its spectrum pass
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(spec + int64_t(c) * (2 * N) + t * (N / 4)),
+                             "r"(uint32_t(N)) : "memory");
             if (have_prev) {
                 output_gate(prev);                  // overlaps the stage-1 MMAs
                 have_prev = false;
