@@ -45,6 +45,8 @@
 // from the filter, then a 16384-point CTA FFT per sub-plane).
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "cta_fft.cuh"
 #include "kernels.h"
@@ -526,6 +528,7 @@ bool cluster_path(const Plan& p, const ConvArgs& a) {
 
 size_t cluster_scratch_bytes() { return size_t(RC) * NI * 4; }
 constexpr int64_t kClusterOversub = 2;
+constexpr int kMaxClusterDevices = 64;
 
 cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspace_bytes, cudaStream_t s) {
     const int64_t npairs = p.C * ((a.B + 1) / 2);
@@ -546,12 +549,21 @@ cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(RC);
-    int max_clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    // the calculator's cluster count, queried once per device
+    static std::atomic<int> g_max_clusters[kMaxClusterDevices];
+    int dev = 0;
+    e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+    if (dev < 0 || dev >= kMaxClusterDevices) return cudaErrorInvalidDevice;
+    int max_clusters = g_max_clusters[dev].load(std::memory_order_relaxed);
+    if (max_clusters == 0) {
+        e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+        g_max_clusters[dev].store(max_clusters, std::memory_order_relaxed);
+    }
     // The occupancy calculator counts one CTA per SM for a kernel that
-    // allocates tensor memory; two fit (256 columns, 128 registers and 93 KB
+    // allocates tensor memory; two fit (256 columns, 127 registers and 114 KB
     // of shared memory each), so twice its cluster count can be resident.
     // One scratch slice per cluster, from the caller's workspace.
     int64_t nclusters = int64_t(workspace_bytes / cluster_scratch_bytes());
