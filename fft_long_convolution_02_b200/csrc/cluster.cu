@@ -296,6 +296,16 @@ __device__ __forceinline__ void f1_step(const ClArgs& p, const PairRows& rw, int
         o.c = __bfloat162float(r[2]);
         return o;
     };
+    // a of item it: a' = 32 (16 half + 2 warp + it / 4) + lane, s' = 4 quad + it % 4
+    auto item_a = [&](int it) { return 32 * (16 * half + 2 * warp + (it >> 2)) + lane + 1024 * (4 * quad + (it & 3)); };
+    // the twiddle base and (after the first step) the scratch values of the
+    // next item are loaded one item ahead, like its staged samples
+    float2 w1n = __ldg(p.wa + item_a(0));
+    uint32_t svn[STEP1 ? 1 : RC];
+    if constexpr (!STEP1) {
+#pragma unroll
+        for (int k1 = 0; k1 < RC; ++k1) svn[k1] = __ldcg(scr + int64_t(k1) * NI + item_a(0));
+    }
     issue(0);
 #pragma unroll 1
     for (int r = 0; r < 2; ++r) {
@@ -307,11 +317,17 @@ __device__ __forceinline__ void f1_step(const ClArgs& p, const PairRows& rw, int
             if (it < 7) issue(it + 1);
             else cp_async_commit();
             const int a = ap + 1024 * (4 * quad + m);
-            const float2 w1 = __ldg(p.wa + a);
+            const float2 w1 = w1n;
             uint32_t sv[STEP1 ? 1 : RC];
-            if constexpr (!STEP1) {
 #pragma unroll
-                for (int k1 = 0; k1 < RC; ++k1) sv[k1] = __ldcg(scr + int64_t(k1) * NI + a);
+            for (int k1 = 0; k1 < (STEP1 ? 1 : RC); ++k1) sv[k1] = svn[k1];
+            if (it < 7) {
+                const int an = item_a(it + 1);
+                w1n = __ldg(p.wa + an);
+                if constexpr (!STEP1) {
+#pragma unroll
+                    for (int k1 = 0; k1 < RC; ++k1) svn[k1] = __ldcg(scr + int64_t(k1) * NI + an);
+                }
             }
             asm volatile("cp.async.wait_group 1;\n" ::: "memory");
             __syncwarp();
