@@ -104,3 +104,17 @@ def test_cluster_reports_a_spectrum_header_mismatch():
     hb.hyena_gated_fftconv(r.u, y, r.spectrum, r.sc_w, None, p.B, p.C, p.shape, p.order, r.workspace)
     hb.hyena_kernel_status()
     assert torch.isfinite(y.float()).all()
+
+
+def test_order4_at_65536_takes_the_multipass_path(orc):
+    """Above order 3 the bf16-operand error would accumulate past the
+    tolerance, so L = 65536 with order 4 runs the fp32 multi-pass kernels:
+    within the bf16 storage tolerance and closer to the oracle than the
+    cluster path's order-3 error."""
+    p = I.WORKLOADS["order3"].with_(B=2, C=2, L=L, order=4, seed=9500)
+    data = I.make_all(p)
+    r = _run(p, data)
+    rows = np.arange(p.B * p.C)
+    ref = oracle_for_rows(orc, p, rows, data, method=2)
+    err = row_rel_err(gpu_rows(from_torch(r.y), p, rows), ref).max()
+    assert err <= 5e-3, err
