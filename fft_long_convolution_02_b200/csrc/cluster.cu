@@ -400,13 +400,13 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_cl[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
+    // the header is requested first and checked after the table setup (which
+    // reads no global memory); every CTA of a cluster reads the same header, so
+    // they all leave together, before the first cluster barrier
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(p.spectrum);
-    // every CTA of a cluster reads the same header, so they all leave together
-    if (!(h->magic == kSpecMagic && h->path == PATH_MULTIPASS_1D && h->C == p.C && h->L == LC &&
-          h->order == p.order && h->tables_off == p.tables_off && h->reserved[0] == p.plane_off)) {
-        if (threadIdx.x == 0) report_status(p.status, kStatusSpectrumMismatch);
-        return;
-    }
+    const SpecHeader hv = *h;
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_MULTIPASS_1D) & (hv.C == p.C) & (hv.L == LC) &
+                        (hv.order == p.order) & (hv.tables_off == p.tables_off) & (hv.reserved[0] == p.plane_off);
     uint8_t* A = smem_cl;
     float4* TW2 = reinterpret_cast<float4*>(smem_cl + kOffTW2c);
     const int t = threadIdx.x;
@@ -418,9 +418,13 @@ k_conv_cluster(const __grid_constant__ ClArgs p) {
     float2* w32 = reinterpret_cast<float2*>(smem_cl);   // operand area, free until the first F1
     fill_w32(w32);
     __syncthreads();
-    fill_dft(smem_cl + kOffB1f, 16, 16, 16, kSBO32, w32);
-    fill_dft(smem_cl + kOffB32c, 32, 32, 32, kSBO64, w32);
-    fill_tw2(TW2, p.even, p.odd);
+    fill_dft<16, 16, 16, kSBO32>(smem_cl + kOffB1f, w32);
+    fill_dft<32, 32, 32, kSBO64>(smem_cl + kOffB32c, w32);
+    fill_tw2(TW2);
+    if (!hdr_ok) {
+        if (t == 0) report_status(p.status, kStatusSpectrumMismatch);
+        return;
+    }
     if (t == 0) tc::mbar_init(&mbar, 1);
     if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
     tc::fence_before_sync();

@@ -77,12 +77,13 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
+    // the header is requested first and checked once the tables below are set
+    // up (they read no global memory), so that its latency overlaps them
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
-    if (!(h->magic == kSpecMagic && h->path == PATH_ONCHIP_1D && h->C == C && h->L == L && h->order == order &&
-          h->spec_row_bytes == int64_t(N) * 8 && h->tables_off == tables_off && h->spec_off == spec_off)) {
-        if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
-        return;
-    }
+    const SpecHeader hv = *h;                       // all fields requested at once (no short-circuit chain)
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_ONCHIP_1D) & (hv.C == C) & (hv.L == L) &
+                        (hv.order == order) & (hv.spec_row_bytes == int64_t(N) * 8) & (hv.tables_off == tables_off) &
+                        (hv.spec_off == spec_off);
     // the layout offsets are kernel parameters (checked against the header above),
     // so that the table pointers need no registers of their own
     const float2* tables = reinterpret_cast<const float2*>(spectrum + tables_off);
@@ -106,10 +107,14 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     float2* w32 = reinterpret_cast<float2*>(smem_tc);
     fill_w32(w32);
     __syncthreads();
-    fill_dft(smem_tc + kOffB1, 16, 16, 8, kSBO16, w32);
-    fill_dft(smem_tc + kOffB32, 32, 32, 32, kSBO64, w32);
-    fill_dft(smem_tc + kOffB1i, 16, 8, 16, kSBO32, w32);
-    fill_tw2(TW2, twist, odd);
+    fill_dft<16, 16, 8, kSBO16>(smem_tc + kOffB1, w32);
+    fill_dft<32, 32, 32, kSBO64>(smem_tc + kOffB32, w32);
+    fill_dft<16, 8, 16, kSBO32>(smem_tc + kOffB1i, w32);
+    fill_tw2(TW2);
+    if (!hdr_ok) {                                  // uniform: every thread read the same header
+        if (t == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
     if (t == 0) tc::mbar_init(&mbar, 1);
     if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
     tc::fence_before_sync();

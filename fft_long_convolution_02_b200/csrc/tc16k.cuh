@@ -111,10 +111,13 @@ __device__ __forceinline__ C2 c2_at(const float (&d)[NCOL], int p) {
 // j = 2 s + (0: re, 1: im) of input s; row n holds output k = 2 (n >> 2) + (n & 1),
 // real part for (n >> 1) & 1 == 0, else imaginary part, so that the accumulator
 // columns of outputs 2p, 2p+1 read (re, re, im, im).  w32 holds (cos, sin) of
-// 2 pi i / 32, i < 32 (R divides 32).
-__device__ inline void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t sbo, const float2* w32) {
-    for (int idx = threadIdx.x; idx < 4 * nout * nin; idx += blockDim.x) {
-        const int n = idx / (2 * nin), j = idx % (2 * nin);
+// 2 pi i / 32, i < 32 (R divides 32).  The sizes are compile-time constants,
+// so that the index arithmetic is shifts and masks.
+template <int R, int NOUT, int NIN, uint32_t SBO>
+__device__ inline void fill_dft(uint8_t* Bm, const float2* w32) {
+    static_assert(32 % R == 0 && (NIN & (NIN - 1)) == 0, "DFT matrix sizes");
+    for (int idx = threadIdx.x; idx < 4 * NOUT * NIN; idx += blockDim.x) {
+        const int n = idx / (2 * NIN), j = idx % (2 * NIN);
         const int k = 2 * (n >> 2) + (n & 1);
         const bool im_row = (n >> 1) & 1;
         const int e = (k * (j >> 1)) % R;
@@ -123,7 +126,7 @@ __device__ inline void fill_dft(uint8_t* Bm, int R, int nout, int nin, uint32_t 
         float v;
         if (!im_row) v = (j & 1) == 0 ? cv : sv;            // re: Re w xr - Im w xi
         else v = (j & 1) == 0 ? -sv : cv;                   // im: Im w xr + Re w xi
-        *reinterpret_cast<bf16*>(Bm + tc::kmaj_off(n, j, sbo)) = __float2bfloat16_rn(v);
+        *reinterpret_cast<bf16*>(Bm + tc::kmaj_off(n, j, SBO)) = __float2bfloat16_rn(v);
     }
 }
 
@@ -203,15 +206,23 @@ __device__ __forceinline__ PairRef pair_ref(int P, int B) {
     return r;
 }
 
+// w1024^e = exp(-2 pi i e / 1024), e < 1024, from sincospif (within an ulp
+// or two of the correctly rounded value).
+__device__ __forceinline__ float2 w1024(int e) {
+    float sv, cv;
+    sincospif(float(e) * (1.0f / 512.0f), &sv, &cv);
+    return make_float2(cv, -sv);
+}
+
 // TW2[(T * 16 + kp) * 8 + l] = (Re w0, Re w1, Im w0, Im w1), w0 = w1024^(b k),
 // w1 = w1024^(b (k+1)), b = 4 l + T, k = 2 kp: the stage-2 / stage-3' twiddles.
-__device__ __forceinline__ void fill_tw2(float4* TW2, const float2* __restrict__ twist,
-                                         const float2* __restrict__ odd) {
+// Computed in place (no global reads), so that the setup does not wait on memory.
+__device__ __forceinline__ void fill_tw2(float4* TW2) {
     for (int idx = threadIdx.x; idx < 4 * 16 * 8; idx += blockDim.x) {
         const int l = idx & 7, kp = (idx >> 3) & 15, T = idx >> 7;
         const int bb = 4 * l + T, k = 2 * kp;
-        const float2 w0 = wN(16 * ((bb * k) & 1023), twist, odd);
-        const float2 w1 = wN(16 * ((bb * (k + 1)) & 1023), twist, odd);
+        const float2 w0 = w1024((bb * k) & 1023);
+        const float2 w1 = w1024((bb * (k + 1)) & 1023);
         TW2[idx] = make_float4(w0.x, w1.x, w0.y, w1.y);
     }
 }
