@@ -547,8 +547,13 @@ bool cluster_path(const Plan& p, const ConvArgs& a) {
 }
 
 size_t cluster_scratch_bytes() { return size_t(RC) * NI * 4; }
-constexpr int64_t kClusterOversub = 2;
 constexpr int kMaxClusterDevices = 64;
+
+// Never launched: the cluster kernel's block size and shared memory without
+// its tensor-memory allocation, for the occupancy calculator (which counts one
+// CTA per SM for any kernel that allocates tensor memory, although two of
+// k_conv_cluster fit: 2 x 256 columns, 2 x 256 threads x 128 registers).
+__global__ void __launch_bounds__(NT, 2) k_cluster_occupancy_probe() {}
 
 cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspace_bytes, cudaStream_t s) {
     const int64_t npairs = p.C * ((a.B + 1) / 2);
@@ -569,7 +574,12 @@ cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(RC);
-    // the calculator's cluster count, queried once per device
+    // Clusters resident at once with two CTAs per SM, queried once per device
+    // on the probe kernel (same block size and shared memory): the grid is
+    // persistent with a static share of pairs per cluster, so a cluster that
+    // could not be resident would start only when another ends.  How many
+    // 8-CTA clusters fit depends on how the SMs are spread over the GPCs (33
+    // on the B200s measured; 34 did not fit).
     static std::atomic<int> g_max_clusters[kMaxClusterDevices];
     int dev = 0;
     e = cudaGetDevice(&dev);
@@ -577,17 +587,23 @@ cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspa
     if (dev < 0 || dev >= kMaxClusterDevices) return cudaErrorInvalidDevice;
     int max_clusters = g_max_clusters[dev].load(std::memory_order_relaxed);
     if (max_clusters == 0) {
-        e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+        // the probe's dynamic shared memory stands for the kernel's dynamic and static parts
+        cudaFuncAttributes fa{};
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t pcfg = cfg;
+        pcfg.dynamicSmemBytes = kSmemC + fa.sharedSizeBytes;
+        e = cudaFuncSetAttribute(k_cluster_occupancy_probe, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(pcfg.dynamicSmemBytes));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveClusters(&max_clusters, k_cluster_occupancy_probe, &pcfg);
         if (e != cudaSuccess) return e;
         if (max_clusters < 1) return cudaErrorInvalidConfiguration;
         g_max_clusters[dev].store(max_clusters, std::memory_order_relaxed);
     }
-    // The occupancy calculator counts one CTA per SM for a kernel that
-    // allocates tensor memory; two fit (256 columns, 127 registers and 114 KB
-    // of shared memory each), so twice its cluster count can be resident.
-    // One scratch slice per cluster, from the caller's workspace.
+    // one scratch slice per cluster, from the caller's workspace
     int64_t nclusters = int64_t(workspace_bytes / cluster_scratch_bytes());
-    if (nclusters > kClusterOversub * int64_t(max_clusters)) nclusters = kClusterOversub * int64_t(max_clusters);
+    if (nclusters > int64_t(max_clusters)) nclusters = int64_t(max_clusters);
     if (nclusters > npairs) nclusters = npairs;
     if (nclusters < 1) return cudaErrorInvalidValue;
     cfg.gridDim = dim3(unsigned(nclusters * RC));

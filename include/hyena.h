@@ -225,8 +225,9 @@ size_t hyena_gated_fftconv_workspace_min_bytes(int64_t C, int ndim, const int64_
  *   workspace, workspace_bytes  device scratch for the multi-pass (L >= 32768)
  *            and 2-D paths; may be NULL/0 for the on-chip path.  Its contents
  *            are undefined after the call.  The cluster path (L = 65536, bf16)
- *            takes 512 KB per cluster in flight from it (up to 30 clusters
- *            on a B200); the minimum workspace runs one cluster.
+ *            takes 512 KB per cluster in flight from it (as many clusters
+ *            as are resident at two CTAs per SM: 33 on the B200s measured);
+ *            the minimum workspace runs one cluster.
  *
  * The spectrum is only read.  Conditions the kernels detect on the device (a
  * spectrum whose header does not match the shape: that kernel writes no
