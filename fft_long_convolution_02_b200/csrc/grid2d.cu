@@ -135,7 +135,7 @@ template <int MH, int MODE, typename WT>
 __global__ void __launch_bounds__(kColThreads2)
 k_2d_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, const float* __restrict__ D, float s8,
-          int64_t SC, int64_t SB) {
+          int64_t SC, int64_t SB, int line0, int line1, int lines_per_block) {
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(MH);
     const int64_t img = img0 + blockIdx.y;
@@ -150,8 +150,9 @@ k_2d_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, i
     } else {
         d = D ? __ldg(D + img) : 0.0f;
     }
-    const int f_begin = MODE == 0 ? int(blockIdx.x) * kCB : 0;
-    const int f_end = MODE == 0 ? min(f_begin + kCB, ncol) : ncol;
+    // spectrum build: this block's lines of the wave [line0, line1) (see spectrum_cols_waves)
+    const int f_begin = MODE == 0 ? int(blockIdx.x) * kCB : line0 + int(blockIdx.x) * lines_per_block;
+    const int f_end = MODE == 0 ? min(f_begin + kCB, ncol) : min(f_begin + lines_per_block, line1);
     const int per = MODE == 0 ? kCB : 1;
     for (int f0 = f_begin; f0 < f_end; f0 += per) {
         const int nc = min(per, f_end - f0);
@@ -644,7 +645,9 @@ k_2dc_cols_spec(float2* __restrict__ rows, T2d tb, int ncol, int64_t row0, int64
     const int64_t r = row0 + blockIdx.y;
     float2* img = rows + int64_t(blockIdx.y) * row_stride;
     const float d = D ? __ldg(D + r) : 0.0f;
-    for (int f = 0; f < ncol; ++f) {
+    // each column is transformed in place (no expansion): the columns of an
+    // image are independent and spread over the blocks of the grid's x
+    for (int f = blockIdx.x; f < ncol; f += gridDim.x) {
         for (int p = threadIdx.x; p < MH; p += blockDim.x) smem[fft_pad(p)] = img[int64_t(f) * MH + p];
         __syncthreads();
         cta_fft_forward<MH>(smem, 1, fft_padded_size(MH), tb.fftH);
@@ -742,6 +745,28 @@ size_t col_smem2(int per) {
     return size_t(2) * per * fft_padded_size(MH) * sizeof(float2);
 }
 
+// The spectrum mode of k_2d_cols works in place: the input of line j sits at
+// entries (n + j) MH .. (n + j + 1) MH of the channel's region (n lines), and
+// line f writes its 2 MH outputs over entries 2 MH f .. 2 MH (f + 1), which
+// hold the inputs of lines 2f - n and 2f + 1 - n.  A wave of lines [a, b)
+// with b <= (a + n) / 2 therefore overwrites only inputs of lines below a,
+// transformed by earlier waves, and the last line only its own input (read
+// into shared memory before it is written), so the n lines run in about
+// log2(n) waves of parallel blocks instead of one block per channel.
+constexpr int kSpecLinesPerBlock = 4;
+template <typename K>
+void spectrum_cols_waves(K kb, int n, unsigned nimg, size_t smem, cudaStream_t s, float2* rows, const T2d& tb,
+                         int W, int C, int64_t img0, int64_t stride, const float* D, float scale) {
+    for (int a0 = 0; a0 < n;) {
+        int b = (a0 + n) / 2;
+        if (b <= a0) b = a0 + 1;             // a0 = n - 1: the last line
+        const unsigned blocks = unsigned((b - a0 + kSpecLinesPerBlock - 1) / kSpecLinesPerBlock);
+        kb<<<dim3(blocks, nimg), kColThreads2, smem, s>>>(rows, nullptr, tb, W, 1, C, 0, img0, stride, 0, D, scale, 0,
+                                                           0, a0, b, kSpecLinesPerBlock);
+        a0 = b;
+    }
+}
+
 template <int MW, int MH>
 cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     const T2d tb = t2d(p, a.spectrum);
@@ -769,8 +794,7 @@ cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
         else
             kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
                                                2, H, i0, stride, upper);
-        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, nullptr, tb, W, 1, p.C, 0, i0, stride,
-                                                           0, a.D, s8, 0, 0);
+        spectrum_cols_waves(kb, W + 1, unsigned(g), smB, s, rows + i0 * stride, tb, W, int(p.C), i0, stride, a.D, s8);
     }
     return cudaGetLastError();
 }
@@ -812,7 +836,7 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
             kb<<<dim3(unsigned((W + 1 + kCB - 1) / kCB), unsigned(g)), kColThreads2, smB, s>>>(
                 ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, nullptr, 0.0f, a.spec_C,
-                a.spec_per_b);
+                a.spec_per_b, 0, 0, 0);
         }
     };
     auto launch_rows_fwd = [&](int64_t i0, int64_t g) {
@@ -876,7 +900,8 @@ cudaError_t spectrum_2dc_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s)
         else
             kh<<<gridA, kRowThreads, smA, s>>>(static_cast<const __nv_bfloat16*>(a.k), rows + i0 * stride, tb, 1, 1,
                                                2, H, i0, stride);
-        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, tb, W / 2 + 1, i0, stride, a.D, s2);
+        kb<<<dim3(unsigned(W / 2 + 1), unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, tb, W / 2 + 1, i0,
+                                                                             stride, a.D, s2);
     }
     return cudaGetLastError();
 }
@@ -973,8 +998,8 @@ cudaError_t spectrum_3d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
                                                                                           N1, 0, ws2_off, stride);
         // k_2d_cols in spectrum mode reads its columns from the upper half
         // (offset ncol * MD = nlines * N1) and writes 2 N1 entries per line
-        kb<<<dim3(1, unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, nullptr, tbd, int(nlines - 1), 1, p.C,
-                                                           0, i0, stride, 0, a.D, s16, 0, 0);
+        spectrum_cols_waves(kb, int(nlines), unsigned(g), smB, s, rows + i0 * stride, tbd, int(nlines - 1), int(p.C),
+                            i0, stride, a.D, s16);
     }
     return cudaGetLastError();
 }
