@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 OBJ = os.path.join(ROOT, "_build", "obj")
 LIB = os.path.join(HERE, "libhyena_b200.so")
 
-CU_SOURCES = ["api.cu", "tables.cu", "onchip.cu", "shortconv.cu", "multipass.cu", "grid2d.cu", "noalloc.cu", "onchip_tc.cu", "status.cu", "proj.cu", "filtergen.cu", "cluster.cu"]
+CU_SOURCES = ["api.cu", "tables.cu", "onchip.cu", "shortconv.cu", "multipass.cu", "grid2d.cu", "noalloc.cu", "onchip_tc.cu", "status.cu", "proj.cu", "filtergen.cu", "cluster.cu", "grid2d_tc.cu"]
 CPP_SOURCES = ["plan.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -165,12 +165,14 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
     if (st != HYENA_OK) return st;
     // the spectrum holds C filters per order step, or B*C (one per (b, c) row)
     size_t spec_total = p.total_bytes;
+    size_t g2_plane = p.g2_plane_off;
     if (per_sample) {
         Plan ps;
         if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
         st = plan_or_fail(B * C, ndim, sizes, order, &ps);
         if (st != HYENA_OK) return st;
         spec_total = ps.total_bytes;
+        g2_plane = ps.g2_plane_off;
     }
     if (!u || !y || !spectrum) return fail(HYENA_ERR_INVALID_ARG, "u, y and spectrum must not be NULL");
     if (B < 1) return fail(HYENA_ERR_INVALID_ARG, "B must be >= 1");
@@ -204,6 +206,7 @@ hyena_status_t prepare_conv(const void* u, void* y, const void* spectrum, size_t
                    static_cast<float2*>(workspace), group};
     pa->spec_C = per_sample ? B * C : C;
     pa->spec_per_b = per_sample ? C : 0;
+    pa->g2_plane_off = g2_plane;
     return HYENA_OK;
 }
 

@@ -425,24 +425,27 @@ k_2df_rows_inv(const T* __restrict__ u, T* __restrict__ y, typename WsOf<T>::typ
 
 // Column pass (convolution): 2H-point FFT of each zero-padded bin column as two
 // H-point chains, times K~ (thread order), inverse, keep p < H.
-template <int MH, typename WT>
+// LAST: only the last bin column (f = W) of every image, thread group cc of
+// block x taking image 16 x + cc (nimg images in the launch).
+template <int MH, typename WT, bool LAST = false>
 __global__ void __launch_bounds__(kFC * (MH / 16), (512 / (kFC * (MH / 16))) > 0 ? 512 / (kFC * (MH / 16)) : 1)
 k_2df_cols(WT* __restrict__ ws, const float2* __restrict__ spec, T2d tb, int W, int64_t B, int64_t C, int step,
-           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, int64_t SC, int64_t SB) {
+           int64_t img0, int64_t ws_img_stride, int64_t spec_row_stride, int64_t SC, int64_t SB, int nimg) {
     extern __shared__ float2 smem[];
     constexpr int TPT = MH / 16;
     constexpr int PS = fft_padded_size(MH);
     const int t = threadIdx.x, cc = t / TPT, g = t - (t / TPT) * TPT;
-    const int64_t img = img0 + blockIdx.y;
-    const int f = blockIdx.x * kFC + cc;
-    const bool active = f <= W;
-    const int fc = active ? f : W;
-    WT* ws_img = ws + int64_t(blockIdx.y) * ws_img_stride;
+    const int li = LAST ? min(int(blockIdx.x) * kFC + cc, nimg - 1) : int(blockIdx.y);
+    const int64_t img = img0 + li;
+    const int f = LAST ? W : int(blockIdx.x) * kFC + cc;
+    const bool active = LAST ? int(blockIdx.x) * kFC + cc < nimg : f <= W;
+    const int fc = LAST ? W : (active ? f : W);
+    WT* ws_img = ws + int64_t(li) * ws_img_stride;
     const int64_t c = img / B, b = img - c * B;
     const float2* sp = spec + (int64_t(step) * SC + b * SB + c) * spec_row_stride + int64_t(fc) * (2 * MH);
-    if (t < kFC) {
+    if (!LAST && t < kFC) {
         // this CTA's spectrum columns into L2 while the forward transform runs
-        const int f2 = blockIdx.x * kFC + t;
+        const int f2 = int(blockIdx.x) * kFC + t;
         if (f2 <= W)
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sp + int64_t(f2 - fc) * (2 * MH)),
                          "r"(uint32_t(2 * MH * sizeof(float2)))
@@ -796,6 +799,11 @@ cudaError_t spectrum_2d_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s) 
                                                2, H, i0, stride, upper);
         spectrum_cols_waves(kb, W + 1, unsigned(g), smB, s, rows + i0 * stride, tb, W, int(p.C), i0, stride, a.D, s8);
     }
+    if (p.g2_plane_off != 0) {
+        const cudaError_t e = launch_spectrum_2d_tc_plane(p, reinterpret_cast<const uint8_t*>(rows), a.spectrum + p.g2_plane_off,
+                                                          nimg, s);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 
@@ -825,12 +833,25 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const size_t smR = size_t(2 * FR) * row_stride_f<MW>() * sizeof(float2);
     const size_t smC = size_t(2 * kFC) * fft_padded_size(MH) * sizeof(float2);
     const size_t smB = col_smem2<MH>(kCB);
+    const bool cols_tc = cols_2d_tc_path(p, a);
+    cudaError_t tc_err = cudaSuccess;
     auto launch_cols = [&](int64_t i0, int64_t g, int st) {
         if constexpr (COLS_REG) {
             auto kb = k_2df_cols<MH, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
-            kb<<<dim3(unsigned((W + 1 + kFC - 1) / kFC), unsigned(g)), NTC, smC, s>>>(
-                ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, a.spec_C, a.spec_per_b);
+            if (cols_tc) {
+                // columns 0 .. W-1 on the tensor cores, the last bin column here
+                const cudaError_t e = launch_cols_2d_tc(p, a, ws, i0, g, st - 1, stride, s);
+                if (tc_err == cudaSuccess) tc_err = e;
+                auto kl = k_2df_cols<MH, WT, true>;
+                cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smC));
+                kl<<<dim3(unsigned((g + kFC - 1) / kFC), 1), NTC, smC, s>>>(ws, spec, tb, W, a.B, p.C, st - 1, i0,
+                                                                             stride, spec_stride, a.spec_C,
+                                                                             a.spec_per_b, int(g));
+            } else {
+                kb<<<dim3(unsigned((W + 1 + kFC - 1) / kFC), unsigned(g)), NTC, smC, s>>>(
+                    ws, spec, tb, W, a.B, p.C, st - 1, i0, stride, spec_stride, a.spec_C, a.spec_per_b, int(g));
+            }
         } else {
             auto kb = k_2d_cols<MH, 0, WT>;
             cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smB));
@@ -872,6 +893,7 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
             launch_rows_inv(i0, g, st == p.order - 1, st < p.order - 1 ? p.order - st - 1 : 0);
         }
     }
+    if (tc_err != cudaSuccess) return tc_err;
     return cudaGetLastError();
 }
 
@@ -1045,7 +1067,7 @@ cudaError_t conv_3d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
             kcf<<<dim3(cblocks, unsigned(g)), kFC * (MH / 16), smC, s>>>(ws, tb, N1, 0, ws2_off, stride);
             kd<<<dim3(dblocks, unsigned(g)), kFC * (MD / 16), smD, s>>>(ws + ws2_off, spec, tbd, int(nlines - 1),
                                                                         a.B, p.C, st - 1, i0, stride, spec_stride,
-                                                                        a.spec_C, a.spec_per_b);
+                                                                        a.spec_C, a.spec_per_b, int(g));
             kci<<<dim3(cblocks, unsigned(g)), kFC * (MH / 16), smC, s>>>(ws, tb, N1, 0, ws2_off, stride);
             if (st < p.order - 1)
                 kca<<<gridR, kRowThreads, row_smem<MW>(), s>>>(u, y, ws, tb, a.B, p.C, p.order, p.order - st - 1,

@@ -1,0 +1,373 @@
+// grid2d_tc.cu -- the column pass of the 2-D non-circular form ([P5] "Native
+// Multi-Dimensional Subquadratic Operators" (gist.science), 方法论: N-D FFT
+// convolution, non-circular by 2x zero padding) with bf16 storage and H = 256
+// on the tensor cores (tcgen05).
+//
+// The row pass leaves, per image, W + 1 bin columns of H = 256 complex values
+// (bf16 (re, im) in the workspace).  Each column needs its 2H = 512-point DFT
+// (rows H .. 2H-1 are zero), the product with its spectrum column and the
+// inverse, keeping rows p < H.  With n = a + 32 s (a < 32, s < 8 non-zero)
+// and bin k = k1 + 16 k2 (k1 < 16, k2 < 32):
+//   X[k1 + 16 k2] = sum_a w32^(a k2) w512^(a k1) sum_s x[a + 32 s] w16^(s k1)
+// so a task of 32 columns (16384 points) runs the first two stages of the
+// 16384-point tensor-core FFT (tc16k.cuh: stage 1 over s, K = 16; stage 2
+// over a, K = 64) with the twiddle w512^(a k1) between them, the spectrum
+// product on the stage-2 accumulators, and the inverse through the same
+// matrices (IDFT(x) = conj(DFT(conj x))): stage 2', the same twiddle, and
+// stage 1' with only the outputs s < 8.  Rows of the stage-1 operand are
+// a_tc = c + 32 a for column c of the task, i.e. b = c and q = a in the row
+// orders of tc16k.cuh.
+//
+// Columns 0 .. W-1 run here (W / 32 tasks per image); the last column (bin W)
+// stays on the register-engine column kernel.  The spectrum comes from a bf16
+// plane in this kernel's thread order, gathered from the complex64 spectrum
+// rows when the spectrum is built.
+//
+// Precision: column values, DFT matrices and the stage operands are bf16
+// (fp32 accumulation), four roundings per transform pair; the 2-D row error
+// stays a few 1e-3.
+#include "common.cuh"
+#include "cta_fft.cuh"
+#include "kernels.h"
+#include "plan_common.h"
+#include "tc16k.cuh"
+#include "tc_util.cuh"
+
+namespace hyena {
+
+namespace {
+
+using namespace tc16k;
+
+constexpr int MH = int(kTc2dH);   // column length H
+constexpr int NCOL = 32;          // columns per task
+constexpr int NT = 256;
+static_assert(NCOL * MH * 2 == N, "a task is one 16384-point transform");
+constexpr uint32_t kB1bytes = 4 * kSBO16;   // N 32 x K 16
+constexpr uint32_t kB1ibytes = 2 * kSBO32;  // N 16 x K 32
+constexpr uint32_t kOffA1 = kAbytes - 128 * kSBO16;   // stage-1 operand (1024 rows x K 16)
+constexpr uint32_t kOffB1 = kAbytes;
+constexpr uint32_t kOffB32 = kOffB1 + kB1bytes;
+constexpr uint32_t kOffB1i = kOffB32 + kB32bytes;
+constexpr uint32_t kOffW512 = kOffB1i + kB1ibytes;
+constexpr size_t kSmem = size_t(kOffW512) + 512 * sizeof(float2);
+static_assert(NCOL * MH * 4 <= kOffA1, "output staging must not overlap the stage-1 operand");
+static_assert(kOffW512 % 16 == 0, "twiddle table alignment");
+constexpr int kPlaneTask = N;     // bf16 (re, im) entries of the spectrum plane per task
+
+// Spectrum plane entry e (uint32 bf16 pair) of task-plane index idx4 (uint4):
+// idx4 = ((Q * 2 + h) * 16 + i) * 32 + lane, i = 4 T + q4 holds, for lane
+// quarter Q, half h and tile T, row (k1 = 4 Q + lane / 8, column c = 4 (lane & 7) + T)
+// and bins k2 = 16 h + 4 q4 + e (e < 4): the order the spectrum pass reads.
+__device__ __forceinline__ void plane_entry(int idx4, int e, int& c, int& k) {
+    const int lane = idx4 & 31, i = (idx4 >> 5) & 15, qh = idx4 >> 9;
+    const int Q = qh >> 1, h = qh & 1, T = i >> 2, q4 = i & 3;
+    const int k1 = 4 * Q + (lane >> 3);
+    c = 4 * (lane & 7) + T;
+    k = k1 + 16 * (16 * h + 4 * q4 + e);
+}
+
+// The plane from the complex64 spectrum rows: per row (W/32 tasks) x 4096 uint4.
+// Bin k of column f sits in the row at f * 2H + (k & 1) * H + the register
+// engine's slot of position fft_bin_pos(k >> 1) (see the 2-D spectrum build).
+__global__ void k_2d_plane_tc(const float2* __restrict__ rows, uint4* __restrict__ plane, int64_t nrows, int W,
+                              int64_t row_stride) {
+    const int64_t per_row = int64_t(W / NCOL) * (kPlaneTask / 4);
+    for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < nrows * per_row;
+         g += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = g / per_row;
+        const int rem = int(g - r * per_row);
+        const int task = rem / (kPlaneTask / 4), idx4 = rem - task * (kPlaneTask / 4);
+        uint32_t v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int c, k;
+            plane_entry(idx4, e, c, k);
+            const int f = NCOL * task + c;
+            const int pos = fft_bin_pos<MH>(k >> 1);
+            const float2 K = rows[r * row_stride + int64_t(f) * (2 * MH) + (k & 1) * MH + (pos & 15) * (MH / 16) +
+                                  (pos >> 4)];
+            v[e] = pack_bf16(K.x, K.y);
+        }
+        plane[g] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum, int C, int W, int64_t B,
+             int step, int64_t img0, int nimg, int64_t ws_img_stride, int64_t plane_off, int64_t SC, int64_t SB,
+             uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_2t[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    // the header is requested first and checked once the tables are set up
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    const SpecHeader hv = *h;
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W) &
+                        (hv.reserved[1] == plane_off);
+    uint8_t* A = smem_2t;
+    uint8_t* A1 = smem_2t + kOffA1;
+    uint32_t* Vs = reinterpret_cast<uint32_t*>(smem_2t);     // output staging [column][p]
+    float2* w512 = reinterpret_cast<float2*>(smem_2t + kOffW512);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+
+    float2* w32 = reinterpret_cast<float2*>(smem_2t);
+    fill_w32(w32);
+    for (int e = t; e < 512; e += NT) {
+        float sv, cv;
+        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);   // w512^e = exp(-2 pi i e / 512)
+        w512[e] = make_float2(cv, -sv);
+    }
+    __syncthreads();
+    fill_dft<16, 16, 8, kSBO16>(smem_2t + kOffB1, w32);
+    fill_dft<32, 32, 32, kSBO64>(smem_2t + kOffB32, w32);
+    fill_dft<16, 8, 16, kSBO32>(smem_2t + kOffB1i, w32);
+    if (!hdr_ok) {
+        if (t == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
+    if (t == 0) tc::mbar_init(&mbar, 1);
+    if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t a1_addr = tc::smem_u32(A1);
+    const uint32_t b1_addr = tc::smem_u32(smem_2t + kOffB1);
+    const uint32_t b32_addr = tc::smem_u32(smem_2t + kOffB32);
+    const uint32_t b1i_addr = tc::smem_u32(smem_2t + kOffB1i);
+    const uint4* plane = reinterpret_cast<const uint4*>(spectrum + plane_off);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int groups = W / NCOL;
+    const int ntasks = nimg * groups;
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int li = task / groups, cg = task - li * groups;
+        const int64_t img = img0 + li;
+        uint32_t* col0 = reinterpret_cast<uint32_t*>(ws + int64_t(li) * ws_img_stride) + int64_t(NCOL * cg) * MH;
+        const int64_t c = img / B, b = img - c * B;
+        const uint4* kq = plane + ((int64_t(step) * SC + b * SB + c) * groups + cg) * (kPlaneTask / 4) +
+                          (Q * 2 + hh) * 16 * 32 + lane;
+        // ---------------- stage-1 operand: rows a_tc = c + 32 a, slots s < 8 (x[c][a + 32 s])
+        {
+            const int chalf = t >> 7, a0 = 8 * (t & 127);
+            const int r0 = rho1(a0);
+            const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
+            uint32_t x[8][4];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int atc = a0 + i, cc = atc & 31, aa = atc >> 5;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[i][j] = col0[cc * MH + aa + 32 * (4 * chalf + j)];
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int jp = 0; jp < 4; jp += 2)
+                    *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u +
+                                              4u * jp) = make_uint2(x[i][jp], x[i][jp + 1]);
+        }
+        stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
+        if (t < 12 && task + int(gridDim.x) < ntasks) {
+            // the next task's 32 columns (32 KB) and spectrum block (64 KB) into L2
+            const int nt = task + int(gridDim.x), nli = nt / groups, ncg = nt - nli * groups;
+            const int64_t nimg_i = img0 + nli, nc = nimg_i / B, nb = nimg_i - nc * B;
+            const uint8_t* src = t < 4 ? reinterpret_cast<const uint8_t*>(reinterpret_cast<const uint32_t*>(
+                                             ws + int64_t(nli) * ws_img_stride) + int64_t(NCOL * ncg) * MH) + 8192 * t
+                                       : reinterpret_cast<const uint8_t*>(
+                                             plane + ((int64_t(step) * SC + nb * SB + nc) * groups + ncg) *
+                                                         (kPlaneTask / 4)) + 8192 * (t - 4);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(8192u) : "memory");
+        }
+        // ---------------- pass 1: twiddle w512^(q k1), q = j + 4 Q + 16 h (= a), rows of stage 2 (k1, b = c)
+        {
+            C2 pw[4], st2[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 beta = w512[j + 4 * Q + 16 * hh];
+                pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
+                st2[j] = c2_splat(cmul(beta, beta));
+            }
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+            const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
+                                  uint32_t(lane & 7) * 16u;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float d[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const int k1 = 8 * half + 2 * pp;
+                    C2 v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[j] = cmul2(c2_at(d[j], pp), pw[j]);
+                        pw[j] = cmul2(pw[j], st2[j]);
+                    }
+                    sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64,
+                           pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
+                           pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+                    sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64,
+                           pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
+                           pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
+                }
+            }
+        }
+        // ---------------- stage 2 (over a); meanwhile this thread loads its spectrum values
+        stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+        {
+            // rows (k1 = 4 Q + lane / 8, b = 4 (lane & 7) + T), bins k2 = 16 h + 4 q4 + e; the
+            // product conj(X K~) goes to the stage-2' row 128 (k1 & 3) + 32 (k1 >> 2) + b,
+            // chunk k2 / 4 (the row order of tc16k's pass 2')
+            uint4 kv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) kv[i] = __ldg(kq + 32 * i);
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+#pragma unroll
+            for (int TH = 0; TH < 8; ++TH) {
+                const int T = TH >> 1;
+                float d[16];
+                tc::tmem_ld16(tl + uint32_t(64 * T + 32 * hh + 16 * (TH & 1)), d);
+                tc::tmem_ld_wait();
+                const int row = 128 * (lane >> 3) + 32 * Q + 4 * (lane & 7) + T;
+#pragma unroll
+                for (int q4 = 2 * (TH & 1); q4 < 2 * (TH & 1) + 2; ++q4) {
+                    const uint4 kk = kv[4 * T + q4];
+                    const C2 K0{make_float2(bf_lo(kk.x), bf_lo(kk.y)), make_float2(bf_hi(kk.x), bf_hi(kk.y))};
+                    const C2 K1{make_float2(bf_lo(kk.z), bf_lo(kk.w)), make_float2(bf_hi(kk.z), bf_hi(kk.w))};
+                    const C2 v0 = cmul2(c2_at(d, 2 * (q4 & 1)), K0);
+                    const C2 v1 = cmul2(c2_at(d, 2 * (q4 & 1) + 1), K1);
+                    sts128(A, tc::chunk_off(row, 4 * hh + q4, kSBO64), pack_bf16(v0.re.x, -v0.im.x),
+                           pack_bf16(v0.re.y, -v0.im.y), pack_bf16(v1.re.x, -v1.im.x), pack_bf16(v1.re.y, -v1.im.y));
+                }
+            }
+        }
+        // ---------------- stage 2' (inverse, on conj)
+        stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+        {
+            // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w512^(q k1)
+            // -> stage-1' row b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
+            const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
+                                  uint32_t(lane & 7) * 16u;
+            C2 pw[4], st2[4];
+#pragma unroll
+            for (int T = 0; T < 4; ++T) {
+                const int k1 = 4 * Q + T;
+                const float2 p0 = w512[(16 * hh * k1) & 511];
+                pw[T] = c2_of(p0, cmul(p0, w512[k1]));
+                st2[T] = c2_splat(w512[(2 * k1) & 511]);
+            }
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+#pragma unroll 1
+            for (int gq = 0; gq < 4; ++gq) {
+                float d[4][8];
+#pragma unroll
+                for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int ip = 0; ip < 2; ++ip) {
+                    C2 v[4];
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) {
+                        v[T] = cmul2(c2_at(d[T], ip), pw[T]);
+                        pw[T] = cmul2(pw[T], st2[T]);
+                    }
+                    const int i = 2 * ip;
+                    sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
+                           pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x),
+                           pack_bf16(v[3].re.x, v[3].im.x));
+                    sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
+                           pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y),
+                           pack_bf16(v[3].re.y, v[3].im.y));
+                }
+            }
+        }
+        // ---------------- stage 1': 8 tiles x (K 32 -> N 16), outputs s < 8 only
+        stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // result conj(D1') at row a_tc = c + 32 a, output s -> Vs[c][a + 32 s], then the
+        // task's 32 columns (contiguous in the workspace) in 16-byte stores
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int atc = 128 * (4 * hh + j) + 32 * Q + lane;
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
+            tc::tmem_ld_wait();
+            const int cc = atc & 31, aa = atc >> 5;
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+                // a warp's lanes are 32 columns (1 KB apart): word p of column cc sits at
+                // p ^ cc, so that they fall in 32 different banks
+                const int col = 4 * (s8 >> 1) + (s8 & 1);                 // re at col, im at col + 2
+                Vs[cc * MH + ((aa + 32 * s8) ^ cc)] = ok ? pack_bf16(d[col], -d[col + 2]) : 0x7fc07fc0u;
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        {
+            // 16-byte group g of column cc (words 4g .. 4g+3) is group g ^ (cc >> 2) with its
+            // words permuted by cc & 3; cc is the same for the 32 lanes of a warp
+            uint4* dst = reinterpret_cast<uint4*>(col0);
+#pragma unroll
+            for (int k = 0; k < NCOL * MH / 4 / NT; ++k) {
+                const int gi = t + NT * k, cc = gi >> 6, g = gi & 63;
+                uint4 v = *reinterpret_cast<const uint4*>(Vs + cc * MH + 4 * (g ^ (cc >> 2)));
+                if (cc & 1) v = make_uint4(v.y, v.x, v.w, v.z);
+                if (cc & 2) v = make_uint4(v.z, v.w, v.x, v.y);
+                dst[gi] = v;
+            }
+        }
+        if (__syncthreads_or(!ok)) {                    // a tensor-core wait ran out (uniform decision)
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+bool cols_2d_tc_path(const Plan& p, const ConvArgs& a) {
+    return p.path == PATH_GRID_2D && p.H == kTc2dH && p.W % NCOL == 0 && a.g2_plane_off != 0 &&
+           a.dtype == DT_BF16 && !a.fp32_transform;
+}
+
+cudaError_t launch_spectrum_2d_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
+                                        cudaStream_t s) {
+    const int64_t n = nrows * int64_t(p.W / NCOL) * (kPlaneTask / 4);
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_2d_plane_tc<<<unsigned(blocks), 256, 0, s>>>(reinterpret_cast<const float2*>(spectrum_rows),
+                                                   reinterpret_cast<uint4*>(plane), nrows, int(p.W),
+                                                   int64_t(p.spec_row_bytes / sizeof(float2)));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cols_2d_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg, int step,
+                              int64_t ws_img_stride, cudaStream_t s) {
+    auto kern = k_2d_cols_tc;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t ntasks = nimg * (p.W / NCOL);
+    if (ntasks > INT32_MAX || nimg > INT32_MAX) return cudaErrorInvalidValue;
+    int64_t grid = int64_t(2) * sms;
+    if (grid > ntasks) grid = ntasks;
+    kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<__nv_bfloat162*>(ws), a.spectrum, int(p.C), int(p.W), a.B, step,
+                                           img0, int(nimg), ws_img_stride, int64_t(a.g2_plane_off), a.spec_C,
+                                           a.spec_per_b, a.wait_budget_ns, a.issue_mma, a.status);
+    return cudaGetLastError();
+}
+
+}  // namespace hyena

@@ -67,9 +67,12 @@ struct ConvArgs {
     int64_t spec_per_b = 0;
     // kernel status word of this device (kStatus* bits)
     uint32_t* status = nullptr;
-    // L = 8192 with bf16 storage: run the fp32 CUDA-core transform instead of
-    // the tensor-core one (HYENA_FLAG_FP32_TRANSFORM)
+    // bf16 storage: run the fp32 CUDA-core transforms instead of the
+    // tensor-core ones (HYENA_FLAG_FP32_TRANSFORM)
     bool fp32_transform = false;
+    // 2-D, H = 256: offset of the tensor-core column pass's spectrum plane in
+    // this spectrum (from the plan of its own filter count: C, or B*C per sample)
+    size_t g2_plane_off = 0;
 };
 
 cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStream_t s);
@@ -86,6 +89,13 @@ cudaError_t launch_spectrum_cluster(const Plan& p, const SpectrumArgs& a, cudaSt
 bool cluster_path(const Plan& p, const ConvArgs& a);
 cudaError_t launch_conv_cluster(const Plan& p, const ConvArgs& a, size_t workspace_bytes, cudaStream_t s);
 cudaError_t launch_spectrum_2d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
+// 2-D with bf16 storage and H = 256 (grid2d_tc.cu): the column pass of columns
+// 0 .. W-1 on the tensor cores, and its spectrum plane from the complex64 rows.
+bool cols_2d_tc_path(const Plan& p, const ConvArgs& a);
+cudaError_t launch_cols_2d_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg, int step,
+                              int64_t ws_img_stride, cudaStream_t s);
+cudaError_t launch_spectrum_2d_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
+                                        cudaStream_t s);
 cudaError_t launch_conv_2d(const Plan& p, const ConvArgs& a, cudaStream_t s);
 cudaError_t launch_spectrum_3d(const Plan& p, const SpectrumArgs& a, cudaStream_t s);
 cudaError_t launch_conv_3d(const Plan& p, const ConvArgs& a, cudaStream_t s);

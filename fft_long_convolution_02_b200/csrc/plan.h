@@ -54,7 +54,7 @@ enum Path {
 constexpr int kCircularFlag = 0x100;
 
 constexpr uint32_t kSpecMagic = 0x4853504Eu;  // "NPSH"
-constexpr uint32_t kSpecVersion = 1;
+constexpr uint32_t kSpecVersion = 2;
 constexpr size_t kHeaderBytes = 256;
 constexpr int kMaxTableSpecs = 24;
 
@@ -62,6 +62,9 @@ constexpr int64_t kOnchipMaxL = 16384;
 // L served by the cluster kernel (bf16 storage): 2L = kClusterR x 16384
 constexpr int64_t kClusterL = 65536;
 constexpr int kClusterR = 8;
+// 2-D column length served by the tensor-core column pass (bf16 storage): a
+// 2H = 512-point transform per column, 32 columns per 16384-point task
+constexpr int64_t kTc2dH = 256;
 constexpr int64_t kMaxL = int64_t(1) << 20;
 constexpr int64_t kMin1D = 16;
 constexpr int64_t kMin2D = 16;
@@ -104,6 +107,10 @@ struct Plan {
     // even / odd powers w_16384^(2j), w_16384^(2j+1) (j < 2048)
     int64_t t_cl_fft = 0, t_cl_wa = 0, t_cl_even = 0, t_cl_odd = 0;
     size_t cl_plane_off = 0;               // 0: no cluster plane
+    // 2-D form with H = 256 and W a multiple of 32: the tensor-core column
+    // pass's spectrum plane (bf16 (re, im), per filter W/32 groups of 32
+    // columns x 512 bins in its thread order); 0: none
+    size_t g2_plane_off = 0;
     TableSpecs specs{};
     size_t tables_off = kHeaderBytes;
     size_t spec_off = 0;

@@ -53,6 +53,7 @@ cudaError_t launch_header_and_tables(const Plan& p, uint8_t* spectrum, cudaStrea
     h.spec_row_bytes = int64_t(p.spec_row_bytes);
     h.total_bytes = int64_t(p.total_bytes);
     h.reserved[0] = int64_t(p.cl_plane_off);
+    h.reserved[1] = int64_t(p.g2_plane_off);
     k_write_header<<<1, 32, 0, s>>>(reinterpret_cast<SpecHeader*>(spectrum), h);
     if (p.specs.total > 0) {
         int blocks = int((p.specs.total + 255) / 256);

@@ -1,0 +1,112 @@
+"""GPU parity: the tensor-core column pass of the 2-D form (grid2d_tc.cu: bf16
+storage, H = 256, columns 0 .. W-1 as 512-point transforms on tcgen05, the
+last bin column on the register engine), against the float64 oracle through
+the C ABI, and against the fp32 register-engine column pass the same shapes
+take with HYENA_FLAG_FP32_TRANSFORM."""
+import numpy as np
+import pytest
+
+from fft_long_convolution_02_b200 import binding as hb
+from fft_long_convolution_02_b200 import inputs as I
+from gpu_helpers import TOL, Run, api_shape, from_torch, oracle_for_rows, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fft_long_convolution_02_b200 import build
+    build.build()
+
+
+def _conv(p, r, flags=0, y=None):
+    import torch
+    hb.hyena_gated_fftconv_ex(r.u, r.y if y is None else y, r.spectrum, r.sc_w, r.sc_b, p.B, p.C, api_shape(p),
+                              p.order, r.workspace, flags=flags)
+    torch.cuda.synchronize()
+    hb.hyena_kernel_status()
+    return from_torch(r.y if y is None else y)
+
+
+def _rows_err(orc, p, data, y):
+    rows = np.arange(p.B * p.C)
+    ref = oracle_for_rows(orc, p, rows, data, method=2).reshape(len(rows), -1)
+    return row_rel_err(y.reshape(len(rows), -1), ref)
+
+
+@pytest.mark.parametrize("W,order,B,C", [(256, 2, 2, 3), (32, 2, 3, 2), (64, 3, 2, 2), (512, 2, 1, 2)])
+def test_tc_columns_against_oracle(orc, W, order, B, C):
+    """Widths of 1, 2, 8 and 16 column groups, orders 2 and 3, odd batch."""
+    p = I.WORKLOADS["grid2d"].with_(B=B, C=C, H=256, W=W, order=order, sigma=(4.0, 64.0), seed=3000 + W + order)
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    y = _conv(p, r)
+    assert np.isfinite(y).all()
+    err = _rows_err(orc, p, data, y)
+    print(f"W={W} order={order}: max image rel err {err.max():.3e}")
+    assert err.max() <= TOL["bf16"], err.max()
+
+
+def test_tc_columns_against_fp32_columns(orc):
+    """The fp32 register column pass (flag) and the tensor-core one agree within
+    the bf16 tolerance, the fp32 one is the closer to the oracle, and they are
+    not the same kernel's output."""
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=4, H=256, W=128, seed=3100)
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    y_tc = _conv(p, r).copy()
+    y_32 = _conv(p, r, flags=hb.HYENA_FLAG_FP32_TRANSFORM)
+    e_tc = _rows_err(orc, p, data, y_tc).max()
+    e_32 = _rows_err(orc, p, data, y_32).max()
+    print(f"tensor-core columns {e_tc:.3e}, fp32 columns {e_32:.3e}")
+    assert e_tc <= TOL["bf16"] and e_32 <= TOL["bf16"]
+    assert e_32 < e_tc
+    assert not np.array_equal(y_tc, y_32)
+
+
+def test_tc_columns_deterministic():
+    import torch
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=64, seed=3200)
+    r = Run(p, I.make_all(p))
+    r.build_spectrum()
+    _conv(p, r)
+    a = r.y.clone()
+    _conv(p, r)
+    assert torch.equal(a, r.y)
+
+
+def test_tc_columns_per_sample(orc):
+    """Per-sample filters: the plane rows follow the spectrum rows (b, c)."""
+    import torch
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=64, per_sample=True, seed=3300)
+    data = I.make_all(p)
+    r = Run(p, data)
+    spec = torch.empty(hb.hyena_spectrum_bytes(p.B * p.C, api_shape(p), p.order), dtype=torch.uint8, device="cuda")
+    hb.hyena_filter_spectrum(r.k, r.D, p.B * p.C, api_shape(p), p.order, spec)
+    hb.hyena_gated_fftconv_per_sample(r.u, r.y, spec, None, None, p.B, p.C, api_shape(p), p.order, r.workspace)
+    torch.cuda.synchronize()
+    hb.hyena_kernel_status()
+    err = _rows_err(orc, p, data, from_torch(r.y))
+    assert err.max() <= TOL["bf16"], err.max()
+
+
+def test_tc_columns_report_a_spectrum_header_mismatch():
+    """A spectrum that was never filled: the tensor-core column kernel writes
+    nothing and the status word reports HYENA_ERR_SPECTRUM_MISMATCH."""
+    import torch
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=64, seed=3400)
+    r = Run(p, I.make_all(p))
+    hb.hyena_kernel_status()
+    fresh = torch.zeros_like(r.spectrum)
+    hb.hyena_gated_fftconv(r.u, r.y, fresh, None, None, p.B, p.C, api_shape(p), p.order, r.workspace)
+    with pytest.raises(hb.HyenaError) as e:
+        hb.hyena_kernel_status()
+    assert e.value.status == 4
+    r.build_spectrum()
+    _conv(p, r)
+    assert np.isfinite(from_torch(r.y)).all()
