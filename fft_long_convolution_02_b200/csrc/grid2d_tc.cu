@@ -46,12 +46,18 @@ static_assert(NCOL * MH * 2 == N, "a task is one 16384-point transform");
 constexpr uint32_t kB1bytes = 4 * kSBO16;   // N 32 x K 16
 constexpr uint32_t kB1ibytes = 2 * kSBO32;  // N 16 x K 32
 constexpr uint32_t kOffA1 = kAbytes - 128 * kSBO16;   // stage-1 operand (1024 rows x K 16)
-constexpr uint32_t kOffB1 = kAbytes;
+// the stage-2' operand's 8-row groups 1168 bytes apart instead of 1152: the
+// spectrum pass writes rows 128 (k1 & 3) + 32 (k1 >> 2) + b, whose 16-byte
+// stores then spread over all eight bank groups
+constexpr uint32_t kSBO64s = kSBO64 + 16;
+constexpr uint32_t kAbytesC = 64 * kSBO64s > kAbytes ? 64 * kSBO64s : kAbytes;
+constexpr uint32_t kOffB1 = kAbytesC;
 constexpr uint32_t kOffB32 = kOffB1 + kB1bytes;
 constexpr uint32_t kOffB1i = kOffB32 + kB32bytes;
 constexpr uint32_t kOffW512 = kOffB1i + kB1ibytes;
 constexpr size_t kSmem = size_t(kOffW512) + 512 * sizeof(float2);
 static_assert(NCOL * MH * 4 <= kOffA1, "output staging must not overlap the stage-1 operand");
+static_assert(kOffA1 + 128 * kSBO16 <= kAbytesC, "stage-1 operand inside the operand area");
 static_assert(kOffW512 % 16 == 0, "twiddle table alignment");
 constexpr int kPlaneTask = N;     // bf16 (re, im) entries of the spectrum plane per task
 
@@ -146,6 +152,21 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     const int groups = W / NCOL;
     const int ntasks = nimg * groups;
 
+    // stage-1 inputs of a task: thread t takes rows a_tc = a0 + i (a0 = 8 (t & 127)) at
+    // slots s = 4 (t >> 7) + j, i.e. x[c][a + 32 s] with c = a_tc & 31, a = a_tc >> 5
+    auto load_build = [&](int tk, uint32_t (&xb)[8][4]) {
+        const int li = tk / groups, cg = tk - li * groups;
+        const uint32_t* cb = reinterpret_cast<const uint32_t*>(ws + int64_t(li) * ws_img_stride) +
+                             int64_t(NCOL * cg) * MH;
+        const int chalf = t >> 7, a0 = 8 * (t & 127);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int atc = a0 + i, cc = atc & 31, aa = atc >> 5;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xb[i][j] = cb[cc * MH + aa + 32 * (4 * chalf + j)];
+        }
+    };
+
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int li = task / groups, cg = task - li * groups;
         const int64_t img = img0 + li;
@@ -155,16 +176,11 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
                           (Q * 2 + hh) * 16 * 32 + lane;
         // ---------------- stage-1 operand: rows a_tc = c + 32 a, slots s < 8 (x[c][a + 32 s])
         {
+            uint32_t x[8][4];
+            load_build(task, x);
             const int chalf = t >> 7, a0 = 8 * (t & 127);
             const int r0 = rho1(a0);
             const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
-            uint32_t x[8][4];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int atc = a0 + i, cc = atc & 31, aa = atc >> 5;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[i][j] = col0[cc * MH + aa + 32 * (4 * chalf + j)];
-            }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -244,13 +260,13 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
                     const C2 K1{make_float2(bf_lo(kk.z), bf_lo(kk.w)), make_float2(bf_hi(kk.z), bf_hi(kk.w))};
                     const C2 v0 = cmul2(c2_at(d, 2 * (q4 & 1)), K0);
                     const C2 v1 = cmul2(c2_at(d, 2 * (q4 & 1) + 1), K1);
-                    sts128(A, tc::chunk_off(row, 4 * hh + q4, kSBO64), pack_bf16(v0.re.x, -v0.im.x),
+                    sts128(A, tc::chunk_off(row, 4 * hh + q4, kSBO64s), pack_bf16(v0.re.x, -v0.im.x),
                            pack_bf16(v0.re.y, -v0.im.y), pack_bf16(v1.re.x, -v1.im.x), pack_bf16(v1.re.y, -v1.im.y));
                 }
             }
         }
         // ---------------- stage 2' (inverse, on conj)
-        stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+        stage_issue(a_addr, kSBO64s, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
         {
             // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w512^(q k1)
             // -> stage-1' row b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
