@@ -447,6 +447,19 @@ hyena_status_t hyena_debug_conv_cluster(const void* u, void* y, const void* spec
                                         void* workspace, size_t workspace_bytes, uint64_t wait_budget_ns,
                                         int issue_mma, void* stream);
 
+/*
+ * The same test hook for the 2-D tensor-core column pass (ndim = 2, H = 256, W
+ * a multiple of 32, bf16 storage, shared filters; sizes = {256, W}; no short
+ * conv; workspace as in hyena_gated_fftconv): the whole 2-D convolution runs,
+ * with the column pass's waits bounded by wait_budget_ns and, for
+ * issue_mma = 0, no tensor-core work issued.  A CTA whose wait ran out writes
+ * NaN columns and stops; the row passes then carry the NaN into y.  Other
+ * shapes return HYENA_ERR_UNSUPPORTED_SHAPE.
+ */
+hyena_status_t hyena_debug_conv_2d_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, int64_t B,
+                                      int64_t C, int64_t W, int order, void* workspace, size_t workspace_bytes,
+                                      uint64_t wait_budget_ns, int issue_mma, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -86,3 +86,33 @@ def test_cluster_wait_timeout_is_reported(orc):
     rows = np.arange(p.B * p.C)
     err = row_rel_err(gpu_rows(from_torch(r.y), p, rows), oracle_for_rows(orc, p, rows, data, method=2))
     assert err.max() <= TOL["bf16"], err.max()
+
+
+def test_2d_tc_column_wait_timeout_is_reported(orc):
+    """The 2-D tensor-core column pass (H = 256, bf16): with no tensor-core work
+    issued each CTA's first wait runs out; the launch completes, the timeout
+    is recorded, the NaN columns reach every output through the inverse row
+    pass, and the next normal call is correct."""
+    import torch
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=64, seed=5103)
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    hb.hyena_kernel_status()
+    spec_before = r.spectrum.clone()
+    y = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_2d_tc(r.u, y, r.spectrum, p.B, p.C, p.W, p.order, r.workspace, wait_budget_ns=1_000_000,
+                              issue_mma=False)
+    torch.cuda.synchronize()
+    with pytest.raises(hb.HyenaError) as ei:
+        hb.hyena_kernel_status()
+    assert ei.value.status == 8                                   # HYENA_ERR_TIMEOUT
+    assert torch.isnan(y.float()).all()
+    assert torch.equal(r.spectrum, spec_before)
+    r.conv()
+    torch.cuda.synchronize()
+    hb.hyena_kernel_status()
+    rows = np.arange(p.B * p.C)
+    ref = oracle_for_rows(orc, p, rows, data, use_shortconv=False, method=2).reshape(len(rows), -1)
+    err = row_rel_err(from_torch(r.y).reshape(len(rows), -1), ref)
+    assert err.max() <= TOL["bf16"], err.max()

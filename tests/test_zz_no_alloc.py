@@ -35,8 +35,8 @@ def _groups(p):
     """Groups of rows the fixed scratch is cut into for problem p."""
     row = hb.hyena_gated_fftconv_workspace_min_bytes(p.C, p.shape, p.order)
     per_group = SCRATCH // row
-    if p.ndim == 1 and p.dtype == "bf16":
-        per_group *= 2          # the four-step workspace holds bf16 pairs with bf16 storage
+    if p.ndim in (1, 2) and p.dtype == "bf16":
+        per_group *= 2          # the four-step and 2-D workspaces hold bf16 pairs with bf16 storage
     return -(-p.B * p.C // per_group)
 
 
@@ -49,12 +49,15 @@ CASES = [
     I.WORKLOADS["vol3d"].with_(B=2, C=4, N1=64, H=128, W=128, seed=1203),
     # 2-D path, fp32: one group
     I.WORKLOADS["grid2d"].with_(B=2, C=5, H=64, W=128, dtype="f32", sigma=(4.0, 32.0), seed=1204),
+    # 2-D path with the tensor-core column pass, bf16: 256 x 512 images (513 bin
+    # columns of 256 bf16 pairs, 0.5 MB of scratch each) -> 62 per group, 70 -> 2 groups
+    I.WORKLOADS["grid2d"].with_(B=2, C=35, H=256, W=512, seed=1207),
     # on-chip path (no scratch needed), bf16
     I.WORKLOADS["d768_l8k"].with_(C=16, seed=1205),
     # cluster path, bf16, order 3, L = 2^16: the scratch holds one 512 KB slice per cluster
     I.WORKLOADS["order3"].with_(B=3, C=7, L=1 << 16, seed=1206),
 ]
-EXPECTED_GROUPS = [3, 2, 8, 1, None, None]
+EXPECTED_GROUPS = [3, 2, 8, 1, 2, None, None]
 
 
 def test_cases_span_several_groups():
