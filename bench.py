@@ -131,7 +131,12 @@ def spectrum_row_bytes(p) -> int:
     if p.ndim == 3:
         return (p.W + 1) * 2 * p.H * 2 * p.N1 * 8
     if p.ndim == 2:
-        return (p.W // 2 + 1) * p.H * 8 if p.circular else (p.W + 1) * 2 * p.H * 8
+        if p.circular:
+            return (p.W // 2 + 1) * p.H * 8
+        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+            # tensor-core column pass: bf16 plane of bins 0..W-1, complex64 last column
+            return p.W * 2 * p.H * 4 + 2 * p.H * 8
+        return (p.W + 1) * 2 * p.H * 8
     if p.L == 8192:
         return 8 * p.L                      # one plane: bf16 2L bins, or fp32 position layout
     if p.L <= 16384:
@@ -300,6 +305,10 @@ def math_of(p, kernel: str) -> str:
         return ("2L-point transform split over 8-CTA clusters: 8-point DFTs, short conv, gates and twiddles fp32 "
                 "on the CUDA cores; 16384-point DFT stages per CTA on tcgen05 tensor cores with bf16 operands and "
                 "fp32 accumulation; exchanges as bf16 pairs; spectrum read as bf16 (re, im)")
+    if p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+        return ("row passes fp32 on the CUDA cores; column pass of bins 0..W-1 as 512-point DFT stages on tcgen05 "
+                "tensor cores (bf16 operands, fp32 accumulation, spectrum read as bf16 (re, im)), last bin column "
+                "fp32; intermediate kept as bf16 pairs in the workspace between passes")
     if p.dtype == "bf16" and (p.ndim > 1 or p.L > 16384):
         return "fp32 (intermediate kept as bf16 pairs in the workspace between passes)"
     return "fp32"
