@@ -885,6 +885,18 @@ cudaError_t conv_2d_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
                                                                               p.order, gnext, H, i0, stride);
         }
     };
+    if constexpr (sizeof(T) == 2) {
+        // the two images of a channel as one complex image (groups of whole pairs)
+        const int64_t Gp = G & ~int64_t(1);
+        if (Gp >= 2 && pairs_2d_tc_path(p, a)) {
+            for (int64_t i0 = 0; i0 < nimg; i0 += Gp) {
+                const int64_t g = nimg - i0 < Gp ? nimg - i0 : Gp;
+                const cudaError_t e = launch_conv_2d_pairs_tc(p, a, ws, i0, g, stride, s);
+                if (e != cudaSuccess) return e;
+            }
+            return cudaGetLastError();
+        }
+    }
     for (int64_t i0 = 0; i0 < nimg; i0 += G) {
         const int64_t g = nimg - i0 < G ? nimg - i0 : G;
         launch_rows_fwd(i0, g);

@@ -73,12 +73,15 @@ __device__ __forceinline__ void plane_entry(int idx4, int e, int& c, int& k) {
     k = k1 + 16 * (16 * h + 4 * q4 + e);
 }
 
-// The plane from the complex64 spectrum rows: per row (W/32 tasks) x 4096 uint4.
-// Bin k of column f sits in the row at f * 2H + (k & 1) * H + the register
-// engine's slot of position fft_bin_pos(k >> 1) (see the 2-D spectrum build).
+// The plane from the complex64 spectrum rows: per row 2W/32 column blocks x
+// 4096 uint4, columns f = 0 .. 2W-1 of the 2H x 2W transform.  Bin k of a
+// stored column f <= W sits in the row at f * 2H + (k & 1) * H + the register
+// engine's slot of position fft_bin_pos(k >> 1) (see the 2-D spectrum build);
+// the columns f > W follow from the symmetry of the transform of a real
+// filter, K~[k][f] = conj K~[-k mod 2H][2W - f].
 __global__ void k_2d_plane_tc(const float2* __restrict__ rows, uint4* __restrict__ plane, int64_t nrows, int W,
                               int64_t row_stride) {
-    const int64_t per_row = int64_t(W / NCOL) * (kPlaneTask / 4);
+    const int64_t per_row = int64_t(2 * W / NCOL) * (kPlaneTask / 4);
     for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < nrows * per_row;
          g += int64_t(gridDim.x) * blockDim.x) {
         const int64_t r = g / per_row;
@@ -90,10 +93,12 @@ __global__ void k_2d_plane_tc(const float2* __restrict__ rows, uint4* __restrict
             int c, k;
             plane_entry(idx4, e, c, k);
             const int f = NCOL * task + c;
-            const int pos = fft_bin_pos<MH>(k >> 1);
-            const float2 K = rows[r * row_stride + int64_t(f) * (2 * MH) + (k & 1) * MH + (pos & 15) * (MH / 16) +
+            const bool mirror = f > W;
+            const int fs = mirror ? 2 * W - f : f, ks = mirror ? (2 * MH - k) & (2 * MH - 1) : k;
+            const int pos = fft_bin_pos<MH>(ks >> 1);
+            const float2 K = rows[r * row_stride + int64_t(fs) * (2 * MH) + (ks & 1) * MH + (pos & 15) * (MH / 16) +
                                   (pos >> 4)];
-            v[e] = pack_bf16(K.x, K.y);
+            v[e] = pack_bf16(K.x, mirror ? -K.y : K.y);
         }
         plane[g] = make_uint4(v[0], v[1], v[2], v[3]);
     }
@@ -102,14 +107,14 @@ __global__ void k_2d_plane_tc(const float2* __restrict__ rows, uint4* __restrict
 __global__ void __launch_bounds__(NT, 2)
 k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum, int C, int W, int64_t B,
              int step, int64_t img0, int nimg, int64_t ws_img_stride, int64_t plane_off, int64_t SC, int64_t SB,
-             uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+             int hdr_W, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_2t[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     // the header is requested first and checked once the tables are set up
     const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
     const SpecHeader hv = *h;
-    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W) &
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == hdr_W) &
                         (hv.reserved[1] == plane_off);
     uint8_t* A = smem_2t;
     uint8_t* A1 = smem_2t + kOffA1;
@@ -149,7 +154,8 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     const uint4* plane = reinterpret_cast<const uint4*>(spectrum + plane_off);
     uint32_t phase = 0;
     bool ok = true;
-    const int groups = W / NCOL;
+    const int groups = W / NCOL;                  // column blocks of an image (its first W columns)
+    const int pgroups = 2 * hdr_W / NCOL;         // column blocks of a plane row
     const int ntasks = nimg * groups;
 
     // stage-1 inputs of a task: thread t takes rows a_tc = a0 + i (a0 = 8 (t & 127)) at
@@ -172,7 +178,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
         const int64_t img = img0 + li;
         uint32_t* col0 = reinterpret_cast<uint32_t*>(ws + int64_t(li) * ws_img_stride) + int64_t(NCOL * cg) * MH;
         const int64_t c = img / B, b = img - c * B;
-        const uint4* kq = plane + ((int64_t(step) * SC + b * SB + c) * groups + cg) * (kPlaneTask / 4) +
+        const uint4* kq = plane + ((int64_t(step) * SC + b * SB + c) * pgroups + cg) * (kPlaneTask / 4) +
                           (Q * 2 + hh) * 16 * 32 + lane;
         // ---------------- stage-1 operand: rows a_tc = c + 32 a, slots s < 8 (x[c][a + 32 s])
         {
@@ -196,7 +202,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
             const uint8_t* src = t < 4 ? reinterpret_cast<const uint8_t*>(reinterpret_cast<const uint32_t*>(
                                              ws + int64_t(nli) * ws_img_stride) + int64_t(NCOL * ncg) * MH) + 8192 * t
                                        : reinterpret_cast<const uint8_t*>(
-                                             plane + ((int64_t(step) * SC + nb * SB + nc) * groups + ncg) *
+                                             plane + ((int64_t(step) * SC + nb * SB + nc) * pgroups + ncg) *
                                                          (kPlaneTask / 4)) + 8192 * (t - 4);
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(8192u) : "memory");
         }
@@ -350,6 +356,391 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+
+// ---------------------------------------------------------------------------
+// Paired images: the two images (b0, b0 + 1) of a channel share the real
+// filter, so they travel as one complex image z = g[b0] + i g[b0 + 1] (g the
+// gated input), and every pass is a plain 512-point complex transform with
+// 256 non-zero inputs: rows forward (here), the column kernel above over all
+// 2W = 512 bin columns, rows inverse with the output gate (below).  The
+// workspace of a pair holds Z[k][row] (k < 512 bins, 256 rows, bf16 pairs).
+// With the unnormalised transforms both ways the spectrum must be
+// (DFT(k) + D) / (4HW), twice the stored (DFT(k) + D) / (8HW), whose other
+// factor two belongs to the packed-real row passes of the unpaired path.
+// ---------------------------------------------------------------------------
+
+constexpr int W2 = 256;           // image width of the paired path (row transform 512)
+constexpr int NROW = 32;          // image rows per task
+
+// z of rows r0 .. r0+31 of a pair -> staging Zs[r][n ^ (8 (r >> 3))] (bf16 pairs):
+// the XOR lets the stage-1 gather below read 32 different banks.
+__device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __restrict__ x_b0, const bf16* __restrict__ x_b1,
+                                                const bf16* __restrict__ v_b0, const bf16* __restrict__ v_b1, int t) {
+#pragma unroll
+    for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
+        const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
+        const int64_t off = int64_t(r) * W2 + n0;
+        const uint4 xa = __ldg(reinterpret_cast<const uint4*>(x_b0 + off));
+        const uint4 xb = __ldg(reinterpret_cast<const uint4*>(x_b1 + off));
+        const uint4 va = __ldg(reinterpret_cast<const uint4*>(v_b0 + off));
+        const uint4 vb = __ldg(reinterpret_cast<const uint4*>(v_b1 + off));
+        const uint32_t xw[2][4] = {{xa.x, xa.y, xa.z, xa.w}, {xb.x, xb.y, xb.z, xb.w}};
+        const uint32_t vw[2][4] = {{va.x, va.y, va.z, va.w}, {vb.x, vb.y, vb.z, vb.w}};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            // samples 2q, 2q+1 of both images: (g[b0], g[b1]) at each
+            const float2 lo = __fmul2_rn(make_float2(bf_lo(xw[0][q]), bf_lo(xw[1][q])),
+                                         make_float2(bf_lo(vw[0][q]), bf_lo(vw[1][q])));
+            const float2 hi = __fmul2_rn(make_float2(bf_hi(xw[0][q]), bf_hi(xw[1][q])),
+                                         make_float2(bf_hi(vw[0][q]), bf_hi(vw[1][q])));
+            o[2 * q] = pack_bf16(lo.x, lo.y);
+            o[2 * q + 1] = pack_bf16(hi.x, hi.y);
+        }
+        uint32_t* dst = Zs + r * W2 + (n0 ^ (8 * (r >> 3)));
+        *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dst + 4) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum,
+                 int64_t B, int64_t C, int order, int64_t pair0, int npairs, int64_t ws_pair_stride,
+                 uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_rf[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    const SpecHeader hv = *h;
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
+    uint8_t* A = smem_rf;
+    uint8_t* A1 = smem_rf + kOffA1;
+    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_rf);     // gated rows, then the output staging
+    float2* w512 = reinterpret_cast<float2*>(smem_rf + kOffW512);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    float2* w32 = reinterpret_cast<float2*>(smem_rf);
+    fill_w32(w32);
+    for (int e = t; e < 512; e += NT) {
+        float sv, cv;
+        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);
+        w512[e] = make_float2(cv, -sv);
+    }
+    __syncthreads();
+    fill_dft<16, 16, 8, kSBO16>(smem_rf + kOffB1, w32);
+    fill_dft<32, 32, 32, kSBO64>(smem_rf + kOffB32, w32);
+    if (!hdr_ok) {
+        if (t == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
+    if (t == 0) tc::mbar_init(&mbar, 1);
+    if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t a1_addr = tc::smem_u32(A1);
+    const uint32_t b1_addr = tc::smem_u32(smem_rf + kOffB1);
+    const uint32_t b32_addr = tc::smem_u32(smem_rf + kOffB32);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(MH) * W2;
+    const int ntasks = npairs * (MH / NROW);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (MH / NROW), rg = task - lp * (MH / NROW);
+        const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
+        const int64_t rowoff = int64_t(NROW * rg) * W2;
+        const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
+        const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
+        stage_pair_rows(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
+        __syncthreads();
+        // ---------------- stage-1 operand: rows a_tc = r + 32 a, slots s < 8 (z[r][a + 32 s])
+        {
+            const int chalf = t >> 7, a0 = 8 * (t & 127);
+            const int r0 = rho1(a0);
+            const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int atc = a0 + i, r = atc & 31, aa = atc >> 5;
+                uint32_t x[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) x[j] = Zs[r * W2 + ((aa + 32 * (4 * chalf + j)) ^ (8 * (r >> 3)))];
+#pragma unroll
+                for (int jp = 0; jp < 4; jp += 2)
+                    *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u +
+                                              4u * jp) = make_uint2(x[jp], x[jp + 1]);
+            }
+        }
+        stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
+        // ---------------- pass 1: twiddle w512^(q k1), rows of stage 2 (k1, b = r)
+        {
+            C2 pw[4], st2[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 beta = w512[j + 4 * Q + 16 * hh];
+                pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
+                st2[j] = c2_splat(cmul(beta, beta));
+            }
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+            const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
+                                  uint32_t(lane & 7) * 16u;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float d[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const int k1 = 8 * half + 2 * pp;
+                    C2 v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[j] = cmul2(c2_at(d[j], pp), pw[j]);
+                        pw[j] = cmul2(pw[j], st2[j]);
+                    }
+                    sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64,
+                           pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
+                           pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+                    sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64,
+                           pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
+                           pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
+                }
+            }
+        }
+        // ---------------- stage 2 (over a): Z[k1 + 16 k2] of row r
+        stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // rows (k1 = 4 Q + lane / 8, r = 4 (lane & 7) + T), bins k2 = 16 h + ..: staging
+        // Os[k][r ^ (k & 3)] (the 32 lanes of a store hit 32 banks), then 128-byte rows
+        // Z[k][32 rg .. 32 rg + 31] of the workspace
+        {
+            uint32_t* Os = reinterpret_cast<uint32_t*>(smem_rf);
+            const int k1 = 4 * Q + (lane >> 3);
+#pragma unroll
+            for (int TH = 0; TH < 8; ++TH) {
+                const int T = TH >> 1;
+                float d[16];
+                tc::tmem_ld16(tl + uint32_t(64 * T + 32 * hh + 16 * (TH & 1)), d);
+                tc::tmem_ld_wait();
+                const int r = 4 * (lane & 7) + T;
+#pragma unroll
+                for (int pcol = 0; pcol < 4; ++pcol) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int k2 = 16 * hh + 8 * (TH & 1) + 2 * pcol + e;
+                        const int k = k1 + 16 * k2;
+                        Os[k * NROW + (r ^ (k & 3))] = ok ? pack_bf16(d[4 * pcol + e], d[4 * pcol + 2 + e]) : 0x7fc07fc0u;
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            __syncthreads();
+            uint32_t* wsp = reinterpret_cast<uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg;
+#pragma unroll 4
+            for (int kk = 0; kk < 512 * NROW / 4 / NT; ++kk) {
+                const int gi = t + NT * kk, k = gi >> 3, g4 = gi & 7;
+                uint4 v = *reinterpret_cast<const uint4*>(Os + k * NROW + 4 * g4);
+                const int m = k & 3;                  // word r sits at r ^ m inside its group of 4
+                if (m & 1) v = make_uint4(v.y, v.x, v.w, v.z);
+                if (m & 2) v = make_uint4(v.z, v.w, v.x, v.y);
+                *reinterpret_cast<uint4*>(wsp + int64_t(k) * MH + 4 * g4) = v;
+            }
+        }
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bfloat162* __restrict__ ws,
+                 const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
+                 int64_t ws_pair_stride, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_ri[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
+    const SpecHeader hv = *h;
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
+    uint8_t* A = smem_ri;
+    uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ri);      // output staging [r][n ^ r]
+    float2* w512 = reinterpret_cast<float2*>(smem_ri + kOffW512);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    float2* w32 = reinterpret_cast<float2*>(smem_ri);
+    fill_w32(w32);
+    for (int e = t; e < 512; e += NT) {
+        float sv, cv;
+        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);
+        w512[e] = make_float2(cv, -sv);
+    }
+    __syncthreads();
+    fill_dft<32, 32, 32, kSBO64>(smem_ri + kOffB32, w32);
+    fill_dft<16, 8, 16, kSBO32>(smem_ri + kOffB1i, w32);
+    if (!hdr_ok) {
+        if (t == 0) report_status(status, kStatusSpectrumMismatch);
+        return;
+    }
+    if (t == 0) tc::mbar_init(&mbar, 1);
+    if (warp == 0) tc::tmem_alloc(&tmem_base, kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t b32_addr = tc::smem_u32(smem_ri + kOffB32);
+    const uint32_t b1i_addr = tc::smem_u32(smem_ri + kOffB1i);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(MH) * W2;
+    const int ntasks = npairs * (MH / NROW);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (MH / NROW), rg = task - lp * (MH / NROW);
+        const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
+        // ---------------- stage-2' operand: conj Y[k1 + 16 k2][r] at row 128 (k1 & 3) +
+        // 32 (k1 >> 2) + r, chunk k2 / 4 (row groups kSBO64s apart); lane = r
+        {
+            const uint32_t* wsp = reinterpret_cast<const uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg + lane;
+#pragma unroll 2
+            for (int m = 0; m < 16; ++m) {
+                const int ci = warp + 8 * m, k1 = ci & 15, ch = ci >> 4;
+                uint32_t q[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) q[e] = wsp[int64_t(k1 + 16 * (4 * ch + e)) * MH] ^ 0x80000000u;
+                const int row = 128 * (k1 & 3) + 32 * (k1 >> 2) + lane;
+                sts128(A, tc::chunk_off(row, ch, kSBO64s), q[0], q[1], q[2], q[3]);
+            }
+        }
+        stage_issue(a_addr, kSBO64s, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
+        // ---------------- pass 2' (twiddle w512^(q k1)) -> stage-1' rows r + 32 q
+        {
+            const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
+                                  uint32_t(lane & 7) * 16u;
+            C2 pw[4], st2[4];
+#pragma unroll
+            for (int T = 0; T < 4; ++T) {
+                const int k1 = 4 * Q + T;
+                const float2 p0 = w512[(16 * hh * k1) & 511];
+                pw[T] = c2_of(p0, cmul(p0, w512[k1]));
+                st2[T] = c2_splat(w512[(2 * k1) & 511]);
+            }
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+#pragma unroll 1
+            for (int gq = 0; gq < 4; ++gq) {
+                float d[4][8];
+#pragma unroll
+                for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int ip = 0; ip < 2; ++ip) {
+                    C2 v[4];
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) {
+                        v[T] = cmul2(c2_at(d[T], ip), pw[T]);
+                        pw[T] = cmul2(pw[T], st2[T]);
+                    }
+                    const int i = 2 * ip;
+                    sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
+                           pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x),
+                           pack_bf16(v[3].re.x, v[3].im.x));
+                    sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
+                           pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y),
+                           pack_bf16(v[3].re.y, v[3].im.y));
+                }
+            }
+        }
+        // ---------------- stage 1': outputs s < 8 (n = a + 32 s < 256)
+        stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // 2 conj(D1') at row a_tc = r + 32 a, output s: (image b0, image b1) of row r,
+        // column n = a + 32 s -> Ys[r][n ^ r]
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int atc = 128 * (4 * hh + j) + 32 * Q + lane;
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(16 * (4 * hh + j)), d);
+            tc::tmem_ld_wait();
+            const int r = atc & 31, aa = atc >> 5;
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+                const int col = 4 * (s8 >> 1) + (s8 & 1);
+                Ys[r * W2 + ((aa + 32 * s8) ^ r)] = pack_bf16(2.0f * d[col], -2.0f * d[col + 2]);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        // output gate: y = x0 * conv for both images, 8 columns of a row per step
+        {
+            const int64_t rowoff = int64_t(NROW * rg) * W2;
+            const bf16* xa = u + (b0 * Ctot + c) * n_img + rowoff;
+            const bf16* xb = xa + Ctot * n_img;
+            bf16* ya = y + (b0 * C + c) * n_img + rowoff;
+            bf16* yb = ya + C * n_img;
+#pragma unroll
+            for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
+                const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
+                const int64_t off = int64_t(r) * W2 + n0;
+                const uint4 x0a = __ldg(reinterpret_cast<const uint4*>(xa + off));
+                const uint4 x0b = __ldg(reinterpret_cast<const uint4*>(xb + off));
+                // word n0 + i sits at (n0 ^ (r & 24)) + (i ^ (r & 7))
+                const uint32_t* src = Ys + r * W2 + (n0 ^ (r & 24));
+                const uint4 g0 = *reinterpret_cast<const uint4*>(src);
+                const uint4 g1 = *reinterpret_cast<const uint4*>(src + 4);
+                uint32_t w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const int m = r & 7;
+                if (m & 1) {
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2) { const uint32_t tmp = w[i]; w[i] = w[i + 1]; w[i + 1] = tmp; }
+                }
+                if (m & 2) {
+#pragma unroll
+                    for (int i = 0; i < 8; i += 4) {
+                        uint32_t tmp = w[i]; w[i] = w[i + 2]; w[i + 2] = tmp;
+                        tmp = w[i + 1]; w[i + 1] = w[i + 3]; w[i + 3] = tmp;
+                    }
+                }
+                if (m & 4) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) { const uint32_t tmp = w[i]; w[i] = w[i + 4]; w[i + 4] = tmp; }
+                }
+                const uint32_t xaw[4] = {x0a.x, x0a.y, x0a.z, x0a.w}, xbw[4] = {x0b.x, x0b.y, x0b.z, x0b.w};
+                uint32_t oa[4], ob[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 lo = __fmul2_rn(make_float2(bf_lo(xaw[q]), bf_lo(xbw[q])),
+                                                 make_float2(bf_lo(w[2 * q]), bf_hi(w[2 * q])));
+                    const float2 hi = __fmul2_rn(make_float2(bf_hi(xaw[q]), bf_hi(xbw[q])),
+                                                 make_float2(bf_lo(w[2 * q + 1]), bf_hi(w[2 * q + 1])));
+                    oa[q] = pack_bf16(lo.x, hi.x);
+                    ob[q] = pack_bf16(lo.y, hi.y);
+                }
+                const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
+                *reinterpret_cast<uint4*>(ya + off) = ok ? make_uint4(oa[0], oa[1], oa[2], oa[3]) : nan4;
+                *reinterpret_cast<uint4*>(yb + off) = ok ? make_uint4(ob[0], ob[1], ob[2], ob[3]) : nan4;
+            }
+        }
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
 }  // namespace
 
 bool cols_2d_tc_path(const Plan& p, const ConvArgs& a) {
@@ -359,7 +750,7 @@ bool cols_2d_tc_path(const Plan& p, const ConvArgs& a) {
 
 cudaError_t launch_spectrum_2d_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
                                         cudaStream_t s) {
-    const int64_t n = nrows * int64_t(p.W / NCOL) * (kPlaneTask / 4);
+    const int64_t n = nrows * int64_t(2 * p.W / NCOL) * (kPlaneTask / 4);
     int64_t blocks = (n + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
     k_2d_plane_tc<<<unsigned(blocks), 256, 0, s>>>(reinterpret_cast<const float2*>(spectrum_rows),
@@ -382,7 +773,39 @@ cudaError_t launch_cols_2d_tc(const Plan& p, const ConvArgs& a, void* ws, int64_
     if (grid > ntasks) grid = ntasks;
     kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<__nv_bfloat162*>(ws), a.spectrum, int(p.C), int(p.W), a.B, step,
                                            img0, int(nimg), ws_img_stride, int64_t(a.g2_plane_off), a.spec_C,
-                                           a.spec_per_b, a.wait_budget_ns, a.issue_mma, a.status);
+                                           a.spec_per_b, int(p.W), a.wait_budget_ns, a.issue_mma, a.status);
+    return cudaGetLastError();
+}
+
+bool pairs_2d_tc_path(const Plan& p, const ConvArgs& a) {
+    return cols_2d_tc_path(p, a) && p.W == W2 && p.order == 2 && a.B % 2 == 0 && a.spec_per_b == 0;
+}
+
+cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg,
+                                    int64_t ws_img_stride, cudaStream_t s) {
+    if (img0 % 2 != 0 || nimg % 2 != 0) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t npairs = nimg / 2, pair0 = img0 / 2, pstride = 2 * ws_img_stride;
+    const int64_t ntasks = npairs * (MH / NROW);
+    if (ntasks > INT32_MAX || npairs * (2 * W2 / NCOL) > INT32_MAX) return cudaErrorInvalidValue;
+    const unsigned grid = unsigned(ntasks < 2 * sms ? ntasks : 2 * sms);
+    const bf16* u = static_cast<const bf16*>(a.u);
+    __nv_bfloat162* w = static_cast<__nv_bfloat162*>(ws);
+    cudaError_t e = cudaFuncSetAttribute(k_2d_rows_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2d_cols_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2d_rows_inv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
+    if (e != cudaSuccess) return e;
+    k_2d_rows_fwd_tc<<<grid, NT, kSmem, s>>>(u, w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride,
+                                             a.wait_budget_ns, a.issue_mma, a.status);
+    // every bin column of a pair (2W), spectrum row c = pair / (B/2)
+    const int64_t ctasks = npairs * (2 * W2 / NCOL);
+    k_2d_cols_tc<<<unsigned(ctasks < 2 * sms ? ctasks : 2 * sms), NT, kSmem, s>>>(
+        w, a.spectrum, int(p.C), 2 * W2, a.B / 2, 0, pair0, int(npairs), pstride, int64_t(a.g2_plane_off), a.spec_C,
+        0, W2, a.wait_budget_ns, a.issue_mma, a.status);
+    k_2d_rows_inv_tc<<<grid, NT, kSmem, s>>>(u, static_cast<bf16*>(a.y), w, a.spectrum, a.B, p.C, p.order, pair0,
+                                             int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
     return cudaGetLastError();
 }
 

@@ -107,9 +107,10 @@ struct Plan {
     // even / odd powers w_16384^(2j), w_16384^(2j+1) (j < 2048)
     int64_t t_cl_fft = 0, t_cl_wa = 0, t_cl_even = 0, t_cl_odd = 0;
     size_t cl_plane_off = 0;               // 0: no cluster plane
-    // 2-D form with H = 256 and W a multiple of 32: the tensor-core column
-    // pass's spectrum plane (bf16 (re, im), per filter W/32 groups of 32
-    // columns x 512 bins in its thread order); 0: none
+    // 2-D form with H = 256 and W a multiple of 32: the tensor-core passes'
+    // spectrum plane (bf16 (re, im), per filter 2W/32 blocks of 32 columns
+    // x 512 bins of the 2H x 2W transform, in the column kernel's thread
+    // order); 0: none
     size_t g2_plane_off = 0;
     TableSpecs specs{};
     size_t tables_off = kHeaderBytes;

@@ -56,9 +56,9 @@ def test_spectrum_bytes_and_workspace(lib):
     assert 256 * 8 * L <= b < 256 * 8 * L + (64 << 20)
     assert lib.hyena_gated_fftconv_workspace_min_bytes(256, 1, _sz(L), 2) == 8 * L
     # 2-D: (W+1) * 2H complex64 per channel, and at H = 256 the tensor-core
-    # column pass's plane, W * 2H bf16 pairs per channel
+    # passes' plane, 2W * 2H bf16 pairs per channel
     b = lib.hyena_spectrum_bytes(256, 2, _sz(256, 256), 2)
-    assert 256 * (257 * 512 * 8 + 256 * 512 * 4) <= b < 256 * (257 * 512 * 8 + 256 * 512 * 4) + (1 << 20)
+    assert 256 * (257 * 512 * 8 + 512 * 512 * 4) <= b < 256 * (257 * 512 * 8 + 512 * 512 * 4) + (1 << 20)
     b = lib.hyena_spectrum_bytes(256, 2, _sz(128, 256), 2)
     assert 256 * 257 * 256 * 8 <= b < 256 * 257 * 256 * 8 + (1 << 20)
     # 2-D circular: (W/2+1) * H complex64 per channel; 1-D circular is refused

@@ -110,3 +110,50 @@ def test_tc_columns_report_a_spectrum_header_mismatch():
     r.build_spectrum()
     _conv(p, r)
     assert np.isfinite(from_torch(r.y)).all()
+
+
+@pytest.mark.parametrize("B,C,order", [(2, 3, 2), (4, 2, 2), (3, 2, 2), (2, 2, 3)])
+def test_paired_images_against_oracle(orc, B, C, order):
+    """256 x 256 images: with an even batch at order 2 the two images of a
+    channel travel as one complex image through tensor-core row, column and
+    row passes; an odd batch or order 3 takes the unpaired passes."""
+    p = I.WORKLOADS["grid2d"].with_(B=B, C=C, H=256, W=256, order=order, seed=3500 + 10 * B + order)
+    data = I.make_all(p)
+    r = Run(p, data)
+    r.build_spectrum()
+    y = _conv(p, r)
+    assert np.isfinite(y).all()
+    err = _rows_err(orc, p, data, y)
+    print(f"B={B} order={order}: max image rel err {err.max():.3e}")
+    assert err.max() <= TOL["bf16"], err.max()
+
+
+def test_paired_images_small_workspace(orc):
+    """Workspaces of one and of three images: pairs are never split (one image
+    of scratch falls back to the unpaired passes), results within the bound."""
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=3, H=256, W=256, seed=3600)
+    data = I.make_all(p)
+    row = hb.hyena_gated_fftconv_workspace_min_bytes(p.C, api_shape(p), p.order)
+    for nrows in (1, 3):
+        r = Run(p, data, workspace_bytes=nrows * row)
+        r.build_spectrum()
+        err = _rows_err(orc, p, data, _conv(p, r))
+        assert err.max() <= TOL["bf16"], (nrows, err.max())
+
+
+def test_paired_images_timeout_is_reported():
+    import torch
+    p = I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=256, seed=3700)
+    r = Run(p, I.make_all(p))
+    r.build_spectrum()
+    hb.hyena_kernel_status()
+    y = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_2d_tc(r.u, y, r.spectrum, p.B, p.C, p.W, p.order, r.workspace, wait_budget_ns=1_000_000,
+                              issue_mma=False)
+    torch.cuda.synchronize()
+    with pytest.raises(hb.HyenaError) as ei:
+        hb.hyena_kernel_status()
+    assert ei.value.status == 8
+    assert torch.isnan(y.float()).all()
+    _conv(p, r)
+    assert np.isfinite(from_torch(r.y)).all()
