@@ -48,6 +48,7 @@ CASES = [
     I.WORKLOADS["order3"].with_(B=3, C=2, L=1 << 16, seed=6006),                          # 8-CTA clusters, order 3
     I.WORKLOADS["grid2d"].with_(B=2, C=3, H=64, W=32, sigma=(4.0, 16.0), seed=6005),      # 2-D
     I.WORKLOADS["grid2d"].with_(B=3, C=2, H=256, W=64, seed=6009),                         # 2-D tensor-core columns
+    I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=256, seed=6010),                        # 2-D paired images
 ]
 
 

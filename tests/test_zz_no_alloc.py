@@ -52,12 +52,14 @@ CASES = [
     # 2-D path with the tensor-core column pass, bf16: 256 x 512 images (513 bin
     # columns of 256 bf16 pairs, 0.5 MB of scratch each) -> 62 per group, 70 -> 2 groups
     I.WORKLOADS["grid2d"].with_(B=2, C=35, H=256, W=512, seed=1207),
+    # 2-D paired images (256 x 256, order 2): 126 images per group, 140 -> 2 groups of whole pairs
+    I.WORKLOADS["grid2d"].with_(B=2, C=70, H=256, W=256, seed=1208),
     # on-chip path (no scratch needed), bf16
     I.WORKLOADS["d768_l8k"].with_(C=16, seed=1205),
     # cluster path, bf16, order 3, L = 2^16: the scratch holds one 512 KB slice per cluster
     I.WORKLOADS["order3"].with_(B=3, C=7, L=1 << 16, seed=1206),
 ]
-EXPECTED_GROUPS = [3, 2, 8, 1, 2, None, None]
+EXPECTED_GROUPS = [3, 2, 8, 1, 2, 2, None, None]
 
 
 def test_cases_span_several_groups():
