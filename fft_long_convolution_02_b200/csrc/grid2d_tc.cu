@@ -613,7 +613,9 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
         // 32 (k1 >> 2) + r, chunk k2 / 4 (row groups kSBO64s apart); lane = r
         {
             const uint32_t* wsp = reinterpret_cast<const uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg + lane;
-#pragma unroll 2
+            // all 64 loads of the thread in flight together (they wait on L2, not on
+            // each other)
+#pragma unroll
             for (int m = 0; m < 16; ++m) {
                 const int ci = warp + 8 * m, k1 = ci & 15, ch = ci >> 4;
                 uint32_t q[4];
