@@ -24,9 +24,9 @@
  *  - dtype selects the storage of u, y (and of k in hyena_filter_spectrum):
  *    HYENA_F32 or HYENA_BF16 (round-to-nearest-even on store).  Arithmetic:
  *    the short conv, the gates, the twiddles and the spectrum products are
- *    fp32 on every path.  With fp32 storage, and on every path other than
- *    1-D L = 8192 with bf16 storage, the transforms are fp32 too and the
- *    spectrum is read as complex64.  At L = 8192 with bf16 storage (order
+ *    fp32 on every path.  With fp32 storage, and on the bf16 paths not named
+ *    below, the transforms are fp32 too and the spectrum is read as
+ *    complex64.  At L = 8192 with bf16 storage (order
  *    <= 3, shared filters) the DFT stages run on the tensor cores: their
  *    operands and the DFT matrices are rounded to bf16 and accumulated in
  *    fp32, and the spectrum is read as bf16 (re, im) pairs (row error a few
@@ -37,9 +37,14 @@
  *    16384-point part on the tensor cores as at L = 8192, the exchanges
  *    between the CTAs and the spectrum as bf16 pairs (row error ~1e-2 at
  *    order 3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 multi-pass
- *    transform there.  With bf16 storage the intermediate of the other
- *    multi-pass (L >= 32768) and N-D paths is kept as bf16 pairs in the
- *    workspace.
+ *    transform there.  2-D with bf16 storage and H = 256 (W a multiple of
+ *    32): the column transforms (512 points) run on the tensor cores the same
+ *    way, with the spectrum read as bf16 pairs; for 256 x 256 images at order
+ *    2 with an even batch and shared filters the two images of a channel
+ *    travel as one complex image and the row transforms run there too (image
+ *    error a few 1e-3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 passes.
+ *    With bf16 storage the intermediate of the multi-pass (L >= 32768) and
+ *    N-D paths is kept as bf16 pairs in the workspace.
  *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
  *    stream) and is asynchronous: no call synchronises the host.
  *  - Arguments are validated before anything is enqueued; on any error
@@ -241,7 +246,8 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
 
 /* Flags of hyena_gated_fftconv_ex. */
 #define HYENA_FLAG_FP32_TRANSFORM 0x1u  /* every transform multiply in fp32 on the CUDA cores (no bf16 tensor-core
-                                           operands); changes only 1-D L = 8192 and 65536 with bf16 storage */
+                                           operands); changes only 1-D L = 8192 and 65536 and 2-D H = 256 with
+                                           bf16 storage */
 
 /*
  * hyena_gated_fftconv_ex -- hyena_gated_fftconv with flags (shared filters).
@@ -448,13 +454,13 @@ hyena_status_t hyena_debug_conv_cluster(const void* u, void* y, const void* spec
                                         int issue_mma, void* stream);
 
 /*
- * The same test hook for the 2-D tensor-core column pass (ndim = 2, H = 256, W
- * a multiple of 32, bf16 storage, shared filters; sizes = {256, W}; no short
+ * The same test hook for the 2-D tensor-core passes (ndim = 2, H = 256, W a
+ * multiple of 32, bf16 storage, shared filters; sizes = {256, W}; no short
  * conv; workspace as in hyena_gated_fftconv): the whole 2-D convolution runs,
- * with the column pass's waits bounded by wait_budget_ns and, for
+ * with the tensor-core kernels' waits bounded by wait_budget_ns and, for
  * issue_mma = 0, no tensor-core work issued.  A CTA whose wait ran out writes
- * NaN columns and stops; the row passes then carry the NaN into y.  Other
- * shapes return HYENA_ERR_UNSUPPORTED_SHAPE.
+ * NaN (workspace columns or rows, or outputs) and stops; the later passes
+ * carry the NaN into y.  Other shapes return HYENA_ERR_UNSUPPORTED_SHAPE.
  */
 hyena_status_t hyena_debug_conv_2d_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, int64_t B,
                                       int64_t C, int64_t W, int order, void* workspace, size_t workspace_bytes,
