@@ -104,6 +104,125 @@ __global__ void k_2d_plane_tc(const float2* __restrict__ rows, uint4* __restrict
     }
 }
 
+
+// Tables of a 2-D tensor-core kernel: the 32 entries of the DFT matrices (in
+// the operand area, free until the first task), w512^e (e < 512), and the
+// DFT matrices the kernel uses (S1: stage 1, K 16 -> N 32; S2: the 32-point
+// stages; S1I: stage 1', K 32 -> N 16).
+template <bool S1, bool S2, bool S1I>
+__device__ __forceinline__ void setup_tables(uint8_t* smem, float2* w512) {
+    float2* w32 = reinterpret_cast<float2*>(smem);
+    fill_w32(w32);
+    for (int e = threadIdx.x; e < 512; e += NT) {
+        float sv, cv;
+        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);   // w512^e = exp(-2 pi i e / 512)
+        w512[e] = make_float2(cv, -sv);
+    }
+    __syncthreads();
+    if (S1) fill_dft<16, 16, 8, kSBO16>(smem + kOffB1, w32);
+    if (S2) fill_dft<32, 32, 32, kSBO64>(smem + kOffB32, w32);
+    if (S1I) fill_dft<16, 8, 16, kSBO32>(smem + kOffB1i, w32);
+}
+
+// Stage-1 operand of a task: rows a_tc = c + 32 a (c < 32 the task's column or
+// row, a < 32), slots s < 8 holding x[c][a + 32 s] = get(c, a, s) (a bf16
+// pair); thread t takes rows a0 .. a0+7 (a0 = 8 (t & 127)) at slots
+// 4 (t >> 7) .. +3 (the store pattern of the L = 8192 kernel's stage 1).
+template <typename Get>
+__device__ __forceinline__ void build_stage1(uint8_t* A1, Get get) {
+    const int t = threadIdx.x;
+    const int chalf = t >> 7, a0 = 8 * (t & 127);
+    const int r0 = rho1(a0);
+    const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
+    uint32_t x[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int atc = a0 + i;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[i][j] = get(atc & 31, atc >> 5, 4 * chalf + j);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int jp = 0; jp < 4; jp += 2)
+            *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u + 4u * jp) =
+                make_uint2(x[i][jp], x[i][jp + 1]);
+}
+
+// Wait for stage 1, then pass 1: twiddle w512^(q k1) (q = j + 4 Q + 16 h, the a
+// of the stage-1 row) into the stage-2 rows (k1, b) of tc16k.cuh's order.
+__device__ __forceinline__ void pass1_512(uint8_t* A, const float2* w512, uint32_t tl, int Q, int hh, int lane,
+                                          uint64_t* mbar, uint32_t& phase, bool& ok, uint64_t budget) {
+    C2 pw[4], st2[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 beta = w512[j + 4 * Q + 16 * hh];
+        pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
+        st2[j] = c2_splat(cmul(beta, beta));
+    }
+    ok = stage_wait(mbar, phase, ok, budget);
+    const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO + uint32_t(lane & 7) * 16u;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        float d[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            const int k1 = 8 * half + 2 * pp;
+            C2 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[j] = cmul2(c2_at(d[j], pp), pw[j]);
+                pw[j] = cmul2(pw[j], st2[j]);
+            }
+            sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64, pack_bf16(v[0].re.x, v[0].im.x),
+                   pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+            sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64, pack_bf16(v[0].re.y, v[0].im.y),
+                   pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
+        }
+    }
+}
+
+// Wait for stage 2', then pass 2': rows (k1 = 4 Q + T, b = lane), outputs q =
+// 16 h + ..; twiddle w512^(q k1) -> stage-1' row b + 32 q, chunk Q (slots k1 =
+// 4 Q .. 4 Q + 3).
+__device__ __forceinline__ void pass2i_512(uint8_t* A, const float2* w512, uint32_t tl, int Q, int hh, int lane,
+                                           uint64_t* mbar, uint32_t& phase, bool& ok, uint64_t budget) {
+    const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO + uint32_t(lane & 7) * 16u;
+    C2 pw[4], st2[4];
+#pragma unroll
+    for (int T = 0; T < 4; ++T) {
+        const int k1 = 4 * Q + T;
+        const float2 p0 = w512[(16 * hh * k1) & 511];
+        pw[T] = c2_of(p0, cmul(p0, w512[k1]));
+        st2[T] = c2_splat(w512[(2 * k1) & 511]);
+    }
+    ok = stage_wait(mbar, phase, ok, budget);
+#pragma unroll 1
+    for (int gq = 0; gq < 4; ++gq) {
+        float d[4][8];
+#pragma unroll
+        for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int ip = 0; ip < 2; ++ip) {
+            C2 v[4];
+#pragma unroll
+            for (int T = 0; T < 4; ++T) {
+                v[T] = cmul2(c2_at(d[T], ip), pw[T]);
+                pw[T] = cmul2(pw[T], st2[T]);
+            }
+            const int i = 2 * ip;
+            sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
+                   pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+            sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
+                   pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NT, 2)
 k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum, int C, int W, int64_t B,
              int step, int64_t img0, int nimg, int64_t ws_img_stride, int64_t plane_off, int64_t SC, int64_t SB,
@@ -124,17 +243,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
 
-    float2* w32 = reinterpret_cast<float2*>(smem_2t);
-    fill_w32(w32);
-    for (int e = t; e < 512; e += NT) {
-        float sv, cv;
-        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);   // w512^e = exp(-2 pi i e / 512)
-        w512[e] = make_float2(cv, -sv);
-    }
-    __syncthreads();
-    fill_dft<16, 16, 8, kSBO16>(smem_2t + kOffB1, w32);
-    fill_dft<32, 32, 32, kSBO64>(smem_2t + kOffB32, w32);
-    fill_dft<16, 8, 16, kSBO32>(smem_2t + kOffB1i, w32);
+    setup_tables<true, true, true>(smem_2t, w512);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -158,21 +267,6 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     const int pgroups = 2 * hdr_W / NCOL;         // column blocks of a plane row
     const int ntasks = nimg * groups;
 
-    // stage-1 inputs of a task: thread t takes rows a_tc = a0 + i (a0 = 8 (t & 127)) at
-    // slots s = 4 (t >> 7) + j, i.e. x[c][a + 32 s] with c = a_tc & 31, a = a_tc >> 5
-    auto load_build = [&](int tk, uint32_t (&xb)[8][4]) {
-        const int li = tk / groups, cg = tk - li * groups;
-        const uint32_t* cb = reinterpret_cast<const uint32_t*>(ws + int64_t(li) * ws_img_stride) +
-                             int64_t(NCOL * cg) * MH;
-        const int chalf = t >> 7, a0 = 8 * (t & 127);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int atc = a0 + i, cc = atc & 31, aa = atc >> 5;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xb[i][j] = cb[cc * MH + aa + 32 * (4 * chalf + j)];
-        }
-    };
-
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int li = task / groups, cg = task - li * groups;
         const int64_t img = img0 + li;
@@ -181,19 +275,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
         const uint4* kq = plane + ((int64_t(step) * SC + b * SB + c) * pgroups + cg) * (kPlaneTask / 4) +
                           (Q * 2 + hh) * 16 * 32 + lane;
         // ---------------- stage-1 operand: rows a_tc = c + 32 a, slots s < 8 (x[c][a + 32 s])
-        {
-            uint32_t x[8][4];
-            load_build(task, x);
-            const int chalf = t >> 7, a0 = 8 * (t & 127);
-            const int r0 = rho1(a0);
-            const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int jp = 0; jp < 4; jp += 2)
-                    *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u +
-                                              4u * jp) = make_uint2(x[i][jp], x[i][jp + 1]);
-        }
+        build_stage1(A1, [&](int cc, int aa, int sl) { return col0[cc * MH + aa + 32 * sl]; });
         stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
         if (t < 12 && task + int(gridDim.x) < ntasks) {
             // the next task's 32 columns (32 KB) and spectrum block (64 KB) into L2
@@ -207,41 +289,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(8192u) : "memory");
         }
         // ---------------- pass 1: twiddle w512^(q k1), q = j + 4 Q + 16 h (= a), rows of stage 2 (k1, b = c)
-        {
-            C2 pw[4], st2[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 beta = w512[j + 4 * Q + 16 * hh];
-                pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
-                st2[j] = c2_splat(cmul(beta, beta));
-            }
-            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
-            const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
-                                  uint32_t(lane & 7) * 16u;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float d[4][16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    const int k1 = 8 * half + 2 * pp;
-                    C2 v[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[j] = cmul2(c2_at(d[j], pp), pw[j]);
-                        pw[j] = cmul2(pw[j], st2[j]);
-                    }
-                    sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64,
-                           pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
-                           pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
-                    sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64,
-                           pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
-                           pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
-                }
-            }
-        }
+        pass1_512(A, w512, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         // ---------------- stage 2 (over a); meanwhile this thread loads its spectrum values
         stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
         {
@@ -273,44 +321,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
         }
         // ---------------- stage 2' (inverse, on conj)
         stage_issue(a_addr, kSBO64s, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
-        {
-            // rows (k1 = 4 Q + T, b = lane), outputs q = 16 h + ..; twiddle w512^(q k1)
-            // -> stage-1' row b + 32 q, chunk Q (slots k1 = 4 Q .. 4 Q + 3)
-            const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
-                                  uint32_t(lane & 7) * 16u;
-            C2 pw[4], st2[4];
-#pragma unroll
-            for (int T = 0; T < 4; ++T) {
-                const int k1 = 4 * Q + T;
-                const float2 p0 = w512[(16 * hh * k1) & 511];
-                pw[T] = c2_of(p0, cmul(p0, w512[k1]));
-                st2[T] = c2_splat(w512[(2 * k1) & 511]);
-            }
-            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
-#pragma unroll 1
-            for (int gq = 0; gq < 4; ++gq) {
-                float d[4][8];
-#pragma unroll
-                for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int ip = 0; ip < 2; ++ip) {
-                    C2 v[4];
-#pragma unroll
-                    for (int T = 0; T < 4; ++T) {
-                        v[T] = cmul2(c2_at(d[T], ip), pw[T]);
-                        pw[T] = cmul2(pw[T], st2[T]);
-                    }
-                    const int i = 2 * ip;
-                    sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
-                           pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x),
-                           pack_bf16(v[3].re.x, v[3].im.x));
-                    sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
-                           pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y),
-                           pack_bf16(v[3].re.y, v[3].im.y));
-                }
-            }
-        }
+        pass2i_512(A, w512, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         // ---------------- stage 1': 8 tiles x (K 32 -> N 16), outputs s < 8 only
         stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
@@ -420,16 +431,7 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, co
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    float2* w32 = reinterpret_cast<float2*>(smem_rf);
-    fill_w32(w32);
-    for (int e = t; e < 512; e += NT) {
-        float sv, cv;
-        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);
-        w512[e] = make_float2(cv, -sv);
-    }
-    __syncthreads();
-    fill_dft<16, 16, 8, kSBO16>(smem_rf + kOffB1, w32);
-    fill_dft<32, 32, 32, kSBO64>(smem_rf + kOffB32, w32);
+    setup_tables<true, true, false>(smem_rf, w512);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -459,59 +461,10 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, co
         stage_pair_rows(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
         __syncthreads();
         // ---------------- stage-1 operand: rows a_tc = r + 32 a, slots s < 8 (z[r][a + 32 s])
-        {
-            const int chalf = t >> 7, a0 = 8 * (t & 127);
-            const int r0 = rho1(a0);
-            const uint32_t base = uint32_t(r0 >> 3) * kSBO16 + uint32_t(chalf) * tc::kLBO + uint32_t(r0 & 7) * 16u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int atc = a0 + i, r = atc & 31, aa = atc >> 5;
-                uint32_t x[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) x[j] = Zs[r * W2 + ((aa + 32 * (4 * chalf + j)) ^ (8 * (r >> 3)))];
-#pragma unroll
-                for (int jp = 0; jp < 4; jp += 2)
-                    *reinterpret_cast<uint2*>(A1 + base + uint32_t(i & 3) * kSBO16 + uint32_t(i >> 2) * 16u +
-                                              4u * jp) = make_uint2(x[jp], x[jp + 1]);
-            }
-        }
+        build_stage1(A1, [&](int r, int aa, int sl) { return Zs[r * W2 + ((aa + 32 * sl) ^ (8 * (r >> 3)))]; });
         stage_issue(a1_addr, kSBO16, b1_addr, kSBO16, 8, 1, tc::idesc_bf16(128, 32), tmem, 32, &mbar, ok && issue_mma);
         // ---------------- pass 1: twiddle w512^(q k1), rows of stage 2 (k1, b = r)
-        {
-            C2 pw[4], st2[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 beta = w512[j + 4 * Q + 16 * hh];
-                pw[j] = c2_of(make_float2(1.0f, 0.0f), beta);
-                st2[j] = c2_splat(cmul(beta, beta));
-            }
-            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
-            const uint32_t base = uint32_t(16 * (lane >> 3)) * kSBO64 + uint32_t(Q + 4 * hh) * tc::kLBO +
-                                  uint32_t(lane & 7) * 16u;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float d[4][16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tc::tmem_ld16(tl + uint32_t(32 * (4 * hh + j) + 16 * half), d[j]);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    const int k1 = 8 * half + 2 * pp;
-                    C2 v[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[j] = cmul2(c2_at(d[j], pp), pw[j]);
-                        pw[j] = cmul2(pw[j], st2[j]);
-                    }
-                    sts128(A, base + uint32_t(4 * (k1 >> 2) + (k1 & 3)) * kSBO64,
-                           pack_bf16(v[0].re.x, v[0].im.x), pack_bf16(v[1].re.x, v[1].im.x),
-                           pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
-                    sts128(A, base + uint32_t(4 * ((k1 + 1) >> 2) + ((k1 + 1) & 3)) * kSBO64,
-                           pack_bf16(v[0].re.y, v[0].im.y), pack_bf16(v[1].re.y, v[1].im.y),
-                           pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
-                }
-            }
-        }
+        pass1_512(A, w512, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         // ---------------- stage 2 (over a): Z[k1 + 16 k2] of row r
         stage_issue(a_addr, kSBO64, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
@@ -577,16 +530,7 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    float2* w32 = reinterpret_cast<float2*>(smem_ri);
-    fill_w32(w32);
-    for (int e = t; e < 512; e += NT) {
-        float sv, cv;
-        sincospif(float(e) * (1.0f / 256.0f), &sv, &cv);
-        w512[e] = make_float2(cv, -sv);
-    }
-    __syncthreads();
-    fill_dft<32, 32, 32, kSBO64>(smem_ri + kOffB32, w32);
-    fill_dft<16, 8, 16, kSBO32>(smem_ri + kOffB1i, w32);
+    setup_tables<false, true, true>(smem_ri, w512);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -627,42 +571,7 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
         }
         stage_issue(a_addr, kSBO64s, b32_addr, kSBO64, 4, 4, tc::idesc_bf16(128, 64), tmem, 64, &mbar, ok && issue_mma);
         // ---------------- pass 2' (twiddle w512^(q k1)) -> stage-1' rows r + 32 q
-        {
-            const uint32_t base = uint32_t((lane >> 3) + 64 * hh) * kSBO32 + uint32_t(Q) * tc::kLBO +
-                                  uint32_t(lane & 7) * 16u;
-            C2 pw[4], st2[4];
-#pragma unroll
-            for (int T = 0; T < 4; ++T) {
-                const int k1 = 4 * Q + T;
-                const float2 p0 = w512[(16 * hh * k1) & 511];
-                pw[T] = c2_of(p0, cmul(p0, w512[k1]));
-                st2[T] = c2_splat(w512[(2 * k1) & 511]);
-            }
-            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
-#pragma unroll 1
-            for (int gq = 0; gq < 4; ++gq) {
-                float d[4][8];
-#pragma unroll
-                for (int T = 0; T < 4; ++T) tc::tmem_ld8(tl + uint32_t(64 * T + 32 * hh + 8 * gq), d[T]);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int ip = 0; ip < 2; ++ip) {
-                    C2 v[4];
-#pragma unroll
-                    for (int T = 0; T < 4; ++T) {
-                        v[T] = cmul2(c2_at(d[T], ip), pw[T]);
-                        pw[T] = cmul2(pw[T], st2[T]);
-                    }
-                    const int i = 2 * ip;
-                    sts128(A, base + uint32_t(16 * gq + 4 * i) * kSBO32, pack_bf16(v[0].re.x, v[0].im.x),
-                           pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x),
-                           pack_bf16(v[3].re.x, v[3].im.x));
-                    sts128(A, base + uint32_t(16 * gq + 4 * (i + 1)) * kSBO32, pack_bf16(v[0].re.y, v[0].im.y),
-                           pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y),
-                           pack_bf16(v[3].re.y, v[3].im.y));
-                }
-            }
-        }
+        pass2i_512(A, w512, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         // ---------------- stage 1': outputs s < 8 (n = a + 32 s < 256)
         stage_issue(a_addr, kSBO32, b1i_addr, kSBO32, 8, 2, tc::idesc_bf16(128, 16), tmem, 16, &mbar, ok && issue_mma);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
