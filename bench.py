@@ -299,6 +299,26 @@ def kernel_of(p) -> str:
     return "multipass" if p.ndim == 1 else ("grid2d" if p.ndim == 2 else "grid3d")
 
 
+def launches_per_step(p) -> int:
+    """Kernels one hyena_gated_fftconv call launches for problem p with the
+    default workspace (the whole batch in one row group), as dispatched."""
+    steps = p.order - 1
+    if p.ndim == 1:
+        if p.L <= 16384 or kernel_of(p) == "k_conv_cluster":
+            return 1                          # every order step inside one kernel
+        return 1 + 2 * steps                  # columns forward, then per step rows and inverse columns
+    if p.ndim == 2:
+        if p.circular:
+            return 1 + 2 * steps              # rows forward, per step columns and rows inverse
+        if (p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.order == 2 and p.B % 2 == 0
+                and not p.per_sample):
+            return 3                          # paired images: rows, columns, rows inverse
+        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+            return 1 + 3 * steps              # per step: tensor-core columns, last column, rows inverse
+        return 1 + 2 * steps
+    return 1 + 4 * steps                      # 3-D: per step columns, depth, columns inverse, rows inverse
+
+
 def math_of(p, kernel: str) -> str:
     """What the measured kernel computes in, as built."""
     if kernel == "k_conv_8192_tc":
@@ -512,7 +532,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": u.numel() * u.element_size(),
                 "d2h_bytes_per_step": y.numel() * y.element_size()},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step(p),
         "fp32_transform": None if fp32_ms is None else {
             "kernel": "k_conv_4096", "flag": "HYENA_FLAG_FP32_TRANSFORM",
             "math": "fp32 throughout (register FFT on the CUDA cores; complex64 spectrum plane)",
