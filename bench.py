@@ -133,10 +133,10 @@ def spectrum_row_bytes(p) -> int:
     if p.ndim == 2:
         if p.circular:
             return (p.W // 2 + 1) * p.H * 8
-        if p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.order == 2 and p.B % 2 == 0 and not p.per_sample:
+        if p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0 and not p.per_sample and p.order <= 3:
             # paired images: the whole 2H x 2W bf16 plane
             return 2 * p.W * 2 * p.H * 4
-        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0 and p.order <= 3:
             # tensor-core column pass: bf16 plane of bins 0..W-1, complex64 last column
             return p.W * 2 * p.H * 4 + 2 * p.H * 8
         return (p.W + 1) * 2 * p.H * 8
@@ -310,10 +310,9 @@ def launches_per_step(p) -> int:
     if p.ndim == 2:
         if p.circular:
             return 1 + 2 * steps              # rows forward, per step columns and rows inverse
-        if (p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.order == 2 and p.B % 2 == 0
-                and not p.per_sample):
-            return 3                          # paired images: rows, columns, rows inverse
-        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+        if p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0 and not p.per_sample and p.order <= 3:
+            return 3 * steps                  # paired images, per step: rows, columns, rows inverse
+        if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0 and p.order <= 3:
             return 1 + 3 * steps              # per step: tensor-core columns, last column, rows inverse
         return 1 + 2 * steps
     return 1 + 4 * steps                      # 3-D: per step columns, depth, columns inverse, rows inverse
@@ -328,12 +327,12 @@ def math_of(p, kernel: str) -> str:
         return ("2L-point transform split over 8-CTA clusters: 8-point DFTs, short conv, gates and twiddles fp32 "
                 "on the CUDA cores; 16384-point DFT stages per CTA on tcgen05 tensor cores with bf16 operands and "
                 "fp32 accumulation; exchanges as bf16 pairs; spectrum read as bf16 (re, im)")
-    if (p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.order == 2
-            and p.B % 2 == 0 and not p.per_sample):
+    if (p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0
+            and not p.per_sample and p.order <= 3):
         return ("the two images of a channel as one complex image: row, column and row passes as 512-point DFT "
                 "stages on tcgen05 tensor cores (bf16 operands, fp32 accumulation), gates and twiddles fp32, "
                 "spectrum read as a bf16 (re, im) plane, intermediate kept as bf16 pairs in the workspace")
-    if p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0:
+    if p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0 and p.order <= 3:
         return ("row passes fp32 on the CUDA cores; column pass of bins 0..W-1 as 512-point DFT stages on tcgen05 "
                 "tensor cores (bf16 operands, fp32 accumulation, spectrum read as bf16 (re, im)), last bin column "
                 "fp32; intermediate kept as bf16 pairs in the workspace between passes")

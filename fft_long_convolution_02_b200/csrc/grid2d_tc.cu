@@ -384,7 +384,10 @@ constexpr int W2 = 256;           // image width of the paired path (row transfo
 constexpr int NROW = 32;          // image rows per task
 
 // z of rows r0 .. r0+31 of a pair -> staging Zs[r][n ^ (8 (r >> 3))] (bf16 pairs):
-// the XOR lets the stage-1 gather below read 32 different banks.
+// the XOR lets the stage-1 gather below read 32 different banks.  GATE: z =
+// x v (the first order step), else z = x (a later step's input, already gated
+// by the previous step's inverse pass).
+template <bool GATE>
 __device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __restrict__ x_b0, const bf16* __restrict__ x_b1,
                                                 const bf16* __restrict__ v_b0, const bf16* __restrict__ v_b1, int t) {
 #pragma unroll
@@ -393,20 +396,29 @@ __device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __rest
         const int64_t off = int64_t(r) * W2 + n0;
         const uint4 xa = __ldg(reinterpret_cast<const uint4*>(x_b0 + off));
         const uint4 xb = __ldg(reinterpret_cast<const uint4*>(x_b1 + off));
-        const uint4 va = __ldg(reinterpret_cast<const uint4*>(v_b0 + off));
-        const uint4 vb = __ldg(reinterpret_cast<const uint4*>(v_b1 + off));
         const uint32_t xw[2][4] = {{xa.x, xa.y, xa.z, xa.w}, {xb.x, xb.y, xb.z, xb.w}};
-        const uint32_t vw[2][4] = {{va.x, va.y, va.z, va.w}, {vb.x, vb.y, vb.z, vb.w}};
         uint32_t o[8];
+        if constexpr (GATE) {
+            const uint4 va = __ldg(reinterpret_cast<const uint4*>(v_b0 + off));
+            const uint4 vb = __ldg(reinterpret_cast<const uint4*>(v_b1 + off));
+            const uint32_t vw[2][4] = {{va.x, va.y, va.z, va.w}, {vb.x, vb.y, vb.z, vb.w}};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            // samples 2q, 2q+1 of both images: (g[b0], g[b1]) at each
-            const float2 lo = __fmul2_rn(make_float2(bf_lo(xw[0][q]), bf_lo(xw[1][q])),
-                                         make_float2(bf_lo(vw[0][q]), bf_lo(vw[1][q])));
-            const float2 hi = __fmul2_rn(make_float2(bf_hi(xw[0][q]), bf_hi(xw[1][q])),
-                                         make_float2(bf_hi(vw[0][q]), bf_hi(vw[1][q])));
-            o[2 * q] = pack_bf16(lo.x, lo.y);
-            o[2 * q + 1] = pack_bf16(hi.x, hi.y);
+            for (int q = 0; q < 4; ++q) {
+                // samples 2q, 2q+1 of both images: (g[b0], g[b1]) at each
+                const float2 lo = __fmul2_rn(make_float2(bf_lo(xw[0][q]), bf_lo(xw[1][q])),
+                                             make_float2(bf_lo(vw[0][q]), bf_lo(vw[1][q])));
+                const float2 hi = __fmul2_rn(make_float2(bf_hi(xw[0][q]), bf_hi(xw[1][q])),
+                                             make_float2(bf_hi(vw[0][q]), bf_hi(vw[1][q])));
+                o[2 * q] = pack_bf16(lo.x, lo.y);
+                o[2 * q + 1] = pack_bf16(hi.x, hi.y);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                // the two images' samples interleaved: (z[b0], z[b1]) per sample
+                o[2 * q] = __byte_perm(xw[0][q], xw[1][q], 0x5410);
+                o[2 * q + 1] = __byte_perm(xw[0][q], xw[1][q], 0x7632);
+            }
         }
         uint32_t* dst = Zs + r * W2 + (n0 ^ (8 * (r >> 3)));
         *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -415,8 +427,9 @@ __device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __rest
 }
 
 __global__ void __launch_bounds__(NT, 2)
-k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum,
-                 int64_t B, int64_t C, int order, int64_t pair0, int npairs, int64_t ws_pair_stride,
+k_2d_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv_bfloat162* __restrict__ ws,
+                 const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
+                 int64_t ws_pair_stride,
                  uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_rf[];
     __shared__ __align__(8) uint64_t mbar;
@@ -456,9 +469,16 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, co
         const int lp = task / (MH / NROW), rg = task - lp * (MH / NROW);
         const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
         const int64_t rowoff = int64_t(NROW * rg) * W2;
-        const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
-        const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
-        stage_pair_rows(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
+        if (zsrc == nullptr) {
+            // first order step: z = x_{order-1} v
+            const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
+            const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
+            stage_pair_rows<true>(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
+        } else {
+            // later steps: z written by the previous step's inverse pass ([B, C, H, W])
+            const bf16* z0 = zsrc + (b0 * C + c) * n_img + rowoff;
+            stage_pair_rows<false>(Zs, z0, z0 + C * n_img, nullptr, nullptr, t);
+        }
         __syncthreads();
         // ---------------- stage-1 operand: rows a_tc = r + 32 a, slots s < 8 (z[r][a + 32 s])
         build_stage1(A1, [&](int r, int aa, int sl) { return Zs[r * W2 + ((aa + 32 * sl) ^ (8 * (r >> 3)))]; });
@@ -516,7 +536,8 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, __nv_bfloat162* __restrict__ ws, co
 
 __global__ void __launch_bounds__(NT, 2)
 k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bfloat162* __restrict__ ws,
-                 const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
+                 const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int gchunk, int64_t pair0,
+                 int npairs,
                  int64_t ws_pair_stride, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
     extern __shared__ __align__(1024) uint8_t smem_ri[];
     __shared__ __align__(8) uint64_t mbar;
@@ -592,10 +613,11 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
         }
         tc::fence_before_sync();
         __syncthreads();
-        // output gate: y = x0 * conv for both images, 8 columns of a row per step
+        // gate: y = x_gchunk * conv for both images (x0 at the last order step,
+        // else the next step's input), 8 columns of a row per step
         {
             const int64_t rowoff = int64_t(NROW * rg) * W2;
-            const bf16* xa = u + (b0 * Ctot + c) * n_img + rowoff;
+            const bf16* xa = u + (b0 * Ctot + int64_t(gchunk) * C + c) * n_img + rowoff;
             const bf16* xb = xa + Ctot * n_img;
             bf16* ya = y + (b0 * C + c) * n_img + rowoff;
             bf16* yb = ya + C * n_img;
@@ -654,9 +676,12 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
 
 }  // namespace
 
+// Orders above kMaxOrderTc keep the fp32 passes, as in 1-D: every order step
+// adds the bf16 roundings of its stage operands (image error ~6e-3, 1e-2 and
+// 1.4e-2 at orders 2, 3 and 4 with the paired passes).
 bool cols_2d_tc_path(const Plan& p, const ConvArgs& a) {
     return p.path == PATH_GRID_2D && p.H == kTc2dH && p.W % NCOL == 0 && a.g2_plane_off != 0 &&
-           a.dtype == DT_BF16 && !a.fp32_transform;
+           a.dtype == DT_BF16 && !a.fp32_transform && p.order <= kMaxOrderTc;
 }
 
 cudaError_t launch_spectrum_2d_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
@@ -689,7 +714,7 @@ cudaError_t launch_cols_2d_tc(const Plan& p, const ConvArgs& a, void* ws, int64_
 }
 
 bool pairs_2d_tc_path(const Plan& p, const ConvArgs& a) {
-    return cols_2d_tc_path(p, a) && p.W == W2 && p.order == 2 && a.B % 2 == 0 && a.spec_per_b == 0;
+    return cols_2d_tc_path(p, a) && p.W == W2 && a.B % 2 == 0 && a.spec_per_b == 0;
 }
 
 cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg,
@@ -708,15 +733,22 @@ cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, 
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2d_cols_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2d_rows_inv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
     if (e != cudaSuccess) return e;
-    k_2d_rows_fwd_tc<<<grid, NT, kSmem, s>>>(u, w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride,
-                                             a.wait_budget_ns, a.issue_mma, a.status);
-    // every bin column of a pair (2W), spectrum row c = pair / (B/2)
+    bf16* y = static_cast<bf16*>(a.y);
     const int64_t ctasks = npairs * (2 * W2 / NCOL);
-    k_2d_cols_tc<<<unsigned(ctasks < 2 * sms ? ctasks : 2 * sms), NT, kSmem, s>>>(
-        w, a.spectrum, int(p.C), 2 * W2, a.B / 2, 0, pair0, int(npairs), pstride, int64_t(a.g2_plane_off), a.spec_C,
-        0, W2, a.wait_budget_ns, a.issue_mma, a.status);
-    k_2d_rows_inv_tc<<<grid, NT, kSmem, s>>>(u, static_cast<bf16*>(a.y), w, a.spectrum, a.B, p.C, p.order, pair0,
-                                             int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
+    for (int st = 1; st < p.order; ++st) {
+        // step st gates with x_{order-st}: the first step's input is x_{order-1} v, a later
+        // step's is x_{order-st} times the previous step's result, which that step's
+        // inverse pass left in y; the last inverse pass applies x0
+        k_2d_rows_fwd_tc<<<grid, NT, kSmem, s>>>(u, st == 1 ? nullptr : y, w, a.spectrum, a.B, p.C, p.order, pair0,
+                                                 int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        // every bin column of a pair (2W), spectrum row (st - 1) C + c, c = pair / (B/2)
+        k_2d_cols_tc<<<unsigned(ctasks < 2 * sms ? ctasks : 2 * sms), NT, kSmem, s>>>(
+            w, a.spectrum, int(p.C), 2 * W2, a.B / 2, st - 1, pair0, int(npairs), pstride, int64_t(a.g2_plane_off),
+            a.spec_C, 0, W2, a.wait_budget_ns, a.issue_mma, a.status);
+        k_2d_rows_inv_tc<<<grid, NT, kSmem, s>>>(u, y, w, a.spectrum, a.B, p.C, p.order,
+                                                 st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs), pstride,
+                                                 a.wait_budget_ns, a.issue_mma, a.status);
+    }
     return cudaGetLastError();
 }
 

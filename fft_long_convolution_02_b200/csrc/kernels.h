@@ -96,7 +96,7 @@ cudaError_t launch_cols_2d_tc(const Plan& p, const ConvArgs& a, void* ws, int64_
                               int64_t ws_img_stride, cudaStream_t s);
 cudaError_t launch_spectrum_2d_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
                                         cudaStream_t s);
-// 256 x 256 images, order 2, even B, shared filters: the two images of a
+// 256 x 256 images, even B, shared filters: the two images of a
 // channel as one complex image, all three passes on the tensor cores
 bool pairs_2d_tc_path(const Plan& p, const ConvArgs& a);
 cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg,

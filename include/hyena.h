@@ -39,8 +39,8 @@
  *    order 3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 multi-pass
  *    transform there.  2-D with bf16 storage and H = 256 (W a multiple of
  *    32): the column transforms (512 points) run on the tensor cores the same
- *    way, with the spectrum read as bf16 pairs; for 256 x 256 images at order
- *    2 with an even batch and shared filters the two images of a channel
+ *    way, with the spectrum read as bf16 pairs (order <= 3); for 256 x 256
+ *    images with an even batch and shared filters the two images of a channel
  *    travel as one complex image and the row transforms run there too (image
  *    error a few 1e-3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 passes.
  *    With bf16 storage the intermediate of the multi-pass (L >= 32768) and

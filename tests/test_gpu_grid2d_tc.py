@@ -112,11 +112,12 @@ def test_tc_columns_report_a_spectrum_header_mismatch():
     assert np.isfinite(from_torch(r.y)).all()
 
 
-@pytest.mark.parametrize("B,C,order", [(2, 3, 2), (4, 2, 2), (3, 2, 2), (2, 2, 3)])
+@pytest.mark.parametrize("B,C,order", [(2, 3, 2), (4, 2, 2), (3, 2, 2), (2, 2, 3), (2, 1, 4)])
 def test_paired_images_against_oracle(orc, B, C, order):
-    """256 x 256 images: with an even batch at order 2 the two images of a
-    channel travel as one complex image through tensor-core row, column and
-    row passes; an odd batch or order 3 takes the unpaired passes."""
+    """256 x 256 images: with an even batch the two images of a channel travel
+    as one complex image through tensor-core row, column and row passes, once
+    per order step (orders 2 and 3); an odd batch takes the unpaired passes,
+    order 4 the fp32 passes."""
     p = I.WORKLOADS["grid2d"].with_(B=B, C=C, H=256, W=256, order=order, seed=3500 + 10 * B + order)
     data = I.make_all(p)
     r = Run(p, data)
