@@ -126,16 +126,23 @@ def algorithmic_bytes(p, spectrum_row_bytes: int) -> int:
     return u + spec + y
 
 
+def paired_2d(p) -> bool:
+    """256 x 256 images with bf16 storage and an even batch: the two images of a
+    channel travel as one complex image through tensor-core passes (both forms)."""
+    return (p.ndim == 2 and p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0
+            and not p.per_sample and p.order <= 3)
+
+
 def spectrum_row_bytes(p) -> int:
     """Spectrum bytes per (step, channel) row the convolution kernel reads."""
     if p.ndim == 3:
         return (p.W + 1) * 2 * p.H * 2 * p.N1 * 8
     if p.ndim == 2:
+        if paired_2d(p):
+            # paired images: the whole bf16 plane (H x W circular, 2H x 2W padded)
+            return (1 if p.circular else 4) * p.W * p.H * 4
         if p.circular:
             return (p.W // 2 + 1) * p.H * 8
-        if p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0 and not p.per_sample and p.order <= 3:
-            # paired images: the whole 2H x 2W bf16 plane
-            return 2 * p.W * 2 * p.H * 4
         if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0 and p.order <= 3:
             # tensor-core column pass: bf16 plane of bins 0..W-1, complex64 last column
             return p.W * 2 * p.H * 4 + 2 * p.H * 8
@@ -308,10 +315,10 @@ def launches_per_step(p) -> int:
             return 1                          # every order step inside one kernel
         return 1 + 2 * steps                  # columns forward, then per step rows and inverse columns
     if p.ndim == 2:
+        if paired_2d(p):
+            return 3 * steps                  # paired images, per step: rows, columns, rows inverse
         if p.circular:
             return 1 + 2 * steps              # rows forward, per step columns and rows inverse
-        if p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0 and not p.per_sample and p.order <= 3:
-            return 3 * steps                  # paired images, per step: rows, columns, rows inverse
         if p.dtype == "bf16" and p.H == 256 and p.W % 32 == 0 and p.order <= 3:
             return 1 + 3 * steps              # per step: tensor-core columns, last column, rows inverse
         return 1 + 2 * steps
@@ -327,8 +334,12 @@ def math_of(p, kernel: str) -> str:
         return ("2L-point transform split over 8-CTA clusters: 8-point DFTs, short conv, gates and twiddles fp32 "
                 "on the CUDA cores; 16384-point DFT stages per CTA on tcgen05 tensor cores with bf16 operands and "
                 "fp32 accumulation; exchanges as bf16 pairs; spectrum read as bf16 (re, im)")
-    if (p.ndim == 2 and not p.circular and p.dtype == "bf16" and p.H == 256 and p.W == 256 and p.B % 2 == 0
-            and not p.per_sample and p.order <= 3):
+    if paired_2d(p) and p.circular:
+        return ("the two images of a channel as one complex image: row, column and row passes as 256-point DFTs "
+                "(two 16-point stages) on tcgen05 tensor cores (bf16 operands, fp32 accumulation), gates and "
+                "twiddles fp32, spectrum read as a bf16 (re, im) plane, intermediate kept as bf16 pairs in the "
+                "workspace")
+    if paired_2d(p):
         return ("the two images of a channel as one complex image: row, column and row passes as 512-point DFT "
                 "stages on tcgen05 tensor cores (bf16 operands, fp32 accumulation), gates and twiddles fp32, "
                 "spectrum read as a bf16 (re, im) plane, intermediate kept as bf16 pairs in the workspace")

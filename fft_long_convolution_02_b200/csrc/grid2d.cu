@@ -22,6 +22,7 @@
 // digit-reversed order its forward DIF leaves behind.
 #include "common.cuh"
 #include "cta_fft.cuh"
+#include "grid2dc_tc.h"
 #include "kernels.h"
 #include "reg_fft.cuh"
 
@@ -937,6 +938,11 @@ cudaError_t spectrum_2dc_t(const Plan& p, const SpectrumArgs& a, cudaStream_t s)
         kb<<<dim3(unsigned(W / 2 + 1), unsigned(g)), kColThreads2, smB, s>>>(rows + i0 * stride, tb, W / 2 + 1, i0,
                                                                              stride, a.D, s2);
     }
+    if (p.g2_plane_off != 0) {
+        const cudaError_t e = launch_spectrum_2dc_tc_plane(p, reinterpret_cast<const uint8_t*>(rows),
+                                                           a.spectrum + p.g2_plane_off, nimg, s);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 
@@ -966,6 +972,19 @@ cudaError_t conv_2dc_t(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
     cudaFuncSetAttribute(kca, cudaFuncAttributeMaxDynamicSharedMemorySize, int(row_smem<MW>()));
     const unsigned cblocks = unsigned((ncol + 2 * kFC - 1) / (2 * kFC));
+    if constexpr (sizeof(T) == 2) {
+        // 256 x 256: the two images of a channel as one complex image on the tensor
+        // cores (groups of whole pairs)
+        const int64_t Gp = G & ~int64_t(1);
+        if (Gp >= 2 && pairs_2dc_tc_path(p, a)) {
+            for (int64_t i0 = 0; i0 < nimg; i0 += Gp) {
+                const int64_t g = nimg - i0 < Gp ? nimg - i0 : Gp;
+                const cudaError_t e = launch_conv_2dc_pairs_tc(p, a, ws, i0, g, stride, s);
+                if (e != cudaSuccess) return e;
+            }
+            return cudaGetLastError();
+        }
+    }
     for (int64_t i0 = 0; i0 < nimg; i0 += G) {
         const int64_t g = nimg - i0 < G ? nimg - i0 : G;
         const dim3 gridR(H / kRB, unsigned(g));

@@ -426,6 +426,56 @@ __device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __rest
     }
 }
 
+// Output gate of 32 rows of a pair: staged result Ys[r][n ^ r] (bf16 pairs
+// (image b0, image b1)) times the gate rows x_b0 / x_b1, stored to y_b0 / y_b1
+// (rows of W2 samples), 8 columns of a row per step; NaN once a wait ran out.
+__device__ __forceinline__ void gate_store_pair_rows(const uint32_t* Ys, const bf16* __restrict__ xa,
+                                                     const bf16* __restrict__ xb, bf16* __restrict__ ya,
+                                                     bf16* __restrict__ yb, int t, bool ok) {
+#pragma unroll
+    for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
+        const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
+        const int64_t off = int64_t(r) * W2 + n0;
+        const uint4 x0a = __ldg(reinterpret_cast<const uint4*>(xa + off));
+        const uint4 x0b = __ldg(reinterpret_cast<const uint4*>(xb + off));
+        // word n0 + i sits at (n0 ^ (r & 24)) + (i ^ (r & 7))
+        const uint32_t* src = Ys + r * W2 + (n0 ^ (r & 24));
+        const uint4 g0 = *reinterpret_cast<const uint4*>(src);
+        const uint4 g1 = *reinterpret_cast<const uint4*>(src + 4);
+        uint32_t w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const int m = r & 7;
+        if (m & 1) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) { const uint32_t tmp = w[i]; w[i] = w[i + 1]; w[i + 1] = tmp; }
+        }
+        if (m & 2) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+                uint32_t tmp = w[i]; w[i] = w[i + 2]; w[i + 2] = tmp;
+                tmp = w[i + 1]; w[i + 1] = w[i + 3]; w[i + 3] = tmp;
+            }
+        }
+        if (m & 4) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { const uint32_t tmp = w[i]; w[i] = w[i + 4]; w[i + 4] = tmp; }
+        }
+        const uint32_t xaw[4] = {x0a.x, x0a.y, x0a.z, x0a.w}, xbw[4] = {x0b.x, x0b.y, x0b.z, x0b.w};
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 lo = __fmul2_rn(make_float2(bf_lo(xaw[q]), bf_lo(xbw[q])),
+                                         make_float2(bf_lo(w[2 * q]), bf_hi(w[2 * q])));
+            const float2 hi = __fmul2_rn(make_float2(bf_hi(xaw[q]), bf_hi(xbw[q])),
+                                         make_float2(bf_lo(w[2 * q + 1]), bf_hi(w[2 * q + 1])));
+            oa[q] = pack_bf16(lo.x, hi.x);
+            ob[q] = pack_bf16(lo.y, hi.y);
+        }
+        const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
+        *reinterpret_cast<uint4*>(ya + off) = ok ? make_uint4(oa[0], oa[1], oa[2], oa[3]) : nan4;
+        *reinterpret_cast<uint4*>(yb + off) = ok ? make_uint4(ob[0], ob[1], ob[2], ob[3]) : nan4;
+    }
+}
+
 __global__ void __launch_bounds__(NT, 2)
 k_2d_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv_bfloat162* __restrict__ ws,
                  const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
@@ -614,55 +664,12 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
         tc::fence_before_sync();
         __syncthreads();
         // gate: y = x_gchunk * conv for both images (x0 at the last order step,
-        // else the next step's input), 8 columns of a row per step
+        // else the next step's input)
         {
             const int64_t rowoff = int64_t(NROW * rg) * W2;
             const bf16* xa = u + (b0 * Ctot + int64_t(gchunk) * C + c) * n_img + rowoff;
-            const bf16* xb = xa + Ctot * n_img;
             bf16* ya = y + (b0 * C + c) * n_img + rowoff;
-            bf16* yb = ya + C * n_img;
-#pragma unroll
-            for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
-                const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
-                const int64_t off = int64_t(r) * W2 + n0;
-                const uint4 x0a = __ldg(reinterpret_cast<const uint4*>(xa + off));
-                const uint4 x0b = __ldg(reinterpret_cast<const uint4*>(xb + off));
-                // word n0 + i sits at (n0 ^ (r & 24)) + (i ^ (r & 7))
-                const uint32_t* src = Ys + r * W2 + (n0 ^ (r & 24));
-                const uint4 g0 = *reinterpret_cast<const uint4*>(src);
-                const uint4 g1 = *reinterpret_cast<const uint4*>(src + 4);
-                uint32_t w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                const int m = r & 7;
-                if (m & 1) {
-#pragma unroll
-                    for (int i = 0; i < 8; i += 2) { const uint32_t tmp = w[i]; w[i] = w[i + 1]; w[i + 1] = tmp; }
-                }
-                if (m & 2) {
-#pragma unroll
-                    for (int i = 0; i < 8; i += 4) {
-                        uint32_t tmp = w[i]; w[i] = w[i + 2]; w[i + 2] = tmp;
-                        tmp = w[i + 1]; w[i + 1] = w[i + 3]; w[i + 3] = tmp;
-                    }
-                }
-                if (m & 4) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) { const uint32_t tmp = w[i]; w[i] = w[i + 4]; w[i + 4] = tmp; }
-                }
-                const uint32_t xaw[4] = {x0a.x, x0a.y, x0a.z, x0a.w}, xbw[4] = {x0b.x, x0b.y, x0b.z, x0b.w};
-                uint32_t oa[4], ob[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 lo = __fmul2_rn(make_float2(bf_lo(xaw[q]), bf_lo(xbw[q])),
-                                                 make_float2(bf_lo(w[2 * q]), bf_hi(w[2 * q])));
-                    const float2 hi = __fmul2_rn(make_float2(bf_hi(xaw[q]), bf_hi(xbw[q])),
-                                                 make_float2(bf_lo(w[2 * q + 1]), bf_hi(w[2 * q + 1])));
-                    oa[q] = pack_bf16(lo.x, hi.x);
-                    ob[q] = pack_bf16(lo.y, hi.y);
-                }
-                const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
-                *reinterpret_cast<uint4*>(ya + off) = ok ? make_uint4(oa[0], oa[1], oa[2], oa[3]) : nan4;
-                *reinterpret_cast<uint4*>(yb + off) = ok ? make_uint4(ob[0], ob[1], ob[2], ob[3]) : nan4;
-            }
+            gate_store_pair_rows(Ys, xa, xa + Ctot * n_img, ya, ya + C * n_img, t, ok);
         }
         if (__syncthreads_or(!ok)) {
             if (t == 0) report_status(status, kStatusTimeout);
@@ -672,6 +679,438 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+
+// ---------------------------------------------------------------------------
+// The circular 2-D form ([P5] "Native Multi-Dimensional Subquadratic
+// Operators", 方法论: the N-D FFT convolution; without the zero padding the
+// product of the transforms is the periodic convolution) at 256 x 256 with
+// bf16 storage, the two images of a channel paired as above.  Every line
+// transform is a 256-point complex DFT, n = n1 + 16 n2, k = k1 + 16 k2:
+//   X[k1 + 16 k2] = sum_n1 w16^(n1 k2) w256^(n1 k1) sum_n2 x[n1 + 16 n2] w16^(n2 k1)
+// two stages with the real form of the full 16-point DFT matrix (K 32 -> N
+// 32) and the twiddle w256^(n1 k1) between them.  The inverse runs on conj
+// through the same matrix and twiddle: a stage over k2 (-> n1), the twiddle
+// w256^(k1 n1), a stage over k1 (-> n2).  A task is 32 lines (8192 points,
+// four tiles of 128 rows); the vector (line l, index i) of every stage sits at
+//   R(l, i) = 128 (i & 3) + 32 (i >> 2) + l,
+// so that thread (lane quarter Q, lane l) holds i = 4 Q + T in tile T and the
+// four slots of each 16-byte chunk it writes.  Three kernels per order step,
+// as for the padded pairs: rows forward (gates, Z[k][row] to the workspace),
+// columns (forward, spectrum product, inverse; in place), rows inverse (output
+// gate).  The spectrum is the full 256 x 256 plane (bf16 pairs) in the column
+// pass's thread order, completed from the stored W/2 + 1 columns by the
+// symmetry of a real filter's transform.
+// ---------------------------------------------------------------------------
+
+constexpr int CN = int(kTc2dH);                  // H = W of the circular tensor-core path
+constexpr uint32_t kSBOc = kSBO32;               // operand rows of K 32 (16 complex slots)
+constexpr uint32_t kAc = 64 * kSBOc;             // 512 rows
+constexpr uint32_t kOffStC = kAc;                // staging: 32 lines x 256 bf16 pairs
+constexpr uint32_t kOffBc = kOffStC + NROW * CN * 4;
+constexpr uint32_t kOffW256 = kOffBc + 4 * kSBOc;   // after the N 32 x K 32 DFT matrix
+constexpr size_t kSmemC = size_t(kOffW256) + CN * sizeof(float2);
+constexpr uint32_t kTmemColsC = 128;             // 4 tiles x 32 columns
+constexpr int kPlaneTaskC = NROW * CN;           // bf16 pairs of the plane per column task
+static_assert(kOffStC % 16 == 0 && kOffW256 % 16 == 0, "table alignment");
+
+__device__ __forceinline__ int rowc(int l, int i) { return 128 * (i & 3) + 32 * (i >> 2) + l; }
+
+// Plane entry e of uint4 idx4 of a column task: idx4 = ((Q * 2 + h) * 8 + 2 T +
+// half) * 32 + lane holds, for column f = 32 fg + lane, bins k = k1 + 16 k2 with
+// k1 = 4 Q + T and k2 = 8 h + 4 half + e.
+__device__ __forceinline__ void plane_entry_c(int idx4, int e, int& l, int& k) {
+    l = idx4 & 31;
+    const int i = (idx4 >> 5) & 7, qh = idx4 >> 8;
+    const int k1 = 4 * (qh >> 1) + (i >> 1);
+    k = k1 + 16 * (8 * (qh & 1) + 4 * (i & 1) + e);
+}
+
+// The plane from the complex64 spectrum rows of the circular form: bin k of a
+// stored column f <= W/2 sits at f * H + the slot of the register engine's
+// position fft_bin_pos(k) (see the circular spectrum build); the columns f >
+// W/2 follow from K~[k][f] = conj K~[-k mod H][W - f].
+__global__ void k_2dc_plane_tc(const float2* __restrict__ rows, uint4* __restrict__ plane, int64_t nrows,
+                               int64_t row_stride) {
+    constexpr int per_task = kPlaneTaskC / 4;
+    const int64_t per_row = int64_t(CN / NROW) * per_task;
+    for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < nrows * per_row;
+         g += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = g / per_row;
+        const int rem = int(g - r * per_row);
+        const int fg = rem / per_task, idx4 = rem - fg * per_task;
+        uint32_t v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int l, k;
+            plane_entry_c(idx4, e, l, k);
+            const int f = NROW * fg + l;
+            const bool mirror = f > CN / 2;
+            const int fs = mirror ? CN - f : f, ks = mirror ? (CN - k) & (CN - 1) : k;
+            const int pos = fft_bin_pos<CN>(ks);
+            const float2 K = rows[r * row_stride + int64_t(fs) * CN + (pos & 15) * (CN / 16) + (pos >> 4)];
+            v[e] = pack_bf16(K.x, mirror ? -K.y : K.y);
+        }
+        plane[g] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+}
+
+// Tables: the real form of the 16-point DFT matrix (B operand) and w256^e.
+__device__ __forceinline__ void setup_tables_c(uint8_t* smem, float2* w256) {
+    float2* w32 = reinterpret_cast<float2*>(smem);
+    fill_w32(w32);
+    for (int e = threadIdx.x; e < CN; e += NT) {
+        float sv, cv;
+        sincospif(float(e) * (1.0f / 128.0f), &sv, &cv);   // w256^e = exp(-2 pi i e / 256)
+        w256[e] = make_float2(cv, -sv);
+    }
+    __syncthreads();
+    fill_dft<16, 16, 16, kSBOc>(smem + kOffBc, w32);
+}
+
+// First operand of a forward transform from the staging Zs[l][n ^ 8 (l >> 3)]
+// (32 lines of 256 bf16 pairs): row R(l, n1), chunk c = slots n2 = 4 c .. 4 c + 3.
+// Thread (warp w, lane l) takes n1 = ((l + w) & 7) + 8 h: the 32 lanes of a
+// gather read 32 banks, and each 8 lanes store 8 rows of one row group.
+__device__ __forceinline__ void build_c(uint8_t* A, const uint32_t* Zs, int warp, int lane) {
+    const uint32_t* zl = Zs + lane * CN;
+    const int sw = 8 * (lane >> 3);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int n1 = ((lane + warp) & 7) + 8 * h;
+        const int row = rowc(lane, n1);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t q[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q[e] = zl[(n1 + 16 * (4 * c + e)) ^ sw];
+            sts128(A, tc::chunk_off(row, c, kSBOc), q[0], q[1], q[2], q[3]);
+        }
+    }
+}
+
+// Wait for a stage, then the twiddle pass: row R(l, i) (l = lane, i = 4 Q + T in
+// tile T), outputs j = 8 h .. 8 h + 7 (columns 16 h ..): value x w256^(i j) ->
+// row R(l, j), chunk Q (slots i = 4 Q .. 4 Q + 3).  The table reads are the same
+// address for the whole warp.
+__device__ __forceinline__ void pass_c(uint8_t* A, const float2* w256, uint32_t tl, int Q, int hh, int lane,
+                                       uint64_t* mbar, uint32_t& phase, bool& ok, uint64_t budget) {
+    ok = stage_wait(mbar, phase, ok, budget);
+    float d[4][16];
+#pragma unroll
+    for (int T = 0; T < 4; ++T) tc::tmem_ld16(tl + uint32_t(32 * T + 16 * hh), d[T]);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int j = 8 * hh + 2 * p;
+        C2 v[4];
+#pragma unroll
+        for (int T = 0; T < 4; ++T) {
+            const int i = 4 * Q + T;
+            v[T] = cmul2(c2_at(d[T], p), c2_of(w256[(i * j) & (CN - 1)], w256[(i * (j + 1)) & (CN - 1)]));
+        }
+        sts128(A, tc::chunk_off(rowc(lane, j), Q, kSBOc), pack_bf16(v[0].re.x, v[0].im.x),
+               pack_bf16(v[1].re.x, v[1].im.x), pack_bf16(v[2].re.x, v[2].im.x), pack_bf16(v[3].re.x, v[3].im.x));
+        sts128(A, tc::chunk_off(rowc(lane, j + 1), Q, kSBOc), pack_bf16(v[0].re.y, v[0].im.y),
+               pack_bf16(v[1].re.y, v[1].im.y), pack_bf16(v[2].re.y, v[2].im.y), pack_bf16(v[3].re.y, v[3].im.y));
+    }
+}
+
+// One DFT16 stage over the four tiles (K 32 -> N 32 each).
+__device__ __forceinline__ void issue_c(uint32_t a_addr, uint32_t b_addr, uint32_t tmem, uint64_t* mbar, bool go) {
+    stage_issue(a_addr, kSBOc, b_addr, kSBOc, 4, 2, tc::idesc_bf16(128, 32), tmem, 32, mbar, go);
+}
+
+// Common prologue of the circular kernels: tables, header check, barrier and
+// tensor memory.  Returns false (status reported) on a header mismatch.
+__device__ __forceinline__ bool prologue_c(uint8_t* smem, float2* w256, bool hdr_ok, uint64_t* mbar,
+                                           uint32_t* tmem_base, uint32_t* status) {
+    setup_tables_c(smem, w256);
+    if (!hdr_ok) {
+        if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
+        return false;
+    }
+    if (threadIdx.x == 0) tc::mbar_init(mbar, 1);
+    if ((threadIdx.x >> 5) == 0) tc::tmem_alloc(tmem_base, kTmemColsC);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    return true;
+}
+
+__device__ __forceinline__ bool header_c(const uint8_t* spectrum, bool check_plane, int64_t plane_off) {
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
+    return (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D_CIRC) & (hv.H == CN) & (hv.W == CN) &
+           (!check_plane | (hv.reserved[1] == plane_off));
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv_bfloat162* __restrict__ ws,
+                  const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
+                  int64_t ws_pair_stride, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_cf[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const bool hdr_ok = header_c(spectrum, false, 0);
+    uint8_t* A = smem_cf;
+    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cf + kOffStC);   // gated rows, then the output staging
+    float2* w256 = reinterpret_cast<float2*>(smem_cf + kOffW256);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    if (!prologue_c(smem_cf, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t b_addr = tc::smem_u32(smem_cf + kOffBc);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(CN) * CN;
+    const int ntasks = npairs * (CN / NROW);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
+        const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
+        const int64_t rowoff = int64_t(NROW * rg) * CN;
+        if (zsrc == nullptr) {
+            const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
+            const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
+            stage_pair_rows<true>(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
+        } else {
+            const bf16* z0 = zsrc + (b0 * C + c) * n_img + rowoff;
+            stage_pair_rows<false>(Zs, z0, z0 + C * n_img, nullptr, nullptr, t);
+        }
+        __syncthreads();
+        build_c(A, Zs, warp, lane);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // rows R(r, k1 = 4 Q + T), bins k2 = 8 h + ..: staging Os[k][r] (a warp's 32
+        // lanes are 32 consecutive words), then 128-byte rows Z[k][32 rg .. 32 rg + 31]
+        uint32_t* Os = Zs;
+#pragma unroll
+        for (int T = 0; T < 4; ++T) {
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(32 * T + 16 * hh), d);
+            tc::tmem_ld_wait();
+            const int k1 = 4 * Q + T;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int k = k1 + 16 * (8 * hh + 2 * p + e);
+                    Os[k * NROW + lane] = ok ? pack_bf16(d[4 * p + e], d[4 * p + 2 + e]) : 0x7fc07fc0u;
+                }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        uint32_t* wsp = reinterpret_cast<uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg;
+#pragma unroll
+        for (int kk = 0; kk < CN * NROW / 4 / NT; ++kk) {
+            const int gi = t + NT * kk, k = gi >> 3, g4 = gi & 7;
+            *reinterpret_cast<uint4*>(wsp + int64_t(k) * CN + 4 * g4) =
+                *reinterpret_cast<const uint4*>(Os + k * NROW + 4 * g4);
+        }
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectrum, int64_t nb2, int step,
+              int64_t pair0, int npairs, int64_t ws_pair_stride, int64_t plane_off, int64_t SC,
+              uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_cc[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const bool hdr_ok = header_c(spectrum, true, plane_off);
+    uint8_t* A = smem_cc;
+    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cc + kOffStC);   // input columns, then the output staging
+    float2* w256 = reinterpret_cast<float2*>(smem_cc + kOffW256);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    if (!prologue_c(smem_cc, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t b_addr = tc::smem_u32(smem_cc + kOffBc);
+    const uint4* plane = reinterpret_cast<const uint4*>(spectrum + plane_off);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int ntasks = npairs * (CN / NROW);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (CN / NROW), fg = task - lp * (CN / NROW);
+        const int64_t c = (pair0 + lp) / nb2;
+        uint32_t* col0 = reinterpret_cast<uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + int64_t(NROW * fg) * CN;
+        const uint4* kq = plane + ((int64_t(step) * SC + c) * (CN / NROW) + fg) * (kPlaneTaskC / 4) +
+                          (Q * 2 + hh) * 256 + lane;
+        // the task's 32 columns (contiguous) -> Zs[l][m ^ 8 (l >> 3)]
+#pragma unroll
+        for (int kk = 0; kk < NROW * CN / 4 / NT; ++kk) {
+            const int gi = t + NT * kk, l = gi >> 6, m0 = 4 * (gi & 63);
+            *reinterpret_cast<uint4*>(Zs + l * CN + (m0 ^ (8 * (l >> 3)))) =
+                __ldg(reinterpret_cast<const uint4*>(col0) + gi);
+        }
+        __syncthreads();
+        build_c(A, Zs, warp, lane);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        {
+            // rows R(l, k1 = 4 Q + T), bins k2 = 8 h + 4 half + e: conj(X K~) to the same
+            // row, chunk 2 h + half (the operand of the inverse stage over k2)
+            uint4 kv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) kv[i] = __ldg(kq + 32 * i);
+            ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+#pragma unroll
+            for (int T = 0; T < 4; ++T) {
+                float d[16];
+                tc::tmem_ld16(tl + uint32_t(32 * T + 16 * hh), d);
+                tc::tmem_ld_wait();
+                const int row = rowc(lane, 4 * Q + T);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const uint4 kk = kv[2 * T + half];
+                    const C2 K0{make_float2(bf_lo(kk.x), bf_lo(kk.y)), make_float2(bf_hi(kk.x), bf_hi(kk.y))};
+                    const C2 K1{make_float2(bf_lo(kk.z), bf_lo(kk.w)), make_float2(bf_hi(kk.z), bf_hi(kk.w))};
+                    const C2 v0 = cmul2(c2_at(d, 2 * half), K0);
+                    const C2 v1 = cmul2(c2_at(d, 2 * half + 1), K1);
+                    sts128(A, tc::chunk_off(row, 2 * hh + half, kSBOc), pack_bf16(v0.re.x, -v0.im.x),
+                           pack_bf16(v0.re.y, -v0.im.y), pack_bf16(v1.re.x, -v1.im.x), pack_bf16(v1.re.y, -v1.im.y));
+                }
+            }
+        }
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // conj of the result at row R(l, n1 = 4 Q + T), output n2: word m = n1 + 16 n2 of
+        // line l at Vs[l][m ^ l] (32 banks for the 32 lanes), then the 32 columns back
+        uint32_t* Vs = Zs;
+#pragma unroll
+        for (int T = 0; T < 4; ++T) {
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(32 * T + 16 * hh), d);
+            tc::tmem_ld_wait();
+            const int n1 = 4 * Q + T;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int m = n1 + 16 * (8 * hh + 2 * p + e);
+                    Vs[lane * CN + (m ^ lane)] = ok ? pack_bf16(d[4 * p + e], -d[4 * p + 2 + e]) : 0x7fc07fc0u;
+                }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        {
+            // 16-byte group g of line l is group g ^ (l >> 2) with its words permuted by l & 3
+            uint4* dst = reinterpret_cast<uint4*>(col0);
+#pragma unroll
+            for (int kk = 0; kk < NROW * CN / 4 / NT; ++kk) {
+                const int gi = t + NT * kk, l = gi >> 6, g = gi & 63;
+                uint4 v = *reinterpret_cast<const uint4*>(Vs + l * CN + 4 * (g ^ (l >> 2)));
+                if (l & 1) v = make_uint4(v.y, v.x, v.w, v.z);
+                if (l & 2) v = make_uint4(v.z, v.w, v.x, v.y);
+                dst[gi] = v;
+            }
+        }
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
+}
+
+__global__ void __launch_bounds__(NT, 2)
+k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bfloat162* __restrict__ ws,
+                  const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int gchunk, int64_t pair0,
+                  int npairs, int64_t ws_pair_stride, uint64_t wait_budget_ns, int issue_mma, uint32_t* status) {
+    extern __shared__ __align__(1024) uint8_t smem_ci[];
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const bool hdr_ok = header_c(spectrum, false, 0);
+    uint8_t* A = smem_ci;
+    uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ci + kOffStC);   // output staging [r][n ^ r]
+    float2* w256 = reinterpret_cast<float2*>(smem_ci + kOffW256);
+    const int t = threadIdx.x;
+    const int warp = t >> 5, lane = t & 31;
+    const int Q = warp & 3, hh = warp >> 2;
+    if (!prologue_c(smem_ci, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    const uint32_t tmem = tmem_base;
+    const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
+    const uint32_t a_addr = tc::smem_u32(A);
+    const uint32_t b_addr = tc::smem_u32(smem_ci + kOffBc);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(CN) * CN;
+    const int ntasks = npairs * (CN / NROW);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
+        const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
+        {
+            // conj Y[k1 + 16 k2][r] at row R(r, k1), chunk k2 / 4; lane = r, the 32 loads
+            // of a thread in flight together
+            const uint32_t* wsp = reinterpret_cast<const uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg + lane;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int ci = warp + 8 * m, k1 = ci & 15, ch = ci >> 4;
+                uint32_t q[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) q[e] = wsp[int64_t(k1 + 16 * (4 * ch + e)) * CN] ^ 0x80000000u;
+                sts128(A, tc::chunk_off(rowc(lane, k1), ch, kSBOc), q[0], q[1], q[2], q[3]);
+            }
+        }
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
+        // 2 conj(D) at row R(r, n1 = 4 Q + T), output n2: (image b0, image b1) of row r,
+        // column n = n1 + 16 n2 -> Ys[r][n ^ r]
+#pragma unroll
+        for (int T = 0; T < 4; ++T) {
+            float d[16];
+            tc::tmem_ld16(tl + uint32_t(32 * T + 16 * hh), d);
+            tc::tmem_ld_wait();
+            const int n1 = 4 * Q + T;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int n = n1 + 16 * (8 * hh + 2 * p + e);
+                    Ys[lane * CN + (n ^ lane)] = pack_bf16(2.0f * d[4 * p + e], -2.0f * d[4 * p + 2 + e]);
+                }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        {
+            const int64_t rowoff = int64_t(NROW * rg) * CN;
+            const bf16* xa = u + (b0 * Ctot + int64_t(gchunk) * C + c) * n_img + rowoff;
+            bf16* ya = y + (b0 * C + c) * n_img + rowoff;
+            gate_store_pair_rows(Ys, xa, xa + Ctot * n_img, ya, ya + C * n_img, t, ok);
+        }
+        if (__syncthreads_or(!ok)) {
+            if (t == 0) report_status(status, kStatusTimeout);
+            break;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
 }
 
 }  // namespace
@@ -748,6 +1187,57 @@ cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, 
         k_2d_rows_inv_tc<<<grid, NT, kSmem, s>>>(u, y, w, a.spectrum, a.B, p.C, p.order,
                                                  st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs), pstride,
                                                  a.wait_budget_ns, a.issue_mma, a.status);
+    }
+    return cudaGetLastError();
+}
+
+
+bool pairs_2dc_tc_path(const Plan& p, const ConvArgs& a) {
+    return p.path == PATH_GRID_2D_CIRC && p.H == CN && p.W == CN && a.g2_plane_off != 0 && a.dtype == DT_BF16 &&
+           !a.fp32_transform && p.order <= kMaxOrderTc && a.B % 2 == 0 && a.spec_per_b == 0;
+}
+
+cudaError_t launch_spectrum_2dc_tc_plane(const Plan& p, const uint8_t* spectrum_rows, uint8_t* plane, int64_t nrows,
+                                         cudaStream_t s) {
+    const int64_t n = nrows * int64_t(CN / NROW) * (kPlaneTaskC / 4);
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_2dc_plane_tc<<<unsigned(blocks), 256, 0, s>>>(reinterpret_cast<const float2*>(spectrum_rows),
+                                                    reinterpret_cast<uint4*>(plane), nrows,
+                                                    int64_t(p.spec_row_bytes / sizeof(float2)));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, int64_t img0, int64_t nimg,
+                                     int64_t ws_img_stride, cudaStream_t s) {
+    if (img0 % 2 != 0 || nimg % 2 != 0) return cudaErrorInvalidValue;
+    if (2 * ws_img_stride < int64_t(CN) * CN) return cudaErrorInvalidValue;   // a pair's Z[k][row]
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t npairs = nimg / 2, pair0 = img0 / 2, pstride = 2 * ws_img_stride;
+    const int64_t ntasks = npairs * (CN / NROW);
+    if (ntasks > INT32_MAX) return cudaErrorInvalidValue;
+    const unsigned grid = unsigned(ntasks < 2 * sms ? ntasks : 2 * sms);
+    cudaError_t e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2dc_cols_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_2dc_rows_inv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    if (e != cudaSuccess) return e;
+    const bf16* u = static_cast<const bf16*>(a.u);
+    bf16* y = static_cast<bf16*>(a.y);
+    __nv_bfloat162* w = static_cast<__nv_bfloat162*>(ws);
+    for (int st = 1; st < p.order; ++st) {
+        // as for the padded pairs: step st gates with x_{order-st}; a later step reads
+        // its input from y, where the previous step's inverse pass left it
+        k_2dc_rows_fwd_tc<<<grid, NT, kSmemC, s>>>(u, st == 1 ? nullptr : y, w, a.spectrum, a.B, p.C, p.order, pair0,
+                                                   int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        k_2dc_cols_tc<<<grid, NT, kSmemC, s>>>(w, a.spectrum, a.B / 2, st - 1, pair0, int(npairs), pstride,
+                                               int64_t(a.g2_plane_off), a.spec_C, a.wait_budget_ns, a.issue_mma,
+                                               a.status);
+        k_2dc_rows_inv_tc<<<grid, NT, kSmemC, s>>>(u, y, w, a.spectrum, a.B, p.C, p.order,
+                                                   st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs),
+                                                   pstride, a.wait_budget_ns, a.issue_mma, a.status);
     }
     return cudaGetLastError();
 }

@@ -168,6 +168,11 @@ bool make_plan(int64_t C, int ndim, const int64_t* sizes, int order, Plan* p, st
         p->g2_plane_off = align_up(p->total_bytes, 256);
         p->total_bytes = p->g2_plane_off + size_t(S) * size_t(C) * size_t(2 * p->W) * size_t(2 * p->H) * 4;
     }
+    if (p->path == PATH_GRID_2D_CIRC && p->H == kTc2dH && p->W == kTc2dH) {
+        // the full H x W plane of the circular transform (bf16 pairs)
+        p->g2_plane_off = align_up(p->total_bytes, 256);
+        p->total_bytes = p->g2_plane_off + size_t(S) * size_t(C) * size_t(p->W) * size_t(p->H) * 4;
+    }
     return true;
 }
 

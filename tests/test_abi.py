@@ -66,6 +66,9 @@ def test_spectrum_bytes_and_workspace(lib):
     b = lib.hyena_spectrum_bytes(256, circ, _sz(256, 128), 2)
     assert 256 * 65 * 256 * 8 <= b < 256 * 65 * 256 * 8 + (1 << 20)
     assert lib.hyena_gated_fftconv_workspace_min_bytes(256, circ, _sz(256, 128), 2) == 65 * 256 * 8
+    # at 256 x 256 also the full H x W bf16 plane of the tensor-core passes
+    b = lib.hyena_spectrum_bytes(256, circ, _sz(256, 256), 2)
+    assert 256 * (129 * 256 * 8 + 256 * 256 * 4) <= b < 256 * (129 * 256 * 8 + 256 * 256 * 4) + (1 << 20)
     assert lib.hyena_spectrum_bytes(64, 1 | 0x100, _sz(1024), 2) == 0
     # 3-D: (W+1) 2H depth lines x 2 N1 complex64 per channel; workspace 3 (W+1) H N1 complex64
     b = lib.hyena_spectrum_bytes(8, 3, _sz(16, 32, 64), 2)

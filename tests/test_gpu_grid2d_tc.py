@@ -158,3 +158,77 @@ def test_paired_images_timeout_is_reported():
     assert torch.isnan(y.float()).all()
     _conv(p, r)
     assert np.isfinite(from_torch(r.y)).all()
+
+
+def _circ(**kw):
+    return I.WORKLOADS["grid2d_circ"].with_(H=256, W=256, **kw)
+
+
+@pytest.mark.parametrize("B,C,order", [(2, 3, 2), (4, 2, 2), (2, 2, 3), (3, 2, 2), (2, 1, 4)])
+def test_circular_pairs_against_oracle(orc, B, C, order):
+    """Circular 256 x 256 images: an even batch pairs the two images of a channel
+    through tensor-core row, column and row passes (256-point transforms, two
+    16-point stages each), once per order step; an odd batch takes the
+    unpaired passes, order 4 the fp32 passes."""
+    p = _circ(B=B, C=C, order=order, seed=3800 + 10 * B + order)
+    data = I.make_all(p)
+    r = Run(p, data, False)
+    r.build_spectrum()
+    y = _conv(p, r)
+    assert np.isfinite(y).all()
+    err = _rows_err(orc, p, data, y)
+    print(f"circular B={B} order={order}: max image rel err {err.max():.3e}")
+    assert err.max() <= TOL["bf16"], err.max()
+
+
+def test_circular_pairs_against_fp32_passes(orc):
+    """The fp32 passes (flag) and the paired tensor-core passes agree within the
+    bf16 tolerance, the fp32 ones are the closer to the oracle, and the outputs
+    differ (two different kernel sets ran)."""
+    p = _circ(B=2, C=3, seed=3900)
+    data = I.make_all(p)
+    r = Run(p, data, False)
+    r.build_spectrum()
+    y_tc = _conv(p, r).copy()
+    y_32 = _conv(p, r, flags=hb.HYENA_FLAG_FP32_TRANSFORM)
+    e_tc = _rows_err(orc, p, data, y_tc).max()
+    e_32 = _rows_err(orc, p, data, y_32).max()
+    print(f"circular: tensor-core pairs {e_tc:.3e}, fp32 passes {e_32:.3e}")
+    assert e_tc <= TOL["bf16"] and e_32 <= TOL["bf16"]
+    assert e_32 < e_tc
+    assert not np.array_equal(y_tc, y_32)
+
+
+def test_circular_pairs_deterministic_and_small_workspace(orc):
+    """Bitwise repeatable; workspaces of one image (unpaired passes) and of
+    three images (one pair per group) stay within the bound."""
+    import torch
+    p = _circ(B=2, C=3, seed=4000)
+    data = I.make_all(p)
+    r = Run(p, data, False)
+    r.build_spectrum()
+    _conv(p, r)
+    a = r.y.clone()
+    _conv(p, r)
+    assert torch.equal(a, r.y)
+    row = hb.hyena_gated_fftconv_workspace_min_bytes(p.C, api_shape(p), p.order)
+    for nrows in (1, 3):
+        rs = Run(p, data, False, workspace_bytes=nrows * row)
+        rs.build_spectrum()
+        err = _rows_err(orc, p, data, _conv(p, rs))
+        assert err.max() <= TOL["bf16"], (nrows, err.max())
+
+
+def test_circular_pairs_report_a_spectrum_header_mismatch():
+    import torch
+    p = _circ(B=2, C=2, seed=4100)
+    r = Run(p, I.make_all(p), False)
+    hb.hyena_kernel_status()
+    fresh = torch.zeros_like(r.spectrum)
+    hb.hyena_gated_fftconv(r.u, r.y, fresh, None, None, p.B, p.C, api_shape(p), p.order, r.workspace)
+    with pytest.raises(hb.HyenaError) as e:
+        hb.hyena_kernel_status()
+    assert e.value.status == 4
+    r.build_spectrum()
+    _conv(p, r)
+    assert np.isfinite(from_torch(r.y)).all()
