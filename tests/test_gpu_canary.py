@@ -7,7 +7,7 @@ import pytest
 
 from fft_long_convolution_02_b200 import binding as hb
 from fft_long_convolution_02_b200 import inputs as I
-from gpu_helpers import TOL, gpu_rows, oracle_for_rows, row_rel_err, to_torch
+from gpu_helpers import TOL, api_shape, gpu_rows, oracle_for_rows, row_rel_err, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +49,7 @@ CASES = [
     I.WORKLOADS["grid2d"].with_(B=2, C=3, H=64, W=32, sigma=(4.0, 16.0), seed=6005),      # 2-D
     I.WORKLOADS["grid2d"].with_(B=3, C=2, H=256, W=64, seed=6009),                         # 2-D tensor-core columns
     I.WORKLOADS["grid2d"].with_(B=2, C=2, H=256, W=256, seed=6010),                        # 2-D paired images
+    I.WORKLOADS["grid2d_circ"].with_(B=2, C=2, H=256, W=256, seed=6011),                   # circular, paired
 ]
 
 
@@ -60,17 +61,17 @@ def test_writes_stay_inside_their_buffers(orc, p):
     k = to_torch(p, data["k"])
     D = torch.from_numpy(data["D"]).cuda()
     sc_w = torch.from_numpy(data["sc_w"]).cuda() if data["sc_w"] is not None else None
-    sb = hb.hyena_spectrum_bytes(p.C, p.shape, p.order)
+    sb = hb.hyena_spectrum_bytes(p.C, api_shape(p), p.order)
     spec_full, spec = _guarded(sb)
     es = u.element_size()
     yb = p.B * p.C * int(np.prod(p.shape)) * es
     y_full, y8 = _guarded(yb)
     y = y8.view(u.dtype).view((p.B, p.C) + p.shape)
-    wb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, p.shape, p.order)
+    wb = hb.hyena_gated_fftconv_workspace_bytes(p.B, p.C, api_shape(p), p.order)
     ws_full, ws = _guarded(wb) if wb else (None, None)
-    hb.hyena_filter_spectrum(k, D, p.C, p.shape, p.order, spec)
-    hb.hyena_gated_fftconv(u, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws)
-    hb.hyena_gated_fftconv(u, y, spec, sc_w, None, p.B, p.C, p.shape, p.order, ws)   # twice: reuse
+    hb.hyena_filter_spectrum(k, D, p.C, api_shape(p), p.order, spec)
+    hb.hyena_gated_fftconv(u, y, spec, sc_w, None, p.B, p.C, api_shape(p), p.order, ws)
+    hb.hyena_gated_fftconv(u, y, spec, sc_w, None, p.B, p.C, api_shape(p), p.order, ws)   # twice: reuse
     torch.cuda.synchronize()
     assert _guards_intact(spec_full, sb), "spectrum guard overwritten"
     assert _guards_intact(y_full, yb), "output guard overwritten"
