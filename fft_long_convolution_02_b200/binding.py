@@ -25,7 +25,7 @@ EXPORTS = ["hyena_version", "hyena_status_string", "hyena_last_error_detail", "h
            "hyena_filter_spectrum", "hyena_shortconv", "hyena_gated_fftconv_workspace_bytes",
            "hyena_gated_fftconv_workspace_min_bytes", "hyena_gated_fftconv", "hyena_gated_fftconv_noalloc",
            "hyena_gated_fftconv_per_sample", "hyena_gated_fftconv_host", "hyena_spectrum_check",
-           "hyena_debug_conv_tc", "hyena_debug_conv_cluster", "hyena_debug_conv_2d_tc", "hyena_gated_fftconv_ex", "hyena_kernel_status", "hyena_in_proj",
+           "hyena_debug_conv_tc", "hyena_debug_conv_cluster", "hyena_debug_conv_2d_tc", "hyena_debug_conv_2dc_tc", "hyena_gated_fftconv_ex", "hyena_kernel_status", "hyena_in_proj",
            "hyena_out_proj", "hyena_implicit_filter_workspace_bytes", "hyena_filter_spectrum_implicit"]
 
 _lock = threading.Lock()
@@ -103,6 +103,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.hyena_debug_conv_2d_tc.restype = ctypes.c_int
         lib.hyena_debug_conv_2d_tc.argtypes = [vp, vp, vp, sz, i64, i64, i64, ctypes.c_int, vp, sz,
                                                ctypes.c_uint64, ctypes.c_int, vp]
+        lib.hyena_debug_conv_2dc_tc.restype = ctypes.c_int
+        lib.hyena_debug_conv_2dc_tc.argtypes = [vp, vp, vp, sz, i64, i64, ctypes.c_int, vp, sz,
+                                                ctypes.c_uint64, ctypes.c_int, vp]
         _lib = lib
     return _lib
 
@@ -324,6 +327,16 @@ def hyena_debug_conv_2d_tc(u, y, spectrum, B: int, C: int, W: int, order: int, w
     _check(load().hyena_debug_conv_2d_tc(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
                                          B, C, W, order, _ptr(workspace), ws_bytes, int(wait_budget_ns),
                                          1 if issue_mma else 0, _stream(stream)))
+
+
+def hyena_debug_conv_2dc_tc(u, y, spectrum, B: int, C: int, order: int, workspace, wait_budget_ns: int,
+                            issue_mma: bool = True, stream=None) -> None:
+    """The same test hook for the circular form's paired tensor-core passes
+    (256 x 256, bf16, even B)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyena_debug_conv_2dc_tc(_ptr(u), _ptr(y), _ptr(spectrum), spectrum.numel() * spectrum.element_size(),
+                                          B, C, order, _ptr(workspace), ws_bytes, int(wait_budget_ns),
+                                          1 if issue_mma else 0, _stream(stream)))
 
 
 def hyena_debug_conv_cluster(u, y, spectrum, sc_w, sc_bias, B: int, C: int, order: int, workspace,

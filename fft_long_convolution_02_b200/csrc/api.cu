@@ -6,6 +6,7 @@
 #include <mutex>
 #include <string>
 
+#include "grid2dc_tc.h"
 #include "hyena.h"
 #include "kernels.h"
 #include "plan.h"
@@ -314,6 +315,26 @@ hyena_status_t hyena_debug_conv_2d_tc(const void* u, void* y, const void* spectr
     if (st != HYENA_OK) return st;
     if (!cols_2d_tc_path(p, a))
         return fail(HYENA_ERR_UNSUPPORTED_SHAPE, "the 2-D tensor-core column pass serves H = 256, W a multiple of 32");
+    if (wait_budget_ns == 0) return fail(HYENA_ERR_INVALID_ARG, "wait_budget_ns must be > 0");
+    a.wait_budget_ns = wait_budget_ns;
+    a.issue_mma = issue_mma ? 1 : 0;
+    cudaError_t e = kernel_status_word(&a.status);
+    if (e != cudaSuccess) return cuda_status(e, "kernel status word");
+    return cuda_status(launch_conv_2d(p, a, static_cast<cudaStream_t>(stream)), "2-D convolution");
+}
+
+hyena_status_t hyena_debug_conv_2dc_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, int64_t B,
+                                       int64_t C, int order, void* workspace, size_t workspace_bytes,
+                                       uint64_t wait_budget_ns, int issue_mma, void* stream) {
+    Plan p;
+    ConvArgs a;
+    const int64_t sizes[2] = {kTc2dH, kTc2dH};
+    hyena_status_t st = prepare_conv(u, y, spectrum, spectrum_bytes, nullptr, nullptr, B, C, 2 | kCircularFlag, sizes,
+                                     order, HYENA_BF16, workspace, workspace_bytes, &p, &a);
+    if (st != HYENA_OK) return st;
+    if (!pairs_2dc_tc_path(p, a))
+        return fail(HYENA_ERR_UNSUPPORTED_SHAPE,
+                    "the circular tensor-core passes serve 256 x 256, an even batch and order <= 3");
     if (wait_budget_ns == 0) return fail(HYENA_ERR_INVALID_ARG, "wait_budget_ns must be > 0");
     a.wait_budget_ns = wait_budget_ns;
     a.issue_mma = issue_mma ? 1 : 0;

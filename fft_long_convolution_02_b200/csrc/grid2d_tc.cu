@@ -383,24 +383,44 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
 constexpr int W2 = 256;           // image width of the paired path (row transform 512)
 constexpr int NROW = 32;          // image rows per task
 
-// z of rows r0 .. r0+31 of a pair -> staging Zs[r][n ^ (8 (r >> 3))] (bf16 pairs):
-// the XOR lets the stage-1 gather below read 32 different banks.  GATE: z =
-// x v (the first order step), else z = x (a later step's input, already gated
-// by the previous step's inverse pass).
+// Raw input rows of a task (32 rows of both images of a pair), held in
+// registers between their loads and the staging: x, and v when GATE.
+constexpr int kRowIt = NROW * W2 / 8 / NT;   // 16-byte groups of a row image per thread
 template <bool GATE>
-__device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __restrict__ x_b0, const bf16* __restrict__ x_b1,
-                                                const bf16* __restrict__ v_b0, const bf16* __restrict__ v_b1, int t) {
+struct PairRows {
+    uint4 x[kRowIt][2];
+    uint4 v[GATE ? kRowIt : 1][2];
+};
+template <bool GATE>
+__device__ __forceinline__ void load_pair_rows(PairRows<GATE>& in, const bf16* __restrict__ x_b0,
+                                               const bf16* __restrict__ x_b1, const bf16* __restrict__ v_b0,
+                                               const bf16* __restrict__ v_b1, int t) {
 #pragma unroll
-    for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
+    for (int jj = 0; jj < kRowIt; ++jj) {
         const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
         const int64_t off = int64_t(r) * W2 + n0;
-        const uint4 xa = __ldg(reinterpret_cast<const uint4*>(x_b0 + off));
-        const uint4 xb = __ldg(reinterpret_cast<const uint4*>(x_b1 + off));
+        in.x[jj][0] = __ldg(reinterpret_cast<const uint4*>(x_b0 + off));
+        in.x[jj][1] = __ldg(reinterpret_cast<const uint4*>(x_b1 + off));
+        if constexpr (GATE) {
+            in.v[jj][0] = __ldg(reinterpret_cast<const uint4*>(v_b0 + off));
+            in.v[jj][1] = __ldg(reinterpret_cast<const uint4*>(v_b1 + off));
+        }
+    }
+}
+// z of the task's rows -> staging Zs[r][n ^ (8 (r >> 3))] (bf16 pairs (z[b0], z[b1])):
+// the XOR lets the stage-1 gathers read 32 different banks.  GATE: z = x v (the
+// first order step), else z = x (a later step's input, already gated by the
+// previous step's inverse pass).
+template <bool GATE>
+__device__ __forceinline__ void store_pair_rows(uint32_t* Zs, const PairRows<GATE>& in, int t) {
+#pragma unroll
+    for (int jj = 0; jj < kRowIt; ++jj) {
+        const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
+        const uint4 xa = in.x[jj][0], xb = in.x[jj][1];
         const uint32_t xw[2][4] = {{xa.x, xa.y, xa.z, xa.w}, {xb.x, xb.y, xb.z, xb.w}};
         uint32_t o[8];
         if constexpr (GATE) {
-            const uint4 va = __ldg(reinterpret_cast<const uint4*>(v_b0 + off));
-            const uint4 vb = __ldg(reinterpret_cast<const uint4*>(v_b1 + off));
+            const uint4 va = in.v[jj][0], vb = in.v[jj][1];
             const uint32_t vw[2][4] = {{va.x, va.y, va.z, va.w}, {vb.x, vb.y, vb.z, vb.w}};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -425,19 +445,35 @@ __device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __rest
         *reinterpret_cast<uint4*>(dst + 4) = make_uint4(o[4], o[5], o[6], o[7]);
     }
 }
+template <bool GATE>
+__device__ __forceinline__ void stage_pair_rows(uint32_t* Zs, const bf16* __restrict__ x_b0, const bf16* __restrict__ x_b1,
+                                                const bf16* __restrict__ v_b0, const bf16* __restrict__ v_b1, int t) {
+    PairRows<GATE> in;
+    load_pair_rows<GATE>(in, x_b0, x_b1, v_b0, v_b1, t);
+    store_pair_rows<GATE>(Zs, in, t);
+}
 
-// Output gate of 32 rows of a pair: staged result Ys[r][n ^ r] (bf16 pairs
-// (image b0, image b1)) times the gate rows x_b0 / x_b1, stored to y_b0 / y_b1
-// (rows of W2 samples), 8 columns of a row per step; NaN once a wait ran out.
-__device__ __forceinline__ void gate_store_pair_rows(const uint32_t* Ys, const bf16* __restrict__ xa,
-                                                     const bf16* __restrict__ xb, bf16* __restrict__ ya,
-                                                     bf16* __restrict__ yb, int t, bool ok) {
+// Output gate of 32 rows of a pair: the gate rows x_b0 / x_b1 (loaded into
+// gx first, so that their loads can be issued early), times the staged result
+// Ys[r][n ^ r] (bf16 pairs (image b0, image b1)), stored to y_b0 / y_b1 (rows of
+// W2 samples), 8 columns of a row per step; NaN once a wait ran out.
+__device__ __forceinline__ void load_gate_rows(uint4 (&gx)[kRowIt][2], const bf16* __restrict__ xa,
+                                               const bf16* __restrict__ xb, int t) {
 #pragma unroll
-    for (int jj = 0; jj < NROW * W2 / 8 / NT; ++jj) {
+    for (int jj = 0; jj < kRowIt; ++jj) {
         const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
         const int64_t off = int64_t(r) * W2 + n0;
-        const uint4 x0a = __ldg(reinterpret_cast<const uint4*>(xa + off));
-        const uint4 x0b = __ldg(reinterpret_cast<const uint4*>(xb + off));
+        gx[jj][0] = __ldg(reinterpret_cast<const uint4*>(xa + off));
+        gx[jj][1] = __ldg(reinterpret_cast<const uint4*>(xb + off));
+    }
+}
+__device__ __forceinline__ void apply_gate_rows(const uint32_t* Ys, const uint4 (&gx)[kRowIt][2], bf16* __restrict__ ya,
+                                                bf16* __restrict__ yb, int t, bool ok) {
+#pragma unroll
+    for (int jj = 0; jj < kRowIt; ++jj) {
+        const int ci = t + NT * jj, r = ci >> 5, n0 = 8 * (ci & 31);
+        const int64_t off = int64_t(r) * W2 + n0;
+        const uint4 x0a = gx[jj][0], x0b = gx[jj][1];
         // word n0 + i sits at (n0 ^ (r & 24)) + (i ^ (r & 7))
         const uint32_t* src = Ys + r * W2 + (n0 ^ (r & 24));
         const uint4 g0 = *reinterpret_cast<const uint4*>(src);
@@ -474,6 +510,13 @@ __device__ __forceinline__ void gate_store_pair_rows(const uint32_t* Ys, const b
         *reinterpret_cast<uint4*>(ya + off) = ok ? make_uint4(oa[0], oa[1], oa[2], oa[3]) : nan4;
         *reinterpret_cast<uint4*>(yb + off) = ok ? make_uint4(ob[0], ob[1], ob[2], ob[3]) : nan4;
     }
+}
+__device__ __forceinline__ void gate_store_pair_rows(const uint32_t* Ys, const bf16* __restrict__ xa,
+                                                     const bf16* __restrict__ xb, bf16* __restrict__ ya,
+                                                     bf16* __restrict__ yb, int t, bool ok) {
+    uint4 gx[kRowIt][2];
+    load_gate_rows(gx, xa, xb, t);
+    apply_gate_rows(Ys, gx, ya, yb, t, ok);
 }
 
 __global__ void __launch_bounds__(NT, 2)
@@ -845,6 +888,8 @@ __device__ __forceinline__ bool header_c(const uint8_t* spectrum, bool check_pla
            (!check_plane | (hv.reserved[1] == plane_off));
 }
 
+// GATE: the first order step (z = x_{order-1} v from u); else z from zsrc.
+template <bool GATE>
 __global__ void __launch_bounds__(NT, 2)
 k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv_bfloat162* __restrict__ ws,
                   const uint8_t* __restrict__ spectrum, int64_t B, int64_t C, int order, int64_t pair0, int npairs,
@@ -868,12 +913,11 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
     bool ok = true;
     const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(CN) * CN;
     const int ntasks = npairs * (CN / NROW);
-
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
         const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
         const int64_t rowoff = int64_t(NROW * rg) * CN;
-        if (zsrc == nullptr) {
+        if constexpr (GATE) {
             const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
             const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
             stage_pair_rows<true>(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
@@ -907,7 +951,7 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
         tc::fence_before_sync();
         __syncthreads();
         uint32_t* wsp = reinterpret_cast<uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg;
-#pragma unroll
+#pragma unroll 4
         for (int kk = 0; kk < CN * NROW / 4 / NT; ++kk) {
             const int gi = t + NT * kk, k = gi >> 3, g4 = gi & 7;
             *reinterpret_cast<uint4*>(wsp + int64_t(k) * CN + 4 * g4) =
@@ -1078,6 +1122,11 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
         issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
         pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        // the gate rows (x_gchunk of both images) are on their way while the last stage runs
+        const int64_t rowoff = int64_t(NROW * rg) * CN;
+        const bf16* xa = u + (b0 * Ctot + int64_t(gchunk) * C + c) * n_img + rowoff;
+        uint4 gx[kRowIt][2];
+        load_gate_rows(gx, xa, xa + Ctot * n_img, t);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         // 2 conj(D) at row R(r, n1 = 4 Q + T), output n2: (image b0, image b1) of row r,
         // column n = n1 + 16 n2 -> Ys[r][n ^ r]
@@ -1098,10 +1147,8 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
         tc::fence_before_sync();
         __syncthreads();
         {
-            const int64_t rowoff = int64_t(NROW * rg) * CN;
-            const bf16* xa = u + (b0 * Ctot + int64_t(gchunk) * C + c) * n_img + rowoff;
             bf16* ya = y + (b0 * C + c) * n_img + rowoff;
-            gate_store_pair_rows(Ys, xa, xa + Ctot * n_img, ya, ya + C * n_img, t, ok);
+            apply_gate_rows(Ys, gx, ya, ya + C * n_img, t, ok);
         }
         if (__syncthreads_or(!ok)) {
             if (t == 0) report_status(status, kStatusTimeout);
@@ -1219,7 +1266,9 @@ cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws,
     const int64_t ntasks = npairs * (CN / NROW);
     if (ntasks > INT32_MAX) return cudaErrorInvalidValue;
     const unsigned grid = unsigned(ntasks < 2 * sms ? ntasks : 2 * sms);
-    cudaError_t e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    cudaError_t e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2dc_cols_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_2dc_rows_inv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
@@ -1230,8 +1279,9 @@ cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws,
     for (int st = 1; st < p.order; ++st) {
         // as for the padded pairs: step st gates with x_{order-st}; a later step reads
         // its input from y, where the previous step's inverse pass left it
-        k_2dc_rows_fwd_tc<<<grid, NT, kSmemC, s>>>(u, st == 1 ? nullptr : y, w, a.spectrum, a.B, p.C, p.order, pair0,
-                                                   int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        (st == 1 ? k_2dc_rows_fwd_tc<true> : k_2dc_rows_fwd_tc<false>)<<<grid, NT, kSmemC, s>>>(
+            u, y, w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride, a.wait_budget_ns, a.issue_mma,
+            a.status);
         k_2dc_cols_tc<<<grid, NT, kSmemC, s>>>(w, a.spectrum, a.B / 2, st - 1, pair0, int(npairs), pstride,
                                                int64_t(a.g2_plane_off), a.spec_C, a.wait_budget_ns, a.issue_mma,
                                                a.status);

@@ -42,7 +42,10 @@
  *    way, with the spectrum read as bf16 pairs (order <= 3); for 256 x 256
  *    images with an even batch and shared filters the two images of a channel
  *    travel as one complex image and the row transforms run there too (image
- *    error a few 1e-3); HYENA_FLAG_FP32_TRANSFORM selects the fp32 passes.
+ *    error a few 1e-3); the circular form at 256 x 256 (bf16, even batch,
+ *    shared filters, order <= 3) runs its 256-point row and column
+ *    transforms the same way, the images paired; HYENA_FLAG_FP32_TRANSFORM
+ *    selects the fp32 passes.
  *    With bf16 storage the intermediate of the multi-pass (L >= 32768) and
  *    N-D paths is kept as bf16 pairs in the workspace.
  *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
@@ -246,8 +249,8 @@ hyena_status_t hyena_gated_fftconv(const void* u, void* y, const void* spectrum,
 
 /* Flags of hyena_gated_fftconv_ex. */
 #define HYENA_FLAG_FP32_TRANSFORM 0x1u  /* every transform multiply in fp32 on the CUDA cores (no bf16 tensor-core
-                                           operands); changes only 1-D L = 8192 and 65536 and 2-D H = 256 with
-                                           bf16 storage */
+                                           operands); changes only 1-D L = 8192 and 65536, 2-D H = 256 and the
+                                           circular 2-D 256 x 256 form with bf16 storage */
 
 /*
  * hyena_gated_fftconv_ex -- hyena_gated_fftconv with flags (shared filters).
@@ -465,6 +468,19 @@ hyena_status_t hyena_debug_conv_cluster(const void* u, void* y, const void* spec
 hyena_status_t hyena_debug_conv_2d_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, int64_t B,
                                       int64_t C, int64_t W, int order, void* workspace, size_t workspace_bytes,
                                       uint64_t wait_budget_ns, int issue_mma, void* stream);
+
+/*
+ * The same test hook for the circular form's paired tensor-core passes
+ * (ndim = 2 | HYENA_CIRCULAR, sizes = {256, 256}, bf16 storage, even B, shared
+ * filters, order <= 3; spectrum and workspace as in hyena_gated_fftconv):
+ * the whole circular convolution runs with the waits of its three kernels
+ * bounded by wait_budget_ns and, for issue_mma = 0, no tensor-core work
+ * issued; a CTA whose wait ran out writes NaN and stops.  Other arguments
+ * return HYENA_ERR_UNSUPPORTED_SHAPE.
+ */
+hyena_status_t hyena_debug_conv_2dc_tc(const void* u, void* y, const void* spectrum, size_t spectrum_bytes, int64_t B,
+                                       int64_t C, int order, void* workspace, size_t workspace_bytes,
+                                       uint64_t wait_budget_ns, int issue_mma, void* stream);
 
 #ifdef __cplusplus
 }

@@ -232,3 +232,23 @@ def test_circular_pairs_report_a_spectrum_header_mismatch():
     r.build_spectrum()
     _conv(p, r)
     assert np.isfinite(from_torch(r.y)).all()
+
+
+def test_circular_pairs_timeout_is_reported():
+    """The circular paired passes' bounded waits: no tensor-core work issued,
+    1 ms budget: HYENA_ERR_TIMEOUT, NaN outputs, the next call correct."""
+    import torch
+    p = _circ(B=2, C=2, seed=4200)
+    r = Run(p, I.make_all(p), False)
+    r.build_spectrum()
+    hb.hyena_kernel_status()
+    y = torch.zeros_like(r.y)
+    hb.hyena_debug_conv_2dc_tc(r.u, y, r.spectrum, p.B, p.C, p.order, r.workspace, wait_budget_ns=1_000_000,
+                               issue_mma=False)
+    torch.cuda.synchronize()
+    with pytest.raises(hb.HyenaError) as ei:
+        hb.hyena_kernel_status()
+    assert ei.value.status == 8
+    assert torch.isnan(y.float()).all()
+    _conv(p, r)
+    assert np.isfinite(from_torch(r.y)).all()
