@@ -757,6 +757,13 @@ constexpr size_t kSmemC = size_t(kOffW256) + CN * sizeof(float2);
 constexpr uint32_t kTmemColsC = 128;             // 4 tiles x 32 columns
 constexpr int kPlaneTaskC = NROW * CN;           // bf16 pairs of the plane per column task
 static_assert(kOffStC % 16 == 0 && kOffW256 % 16 == 0, "table alignment");
+// the rows-forward kernel stages the raw rows of x and v of both images (four
+// 16 KB planes) in place of the 32 KB staging, its tables after them
+constexpr uint32_t kRawPlane = NROW * CN * 2;
+constexpr uint32_t kOffBcF = kOffStC + 4 * kRawPlane;
+constexpr uint32_t kOffW256F = kOffBcF + 4 * kSBOc;
+constexpr size_t kSmemCF = size_t(kOffW256F) + CN * sizeof(float2);
+static_assert(2 * (kSmemCF + 2048) <= 227 * 1024, "two rows-forward CTAs per SM");
 
 __device__ __forceinline__ int rowc(int l, int i) { return 128 * (i & 3) + 32 * (i >> 2) + l; }
 
@@ -800,6 +807,7 @@ __global__ void k_2dc_plane_tc(const float2* __restrict__ rows, uint4* __restric
 }
 
 // Tables: the real form of the 16-point DFT matrix (B operand) and w256^e.
+template <uint32_t OFF_B>
 __device__ __forceinline__ void setup_tables_c(uint8_t* smem, float2* w256) {
     float2* w32 = reinterpret_cast<float2*>(smem);
     fill_w32(w32);
@@ -809,7 +817,7 @@ __device__ __forceinline__ void setup_tables_c(uint8_t* smem, float2* w256) {
         w256[e] = make_float2(cv, -sv);
     }
     __syncthreads();
-    fill_dft<16, 16, 16, kSBOc>(smem + kOffBc, w32);
+    fill_dft<16, 16, 16, kSBOc>(smem + OFF_B, w32);
 }
 
 // First operand of a forward transform from the staging Zs[l][n ^ 8 (l >> 3)]
@@ -867,9 +875,10 @@ __device__ __forceinline__ void issue_c(uint32_t a_addr, uint32_t b_addr, uint32
 
 // Common prologue of the circular kernels: tables, header check, barrier and
 // tensor memory.  Returns false (status reported) on a header mismatch.
+template <uint32_t OFF_B = kOffBc>
 __device__ __forceinline__ bool prologue_c(uint8_t* smem, float2* w256, bool hdr_ok, uint64_t* mbar,
                                            uint32_t* tmem_base, uint32_t* status) {
-    setup_tables_c(smem, w256);
+    setup_tables_c<OFF_B>(smem, w256);
     if (!hdr_ok) {
         if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return false;
@@ -899,41 +908,75 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
     __shared__ uint32_t tmem_base;
     const bool hdr_ok = header_c(spectrum, false, 0);
     uint8_t* A = smem_cf;
-    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cf + kOffStC);   // gated rows, then the output staging
-    float2* w256 = reinterpret_cast<float2*>(smem_cf + kOffW256);
+    uint8_t* Rw = smem_cf + kOffStC;                                 // raw rows: x_b0, x_b1 (, v_b0, v_b1)
+    uint32_t* Zs = reinterpret_cast<uint32_t*>(Rw);                  // gated rows (over the raw ones)
+    uint32_t* Os = reinterpret_cast<uint32_t*>(smem_cf);             // output staging (the operand area)
+    float2* w256 = reinterpret_cast<float2*>(smem_cf + kOffW256F);
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    if (!prologue_c(smem_cf, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    if (!prologue_c<kOffBcF>(smem_cf, w256, hdr_ok, &mbar, &tmem_base, status)) return;
     const uint32_t tmem = tmem_base;
     const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
     const uint32_t a_addr = tc::smem_u32(A);
-    const uint32_t b_addr = tc::smem_u32(smem_cf + kOffBc);
+    const uint32_t b_addr = tc::smem_u32(smem_cf + kOffBcF);
     uint32_t phase = 0;
     bool ok = true;
     const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(CN) * CN;
     const int ntasks = npairs * (CN / NROW);
-    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+    // a task's raw rows (each plane 16 KB contiguous) into Rw by cp.async: the next
+    // task's are copied while this one is transformed
+    constexpr int kPlanes = GATE ? 4 : 2;
+    auto stage_raw = [&](int task) {
         const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
         const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
         const int64_t rowoff = int64_t(NROW * rg) * CN;
-        if constexpr (GATE) {
-            const bf16* x0 = u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff;
-            const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
-            stage_pair_rows<true>(Zs, x0, x0 + Ctot * n_img, v0, v0 + Ctot * n_img, t);
-        } else {
-            const bf16* z0 = zsrc + (b0 * C + c) * n_img + rowoff;
-            stage_pair_rows<false>(Zs, z0, z0 + C * n_img, nullptr, nullptr, t);
+        const bf16* x0 = GATE ? u + (b0 * Ctot + int64_t(order - 1) * C + c) * n_img + rowoff
+                              : zsrc + (b0 * C + c) * n_img + rowoff;
+        const int64_t xs = GATE ? Ctot * n_img : C * n_img;                  // image b0 -> b0 + 1
+        const bf16* v0 = u + (b0 * Ctot + int64_t(order) * C + c) * n_img + rowoff;
+#pragma unroll
+        for (int pl = 0; pl < kPlanes; ++pl) {
+            const bf16* src = (pl < 2 ? x0 : v0) + (pl & 1) * xs;
+#pragma unroll
+            for (int kk = 0; kk < int(kRawPlane / 16) / NT; ++kk) {
+                const int gi = t + NT * kk;
+                cp_async_bytes16(Rw + pl * kRawPlane + 16 * gi, reinterpret_cast<const uint4*>(src) + gi);
+            }
+        }
+        cp_async_commit();
+    };
+    if (int(blockIdx.x) < ntasks) stage_raw(blockIdx.x);
+
+    for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
+        cp_async_wait_all();
+        __syncthreads();
+        {
+            // this thread's raw values into registers, then (every thread done reading) the
+            // gated rows over them
+            PairRows<GATE> in;
+#pragma unroll
+            for (int jj = 0; jj < kRowIt; ++jj) {
+                const int ci = t + NT * jj;                 // 16-byte group ci of a plane
+#pragma unroll
+                for (int im = 0; im < 2; ++im) {
+                    in.x[jj][im] = *reinterpret_cast<const uint4*>(Rw + im * kRawPlane + 16 * ci);
+                    if constexpr (GATE) in.v[jj][im] = *reinterpret_cast<const uint4*>(Rw + (2 + im) * kRawPlane + 16 * ci);
+                }
+            }
+            __syncthreads();
+            store_pair_rows<GATE>(Zs, in, t);
         }
         __syncthreads();
         build_c(A, Zs, warp, lane);
-        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);   // every thread is past its build: Rw is free
+        if (task + int(gridDim.x) < ntasks) stage_raw(task + int(gridDim.x));
         pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         // rows R(r, k1 = 4 Q + T), bins k2 = 8 h + ..: staging Os[k][r] (a warp's 32
         // lanes are 32 consecutive words), then 128-byte rows Z[k][32 rg .. 32 rg + 31]
-        uint32_t* Os = Zs;
 #pragma unroll
         for (int T = 0; T < 4; ++T) {
             float d[16];
@@ -962,6 +1005,7 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
             break;
         }
     }
+    cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
@@ -976,7 +1020,8 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
     __shared__ uint32_t tmem_base;
     const bool hdr_ok = header_c(spectrum, true, plane_off);
     uint8_t* A = smem_cc;
-    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cc + kOffStC);   // input columns, then the output staging
+    uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cc + kOffStC);   // input columns
+    uint32_t* Vs = reinterpret_cast<uint32_t*>(smem_cc);             // output staging (the operand area)
     float2* w256 = reinterpret_cast<float2*>(smem_cc + kOffW256);
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
@@ -991,22 +1036,33 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
     bool ok = true;
     const int ntasks = npairs * (CN / NROW);
 
+    // a task's 32 columns (contiguous in the workspace) -> Zs[l][m ^ 8 (l >> 3)] by
+    // cp.async: the next task's are copied while this one is transformed
+    auto stage_cols = [&](int task) {
+        const int lp = task / (CN / NROW), fg = task - lp * (CN / NROW);
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint32_t*>(
+                                                              ws + int64_t(lp) * ws_pair_stride) +
+                                                          int64_t(NROW * fg) * CN);
+#pragma unroll
+        for (int kk = 0; kk < NROW * CN / 4 / NT; ++kk) {
+            const int gi = t + NT * kk, l = gi >> 6, m0 = 4 * (gi & 63);
+            cp_async_bytes16(Zs + l * CN + (m0 ^ (8 * (l >> 3))), src + gi);
+        }
+        cp_async_commit();
+    };
+    if (int(blockIdx.x) < ntasks) stage_cols(blockIdx.x);
+
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int lp = task / (CN / NROW), fg = task - lp * (CN / NROW);
         const int64_t c = (pair0 + lp) / nb2;
         uint32_t* col0 = reinterpret_cast<uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + int64_t(NROW * fg) * CN;
         const uint4* kq = plane + ((int64_t(step) * SC + c) * (CN / NROW) + fg) * (kPlaneTaskC / 4) +
                           (Q * 2 + hh) * 256 + lane;
-        // the task's 32 columns (contiguous) -> Zs[l][m ^ 8 (l >> 3)]
-#pragma unroll
-        for (int kk = 0; kk < NROW * CN / 4 / NT; ++kk) {
-            const int gi = t + NT * kk, l = gi >> 6, m0 = 4 * (gi & 63);
-            *reinterpret_cast<uint4*>(Zs + l * CN + (m0 ^ (8 * (l >> 3)))) =
-                __ldg(reinterpret_cast<const uint4*>(col0) + gi);
-        }
+        cp_async_wait_all();
         __syncthreads();
         build_c(A, Zs, warp, lane);
-        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);   // every thread is past its build: Zs is free
+        if (task + int(gridDim.x) < ntasks) stage_cols(task + int(gridDim.x));
         pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
         {
@@ -1040,7 +1096,6 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
         ok = stage_wait(&mbar, phase, ok, wait_budget_ns);
         // conj of the result at row R(l, n1 = 4 Q + T), output n2: word m = n1 + 16 n2 of
         // line l at Vs[l][m ^ l] (32 banks for the 32 lanes), then the 32 columns back
-        uint32_t* Vs = Zs;
 #pragma unroll
         for (int T = 0; T < 4; ++T) {
             float d[16];
@@ -1074,6 +1129,7 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
             break;
         }
     }
+    cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
@@ -1088,7 +1144,8 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
     __shared__ uint32_t tmem_base;
     const bool hdr_ok = header_c(spectrum, false, 0);
     uint8_t* A = smem_ci;
-    uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ci + kOffStC);   // output staging [r][n ^ r]
+    uint32_t* Ws = reinterpret_cast<uint32_t*>(smem_ci + kOffStC);   // the task's Y[k][32 rows]
+    uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ci);             // output staging [r][n ^ r] (operand area)
     float2* w256 = reinterpret_cast<float2*>(smem_ci + kOffW256);
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
@@ -1103,23 +1160,39 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
     const int64_t nb2 = B / 2, Ctot = int64_t(order + 1) * C, n_img = int64_t(CN) * CN;
     const int ntasks = npairs * (CN / NROW);
 
+    // a task's Y[k][32 rg .. 32 rg + 31] (256 rows of 128 bytes in the workspace) ->
+    // Ws[k][r] by cp.async: the next task's are copied while this one is transformed
+    auto stage_rows = [&](int task) {
+        const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
+        const uint32_t* wsp = reinterpret_cast<const uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg;
+#pragma unroll
+        for (int kk = 0; kk < CN * NROW / 4 / NT; ++kk) {
+            const int gi = t + NT * kk, k = gi >> 3, g4 = gi & 7;
+            cp_async_bytes16(Ws + k * NROW + 4 * g4, wsp + int64_t(k) * CN + 4 * g4);
+        }
+        cp_async_commit();
+    };
+    if (int(blockIdx.x) < ntasks) stage_rows(blockIdx.x);
+
     for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
         const int lp = task / (CN / NROW), rg = task - lp * (CN / NROW);
         const int64_t pr = pair0 + lp, c = pr / nb2, b0 = 2 * (pr - c * nb2);
+        cp_async_wait_all();
+        __syncthreads();
         {
-            // conj Y[k1 + 16 k2][r] at row R(r, k1), chunk k2 / 4; lane = r, the 32 loads
-            // of a thread in flight together
-            const uint32_t* wsp = reinterpret_cast<const uint32_t*>(ws + int64_t(lp) * ws_pair_stride) + NROW * rg + lane;
+            // conj Y[k1 + 16 k2][r] at row R(r, k1), chunk k2 / 4; lane = r (a warp reads
+            // 32 consecutive words)
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int ci = warp + 8 * m, k1 = ci & 15, ch = ci >> 4;
                 uint32_t q[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) q[e] = wsp[int64_t(k1 + 16 * (4 * ch + e)) * CN] ^ 0x80000000u;
+                for (int e = 0; e < 4; ++e) q[e] = Ws[(k1 + 16 * (4 * ch + e)) * NROW + lane] ^ 0x80000000u;
                 sts128(A, tc::chunk_off(rowc(lane, k1), ch, kSBOc), q[0], q[1], q[2], q[3]);
             }
         }
-        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
+        issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);   // every thread is past its build: Ws is free
+        if (task + int(gridDim.x) < ntasks) stage_rows(task + int(gridDim.x));
         pass_c(A, w256, tl, Q, hh, lane, &mbar, phase, ok, wait_budget_ns);
         issue_c(a_addr, b_addr, tmem, &mbar, ok && issue_mma);
         // the gate rows (x_gchunk of both images) are on their way while the last stage runs
@@ -1155,6 +1228,7 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
             break;
         }
     }
+    cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemColsC);
@@ -1266,9 +1340,9 @@ cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws,
     const int64_t ntasks = npairs * (CN / NROW);
     if (ntasks > INT32_MAX) return cudaErrorInvalidValue;
     const unsigned grid = unsigned(ntasks < 2 * sms ? ntasks : 2 * sms);
-    cudaError_t e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+    cudaError_t e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemCF));
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
+        e = cudaFuncSetAttribute(k_2dc_rows_fwd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemCF));
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_2dc_cols_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_2dc_rows_inv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemC));
@@ -1279,7 +1353,7 @@ cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws,
     for (int st = 1; st < p.order; ++st) {
         // as for the padded pairs: step st gates with x_{order-st}; a later step reads
         // its input from y, where the previous step's inverse pass left it
-        (st == 1 ? k_2dc_rows_fwd_tc<true> : k_2dc_rows_fwd_tc<false>)<<<grid, NT, kSmemC, s>>>(
+        (st == 1 ? k_2dc_rows_fwd_tc<true> : k_2dc_rows_fwd_tc<false>)<<<grid, NT, kSmemCF, s>>>(
             u, y, w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride, a.wait_budget_ns, a.issue_mma,
             a.status);
         k_2dc_cols_tc<<<grid, NT, kSmemC, s>>>(w, a.spectrum, a.B / 2, st - 1, pair0, int(npairs), pstride,
