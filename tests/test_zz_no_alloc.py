@@ -15,7 +15,7 @@ import pytest
 
 from fft_long_convolution_02_b200 import binding as hb
 from fft_long_convolution_02_b200 import inputs as I
-from gpu_helpers import TOL, Run, oracle_for_rows, row_rel_err
+from gpu_helpers import TOL, Run, api_shape, oracle_for_rows, row_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,7 @@ def _cuda():
 
 def _groups(p):
     """Groups of rows the fixed scratch is cut into for problem p."""
-    row = hb.hyena_gated_fftconv_workspace_min_bytes(p.C, p.shape, p.order)
+    row = hb.hyena_gated_fftconv_workspace_min_bytes(p.C, api_shape(p), p.order)
     per_group = SCRATCH // row
     if p.ndim in (1, 2) and p.dtype == "bf16":
         per_group *= 2          # the four-step and 2-D workspaces hold bf16 pairs with bf16 storage
@@ -58,8 +58,10 @@ CASES = [
     I.WORKLOADS["d768_l8k"].with_(C=16, seed=1205),
     # cluster path, bf16, order 3, L = 2^16: the scratch holds one 512 KB slice per cluster
     I.WORKLOADS["order3"].with_(B=3, C=7, L=1 << 16, seed=1206),
+    # circular 2-D paired images (256 x 256, order 2): 254 images per group, 280 -> 2 groups of whole pairs
+    I.WORKLOADS["grid2d_circ"].with_(B=2, C=140, seed=1209),
 ]
-EXPECTED_GROUPS = [3, 2, 8, 1, 2, 2, None, None]
+EXPECTED_GROUPS = [3, 2, 8, 1, 2, 2, None, None, 2]
 
 
 def test_cases_span_several_groups():
@@ -76,7 +78,7 @@ def test_noalloc_matches_workspace_entry_point(p):
     ref = r.run()                      # hyena_gated_fftconv with a workspace
     for _ in range(2):                 # two calls in a row share the fixed scratch
         y = torch.full_like(r.y, float("nan"))
-        hb.hyena_gated_fftconv_noalloc(r.u, y, r.spectrum, r.sc_w, r.sc_b, p.B, p.C, p.shape, p.order)
+        hb.hyena_gated_fftconv_noalloc(r.u, y, r.spectrum, r.sc_w, r.sc_b, p.B, p.C, api_shape(p), p.order)
         torch.cuda.synchronize()
         got = y.double().cpu().numpy()
         assert np.isfinite(got).all()
