@@ -8,6 +8,9 @@ all order steps, output gate) with inputs resident in HBM.  Default workload:
 B=4, C=768, L=8192, order 2, bf16 storage / fp32 math (the 1-D operator at
 width 768 and 8K context).  The spectrum cache is built once, before timing.
 Every step reads ~252 MB (> the 126 MB L2), so no explicit L2 flush is needed.
+The K timed steps run back to back between two CUDA events on the launching
+stream; the roofline's launch duration is that region's time per step (one
+step is one call: at L = 8192 one kernel launch).
 
 N > 1 (torchrun): every rank runs the same per-GPU workload on its own GPU
 (rows are independent: no exchange), so scaling is weak; the time is the max
@@ -443,24 +446,24 @@ def main():
         for _ in range(8):
             step()
         torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push("hyena timed steps")
+    # the K steps back to back between two events on the launching stream (events
+    # between the steps would add their own gaps); a step is one call, so the
+    # average step of this region is the average duration of the call's kernels
     t_start.record(stream)
     for i in range(args.steps):
-        ev[i][0].record(stream)
         step()
-        ev[i][1].record(stream)
     t_stop.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_stop)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    launch_ms = [elapsed_ms / args.steps]
     elapsed_ms = hd.max_over_ranks(elapsed_ms, dev)
 
     # the same workload with every transform multiply in fp32 (bf16 storage,
