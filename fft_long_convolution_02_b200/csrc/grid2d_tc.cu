@@ -873,12 +873,24 @@ __device__ __forceinline__ void issue_c(uint32_t a_addr, uint32_t b_addr, uint32
     stage_issue(a_addr, kSBOc, b_addr, kSBOc, 4, 2, tc::idesc_bf16(128, 32), tmem, 32, mbar, go);
 }
 
-// Common prologue of the circular kernels: tables, header check, barrier and
-// tensor memory.  Returns false (status reported) on a header mismatch.
+__device__ __forceinline__ bool header_c(const uint8_t* spectrum, bool check_plane, int64_t plane_off) {
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
+    return (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D_CIRC) & (hv.H == CN) & (hv.W == CN) &
+           (!check_plane | (hv.reserved[1] == plane_off));
+}
+
+// Common prologue of the circular kernels: tables (no global memory), then the
+// wait for the grids this launch depends on (the kernels are launched with
+// programmatic stream serialisation: the tables are built while the previous
+// kernel finishes), the header check, barrier and tensor memory.  Returns false
+// (status reported) on a header mismatch.
 template <uint32_t OFF_B = kOffBc>
-__device__ __forceinline__ bool prologue_c(uint8_t* smem, float2* w256, bool hdr_ok, uint64_t* mbar,
-                                           uint32_t* tmem_base, uint32_t* status) {
+__device__ __forceinline__ bool prologue_c(uint8_t* smem, float2* w256, const uint8_t* spectrum, bool check_plane,
+                                           int64_t plane_off, uint64_t* mbar, uint32_t* tmem_base,
+                                           uint32_t* status) {
     setup_tables_c<OFF_B>(smem, w256);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const bool hdr_ok = header_c(spectrum, check_plane, plane_off);
     if (!hdr_ok) {
         if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return false;
@@ -891,12 +903,6 @@ __device__ __forceinline__ bool prologue_c(uint8_t* smem, float2* w256, bool hdr
     return true;
 }
 
-__device__ __forceinline__ bool header_c(const uint8_t* spectrum, bool check_plane, int64_t plane_off) {
-    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
-    return (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D_CIRC) & (hv.H == CN) & (hv.W == CN) &
-           (!check_plane | (hv.reserved[1] == plane_off));
-}
-
 // GATE: the first order step (z = x_{order-1} v from u); else z from zsrc.
 template <bool GATE>
 __global__ void __launch_bounds__(NT, 2)
@@ -906,7 +912,6 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
     extern __shared__ __align__(1024) uint8_t smem_cf[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const bool hdr_ok = header_c(spectrum, false, 0);
     uint8_t* A = smem_cf;
     uint8_t* Rw = smem_cf + kOffStC;                                 // raw rows: x_b0, x_b1 (, v_b0, v_b1)
     uint32_t* Zs = reinterpret_cast<uint32_t*>(Rw);                  // gated rows (over the raw ones)
@@ -915,7 +920,7 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    if (!prologue_c<kOffBcF>(smem_cf, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    if (!prologue_c<kOffBcF>(smem_cf, w256, spectrum, false, 0, &mbar, &tmem_base, status)) return;
     const uint32_t tmem = tmem_base;
     const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
     const uint32_t a_addr = tc::smem_u32(A);
@@ -1005,6 +1010,7 @@ k_2dc_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __n
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
@@ -1018,7 +1024,6 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
     extern __shared__ __align__(1024) uint8_t smem_cc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const bool hdr_ok = header_c(spectrum, true, plane_off);
     uint8_t* A = smem_cc;
     uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_cc + kOffStC);   // input columns
     uint32_t* Vs = reinterpret_cast<uint32_t*>(smem_cc);             // output staging (the operand area)
@@ -1026,7 +1031,7 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    if (!prologue_c(smem_cc, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    if (!prologue_c(smem_cc, w256, spectrum, true, plane_off, &mbar, &tmem_base, status)) return;
     const uint32_t tmem = tmem_base;
     const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
     const uint32_t a_addr = tc::smem_u32(A);
@@ -1129,6 +1134,7 @@ k_2dc_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spect
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
@@ -1142,7 +1148,6 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
     extern __shared__ __align__(1024) uint8_t smem_ci[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const bool hdr_ok = header_c(spectrum, false, 0);
     uint8_t* A = smem_ci;
     uint32_t* Ws = reinterpret_cast<uint32_t*>(smem_ci + kOffStC);   // the task's Y[k][32 rows]
     uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ci);             // output staging [r][n ^ r] (operand area)
@@ -1150,7 +1155,7 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
     const int t = threadIdx.x;
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
-    if (!prologue_c(smem_ci, w256, hdr_ok, &mbar, &tmem_base, status)) return;
+    if (!prologue_c(smem_ci, w256, spectrum, false, 0, &mbar, &tmem_base, status)) return;
     const uint32_t tmem = tmem_base;
     const uint32_t tl = tmem + (uint32_t(32 * Q) << 16);
     const uint32_t a_addr = tc::smem_u32(A);
@@ -1228,6 +1233,7 @@ k_2dc_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_b
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     cp_async_wait_all();   // no copy into this CTA's shared memory outlives it
     tc::fence_before_sync();
     __syncthreads();
@@ -1350,19 +1356,37 @@ cudaError_t launch_conv_2dc_pairs_tc(const Plan& p, const ConvArgs& a, void* ws,
     const bf16* u = static_cast<const bf16*>(a.u);
     bf16* y = static_cast<bf16*>(a.y);
     __nv_bfloat162* w = static_cast<__nv_bfloat162*>(ws);
-    for (int st = 1; st < p.order; ++st) {
+    // programmatic stream serialisation: each kernel sets up its tables while the one
+    // before it finishes, and waits for it (griddepcontrol.wait) before its first read
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    auto cfg = [&](size_t smem) {
+        cudaLaunchConfig_t c = {};
+        c.gridDim = dim3(grid);
+        c.blockDim = dim3(NT);
+        c.dynamicSmemBytes = smem;
+        c.stream = s;
+        c.attrs = pdl;
+        c.numAttrs = 1;
+        return c;
+    };
+    const cudaLaunchConfig_t cf = cfg(kSmemCF), cc = cfg(kSmemC);
+    for (int st = 1; st < p.order && e == cudaSuccess; ++st) {
         // as for the padded pairs: step st gates with x_{order-st}; a later step reads
         // its input from y, where the previous step's inverse pass left it
-        (st == 1 ? k_2dc_rows_fwd_tc<true> : k_2dc_rows_fwd_tc<false>)<<<grid, NT, kSmemCF, s>>>(
-            u, y, w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride, a.wait_budget_ns, a.issue_mma,
-            a.status);
-        k_2dc_cols_tc<<<grid, NT, kSmemC, s>>>(w, a.spectrum, a.B / 2, st - 1, pair0, int(npairs), pstride,
-                                               int64_t(a.g2_plane_off), a.spec_C, a.wait_budget_ns, a.issue_mma,
-                                               a.status);
-        k_2dc_rows_inv_tc<<<grid, NT, kSmemC, s>>>(u, y, w, a.spectrum, a.B, p.C, p.order,
-                                                   st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs),
-                                                   pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        e = cudaLaunchKernelEx(&cf, st == 1 ? k_2dc_rows_fwd_tc<true> : k_2dc_rows_fwd_tc<false>, u,
+                               static_cast<const bf16*>(y), w, a.spectrum, a.B, p.C, p.order, pair0, int(npairs),
+                               pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        if (e == cudaSuccess)
+            e = cudaLaunchKernelEx(&cc, k_2dc_cols_tc, w, a.spectrum, a.B / 2, st - 1, pair0, int(npairs), pstride,
+                                   int64_t(a.g2_plane_off), a.spec_C, a.wait_budget_ns, a.issue_mma, a.status);
+        if (e == cudaSuccess)
+            e = cudaLaunchKernelEx(&cc, k_2dc_rows_inv_tc, u, y, static_cast<const __nv_bfloat162*>(w), a.spectrum,
+                                   a.B, p.C, p.order, st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs),
+                                   pstride, a.wait_budget_ns, a.issue_mma, a.status);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
