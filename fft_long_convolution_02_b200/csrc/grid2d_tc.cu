@@ -230,11 +230,6 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     extern __shared__ __align__(1024) uint8_t smem_2t[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    // the header is requested first and checked once the tables are set up
-    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
-    const SpecHeader hv = *h;
-    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == hdr_W) &
-                        (hv.reserved[1] == plane_off);
     uint8_t* A = smem_2t;
     uint8_t* A1 = smem_2t + kOffA1;
     uint32_t* Vs = reinterpret_cast<uint32_t*>(smem_2t);     // output staging [column][p]
@@ -244,6 +239,13 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
     const int Q = warp & 3, hh = warp >> 2;
 
     setup_tables<true, true, true>(smem_2t, w512);
+    // launched with programmatic stream serialisation in the paired passes: the
+    // tables are built while the previous kernel finishes; nothing global is read
+    // or written before this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == hdr_W) &
+                        (hv.reserved[1] == plane_off);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -362,6 +364,7 @@ k_2d_cols_tc(__nv_bfloat162* __restrict__ ws, const uint8_t* __restrict__ spectr
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
@@ -527,9 +530,6 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv
     extern __shared__ __align__(1024) uint8_t smem_rf[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
-    const SpecHeader hv = *h;
-    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
     uint8_t* A = smem_rf;
     uint8_t* A1 = smem_rf + kOffA1;
     uint32_t* Zs = reinterpret_cast<uint32_t*>(smem_rf);     // gated rows, then the output staging
@@ -538,6 +538,9 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
     setup_tables<true, true, false>(smem_rf, w512);
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // as in k_2d_cols_tc
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -622,6 +625,7 @@ k_2d_rows_fwd_tc(const bf16* __restrict__ u, const bf16* __restrict__ zsrc, __nv
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
@@ -635,9 +639,6 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
     extern __shared__ __align__(1024) uint8_t smem_ri[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
-    const SpecHeader hv = *h;
-    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
     uint8_t* A = smem_ri;
     uint32_t* Ys = reinterpret_cast<uint32_t*>(smem_ri);      // output staging [r][n ^ r]
     float2* w512 = reinterpret_cast<float2*>(smem_ri + kOffW512);
@@ -645,6 +646,9 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
     const int warp = t >> 5, lane = t & 31;
     const int Q = warp & 3, hh = warp >> 2;
     setup_tables<false, true, true>(smem_ri, w512);
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // as in k_2d_cols_tc
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_GRID_2D) & (hv.H == MH) & (hv.W == W2);
     if (!hdr_ok) {
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -719,6 +723,7 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
             break;
         }
     }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the next kernel may start its setup
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
@@ -1301,20 +1306,39 @@ cudaError_t launch_conv_2d_pairs_tc(const Plan& p, const ConvArgs& a, void* ws, 
     if (e != cudaSuccess) return e;
     bf16* y = static_cast<bf16*>(a.y);
     const int64_t ctasks = npairs * (2 * W2 / NCOL);
-    for (int st = 1; st < p.order; ++st) {
+    // programmatic stream serialisation, as for the circular passes
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    auto cfg = [&](unsigned g) {
+        cudaLaunchConfig_t c = {};
+        c.gridDim = dim3(g);
+        c.blockDim = dim3(NT);
+        c.dynamicSmemBytes = kSmem;
+        c.stream = s;
+        c.attrs = pdl;
+        c.numAttrs = 1;
+        return c;
+    };
+    const cudaLaunchConfig_t cr = cfg(grid), ccl = cfg(unsigned(ctasks < 2 * sms ? ctasks : 2 * sms));
+    for (int st = 1; st < p.order && e == cudaSuccess; ++st) {
         // step st gates with x_{order-st}: the first step's input is x_{order-1} v, a later
         // step's is x_{order-st} times the previous step's result, which that step's
         // inverse pass left in y; the last inverse pass applies x0
-        k_2d_rows_fwd_tc<<<grid, NT, kSmem, s>>>(u, st == 1 ? nullptr : y, w, a.spectrum, a.B, p.C, p.order, pair0,
-                                                 int(npairs), pstride, a.wait_budget_ns, a.issue_mma, a.status);
+        e = cudaLaunchKernelEx(&cr, k_2d_rows_fwd_tc, u, st == 1 ? static_cast<const bf16*>(nullptr) : y, w,
+                               a.spectrum, a.B, p.C, p.order, pair0, int(npairs), pstride, a.wait_budget_ns,
+                               a.issue_mma, a.status);
         // every bin column of a pair (2W), spectrum row (st - 1) C + c, c = pair / (B/2)
-        k_2d_cols_tc<<<unsigned(ctasks < 2 * sms ? ctasks : 2 * sms), NT, kSmem, s>>>(
-            w, a.spectrum, int(p.C), 2 * W2, a.B / 2, st - 1, pair0, int(npairs), pstride, int64_t(a.g2_plane_off),
-            a.spec_C, 0, W2, a.wait_budget_ns, a.issue_mma, a.status);
-        k_2d_rows_inv_tc<<<grid, NT, kSmem, s>>>(u, y, w, a.spectrum, a.B, p.C, p.order,
-                                                 st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs), pstride,
-                                                 a.wait_budget_ns, a.issue_mma, a.status);
+        if (e == cudaSuccess)
+            e = cudaLaunchKernelEx(&ccl, k_2d_cols_tc, w, a.spectrum, int(p.C), 2 * W2, a.B / 2, st - 1, pair0,
+                                   int(npairs), pstride, int64_t(a.g2_plane_off), a.spec_C, int64_t(0), W2,
+                                   a.wait_budget_ns, a.issue_mma, a.status);
+        if (e == cudaSuccess)
+            e = cudaLaunchKernelEx(&cr, k_2d_rows_inv_tc, u, y, static_cast<const __nv_bfloat162*>(w), a.spectrum,
+                                   a.B, p.C, p.order, st == p.order - 1 ? 0 : p.order - st - 1, pair0, int(npairs),
+                                   pstride, a.wait_budget_ns, a.issue_mma, a.status);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
