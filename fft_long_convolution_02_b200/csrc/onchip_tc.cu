@@ -77,13 +77,6 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     extern __shared__ __align__(1024) uint8_t smem_tc[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    // the header is requested first and checked once the tables below are set
-    // up (they read no global memory), so that its latency overlaps them
-    const SpecHeader* h = reinterpret_cast<const SpecHeader*>(spectrum);
-    const SpecHeader hv = *h;                       // all fields requested at once (no short-circuit chain)
-    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_ONCHIP_1D) & (hv.C == C) & (hv.L == L) &
-                        (hv.order == order) & (hv.spec_row_bytes == int64_t(N) * 8) & (hv.tables_off == tables_off) &
-                        (hv.spec_off == spec_off);
     // the layout offsets are kernel parameters (checked against the header above),
     // so that the table pointers need no registers of their own
     const float2* tables = reinterpret_cast<const float2*>(spectrum + tables_off);
@@ -111,6 +104,14 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     fill_dft<32, 32, 32, kSBO64>(smem_tc + kOffB32, w32);
     fill_dft<16, 8, 16, kSBO32>(smem_tc + kOffB1i, w32);
     fill_tw2(TW2);
+    // launched with programmatic stream serialisation: the tables above (no global
+    // memory) are built while the previous kernel on the stream finishes; nothing
+    // global is read or written before this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const SpecHeader hv = *reinterpret_cast<const SpecHeader*>(spectrum);   // all fields at once
+    const bool hdr_ok = (hv.magic == kSpecMagic) & (hv.path == PATH_ONCHIP_1D) & (hv.C == C) & (hv.L == L) &
+                        (hv.order == order) & (hv.spec_row_bytes == int64_t(N) * 8) & (hv.tables_off == tables_off) &
+                        (hv.spec_off == spec_off);
     if (!hdr_ok) {                                  // uniform: every thread read the same header
         if (t == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -177,6 +178,9 @@ k_conv_8192_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const uint8_t* 
     bool have_prev = false;
 
     for (int P = blockIdx.x; P < npairs; P += gridDim.x) {
+        // this CTA's last pair: the next kernel may start its setup on the slots that
+        // the CTAs already done leave free
+        if (P + int(gridDim.x) >= npairs) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         const PairRef pr = pair_ref(P, B);
         const int c = pr.c;
         const bf16* u0 = u + int64_t(pr.b0) * Ctot * L;
@@ -302,11 +306,21 @@ cudaError_t launch_conv_8192_tc(const Plan& p, const ConvArgs& a, cudaStream_t s
     if (npairs > INT32_MAX || a.B > INT32_MAX) return cudaErrorInvalidValue;   // 32-bit pair indices
     int64_t grid = int64_t(2) * sms;
     if (grid > npairs) grid = npairs;
-    kern<<<unsigned(grid), NT, kSmem, s>>>(static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
-                                           a.sc_b, int(a.B), int(p.C), p.order, int(npairs), int64_t(p.tables_off),
-                                           int64_t(p.spec_off), int64_t(p.order + 1) * p.C, a.wait_budget_ns, a.issue_mma,
-                                           a.status);
-    return cudaGetLastError();
+    // programmatic stream serialisation (see the kernel's prologue)
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = s;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const bf16*>(a.u), static_cast<bf16*>(a.y), a.spectrum, a.sc_w,
+                              a.sc_b, int(a.B), int(p.C), p.order, int(npairs), int64_t(p.tables_off),
+                              int64_t(p.spec_off), int64_t(p.order + 1) * p.C, a.wait_budget_ns, a.issue_mma,
+                              a.status);
 }
 
 }  // namespace hyena
