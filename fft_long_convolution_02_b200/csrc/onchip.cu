@@ -176,6 +176,11 @@ k_conv_onchip(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restr
     extern __shared__ float2 smem[];
     constexpr int PS = fft_padded_size(M);
     constexpr int L = 2 * M;
+    // launched with programmatic stream serialisation: wait for the kernel before
+    // this one on the stream (its writes visible), then let the next one be
+    // scheduled once every CTA of this grid has started
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!header_ok(spectrum, SC, L, order)) {
         if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -353,6 +358,8 @@ k_conv_4096(const T* __restrict__ u, T* __restrict__ y, const uint8_t* __restric
             const float* __restrict__ sc_w, const float* __restrict__ sc_b, int64_t B, int64_t C, int order,
             int64_t rows, int64_t SC, int64_t SB, uint32_t* status) {
     extern __shared__ float2 smem[];
+    asm volatile("griddepcontrol.wait;" ::: "memory");               // as in k_conv_onchip
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!header_ok(spectrum, SC, L, order)) {
         if (threadIdx.x == 0) report_status(status, kStatusSpectrumMismatch);
         return;
@@ -668,6 +675,25 @@ cudaError_t spectrum_m(const Plan& p, const SpectrumArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Launch configuration with programmatic stream serialisation (the kernel waits
+// for its predecessor with griddepcontrol.wait before anything else).
+inline cudaLaunchConfig_t pdl_config(unsigned grid, unsigned threads, size_t smem, cudaStream_t s) {
+    static const cudaLaunchAttribute kAttr = [] {          // initialised once, read-only after
+        cudaLaunchAttribute at = {};
+        at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at.val.programmaticStreamSerializationAllowed = 1;
+        return at;
+    }();
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(grid);
+    c.blockDim = dim3(threads);
+    c.dynamicSmemBytes = smem;
+    c.stream = s;
+    c.attrs = const_cast<cudaLaunchAttribute*>(&kAttr);
+    c.numAttrs = 1;
+    return c;
+}
+
 template <typename T>
 cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     auto kern = r16::k_conv_4096<T>;
@@ -679,10 +705,9 @@ cudaError_t conv_4096(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     const int64_t rows = a.B * p.C;
     int64_t grid = int64_t(2) * sms;
     if (grid > rows) grid = rows;
-    kern<<<unsigned(grid), r16::NT, smem, s>>>(static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum,
-                                                    a.sc_w, a.sc_b, a.B, p.C, p.order, rows, a.spec_C, a.spec_per_b,
-                                                    a.status);
-    return cudaGetLastError();
+    const cudaLaunchConfig_t cfg = pdl_config(unsigned(grid), r16::NT, smem, s);
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(a.u), static_cast<T*>(a.y), a.spectrum, a.sc_w,
+                              a.sc_b, a.B, int64_t(p.C), p.order, rows, a.spec_C, a.spec_per_b, a.status);
 }
 
 template <int M>
@@ -700,19 +725,18 @@ cudaError_t conv_m(const Plan& p, const ConvArgs& a, cudaStream_t s) {
     constexpr int NT = onchip_threads<M>();
     const size_t smem = size_t(2) * fft_padded_size(M) * sizeof(float2);
     const unsigned grid = unsigned(a.B * p.C);
+    const cudaLaunchConfig_t cfg = pdl_config(grid, NT, smem, s);
     if (a.dtype == DT_F32) {
         auto kern = k_conv_onchip<M, float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        kern<<<grid, NT, smem, s>>>(static_cast<const float*>(a.u), static_cast<float*>(a.y), a.spectrum,
-                                    a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b, a.status);
-    } else {
-        auto kern = k_conv_onchip<M, __nv_bfloat16>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        kern<<<grid, NT, smem, s>>>(static_cast<const __nv_bfloat16*>(a.u), static_cast<__nv_bfloat16*>(a.y),
-                                    a.spectrum, a.sc_w, a.sc_b, a.B, p.C, p.order, a.spec_C, a.spec_per_b,
-                                    a.status);
+        return cudaLaunchKernelEx(&cfg, kern, static_cast<const float*>(a.u), static_cast<float*>(a.y), a.spectrum,
+                                  a.sc_w, a.sc_b, a.B, int64_t(p.C), p.order, a.spec_C, a.spec_per_b, a.status);
     }
-    return cudaGetLastError();
+    auto kern = k_conv_onchip<M, __nv_bfloat16>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(a.u), static_cast<__nv_bfloat16*>(a.y),
+                              a.spectrum, a.sc_w, a.sc_b, a.B, int64_t(p.C), p.order, a.spec_C, a.spec_per_b,
+                              a.status);
 }
 
 #define HYENA_ONCHIP_SWITCH(FN)          \
