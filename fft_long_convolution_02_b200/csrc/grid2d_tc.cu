@@ -1,7 +1,9 @@
-// grid2d_tc.cu -- the column pass of the 2-D non-circular form ([P5] "Native
-// Multi-Dimensional Subquadratic Operators" (gist.science), 方法论: N-D FFT
-// convolution, non-circular by 2x zero padding) with bf16 storage and H = 256
-// on the tensor cores (tcgen05).
+// grid2d_tc.cu -- the 2-D forms on the tensor cores (tcgen05) with bf16
+// storage ([P5] "Native Multi-Dimensional Subquadratic Operators"
+// (gist.science), 方法论: N-D FFT convolution, non-circular by 2x zero
+// padding): the column pass of the non-circular form at H = 256 (first part),
+// the paired-image row, column and row passes at 256 x 256 (second part), and
+// the circular form's paired passes at 256 x 256 (third part).
 //
 // The row pass leaves, per image, W + 1 bin columns of H = 256 complex values
 // (bf16 (re, im) in the workspace).  Each column needs its 2H = 512-point DFT
@@ -749,7 +751,10 @@ k_2d_rows_inv_tc(const bf16* __restrict__ u, bf16* __restrict__ y, const __nv_bf
 // columns (forward, spectrum product, inverse; in place), rows inverse (output
 // gate).  The spectrum is the full 256 x 256 plane (bf16 pairs) in the column
 // pass's thread order, completed from the stored W/2 + 1 columns by the
-// symmetry of a real filter's transform.
+// symmetry of a real filter's transform.  Each kernel copies the next task's
+// inputs into shared memory with cp.async while the current task is
+// transformed; its output staging reuses the operand area, which is free once
+// the last stage is done.
 // ---------------------------------------------------------------------------
 
 constexpr int CN = int(kTc2dH);                  // H = W of the circular tensor-core path
