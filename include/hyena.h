@@ -49,7 +49,11 @@
  *    With bf16 storage the intermediate of the multi-pass (L >= 32768) and
  *    N-D paths is kept as bf16 pairs in the workspace.
  *  - All work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
- *    stream) and is asynchronous: no call synchronises the host.
+ *    stream) and is asynchronous: no call synchronises the host.  The
+ *    convolution kernels are launched with programmatic stream serialisation:
+ *    one may begin (build its tables in shared memory) while the kernel before
+ *    it on the stream finishes, but reads and writes no global memory before
+ *    that kernel has completed, so plain stream order holds for the data.
  *  - Arguments are validated before anything is enqueued; on any error
  *    nothing is launched and a status other than HYENA_OK is returned, with a
  *    thread-local message available from hyena_last_error_detail().
